@@ -1,0 +1,132 @@
+"""Seeded Gaussian-mixture generator and seeded initial-centroid choice.
+
+Recipe (every draw comes from torch.Generator objects seeded from `seed`, one
+independent stream per purpose, so changing one draw leaves the others unchanged):
+
+  centers   n_comp x d, iid U[-1, 1] ("uniform") or iid N(0, 1) ("normal");
+  component per point, iid categorical: equal weights, or Zipf weights w_j ~ j^-s
+            (rank j = 1..n_comp), drawn by inverse CDF of a uniform;
+  point     = center[component] + sigma * N(0, I), computed in fp32, then stored as
+            fp32 or rounded (nearest even) to bf16;
+  init      = the first K entries of a seeded random permutation of [0, N): K distinct
+            point indices; the initial centroids are those points.
+
+Generation on a CUDA device uses the device generator (fast for the 10^8-point case);
+generation on the CPU uses the CPU generator.  The two give different (but equally
+distributed) data; any comparison between the oracle and the GPU uses one generated
+array, copied to wherever it is needed.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass, replace
+
+import torch
+
+# Stream ids for the independent generators derived from one seed.
+_S_CENTERS, _S_COMP, _S_NOISE, _S_INIT = 11, 23, 37, 41
+
+
+@dataclass(frozen=True)
+class MixtureSpec:
+    name: str
+    n: int
+    d: int
+    k: int                 # number of clusters (centroids) and of mixture components
+    dtype: str             # "f32" or "bf16": storage type of X (and the MMA operand)
+    centers: str           # "uniform" in [-1,1]^d or "normal" N(0, I)
+    sigma: float
+    weights: str           # "equal" or "zipf"
+    zipf_s: float = 1.2
+    metric: str = "l2"     # "l2" or "cosine"
+    niter: int = 5
+    seed: int = 0
+
+
+# The five workloads: shapes, distributions and iteration counts.
+CONFIGS = {
+    1: MixtureSpec("tiny_65536x128_k256_f32", 65_536, 128, 256, "f32", "uniform", 0.1,
+                   "equal", niter=5),
+    2: MixtureSpec("ivf_1000000x768_k4096_f32_cosine", 1_000_000, 768, 4096, "f32",
+                   "normal", 0.3, "equal", metric="cosine", niter=20),
+    3: MixtureSpec("mid_10000000x128_k1024_f32", 10_000_000, 128, 1024, "f32",
+                   "uniform", 0.2, "equal", niter=10),
+    4: MixtureSpec("zipf_16000000x128_k65536_f32", 16_000_000, 128, 65_536, "f32",
+                   "normal", 0.15, "zipf", zipf_s=1.2, niter=5),
+    5: MixtureSpec("large_100000000x128_k32768_bf16", 100_000_000, 128, 32_768, "bf16",
+                   "normal", 0.25, "equal", niter=3),
+}
+
+
+def _gen(device, seed: int, stream: int) -> torch.Generator:
+    g = torch.Generator(device=device)
+    g.manual_seed(seed * 1_000_003 + stream)
+    return g
+
+
+def _torch_dtype(dtype: str):
+    return {"f32": torch.float32, "bf16": torch.bfloat16}[dtype]
+
+
+def gaussian_mixture(n: int, d: int, n_comp: int, *, centers: str = "normal",
+                     sigma: float = 0.1, weights: str = "equal", zipf_s: float = 1.2,
+                     dtype: str = "f32", seed: int = 0, device="cpu",
+                     chunk_rows: int = 1 << 22):
+    """Return (X [n, d] fp32 or bf16, comp [n] int32 component ids, centers [n_comp, d]
+    fp32), all on `device`."""
+    device = torch.device(device)
+    gc = _gen(device, seed, _S_CENTERS)
+    if centers == "uniform":
+        cen = torch.rand(n_comp, d, generator=gc, device=device) * 2.0 - 1.0
+    elif centers == "normal":
+        cen = torch.randn(n_comp, d, generator=gc, device=device)
+    else:
+        raise ValueError(centers)
+
+    gk = _gen(device, seed, _S_COMP)
+    if weights == "equal":
+        comp = torch.randint(0, n_comp, (n,), generator=gk, device=device,
+                             dtype=torch.int64)
+    elif weights == "zipf":
+        w = torch.arange(1, n_comp + 1, device=device, dtype=torch.float64) ** (-zipf_s)
+        cdf = torch.cumsum(w / w.sum(), 0)
+        cdf[-1] = 1.0
+        u = torch.rand(n, generator=gk, device=device, dtype=torch.float64)
+        comp = torch.searchsorted(cdf, u, right=True).clamp_(max=n_comp - 1)
+    else:
+        raise ValueError(weights)
+
+    gn = _gen(device, seed, _S_NOISE)
+    X = torch.empty(n, d, dtype=_torch_dtype(dtype), device=device)
+    for r0 in range(0, n, chunk_rows):
+        r1 = min(n, r0 + chunk_rows)
+        noise = torch.randn(r1 - r0, d, generator=gn, device=device)
+        X[r0:r1] = (cen[comp[r0:r1]] + sigma * noise).to(X.dtype)
+        del noise
+    return X, comp.to(torch.int32), cen
+
+
+def init_indices(n: int, k: int, seed: int = 0, device="cpu") -> torch.Tensor:
+    """First k entries of a seeded random permutation of [0, n): k distinct indices."""
+    if k > n:
+        raise ValueError("k > n")
+    g = _gen(torch.device(device), seed, _S_INIT)
+    return torch.randperm(n, generator=g, device=device)[:k]
+
+
+def make_config(cfg, device="cpu", n: int | None = None, **overrides):
+    """Materialise a workload: returns (spec, X, C0 fp32, comp, centers).
+
+    `cfg` is a key of CONFIGS or a MixtureSpec; `n` (and any MixtureSpec field given in
+    `overrides`) shrinks or alters the spec for small test cases."""
+    spec = CONFIGS[cfg] if not isinstance(cfg, MixtureSpec) else cfg
+    if n is not None:
+        overrides["n"] = n
+    if overrides:
+        spec = replace(spec, **overrides)
+    X, comp, cen = gaussian_mixture(spec.n, spec.d, spec.k, centers=spec.centers,
+                                    sigma=spec.sigma, weights=spec.weights,
+                                    zipf_s=spec.zipf_s, dtype=spec.dtype, seed=spec.seed,
+                                    device=device)
+    idx = init_indices(spec.n, spec.k, spec.seed, device=device)
+    C0 = X[idx].float().contiguous()
+    return spec, X, C0, comp, cen
