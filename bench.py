@@ -1,0 +1,400 @@
+"""Throughput of exact Lloyd's k-means on B200 through the C ABI (libfk.so).
+
+A step is one fk_lloyd call: one complete k-means run of `niter` Lloyd iterations (cosine
+normalisation once, then assign + sort + update per iteration) over the workload's N
+synthetic points, starting from the same initial centroids every step.  The metric is
+points x iterations per second for the whole job.
+
+Default workload: N = 1,000,000 points, d = 768, K = 4096, fp32, cosine, 20 iterations
+(the IVF coarse-quantizer build shape of the LEANN FlashLib guide, section "性能对比").
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config 1..5] [--impl reference]
+
+Under torchrun every rank runs its own independent copy of the workload (its own seed), so
+per-GPU work is fixed (weak scaling); the whole-job value divides all ranks' points x
+iterations by the slowest rank's device time.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "points·iterations/sec per Lloyd iter (assign+update) on 1 B200; % of roofline"
+UNIT = "points*iter/s"
+# The pages' own figure for the default workload: a 1M x 768, nlist 4096 k-means build
+# (default niter 20) in 10.6 s on an H200 (another machine; context only).
+PAGES_BUILD_RATE = 1_000_000 * 20 / 10.6
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=5)
+    p.add_argument("--warmup", type=int, default=3)
+    p.add_argument("--config", type=int, default=2)
+    p.add_argument("--niter", type=int, default=None)
+    p.add_argument("--impl", default="fk", choices=["fk", "reference"])
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--cpu-seconds", type=float, default=12.0)
+    return p.parse_args()
+
+
+# ----------------------------------------------------------------------------- helpers
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": p["hbm_gbs"], "bf16": p["bf16_tflops"],
+                "bf16_sustained": p["bf16_tflops_sustained"], "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16": 1590.0, "bf16_sustained": 1400.0, "source": "fallback"}
+
+
+def assign_traffic_record():
+    """DRAM bytes per assign launch from a committed ncu summary, if it was taken on the
+    current kernel source (else None)."""
+    path = os.path.join(ROOT, "profiles", "assign_traffic.json")
+    src = os.path.join(ROOT, "exact_lloyd_means_b200", "csrc", "assign_sm100.cu")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        rec = json.load(f)
+    h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    return rec if rec.get("kernel_sha") == h else None
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms while running."""
+
+    FIELDS = ("index,uuid,clocks.sm,clocks.max.sm,power.draw,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid):
+        self.uuid = str(uuid or "").lower().replace("gpu-", "")
+        self.proc = None
+        self.path = os.path.join("/tmp", f"fk_clocks_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=self.f, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.f.close()
+        rows = []
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            if self.uuid and self.uuid not in parts[1].lower():
+                continue
+            rows.append(parts)
+        os.remove(self.path)
+        if not rows:
+            return None
+        sm = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        mx = [float(r[3]) for r in rows if r[3].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[j] for r in rows for j in range(4)
+                          if r[5 + j].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(rows)}
+
+
+def cpu_baseline(X_host, C0_host, metric, precision, seconds):
+    """The oracle as it stands (fp64 C + OpenMP), timed on this host's cores on a bounded
+    sample: one Lloyd iteration (assign against all K centroids, CSR, update, objective)
+    over S sampled points.  Returns (points*iter/s, threads, description)."""
+    import oracle
+
+    def one(S):
+        Xs = X_host[:S]
+        t0 = time.perf_counter()
+        Xd = oracle.normalize_rows(Xs) if metric == "cosine" else oracle._f64(Xs)
+        C = oracle.normalize_rows(C0_host) if metric == "cosine" else oracle._f64(C0_host)
+        C = oracle.round_bf16(C) if precision == "bf16" else C
+        lab, _, _ = oracle.assign(Xd, C)
+        oracle.csr(lab, C.shape[0])
+        oracle.update(Xd, lab, C)
+        oracle.objective(Xd, C, lab)
+        return time.perf_counter() - t0
+
+    S = 64
+    t = one(S)
+    while t < 1.0 and S < X_host.shape[0]:
+        S = min(X_host.shape[0], S * 4)
+        t = one(S)
+    S2 = int(min(X_host.shape[0], max(S, S * seconds / max(t, 1e-9))))
+    t2 = one(S2)
+    return S2 / t2, oracle.threads(), f"one oracle Lloyd iteration over the first {S2} points"
+
+
+# ----------------------------------------------------------------------------- arms
+
+
+def reference_arm(args, spec, rank, world):
+    """The oracle timed on the host as the reference arm: each step is one Lloyd iteration
+    over a bounded sample of the workload's points."""
+    if rank != 0:
+        return
+    import numpy as np
+    import torch
+
+    import oracle
+    from synth import gaussian_mixture, init_indices
+    S = 256 if spec.d * spec.k > 1_000_000 else 4096
+    n_gen = 2 * max(S, spec.k)
+    X, _, _ = gaussian_mixture(n_gen, spec.d, spec.k, centers=spec.centers, sigma=spec.sigma,
+                               weights=spec.weights, zipf_s=spec.zipf_s, dtype=spec.dtype,
+                               seed=spec.seed)
+    idx = init_indices(n_gen, spec.k, spec.seed)
+    C0 = X[idx].float().numpy()
+    Xh = X[:S].double().numpy() if spec.dtype == "bf16" else X[:S].numpy()
+    prec = "bf16" if spec.dtype == "bf16" else "f32"
+
+    def step():
+        Xd = oracle.normalize_rows(Xh) if spec.metric == "cosine" else oracle._f64(Xh)
+        C = oracle.normalize_rows(C0) if spec.metric == "cosine" else oracle._f64(C0)
+        C = oracle.round_bf16(C) if prec == "bf16" else C
+        lab, _, _ = oracle.assign(Xd, C)
+        oracle.csr(lab, C.shape[0])
+        oracle.update(Xd, lab, C)
+        oracle.objective(Xd, C, lab)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = time.perf_counter() - t0
+    value = S * args.steps / dt
+    sample = f"one oracle Lloyd iteration over {S} points of the workload per step"
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": dt * 1e3 / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": spec.name, "N": spec.n, "d": spec.d, "K": spec.k,
+                   "metric": spec.metric, "sample_points": S},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle.threads(),
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0}}), flush=True)
+
+
+def fk_arm(args, spec, rank, world, dist):
+    import torch
+
+    from exact_lloyd_means_b200 import fk
+    from synth import gaussian_mixture, init_indices
+
+    dev = torch.device("cuda", torch.cuda.current_device())
+    niter = args.niter or spec.niter
+    seed = spec.seed + rank
+    X, _, _ = gaussian_mixture(spec.n, spec.d, spec.k, centers=spec.centers, sigma=spec.sigma,
+                               weights=spec.weights, zipf_s=spec.zipf_s, dtype=spec.dtype,
+                               seed=seed, device=dev)
+    C0 = X[init_indices(spec.n, spec.k, seed, device=dev)].float().contiguous()
+    C = torch.empty_like(C0)
+    labels = torch.empty(spec.n, dtype=torch.int32, device=dev)
+    counts = torch.empty(spec.k, dtype=torch.int32, device=dev)
+    ws = fk.workspace(spec.n, spec.d, spec.k, X.dtype, spec.metric, device=dev)
+    torch.cuda.synchronize()
+
+    def step(acc):
+        C.copy_(C0)
+        objs, tm = fk.fk_lloyd(X, C, niter, labels, ws, metric=spec.metric, counts=counts,
+                               timing=True)
+        if acc is not None:
+            for k in ("ms_setup", "ms_prep", "ms_assign", "ms_sort", "ms_update"):
+                acc[k] = acc.get(k, 0.0) + tm[k]
+            acc["launches"] = acc.get("launches", 0) + tm["launches"]
+        return objs
+
+    for _ in range(args.warmup):
+        step(None)
+
+    uuid = None
+    try:
+        uuid = torch.cuda.get_device_properties(dev).uuid
+    except Exception:
+        pass
+    sampler = ClockSampler(uuid)
+    sampler.start()
+    time.sleep(0.4)
+    acc = {}
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        objs = step(acc)
+    e1.record()
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    clocks = sampler.stop()
+    ms = e0.elapsed_time(e1)
+    if dist:
+        t = torch.tensor([ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = t.item()
+
+    pts_iter = spec.n * niter * args.steps * world
+    value = pts_iter / (ms / 1e3)
+
+    # roofline of the dominant kernel (assign), from the per-launch device times that
+    # fk_lloyd recorded with CUDA events on this stream during the timed steps
+    peaks = load_peaks()
+    n_assign = niter * args.steps
+    assign_ms = acc["ms_assign"] / n_assign
+    flops = 2.0 * spec.n * spec.k * spec.d
+    achieved = flops / (assign_ms / 1e3) / 1e12
+    if spec.dtype == "f32":
+        peak = peaks["bf16_sustained"] / 3.0
+        peak_note = ("fp32 products as 3 bf16 tensor-core products: measured sustained bf16 "
+                     f"dense {peaks['bf16_sustained']} TFLOP/s / 3 ({peaks['source']})")
+    else:
+        peak = peaks["bf16_sustained"]
+        peak_note = f"measured sustained bf16 dense TFLOP/s ({peaks['source']})"
+    trec = assign_traffic_record()
+    roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+            "frac": achieved / peak, "traffic": trec["bytes_per_launch"] if trec else None,
+            "kernel": "assign_kernel (tcgen05)", "algorithmic_flops_per_launch": flops,
+            "avg_launch_ms": assign_ms, "peak_note": peak_note}
+    upd_ms = (acc["ms_sort"] + acc["ms_update"]) / n_assign
+    e_bytes = 4 if spec.dtype == "f32" else 2
+    upd_bytes = spec.n * spec.d * e_bytes + 24.0 * spec.n
+    phases = {k: acc[k] / args.steps for k in ("ms_setup", "ms_prep", "ms_assign",
+                                                "ms_sort", "ms_update")}
+
+    out = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
+           "higher_is_better": True, "scaling": "weak",
+           "vs_baseline": value / PAGES_BUILD_RATE if args.config == 2 and niter == 20
+           else None,
+           "vs_baseline_note": "pages' 1M x 768 nlist 4096 build: 10.6 s for 20 iterations "
+                               "on an H200 (another machine; context)",
+           "dtype": spec.dtype, "data": "synthetic",
+           "config": {"workload": spec.name, "N": spec.n, "d": spec.d, "K": spec.k,
+                      "metric": spec.metric, "niter_per_step": niter,
+                      "parallelism": f"replica x{world}",
+                      "l2": f"inputs larger than L2 (X = {spec.n * spec.d * e_bytes / 1e9:.2f}"
+                            " GB per rank)"},
+           "roofline": roof,
+           "update_hbm": {"achieved_gbs": upd_bytes / (upd_ms / 1e3) / 1e9,
+                          "peak_gbs": peaks["hbm_gbs"],
+                          "frac": upd_bytes / (upd_ms / 1e3) / 1e9 / peaks["hbm_gbs"],
+                          "avg_ms": upd_ms},
+           "phase_ms_per_step": phases,
+           "gpu_launches": acc["launches"], "final_objective": objs[-1],
+           "clocks": clocks}
+
+    # end to end through the public API with host buffers
+    if not args.no_e2e:
+        Xh = torch.empty(X.shape, dtype=X.dtype, pin_memory=True)
+        Xh.copy_(X)
+        C0h = torch.empty(C0.shape, dtype=torch.float32, pin_memory=True)
+        C0h.copy_(C0)
+        labh = torch.empty(spec.n, dtype=torch.int32, pin_memory=True)
+        Ch = torch.empty(C0.shape, dtype=torch.float32, pin_memory=True)
+        Xd = torch.empty_like(X)
+        ke = max(1, min(args.steps, 3))
+
+        def e2e_step():
+            Xd.copy_(Xh, non_blocking=True)
+            C.copy_(C0h, non_blocking=True)
+            fk.fk_lloyd(Xd, C, niter, labels, ws, metric=spec.metric)
+            labh.copy_(labels, non_blocking=True)
+            Ch.copy_(C, non_blocking=True)
+            torch.cuda.synchronize()
+
+        e2e_step()
+        if dist:
+            dist.barrier()
+        torch.cuda.synchronize()
+        f0 = torch.cuda.Event(enable_timing=True)
+        f1 = torch.cuda.Event(enable_timing=True)
+        f0.record()
+        for _ in range(ke):
+            e2e_step()
+        f1.record()
+        torch.cuda.synchronize()
+        ems = f0.elapsed_time(f1)
+        if dist:
+            t = torch.tensor([ems], device=dev, dtype=torch.float64)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ems = t.item()
+        out["e2e"] = {"value": spec.n * niter * ke * world / (ems / 1e3), "unit": UNIT,
+                      "h2d_bytes_per_step": X.numel() * X.element_size() + C0.numel() * 4,
+                      "d2h_bytes_per_step": spec.n * 4 + C0.numel() * 4 + niter * 8,
+                      "steps": ke}
+        del Xh, Xd
+
+    if not args.no_cpu_baseline and world == 1 and rank == 0:
+        S = min(spec.n, 1 << 16)
+        Xs = X[:S].cpu()
+        Xs = Xs.double().numpy() if spec.dtype == "bf16" else Xs.numpy()
+        v, cores, sample = cpu_baseline(Xs, C0.cpu().numpy(), spec.metric,
+                                        "bf16" if spec.dtype == "bf16" else "f32",
+                                        args.cpu_seconds)
+        out["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle",
+                               "sample": sample, "host_nproc": os.cpu_count()}
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+
+
+def main():
+    args = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    from synth import CONFIGS
+    spec = CONFIGS[args.config]
+    if args.impl == "reference":
+        reference_arm(args, spec, rank, world)
+        return
+    import torch
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as tdist
+        local = int(os.environ.get("LOCAL_RANK", "0"))
+        torch.cuda.set_device(local)
+        tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600))
+        dist = tdist
+    fk_arm(args, spec, rank, world, dist)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

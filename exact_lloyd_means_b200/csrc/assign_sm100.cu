@@ -1,0 +1,357 @@
+// assign_sm100.cu -- fused nearest-centroid assignment on B200 tensor cores.
+//
+// Flash-KMeans article, section "FlashAssign：把距离矩阵按块切成流水线": distances of a
+// block of points to all centroids are produced on the fly and reduced to an argmin on
+// chip, so the N x K distance matrix never reaches memory and only O(Nd + Kd) bytes move.
+//
+// B200 design (a new kernel; the article's H200 kernel is prior art only):
+//   * persistent grid, one CTA per SM; a CTA owns 128-row blocks of X in turn and sweeps
+//     all centroid tiles of 256 for each;
+//   * warp 0, one thread: TMA producer.  Per 64-column chunk of d it loads the X chunk(s)
+//     (128 x 64 bf16 per plane) and the centroid chunk(s) (256 x 64 bf16 per plane) into
+//     a ring of shared-memory stages, 128-byte swizzled; completion by mbarrier tx-count;
+//   * warp 1, one thread: tcgen05.mma issuer, kind::f16 (bf16 x bf16 -> fp32), M=128,
+//     N=256, K=16 per instruction, accumulating a 128 x 256 fp32 tile in tensor memory;
+//     two accumulators (512 TMEM columns) so the epilogue of tile t overlaps the MMAs of
+//     tile t+1; tcgen05.commit releases smem stages and hands tiles to the epilogue;
+//   * warps 2..5 (128 threads, one per row / TMEM lane): epilogue.  tcgen05.ld 32 columns
+//     at a time, v = acc + ||c||^2 (the B operand holds -2c), chunk minimum, and a running
+//     (min, argmin) per row in registers; ties keep the lowest centroid index.  Only the
+//     label (and optionally the minimum) is written to HBM.
+//   * fp32 points (NP = 2): x.c is formed from three bf16 products hi*hi' + lo*hi' +
+//     hi*lo' into one fp32 accumulator (the X and centroid planes come split from prep).
+//     bf16 points (NP = 1): one product, exact in fp32.
+//   * every mbarrier wait is bounded; on expiry the CTA raises the abort flag, records
+//     the timeout in the workspace error word and winds down (TMEM is always freed).
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include "fk_common.cuh"
+#include "ptx_sm100.cuh"
+
+namespace fk {
+namespace {
+
+
+template <int NP>
+struct AsgCfg {
+    static constexpr int kABytes = kBM * kBK * 2;  // 16 KB: one X plane chunk
+    static constexpr int kBBytes = kBN * kBK * 2;  // 32 KB: one centroid plane chunk
+    static constexpr int kStageBytes = NP * (kABytes + kBBytes);
+    static constexpr int kStages = NP == 2 ? 2 : 4;
+    static constexpr int kDataBytes = kStages * kStageBytes;  // 192 KB
+    static constexpr int kBarBytes = 256;
+    static constexpr int kSmemBytes = kDataBytes + kBarBytes + 1024;  // + alignment slack
+    static constexpr int kThreads = 192;
+    static constexpr int kTmemCols = 2 * kBN;  // two 256-column fp32 accumulators
+};
+
+__device__ __forceinline__ void raise_timeout(volatile uint32_t *abort_flag, uint32_t *err) {
+    *abort_flag = 1u;
+    err[0] = kErrTimeout;
+}
+
+// Warp-uniform bounded wait: lane 0 polls, the verdict is broadcast to the warp so every
+// lane takes the same path (the tcgen05.ld that follows is a warp-aligned instruction).
+__device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity,
+                                          volatile uint32_t *abort_flag, uint64_t wait_ns) {
+    uint32_t ok = 0;
+    if ((threadIdx.x & 31) == 0) ok = ptx::mbar_wait(bar, parity, abort_flag, wait_ns);
+    return __shfl_sync(0xffffffffu, ok, 0) != 0;
+}
+
+template <int NP>
+__global__ void __launch_bounds__(AsgCfg<NP>::kThreads, 1)
+    assign_kernel(const __grid_constant__ CUtensorMap tmA0,
+                  const __grid_constant__ CUtensorMap tmA1,
+                  const __grid_constant__ CUtensorMap tmB0,
+                  const __grid_constant__ CUtensorMap tmB1, const float *__restrict__ cn,
+                  int64_t N, int nkc, int ntiles, int64_t nmb, int32_t *__restrict__ labels,
+                  float *__restrict__ best_out, const float *__restrict__ xnorm,
+                  float *__restrict__ mind, uint32_t *__restrict__ err, uint64_t wait_ns) {
+    using Cfg = AsgCfg<NP>;
+    constexpr int S = Cfg::kStages;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + Cfg::kDataBytes);
+    uint64_t *empty = full + S;
+    uint64_t *tfull = empty + S;
+    uint64_t *tempty = tfull + 2;
+    uint64_t *drain = tempty + 2;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
+    volatile uint32_t *abort_flag = tmem_slot + 1;
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S; ++s) {
+            ptx::mbar_init(&full[s], 1);
+            ptx::mbar_init(&empty[s], 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            ptx::mbar_init(&tfull[a], 1);
+            ptx::mbar_init(&tempty[a], 4 * 32);
+        }
+        ptx::mbar_init(drain, 1);
+        *abort_flag = 0u;
+        ptx::fence_mbar_init();
+    }
+    if (warp == 0 && lane == 0) {
+        ptx::prefetch_tmap(&tmA0);
+        ptx::prefetch_tmap(&tmB0);
+        if (NP == 2) {
+            ptx::prefetch_tmap(&tmA1);
+            ptx::prefetch_tmap(&tmB1);
+        }
+    }
+    if (warp == 1) {
+        ptx::tmem_alloc(tmem_slot, Cfg::kTmemCols);
+        ptx::tmem_relinquish();
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            uint32_t stage = 0, phase = 0;
+            uint32_t issued_mask = 0, issued_par = 0;  // per stage: loaded at least once,
+                                                       // parity of the last load
+            bool ok = true;
+            for (int64_t mb = blockIdx.x; mb < nmb && ok; mb += gridDim.x) {
+                const int row0 = static_cast<int>(mb * kBM);
+                for (int nt = 0; nt < ntiles && ok; ++nt) {
+                    for (int kc = 0; kc < nkc; ++kc) {
+                        if (!ptx::mbar_wait(&empty[stage], phase ^ 1u, abort_flag, wait_ns)) {
+                            raise_timeout(abort_flag, err);
+                            ok = false;
+                            break;
+                        }
+                        ptx::mbar_arrive_expect_tx(&full[stage], Cfg::kStageBytes);
+                        uint8_t *st = smem + stage * Cfg::kStageBytes;
+                        ptx::tma_load_2d(st, &tmA0, &full[stage], kc * kBK, row0);
+                        if (NP == 2)
+                            ptx::tma_load_2d(st + Cfg::kABytes, &tmA1, &full[stage], kc * kBK,
+                                             row0);
+                        uint8_t *sb = st + NP * Cfg::kABytes;
+                        ptx::tma_load_2d(sb, &tmB0, &full[stage], kc * kBK, nt * kBN);
+                        if (NP == 2)
+                            ptx::tma_load_2d(sb + Cfg::kBBytes, &tmB1, &full[stage], kc * kBK,
+                                             nt * kBN);
+                        issued_mask |= 1u << stage;
+                        issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
+                        if (++stage == S) {
+                            stage = 0;
+                            phase ^= 1u;
+                        }
+                    }
+                }
+            }
+            if (!ok) {
+                // Let every load already issued land before the CTA can exit.
+                for (int s = 0; s < S; ++s)
+                    if (issued_mask & (1u << s))
+                        ptx::mbar_wait(&full[s], (issued_par >> s) & 1u, nullptr, wait_ns);
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc = ptx::idesc_bf16_f32(kBM, kBN);
+            uint32_t stage = 0, phase = 0, titer = 0;
+            bool ok = true;
+            for (int64_t mb = blockIdx.x; mb < nmb && ok; mb += gridDim.x) {
+                for (int nt = 0; nt < ntiles && ok; ++nt, ++titer) {
+                    const uint32_t acc = titer & 1u;
+                    const uint32_t aphase = (titer >> 1) & 1u;
+                    if (!ptx::mbar_wait(&tempty[acc], aphase ^ 1u, abort_flag, wait_ns)) {
+                        raise_timeout(abort_flag, err);
+                        ok = false;
+                        break;
+                    }
+                    ptx::tc_fence_after();
+                    const uint32_t dt = tmem + acc * kBN;
+                    for (int kc = 0; kc < nkc; ++kc) {
+                        if (!ptx::mbar_wait(&full[stage], phase, abort_flag, wait_ns)) {
+                            raise_timeout(abort_flag, err);
+                            ok = false;
+                            break;
+                        }
+                        ptx::tc_fence_after();
+                        const uint32_t a0 = ptx::smem_u32(smem + stage * Cfg::kStageBytes);
+                        const uint32_t a1 = a0 + Cfg::kABytes;
+                        const uint32_t b0 = a0 + NP * Cfg::kABytes;
+                        const uint32_t b1 = b0 + Cfg::kBBytes;
+#pragma unroll
+                        for (int ks = 0; ks < kBK / 16; ++ks) {
+                            const uint32_t off = ks * 32;  // 16 bf16 = 32 bytes along K
+                            ptx::mma_bf16_ss(dt, ptx::sdesc_k_sw128(a0 + off),
+                                             ptx::sdesc_k_sw128(b0 + off), idesc,
+                                             (kc | ks) != 0 ? 1u : 0u);
+                            if (NP == 2) {
+                                ptx::mma_bf16_ss(dt, ptx::sdesc_k_sw128(a1 + off),
+                                                 ptx::sdesc_k_sw128(b0 + off), idesc, 1u);
+                                ptx::mma_bf16_ss(dt, ptx::sdesc_k_sw128(a0 + off),
+                                                 ptx::sdesc_k_sw128(b1 + off), idesc, 1u);
+                            }
+                        }
+                        ptx::mma_commit(&empty[stage]);
+                        if (++stage == S) {
+                            stage = 0;
+                            phase ^= 1u;
+                        }
+                    }
+                    if (!ok) break;
+                    ptx::mma_commit(&tfull[acc]);
+                }
+            }
+            if (!ok) {
+                // Make sure no MMA issued by this thread is still writing tensor memory.
+                ptx::mma_commit(drain);
+                ptx::mbar_wait(drain, 0u, nullptr, wait_ns);
+            }
+        }
+    } else {
+        // ------------------------------------------------------------ epilogue
+        const int q = warp & 3;  // TMEM lane quarter this warp may access
+        const int r = q * 32 + lane;
+        uint32_t titer = 0;
+        bool ok = true;
+        for (int64_t mb = blockIdx.x; mb < nmb && ok; mb += gridDim.x) {
+            float best = __int_as_float(0x7f800000);
+            int bestk = 0;
+            for (int nt = 0; nt < ntiles; ++nt, ++titer) {
+                const uint32_t acc = titer & 1u;
+                const uint32_t aphase = (titer >> 1) & 1u;
+                if (!warp_wait(&tfull[acc], aphase, abort_flag, wait_ns)) {
+                    if (lane == 0) raise_timeout(abort_flag, err);
+                    ok = false;
+                    break;
+                }
+                ptx::tc_fence_after();
+                const uint32_t tbase = tmem + (static_cast<uint32_t>(q * 32) << 16) + acc * kBN;
+                const float4 *cn4 = reinterpret_cast<const float4 *>(cn + nt * kBN);
+#pragma unroll 1
+                for (int ch = 0; ch < kBN / 32; ++ch) {
+                    __syncwarp();
+                    float v[32];
+                    ptx::tmem_ld32_sync(tbase + ch * 32, v);
+#pragma unroll
+                    for (int j4 = 0; j4 < 8; ++j4) {
+                        const float4 c = __ldg(cn4 + ch * 8 + j4);
+                        v[4 * j4 + 0] += c.x;
+                        v[4 * j4 + 1] += c.y;
+                        v[4 * j4 + 2] += c.z;
+                        v[4 * j4 + 3] += c.w;
+                    }
+                    float m = v[0];
+#pragma unroll
+                    for (int j = 1; j < 32; ++j) m = fminf(m, v[j]);
+                    if (m < best) {
+                        int idx = 0;
+#pragma unroll
+                        for (int j = 31; j >= 0; --j)
+                            if (v[j] == m) idx = j;
+                        best = m;
+                        bestk = nt * kBN + ch * 32 + idx;
+                    }
+                }
+                ptx::tc_fence_before();
+                ptx::mbar_arrive(&tempty[acc]);
+            }
+            if (!ok) break;
+            const int64_t row = mb * kBM + r;
+            if (row < N) {
+                labels[row] = bestk;
+                if (best_out) best_out[row] = best;
+                if (mind) mind[row] = xnorm[row] + best;
+            }
+        }
+    }
+
+    // ---------------------------------------------------------------- teardown
+    ptx::tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        ptx::tc_fence_after();
+        ptx::tmem_dealloc(tmem, Cfg::kTmemCols);
+    }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 tmap_encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }
+    return fn;
+}
+
+// 2-D bf16 tensor map over a row-major [rows][cols] plane with the given row stride,
+// 64 x box_rows boxes, 128-byte swizzle; out-of-range rows/columns read as zero.
+bool make_tmap(CUtensorMap *m, const void *base, int64_t rows, int64_t cols,
+               int64_t row_stride_elems, int box_rows) {
+    auto fn = tmap_encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(row_stride_elems * 2)};
+    cuuint32_t box[2] = {static_cast<cuuint32_t>(kBK), static_cast<cuuint32_t>(box_rows)};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims,
+                    strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+template <int NP>
+cudaError_t launch_assign_np(const AssignArgs &a, cudaStream_t st) {
+    using Cfg = AsgCfg<NP>;
+    CUtensorMap tA[2], tB[2];
+    const uint16_t *ap = static_cast<const uint16_t *>(a.a_planes);
+    const uint16_t *bp = static_cast<const uint16_t *>(a.b_planes);
+    for (int p = 0; p < NP; ++p) {
+        if (!make_tmap(&tA[p], ap + p * a.N * a.lda, a.N, a.dp, a.lda, kBM))
+            return cudaErrorInvalidValue;
+        if (!make_tmap(&tB[p], bp + p * static_cast<int64_t>(a.Kp) * a.dp, a.Kp, a.dp, a.dp,
+                       kBN))
+            return cudaErrorInvalidValue;
+    }
+    if (NP == 1) {
+        tA[1] = tA[0];
+        tB[1] = tB[0];
+    }
+    static bool attr_set = false;
+    if (!attr_set) {
+        cudaError_t e = cudaFuncSetAttribute(
+            assign_kernel<NP>, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes);
+        if (e != cudaSuccess) return e;
+        attr_set = true;
+    }
+    const int64_t nmb = ceil_div(a.N, kBM);
+    const int64_t sms = device_sm_count();
+    const int grid = static_cast<int>(nmb < sms ? nmb : sms);
+    assign_kernel<NP><<<grid, Cfg::kThreads, Cfg::kSmemBytes, st>>>(
+        tA[0], tA[1], tB[0], tB[1], a.cn, a.N, static_cast<int>(a.dp / kBK),
+        static_cast<int>(a.Kp / kBN), nmb, a.labels, a.best, a.xnorm, a.mind, a.err,
+        a.wait_ns);
+    note_launch();
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_assign(const AssignArgs &a, cudaStream_t st) {
+    if (a.N <= 0) return cudaSuccess;
+    return a.a_nplanes == 2 ? launch_assign_np<2>(a, st) : launch_assign_np<1>(a, st);
+}
+
+}  // namespace fk

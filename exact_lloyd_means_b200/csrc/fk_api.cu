@@ -1,0 +1,414 @@
+// fk_api.cu -- the extern "C" boundary of libfk: argument validation, workspace carving,
+// stream plumbing and the Lloyd loop.  Every arithmetic step runs in the kernels of
+// prep.cu, assign_sm100.cu, sort_csr.cu and update.cu; this file only launches them.
+#include <cstring>
+#include <vector>
+
+#include "fk_common.cuh"
+#include "ptx_sm100.cuh"
+
+namespace fk {
+
+thread_local long g_launches = 0;
+
+int device_sm_count() {
+    static int cached[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+    if (dev >= 0 && dev < 64 && cached[dev]) return cached[dev];
+    int n = 148;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) n = 148;
+    if (dev >= 0 && dev < 64) cached[dev] = n;
+    return n;
+}
+
+namespace {
+
+constexpr uint64_t kDefaultWaitNs = 2000000000ull;  // 2 s bound on any in-kernel wait
+
+fk_status check_device() {
+    static int verdict[64] = {0};  // 0 unknown, 1 ok, 2 unsupported
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return FK_ERR_CUDA;
+    if (dev >= 0 && dev < 64 && verdict[dev]) return verdict[dev] == 1 ? FK_OK : FK_ERR_UNSUPPORTED;
+    int major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+        return FK_ERR_CUDA;
+    const bool ok = major == 10 && minor == 0;
+    if (dev >= 0 && dev < 64) verdict[dev] = ok ? 1 : 2;
+    return ok ? FK_OK : FK_ERR_UNSUPPORTED;
+}
+
+bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+fk_status validate_shape(int64_t N, int d, int K, fk_dtype dtype, fk_metric metric) {
+    if (N < 1 || N > 2147483647LL - 1) return FK_ERR_INVALID_ARG;
+    if (d < 1 || K < 1 || K > N) return FK_ERR_INVALID_ARG;
+    if (dtype != FK_F32 && dtype != FK_BF16) return FK_ERR_UNSUPPORTED;
+    if (metric != FK_L2 && metric != FK_COSINE) return FK_ERR_UNSUPPORTED;
+    if (dtype == FK_F32 && d % 4 != 0) return FK_ERR_UNSUPPORTED;
+    if (dtype == FK_BF16 && d % 8 != 0) return FK_ERR_UNSUPPORTED;
+    if (metric == FK_COSINE && dtype != FK_F32) return FK_ERR_UNSUPPORTED;
+    if (static_cast<int64_t>(K) * d > 2147483647LL) return FK_ERR_UNSUPPORTED;
+    return FK_OK;
+}
+
+fk_status check_ws(void *ws, size_t ws_bytes, const WsLayout &L) {
+    if (ws == nullptr || !aligned(ws, 256) || ws_bytes < L.total) return FK_ERR_WORKSPACE;
+    return FK_OK;
+}
+
+bool overlap(const void *a, size_t an, const void *b, size_t bn) {
+    const char *pa = static_cast<const char *>(a), *pb = static_cast<const char *>(b);
+    return pa < pb + bn && pb < pa + an;
+}
+
+#define FK_TRY_CUDA(expr)                              \
+    do {                                               \
+        if ((expr) != cudaSuccess) return FK_ERR_CUDA; \
+    } while (0)
+
+// The operand X planes the assign kernel reads, prepared from the (possibly normalised)
+// points.  Returns the planes pointer, plane count and row stride.
+fk_status prepare_x(const void *Xp, fk_dtype dtype, int64_t N, int d, const WsLayout &L,
+                    void *ws, float *xnorm, cudaStream_t st, const void **planes,
+                    int *nplanes, int64_t *lda) {
+    uint16_t *xs = ws_ptr<uint16_t>(ws, L.xs);
+    if (dtype == FK_F32) {
+        FK_TRY_CUDA(launch_split_x(static_cast<const float *>(Xp), N, d, L.dp, xs, xs + N * L.dp,
+                                   xnorm, st));
+        *planes = xs;
+        *nplanes = 2;
+        *lda = L.dp;
+    } else {
+        if (xnorm)
+            FK_TRY_CUDA(launch_xnorm_bf16(static_cast<const uint16_t *>(Xp), N, d, xnorm, st));
+        if (L.xplanes == 1) {
+            FK_TRY_CUDA(launch_pad_bf16(static_cast<const uint16_t *>(Xp), N, d, L.dp, xs, st));
+            *planes = xs;
+            *lda = L.dp;
+        } else {
+            *planes = Xp;
+            *lda = d;
+        }
+        *nplanes = 1;
+    }
+    return FK_OK;
+}
+
+fk_status run_assign(const void *planes, int nplanes, int64_t lda, int64_t N, int d, int K,
+                     const WsLayout &L, void *ws, int32_t *labels, const float *xnorm,
+                     float *mind, cudaStream_t st) {
+    AssignArgs a{};
+    a.a_planes = planes;
+    a.a_nplanes = nplanes;
+    a.lda = lda;
+    a.b_planes = ws_ptr<uint16_t>(ws, L.cs);
+    a.cn = ws_ptr<float>(ws, L.cn);
+    a.N = N;
+    a.d = d;
+    a.dp = static_cast<int>(L.dp);
+    a.K = K;
+    a.Kp = static_cast<int>(L.Kp);
+    a.labels = labels;
+    a.best = nullptr;
+    a.xnorm = xnorm;
+    a.mind = mind;
+    a.err = ws_ptr<uint32_t>(ws, L.err);
+    a.wait_ns = kDefaultWaitNs;
+    FK_TRY_CUDA(launch_assign(a, st));
+    return FK_OK;
+}
+
+fk_status run_update(const void *Xp, fk_dtype dtype, int64_t N, int d, int K,
+                     const WsLayout &L, void *ws, const int32_t *labels, const float *C_old,
+                     const float *C_used, float *C_new, int32_t *counts, int32_t *offsets,
+                     int32_t *perm_out, double *objective, cudaStream_t st) {
+    const int32_t *skeys = nullptr, *perm = nullptr;
+    FK_TRY_CUDA(launch_sort_csr(labels, N, K, L.sp, ws_ptr<int32_t>(ws, L.keys0),
+                                ws_ptr<int32_t>(ws, L.keys1), ws_ptr<int32_t>(ws, L.vals0),
+                                ws_ptr<int32_t>(ws, L.vals1), perm_out,
+                                ws_ptr<uint32_t>(ws, L.hist), ws_ptr<uint32_t>(ws, L.dtot),
+                                offsets, &skeys, &perm, ws_ptr<uint32_t>(ws, L.err), st));
+    FK_TRY_CUDA(launch_update(Xp, dtype, N, d, K, L.up, skeys, perm, offsets, C_old, C_used,
+                              C_new, counts, ws_ptr<double>(ws, L.pieces),
+                              ws_ptr<int32_t>(ws, L.pkeys), ws_ptr<double>(ws, L.piecesb),
+                              ws_ptr<int32_t>(ws, L.pkeysb), ws_ptr<double>(ws, L.jpart),
+                              objective, st));
+    return FK_OK;
+}
+
+// Read (and optionally clear) the two device error words after a stream sync.
+fk_status read_err(void *ws, const WsLayout &L, cudaStream_t st, bool clear, int *code) {
+    uint32_t e[2] = {0, 0};
+    uint32_t *dev = ws_ptr<uint32_t>(ws, L.err);
+    FK_TRY_CUDA(cudaMemcpyAsync(e, dev, sizeof(e), cudaMemcpyDeviceToHost, st));
+    if (clear) FK_TRY_CUDA(cudaMemsetAsync(dev, 0, sizeof(e), st));
+    FK_TRY_CUDA(cudaStreamSynchronize(st));
+    *code = e[0] ? FK_ERR_TIMEOUT : (e[1] ? FK_ERR_DEVICE : FK_OK);
+    return FK_OK;
+}
+
+// A kernel whose mbarrier is never arrived on: its bounded wait must expire and record
+// a timeout in the workspace error word (exercises the failure path without a fault).
+__global__ void wait_selftest_kernel(uint32_t *err, uint64_t limit_ns) {
+    __shared__ __align__(8) uint64_t bar;
+    if (threadIdx.x == 0) {
+        ptx::mbar_init(&bar, 1);
+        ptx::fence_mbar_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        if (!ptx::mbar_wait(&bar, 0u, nullptr, limit_ns)) err[0] = kErrTimeout;
+    }
+}
+
+}  // namespace
+}  // namespace fk
+
+using namespace fk;
+
+extern "C" {
+
+const char *fk_status_string(fk_status s) {
+    switch (s) {
+        case FK_OK: return "FK_OK";
+        case FK_ERR_INVALID_ARG: return "FK_ERR_INVALID_ARG";
+        case FK_ERR_UNSUPPORTED: return "FK_ERR_UNSUPPORTED";
+        case FK_ERR_WORKSPACE: return "FK_ERR_WORKSPACE";
+        case FK_ERR_CUDA: return "FK_ERR_CUDA";
+        case FK_ERR_TIMEOUT: return "FK_ERR_TIMEOUT";
+        case FK_ERR_DEVICE: return "FK_ERR_DEVICE";
+    }
+    return "FK_UNKNOWN_STATUS";
+}
+
+int fk_version(void) { return 1; }
+
+fk_status fk_workspace_size(int64_t N, int d, int K, fk_dtype dtype, fk_metric metric,
+                            size_t *bytes) {
+    if (!bytes) return FK_ERR_INVALID_ARG;
+    fk_status s = validate_shape(N, d, K, dtype, metric);
+    if (s != FK_OK) return s;
+    const size_t a = ws_layout(N, d, K, dtype, metric).total;
+    const size_t b = ws_layout(N, d, K, dtype, FK_L2).total;
+    *bytes = a > b ? a : b;
+    return FK_OK;
+}
+
+fk_status fk_normalize_rows(const float *X_in, float *X_out, int64_t N, int d,
+                            fk_stream_t stream) {
+    if (N < 0 || d < 1 || !X_in || !X_out) return FK_ERR_INVALID_ARG;
+    if (d % 4 != 0 || !aligned(X_in, 16) || !aligned(X_out, 16)) return FK_ERR_UNSUPPORTED;
+    if (N == 0) return FK_OK;
+    fk_status s = check_device();
+    if (s != FK_OK) return s;
+    FK_TRY_CUDA(launch_normalize(X_in, X_out, N, d, stream));
+    return FK_OK;
+}
+
+fk_status fk_centroid_norms(const float *C, int K, int d, fk_dtype dtype, float *cn,
+                            fk_stream_t stream) {
+    if (K < 1 || d < 1 || !C || !cn) return FK_ERR_INVALID_ARG;
+    if (dtype != FK_F32 && dtype != FK_BF16) return FK_ERR_UNSUPPORTED;
+    fk_status s = check_device();
+    if (s != FK_OK) return s;
+    FK_TRY_CUDA(launch_centroid_norms(C, K, d, dtype, cn, stream));
+    return FK_OK;
+}
+
+fk_status fk_assign(const void *X, fk_dtype dtype, int64_t N, int d, const float *C, int K,
+                    int32_t *labels, float *mind, void *ws, size_t ws_bytes,
+                    fk_stream_t stream) {
+    fk_status s = validate_shape(N, d, K, dtype, FK_L2);
+    if (s != FK_OK) return s;
+    if (!X || !C || !labels) return FK_ERR_INVALID_ARG;
+    if (!aligned(X, 16) || !aligned(C, 4) || !aligned(labels, 4) || (mind && !aligned(mind, 4)))
+        return FK_ERR_UNSUPPORTED;
+    const WsLayout L = ws_layout(N, d, K, dtype, FK_L2);
+    if ((s = check_ws(ws, ws_bytes, L)) != FK_OK) return s;
+    if ((s = check_device()) != FK_OK) return s;
+    cudaStream_t st = stream;
+    FK_TRY_CUDA(launch_prep_centroids(C, K, d, L.Kp, L.dp, dtype, ws_ptr<uint16_t>(ws, L.cs),
+                                      ws_ptr<float>(ws, L.cn), ws_ptr<float>(ws, L.cused), st));
+    float *xnorm = mind ? ws_ptr<float>(ws, L.xnorm) : nullptr;
+    const void *planes = nullptr;
+    int nplanes = 0;
+    int64_t lda = 0;
+    if ((s = prepare_x(X, dtype, N, d, L, ws, xnorm, st, &planes, &nplanes, &lda)) != FK_OK)
+        return s;
+    return run_assign(planes, nplanes, lda, N, d, K, L, ws, labels, xnorm, mind, st);
+}
+
+fk_status fk_update(const void *X, fk_dtype dtype, int64_t N, int d, int K,
+                    const int32_t *labels, const float *C_old, float *C_new, int32_t *counts,
+                    int32_t *offsets, int32_t *perm, double *objective, void *ws,
+                    size_t ws_bytes, fk_stream_t stream) {
+    fk_status s = validate_shape(N, d, K, dtype, FK_L2);
+    if (s != FK_OK) return s;
+    if (!X || !labels || !C_old || !C_new || !counts || !offsets) return FK_ERR_INVALID_ARG;
+    const size_t cbytes = sizeof(float) * static_cast<size_t>(K) * d;
+    if (overlap(C_old, cbytes, C_new, cbytes)) return FK_ERR_INVALID_ARG;
+    if (!aligned(X, 16) || !aligned(C_old, 16) || !aligned(C_new, 16) || !aligned(labels, 4) ||
+        !aligned(counts, 4) || !aligned(offsets, 4) || (perm && !aligned(perm, 4)) ||
+        (objective && !aligned(objective, 8)))
+        return FK_ERR_UNSUPPORTED;
+    const WsLayout L = ws_layout(N, d, K, dtype, FK_L2);
+    if ((s = check_ws(ws, ws_bytes, L)) != FK_OK) return s;
+    if ((s = check_device()) != FK_OK) return s;
+    cudaStream_t st = stream;
+    const float *C_used = C_old;
+    if (dtype == FK_BF16) {
+        FK_TRY_CUDA(launch_prep_centroids(C_old, K, d, L.Kp, L.dp, dtype,
+                                          ws_ptr<uint16_t>(ws, L.cs), ws_ptr<float>(ws, L.cn),
+                                          ws_ptr<float>(ws, L.cused), st));
+        C_used = ws_ptr<float>(ws, L.cused);
+    }
+    return run_update(X, dtype, N, d, K, L, ws, labels, C_old, C_used, C_new, counts, offsets,
+                      perm, objective, st);
+}
+
+fk_status fk_lloyd(const void *X, fk_dtype dtype, int64_t N, int d, int K, fk_metric metric,
+                   int niter, float *C, int32_t *labels, int32_t *counts, int32_t *offsets,
+                   double *objective_host, fk_timing *timing, void *ws, size_t ws_bytes,
+                   fk_stream_t stream) {
+    fk_status s = validate_shape(N, d, K, dtype, metric);
+    if (s != FK_OK) return s;
+    if (!X || !C || !labels || niter < 0) return FK_ERR_INVALID_ARG;
+    if (!aligned(X, 16) || !aligned(C, 16) || !aligned(labels, 4) ||
+        (counts && !aligned(counts, 4)) || (offsets && !aligned(offsets, 4)))
+        return FK_ERR_UNSUPPORTED;
+    const WsLayout L = ws_layout(N, d, K, dtype, metric);
+    if ((s = check_ws(ws, ws_bytes, L)) != FK_OK) return s;
+    if ((s = check_device()) != FK_OK) return s;
+    cudaStream_t st = stream;
+
+    // events: [0] start, [1] after setup, then 4 per iteration
+    std::vector<cudaEvent_t> ev;
+    auto rec = [&]() -> bool {
+        if (!timing) return true;
+        cudaEvent_t e;
+        if (cudaEventCreate(&e) != cudaSuccess) return false;
+        ev.push_back(e);
+        return cudaEventRecord(e, st) == cudaSuccess;
+    };
+    auto cleanup = [&]() {
+        for (auto e : ev) cudaEventDestroy(e);
+    };
+    auto fail = [&](fk_status f) {
+        cleanup();
+        return f;
+    };
+
+    if (cudaMemsetAsync(ws_ptr<uint32_t>(ws, L.err), 0, 2 * sizeof(uint32_t), st) != cudaSuccess)
+        return FK_ERR_CUDA;
+    const long launches0 = g_launches;
+    if (!rec()) return fail(FK_ERR_CUDA);
+    const void *Xp = X;
+    if (metric == FK_COSINE) {
+        float *xn = ws_ptr<float>(ws, L.xn);
+        if (launch_normalize(static_cast<const float *>(X), xn, N, d, st) != cudaSuccess ||
+            launch_normalize(C, C, K, d, st) != cudaSuccess)
+            return fail(FK_ERR_CUDA);
+        Xp = xn;
+    }
+    const void *planes = nullptr;
+    int nplanes = 0;
+    int64_t lda = 0;
+    if (niter > 0 &&
+        (s = prepare_x(Xp, dtype, N, d, L, ws, nullptr, st, &planes, &nplanes, &lda)) != FK_OK)
+        return fail(s);
+    if (!rec()) return fail(FK_ERR_CUDA);
+
+    float *Ccur = C, *Cnext = ws_ptr<float>(ws, L.calt);
+    int32_t *cnt = counts ? counts : ws_ptr<int32_t>(ws, L.cnt);
+    int32_t *off = offsets ? offsets : ws_ptr<int32_t>(ws, L.off);
+    double *obj = ws_ptr<double>(ws, L.obj);
+    float *cused = ws_ptr<float>(ws, L.cused);
+    int copied = 0;
+    for (int t = 0; t < niter; ++t) {
+        if (launch_prep_centroids(Ccur, K, d, L.Kp, L.dp, dtype, ws_ptr<uint16_t>(ws, L.cs),
+                                  ws_ptr<float>(ws, L.cn), cused, st) != cudaSuccess)
+            return fail(FK_ERR_CUDA);
+        if (!rec()) return fail(FK_ERR_CUDA);
+        if ((s = run_assign(planes, nplanes, lda, N, d, K, L, ws, labels, nullptr, nullptr,
+                            st)) != FK_OK)
+            return fail(s);
+        if (!rec()) return fail(FK_ERR_CUDA);
+        const int32_t *skeys = nullptr, *perm = nullptr;
+        if (launch_sort_csr(labels, N, K, L.sp, ws_ptr<int32_t>(ws, L.keys0),
+                            ws_ptr<int32_t>(ws, L.keys1), ws_ptr<int32_t>(ws, L.vals0),
+                            ws_ptr<int32_t>(ws, L.vals1), nullptr,
+                            ws_ptr<uint32_t>(ws, L.hist), ws_ptr<uint32_t>(ws, L.dtot), off,
+                            &skeys, &perm, ws_ptr<uint32_t>(ws, L.err), st) != cudaSuccess)
+            return fail(FK_ERR_CUDA);
+        if (!rec()) return fail(FK_ERR_CUDA);
+        if (launch_update(Xp, dtype, N, d, K, L.up, skeys, perm, off, Ccur,
+                          dtype == FK_F32 ? Ccur : cused, Cnext, cnt,
+                          ws_ptr<double>(ws, L.pieces), ws_ptr<int32_t>(ws, L.pkeys),
+                          ws_ptr<double>(ws, L.piecesb), ws_ptr<int32_t>(ws, L.pkeysb),
+                          ws_ptr<double>(ws, L.jpart), obj + (t % kObjRing), st) != cudaSuccess)
+            return fail(FK_ERR_CUDA);
+        if (!rec()) return fail(FK_ERR_CUDA);
+        float *tmp = Ccur;
+        Ccur = Cnext;
+        Cnext = tmp;
+        if (objective_host && (t + 1) % kObjRing == 0) {
+            if (cudaMemcpyAsync(objective_host + copied, obj, sizeof(double) * kObjRing,
+                                cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+                cudaStreamSynchronize(st) != cudaSuccess)
+                return fail(FK_ERR_CUDA);
+            copied += kObjRing;
+        }
+    }
+    if (Ccur != C &&
+        cudaMemcpyAsync(C, Ccur, sizeof(float) * static_cast<size_t>(K) * d,
+                        cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+        return fail(FK_ERR_CUDA);
+    if (objective_host && niter > copied &&
+        cudaMemcpyAsync(objective_host + copied, obj, sizeof(double) * (niter - copied),
+                        cudaMemcpyDeviceToHost, st) != cudaSuccess)
+        return fail(FK_ERR_CUDA);
+    int code = FK_OK;
+    if (read_err(ws, L, st, true, &code) != FK_OK) return fail(FK_ERR_CUDA);
+    if (timing && ev.size() >= 2) {
+        float ms = 0.f;
+        std::memset(timing, 0, sizeof(*timing));
+        cudaEventElapsedTime(&ms, ev[0], ev[1]);
+        timing->ms_setup = ms;
+        double *slot[4] = {&timing->ms_prep, &timing->ms_assign, &timing->ms_sort,
+                           &timing->ms_update};
+        for (int t = 0; t < niter; ++t) {
+            for (int p = 0; p < 4; ++p) {
+                const size_t a = 1 + 4 * t + p;
+                if (a + 1 < ev.size() && cudaEventElapsedTime(&ms, ev[a], ev[a + 1]) == cudaSuccess)
+                    *slot[p] += ms;
+            }
+        }
+        timing->iterations = niter;
+        timing->launches = static_cast<int>(g_launches - launches0);
+    }
+    cleanup();
+    return static_cast<fk_status>(code);
+}
+
+fk_status fk_get_device_error(void *ws, size_t ws_bytes, int *code, fk_stream_t stream) {
+    if (!ws || !code || ws_bytes < 256 || !aligned(ws, 256)) return FK_ERR_INVALID_ARG;
+    WsLayout L;
+    L.err = 0;
+    return read_err(ws, L, stream, true, code);
+}
+
+fk_status fk_selftest_timeout(void *ws, size_t ws_bytes, uint64_t limit_ns,
+                              fk_stream_t stream) {
+    if (!ws || ws_bytes < 256 || !aligned(ws, 256)) return FK_ERR_INVALID_ARG;
+    fk_status s = check_device();
+    if (s != FK_OK) return s;
+    if (limit_ns > 10000000000ull) return FK_ERR_INVALID_ARG;
+    wait_selftest_kernel<<<1, 32, 0, stream>>>(static_cast<uint32_t *>(ws), limit_ns);
+    note_launch();
+    return cudaGetLastError() == cudaSuccess ? FK_OK : FK_ERR_CUDA;
+}
+
+}  // extern "C"

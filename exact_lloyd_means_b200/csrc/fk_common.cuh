@@ -1,0 +1,193 @@
+// fk_common.cuh -- constants, workspace layout and small helpers shared by the kernels
+// and the C-ABI host code of libfk.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "../../include/fk.h"
+
+namespace fk {
+
+// ----------------------------------------------------------------- assign tiling
+constexpr int kBM = 128;  // rows of X per tile (one TMEM lane per row)
+constexpr int kBN = 256;  // centroids per tile (fp32 accumulator columns)
+constexpr int kBK = 64;   // bf16 elements per 128-byte swizzle row
+
+// ----------------------------------------------------------------- sort tiling
+constexpr int kSortThreads = 256;
+constexpr int kSortItems = 16;
+constexpr int kSortTile = kSortThreads * kSortItems;  // keys per block
+constexpr int kSortMaxBits = 11;                      // digit width bound: 2048 bins
+
+// ----------------------------------------------------------------- update tiling
+constexpr int kRowsPerWarp = 512;  // sorted positions per warp chunk
+constexpr int kUpdWarps = 8;
+constexpr int kMaxSlices = 8;      // 128-column slices per lane group (d <= 1024 per pass)
+
+// Objective slots kept on the device by fk_lloyd before a copy to the host.
+constexpr int kObjRing = 4096;
+
+// Device error word bits (workspace offset 0).
+constexpr uint32_t kErrTimeout = 1u;
+constexpr uint32_t kErrLabel = 2u;
+
+inline int64_t round_up(int64_t a, int64_t b) { return (a + b - 1) / b * b; }
+inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+inline int key_bits(int K) {
+    if (K <= 1) return 0;
+    unsigned v = static_cast<unsigned>(K - 1);
+    int b = 0;
+    while (v) {
+        ++b;
+        v >>= 1;
+    }
+    return b;
+}
+
+struct SortPlan {
+    int nbits = 0;
+    int passes = 0;
+    int bits = 0;  // digit width per pass (last pass may use fewer significant bits)
+    int64_t nblocks = 0;
+};
+
+inline SortPlan sort_plan(int64_t N, int K) {
+    SortPlan p;
+    p.nbits = key_bits(K);
+    p.passes = p.nbits == 0 ? 0 : static_cast<int>(ceil_div(p.nbits, kSortMaxBits));
+    p.bits = p.passes == 0 ? 0 : static_cast<int>(ceil_div(p.nbits, p.passes));
+    p.nblocks = ceil_div(N, kSortTile);
+    return p;
+}
+
+struct UpdPlan {
+    int slices = 1;    // 128-column slices per pass
+    int ncolblk = 1;   // column passes
+    int dcov = 128;    // padded row length covered by the passes
+    int64_t nwarps = 0;
+};
+
+inline UpdPlan upd_plan(int64_t N, int d) {
+    UpdPlan p;
+    int sl = static_cast<int>(ceil_div(d, 128));
+    p.slices = sl < kMaxSlices ? sl : kMaxSlices;
+    p.ncolblk = static_cast<int>(ceil_div(d, 128 * p.slices));
+    p.dcov = p.ncolblk * 128 * p.slices;
+    p.nwarps = ceil_div(N, kRowsPerWarp);
+    return p;
+}
+
+// Byte offsets of every scratch buffer inside the caller's workspace (256-byte aligned).
+struct WsLayout {
+    size_t err = 0, obj = 0, xn = 0, xs = 0, xnorm = 0, cs = 0, cn = 0, cused = 0,
+           calt = 0, keys0 = 0, keys1 = 0, vals0 = 0, vals1 = 0, hist = 0, dtot = 0,
+           pieces = 0, pkeys = 0, piecesb = 0, pkeysb = 0, jpart = 0, jdev = 0, cnt = 0,
+           off = 0, total = 0;
+    int64_t dp = 0, Kp = 0;
+    int xplanes = 0;  // bf16 planes of X prepared in the workspace (0, 1 or 2)
+    int cplanes = 0;  // bf16 planes of the centroids (1 or 2)
+    SortPlan sp;
+    UpdPlan up;
+};
+
+inline WsLayout ws_layout(int64_t N, int d, int K, fk_dtype dtype, fk_metric metric) {
+    WsLayout L;
+    L.dp = round_up(d, kBK);
+    L.Kp = round_up(K, kBN);
+    L.cplanes = dtype == FK_F32 ? 2 : 1;
+    L.xplanes = dtype == FK_F32 ? 2 : ((d % kBK) != 0 ? 1 : 0);
+    L.sp = sort_plan(N, K);
+    L.up = upd_plan(N, d);
+    size_t o = 0;
+    auto take = [&](size_t bytes) {
+        size_t at = o;
+        o += static_cast<size_t>(round_up(static_cast<int64_t>(bytes > 0 ? bytes : 1), 256));
+        return at;
+    };
+    L.err = take(256);
+    L.obj = take(sizeof(double) * kObjRing);
+    L.xn = take(metric == FK_COSINE ? sizeof(float) * N * d : 0);
+    L.xs = take(sizeof(uint16_t) * L.xplanes * N * L.dp);
+    L.xnorm = take(sizeof(float) * N);
+    L.cs = take(sizeof(uint16_t) * L.cplanes * L.Kp * L.dp);
+    L.cn = take(sizeof(float) * L.Kp);
+    L.cused = take(sizeof(float) * K * d);
+    L.calt = take(sizeof(float) * K * d);
+    L.keys0 = take(sizeof(int32_t) * N);
+    L.keys1 = take(sizeof(int32_t) * N);
+    L.vals0 = take(sizeof(int32_t) * N);
+    L.vals1 = take(sizeof(int32_t) * N);
+    const int64_t bins = int64_t(1) << (L.sp.bits > 0 ? L.sp.bits : 1);
+    L.hist = take(sizeof(uint32_t) * bins * L.sp.nblocks);
+    L.dtot = take(sizeof(uint32_t) * bins);
+    L.pieces = take(sizeof(double) * L.up.nwarps * 2 * L.up.dcov);
+    L.pkeys = take(sizeof(int32_t) * L.up.nwarps * 2);
+    const int64_t units2 = ceil_div(L.up.nwarps, 64) + 1;
+    L.piecesb = take(sizeof(double) * units2 * 2 * L.up.dcov);
+    L.pkeysb = take(sizeof(int32_t) * units2 * 2);
+    L.jpart = take(sizeof(double) * L.up.nwarps * L.up.ncolblk);
+    L.jdev = take(sizeof(double) * 2);
+    L.cnt = take(sizeof(int32_t) * K);
+    L.off = take(sizeof(int32_t) * (K + 1));
+    L.total = o;
+    return L;
+}
+
+template <typename T>
+inline T *ws_ptr(void *ws, size_t off) {
+    return reinterpret_cast<T *>(static_cast<char *>(ws) + off);
+}
+
+// ----------------------------------------------------------------- launch helpers
+// (declared here, defined in the .cu files)
+struct AssignArgs {
+    const void *a_planes;  // bf16 X planes: [xplanes][N][lda]
+    int a_nplanes;         // 2 = hi/lo (fp32 emulation), 1 = bf16
+    int64_t lda;           // row stride of an X plane, elements
+    const void *b_planes;  // bf16 centroid planes [cplanes][Kp][dp], scaled by -2
+    const float *cn;       // [Kp], +inf beyond K
+    int64_t N;
+    int d, dp, K, Kp;
+    int32_t *labels;
+    float *best;           // optional [N]: min_k (cn_k - 2 x.c_k)
+    const float *xnorm;    // optional [N]: ||x||^2, with mind
+    float *mind;           // optional [N]
+    uint32_t *err;         // workspace error words
+    uint64_t wait_ns;      // bound on every mbarrier wait inside the kernel
+};
+
+cudaError_t launch_split_x(const float *X, int64_t N, int d, int64_t dp, uint16_t *hi,
+                           uint16_t *lo, float *xnorm, cudaStream_t st);
+cudaError_t launch_pad_bf16(const uint16_t *X, int64_t N, int d, int64_t dp, uint16_t *out,
+                            cudaStream_t st);
+cudaError_t launch_normalize(const float *X, float *Y, int64_t N, int d, cudaStream_t st);
+cudaError_t launch_xnorm_bf16(const uint16_t *X, int64_t N, int d, float *xnorm,
+                              cudaStream_t st);
+cudaError_t launch_prep_centroids(const float *C, int K, int d, int64_t Kp, int64_t dp,
+                                  fk_dtype dtype, uint16_t *planes, float *cn, float *cused,
+                                  cudaStream_t st);
+cudaError_t launch_centroid_norms(const float *C, int K, int d, fk_dtype dtype, float *cn,
+                                  cudaStream_t st);
+cudaError_t launch_assign(const AssignArgs &a, cudaStream_t st);
+cudaError_t launch_sort_csr(const int32_t *labels, int64_t N, int K, const SortPlan &sp,
+                            int32_t *keys0, int32_t *keys1, int32_t *vals0, int32_t *vals1,
+                            int32_t *perm_out, uint32_t *hist, uint32_t *dtot,
+                            int32_t *offsets, const int32_t **sorted_keys,
+                            const int32_t **perm, uint32_t *err, cudaStream_t st);
+cudaError_t launch_update(const void *X, fk_dtype dtype, int64_t N, int d, int K,
+                          const UpdPlan &up, const int32_t *skeys, const int32_t *perm,
+                          const int32_t *offsets, const float *C_old, const float *C_used,
+                          float *C_new, int32_t *counts, double *pieces_a, int32_t *pkeys_a,
+                          double *pieces_b, int32_t *pkeys_b, double *jpart,
+                          double *objective, cudaStream_t st);
+
+int device_sm_count();
+
+// Kernels launched by this host thread since the last reset (fk_lloyd reports it).
+extern thread_local long g_launches;
+inline void note_launch(int n = 1) { g_launches += n; }
+
+}  // namespace fk

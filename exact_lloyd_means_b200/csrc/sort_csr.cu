@@ -1,0 +1,293 @@
+// sort_csr.cu -- labels -> sorted inverse index (perm) + CSR cluster offsets.
+//
+// Flash-KMeans article, section "Sort-Inverse Update：原子操作的另一种解法": the
+// assignments are sorted by cluster id into an inverse index so that each cluster's
+// points can be read contiguously; LEANN FlashLib guide, section "工作原理": the coarse
+// quantizer's output is CSR offsets plus cell-ordered row ids.
+//
+// A stable least-significant-digit radix sort with digits of up to 11 bits (one pass for
+// K <= 2048, two for K <= 2^22), written without atomics:
+//   upsweep   : each block of 4096 keys counts its digits; every warp keeps a private
+//               histogram in shared memory that only the elected leader of each group of
+//               equal digits (__match_any_sync) updates, so no two lanes write one counter;
+//   scan      : one block per digit scans the per-block counts (digit-major order) and
+//               stores the digit total;
+//   downsweep : each block recounts, turns warp counts into exclusive offsets (digits in
+//               order, then blocks in order, then warps in order) and scatters every key
+//               to base + rank, rank = #equal digits before it in the warp (popc of the
+//               match mask below the lane).  Keys are visited in index order, so the sort
+//               is stable and the output is unique.
+// offsets[k] = first sorted position whose key is >= k, written once per k.
+#include "fk_common.cuh"
+
+namespace fk {
+namespace {
+
+constexpr int kWarps = kSortThreads / 32;
+
+__device__ __forceinline__ uint32_t lanemask_lt() {
+    uint32_t m;
+    asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
+    return m;
+}
+
+// Check labels (first pass) and count digits of one 4096-key tile into per-warp
+// histograms wh[kWarps][bins].
+__device__ __forceinline__ void count_tile(const int32_t *__restrict__ keys, int64_t n,
+                                           int64_t tile0, int shift, uint32_t mask, int K,
+                                           uint32_t *__restrict__ err, int check,
+                                           uint32_t *wh, int bins) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    uint32_t *h = wh + warp * bins;
+    const int64_t base = tile0 + static_cast<int64_t>(warp) * (32 * kSortItems);
+    for (int step = 0; step < kSortItems; ++step) {
+        const int64_t idx = base + step * 32 + lane;
+        const bool valid = idx < n;
+        int key = valid ? keys[idx] : 0;
+        if (check && valid && (key < 0 || key >= K)) {
+            err[1] = 1u;
+            key = key < 0 ? 0 : K - 1;
+        }
+        const uint32_t digit = (static_cast<uint32_t>(key) >> shift) & mask;
+        const uint32_t vmask = __ballot_sync(0xffffffffu, valid);
+        if (valid) {
+            const uint32_t peers = __match_any_sync(vmask, digit);
+            if (lane == __ffs(peers) - 1) h[digit] += __popc(peers);
+        }
+        __syncwarp();
+    }
+}
+
+__global__ void __launch_bounds__(kSortThreads)
+    upsweep_kernel(const int32_t *__restrict__ keys, int64_t n, int shift, int bits, int K,
+                   uint32_t *__restrict__ hist, int64_t nblocks, uint32_t *__restrict__ err,
+                   int check) {
+    extern __shared__ uint32_t wh[];
+    const int bins = 1 << bits;
+    for (int i = threadIdx.x; i < kWarps * bins; i += blockDim.x) wh[i] = 0;
+    __syncthreads();
+    count_tile(keys, n, static_cast<int64_t>(blockIdx.x) * kSortTile, shift, bins - 1, K, err,
+               check, wh, bins);
+    __syncthreads();
+    for (int b = threadIdx.x; b < bins; b += blockDim.x) {
+        uint32_t t = 0;
+        for (int w = 0; w < kWarps; ++w) t += wh[w * bins + b];
+        hist[static_cast<int64_t>(b) * nblocks + blockIdx.x] = t;
+    }
+}
+
+// Exclusive scan of 1024 per-thread values held in registers; returns the exclusive
+// prefix of this thread and writes the block total to *total.
+__device__ __forceinline__ uint32_t block_exclusive_scan_1024(uint32_t v, uint32_t *sh,
+                                                              uint32_t *total) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    uint32_t x = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+    }
+    if (lane == 31) sh[warp] = x;
+    __syncthreads();
+    if (warp == 0) {
+        uint32_t w = lane < (blockDim.x >> 5) ? sh[lane] : 0;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t y = __shfl_up_sync(0xffffffffu, w, o);
+            if (lane >= o) w += y;
+        }
+        sh[32 + lane] = w;  // inclusive warp totals
+    }
+    __syncthreads();
+    const uint32_t warp_base = warp == 0 ? 0 : sh[32 + warp - 1];
+    *total = sh[32 + (blockDim.x >> 5) - 1];
+    return warp_base + x - v;
+}
+
+// One block (1024 threads) per digit: exclusive scan of hist[b][0..nblocks).
+__global__ void __launch_bounds__(1024)
+    scan_rows_kernel(uint32_t *__restrict__ hist, int64_t nblocks, uint32_t *__restrict__ dtot) {
+    __shared__ uint32_t sh[64];
+    uint32_t *row = hist + static_cast<int64_t>(blockIdx.x) * nblocks;
+    const int64_t per = (nblocks + blockDim.x - 1) / blockDim.x;
+    const int64_t lo = threadIdx.x * per;
+    const int64_t hi = lo + per < nblocks ? lo + per : nblocks;
+    uint32_t s = 0;
+    for (int64_t i = lo; i < hi; ++i) s += row[i];
+    uint32_t total;
+    uint32_t run = block_exclusive_scan_1024(s, sh, &total);
+    for (int64_t i = lo; i < hi; ++i) {
+        const uint32_t t = row[i];
+        row[i] = run;
+        run += t;
+    }
+    if (threadIdx.x == 0) dtot[blockIdx.x] = total;
+}
+
+__global__ void __launch_bounds__(kSortThreads)
+    downsweep_kernel(const int32_t *__restrict__ kin, const int32_t *__restrict__ vin,
+                     int32_t *__restrict__ kout, int32_t *__restrict__ vout, int64_t n,
+                     int shift, int bits, int K, const uint32_t *__restrict__ hist,
+                     const uint32_t *__restrict__ dtot, int64_t nblocks) {
+    extern __shared__ uint32_t sm[];
+    const int bins = 1 << bits;
+    const uint32_t mask = bins - 1;
+    uint32_t *wh = sm;                   // [kWarps][bins]
+    uint32_t *dbase = sm + kWarps * bins;  // [bins] exclusive scan of digit totals
+    __shared__ uint32_t part[kSortThreads];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    for (int i = threadIdx.x; i < kWarps * bins; i += blockDim.x) wh[i] = 0;
+    // digit bases: thread t scans a contiguous run of digits, then the runs are combined
+    {
+        const int per = (bins + kSortThreads - 1) / kSortThreads;
+        const int lo = threadIdx.x * per;
+        const int hi = lo + per < bins ? lo + per : bins;
+        uint32_t s = 0;
+        for (int b = lo; b < hi; ++b) s += dtot[b];
+        part[threadIdx.x] = s;
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            uint32_t run = 0;
+            for (int t = 0; t < kSortThreads; ++t) {
+                const uint32_t v = part[t];
+                part[t] = run;
+                run += v;
+            }
+        }
+        __syncthreads();
+        uint32_t run = part[threadIdx.x];
+        for (int b = lo; b < hi; ++b) {
+            dbase[b] = run;
+            run += dtot[b];
+        }
+    }
+    __syncthreads();
+
+    const int64_t tile0 = static_cast<int64_t>(blockIdx.x) * kSortTile;
+    count_tile(kin, n, tile0, shift, mask, K, nullptr, 0, wh, bins);
+    __syncthreads();
+    for (int b = threadIdx.x; b < bins; b += blockDim.x) {
+        uint32_t run = dbase[b] + hist[static_cast<int64_t>(b) * nblocks + blockIdx.x];
+        for (int w = 0; w < kWarps; ++w) {
+            const uint32_t t = wh[w * bins + b];
+            wh[w * bins + b] = run;
+            run += t;
+        }
+    }
+    __syncthreads();
+
+    uint32_t *h = wh + warp * bins;
+    const uint32_t lt = lanemask_lt();
+    const int64_t base = tile0 + static_cast<int64_t>(warp) * (32 * kSortItems);
+    for (int step = 0; step < kSortItems; ++step) {
+        const int64_t idx = base + step * 32 + lane;
+        const bool valid = idx < n;
+        int key = 0, val = 0;
+        if (valid) {
+            key = kin[idx];
+            key = key < 0 ? 0 : (key >= K ? K - 1 : key);
+            val = vin ? vin[idx] : static_cast<int32_t>(idx);
+        }
+        const uint32_t digit = (static_cast<uint32_t>(key) >> shift) & mask;
+        const uint32_t vmask = __ballot_sync(0xffffffffu, valid);
+        uint32_t peers = 0, pos = 0;
+        if (valid) {
+            peers = __match_any_sync(vmask, digit);
+            pos = h[digit] + __popc(peers & lt);
+        }
+        __syncwarp();
+        if (valid) {
+            if (lane == __ffs(peers) - 1) h[digit] += __popc(peers);
+            kout[pos] = key;
+            vout[pos] = val;
+        }
+        __syncwarp();
+    }
+}
+
+// K == 1: nothing to sort; check the labels and emit the identity permutation.
+__global__ void single_cluster_kernel(const int32_t *__restrict__ labels, int64_t n,
+                                      int32_t *__restrict__ kout, int32_t *__restrict__ vout,
+                                      uint32_t *__restrict__ err) {
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+         i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        if (labels[i] != 0) err[1] = 1u;
+        kout[i] = 0;
+        vout[i] = static_cast<int32_t>(i);
+    }
+}
+
+// offsets[k] = first position p with skeys[p] >= k (offsets[K] = n): position i writes
+// every k in (skeys[i-1], skeys[i]], so each entry is written exactly once.
+__global__ void csr_offsets_kernel(const int32_t *__restrict__ skeys, int64_t n, int K,
+                                   int32_t *__restrict__ offsets) {
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i <= n;
+         i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const int prev = i == 0 ? -1 : skeys[i - 1];
+        const int cur = i == n ? K : skeys[i];
+        for (int k = prev + 1; k <= cur; ++k) offsets[k] = static_cast<int32_t>(i);
+    }
+}
+
+int grid_cap(int64_t items, int threads) {
+    int64_t g = (items + threads - 1) / threads;
+    const int64_t cap = static_cast<int64_t>(device_sm_count()) * 32;
+    if (g > cap) g = cap;
+    return static_cast<int>(g < 1 ? 1 : g);
+}
+
+}  // namespace
+
+cudaError_t launch_sort_csr(const int32_t *labels, int64_t N, int K, const SortPlan &sp,
+                            int32_t *keys0, int32_t *keys1, int32_t *vals0, int32_t *vals1,
+                            int32_t *perm_out, uint32_t *hist, uint32_t *dtot,
+                            int32_t *offsets, const int32_t **sorted_keys,
+                            const int32_t **perm, uint32_t *err, cudaStream_t st) {
+    if (sp.passes == 0) {
+        int32_t *vo = perm_out ? perm_out : vals0;
+        single_cluster_kernel<<<grid_cap(N, 256), 256, 0, st>>>(labels, N, keys0, vo, err);
+        note_launch();
+        *sorted_keys = keys0;
+        *perm = vo;
+    } else {
+        const int bins = 1 << sp.bits;
+        const size_t up_smem = sizeof(uint32_t) * kWarps * bins;
+        const size_t dn_smem = sizeof(uint32_t) * (kWarps + 1) * bins;
+        static bool attr = false;
+        if (!attr) {
+            const int maxb = 1 << kSortMaxBits;
+            cudaFuncSetAttribute(upsweep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(sizeof(uint32_t) * kWarps * maxb));
+            cudaFuncSetAttribute(downsweep_kernel,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(sizeof(uint32_t) * (kWarps + 1) * maxb));
+            attr = true;
+        }
+        const int32_t *kin = labels;
+        const int32_t *vin = nullptr;
+        int32_t *kb[2] = {keys0, keys1};
+        int32_t *vb[2] = {vals0, vals1};
+        for (int p = 0; p < sp.passes; ++p) {
+            const int shift = p * sp.bits;
+            upsweep_kernel<<<static_cast<unsigned>(sp.nblocks), kSortThreads, up_smem, st>>>(
+                kin, N, shift, sp.bits, K, hist, sp.nblocks, err, p == 0 ? 1 : 0);
+            note_launch();
+            scan_rows_kernel<<<bins, 1024, 0, st>>>(hist, sp.nblocks, dtot);
+            note_launch();
+            int32_t *vo = (p == sp.passes - 1 && perm_out) ? perm_out : vb[p & 1];
+            downsweep_kernel<<<static_cast<unsigned>(sp.nblocks), kSortThreads, dn_smem, st>>>(
+                kin, vin, kb[p & 1], vo, N, shift, sp.bits, K, hist, dtot, sp.nblocks);
+            note_launch();
+            kin = kb[p & 1];
+            vin = vo;
+        }
+        *sorted_keys = kin;
+        *perm = vin;
+    }
+    csr_offsets_kernel<<<grid_cap(N + 1, 256), 256, 0, st>>>(*sorted_keys, N, K, offsets);
+    note_launch();
+    return cudaGetLastError();
+}
+
+}  // namespace fk

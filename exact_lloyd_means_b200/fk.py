@@ -1,0 +1,223 @@
+"""ctypes binding of libfk.so, the C-ABI CUDA library (include/fk.h).
+
+Argument marshalling only: every function here checks tensor dtypes, shapes, devices and
+contiguity, passes raw device pointers, sizes and the current CUDA stream to the function
+of the same name in libfk.so, and raises FkError on a non-zero status.  All arithmetic
+runs in the library's sm_100a kernels; PyTorch only provides device memory and streams.
+Importing this module fails loudly when libfk.so has not been built.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libfk.so")
+
+FK_OK, FK_ERR_INVALID_ARG, FK_ERR_UNSUPPORTED, FK_ERR_WORKSPACE = 0, 1, 2, 3
+FK_ERR_CUDA, FK_ERR_TIMEOUT, FK_ERR_DEVICE = 4, 5, 6
+FK_F32, FK_BF16 = 0, 1
+FK_L2, FK_COSINE = 0, 1
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"{LIB_PATH} is missing: build the CUDA library first "
+        "(python -c 'import __graft_entry__; __graft_entry__.build()' or "
+        "python exact_lloyd_means_b200/build.py)")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+_vp, _i64, _int, _sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
+
+
+class FkTiming(ctypes.Structure):
+    _fields_ = [("ms_setup", ctypes.c_double), ("ms_prep", ctypes.c_double),
+                ("ms_assign", ctypes.c_double), ("ms_sort", ctypes.c_double),
+                ("ms_update", ctypes.c_double), ("iterations", ctypes.c_int),
+                ("launches", ctypes.c_int)]
+
+
+def _sig(name, args, res=ctypes.c_int):
+    f = getattr(_lib, name)
+    f.argtypes = args
+    f.restype = res
+    return f
+
+
+_lib.fk_status_string.argtypes = [ctypes.c_int]
+_lib.fk_status_string.restype = ctypes.c_char_p
+_sig("fk_version", [])
+_sig("fk_workspace_size", [_i64, _int, _int, _int, _int, ctypes.POINTER(_sz)])
+_sig("fk_normalize_rows", [_vp, _vp, _i64, _int, _vp])
+_sig("fk_centroid_norms", [_vp, _int, _int, _int, _vp, _vp])
+_sig("fk_assign", [_vp, _int, _i64, _int, _vp, _int, _vp, _vp, _vp, _sz, _vp])
+_sig("fk_update", [_vp, _int, _i64, _int, _int, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                   _sz, _vp])
+_sig("fk_lloyd", [_vp, _int, _i64, _int, _int, _int, _int, _vp, _vp, _vp, _vp,
+                  ctypes.POINTER(ctypes.c_double), ctypes.POINTER(FkTiming), _vp, _sz, _vp])
+_sig("fk_get_device_error", [_vp, _sz, ctypes.POINTER(ctypes.c_int), _vp])
+_sig("fk_selftest_timeout", [_vp, _sz, ctypes.c_uint64, _vp])
+
+EXPORTED = ["fk_status_string", "fk_version", "fk_workspace_size", "fk_normalize_rows",
+            "fk_centroid_norms", "fk_assign", "fk_update", "fk_lloyd",
+            "fk_get_device_error", "fk_selftest_timeout"]
+
+
+class FkError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {_lib.fk_status_string(status).decode()}")
+
+
+def _check(status: int, where: str):
+    if status != FK_OK:
+        raise FkError(status, where)
+
+
+def status_string(status: int) -> str:
+    return _lib.fk_status_string(status).decode()
+
+
+def version() -> int:
+    return _lib.fk_version()
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return FK_F32
+    if t.dtype == torch.bfloat16:
+        return FK_BF16
+    raise TypeError(f"unsupported point dtype {t.dtype}")
+
+
+def _metric_code(metric) -> int:
+    if metric in ("l2", FK_L2):
+        return FK_L2
+    if metric in ("cosine", FK_COSINE):
+        return FK_COSINE
+    raise ValueError(metric)
+
+
+def _dev(t: torch.Tensor, name: str, dtype=None, shape=None):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.device.type != "cuda":
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    return t.data_ptr()
+
+
+def _opt(t, name, dtype=None, shape=None):
+    return None if t is None else _dev(t, name, dtype, shape)
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def fk_workspace_size(N: int, d: int, K: int, dtype=torch.float32, metric="l2") -> int:
+    code = dtype if isinstance(dtype, int) else (FK_F32 if dtype == torch.float32 else
+                                                 FK_BF16 if dtype == torch.bfloat16 else -1)
+    out = _sz(0)
+    _check(_lib.fk_workspace_size(N, d, K, code, _metric_code(metric), ctypes.byref(out)),
+           "fk_workspace_size")
+    return out.value
+
+
+def workspace(N: int, d: int, K: int, dtype=torch.float32, metric="l2", device="cuda"):
+    """A zeroed uint8 workspace tensor of the size libfk asks for (256-byte aligned by the
+    CUDA caching allocator)."""
+    nbytes = fk_workspace_size(N, d, K, dtype, metric)
+    ws = torch.zeros(nbytes, dtype=torch.uint8, device=device)
+    if ws.data_ptr() % 256:
+        raise RuntimeError("workspace is not 256-byte aligned")
+    return ws
+
+
+def fk_normalize_rows(X_in: torch.Tensor, X_out: torch.Tensor, stream=None):
+    N, d = X_in.shape
+    _check(_lib.fk_normalize_rows(_dev(X_in, "X_in", torch.float32),
+                                  _dev(X_out, "X_out", torch.float32, (N, d)), N, d,
+                                  _stream(stream)), "fk_normalize_rows")
+
+
+def fk_centroid_norms(C: torch.Tensor, cn: torch.Tensor, dtype=torch.float32, stream=None):
+    K, d = C.shape
+    code = FK_F32 if dtype == torch.float32 else FK_BF16
+    _check(_lib.fk_centroid_norms(_dev(C, "C", torch.float32), K, d, code,
+                                  _dev(cn, "cn", torch.float32, (K,)), _stream(stream)),
+           "fk_centroid_norms")
+
+
+def fk_assign(X: torch.Tensor, C: torch.Tensor, labels: torch.Tensor, ws: torch.Tensor,
+              mind: torch.Tensor | None = None, stream=None):
+    N, d = X.shape
+    K = C.shape[0]
+    _check(_lib.fk_assign(_dev(X, "X"), _dtype_code(X), N, d,
+                          _dev(C, "C", torch.float32, (K, d)), K,
+                          _dev(labels, "labels", torch.int32, (N,)),
+                          _opt(mind, "mind", torch.float32, (N,)),
+                          _dev(ws, "ws", torch.uint8), ws.numel(), _stream(stream)),
+           "fk_assign")
+
+
+def fk_update(X: torch.Tensor, labels: torch.Tensor, C_old: torch.Tensor,
+              C_new: torch.Tensor, counts: torch.Tensor, offsets: torch.Tensor,
+              ws: torch.Tensor, perm: torch.Tensor | None = None,
+              objective: torch.Tensor | None = None, stream=None):
+    N, d = X.shape
+    K = C_old.shape[0]
+    _check(_lib.fk_update(_dev(X, "X"), _dtype_code(X), N, d, K,
+                          _dev(labels, "labels", torch.int32, (N,)),
+                          _dev(C_old, "C_old", torch.float32, (K, d)),
+                          _dev(C_new, "C_new", torch.float32, (K, d)),
+                          _dev(counts, "counts", torch.int32, (K,)),
+                          _dev(offsets, "offsets", torch.int32, (K + 1,)),
+                          _opt(perm, "perm", torch.int32, (N,)),
+                          _opt(objective, "objective", torch.float64, (1,)),
+                          _dev(ws, "ws", torch.uint8), ws.numel(), _stream(stream)),
+           "fk_update")
+
+
+def fk_lloyd(X: torch.Tensor, C: torch.Tensor, niter: int, labels: torch.Tensor,
+             ws: torch.Tensor, metric="l2", counts: torch.Tensor | None = None,
+             offsets: torch.Tensor | None = None, timing: bool = False, stream=None):
+    """Run niter iterations in place on C.  Returns (objectives list, timing dict|None)."""
+    N, d = X.shape
+    K = C.shape[0]
+    obj = (ctypes.c_double * max(niter, 1))()
+    tm = FkTiming() if timing else None
+    _check(_lib.fk_lloyd(_dev(X, "X"), _dtype_code(X), N, d, K, _metric_code(metric), niter,
+                         _dev(C, "C", torch.float32, (K, d)),
+                         _dev(labels, "labels", torch.int32, (N,)),
+                         _opt(counts, "counts", torch.int32, (K,)),
+                         _opt(offsets, "offsets", torch.int32, (K + 1,)), obj,
+                         ctypes.byref(tm) if tm is not None else None,
+                         _dev(ws, "ws", torch.uint8), ws.numel(), _stream(stream)),
+           "fk_lloyd")
+    t = None
+    if tm is not None:
+        t = {f: getattr(tm, f) for f, _ in FkTiming._fields_}
+    return [obj[i] for i in range(niter)], t
+
+
+def fk_get_device_error(ws: torch.Tensor, stream=None) -> int:
+    code = ctypes.c_int(0)
+    _check(_lib.fk_get_device_error(_dev(ws, "ws", torch.uint8), ws.numel(),
+                                    ctypes.byref(code), _stream(stream)),
+           "fk_get_device_error")
+    return code.value
+
+
+def fk_selftest_timeout(ws: torch.Tensor, limit_ns: int, stream=None):
+    _check(_lib.fk_selftest_timeout(_dev(ws, "ws", torch.uint8), ws.numel(), int(limit_ns),
+                                    _stream(stream)), "fk_selftest_timeout")

@@ -1,0 +1,187 @@
+/*
+ * fk.h -- C ABI of the exact Lloyd's k-means library (libfk.so), sm_100a (B200).
+ *
+ * One Lloyd iteration = (1) assign every point to its nearest centroid under squared
+ * L2, without materialising the N x K distance matrix, and (2) recompute every centroid
+ * as the mean of its points through a sorted inverse index, with no atomics.  Sources:
+ *   - Flash-KMeans article (lumevalley.com, "UC Berkeley + UT Austin Flash-KMeans"),
+ *     opening paragraph: exact standard Lloyd's, no approximation;
+ *     section "为什么"快"这件事被拖了这么久": an iteration assigns N points to K
+ *     clusters, then recomputes the centroids;
+ *     section "FlashAssign：把距离矩阵按块切成流水线": distances are computed tile by
+ *     tile and reduced to an argmin on chip, so only O(Nd + Kd) data moves;
+ *     section "Sort-Inverse Update：原子操作的另一种解法": sort the assignments by
+ *     cluster id into an inverse index, then reduce each cluster by reading its points
+ *     contiguously, with no atomics;
+ *     section "它不是银弹，但切中了一个真痛点": L2 and cosine only.
+ *   - LEANN FlashLib guide (mhpn.cn, "LEANN FlashLib 后端实战指南"),
+ *     section "距离度量只有 squared L2如何支持 mips / cosine": cosine = L2-normalise the
+ *     vectors, a zero-norm vector is divided by 1;
+ *     section "nlist 与 nprobe 的推导规则": the cluster count is clamped to n (here
+ *     K > N is an argument error; a caller may clamp);
+ *     section "工作原理": the build output is CSR cluster offsets plus cell-ordered row
+ *     ids.
+ *
+ * Conventions for every call:
+ *   - All matrices are row-major and contiguous: X is N x d, centroids are K x d.
+ *   - Pointers are DEVICE pointers unless a parameter says "host".  Input buffers are
+ *     read-only unless stated; the caller owns every buffer, including the workspace.
+ *   - The library never allocates device memory: scratch comes from the caller's
+ *     workspace `ws` of `ws_bytes` bytes (query the size with fk_workspace_size; the
+ *     pointer must be 256-byte aligned).  One workspace must not be used by two calls
+ *     that can run at the same time.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy default
+ *     stream) unless stated.  Argument checks are synchronous and return an error before
+ *     anything is launched.  A failed launch returns FK_ERR_CUDA.
+ *   - Device-side checks (a label outside [0, K), a bounded wait that expired inside a
+ *     kernel) set an error word in the first 256 bytes of the workspace; fk_lloyd clears
+ *     it on entry and reports it on return, fk_get_device_error reads and clears it for
+ *     the asynchronous calls.  Zero a new workspace once (or call fk_get_device_error on
+ *     it) before the first fk_assign / fk_update.  No kernel traps.
+ *   - Results are deterministic: the same inputs on the same device give the same bits,
+ *     run after run (no atomics on any floating-point value, fixed reduction orders).
+ *   - Limits: 1 <= K <= N < 2^31, d >= 1; FK_F32 needs d % 4 == 0 and X 16-byte
+ *     aligned; FK_BF16 needs d % 8 == 0 and X 16-byte aligned; FK_COSINE needs FK_F32.
+ *     Violations return FK_ERR_INVALID_ARG (shape/pointer) or FK_ERR_UNSUPPORTED
+ *     (dtype/alignment/device other than sm_100).
+ */
+#ifndef FK_H
+#define FK_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define FK_API __attribute__((visibility("default")))
+#else
+#define FK_API
+#endif
+
+typedef struct CUstream_st *fk_stream_t; /* same type as cudaStream_t */
+
+typedef enum fk_status {
+    FK_OK = 0,
+    FK_ERR_INVALID_ARG = 1, /* bad shape, null required pointer, K > N, ...          */
+    FK_ERR_UNSUPPORTED = 2, /* dtype/metric/alignment/device not supported            */
+    FK_ERR_WORKSPACE = 3,   /* ws null, misaligned or smaller than fk_workspace_size  */
+    FK_ERR_CUDA = 4,        /* a CUDA runtime/driver call or a launch failed          */
+    FK_ERR_TIMEOUT = 5,     /* a bounded wait inside a kernel expired                 */
+    FK_ERR_DEVICE = 6       /* a device-side argument check failed (label range)      */
+} fk_status;
+
+typedef enum fk_dtype {
+    FK_F32 = 0,  /* fp32 points; products emulated to fp32 accuracy with three bf16
+                    tensor-core products (hi*hi + lo*hi + hi*lo)                      */
+    FK_BF16 = 1  /* bf16 points; bf16 tensor-core products (exact), fp32 accumulation  */
+} fk_dtype;
+
+typedef enum fk_metric {
+    FK_L2 = 0,     /* squared Euclidean distance                                     */
+    FK_COSINE = 1  /* L2-normalise points and initial centroids, then squared L2     */
+} fk_metric;
+
+/* Per-phase device time of an fk_lloyd call, summed over its iterations (CUDA events
+ * recorded on the caller's stream around each phase). */
+typedef struct fk_timing {
+    double ms_setup;   /* once per call: normalisation (cosine) and the fp32 split of X */
+    double ms_prep;    /* per iteration: centroid norms and operand preparation        */
+    double ms_assign;  /* per iteration: the fused tensor-core assign kernel           */
+    double ms_sort;    /* per iteration: radix sort of labels -> perm + CSR offsets   */
+    double ms_update;  /* per iteration: segmented reduction, combine, finalize, J     */
+    int iterations;
+    int launches;      /* kernels this call launched (library kernels only)            */
+} fk_timing;
+
+/* Human-readable name of a status code (static string, never NULL). */
+FK_API const char *fk_status_string(fk_status s);
+
+/* Library ABI version (incremented on any signature change). */
+FK_API int fk_version(void);
+
+/* Bytes of workspace that fk_assign, fk_update and fk_lloyd need for this problem
+ * (any of them; the largest need).  Host-only, synchronous.  `bytes` is a host pointer. */
+FK_API fk_status fk_workspace_size(int64_t N, int d, int K, fk_dtype dtype, fk_metric metric,
+                            size_t *bytes);
+
+/* Row L2 normalisation (cosine mode, step 0): X_out[i] = X_in[i] / ||X_in[i]||, where a
+ * zero norm is replaced by 1 (LEANN FlashLib guide, "距离度量只有 squared L2如何支持
+ * mips / cosine").  The norm is accumulated in fp64 and each output is rounded once to
+ * fp32.  fp32 only; X_out may equal X_in (in place).  N x d row-major. */
+FK_API fk_status fk_normalize_rows(const float *X_in, float *X_out, int64_t N, int d,
+                            fk_stream_t stream);
+
+/* Centroid norms: cn[k] = sum_j c_kj^2 over the values the tensor cores consume (the
+ * fp32 centroids for FK_F32, their bf16 rounding for FK_BF16), accumulated in fp64 and
+ * rounded once to fp32.  C is K x d fp32; cn has K floats. */
+FK_API fk_status fk_centroid_norms(const float *C, int K, int d, fk_dtype dtype, float *cn,
+                            fk_stream_t stream);
+
+/* Assignment step (Flash-KMeans article, "FlashAssign：把距离矩阵按块切成流水线").
+ *   labels[i] = argmin_k ||x_i - c_k||^2, lowest k on exact ties, for i < N.
+ *   mind[i]   = ||x_i||^2 + min_k (||c_k||^2 - 2 x_i.c_k)  (expansion form; optional,
+ *               pass NULL to skip).
+ * X: N x d, dtype `dtype`.  C: K x d fp32 (for FK_BF16 the kernel uses C rounded to
+ * bf16).  labels: N int32.  The N x K distance matrix is never stored: a tcgen05 kernel
+ * keeps one 128 x 256 fp32 tile in tensor memory and a running min/argmin per row.
+ * For FK_F32 each call first splits X into bf16 hi/lo planes inside `ws` (one extra
+ * pass over X; fk_lloyd does this once per call instead of once per iteration). */
+FK_API fk_status fk_assign(const void *X, fk_dtype dtype, int64_t N, int d, const float *C,
+                    int K, int32_t *labels, float *mind, void *ws, size_t ws_bytes,
+                    fk_stream_t stream);
+
+/* Update step (Flash-KMeans article, "Sort-Inverse Update：原子操作的另一种解法").
+ *   counts[k]  = #{i : labels[i] == k}                         (K int32, required)
+ *   offsets    = exclusive prefix sum of counts, offsets[K] = N (K+1 int32, required)
+ *   perm       = point indices ordered by (label, index)        (N int32, optional)
+ *   C_new[k]   = mean of the points with label k, or C_old[k] bit for bit when the
+ *                cluster is empty                              (K x d fp32, required;
+ *                must not overlap C_old)
+ *   *objective = sum_i ||x_i - c_old[labels[i]]||^2 in fp64 (device double, optional),
+ *                where c_old is C_old for FK_F32 and C_old rounded to bf16 for FK_BF16
+ *                (the centroids the labels were assigned with).
+ * The labels are sorted with an atomic-free, stable LSD radix sort; each cluster's sum is
+ * accumulated in fp64 in a fixed order (rows in index order within fixed chunks, chunk
+ * partials combined in chunk order), so the result does not depend on timing.
+ * A label outside [0, K) sets FK_ERR_DEVICE in the workspace error word. */
+FK_API fk_status fk_update(const void *X, fk_dtype dtype, int64_t N, int d, int K,
+                    const int32_t *labels, const float *C_old, float *C_new,
+                    int32_t *counts, int32_t *offsets, int32_t *perm, double *objective,
+                    void *ws, size_t ws_bytes, fk_stream_t stream);
+
+/* `niter` Lloyd iterations from the initial centroids in C (K x d fp32, overwritten with
+ * the final centroids).  Cosine mode normalises X (into the workspace; X itself is not
+ * modified) and the initial C first.  On return (this call synchronises `stream` once,
+ * at the end):
+ *   labels           N int32, the labels of the last assignment (device);
+ *   counts, offsets  of the last assignment (device; optional, may be NULL);
+ *   objective_host   niter doubles (HOST pointer, optional): entry t is the objective
+ *                    of iteration t's labels against the centroids they were assigned
+ *                    with;
+ *   timing           HOST pointer (optional): per-phase device milliseconds.
+ * niter = 0 only normalises C (cosine) and returns. */
+FK_API fk_status fk_lloyd(const void *X, fk_dtype dtype, int64_t N, int d, int K,
+                   fk_metric metric, int niter, float *C, int32_t *labels,
+                   int32_t *counts, int32_t *offsets, double *objective_host,
+                   fk_timing *timing, void *ws, size_t ws_bytes, fk_stream_t stream);
+
+/* Diagnostics for the failure path, without any fault: launches a one-warp kernel that
+ * waits (bounded by limit_ns, at most 10 s) on an mbarrier nothing ever arrives on; the
+ * wait expires and the kernel records FK_ERR_TIMEOUT in the workspace error word, which
+ * fk_get_device_error then returns.  Asynchronous on `stream`. */
+FK_API fk_status fk_selftest_timeout(void *ws, size_t ws_bytes, uint64_t limit_ns,
+                              fk_stream_t stream);
+
+/* Synchronise `stream`, then read and clear the workspace's device error word.
+ * *code (host int) receives FK_OK, FK_ERR_TIMEOUT or FK_ERR_DEVICE; the return value
+ * is FK_OK unless reading failed. */
+FK_API fk_status fk_get_device_error(void *ws, size_t ws_bytes, int *code, fk_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FK_H */

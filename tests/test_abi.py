@@ -1,0 +1,93 @@
+"""The C-ABI library loads, exports every symbol include/fk.h declares, and rejects bad
+arguments on the host before any device work (no GPU needed)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def fk():
+    import __graft_entry__
+    __graft_entry__.build()
+    from exact_lloyd_means_b200 import fk as m
+    return m
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "fk.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(fk_[a-z_]+)\s*\(", src)))
+
+
+def test_every_declared_symbol_is_exported(fk):
+    lib = ctypes.CDLL(fk.LIB_PATH)
+    names = _declared()
+    assert "fk_lloyd" in names and "fk_assign" in names and "fk_update" in names
+    for n in names:
+        assert hasattr(lib, n), n
+    assert sorted(fk.EXPORTED) == names
+
+
+def test_only_declared_symbols_are_exported(fk):
+    out = os.popen(f"nm -D --defined-only {fk.LIB_PATH}").read()
+    exported = sorted(set(re.findall(r"\bT (fk_[a-z_]+)\b", out)))
+    assert exported == _declared()
+
+
+def test_status_strings(fk):
+    for code, name in [(0, "FK_OK"), (1, "FK_ERR_INVALID_ARG"), (2, "FK_ERR_UNSUPPORTED"),
+                       (3, "FK_ERR_WORKSPACE"), (4, "FK_ERR_CUDA"), (5, "FK_ERR_TIMEOUT"),
+                       (6, "FK_ERR_DEVICE")]:
+        assert fk.status_string(code) == name
+    assert fk.version() >= 1
+
+
+def test_workspace_size_validation(fk):
+    import torch
+    n = fk.fk_workspace_size(65536, 128, 256, torch.float32, "l2")
+    assert n > 65536 * 128 * 4  # holds the two bf16 planes of X
+    assert fk.fk_workspace_size(65536, 128, 256, torch.bfloat16, "l2") < n
+    assert fk.fk_workspace_size(65536, 128, 256, torch.float32, "cosine") > n
+    for args, code in [((10, 128, 11), fk.FK_ERR_INVALID_ARG),
+                       ((10, 0, 2), fk.FK_ERR_INVALID_ARG),
+                       ((0, 8, 1), fk.FK_ERR_INVALID_ARG),
+                       ((10, 6, 2), fk.FK_ERR_UNSUPPORTED),
+                       ((2 ** 31, 8, 2), fk.FK_ERR_INVALID_ARG)]:
+        with pytest.raises(fk.FkError) as e:
+            fk.fk_workspace_size(*args, torch.float32, "l2")
+        assert e.value.status == code
+    with pytest.raises(fk.FkError) as e:
+        fk.fk_workspace_size(100, 12, 4, torch.bfloat16, "l2")
+    assert e.value.status == fk.FK_ERR_UNSUPPORTED
+    with pytest.raises(fk.FkError) as e:
+        fk.fk_workspace_size(100, 16, 4, torch.bfloat16, "cosine")
+    assert e.value.status == fk.FK_ERR_UNSUPPORTED
+
+
+def test_host_side_checks_need_no_device(fk):
+    lib = fk._lib
+    # null workspace / null inputs are rejected before any CUDA call
+    assert lib.fk_assign(None, 0, 100, 8, None, 4, None, None, None, 0, None) == \
+        fk.FK_ERR_INVALID_ARG
+    assert lib.fk_assign(16, 0, 100, 8, 16, 4, 16, None, None, 0, None) == fk.FK_ERR_WORKSPACE
+    assert lib.fk_assign(16, 0, 100, 8, 16, 4, 16, None, 256, 10, None) == fk.FK_ERR_WORKSPACE
+    assert lib.fk_assign(8, 0, 100, 8, 16, 4, 16, None, 256, 1 << 30, None) == \
+        fk.FK_ERR_UNSUPPORTED  # X not 16-byte aligned
+    assert lib.fk_lloyd(16, 0, 100, 8, 4, 0, -1, 16, 16, None, None, None, None, 256, 1 << 30,
+                        None) == fk.FK_ERR_INVALID_ARG
+    # C_new overlapping C_old
+    assert lib.fk_update(16, 0, 100, 8, 4, 16, 4096, 4100, 16, 16, None, None, 256, 1 << 30,
+                         None) == fk.FK_ERR_INVALID_ARG
+    assert lib.fk_get_device_error(None, 0, None, None) == fk.FK_ERR_INVALID_ARG
+
+
+def test_binding_rejects_cpu_tensors(fk):
+    import torch
+    X = torch.zeros(10, 8)
+    with pytest.raises(ValueError):
+        fk.fk_assign(X, torch.zeros(2, 8), torch.zeros(10, dtype=torch.int32),
+                     torch.zeros(256, dtype=torch.uint8))

@@ -1,0 +1,244 @@
+"""GPU parity: the CUDA path through the C ABI against the fp64 oracle, element by element
+on the same seeded inputs, at sizes spanning several tiles with ragged tails.
+
+Parity rules (written here, applied in every test):
+  labels   bit-exact except at tie points (oracle top-2 gap < 1e-4 (||x||^2 + max||c||^2));
+  counts, offsets, perm  bit-exact;
+  centroids (given identical labels)  max |dc| <= 1e-5 max |c_ref| per centroid;
+  objective  relative error <= 1e-5.
+Inputs reach the GPU from the generator or from the oracle (lockstep); nothing computed on
+the GPU is ever handed to the oracle."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from synth import gaussian_mixture, init_indices
+from tests.gpu_helpers import (CENTROID_TOL, OBJECTIVE_TOL, centroid_rel_err, fk, gpu_assign,
+                               gpu_update, label_mismatches)
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+
+def _mixture(N, d, K, dtype="f32", seed=0, centers="uniform", sigma=0.1, weights="equal"):
+    X, comp, cen = gaussian_mixture(N, d, K, centers=centers, sigma=sigma, weights=weights,
+                                    dtype=dtype, seed=seed)
+    C0 = X[init_indices(N, K, seed)].float().contiguous()
+    return X, C0, comp
+
+
+ASSIGN_SHAPES = [(1000, 64, 10), (4097, 128, 256), (3001, 96, 300), (5000, 8, 7),
+                 (777, 768, 513), (300, 128, 1), (129, 16, 129), (20000, 128, 1000)]
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("N,d,K", ASSIGN_SHAPES)
+def test_assign_matches_oracle(N, d, K, dtype):
+    X, C0, _ = _mixture(N, d, K, dtype, seed=N + d + K)
+    Cref = oracle.round_bf16(C0.numpy()) if dtype == "bf16" else C0.numpy()
+    ref, dmin, d2nd = oracle.assign(X, Cref)
+    ties = oracle.tie_mask(X, Cref, dmin, d2nd)
+    lab, mind = gpu_assign(X.to(DEV), C0.to(DEV), with_mind=True)
+    assert (lab >= 0).all() and (lab < K).all()
+    assert label_mismatches(lab, ref, ties) == 0, f"ties={int(ties.sum())}"
+    # mind is the expansion form: within the same window the tie rule uses
+    Xd = X.double().numpy()
+    s = (Xd * Xd).sum(1) + (Cref.astype(np.float64) ** 2).sum(1).max()
+    assert (np.abs(mind.astype(np.float64) - dmin) <= 1e-4 * s).all()
+
+
+def test_assign_points_as_centroids():
+    X, _, _ = _mixture(1000, 64, 50, seed=3)
+    lab, _ = gpu_assign(X.to(DEV), X.to(DEV).clone())
+    assert (lab == np.arange(1000)).all()
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_assign_duplicate_centroid_lowest_index(dtype):
+    X, C0, _ = _mixture(3000, 128, 40, dtype, seed=4)
+    C = torch.cat([C0, C0[5:6], C0[17:18]])  # 40 duplicates 5, 41 duplicates 17
+    lab, _ = gpu_assign(X.to(DEV), C.to(DEV))
+    assert not np.isin(lab, [40, 41]).any()
+    assert (lab == 5).any() and (lab == 17).any()
+
+
+def test_assign_tight_mixture_recovers_components():
+    X, comp, cen = gaussian_mixture(5000, 128, 300, centers="uniform", sigma=1e-3, seed=5)
+    lab, _ = gpu_assign(X.to(DEV), cen.float().to(DEV))
+    assert (lab == comp.numpy()).all()
+
+
+UPDATE_SHAPES = [(1000, 64, 10, "equal"), (20000, 128, 37, "equal"), (70000, 128, 3, "equal"),
+                 (5000, 768, 50, "equal"), (3000, 1032, 20, "equal"), (200000, 16, 2, "equal"),
+                 (150000, 128, 4096, "zipf"), (777, 8, 700, "equal")]
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("N,d,K,weights", UPDATE_SHAPES)
+def test_update_matches_oracle(N, d, K, weights, dtype):
+    if dtype == "bf16" and d % 8:
+        pytest.skip("bf16 needs d % 8 == 0")
+    X, C0, comp = _mixture(N, d, K, dtype, seed=N + K, weights=weights, centers="normal")
+    labels = comp.numpy().astype(np.int32)  # generator labels: Zipf gives huge clusters
+    labels[labels == K // 2] = (K // 2 + 1) % K  # force an empty cluster
+    C_old = torch.randn(K, d, generator=torch.Generator().manual_seed(1))
+    counts, offsets, perm = oracle.csr(labels, K)
+    C_ref = oracle.update(X, labels, C_old.numpy())
+    C_used = oracle.round_bf16(C_old.numpy()) if dtype == "bf16" else C_old.numpy()
+    J_ref = oracle.objective(X, C_used, labels)
+
+    g = gpu_update(X.to(DEV), labels, C_old.to(DEV))
+    assert (g["counts"] == counts).all()
+    assert (g["offsets"] == offsets).all()
+    assert (g["perm"] == perm).all()
+    nonempty = counts > 0
+    assert centroid_rel_err(g["C_new"][nonempty], C_ref[nonempty]) <= CENTROID_TOL
+    # an empty cluster keeps its previous centroid bit for bit
+    assert (g["C_new"][~nonempty] == C_old.numpy()[~nonempty].astype(np.float64)).all()
+    assert abs(g["J"] - J_ref) <= OBJECTIVE_TOL * J_ref
+
+
+def test_update_single_cluster_is_global_mean():
+    X, _, _ = _mixture(50000, 128, 1, seed=9)
+    g = gpu_update(X.to(DEV), np.zeros(50000, np.int32), torch.zeros(1, 128, device=DEV))
+    mean = X.double().numpy().mean(axis=0)
+    assert centroid_rel_err(g["C_new"], mean[None]) <= 1e-6
+    assert (g["perm"] == np.arange(50000)).all() and g["offsets"].tolist() == [0, 50000]
+
+
+@pytest.mark.parametrize("case", ["tiny_f32", "tiny_bf16", "cosine_768"])
+def test_lockstep_lloyd_matches_oracle(case):
+    """Lockstep: each iteration the GPU assigns with the oracle's centroids and updates
+    with the oracle's labels; every output is compared with the oracle's."""
+    if case == "tiny_f32":
+        X, C0, _ = _mixture(65536, 128, 256, "f32", seed=0, sigma=0.1)
+        niter, prec, metric = 3, "f32", "l2"
+    elif case == "tiny_bf16":
+        X, C0, _ = _mixture(30000, 128, 500, "bf16", seed=1, centers="normal", sigma=0.25)
+        niter, prec, metric = 3, "bf16", "l2"
+    else:
+        X, C0, _ = _mixture(20000, 768, 64, "f32", seed=2, centers="normal", sigma=0.3)
+        niter, prec, metric = 3, "f32", "cosine"
+    ref = oracle.lloyd(X, C0, niter, metric=metric, precision=prec)
+    Xg = X.to(DEV)
+    if metric == "cosine":
+        Xn = torch.empty_like(Xg)
+        fk().fk_normalize_rows(Xg, Xn)
+        dn = np.abs(Xn.cpu().double().numpy() - ref["X"])
+        assert (dn <= 2 ** -23 * np.abs(ref["X"]) + 1e-30).all()  # <= 1 ulp of fp32
+        Xg = Xn
+    C_master = [C0.double().numpy()] + ref["C_next"]
+    if metric == "cosine":
+        C_master[0] = oracle.round_f32(oracle.normalize_rows(C0.numpy()))
+    total_ties = 0
+    for t in range(niter):
+        Cm = torch.as_tensor(C_master[t], dtype=torch.float32)
+        lab, _ = gpu_assign(Xg, Cm.to(DEV))
+        ties = ref["ties"][t]
+        total_ties += int(ties.sum())
+        assert label_mismatches(lab, ref["labels"][t], ties) == 0, f"iteration {t}"
+        g = gpu_update(Xg, ref["labels"][t], Cm.to(DEV))
+        assert (g["counts"] == ref["counts"][t]).all()
+        assert (g["offsets"] == ref["offsets"][t]).all()
+        assert (g["perm"] == ref["perm"][t]).all()
+        assert centroid_rel_err(g["C_new"], ref["C_next"][t]) <= CENTROID_TOL
+        assert abs(g["J"] - ref["J"][t]) <= OBJECTIVE_TOL * ref["J"][t]
+    print(f"{case}: tie points over {niter} iterations: {total_ties}")
+
+
+@pytest.mark.parametrize("metric", ["l2", "cosine"])
+def test_fk_lloyd_free_running_objective(metric):
+    """fk_lloyd end to end from the same C0 as the oracle's own free-running Lloyd.
+
+    Iteration 0 sees identical centroids, so its objective must agree to 1e-5.  Later
+    iterations may legitimately drift: a point inside the tie window may take the other
+    label (allowed by the parity rule), which moves two centroids by |x - c| / n_k and
+    changes the rest of the trajectory; the lockstep test above is the parity gate for
+    every later iteration.  Here the later objectives are held to 1e-3 and the run's own
+    invariants are checked exactly."""
+    X, C0, _ = _mixture(40000, 64 if metric == "l2" else 256, 100, seed=7, centers="normal",
+                        sigma=0.3)
+    niter = 4
+    ref = oracle.lloyd(X, C0, niter, metric=metric)
+    m = fk()
+    C = C0.to(DEV).clone()
+    labels = torch.empty(X.shape[0], dtype=torch.int32, device=DEV)
+    counts = torch.empty(100, dtype=torch.int32, device=DEV)
+    offsets = torch.empty(101, dtype=torch.int32, device=DEV)
+    ws = m.workspace(X.shape[0], X.shape[1], 100, torch.float32, metric)
+    objs, tm = m.fk_lloyd(X.to(DEV), C, niter, labels, ws, metric=metric, counts=counts,
+                          offsets=offsets, timing=True)
+    assert abs(objs[0] - ref["J"][0]) <= OBJECTIVE_TOL * ref["J"][0]
+    for t in range(1, niter):
+        assert abs(objs[t] - ref["J"][t]) <= 1e-3 * ref["J"][t], t
+    assert tm["iterations"] == niter and tm["ms_assign"] > 0 and tm["launches"] > 4 * niter
+    lab = labels.cpu().numpy()
+    assert (np.bincount(lab, minlength=100) == counts.cpu().numpy()).all()
+    assert offsets.cpu().numpy()[-1] == X.shape[0]
+    # objective never increases (beyond fp32 rounding of the centroids)
+    for t in range(1, niter):
+        assert objs[t] <= objs[t - 1] * (1 + 1e-6)
+
+
+def test_fk_lloyd_deterministic_and_resumable():
+    X, C0, _ = _mixture(30000, 128, 200, seed=8, centers="normal", sigma=0.3)
+    m = fk()
+    Xg = X.to(DEV)
+    ws = m.workspace(30000, 128, 200, torch.float32, "l2")
+
+    def run(C, n):
+        labels = torch.empty(30000, dtype=torch.int32, device=DEV)
+        objs, _ = m.fk_lloyd(Xg, C, n, labels, ws)
+        return C, labels, objs
+
+    a = run(C0.to(DEV).clone(), 5)
+    b = run(C0.to(DEV).clone(), 5)
+    assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1]) and a[2] == b[2]
+    # checkpoint/resume: 2 iterations then 3 more from the saved centroids == 5 at once
+    c = run(C0.to(DEV).clone(), 2)
+    d = run(c[0].clone(), 3)
+    assert torch.equal(d[0], a[0]) and torch.equal(d[1], a[1]) and d[2] == a[2][2:]
+
+
+def test_fk_lloyd_k_equals_one_and_k_equals_n():
+    m = fk()
+    X, _, _ = _mixture(513, 32, 4, seed=10)
+    Xg = X.to(DEV)
+    for K, C in [(1, X[:1].clone()), (513, X.clone())]:
+        ws = m.workspace(513, 32, K, torch.float32, "l2")
+        labels = torch.empty(513, dtype=torch.int32, device=DEV)
+        Cg = C.to(DEV).contiguous()
+        objs, _ = m.fk_lloyd(Xg, Cg, 1, labels, ws)
+        lab = labels.cpu().numpy()
+        if K == 1:
+            assert (lab == 0).all()
+            assert centroid_rel_err(Cg.cpu().numpy(), X.double().numpy().mean(0)[None]) < 1e-6
+        else:
+            assert (lab == np.arange(513)).all() and objs[0] == 0.0
+            assert torch.equal(Cg.cpu(), X)
+
+
+def test_device_error_paths_without_fault():
+    """A wait that nothing ends expires and is reported; a bad label is reported; the
+    context stays usable afterwards."""
+    m = fk()
+    ws = m.workspace(1000, 64, 10, torch.float32, "l2")
+    assert m.fk_get_device_error(ws) == m.FK_OK
+    m.fk_selftest_timeout(ws, 20_000_000)  # 20 ms
+    assert m.fk_get_device_error(ws) == m.FK_ERR_TIMEOUT
+    assert m.fk_get_device_error(ws) == m.FK_OK  # read clears it
+    X, C0, _ = _mixture(1000, 64, 10, seed=11)
+    labels = np.zeros(1000, np.int32)
+    labels[7] = 10  # == K: out of range
+    m2 = fk()
+    Xg = X.to(DEV)
+    lab = torch.as_tensor(labels).to(DEV)
+    C_new = torch.empty(10, 64, device=DEV)
+    counts = torch.empty(10, dtype=torch.int32, device=DEV)
+    offsets = torch.empty(11, dtype=torch.int32, device=DEV)
+    m2.fk_update(Xg, lab, C0.to(DEV), C_new, counts, offsets, ws)
+    assert m2.fk_get_device_error(ws) == m2.FK_ERR_DEVICE
+    lab2, _ = gpu_assign(Xg, C0.to(DEV))  # still works
+    assert (lab2 >= 0).all()
