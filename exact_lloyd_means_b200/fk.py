@@ -59,10 +59,14 @@ _sig("fk_lloyd", [_vp, _int, _i64, _int, _int, _int, _int, _vp, _vp, _vp, _vp,
                   ctypes.POINTER(ctypes.c_double), ctypes.POINTER(FkTiming), _vp, _sz, _vp])
 _sig("fk_get_device_error", [_vp, _sz, ctypes.POINTER(ctypes.c_int), _vp])
 _sig("fk_selftest_timeout", [_vp, _sz, ctypes.c_uint64, _vp])
+_sig("fk_assign_noalloc", [_vp, _int, _i64, _int, _vp, _int, _vp, _vp])
 
 EXPORTED = ["fk_status_string", "fk_version", "fk_workspace_size", "fk_normalize_rows",
             "fk_centroid_norms", "fk_assign", "fk_update", "fk_lloyd",
-            "fk_get_device_error", "fk_selftest_timeout"]
+            "fk_get_device_error", "fk_selftest_timeout", "fk_assign_noalloc"]
+
+# Bytes of the static device array fk_assign_noalloc takes its scratch from.
+NOALLOC_SCRATCH_BYTES = 8 << 20
 
 
 class FkError(RuntimeError):
@@ -221,3 +225,14 @@ def fk_get_device_error(ws: torch.Tensor, stream=None) -> int:
 def fk_selftest_timeout(ws: torch.Tensor, limit_ns: int, stream=None):
     _check(_lib.fk_selftest_timeout(_dev(ws, "ws", torch.uint8), ws.numel(), int(limit_ns),
                                     _stream(stream)), "fk_selftest_timeout")
+
+
+def fk_assign_noalloc(X: torch.Tensor, C: torch.Tensor, labels: torch.Tensor, stream=None):
+    """fk_assign without a workspace: scratch comes from the library's static device array
+    (for callers that cannot allocate device memory).  Synchronous."""
+    N, d = X.shape
+    K = C.shape[0]
+    _check(_lib.fk_assign_noalloc(_dev(X, "X"), _dtype_code(X), N, d,
+                                  _dev(C, "C", torch.float32, (K, d)), K,
+                                  _dev(labels, "labels", torch.int32, (N,)), _stream(stream)),
+           "fk_assign_noalloc")

@@ -168,6 +168,34 @@ FK_API fk_status fk_lloyd(const void *X, fk_dtype dtype, int64_t N, int d, int K
                    int32_t *counts, int32_t *offsets, double *objective_host,
                    fk_timing *timing, void *ws, size_t ws_bytes, fk_stream_t stream);
 
+/* Scratch held by fk_assign_noalloc: one static device array of this many bytes. */
+#define FK_NOALLOC_SCRATCH_BYTES (8u << 20)
+
+/* fk_assign without a workspace, for callers that cannot allocate device memory: code
+ * that runs under another framework's memory manager (which owns all device memory and
+ * does not allow cudaMalloc behind its back), or on a latency-critical path where
+ * cudaMalloc / cudaFree would implicitly synchronise the device.  The paper has no
+ * counterpart; it is an interface variant of the assignment step above, with the same
+ * labels (bit for bit) as fk_assign on the same inputs.
+ *   - Scratch (error words, centroid operand planes and norms, and for FK_F32 -- or
+ *     FK_BF16 with d % 64 != 0 -- the bf16 planes of X) lives in one file-scope device
+ *     array of FK_NOALLOC_SCRATCH_BYTES (8 MiB) inside libfk; every GPU that loads the
+ *     library holds it until the process exits.  The call allocates and frees nothing.
+ *   - A problem whose scratch does not fit returns FK_ERR_WORKSPACE before any launch
+ *     (roughly: FK_F32 needs 4*N*roundup(d,64) + 4*roundup(K,256)*roundup(d,64) bytes,
+ *     FK_BF16 with d % 64 == 0 needs 2*roundup(K,256)*d bytes, plus a few KB).
+ *   - The first call on a device looks up the array's device address there
+ *     (cudaGetSymbolAddress, with that device current) and caches it; make that first
+ *     call before any stream capture.
+ *   - Every call shares the one array and it keeps the previous call's contents (the
+ *     call clears its error words itself).  Calls whose kernels overlap on the GPU (two
+ *     host threads, two streams) race on it: serialise them.
+ *   - No mind output.  The call is synchronous: it waits for `stream` and returns
+ *     FK_ERR_TIMEOUT if a bounded wait inside the kernel expired. */
+FK_API fk_status fk_assign_noalloc(const void *X, fk_dtype dtype, int64_t N, int d,
+                                   const float *C, int K, int32_t *labels,
+                                   fk_stream_t stream);
+
 /* Diagnostics for the failure path, without any fault: launches a one-warp kernel that
  * waits (bounded by limit_ns, at most 10 s) on an mbarrier nothing ever arrives on; the
  * wait expires and the kernel records FK_ERR_TIMEOUT in the workspace error word, which
