@@ -42,6 +42,8 @@ def parse():
     p.add_argument("--warmup", type=int, default=3)
     p.add_argument("--config", type=int, default=2)
     p.add_argument("--niter", type=int, default=None)
+    p.add_argument("--n", type=int, default=None,
+                   help="override N (smaller cases for profiling captures)")
     p.add_argument("--impl", default="fk", choices=["fk", "reference"])
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
@@ -375,8 +377,13 @@ def main():
     args = parse()
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
+    from dataclasses import replace
+
     from synth import CONFIGS
     spec = CONFIGS[args.config]
+    if args.n:
+        spec = replace(spec, n=args.n, name=spec.name.replace(
+            str(CONFIGS[args.config].n), str(args.n)))
     if args.impl == "reference":
         reference_arm(args, spec, rank, world)
         return

@@ -33,17 +33,29 @@ namespace fk {
 namespace {
 
 
-template <int NP>
+// Tile configuration.  NP = bf16 planes per operand (2: fp32 emulation hi/lo, 1: bf16).
+// RES = the 128-row X block stays resident in shared memory for the whole sweep over the
+// centroid tiles (d <= 128 only), so only centroid chunks stream through the ring; the X
+// block is double-buffered when it is small enough (NP = 1) so the next block's load
+// overlaps the current block's MMAs.
+template <int NP, bool RES>
 struct AsgCfg {
     static constexpr int kABytes = kBM * kBK * 2;  // 16 KB: one X plane chunk
     static constexpr int kBBytes = kBN * kBK * 2;  // 32 KB: one centroid plane chunk
-    static constexpr int kStageBytes = NP * (kABytes + kBBytes);
-    static constexpr int kStages = NP == 2 ? 2 : 4;
-    static constexpr int kDataBytes = kStages * kStageBytes;  // 192 KB
-    static constexpr int kBarBytes = 256;
-    static constexpr int kSmemBytes = kDataBytes + kBarBytes + 1024;  // + alignment slack
-    static constexpr int kThreads = 192;
+    static constexpr int kAChunks = RES ? 2 : 0;   // resident k-chunks (d <= 128)
+    static constexpr int kABufs = RES ? (NP == 1 ? 2 : 1) : 0;
+    static constexpr int kABufBytes = kAChunks * NP * kABytes;
+    static constexpr int kARegion = kABufs * kABufBytes;
+    static constexpr int kStageBytes = RES ? NP * kBBytes : NP * (kABytes + kBBytes);
+    static constexpr int kStages = RES ? (NP == 1 ? 4 : 2) : (NP == 2 ? 2 : 4);
+    static constexpr int kDataBytes = kARegion + kStages * kStageBytes;  // 192 KB
+    static constexpr int kBarBytes = 512;
+    static constexpr int kRedBytes = 2 * 2 * kBM * 4;  // per-row (min, argmin), 2 slots
+    static constexpr int kSmemBytes = kDataBytes + kBarBytes + kRedBytes + 1024;
+    static constexpr int kEpiWarps = 8;  // two warpgroups, one per half of the columns
+    static constexpr int kThreads = 64 + kEpiWarps * 32;
     static constexpr int kTmemCols = 2 * kBN;  // two 256-column fp32 accumulators
+    static_assert(kSmemBytes <= 232448, "shared memory");
 };
 
 __device__ __forceinline__ void raise_timeout(volatile uint32_t *abort_flag, uint32_t *err) {
@@ -60,8 +72,23 @@ __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity,
     return __shfl_sync(0xffffffffu, ok, 0) != 0;
 }
 
-template <int NP>
-__global__ void __launch_bounds__(AsgCfg<NP>::kThreads, 1)
+// Minimum of 64 values with three-input mins: 21 + 7 + 3 + 1 instructions.
+__device__ __forceinline__ float min64(const float (&v)[64]) {
+    float t[22];
+#pragma unroll
+    for (int i = 0; i < 21; ++i) t[i] = ptx::fmin3(v[3 * i], v[3 * i + 1], v[3 * i + 2]);
+    t[21] = v[63];
+    float u[8];
+#pragma unroll
+    for (int i = 0; i < 7; ++i) u[i] = ptx::fmin3(t[3 * i], t[3 * i + 1], t[3 * i + 2]);
+    u[7] = t[21];
+    const float a = ptx::fmin3(u[0], u[1], u[2]);
+    const float b = ptx::fmin3(u[3], u[4], u[5]);
+    return ptx::fmin3(a, b, fminf(u[6], u[7]));
+}
+
+template <int NP, bool RES>
+__global__ void __launch_bounds__(AsgCfg<NP, RES>::kThreads, 1)
     assign_kernel(const __grid_constant__ CUtensorMap tmA0,
                   const __grid_constant__ CUtensorMap tmA1,
                   const __grid_constant__ CUtensorMap tmB0,
@@ -69,18 +96,25 @@ __global__ void __launch_bounds__(AsgCfg<NP>::kThreads, 1)
                   int64_t N, int nkc, int ntiles, int64_t nmb, int32_t *__restrict__ labels,
                   float *__restrict__ best_out, const float *__restrict__ xnorm,
                   float *__restrict__ mind, uint32_t *__restrict__ err, uint64_t wait_ns) {
-    using Cfg = AsgCfg<NP>;
+    using Cfg = AsgCfg<NP, RES>;
     constexpr int S = Cfg::kStages;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    uint8_t *ring = smem + Cfg::kARegion;
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + Cfg::kDataBytes);
     uint64_t *empty = full + S;
     uint64_t *tfull = empty + S;
     uint64_t *tempty = tfull + 2;
-    uint64_t *drain = tempty + 2;
+    uint64_t *afull = tempty + 2;
+    uint64_t *aempty = afull + 2;
+    uint64_t *redfull = aempty + 2;
+    uint64_t *redempty = redfull + 2;
+    uint64_t *drain = redempty + 2;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
     volatile uint32_t *abort_flag = tmem_slot + 1;
+    float *red_v = reinterpret_cast<float *>(smem + Cfg::kDataBytes + Cfg::kBarBytes);
+    int *red_k = reinterpret_cast<int *>(red_v + 2 * kBM);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -92,7 +126,11 @@ __global__ void __launch_bounds__(AsgCfg<NP>::kThreads, 1)
         }
         for (int a = 0; a < 2; ++a) {
             ptx::mbar_init(&tfull[a], 1);
-            ptx::mbar_init(&tempty[a], 4 * 32);
+            ptx::mbar_init(&tempty[a], Cfg::kEpiWarps * 32);
+            ptx::mbar_init(&afull[a], 1);
+            ptx::mbar_init(&aempty[a], 1);
+            ptx::mbar_init(&redfull[a], kBM);
+            ptx::mbar_init(&redempty[a], kBM);
         }
         ptx::mbar_init(drain, 1);
         *abort_flag = 0u;
@@ -118,12 +156,32 @@ __global__ void __launch_bounds__(AsgCfg<NP>::kThreads, 1)
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
-            uint32_t stage = 0, phase = 0;
-            uint32_t issued_mask = 0, issued_par = 0;  // per stage: loaded at least once,
-                                                       // parity of the last load
+            uint32_t stage = 0, phase = 0, mbi = 0;
+            uint32_t issued_mask = 0, issued_par = 0;    // ring stages: loaded, last parity
+            uint32_t a_mask = 0, a_par = 0;              // resident X buffers
             bool ok = true;
-            for (int64_t mb = blockIdx.x; mb < nmb && ok; mb += gridDim.x) {
+            for (int64_t mb = blockIdx.x; mb < nmb && ok; mb += gridDim.x, ++mbi) {
                 const int row0 = static_cast<int>(mb * kBM);
+                if (RES) {
+                    const uint32_t ab = mbi % Cfg::kABufs;
+                    const uint32_t apar = (mbi / Cfg::kABufs) & 1u;
+                    if (!ptx::mbar_wait(&aempty[ab], apar ^ 1u, abort_flag, wait_ns)) {
+                        raise_timeout(abort_flag, err);
+                        ok = false;
+                        break;
+                    }
+                    ptx::mbar_arrive_expect_tx(&afull[ab], nkc * NP * Cfg::kABytes);
+                    uint8_t *ar = smem + ab * Cfg::kABufBytes;
+                    for (int kc = 0; kc < nkc; ++kc) {
+                        ptx::tma_load_2d(ar + (kc * NP) * Cfg::kABytes, &tmA0, &afull[ab],
+                                         kc * kBK, row0);
+                        if (NP == 2)
+                            ptx::tma_load_2d(ar + (kc * NP + 1) * Cfg::kABytes, &tmA1,
+                                             &afull[ab], kc * kBK, row0);
+                    }
+                    a_mask |= 1u << ab;
+                    a_par = (a_par & ~(1u << ab)) | (apar << ab);
+                }
                 for (int nt = 0; nt < ntiles && ok; ++nt) {
                     for (int kc = 0; kc < nkc; ++kc) {
                         if (!ptx::mbar_wait(&empty[stage], phase ^ 1u, abort_flag, wait_ns)) {
@@ -132,12 +190,15 @@ __global__ void __launch_bounds__(AsgCfg<NP>::kThreads, 1)
                             break;
                         }
                         ptx::mbar_arrive_expect_tx(&full[stage], Cfg::kStageBytes);
-                        uint8_t *st = smem + stage * Cfg::kStageBytes;
-                        ptx::tma_load_2d(st, &tmA0, &full[stage], kc * kBK, row0);
-                        if (NP == 2)
-                            ptx::tma_load_2d(st + Cfg::kABytes, &tmA1, &full[stage], kc * kBK,
-                                             row0);
-                        uint8_t *sb = st + NP * Cfg::kABytes;
+                        uint8_t *st = ring + stage * Cfg::kStageBytes;
+                        uint8_t *sb = st;
+                        if (!RES) {
+                            ptx::tma_load_2d(st, &tmA0, &full[stage], kc * kBK, row0);
+                            if (NP == 2)
+                                ptx::tma_load_2d(st + Cfg::kABytes, &tmA1, &full[stage],
+                                                 kc * kBK, row0);
+                            sb = st + NP * Cfg::kABytes;
+                        }
                         ptx::tma_load_2d(sb, &tmB0, &full[stage], kc * kBK, nt * kBN);
                         if (NP == 2)
                             ptx::tma_load_2d(sb + Cfg::kBBytes, &tmB1, &full[stage], kc * kBK,
@@ -156,15 +217,30 @@ __global__ void __launch_bounds__(AsgCfg<NP>::kThreads, 1)
                 for (int s = 0; s < S; ++s)
                     if (issued_mask & (1u << s))
                         ptx::mbar_wait(&full[s], (issued_par >> s) & 1u, nullptr, wait_ns);
+                for (int s = 0; s < 2; ++s)
+                    if (a_mask & (1u << s))
+                        ptx::mbar_wait(&afull[s], (a_par >> s) & 1u, nullptr, wait_ns);
             }
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             constexpr uint32_t idesc = ptx::idesc_bf16_f32(kBM, kBN);
-            uint32_t stage = 0, phase = 0, titer = 0;
+            uint32_t stage = 0, phase = 0, titer = 0, mbi = 0;
             bool ok = true;
-            for (int64_t mb = blockIdx.x; mb < nmb && ok; mb += gridDim.x) {
+            for (int64_t mb = blockIdx.x; mb < nmb && ok; mb += gridDim.x, ++mbi) {
+                uint32_t abase = 0, ab = 0;
+                if (RES) {
+                    ab = mbi % Cfg::kABufs;
+                    const uint32_t apar = (mbi / Cfg::kABufs) & 1u;
+                    if (!ptx::mbar_wait(&afull[ab], apar, abort_flag, wait_ns)) {
+                        raise_timeout(abort_flag, err);
+                        ok = false;
+                        break;
+                    }
+                    ptx::tc_fence_after();
+                    abase = ptx::smem_u32(smem + ab * Cfg::kABufBytes);
+                }
                 for (int nt = 0; nt < ntiles && ok; ++nt, ++titer) {
                     const uint32_t acc = titer & 1u;
                     const uint32_t aphase = (titer >> 1) & 1u;
@@ -182,9 +258,10 @@ __global__ void __launch_bounds__(AsgCfg<NP>::kThreads, 1)
                             break;
                         }
                         ptx::tc_fence_after();
-                        const uint32_t a0 = ptx::smem_u32(smem + stage * Cfg::kStageBytes);
+                        const uint32_t st = ptx::smem_u32(ring + stage * Cfg::kStageBytes);
+                        const uint32_t a0 = RES ? abase + (kc * NP) * Cfg::kABytes : st;
                         const uint32_t a1 = a0 + Cfg::kABytes;
-                        const uint32_t b0 = a0 + NP * Cfg::kABytes;
+                        const uint32_t b0 = RES ? st : st + NP * Cfg::kABytes;
                         const uint32_t b1 = b0 + Cfg::kBBytes;
 #pragma unroll
                         for (int ks = 0; ks < kBK / 16; ++ks) {
@@ -208,6 +285,7 @@ __global__ void __launch_bounds__(AsgCfg<NP>::kThreads, 1)
                     if (!ok) break;
                     ptx::mma_commit(&tfull[acc]);
                 }
+                if (RES && ok) ptx::mma_commit(&aempty[ab]);  // X buffer free after these MMAs
             }
             if (!ok) {
                 // Make sure no MMA issued by this thread is still writing tensor memory.
@@ -217,11 +295,14 @@ __global__ void __launch_bounds__(AsgCfg<NP>::kThreads, 1)
         }
     } else {
         // ------------------------------------------------------------ epilogue
-        const int q = warp & 3;  // TMEM lane quarter this warp may access
+        // Warpgroup g (warps 2-5: g = 0, warps 6-9: g = 1) scans columns [128 g, 128 g + 128)
+        // of every tile; warp w may read TMEM lanes 32 (w % 4) .. 32 (w % 4) + 31, i.e. rows.
+        const int g = (warp - 2) >> 2;
+        const int q = warp & 3;
         const int r = q * 32 + lane;
-        uint32_t titer = 0;
+        uint32_t titer = 0, mbi = 0;
         bool ok = true;
-        for (int64_t mb = blockIdx.x; mb < nmb && ok; mb += gridDim.x) {
+        for (int64_t mb = blockIdx.x; mb < nmb && ok; mb += gridDim.x, ++mbi) {
             float best = __int_as_float(0x7f800000);
             int bestk = 0;
             for (int nt = 0; nt < ntiles; ++nt, ++titer) {
@@ -233,42 +314,68 @@ __global__ void __launch_bounds__(AsgCfg<NP>::kThreads, 1)
                     break;
                 }
                 ptx::tc_fence_after();
-                const uint32_t tbase = tmem + (static_cast<uint32_t>(q * 32) << 16) + acc * kBN;
-                const float4 *cn4 = reinterpret_cast<const float4 *>(cn + nt * kBN);
+                const uint32_t tb = tmem + (static_cast<uint32_t>(q * 32) << 16) + acc * kBN +
+                                    g * (kBN / 2);
+                const int colbase = nt * kBN + g * (kBN / 2);
+                const float4 *cn4 = reinterpret_cast<const float4 *>(cn + colbase);
 #pragma unroll 1
-                for (int ch = 0; ch < kBN / 32; ++ch) {
+                for (int h = 0; h < 2; ++h) {
                     __syncwarp();
-                    float v[32];
-                    ptx::tmem_ld32_sync(tbase + ch * 32, v);
+                    float v[64];
+                    ptx::tmem_ld64_sync(tb + h * 64, v);
 #pragma unroll
-                    for (int j4 = 0; j4 < 8; ++j4) {
-                        const float4 c = __ldg(cn4 + ch * 8 + j4);
+                    for (int j4 = 0; j4 < 16; ++j4) {
+                        const float4 c = __ldg(cn4 + h * 16 + j4);
                         v[4 * j4 + 0] += c.x;
                         v[4 * j4 + 1] += c.y;
                         v[4 * j4 + 2] += c.z;
                         v[4 * j4 + 3] += c.w;
                     }
-                    float m = v[0];
-#pragma unroll
-                    for (int j = 1; j < 32; ++j) m = fminf(m, v[j]);
+                    const float m = min64(v);
                     if (m < best) {
                         int idx = 0;
 #pragma unroll
-                        for (int j = 31; j >= 0; --j)
+                        for (int j = 63; j >= 0; --j)
                             if (v[j] == m) idx = j;
                         best = m;
-                        bestk = nt * kBN + ch * 32 + idx;
+                        bestk = colbase + h * 64 + idx;
                     }
                 }
                 ptx::tc_fence_before();
                 ptx::mbar_arrive(&tempty[acc]);
             }
             if (!ok) break;
-            const int64_t row = mb * kBM + r;
-            if (row < N) {
-                labels[row] = bestk;
-                if (best_out) best_out[row] = best;
-                if (mind) mind[row] = xnorm[row] + best;
+            // combine the two column halves of each row: (min, lowest index)
+            const uint32_t slot = mbi & 1u;
+            const uint32_t spar = (mbi >> 1) & 1u;
+            if (g == 1) {
+                if (!warp_wait(&redempty[slot], spar ^ 1u, abort_flag, wait_ns)) {
+                    if (lane == 0) raise_timeout(abort_flag, err);
+                    ok = false;
+                    break;
+                }
+                red_v[slot * kBM + r] = best;
+                red_k[slot * kBM + r] = bestk;
+                ptx::mbar_arrive(&redfull[slot]);
+            } else {
+                if (!warp_wait(&redfull[slot], spar, abort_flag, wait_ns)) {
+                    if (lane == 0) raise_timeout(abort_flag, err);
+                    ok = false;
+                    break;
+                }
+                const float b1 = red_v[slot * kBM + r];
+                const int k1 = red_k[slot * kBM + r];
+                ptx::mbar_arrive(&redempty[slot]);
+                if (b1 < best || (b1 == best && k1 < bestk)) {
+                    best = b1;
+                    bestk = k1;
+                }
+                const int64_t row = mb * kBM + r;
+                if (row < N) {
+                    labels[row] = bestk;
+                    if (best_out) best_out[row] = best;
+                    if (mind) mind[row] = xnorm[row] + best;
+                }
             }
         }
     }
@@ -312,9 +419,31 @@ bool make_tmap(CUtensorMap *m, const void *base, int64_t rows, int64_t cols,
     return r == CUDA_SUCCESS;
 }
 
+template <int NP, bool RES>
+cudaError_t launch_assign_cfg(const AssignArgs &a, const CUtensorMap (&tA)[2],
+                              const CUtensorMap (&tB)[2], cudaStream_t st) {
+    using Cfg = AsgCfg<NP, RES>;
+    static bool attr_set = false;
+    if (!attr_set) {
+        cudaError_t e = cudaFuncSetAttribute(assign_kernel<NP, RES>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             Cfg::kSmemBytes);
+        if (e != cudaSuccess) return e;
+        attr_set = true;
+    }
+    const int64_t nmb = ceil_div(a.N, kBM);
+    const int64_t sms = device_sm_count();
+    const int grid = static_cast<int>(nmb < sms ? nmb : sms);
+    assign_kernel<NP, RES><<<grid, Cfg::kThreads, Cfg::kSmemBytes, st>>>(
+        tA[0], tA[1], tB[0], tB[1], a.cn, a.N, static_cast<int>(a.dp / kBK),
+        static_cast<int>(a.Kp / kBN), nmb, a.labels, a.best, a.xnorm, a.mind, a.err,
+        a.wait_ns);
+    note_launch();
+    return cudaGetLastError();
+}
+
 template <int NP>
 cudaError_t launch_assign_np(const AssignArgs &a, cudaStream_t st) {
-    using Cfg = AsgCfg<NP>;
     CUtensorMap tA[2], tB[2];
     const uint16_t *ap = static_cast<const uint16_t *>(a.a_planes);
     const uint16_t *bp = static_cast<const uint16_t *>(a.b_planes);
@@ -329,22 +458,14 @@ cudaError_t launch_assign_np(const AssignArgs &a, cudaStream_t st) {
         tA[1] = tA[0];
         tB[1] = tB[0];
     }
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(
-            assign_kernel<NP>, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes);
-        if (e != cudaSuccess) return e;
-        attr_set = true;
-    }
-    const int64_t nmb = ceil_div(a.N, kBM);
-    const int64_t sms = device_sm_count();
-    const int grid = static_cast<int>(nmb < sms ? nmb : sms);
-    assign_kernel<NP><<<grid, Cfg::kThreads, Cfg::kSmemBytes, st>>>(
-        tA[0], tA[1], tB[0], tB[1], a.cn, a.N, static_cast<int>(a.dp / kBK),
-        static_cast<int>(a.Kp / kBN), nmb, a.labels, a.best, a.xnorm, a.mind, a.err,
-        a.wait_ns);
-    note_launch();
-    return cudaGetLastError();
+    // X block resident in shared memory when it fits (d <= 128) and, for the fp32
+    // emulation (one X buffer, so a short gap at each new block), when the sweep over
+    // the centroid tiles is long enough to hide that gap.
+    const int nkc = a.dp / kBK;
+    const int ntiles = a.Kp / kBN;
+    const bool res = nkc <= 2 && (NP == 1 || ntiles >= 16);
+    if (res) return launch_assign_cfg<NP, true>(a, tA, tB, st);
+    return launch_assign_cfg<NP, false>(a, tA, tB, st);
 }
 
 }  // namespace

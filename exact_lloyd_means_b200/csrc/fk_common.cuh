@@ -22,9 +22,10 @@ constexpr int kSortTile = kSortThreads * kSortItems;  // keys per block
 constexpr int kSortMaxBits = 11;                      // digit width bound: 2048 bins
 
 // ----------------------------------------------------------------- update tiling
-constexpr int kRowsPerWarp = 512;  // sorted positions per warp chunk
-constexpr int kUpdWarps = 8;
-constexpr int kMaxSlices = 8;      // 128-column slices per lane group (d <= 1024 per pass)
+constexpr int kUpdWarps = 8;          // warps per block of the level-1 kernel
+constexpr int kUpdMinRows = 32;       // smallest chunk of sorted positions per warp
+constexpr int kUpdMaxRows = 256;      // largest chunk
+constexpr int64_t kUpdTargetWarps = 148 * 64;  // enough warps to cover the GPU twice
 
 // Objective slots kept on the device by fk_lloyd before a copy to the host.
 constexpr int kObjRing = 4096;
@@ -63,20 +64,26 @@ inline SortPlan sort_plan(int64_t N, int K) {
     return p;
 }
 
+// Level-1 work split of the update: a warp owns `rows` consecutive sorted positions and one
+// 128-column block of the rows (grid.y = column blocks), so a 3 KB row (d = 768) is read
+// by six warps as six contiguous 512-byte pieces.  `rows` is a power of two chosen so the
+// grid has enough warps to hide memory latency even for small N.
 struct UpdPlan {
-    int slices = 1;    // 128-column slices per pass
-    int ncolblk = 1;   // column passes
-    int dcov = 128;    // padded row length covered by the passes
-    int64_t nwarps = 0;
+    int ncolblk = 1;   // 128-column blocks
+    int dcov = 128;    // padded row length of a piece (ncolblk * 128)
+    int rows = kUpdMaxRows;
+    int64_t nwarps = 0;  // warps per column block
 };
 
 inline UpdPlan upd_plan(int64_t N, int d) {
     UpdPlan p;
-    int sl = static_cast<int>(ceil_div(d, 128));
-    p.slices = sl < kMaxSlices ? sl : kMaxSlices;
-    p.ncolblk = static_cast<int>(ceil_div(d, 128 * p.slices));
-    p.dcov = p.ncolblk * 128 * p.slices;
-    p.nwarps = ceil_div(N, kRowsPerWarp);
+    p.ncolblk = static_cast<int>(ceil_div(d, 128));
+    p.dcov = p.ncolblk * 128;
+    int64_t r = N * p.ncolblk / kUpdTargetWarps;
+    int rows = kUpdMinRows;
+    while (rows < kUpdMaxRows && rows * 2 <= r) rows *= 2;
+    p.rows = rows;
+    p.nwarps = ceil_div(N, rows);
     return p;
 }
 

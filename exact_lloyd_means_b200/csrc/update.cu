@@ -7,17 +7,18 @@
 // "为什么"快"这件事被拖了这么久"); an empty cluster keeps its previous centroid.
 //
 // B200 design:
-//   level 1  : the sorted order [0, N) is cut into fixed chunks of 512 positions, one per
-//              warp, independent of where clusters start.  A warp gathers its rows through
-//              perm (each row is d contiguous values, read as 16-byte vectors across the
-//              lanes, several rows in flight), adds them in position order in fp64 and,
+//   level 1  : the sorted order [0, N) is cut into fixed chunks of R positions (a power of
+//              two, 32..256, chosen from N), one per warp and 128-column block, independent
+//              of where clusters start.  A warp gathers its rows through perm (512
+//              contiguous bytes of a row per warp, read as 16-byte vectors across the lanes,
+//              eight rows in flight), adds them in position order in fp64 and,
 //              whenever the cluster id changes, either finishes the cluster (all of it
 //              lies in this chunk: mean = sum / count, rounded once to fp32) or emits a
 //              "piece" (the chunk's first or last cluster, which continues outside).  The
 //              same pass accumulates the objective sum ||x - c_used[label]||^2 in fp64.
 //   level L>1: groups of 64 consecutive units of the previous level are reduced the same
 //              way over their pieces, in piece order.  A cluster is finished at the first
-//              level whose unit (512 * 64^(L-1) positions) contains all of it, so a
+//              level whose unit (R * 64^(L-1) positions) contains all of it, so a
 //              cluster with millions of points is split over thousands of warps at
 //              level 1 and finished after a few levels with short, parallel sums.
 //   finalize : counts from the CSR offsets; empty clusters copy C_old bit for bit.
@@ -33,23 +34,6 @@ namespace {
 
 constexpr int kGroup = 64;  // units of level L-1 per unit of level L
 
-template <bool BF16>
-__device__ __forceinline__ void load4(const void *X, int64_t off, float (&v)[4]) {
-    if constexpr (BF16) {
-        const uint2 u = *reinterpret_cast<const uint2 *>(static_cast<const uint16_t *>(X) + off);
-        v[0] = __uint_as_float(u.x << 16);
-        v[1] = __uint_as_float(u.x & 0xffff0000u);
-        v[2] = __uint_as_float(u.y << 16);
-        v[3] = __uint_as_float(u.y & 0xffff0000u);
-    } else {
-        const float4 f = *reinterpret_cast<const float4 *>(static_cast<const float *>(X) + off);
-        v[0] = f.x;
-        v[1] = f.y;
-        v[2] = f.z;
-        v[3] = f.w;
-    }
-}
-
 // Write the mean of a finished cluster: C_new[k][col..col+3] = acc / cnt.
 __device__ __forceinline__ void store_mean(float *C_new, int64_t k, int d, int col,
                                            const double (&acc)[4], double cnt) {
@@ -61,108 +45,176 @@ __device__ __forceinline__ void store_mean(float *C_new, int64_t k, int d, int c
     *reinterpret_cast<float4 *>(C_new + k * d + col) = o;
 }
 
-// Level 1.  grid.x covers warps (8 per block), grid.y the column passes.
-template <int SL, bool BF16>
-__global__ void __launch_bounds__(kUpdWarps * 32)
-    seg_rows_kernel(const void *__restrict__ X, int64_t N, int d, int64_t nwarps, int dcov,
-                    const int32_t *__restrict__ skeys, const int32_t *__restrict__ perm,
-                    const int32_t *__restrict__ offsets, const float *__restrict__ C_used,
-                    float *__restrict__ C_new, double *__restrict__ pieces,
-                    int32_t *__restrict__ pkeys, double *__restrict__ jpart) {
-    constexpr int B = SL >= 4 ? 2 : (SL >= 2 ? 4 : 8);  // rows in flight per lane
+__device__ __forceinline__ void store_piece(double *dst, const double (&acc)[4]) {
+    double2 *q = reinterpret_cast<double2 *>(dst);
+    q[0] = make_double2(acc[0], acc[1]);
+    q[1] = make_double2(acc[2], acc[3]);
+}
+
+// Level 1.  A warp owns sorted positions [w*R, w*R + R) and the 128 columns of block
+// blockIdx.y (lane l holds columns 4l .. 4l+3).  The warp first stages the R cluster ids
+// and row ids of its chunk in shared memory (one coalesced read), so row fetches never
+// wait on an index load; rows are then fetched B at a time (B = 8 fp32 / 16 bf16 rows,
+// 16 / 8 bytes per lane per row) with the next batch in flight while the current one is
+// added.  When a batch lies in one cluster its rows are first added pairwise in fp32 (a
+// fixed tree) and the batch sum is added to the fp64 accumulator once; otherwise rows are
+// added one by one in fp64.  The objective term (x - c_used)^2 of a row is formed in fp32
+// and accumulated in fp64.
+template <bool BF16>
+struct RowVec;
+template <>
+struct RowVec<false> {
+    using T = float4;
+    static constexpr int kBatch = 8;
+    __device__ static void unpack(const float4 &v, float (&f)[4]) {
+        f[0] = v.x;
+        f[1] = v.y;
+        f[2] = v.z;
+        f[3] = v.w;
+    }
+    __device__ static float4 zero() { return make_float4(0.f, 0.f, 0.f, 0.f); }
+};
+template <>
+struct RowVec<true> {
+    using T = uint2;
+    static constexpr int kBatch = 16;
+    __device__ static void unpack(const uint2 &u, float (&f)[4]) {
+        f[0] = __uint_as_float(u.x << 16);
+        f[1] = __uint_as_float(u.x & 0xffff0000u);
+        f[2] = __uint_as_float(u.y << 16);
+        f[3] = __uint_as_float(u.y & 0xffff0000u);
+    }
+    __device__ static uint2 zero() { return make_uint2(0u, 0u); }
+};
+
+template <bool BF16>
+__global__ void __launch_bounds__(kUpdWarps * 32, 2)
+    seg_rows_kernel(const void *__restrict__ X, int64_t N, int d, int R, int64_t nwarps,
+                    int dcov, const int32_t *__restrict__ skeys,
+                    const int32_t *__restrict__ perm, const int32_t *__restrict__ offsets,
+                    const float *__restrict__ C_used, float *__restrict__ C_new,
+                    double *__restrict__ pieces, int32_t *__restrict__ pkeys,
+                    double *__restrict__ jpart) {
+    using RV = RowVec<BF16>;
+    using V = typename RV::T;
+    constexpr int B = RV::kBatch;
+    __shared__ int32_t s_key[kUpdWarps][kUpdMaxRows];
+    __shared__ int32_t s_row[kUpdWarps][kUpdMaxRows];
     const int lane = threadIdx.x & 31;
-    const int64_t w = static_cast<int64_t>(blockIdx.x) * kUpdWarps + (threadIdx.x >> 5);
+    const int wib = threadIdx.x >> 5;
+    const int64_t w = static_cast<int64_t>(blockIdx.x) * kUpdWarps + wib;
     if (w >= nwarps) return;
     const int cb = blockIdx.y;
-    const int col0 = cb * 128 * SL;
-    const int64_t p0 = w * kRowsPerWarp;
-    const int64_t p1 = p0 + kRowsPerWarp < N ? p0 + kRowsPerWarp : N;
+    const int col = cb * 128 + lane * 4;
+    const bool colv = col < d;
+    const int64_t p0 = w * R;
+    const int n = static_cast<int>((p0 + R < N ? p0 + R : N) - p0);
+    const int64_t p1 = p0 + n;
+    int32_t *sk = s_key[wib];
+    int32_t *si = s_row[wib];
+    for (int j = lane; j < n; j += 32) {
+        sk[j] = skeys[p0 + j];
+        si[j] = perm[p0 + j];
+    }
+    __syncwarp();
 
-    double acc[SL][4];
-    float cu[SL][4];
+    const V *Xv = static_cast<const V *>(X);
+    double acc[4] = {0.0, 0.0, 0.0, 0.0};
+    float cu[4] = {0.f, 0.f, 0.f, 0.f};
     double jacc = 0.0;
     int cur = -1, first = -1, slot1 = -1;
 
     auto flush = [&](int k) {
         const int64_t lo = offsets[k], hi = offsets[k + 1];
         if (lo >= p0 && hi <= p1) {
-            const double cnt = static_cast<double>(hi - lo);
-#pragma unroll
-            for (int s = 0; s < SL; ++s) {
-                const int col = col0 + s * 128 + lane * 4;
-                if (col < d) store_mean(C_new, k, d, col, acc[s], cnt);
-            }
+            if (colv) store_mean(C_new, k, d, col, acc, static_cast<double>(hi - lo));
         } else {
             const int slot = (k == first) ? 0 : 1;
             if (slot == 1) slot1 = k;
-            double *dst = pieces + (w * 2 + slot) * static_cast<int64_t>(dcov) + col0;
+            store_piece(pieces + (w * 2 + slot) * static_cast<int64_t>(dcov) + col, acc);
+        }
+    };
+    auto start = [&](int k) {
+        if (cur >= 0) flush(cur);
+        if (cur < 0) first = k;
+        cur = k;
+        acc[0] = acc[1] = acc[2] = acc[3] = 0.0;
+        if (colv) {
+            const float4 c = *reinterpret_cast<const float4 *>(C_used + int64_t(k) * d + col);
+            cu[0] = c.x;
+            cu[1] = c.y;
+            cu[2] = c.z;
+            cu[3] = c.w;
+        }
+    };
+    auto issue = [&](int b, V (&buf)[B]) {
 #pragma unroll
-            for (int s = 0; s < SL; ++s) {
-                double2 *q = reinterpret_cast<double2 *>(dst + s * 128 + lane * 4);
-                q[0] = make_double2(acc[s][0], acc[s][1]);
-                q[1] = make_double2(acc[s][2], acc[s][3]);
+        for (int j = 0; j < B; ++j) {
+            const int q = b + j;
+            buf[j] = (q < n && colv)
+                         ? __ldg(Xv + (static_cast<int64_t>(si[q]) * d + col) / 4)
+                         : RV::zero();
+        }
+    };
+    auto process = [&](int b, const V (&buf)[B]) {
+        const int nb = n - b < B ? n - b : B;
+        const int kf = sk[b], kl = sk[b + nb - 1];
+        if (kf == kl) {
+            if (kf != cur) start(kf);
+            float xs[B][4];
+            float jr[B];
+#pragma unroll
+            for (int j = 0; j < B; ++j) {
+                RV::unpack(buf[j], xs[j]);
+                float t = 0.f;
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float df = j < nb ? xs[j][e] - cu[e] : 0.f;
+                    t = fmaf(df, df, t);
+                }
+                jr[j] = t;
+            }
+#pragma unroll
+            for (int h = B / 2; h > 0; h >>= 1) {
+#pragma unroll
+                for (int j = 0; j < h; ++j) {
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) xs[j][e] += xs[j + h][e];
+                    jr[j] += jr[j + h];
+                }
+            }
+#pragma unroll
+            for (int e = 0; e < 4; ++e) acc[e] += static_cast<double>(xs[0][e]);
+            jacc += static_cast<double>(jr[0]);
+        } else {
+#pragma unroll
+            for (int j = 0; j < B; ++j) {
+                if (j < nb) {
+                    const int k = sk[b + j];
+                    if (k != cur) start(k);
+                    float x[4];
+                    RV::unpack(buf[j], x);
+                    float t = 0.f;
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        acc[e] += static_cast<double>(x[e]);
+                        const float df = x[e] - cu[e];
+                        t = fmaf(df, df, t);
+                    }
+                    jacc += static_cast<double>(t);
+                }
             }
         }
     };
 
-    for (int64_t p = p0; p < p1; p += B) {
-        const int nb = p1 - p < B ? static_cast<int>(p1 - p) : B;
-        int myk = 0, myi = 0;
-        if (lane < nb) {
-            myk = skeys[p + lane];
-            myi = perm[p + lane];
-        }
-        float xr[B][SL][4];
-#pragma unroll
-        for (int j = 0; j < B; ++j) {
-            const int i = __shfl_sync(0xffffffffu, myi, j);
-#pragma unroll
-            for (int s = 0; s < SL; ++s) {
-                const int col = col0 + s * 128 + lane * 4;
-                if (j < nb && col < d) {
-                    load4<BF16>(X, static_cast<int64_t>(i) * d + col, xr[j][s]);
-                } else {
-                    xr[j][s][0] = xr[j][s][1] = xr[j][s][2] = xr[j][s][3] = 0.f;
-                }
-            }
-        }
-#pragma unroll
-        for (int j = 0; j < B; ++j) {
-            const int k = __shfl_sync(0xffffffffu, myk, j);
-            if (j < nb) {
-                if (k != cur) {
-                    if (cur >= 0) flush(cur);
-                    if (cur < 0) first = k;
-                    cur = k;
-#pragma unroll
-                    for (int s = 0; s < SL; ++s) {
-                        const int col = col0 + s * 128 + lane * 4;
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) acc[s][e] = 0.0;
-                        if (col < d) {
-                            const float4 c =
-                                *reinterpret_cast<const float4 *>(C_used + int64_t(k) * d + col);
-                            cu[s][0] = c.x;
-                            cu[s][1] = c.y;
-                            cu[s][2] = c.z;
-                            cu[s][3] = c.w;
-                        } else {
-                            cu[s][0] = cu[s][1] = cu[s][2] = cu[s][3] = 0.f;
-                        }
-                    }
-                }
-#pragma unroll
-                for (int s = 0; s < SL; ++s) {
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const double xv = xr[j][s][e];
-                        acc[s][e] += xv;
-                        const double df = xv - static_cast<double>(cu[s][e]);
-                        jacc += df * df;
-                    }
-                }
-            }
-        }
+    V bufA[B], bufB[B];
+    issue(0, bufA);
+    for (int b = 0; b < n; b += 2 * B) {
+        issue(b + B, bufB);
+        process(b, bufA);
+        if (b + B >= n) break;
+        issue(b + 2 * B, bufA);
+        process(b + B, bufB);
     }
     if (cur >= 0) flush(cur);
     if (cb == 0 && lane == 0) {
@@ -178,22 +230,30 @@ __global__ void __launch_bounds__(kUpdWarps * 32)
 }
 
 // Level L >= 2: one warp per group of kGroup units of the previous level (2 piece slots
-// each).  `span` = positions covered by one unit of THIS level.
-template <int SL>
+// each), one 128-column block per grid.y.  `span` = sorted positions covered by one unit
+// of THIS level.  The group's slot keys are staged in shared memory first and the pieces
+// are read 8 slots at a time, so the loop is not a chain of dependent loads.
 __global__ void __launch_bounds__(kUpdWarps * 32)
     seg_pieces_kernel(const double *__restrict__ pin, const int32_t *__restrict__ kin,
                       int64_t nslots_in, double *__restrict__ pout,
                       int32_t *__restrict__ kout, int64_t nunits, int64_t span, int d,
                       int dcov, const int32_t *__restrict__ offsets, float *__restrict__ C_new) {
+    constexpr int S = 2 * kGroup;
+    constexpr int B = 8;
+    __shared__ int32_t s_key[kUpdWarps][S];
     const int lane = threadIdx.x & 31;
-    const int64_t u = static_cast<int64_t>(blockIdx.x) * kUpdWarps + (threadIdx.x >> 5);
+    const int wib = threadIdx.x >> 5;
+    const int64_t u = static_cast<int64_t>(blockIdx.x) * kUpdWarps + wib;
     if (u >= nunits) return;
     const int cb = blockIdx.y;
-    const int col0 = cb * 128 * SL;
-    const int64_t s0 = u * 2 * kGroup;
-    const int64_t s1 = s0 + 2 * kGroup < nslots_in ? s0 + 2 * kGroup : nslots_in;
+    const int col = cb * 128 + lane * 4;
+    const int64_t s0 = u * S;
+    const int ns = static_cast<int>((s0 + S < nslots_in ? s0 + S : nslots_in) - s0);
+    int32_t *sk = s_key[wib];
+    for (int j = lane; j < ns; j += 32) sk[j] = kin[s0 + j];
+    __syncwarp();
 
-    double acc[SL][4];
+    double acc[4] = {0.0, 0.0, 0.0, 0.0};
     int cur = -1, first = -1, slot1 = -1;
     bool first_done = false;
 
@@ -202,52 +262,45 @@ __global__ void __launch_bounds__(kUpdWarps * 32)
         const bool done = (lo / span) == ((hi - 1) / span);
         if (k == first) first_done = done;
         if (done) {
-            const double cnt = static_cast<double>(hi - lo);
-#pragma unroll
-            for (int s = 0; s < SL; ++s) {
-                const int col = col0 + s * 128 + lane * 4;
-                if (col < d) store_mean(C_new, k, d, col, acc[s], cnt);
-            }
+            if (col < d) store_mean(C_new, k, d, col, acc, static_cast<double>(hi - lo));
         } else {
             const int slot = (k == first) ? 0 : 1;
             if (slot == 1) slot1 = k;
-            double *dst = pout + (u * 2 + slot) * static_cast<int64_t>(dcov) + col0;
-#pragma unroll
-            for (int s = 0; s < SL; ++s) {
-                double2 *q = reinterpret_cast<double2 *>(dst + s * 128 + lane * 4);
-                q[0] = make_double2(acc[s][0], acc[s][1]);
-                q[1] = make_double2(acc[s][2], acc[s][3]);
-            }
+            store_piece(pout + (u * 2 + slot) * static_cast<int64_t>(dcov) + col, acc);
         }
     };
 
-    for (int64_t sl = s0; sl < s1; ++sl) {
-        const int k = kin[sl];
-        if (k < 0) continue;
-        const double *src = pin + sl * static_cast<int64_t>(dcov) + col0;
-        double v[SL][4];
+    for (int b = 0; b < ns; b += B) {
+        double2 va[B], vb[B];
 #pragma unroll
-        for (int s = 0; s < SL; ++s) {
-            const double2 *q = reinterpret_cast<const double2 *>(src + s * 128 + lane * 4);
-            const double2 a = q[0], b = q[1];
-            v[s][0] = a.x;
-            v[s][1] = a.y;
-            v[s][2] = b.x;
-            v[s][3] = b.y;
-        }
-        if (k != cur) {
-            if (cur >= 0) flush(cur);
-            if (cur < 0) first = k;
-            cur = k;
-#pragma unroll
-            for (int s = 0; s < SL; ++s)
-#pragma unroll
-                for (int e = 0; e < 4; ++e) acc[s][e] = 0.0;
+        for (int j = 0; j < B; ++j) {
+            const int q = b + j;
+            if (q < ns && sk[q] >= 0) {
+                const double2 *src =
+                    reinterpret_cast<const double2 *>(pin + (s0 + q) * int64_t(dcov) + col);
+                va[j] = src[0];
+                vb[j] = src[1];
+            } else {
+                va[j] = vb[j] = make_double2(0.0, 0.0);
+            }
         }
 #pragma unroll
-        for (int s = 0; s < SL; ++s)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) acc[s][e] += v[s][e];
+        for (int j = 0; j < B; ++j) {
+            const int q = b + j;
+            if (q >= ns) break;
+            const int k = sk[q];
+            if (k < 0) continue;
+            if (k != cur) {
+                if (cur >= 0) flush(cur);
+                if (cur < 0) first = k;
+                cur = k;
+                acc[0] = acc[1] = acc[2] = acc[3] = 0.0;
+            }
+            acc[0] += va[j].x;
+            acc[1] += va[j].y;
+            acc[2] += vb[j].x;
+            acc[3] += vb[j].y;
+        }
     }
     if (cur >= 0) flush(cur);
     if (cb == 0 && lane == 0) {
@@ -286,7 +339,6 @@ __global__ void __launch_bounds__(1024)
     if (threadIdx.x == 0) *out = sh[0];
 }
 
-template <int SL>
 cudaError_t run_levels(const void *X, bool bf16, int64_t N, int d, const UpdPlan &up,
                        const int32_t *skeys, const int32_t *perm, const int32_t *offsets,
                        const float *C_used, float *C_new, double *pa, int32_t *ka,
@@ -294,24 +346,24 @@ cudaError_t run_levels(const void *X, bool bf16, int64_t N, int d, const UpdPlan
     const dim3 block(kUpdWarps * 32);
     dim3 grid(static_cast<unsigned>(ceil_div(up.nwarps, kUpdWarps)), up.ncolblk);
     if (bf16)
-        seg_rows_kernel<SL, true><<<grid, block, 0, st>>>(X, N, d, up.nwarps, up.dcov, skeys,
-                                                          perm, offsets, C_used, C_new, pa, ka,
-                                                          jpart);
+        seg_rows_kernel<true><<<grid, block, 0, st>>>(X, N, d, up.rows, up.nwarps, up.dcov,
+                                                      skeys, perm, offsets, C_used, C_new, pa,
+                                                      ka, jpart);
     else
-        seg_rows_kernel<SL, false><<<grid, block, 0, st>>>(X, N, d, up.nwarps, up.dcov, skeys,
-                                                           perm, offsets, C_used, C_new, pa,
-                                                           ka, jpart);
+        seg_rows_kernel<false><<<grid, block, 0, st>>>(X, N, d, up.rows, up.nwarps, up.dcov,
+                                                       skeys, perm, offsets, C_used, C_new, pa,
+                                                       ka, jpart);
     note_launch();
     int64_t units = up.nwarps;
-    int64_t span = kRowsPerWarp;
+    int64_t span = up.rows;
     double *pin = pa, *pout = pb;
     int32_t *kin = ka, *kout = kb;
     while (units > 1) {
         const int64_t nunits = ceil_div(units, kGroup);
         span *= kGroup;
         dim3 g2(static_cast<unsigned>(ceil_div(nunits, kUpdWarps)), up.ncolblk);
-        seg_pieces_kernel<SL><<<g2, block, 0, st>>>(pin, kin, units * 2, pout, kout, nunits,
-                                                    span, d, up.dcov, offsets, C_new);
+        seg_pieces_kernel<<<g2, block, 0, st>>>(pin, kin, units * 2, pout, kout, nunits, span, d,
+                                                up.dcov, offsets, C_new);
         note_launch();
         units = nunits;
         double *tp = pin;
@@ -333,25 +385,8 @@ cudaError_t launch_update(const void *X, fk_dtype dtype, int64_t N, int d, int K
                           double *pieces_b, int32_t *pkeys_b, double *jpart,
                           double *objective, cudaStream_t st) {
     const bool bf16 = dtype == FK_BF16;
-    cudaError_t e;
-    switch (up.slices) {
-#define FK_SL(n)                                                                            \
-    case n:                                                                                 \
-        e = run_levels<n>(X, bf16, N, d, up, skeys, perm, offsets, C_used, C_new, pieces_a, \
-                          pkeys_a, pieces_b, pkeys_b, jpart, st);                           \
-        break;
-        FK_SL(1)
-        FK_SL(2)
-        FK_SL(3)
-        FK_SL(4)
-        FK_SL(5)
-        FK_SL(6)
-        FK_SL(7)
-        FK_SL(8)
-#undef FK_SL
-        default:
-            return cudaErrorInvalidValue;
-    }
+    cudaError_t e = run_levels(X, bf16, N, d, up, skeys, perm, offsets, C_used, C_new,
+                               pieces_a, pkeys_a, pieces_b, pkeys_b, jpart, st);
     if (e != cudaSuccess) return e;
     int64_t fgrid = ceil_div(K, 8);
     const int64_t cap = static_cast<int64_t>(device_sm_count()) * 16;
