@@ -14,10 +14,13 @@
 //     N=256, K=16 per instruction, accumulating a 128 x 256 fp32 tile in tensor memory;
 //     two accumulators (512 TMEM columns) so the epilogue of tile t overlaps the MMAs of
 //     tile t+1; tcgen05.commit releases smem stages and hands tiles to the epilogue;
-//   * warps 2..5 (128 threads, one per row / TMEM lane): epilogue.  tcgen05.ld 32 columns
-//     at a time, v = acc + ||c||^2 (the B operand holds -2c), chunk minimum, and a running
-//     (min, argmin) per row in registers; ties keep the lowest centroid index.  Only the
-//     label (and optionally the minimum) is written to HBM.
+//   * warps 2..17 (four warpgroups, one per 64-column quarter of the tile; within a group
+//     one thread per row / TMEM lane): epilogue.  tcgen05.ld of 64 columns, v = acc +
+//     ||c||^2 (the B operand holds -2c; the norms arrive in shared memory by bulk copy),
+//     a three-input-min reduction and a running (min, argmin) per row in registers; ties
+//     keep the lowest centroid index.  The four quarters are merged per 128-row block
+//     through mbarrier-guarded shared memory.  Only the label (and optionally the minimum)
+//     is written to HBM.
 //   * fp32 points (NP = 2): x.c is formed from three bf16 products hi*hi' + lo*hi' +
 //     hi*lo' into one fp32 accumulator (the X and centroid planes come split from prep).
 //     bf16 points (NP = 1): one product, exact in fp32.
@@ -43,16 +46,20 @@ struct AsgCfg {
     static constexpr int kABytes = kBM * kBK * 2;  // 16 KB: one X plane chunk
     static constexpr int kBBytes = kBN * kBK * 2;  // 32 KB: one centroid plane chunk
     static constexpr int kAChunks = RES ? 2 : 0;   // resident k-chunks (d <= 128)
-    static constexpr int kABufs = RES ? (NP == 1 ? 2 : 1) : 0;
+    static constexpr int kABufs = RES ? (NP == 1 ? 2 : 1) : 1;  // (1 unused when !RES)
     static constexpr int kABufBytes = kAChunks * NP * kABytes;
-    static constexpr int kARegion = kABufs * kABufBytes;
+    static constexpr int kARegion = RES ? kABufs * kABufBytes : 0;
     static constexpr int kStageBytes = RES ? NP * kBBytes : NP * (kABytes + kBBytes);
     static constexpr int kStages = RES ? (NP == 1 ? 4 : 2) : (NP == 2 ? 2 : 4);
     static constexpr int kDataBytes = kARegion + kStages * kStageBytes;  // 192 KB
     static constexpr int kBarBytes = 512;
-    static constexpr int kRedBytes = 2 * 2 * kBM * 4;  // per-row (min, argmin), 2 slots
-    static constexpr int kSmemBytes = kDataBytes + kBarBytes + kRedBytes + 1024;
-    static constexpr int kEpiWarps = 8;  // two warpgroups, one per half of the columns
+    static constexpr int kEpiGroups = 4;               // warpgroups splitting the columns
+    static constexpr int kEpiCols = kBN / kEpiGroups;  // 64 columns per group per tile
+    // per-row (min, argmin) of groups 1..3, two slots
+    static constexpr int kRedBytes = (kEpiGroups - 1) * 2 * kBM * 8;
+    static constexpr int kCnBytes = 2 * kBN * 4;       // ||c||^2 of the tile per accumulator
+    static constexpr int kSmemBytes = kDataBytes + kBarBytes + kRedBytes + kCnBytes + 1024;
+    static constexpr int kEpiWarps = 4 * kEpiGroups;
     static constexpr int kThreads = 64 + kEpiWarps * 32;
     static constexpr int kTmemCols = 2 * kBN;  // two 256-column fp32 accumulators
     static_assert(kSmemBytes <= 232448, "shared memory");
@@ -110,11 +117,14 @@ __global__ void __launch_bounds__(AsgCfg<NP, RES>::kThreads, 1)
     uint64_t *aempty = afull + 2;
     uint64_t *redfull = aempty + 2;
     uint64_t *redempty = redfull + 2;
-    uint64_t *drain = redempty + 2;
+    uint64_t *cnfull = redempty + 2;
+    uint64_t *drain = cnfull + 2;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
     volatile uint32_t *abort_flag = tmem_slot + 1;
+    // [group-1][slot][row]
     float *red_v = reinterpret_cast<float *>(smem + Cfg::kDataBytes + Cfg::kBarBytes);
-    int *red_k = reinterpret_cast<int *>(red_v + 2 * kBM);
+    int *red_k = reinterpret_cast<int *>(red_v + (Cfg::kEpiGroups - 1) * 2 * kBM);
+    float *cn_s = reinterpret_cast<float *>(red_k + (Cfg::kEpiGroups - 1) * 2 * kBM);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -129,8 +139,9 @@ __global__ void __launch_bounds__(AsgCfg<NP, RES>::kThreads, 1)
             ptx::mbar_init(&tempty[a], Cfg::kEpiWarps * 32);
             ptx::mbar_init(&afull[a], 1);
             ptx::mbar_init(&aempty[a], 1);
-            ptx::mbar_init(&redfull[a], kBM);
+            ptx::mbar_init(&redfull[a], (Cfg::kEpiGroups - 1) * kBM);
             ptx::mbar_init(&redempty[a], kBM);
+            ptx::mbar_init(&cnfull[a], 1);
         }
         ptx::mbar_init(drain, 1);
         *abort_flag = 0u;
@@ -227,6 +238,7 @@ __global__ void __launch_bounds__(AsgCfg<NP, RES>::kThreads, 1)
         if (lane == 0) {
             constexpr uint32_t idesc = ptx::idesc_bf16_f32(kBM, kBN);
             uint32_t stage = 0, phase = 0, titer = 0, mbi = 0;
+            uint32_t cn_issued = 0, cn_par = 0;
             bool ok = true;
             for (int64_t mb = blockIdx.x; mb < nmb && ok; mb += gridDim.x, ++mbi) {
                 uint32_t abase = 0, ab = 0;
@@ -250,6 +262,12 @@ __global__ void __launch_bounds__(AsgCfg<NP, RES>::kThreads, 1)
                         break;
                     }
                     ptx::tc_fence_after();
+                    // this tile's centroid norms into the slot of its accumulator (the
+                    // epilogue released the slot together with the accumulator)
+                    ptx::mbar_arrive_expect_tx(&cnfull[acc], kBN * 4);
+                    ptx::bulk_load(cn_s + acc * kBN, cn + nt * kBN, kBN * 4, &cnfull[acc]);
+                    cn_issued |= 1u << acc;
+                    cn_par = (cn_par & ~(1u << acc)) | (aphase << acc);
                     const uint32_t dt = tmem + acc * kBN;
                     for (int kc = 0; kc < nkc; ++kc) {
                         if (!ptx::mbar_wait(&full[stage], phase, abort_flag, wait_ns)) {
@@ -288,15 +306,20 @@ __global__ void __launch_bounds__(AsgCfg<NP, RES>::kThreads, 1)
                 if (RES && ok) ptx::mma_commit(&aempty[ab]);  // X buffer free after these MMAs
             }
             if (!ok) {
-                // Make sure no MMA issued by this thread is still writing tensor memory.
+                // Make sure no MMA issued by this thread is still writing tensor memory and
+                // every norm copy it started has landed.
                 ptx::mma_commit(drain);
                 ptx::mbar_wait(drain, 0u, nullptr, wait_ns);
+                for (int a = 0; a < 2; ++a)
+                    if (cn_issued & (1u << a))
+                        ptx::mbar_wait(&cnfull[a], (cn_par >> a) & 1u, nullptr, wait_ns);
             }
         }
     } else {
         // ------------------------------------------------------------ epilogue
-        // Warpgroup g (warps 2-5: g = 0, warps 6-9: g = 1) scans columns [128 g, 128 g + 128)
-        // of every tile; warp w may read TMEM lanes 32 (w % 4) .. 32 (w % 4) + 31, i.e. rows.
+        // Warpgroup g (warps 2+4g .. 5+4g) scans columns [64 g, 64 g + 64) of every tile;
+        // warp w may read TMEM lanes 32 (w % 4) .. 32 (w % 4) + 31, i.e. those rows.
+        constexpr int EC = Cfg::kEpiCols;
         const int g = (warp - 2) >> 2;
         const int q = warp & 3;
         const int r = q * 32 + lane;
@@ -308,54 +331,53 @@ __global__ void __launch_bounds__(AsgCfg<NP, RES>::kThreads, 1)
             for (int nt = 0; nt < ntiles; ++nt, ++titer) {
                 const uint32_t acc = titer & 1u;
                 const uint32_t aphase = (titer >> 1) & 1u;
-                if (!warp_wait(&tfull[acc], aphase, abort_flag, wait_ns)) {
+                if (!warp_wait(&tfull[acc], aphase, abort_flag, wait_ns) ||
+                    !warp_wait(&cnfull[acc], aphase, abort_flag, wait_ns)) {
                     if (lane == 0) raise_timeout(abort_flag, err);
                     ok = false;
                     break;
                 }
                 ptx::tc_fence_after();
-                const uint32_t tb = tmem + (static_cast<uint32_t>(q * 32) << 16) + acc * kBN +
-                                    g * (kBN / 2);
-                const int colbase = nt * kBN + g * (kBN / 2);
-                const float4 *cn4 = reinterpret_cast<const float4 *>(cn + colbase);
-#pragma unroll 1
-                for (int h = 0; h < 2; ++h) {
-                    __syncwarp();
-                    float v[64];
-                    ptx::tmem_ld64_sync(tb + h * 64, v);
+                const uint32_t tb =
+                    tmem + (static_cast<uint32_t>(q * 32) << 16) + acc * kBN + g * EC;
+                const int colbase = nt * kBN + g * EC;
+                const float4 *cn4 =
+                    reinterpret_cast<const float4 *>(cn_s + acc * kBN + g * EC);
+                __syncwarp();
+                float v[EC];
+                ptx::tmem_ld64_sync(tb, v);
 #pragma unroll
-                    for (int j4 = 0; j4 < 16; ++j4) {
-                        const float4 c = __ldg(cn4 + h * 16 + j4);
-                        v[4 * j4 + 0] += c.x;
-                        v[4 * j4 + 1] += c.y;
-                        v[4 * j4 + 2] += c.z;
-                        v[4 * j4 + 3] += c.w;
-                    }
-                    const float m = min64(v);
-                    if (m < best) {
-                        int idx = 0;
-#pragma unroll
-                        for (int j = 63; j >= 0; --j)
-                            if (v[j] == m) idx = j;
-                        best = m;
-                        bestk = colbase + h * 64 + idx;
-                    }
+                for (int j4 = 0; j4 < EC / 4; ++j4) {
+                    const float4 c = cn4[j4];
+                    v[4 * j4 + 0] += c.x;
+                    v[4 * j4 + 1] += c.y;
+                    v[4 * j4 + 2] += c.z;
+                    v[4 * j4 + 3] += c.w;
                 }
                 ptx::tc_fence_before();
-                ptx::mbar_arrive(&tempty[acc]);
+                ptx::mbar_arrive(&tempty[acc]);  // accumulator and norm slot consumed
+                const float m = min64(v);
+                if (m < best) {
+                    int idx = 0;
+#pragma unroll
+                    for (int j = EC - 1; j >= 0; --j)
+                        if (v[j] == m) idx = j;
+                    best = m;
+                    bestk = colbase + idx;
+                }
             }
             if (!ok) break;
-            // combine the two column halves of each row: (min, lowest index)
+            // combine the column groups of each row: (min, lowest index)
             const uint32_t slot = mbi & 1u;
             const uint32_t spar = (mbi >> 1) & 1u;
-            if (g == 1) {
+            if (g > 0) {
                 if (!warp_wait(&redempty[slot], spar ^ 1u, abort_flag, wait_ns)) {
                     if (lane == 0) raise_timeout(abort_flag, err);
                     ok = false;
                     break;
                 }
-                red_v[slot * kBM + r] = best;
-                red_k[slot * kBM + r] = bestk;
+                red_v[((g - 1) * 2 + slot) * kBM + r] = best;
+                red_k[((g - 1) * 2 + slot) * kBM + r] = bestk;
                 ptx::mbar_arrive(&redfull[slot]);
             } else {
                 if (!warp_wait(&redfull[slot], spar, abort_flag, wait_ns)) {
@@ -363,13 +385,16 @@ __global__ void __launch_bounds__(AsgCfg<NP, RES>::kThreads, 1)
                     ok = false;
                     break;
                 }
-                const float b1 = red_v[slot * kBM + r];
-                const int k1 = red_k[slot * kBM + r];
-                ptx::mbar_arrive(&redempty[slot]);
-                if (b1 < best || (b1 == best && k1 < bestk)) {
-                    best = b1;
-                    bestk = k1;
+#pragma unroll
+                for (int gg = 0; gg < Cfg::kEpiGroups - 1; ++gg) {
+                    const float b1 = red_v[(gg * 2 + slot) * kBM + r];
+                    const int k1 = red_k[(gg * 2 + slot) * kBM + r];
+                    if (b1 < best || (b1 == best && k1 < bestk)) {
+                        best = b1;
+                        bestk = k1;
+                    }
                 }
+                ptx::mbar_arrive(&redempty[slot]);
                 const int64_t row = mb * kBM + r;
                 if (row < N) {
                     labels[row] = bestk;
