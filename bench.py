@@ -8,7 +8,7 @@ points x iterations per second for the whole job.
 Default workload: N = 1,000,000 points, d = 768, K = 4096, fp32, cosine, 20 iterations
 (the IVF coarse-quantizer build shape of the LEANN FlashLib guide, section "性能对比").
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--config 1..5] [--impl reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
 
 Under torchrun every rank runs its own independent copy of the workload (its own seed), so
 per-GPU work is fixed (weak scaling); the whole-job value divides all ranks' points x
@@ -40,7 +40,8 @@ def parse():
     p.add_argument("--gpus", type=int, default=1)
     p.add_argument("--steps", type=int, default=5)
     p.add_argument("--warmup", type=int, default=3)
-    p.add_argument("--config", type=int, default=2)
+    p.add_argument("--workload", default="ivf_1000000x768_k4096_f32_cosine",
+                   help="one of synth.CONFIGS")
     p.add_argument("--niter", type=int, default=None)
     p.add_argument("--n", type=int, default=None,
                    help="override N (smaller cases for profiling captures)")
@@ -300,8 +301,8 @@ def fk_arm(args, spec, rank, world, dist):
     out = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
            "higher_is_better": True, "scaling": "weak",
-           "vs_baseline": value / PAGES_BUILD_RATE if args.config == 2 and niter == 20
-           else None,
+           "vs_baseline": value / PAGES_BUILD_RATE
+           if spec.name == "ivf_1000000x768_k4096_f32_cosine" and niter == 20 else None,
            "vs_baseline_note": "pages' 1M x 768 nlist 4096 build: 10.6 s for 20 iterations "
                                "on an H200 (another machine; context)",
            "dtype": spec.dtype, "data": "synthetic",
@@ -380,10 +381,9 @@ def main():
     from dataclasses import replace
 
     from synth import CONFIGS
-    spec = CONFIGS[args.config]
+    spec = CONFIGS[args.workload]
     if args.n:
-        spec = replace(spec, n=args.n, name=spec.name.replace(
-            str(CONFIGS[args.config].n), str(args.n)))
+        spec = replace(spec, n=args.n, name=spec.name.replace(str(spec.n), str(args.n)))
     if args.impl == "reference":
         reference_arm(args, spec, rank, world)
         return

@@ -42,19 +42,21 @@ class MixtureSpec:
     seed: int = 0
 
 
-# The five workloads: shapes, distributions and iteration counts.
-CONFIGS = {
-    1: MixtureSpec("tiny_65536x128_k256_f32", 65_536, 128, 256, "f32", "uniform", 0.1,
-                   "equal", niter=5),
-    2: MixtureSpec("ivf_1000000x768_k4096_f32_cosine", 1_000_000, 768, 4096, "f32",
-                   "normal", 0.3, "equal", metric="cosine", niter=20),
-    3: MixtureSpec("mid_10000000x128_k1024_f32", 10_000_000, 128, 1024, "f32",
-                   "uniform", 0.2, "equal", niter=10),
-    4: MixtureSpec("zipf_16000000x128_k65536_f32", 16_000_000, 128, 65_536, "f32",
-                   "normal", 0.15, "zipf", zipf_s=1.2, niter=5),
-    5: MixtureSpec("large_100000000x128_k32768_bf16", 100_000_000, 128, 32_768, "bf16",
-                   "normal", 0.25, "equal", niter=3),
-}
+# The workloads: shapes, distributions and iteration counts, keyed by name.
+_SPECS = [
+    MixtureSpec("tiny_65536x128_k256_f32", 65_536, 128, 256, "f32", "uniform", 0.1,
+                "equal", niter=5),
+    MixtureSpec("ivf_1000000x768_k4096_f32_cosine", 1_000_000, 768, 4096, "f32",
+                "normal", 0.3, "equal", metric="cosine", niter=20),
+    MixtureSpec("mid_10000000x128_k1024_f32", 10_000_000, 128, 1024, "f32",
+                "uniform", 0.2, "equal", niter=10),
+    MixtureSpec("zipf_16000000x128_k65536_f32", 16_000_000, 128, 65_536, "f32",
+                "normal", 0.15, "zipf", zipf_s=1.2, niter=5),
+    MixtureSpec("large_100000000x128_k32768_bf16", 100_000_000, 128, 32_768, "bf16",
+                "normal", 0.25, "equal", niter=3),
+]
+CONFIGS = {s.name: s for s in _SPECS}
+TINY, IVF, MID, ZIPF, LARGE = (s.name for s in _SPECS)
 
 
 def _gen(device, seed: int, stream: int) -> torch.Generator:
@@ -116,7 +118,7 @@ def init_indices(n: int, k: int, seed: int = 0, device="cpu") -> torch.Tensor:
 def make_config(cfg, device="cpu", n: int | None = None, **overrides):
     """Materialise a workload: returns (spec, X, C0 fp32, comp, centers).
 
-    `cfg` is a key of CONFIGS or a MixtureSpec; `n` (and any MixtureSpec field given in
+    `cfg` is a workload name (a key of CONFIGS) or a MixtureSpec; `n` (and any MixtureSpec field given in
     `overrides`) shrinks or alters the spec for small test cases."""
     spec = CONFIGS[cfg] if not isinstance(cfg, MixtureSpec) else cfg
     if n is not None:

@@ -15,12 +15,12 @@ import pytest
 import torch
 
 import oracle
-from synth import CONFIGS, gaussian_mixture, init_indices
+from synth import CONFIGS, IVF, LARGE, MID, ZIPF, gaussian_mixture, init_indices
 from tests.gpu_helpers import CENTROID_TOL, OBJECTIVE_TOL, centroid_rel_err, fk
 
 pytestmark = [pytest.mark.gpu, pytest.mark.slow]
 
-SAMPLE_ROWS = {2: 1024, 3: 4096, 4: 1024, 5: 768}
+SAMPLE_ROWS = {IVF: 1024, MID: 4096, ZIPF: 1024, LARGE: 768}
 
 
 def _data(cfg):
@@ -36,7 +36,7 @@ def _rows64(X, idx):
     return X[torch.as_tensor(idx, device=X.device)].double().cpu().numpy()
 
 
-@pytest.mark.parametrize("cfg", [2, 3, 4, 5])
+@pytest.mark.parametrize("cfg", [IVF, MID, ZIPF, LARGE])
 def test_fullsize_assign_sampled_rows(cfg):
     spec, X, _, C0 = _data(cfg)
     m = fk()
@@ -53,7 +53,7 @@ def test_fullsize_assign_sampled_rows(cfg):
     lab = labels.cpu().numpy()
     assert lab.min() >= 0 and lab.max() < spec.k
     del ws
-    rng = np.random.default_rng(cfg)
+    rng = np.random.default_rng(len(cfg))
     idx = np.sort(rng.choice(spec.n, SAMPLE_ROWS[cfg], replace=False))
     Xs = _rows64(X, idx)
     C = C0.double().cpu().numpy()
@@ -66,11 +66,11 @@ def test_fullsize_assign_sampled_rows(cfg):
     ref, dmin, d2nd = oracle.assign(Xs, C)
     ties = oracle.tie_mask(Xs, C, dmin, d2nd)
     bad = int(((lab[idx] != ref) & ~ties).sum())
-    print(f"config {cfg}: {len(idx)} sampled rows, {int(ties.sum())} tie points, {bad} bad")
+    print(f"{cfg}: {len(idx)} sampled rows, {int(ties.sum())} tie points, {bad} bad")
     assert bad == 0
 
 
-@pytest.mark.parametrize("cfg", [3, 4, 5])
+@pytest.mark.parametrize("cfg", [MID, ZIPF, LARGE])
 def test_fullsize_update_given_labels(cfg):
     spec, X, comp, C0 = _data(cfg)
     m = fk()
@@ -91,7 +91,7 @@ def test_fullsize_update_given_labels(cfg):
     assert (offsets.cpu().numpy() == off_ref).all()
 
     # centroids of sampled clusters (the largest always among them)
-    rng = np.random.default_rng(100 + cfg)
+    rng = np.random.default_rng(100 + len(cfg))
     nonempty = np.flatnonzero(cnt_ref)
     pick = np.unique(np.concatenate([[int(np.argmax(cnt_ref))],
                                      rng.choice(nonempty, min(64, len(nonempty)),
@@ -120,7 +120,7 @@ def test_fullsize_update_given_labels(cfg):
     assert abs(obj.item() - J) <= OBJECTIVE_TOL * J
 
 
-@pytest.mark.parametrize("cfg", [3, 4])
+@pytest.mark.parametrize("cfg", [MID, ZIPF])
 def test_fullsize_lloyd_invariants(cfg):
     spec, X, _, C0 = _data(cfg)
     m = fk()

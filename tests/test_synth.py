@@ -1,7 +1,7 @@
 """The seeded generator: determinism, shapes and the distributions the recipe states."""
 import torch
 
-from synth import CONFIGS, gaussian_mixture, init_indices, make_config
+from synth import CONFIGS, IVF, LARGE, TINY, gaussian_mixture, init_indices, make_config
 
 
 def test_deterministic_and_seed_sensitive():
@@ -42,6 +42,6 @@ def test_init_indices_distinct():
 
 
 def test_make_config_shapes():
-    spec, X, C0, comp, cen = make_config(1, n=4096, k=32)
+    spec, X, C0, comp, cen = make_config(TINY, n=4096, k=32)
     assert X.shape == (4096, 128) and C0.shape == (32, 128) and C0.dtype == torch.float32
-    assert CONFIGS[5].dtype == "bf16" and CONFIGS[2].metric == "cosine"
+    assert CONFIGS[LARGE].dtype == "bf16" and CONFIGS[IVF].metric == "cosine"
