@@ -57,8 +57,10 @@ struct AsgCfg {
     static constexpr int kEpiCols = kBN / kEpiGroups;  // 64 columns per group per tile
     // per-row (min, argmin) of groups 1..3, two slots
     static constexpr int kRedBytes = (kEpiGroups - 1) * 2 * kBM * 8;
-    static constexpr int kCnBytes = 2 * kBN * 4;       // ||c||^2 of the tile per accumulator
-    static constexpr int kSmemBytes = kDataBytes + kBarBytes + kRedBytes + kCnBytes + 1024;
+    static constexpr int kAugA = kBM * kAug * 2;       // 4 KB: constant (1, 1, 1, 0, ...) rows
+    static constexpr int kAugB = kBN * kAug * 2;       // 8 KB: tile's ||c||^2 pieces
+    static constexpr int kAugRegion = kAugA + 2 * kAugB;
+    static constexpr int kSmemBytes = kDataBytes + kAugRegion + kBarBytes + kRedBytes + 1024;
     static constexpr int kEpiWarps = 4 * kEpiGroups;
     static constexpr int kThreads = 64 + kEpiWarps * 32;
     static constexpr int kTmemCols = 2 * kBN;  // two 256-column fp32 accumulators
@@ -77,6 +79,19 @@ __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity,
     uint32_t ok = 0;
     if ((threadIdx.x & 31) == 0) ok = ptx::mbar_wait(bar, parity, abort_flag, wait_ns);
     return __shfl_sync(0xffffffffu, ok, 0) != 0;
+}
+
+// The constant A block of the norm-folding K step: 128 rows of (1, 1, 1, 0, ..., 0) bf16
+// (16 columns, 32 bytes per row) in the 32-byte-swizzled K-major layout (the two 16-byte
+// halves of row r are swapped when bit 2 of r is set).  One thread per row; the caller
+// fences the generic-proxy writes before the tensor core reads them.
+__device__ __forceinline__ void init_aug_a(uint8_t *aaug, int r) {
+    const uint4 ones = make_uint4(0x3f803f80u, 0x00003f80u, 0u, 0u);  // 1, 1, 1, 0, ...
+    const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
+    uint4 *row = reinterpret_cast<uint4 *>(aaug + r * 32);
+    const int sw = (r >> 2) & 1;
+    row[0 ^ sw] = ones;
+    row[1 ^ sw] = zero;
 }
 
 // Minimum of 64 values with three-input mins: 21 + 7 + 3 + 1 instructions.
@@ -99,7 +114,8 @@ __global__ void __launch_bounds__(AsgCfg<NP, RES>::kThreads, 1)
     assign_kernel(const __grid_constant__ CUtensorMap tmA0,
                   const __grid_constant__ CUtensorMap tmA1,
                   const __grid_constant__ CUtensorMap tmB0,
-                  const __grid_constant__ CUtensorMap tmB1, const float *__restrict__ cn,
+                  const __grid_constant__ CUtensorMap tmB1,
+                  const __grid_constant__ CUtensorMap tmC,
                   int64_t N, int nkc, int ntiles, int64_t nmb, int32_t *__restrict__ labels,
                   float *__restrict__ best_out, const float *__restrict__ xnorm,
                   float *__restrict__ mind, uint32_t *__restrict__ err, uint64_t wait_ns) {
@@ -109,7 +125,9 @@ __global__ void __launch_bounds__(AsgCfg<NP, RES>::kThreads, 1)
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     uint8_t *ring = smem + Cfg::kARegion;
-    uint64_t *full = reinterpret_cast<uint64_t *>(smem + Cfg::kDataBytes);
+    uint8_t *aaug = smem + Cfg::kDataBytes;  // constant A block of the norm step
+    uint8_t *baug = aaug + Cfg::kAugA;       // [2][256 rows][32 B], one slot per accumulator
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + Cfg::kDataBytes + Cfg::kAugRegion);
     uint64_t *empty = full + S;
     uint64_t *tfull = empty + S;
     uint64_t *tempty = tfull + 2;
@@ -117,14 +135,14 @@ __global__ void __launch_bounds__(AsgCfg<NP, RES>::kThreads, 1)
     uint64_t *aempty = afull + 2;
     uint64_t *redfull = aempty + 2;
     uint64_t *redempty = redfull + 2;
-    uint64_t *cnfull = redempty + 2;
-    uint64_t *drain = cnfull + 2;
+    uint64_t *augfull = redempty + 2;
+    uint64_t *drain = augfull + 2;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
     volatile uint32_t *abort_flag = tmem_slot + 1;
     // [group-1][slot][row]
-    float *red_v = reinterpret_cast<float *>(smem + Cfg::kDataBytes + Cfg::kBarBytes);
+    float *red_v = reinterpret_cast<float *>(smem + Cfg::kDataBytes + Cfg::kAugRegion +
+                                             Cfg::kBarBytes);
     int *red_k = reinterpret_cast<int *>(red_v + (Cfg::kEpiGroups - 1) * 2 * kBM);
-    float *cn_s = reinterpret_cast<float *>(red_k + (Cfg::kEpiGroups - 1) * 2 * kBM);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -141,7 +159,7 @@ __global__ void __launch_bounds__(AsgCfg<NP, RES>::kThreads, 1)
             ptx::mbar_init(&aempty[a], 1);
             ptx::mbar_init(&redfull[a], (Cfg::kEpiGroups - 1) * kBM);
             ptx::mbar_init(&redempty[a], kBM);
-            ptx::mbar_init(&cnfull[a], 1);
+            ptx::mbar_init(&augfull[a], 1);
         }
         ptx::mbar_init(drain, 1);
         *abort_flag = 0u;
@@ -150,6 +168,7 @@ __global__ void __launch_bounds__(AsgCfg<NP, RES>::kThreads, 1)
     if (warp == 0 && lane == 0) {
         ptx::prefetch_tmap(&tmA0);
         ptx::prefetch_tmap(&tmB0);
+        ptx::prefetch_tmap(&tmC);
         if (NP == 2) {
             ptx::prefetch_tmap(&tmA1);
             ptx::prefetch_tmap(&tmB1);
@@ -159,6 +178,10 @@ __global__ void __launch_bounds__(AsgCfg<NP, RES>::kThreads, 1)
         ptx::tmem_alloc(tmem_slot, Cfg::kTmemCols);
         ptx::tmem_relinquish();
     }
+    if (warp >= 2 && warp < 6) {
+        init_aug_a(aaug, (warp & 3) * 32 + lane);
+        ptx::fence_proxy_async_smem();  // visible to the tensor core (async proxy)
+    }
     ptx::tc_fence_before();
     __syncthreads();
     ptx::tc_fence_after();
@@ -167,8 +190,9 @@ __global__ void __launch_bounds__(AsgCfg<NP, RES>::kThreads, 1)
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
-            uint32_t stage = 0, phase = 0, mbi = 0;
+            uint32_t stage = 0, phase = 0, mbi = 0, titer = 0;
             uint32_t issued_mask = 0, issued_par = 0;    // ring stages: loaded, last parity
+            uint32_t g_mask = 0, g_par = 0;              // norm slots
             uint32_t a_mask = 0, a_par = 0;              // resident X buffers
             bool ok = true;
             for (int64_t mb = blockIdx.x; mb < nmb && ok; mb += gridDim.x, ++mbi) {
@@ -193,7 +217,23 @@ __global__ void __launch_bounds__(AsgCfg<NP, RES>::kThreads, 1)
                     a_mask |= 1u << ab;
                     a_par = (a_par & ~(1u << ab)) | (apar << ab);
                 }
-                for (int nt = 0; nt < ntiles && ok; ++nt) {
+                for (int nt = 0; nt < ntiles && ok; ++nt, ++titer) {
+                    {
+                        // the norm slot of this accumulator is free once the MMAs of the tile
+                        // two back (same slot) are complete, i.e. its accumulator is full
+                        const uint32_t acc = titer & 1u;
+                        const uint32_t aphase = (titer >> 1) & 1u;
+                        if (!ptx::mbar_wait(&tfull[acc], aphase ^ 1u, abort_flag, wait_ns)) {
+                            raise_timeout(abort_flag, err);
+                            ok = false;
+                            break;
+                        }
+                        ptx::mbar_arrive_expect_tx(&augfull[acc], Cfg::kAugB);
+                        ptx::tma_load_2d(baug + acc * Cfg::kAugB, &tmC, &augfull[acc], 0,
+                                         nt * kBN);
+                        g_mask |= 1u << acc;
+                        g_par = (g_par & ~(1u << acc)) | (aphase << acc);
+                    }
                     for (int kc = 0; kc < nkc; ++kc) {
                         if (!ptx::mbar_wait(&empty[stage], phase ^ 1u, abort_flag, wait_ns)) {
                             raise_timeout(abort_flag, err);
@@ -228,9 +268,12 @@ __global__ void __launch_bounds__(AsgCfg<NP, RES>::kThreads, 1)
                 for (int s = 0; s < S; ++s)
                     if (issued_mask & (1u << s))
                         ptx::mbar_wait(&full[s], (issued_par >> s) & 1u, nullptr, wait_ns);
-                for (int s = 0; s < 2; ++s)
+                for (int s = 0; s < 2; ++s) {
                     if (a_mask & (1u << s))
                         ptx::mbar_wait(&afull[s], (a_par >> s) & 1u, nullptr, wait_ns);
+                    if (g_mask & (1u << s))
+                        ptx::mbar_wait(&augfull[s], (g_par >> s) & 1u, nullptr, wait_ns);
+                }
             }
         }
     } else if (warp == 1) {
@@ -238,7 +281,8 @@ __global__ void __launch_bounds__(AsgCfg<NP, RES>::kThreads, 1)
         if (lane == 0) {
             constexpr uint32_t idesc = ptx::idesc_bf16_f32(kBM, kBN);
             uint32_t stage = 0, phase = 0, titer = 0, mbi = 0;
-            uint32_t cn_issued = 0, cn_par = 0;
+            const uint32_t aaug_s = ptx::smem_u32(aaug);
+            const uint32_t baug_s = ptx::smem_u32(baug);
             bool ok = true;
             for (int64_t mb = blockIdx.x; mb < nmb && ok; mb += gridDim.x, ++mbi) {
                 uint32_t abase = 0, ab = 0;
@@ -261,14 +305,16 @@ __global__ void __launch_bounds__(AsgCfg<NP, RES>::kThreads, 1)
                         ok = false;
                         break;
                     }
+                    if (!ptx::mbar_wait(&augfull[acc], aphase, abort_flag, wait_ns)) {
+                        raise_timeout(abort_flag, err);
+                        ok = false;
+                        break;
+                    }
                     ptx::tc_fence_after();
-                    // this tile's centroid norms into the slot of its accumulator (the
-                    // epilogue released the slot together with the accumulator)
-                    ptx::mbar_arrive_expect_tx(&cnfull[acc], kBN * 4);
-                    ptx::bulk_load(cn_s + acc * kBN, cn + nt * kBN, kBN * 4, &cnfull[acc]);
-                    cn_issued |= 1u << acc;
-                    cn_par = (cn_par & ~(1u << acc)) | (aphase << acc);
                     const uint32_t dt = tmem + acc * kBN;
+                    // D = ||c||^2 (hi + mid + lo against the constant ones): the norm step
+                    ptx::mma_bf16_ss(dt, ptx::sdesc_k_sw32(aaug_s),
+                                     ptx::sdesc_k_sw32(baug_s + acc * Cfg::kAugB), idesc, 0u);
                     for (int kc = 0; kc < nkc; ++kc) {
                         if (!ptx::mbar_wait(&full[stage], phase, abort_flag, wait_ns)) {
                             raise_timeout(abort_flag, err);
@@ -281,17 +327,17 @@ __global__ void __launch_bounds__(AsgCfg<NP, RES>::kThreads, 1)
                         const uint32_t a1 = a0 + Cfg::kABytes;
                         const uint32_t b0 = RES ? st : st + NP * Cfg::kABytes;
                         const uint32_t b1 = b0 + Cfg::kBBytes;
+                        // descriptors built once; +2 advances the start address by 32 bytes
+                        // (16 bf16 along K) inside the 128-byte swizzle row
+                        const uint64_t da0 = ptx::sdesc_k_sw128(a0), da1 = ptx::sdesc_k_sw128(a1);
+                        const uint64_t db0 = ptx::sdesc_k_sw128(b0), db1 = ptx::sdesc_k_sw128(b1);
 #pragma unroll
                         for (int ks = 0; ks < kBK / 16; ++ks) {
-                            const uint32_t off = ks * 32;  // 16 bf16 = 32 bytes along K
-                            ptx::mma_bf16_ss(dt, ptx::sdesc_k_sw128(a0 + off),
-                                             ptx::sdesc_k_sw128(b0 + off), idesc,
-                                             (kc | ks) != 0 ? 1u : 0u);
+                            const uint64_t o = 2u * ks;
+                            ptx::mma_bf16_ss(dt, da0 + o, db0 + o, idesc, 1u);
                             if (NP == 2) {
-                                ptx::mma_bf16_ss(dt, ptx::sdesc_k_sw128(a1 + off),
-                                                 ptx::sdesc_k_sw128(b0 + off), idesc, 1u);
-                                ptx::mma_bf16_ss(dt, ptx::sdesc_k_sw128(a0 + off),
-                                                 ptx::sdesc_k_sw128(b1 + off), idesc, 1u);
+                                ptx::mma_bf16_ss(dt, da1 + o, db0 + o, idesc, 1u);
+                                ptx::mma_bf16_ss(dt, da0 + o, db1 + o, idesc, 1u);
                             }
                         }
                         ptx::mma_commit(&empty[stage]);
@@ -301,7 +347,7 @@ __global__ void __launch_bounds__(AsgCfg<NP, RES>::kThreads, 1)
                         }
                     }
                     if (!ok) break;
-                    ptx::mma_commit(&tfull[acc]);
+                    ptx::mma_commit(&tfull[acc]);  // also frees this tile's norm slot
                 }
                 if (RES && ok) ptx::mma_commit(&aempty[ab]);  // X buffer free after these MMAs
             }
@@ -310,9 +356,6 @@ __global__ void __launch_bounds__(AsgCfg<NP, RES>::kThreads, 1)
                 // every norm copy it started has landed.
                 ptx::mma_commit(drain);
                 ptx::mbar_wait(drain, 0u, nullptr, wait_ns);
-                for (int a = 0; a < 2; ++a)
-                    if (cn_issued & (1u << a))
-                        ptx::mbar_wait(&cnfull[a], (cn_par >> a) & 1u, nullptr, wait_ns);
             }
         }
     } else {
@@ -331,8 +374,7 @@ __global__ void __launch_bounds__(AsgCfg<NP, RES>::kThreads, 1)
             for (int nt = 0; nt < ntiles; ++nt, ++titer) {
                 const uint32_t acc = titer & 1u;
                 const uint32_t aphase = (titer >> 1) & 1u;
-                if (!warp_wait(&tfull[acc], aphase, abort_flag, wait_ns) ||
-                    !warp_wait(&cnfull[acc], aphase, abort_flag, wait_ns)) {
+                if (!warp_wait(&tfull[acc], aphase, abort_flag, wait_ns)) {
                     if (lane == 0) raise_timeout(abort_flag, err);
                     ok = false;
                     break;
@@ -341,21 +383,11 @@ __global__ void __launch_bounds__(AsgCfg<NP, RES>::kThreads, 1)
                 const uint32_t tb =
                     tmem + (static_cast<uint32_t>(q * 32) << 16) + acc * kBN + g * EC;
                 const int colbase = nt * kBN + g * EC;
-                const float4 *cn4 =
-                    reinterpret_cast<const float4 *>(cn_s + acc * kBN + g * EC);
                 __syncwarp();
-                float v[EC];
+                float v[EC];  // ||c||^2 - 2 x.c, the norm already folded in by the MMA
                 ptx::tmem_ld64_sync(tb, v);
-#pragma unroll
-                for (int j4 = 0; j4 < EC / 4; ++j4) {
-                    const float4 c = cn4[j4];
-                    v[4 * j4 + 0] += c.x;
-                    v[4 * j4 + 1] += c.y;
-                    v[4 * j4 + 2] += c.z;
-                    v[4 * j4 + 3] += c.w;
-                }
                 ptx::tc_fence_before();
-                ptx::mbar_arrive(&tempty[acc]);  // accumulator and norm slot consumed
+                ptx::mbar_arrive(&tempty[acc]);  // accumulator consumed
                 const float m = min64(v);
                 if (m < best) {
                     int idx = 0;
@@ -414,6 +446,397 @@ __global__ void __launch_bounds__(AsgCfg<NP, RES>::kThreads, 1)
     }
 }
 
+// ============================================================================ CTA pairs
+// The same computation on a cluster of two CTAs (two SMs) with cta_group::2 MMAs: the
+// pair owns a 256-row block of X, each CTA staging its own 128 rows and its own half (128
+// centroids) of every 256-centroid tile; the even CTA issues M = 256, N = 256 MMAs that
+// read A and B from both CTAs' shared memory and leave each CTA's 128 x 256 accumulator
+// in its own tensor memory.  Shared-memory operand traffic per flop is half that of the
+// single-CTA kernel.  Stage and accumulator hand-offs are mbarriers: loads of both CTAs
+// complete on the even CTA's barriers, MMA completion is signalled to both CTAs
+// (tcgen05.commit multicast), and both CTAs' epilogues release the accumulator to the
+// even CTA by remote arrive.  No load is multicast.
+template <int NP, bool RES>
+struct PairCfg {
+    static constexpr int kABytes = kBM * kBK * 2;         // 16 KB: 128 X rows, one chunk
+    static constexpr int kBBytes = (kBN / 2) * kBK * 2;   // 16 KB: 128 centroids, one chunk
+    static constexpr int kAChunks = RES ? 2 : 0;
+    static constexpr int kABufs = RES ? (NP == 1 ? 2 : 1) : 1;
+    static constexpr int kABufBytes = kAChunks * NP * kABytes;
+    static constexpr int kARegion = RES ? kABufs * kABufBytes : 0;
+    // resident X: one stage holds all (<= 2) k-chunks of a tile's centroids, so a tile costs
+    // one full-wait and one empty-commit; streamed X: one k-chunk of X and centroids
+    static constexpr int kStageChunks = RES ? kAChunks : 1;
+    static constexpr int kStageBytes =
+        RES ? kStageChunks * NP * kBBytes : NP * (kABytes + kBBytes);
+    static constexpr int kStages = RES ? (NP == 1 ? 4 : 2) : (NP == 2 ? 3 : 6);
+    static constexpr int kDataBytes = kARegion + kStages * kStageBytes;  // 192 KB
+    static constexpr int kBarBytes = 512;
+    static constexpr int kEpiGroups = 4;
+    static constexpr int kEpiCols = kBN / kEpiGroups;
+    static constexpr int kRedBytes = (kEpiGroups - 1) * 2 * kBM * 8;
+    static constexpr int kAugA = kBM * kAug * 2;         // 4 KB: constant (1, 1, 1, 0, ...)
+    static constexpr int kAugB = (kBN / 2) * kAug * 2;   // 4 KB: this CTA's 128 norms
+    static constexpr int kAugRegion = kAugA + 2 * kAugB;
+    static constexpr int kSmemBytes = kDataBytes + kAugRegion + kBarBytes + kRedBytes + 1024;
+    static constexpr int kEpiWarps = 4 * kEpiGroups;
+    static constexpr int kThreads = 64 + kEpiWarps * 32;
+    static constexpr int kTmemCols = 2 * kBN;
+    static_assert(kStages <= 8, "stage masks");
+    static_assert(kSmemBytes <= 232448, "shared memory");
+};
+
+template <int NP, bool RES>
+__global__ void __launch_bounds__(PairCfg<NP, RES>::kThreads, 1)
+    assign_pair_kernel(const __grid_constant__ CUtensorMap tmA0,
+                       const __grid_constant__ CUtensorMap tmA1,
+                       const __grid_constant__ CUtensorMap tmB0,
+                       const __grid_constant__ CUtensorMap tmB1,
+                       const __grid_constant__ CUtensorMap tmC,
+                       int64_t N, int nkc, int ntiles, int64_t nmb,
+                       int32_t *__restrict__ labels, float *__restrict__ best_out,
+                       const float *__restrict__ xnorm, float *__restrict__ mind,
+                       uint32_t *__restrict__ err, uint64_t wait_ns) {
+    using Cfg = PairCfg<NP, RES>;
+    constexpr int S = Cfg::kStages;
+    constexpr int EC = Cfg::kEpiCols;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    uint8_t *ring = smem + Cfg::kARegion;
+    uint8_t *aaug = smem + Cfg::kDataBytes;  // constant A block of the norm step
+    uint8_t *baug = aaug + Cfg::kAugA;       // [2][128 rows][32 B]
+    uint64_t *full =
+        reinterpret_cast<uint64_t *>(smem + Cfg::kDataBytes + Cfg::kAugRegion);  // even CTA
+    uint64_t *empty = full + S;
+    uint64_t *tfull = empty + S;
+    uint64_t *tempty = tfull + 2;  // even CTA
+    uint64_t *afull = tempty + 2;  // even CTA
+    uint64_t *aempty = afull + 2;
+    uint64_t *redfull = aempty + 2;
+    uint64_t *redempty = redfull + 2;
+    uint64_t *augfull = redempty + 2;  // even CTA
+    uint64_t *drain = augfull + 2;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
+    volatile uint32_t *abort_flag = tmem_slot + 1;
+    float *red_v = reinterpret_cast<float *>(smem + Cfg::kDataBytes + Cfg::kAugRegion +
+                                             Cfg::kBarBytes);
+    int *red_k = reinterpret_cast<int *>(red_v + (Cfg::kEpiGroups - 1) * 2 * kBM);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const uint32_t rank = ptx::cluster_ctarank();
+    const int64_t pair = blockIdx.x >> 1;
+    const int64_t npairs = gridDim.x >> 1;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S; ++s) {
+            ptx::mbar_init(&full[s], 1);
+            ptx::mbar_init(&empty[s], 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            ptx::mbar_init(&tfull[a], 1);
+            ptx::mbar_init(&tempty[a], 2 * Cfg::kEpiWarps);
+            ptx::mbar_init(&afull[a], 1);
+            ptx::mbar_init(&aempty[a], 1);
+            ptx::mbar_init(&redfull[a], (Cfg::kEpiGroups - 1) * kBM);
+            ptx::mbar_init(&redempty[a], kBM);
+            ptx::mbar_init(&augfull[a], 1);
+        }
+        ptx::mbar_init(drain, 1);
+        *abort_flag = 0u;
+        ptx::fence_mbar_init();
+    }
+    if (warp == 0 && lane == 0) {
+        ptx::prefetch_tmap(&tmA0);
+        ptx::prefetch_tmap(&tmB0);
+        ptx::prefetch_tmap(&tmC);
+        if (NP == 2) {
+            ptx::prefetch_tmap(&tmA1);
+            ptx::prefetch_tmap(&tmB1);
+        }
+    }
+    if (warp == 1) {
+        ptx::tmem_alloc_pair(tmem_slot, Cfg::kTmemCols);
+        ptx::tmem_relinquish_pair();
+    }
+    if (warp >= 2 && warp < 6) {
+        init_aug_a(aaug, (warp & 3) * 32 + lane);
+        ptx::fence_proxy_async_smem();  // visible to the tensor core (async proxy)
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::cluster_sync();  // barriers of both CTAs initialised, tensor memory allocated
+    ptx::tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    // shared::cluster addresses of the even CTA's barriers
+    const uint32_t full_c = ptx::mapa_shared(ptx::smem_u32(full), 0);
+    const uint32_t afull_c = ptx::mapa_shared(ptx::smem_u32(afull), 0);
+    const uint32_t tempty_c = ptx::mapa_shared(ptx::smem_u32(tempty), 0);
+    const uint32_t augfull_c = ptx::mapa_shared(ptx::smem_u32(augfull), 0);
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ TMA producer (both)
+        if (lane == 0) {
+            uint32_t stage = 0, phase = 0, mbi = 0, titer = 0;
+            bool ok = true;
+            for (int64_t mb = pair; mb < nmb && ok; mb += npairs, ++mbi) {
+                const int row0 = static_cast<int>(mb * 2 * kBM + rank * kBM);
+                if (RES) {
+                    const uint32_t ab = mbi % Cfg::kABufs;
+                    const uint32_t apar = (mbi / Cfg::kABufs) & 1u;
+                    if (!ptx::mbar_wait(&aempty[ab], apar ^ 1u, abort_flag, wait_ns)) {
+                        raise_timeout(abort_flag, err);
+                        ok = false;
+                        break;
+                    }
+                    if (rank == 0)
+                        ptx::mbar_arrive_expect_tx(&afull[ab], 2 * nkc * NP * Cfg::kABytes);
+                    uint8_t *ar = smem + ab * Cfg::kABufBytes;
+                    for (int kc = 0; kc < nkc; ++kc) {
+                        ptx::tma_load_2d_pair(ar + (kc * NP) * Cfg::kABytes, &tmA0,
+                                              afull_c + ab * 8, kc * kBK, row0);
+                        if (NP == 2)
+                            ptx::tma_load_2d_pair(ar + (kc * NP + 1) * Cfg::kABytes, &tmA1,
+                                                  afull_c + ab * 8, kc * kBK, row0);
+                    }
+                }
+                for (int nt = 0; nt < ntiles && ok; ++nt, ++titer) {
+                    const int crow = nt * kBN + static_cast<int>(rank) * (kBN / 2);
+                    {
+                        // the norm slot is free once the tile two back (same slot) completed
+                        const uint32_t acc = titer & 1u;
+                        const uint32_t aphase = (titer >> 1) & 1u;
+                        if (!ptx::mbar_wait(&tfull[acc], aphase ^ 1u, abort_flag, wait_ns)) {
+                            raise_timeout(abort_flag, err);
+                            ok = false;
+                            break;
+                        }
+                        if (rank == 0) ptx::mbar_arrive_expect_tx(&augfull[acc], 2 * Cfg::kAugB);
+                        ptx::tma_load_2d_pair(baug + acc * Cfg::kAugB, &tmC, augfull_c + acc * 8,
+                                              0, crow);
+                    }
+                    for (int kc = 0; kc < nkc; kc += Cfg::kStageChunks) {
+                        if (!ptx::mbar_wait(&empty[stage], phase ^ 1u, abort_flag, wait_ns)) {
+                            raise_timeout(abort_flag, err);
+                            ok = false;
+                            break;
+                        }
+                        const int nch = nkc - kc < Cfg::kStageChunks ? nkc - kc
+                                                                     : Cfg::kStageChunks;
+                        if (rank == 0)
+                            ptx::mbar_arrive_expect_tx(&full[stage],
+                                                       2 * nch * NP * (RES ? Cfg::kBBytes
+                                                                           : Cfg::kABytes +
+                                                                                 Cfg::kBBytes));
+                        uint8_t *st = ring + stage * Cfg::kStageBytes;
+                        const uint32_t fb = full_c + stage * 8;
+                        for (int c = 0; c < nch; ++c) {
+                            uint8_t *sb = st + c * NP * Cfg::kBBytes;
+                            if (!RES) {
+                                ptx::tma_load_2d_pair(st, &tmA0, fb, (kc + c) * kBK, row0);
+                                if (NP == 2)
+                                    ptx::tma_load_2d_pair(st + Cfg::kABytes, &tmA1, fb,
+                                                          (kc + c) * kBK, row0);
+                                sb = st + NP * Cfg::kABytes;
+                            }
+                            ptx::tma_load_2d_pair(sb, &tmB0, fb, (kc + c) * kBK, crow);
+                            if (NP == 2)
+                                ptx::tma_load_2d_pair(sb + Cfg::kBBytes, &tmB1, fb,
+                                                      (kc + c) * kBK, crow);
+                        }
+                        if (++stage == S) {
+                            stage = 0;
+                            phase ^= 1u;
+                        }
+                    }
+                }
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            uint32_t titer = 0;
+            bool ok = true;
+            if (rank == 0) {
+                // -------------------------------------------------- MMA issuer (even CTA)
+                constexpr uint32_t idesc = ptx::idesc_bf16_f32(2 * kBM, kBN);
+                uint32_t stage = 0, phase = 0, mbi = 0;
+                const uint32_t aaug_s = ptx::smem_u32(aaug);
+                const uint32_t baug_s = ptx::smem_u32(baug);
+                for (int64_t mb = pair; mb < nmb && ok; mb += npairs, ++mbi) {
+                    uint32_t abase = 0, ab = 0;
+                    if (RES) {
+                        ab = mbi % Cfg::kABufs;
+                        const uint32_t apar = (mbi / Cfg::kABufs) & 1u;
+                        if (!ptx::mbar_wait(&afull[ab], apar, abort_flag, wait_ns)) {
+                            raise_timeout(abort_flag, err);
+                            ok = false;
+                            break;
+                        }
+                        ptx::tc_fence_after();
+                        abase = ptx::smem_u32(smem + ab * Cfg::kABufBytes);
+                    }
+                    for (int nt = 0; nt < ntiles && ok; ++nt, ++titer) {
+                        const uint32_t acc = titer & 1u;
+                        const uint32_t aphase = (titer >> 1) & 1u;
+                        if (!ptx::mbar_wait_cluster(&tempty[acc], aphase ^ 1u, abort_flag,
+                                                    wait_ns)) {
+                            raise_timeout(abort_flag, err);
+                            ok = false;
+                            break;
+                        }
+                        if (!ptx::mbar_wait(&augfull[acc], aphase, abort_flag, wait_ns)) {
+                            raise_timeout(abort_flag, err);
+                            ok = false;
+                            break;
+                        }
+                        ptx::tc_fence_after();
+                        const uint32_t dt = tmem + acc * kBN;
+                        // D = ||c||^2 (hi + mid + lo against the constant ones)
+                        ptx::mma_bf16_ss_pair(dt, ptx::sdesc_k_sw32(aaug_s),
+                                              ptx::sdesc_k_sw32(baug_s + acc * Cfg::kAugB),
+                                              idesc, 0u);
+                        for (int kc = 0; kc < nkc; kc += Cfg::kStageChunks) {
+                            if (!ptx::mbar_wait(&full[stage], phase, abort_flag, wait_ns)) {
+                                raise_timeout(abort_flag, err);
+                                ok = false;
+                                break;
+                            }
+                            ptx::tc_fence_after();
+                            const int nch = nkc - kc < Cfg::kStageChunks ? nkc - kc
+                                                                         : Cfg::kStageChunks;
+                            const uint32_t st = ptx::smem_u32(ring + stage * Cfg::kStageBytes);
+                            for (int c = 0; c < nch; ++c) {
+                                const uint32_t a0 =
+                                    RES ? abase + ((kc + c) * NP) * Cfg::kABytes : st;
+                                const uint32_t a1 = a0 + Cfg::kABytes;
+                                const uint32_t b0 =
+                                    RES ? st + c * NP * Cfg::kBBytes : st + NP * Cfg::kABytes;
+                                const uint32_t b1 = b0 + Cfg::kBBytes;
+                                const uint64_t da0 = ptx::sdesc_k_sw128(a0);
+                                const uint64_t da1 = ptx::sdesc_k_sw128(a1);
+                                const uint64_t db0 = ptx::sdesc_k_sw128(b0);
+                                const uint64_t db1 = ptx::sdesc_k_sw128(b1);
+#pragma unroll
+                                for (int ks = 0; ks < kBK / 16; ++ks) {
+                                    const uint64_t o = 2u * ks;  // +32 bytes along K
+                                    ptx::mma_bf16_ss_pair(dt, da0 + o, db0 + o, idesc, 1u);
+                                    if (NP == 2) {
+                                        ptx::mma_bf16_ss_pair(dt, da1 + o, db0 + o, idesc, 1u);
+                                        ptx::mma_bf16_ss_pair(dt, da0 + o, db1 + o, idesc, 1u);
+                                    }
+                                }
+                            }
+                            ptx::mma_commit_pair(&empty[stage], 0x3);
+                            if (++stage == S) {
+                                stage = 0;
+                                phase ^= 1u;
+                            }
+                        }
+                        if (!ok) break;
+                        ptx::mma_commit_pair(&tfull[acc], 0x3);  // also frees the norm slot
+                    }
+                    if (RES && ok) ptx::mma_commit_pair(&aempty[ab], 0x3);
+                }
+                if (!ok) {
+                    ptx::mma_commit_pair(drain, 0x1);
+                    ptx::mbar_wait(drain, 0u, nullptr, wait_ns);
+                }
+            }
+        }
+    } else {
+        // ------------------------------------------------------------ epilogue (both)
+        const int g = (warp - 2) >> 2;
+        const int q = warp & 3;
+        const int r = q * 32 + lane;
+        uint32_t titer = 0, mbi = 0;
+        bool ok = true;
+        for (int64_t mb = pair; mb < nmb && ok; mb += npairs, ++mbi) {
+            float best = __int_as_float(0x7f800000);
+            int bestk = 0;
+            for (int nt = 0; nt < ntiles; ++nt, ++titer) {
+                const uint32_t acc = titer & 1u;
+                const uint32_t aphase = (titer >> 1) & 1u;
+                if (!warp_wait(&tfull[acc], aphase, abort_flag, wait_ns)) {
+                    if (lane == 0) raise_timeout(abort_flag, err);
+                    ok = false;
+                    break;
+                }
+                ptx::tc_fence_after();
+                const uint32_t tb =
+                    tmem + (static_cast<uint32_t>(q * 32) << 16) + acc * kBN + g * EC;
+                const int colbase = nt * kBN + g * EC;
+                __syncwarp();
+                float v[EC];  // ||c||^2 - 2 x.c, the norm already folded in by the MMA
+                ptx::tmem_ld64_sync(tb, v);
+                ptx::tc_fence_before();
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive_cluster(tempty_c + acc * 8);  // consumed
+                const float m = min64(v);
+                if (m < best) {
+                    int idx = 0;
+#pragma unroll
+                    for (int j = EC - 1; j >= 0; --j)
+                        if (v[j] == m) idx = j;
+                    best = m;
+                    bestk = colbase + idx;
+                }
+            }
+            if (!ok) break;
+            const uint32_t slot = mbi & 1u;
+            const uint32_t spar = (mbi >> 1) & 1u;
+            if (g > 0) {
+                if (!warp_wait(&redempty[slot], spar ^ 1u, abort_flag, wait_ns)) {
+                    if (lane == 0) raise_timeout(abort_flag, err);
+                    ok = false;
+                    break;
+                }
+                red_v[((g - 1) * 2 + slot) * kBM + r] = best;
+                red_k[((g - 1) * 2 + slot) * kBM + r] = bestk;
+                ptx::mbar_arrive(&redfull[slot]);
+            } else {
+                if (!warp_wait(&redfull[slot], spar, abort_flag, wait_ns)) {
+                    if (lane == 0) raise_timeout(abort_flag, err);
+                    ok = false;
+                    break;
+                }
+#pragma unroll
+                for (int gg = 0; gg < Cfg::kEpiGroups - 1; ++gg) {
+                    const float b1 = red_v[(gg * 2 + slot) * kBM + r];
+                    const int k1 = red_k[(gg * 2 + slot) * kBM + r];
+                    if (b1 < best || (b1 == best && k1 < bestk)) {
+                        best = b1;
+                        bestk = k1;
+                    }
+                }
+                ptx::mbar_arrive(&redempty[slot]);
+                const int64_t row = mb * 2 * kBM + static_cast<int64_t>(rank) * kBM + r;
+                if (row < N) {
+                    labels[row] = bestk;
+                    if (best_out) best_out[row] = best;
+                    if (mind) mind[row] = xnorm[row] + best;
+                }
+            }
+        }
+    }
+
+    // ---------------------------------------------------------------- teardown
+    ptx::tc_fence_before();
+    __syncthreads();
+    __syncwarp();
+    ptx::cluster_sync();  // neither CTA leaves while the pair may still touch its memory
+    if (*abort_flag) {
+        // after a timeout, give copies already in flight a moment to land (bounded)
+        const uint64_t t0 = ptx::globaltimer_ns();
+        while (ptx::globaltimer_ns() - t0 < 200000ull) {
+        }
+    }
+    if (warp == 1) {
+        ptx::tc_fence_after();
+        ptx::tmem_dealloc_pair(tmem, Cfg::kTmemCols);
+    }
+}
+
 PFN_cuTensorMapEncodeTiled_v12000 tmap_encode_fn() {
     static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
     if (!fn) {
@@ -428,25 +851,28 @@ PFN_cuTensorMapEncodeTiled_v12000 tmap_encode_fn() {
 }
 
 // 2-D bf16 tensor map over a row-major [rows][cols] plane with the given row stride,
-// 64 x box_rows boxes, 128-byte swizzle; out-of-range rows/columns read as zero.
+// box_cols x box_rows boxes (64 columns = 128 bytes with 128-byte swizzle, or 16 columns =
+// 32 bytes with 32-byte swizzle); out-of-range rows/columns read as zero.
 bool make_tmap(CUtensorMap *m, const void *base, int64_t rows, int64_t cols,
-               int64_t row_stride_elems, int box_rows) {
+               int64_t row_stride_elems, int box_rows, int box_cols = kBK) {
     auto fn = tmap_encode_fn();
     if (!fn) return false;
     cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
     cuuint64_t strides[1] = {static_cast<cuuint64_t>(row_stride_elems * 2)};
-    cuuint32_t box[2] = {static_cast<cuuint32_t>(kBK), static_cast<cuuint32_t>(box_rows)};
+    cuuint32_t box[2] = {static_cast<cuuint32_t>(box_cols), static_cast<cuuint32_t>(box_rows)};
     cuuint32_t estr[2] = {1, 1};
     CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims,
                     strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                    CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    box_cols == kAug ? CU_TENSOR_MAP_SWIZZLE_32B : CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
 
 template <int NP, bool RES>
 cudaError_t launch_assign_cfg(const AssignArgs &a, const CUtensorMap (&tA)[2],
-                              const CUtensorMap (&tB)[2], cudaStream_t st) {
+                              const CUtensorMap (&tB)[2], const CUtensorMap &tC,
+                              cudaStream_t st) {
     using Cfg = AsgCfg<NP, RES>;
     static bool attr_set = false;
     if (!attr_set) {
@@ -460,11 +886,95 @@ cudaError_t launch_assign_cfg(const AssignArgs &a, const CUtensorMap (&tA)[2],
     const int64_t sms = device_sm_count();
     const int grid = static_cast<int>(nmb < sms ? nmb : sms);
     assign_kernel<NP, RES><<<grid, Cfg::kThreads, Cfg::kSmemBytes, st>>>(
-        tA[0], tA[1], tB[0], tB[1], a.cn, a.N, static_cast<int>(a.dp / kBK),
+        tA[0], tA[1], tB[0], tB[1], tC, a.N, static_cast<int>(a.dp / kBK),
         static_cast<int>(a.Kp / kBN), nmb, a.labels, a.best, a.xnorm, a.mind, a.err,
         a.wait_ns);
     note_launch();
     return cudaGetLastError();
+}
+
+template <int NP, bool RES>
+cudaError_t launch_assign_pair_cfg(const AssignArgs &a, const CUtensorMap (&tA)[2],
+                                   const CUtensorMap (&tB)[2], const CUtensorMap &tC,
+                                   int max_pairs, cudaStream_t st) {
+    using Cfg = PairCfg<NP, RES>;
+    const int64_t nmb = ceil_div(a.N, 2 * kBM);
+    const int pairs = static_cast<int>(nmb < max_pairs ? nmb : max_pairs);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * pairs);
+    cfg.blockDim = dim3(Cfg::kThreads);
+    cfg.dynamicSmemBytes = Cfg::kSmemBytes;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, assign_pair_kernel<NP, RES>, tA[0], tA[1], tB[0],
+                                       tB[1], tC, a.N, static_cast<int>(a.dp / kBK),
+                                       static_cast<int>(a.Kp / kBN), nmb, a.labels, a.best,
+                                       a.xnorm, a.mind, a.err, a.wait_ns);
+    note_launch();
+    return e;
+}
+
+// Largest number of CTA pairs of this configuration that can be resident at once (the
+// persistent grid must not exceed it, or part of it would wait for a second wave).
+template <int NP, bool RES>
+int max_resident_pairs() {
+    using Cfg = PairCfg<NP, RES>;
+    static int cached[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+    if (cached[dev]) return cached[dev];
+    if (cudaFuncSetAttribute(assign_pair_kernel<NP, RES>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             Cfg::kSmemBytes) != cudaSuccess)
+        return 0;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * 74);
+    cfg.blockDim = dim3(Cfg::kThreads);
+    cfg.dynamicSmemBytes = Cfg::kSmemBytes;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, assign_pair_kernel<NP, RES>, &cfg) != cudaSuccess)
+        n = 0;
+    cached[dev] = n;
+    return n;
+}
+
+template <int NP>
+cudaError_t launch_assign_pair(const AssignArgs &a, cudaStream_t st, bool res, bool *done) {
+    *done = false;
+    const int mp = res ? max_resident_pairs<NP, true>() : max_resident_pairs<NP, false>();
+    if (mp <= 0) return cudaSuccess;  // pairs cannot be scheduled: use the single-CTA form
+    CUtensorMap tA[2], tB[2];
+    const uint16_t *ap = static_cast<const uint16_t *>(a.a_planes);
+    const uint16_t *bp = static_cast<const uint16_t *>(a.b_planes);
+    for (int p = 0; p < NP; ++p) {
+        if (!make_tmap(&tA[p], ap + p * a.N * a.lda, a.N, a.dp, a.lda, kBM))
+            return cudaErrorInvalidValue;
+        if (!make_tmap(&tB[p], bp + p * static_cast<int64_t>(a.Kp) * a.dp, a.Kp, a.dp, a.dp,
+                       kBN / 2))
+            return cudaErrorInvalidValue;
+    }
+    if (NP == 1) {
+        tA[1] = tA[0];
+        tB[1] = tB[0];
+    }
+    CUtensorMap tC;
+    if (!make_tmap(&tC, a.caug, a.Kp, kAug, kAug, kBN / 2, kAug)) return cudaErrorInvalidValue;
+    *done = true;
+    return res ? launch_assign_pair_cfg<NP, true>(a, tA, tB, tC, mp, st)
+               : launch_assign_pair_cfg<NP, false>(a, tA, tB, tC, mp, st);
 }
 
 template <int NP>
@@ -489,8 +999,16 @@ cudaError_t launch_assign_np(const AssignArgs &a, cudaStream_t st) {
     const int nkc = a.dp / kBK;
     const int ntiles = a.Kp / kBN;
     const bool res = nkc <= 2 && (NP == 1 || ntiles >= 16);
-    if (res) return launch_assign_cfg<NP, true>(a, tA, tB, st);
-    return launch_assign_cfg<NP, false>(a, tA, tB, st);
+    // CTA pairs (M = 256 per MMA) once there are enough 256-row blocks to fill the GPU
+    if (a.N >= int64_t(2 * kBM) * device_sm_count() / 2) {
+        bool done = false;
+        const cudaError_t e = launch_assign_pair<NP>(a, st, res, &done);
+        if (done || e != cudaSuccess) return e;
+    }
+    CUtensorMap tC;
+    if (!make_tmap(&tC, a.caug, a.Kp, kAug, kAug, kBN, kAug)) return cudaErrorInvalidValue;
+    if (res) return launch_assign_cfg<NP, true>(a, tA, tB, tC, st);
+    return launch_assign_cfg<NP, false>(a, tA, tB, tC, st);
 }
 
 }  // namespace

@@ -106,6 +106,7 @@ fk_status run_assign(const void *planes, int nplanes, int64_t lda, int64_t N, in
     a.lda = lda;
     a.b_planes = ws_ptr<uint16_t>(ws, L.cs);
     a.cn = ws_ptr<float>(ws, L.cn);
+    a.caug = ws_ptr<uint16_t>(ws, L.caug);
     a.N = N;
     a.d = d;
     a.dp = static_cast<int>(L.dp);
@@ -231,7 +232,8 @@ fk_status fk_assign(const void *X, fk_dtype dtype, int64_t N, int d, const float
     if ((s = check_device()) != FK_OK) return s;
     cudaStream_t st = stream;
     FK_TRY_CUDA(launch_prep_centroids(C, K, d, L.Kp, L.dp, dtype, ws_ptr<uint16_t>(ws, L.cs),
-                                      ws_ptr<float>(ws, L.cn), ws_ptr<float>(ws, L.cused), st));
+                                      ws_ptr<float>(ws, L.cn), ws_ptr<float>(ws, L.cused),
+                                      ws_ptr<uint16_t>(ws, L.caug), st));
     float *xnorm = mind ? ws_ptr<float>(ws, L.xnorm) : nullptr;
     const void *planes = nullptr;
     int nplanes = 0;
@@ -262,7 +264,7 @@ fk_status fk_update(const void *X, fk_dtype dtype, int64_t N, int d, int K,
     if (dtype == FK_BF16) {
         FK_TRY_CUDA(launch_prep_centroids(C_old, K, d, L.Kp, L.dp, dtype,
                                           ws_ptr<uint16_t>(ws, L.cs), ws_ptr<float>(ws, L.cn),
-                                          ws_ptr<float>(ws, L.cused), st));
+                                          ws_ptr<float>(ws, L.cused), nullptr, st));
         C_used = ws_ptr<float>(ws, L.cused);
     }
     return run_update(X, dtype, N, d, K, L, ws, labels, C_old, C_used, C_new, counts, offsets,
@@ -329,7 +331,8 @@ fk_status fk_lloyd(const void *X, fk_dtype dtype, int64_t N, int d, int K, fk_me
     int copied = 0;
     for (int t = 0; t < niter; ++t) {
         if (launch_prep_centroids(Ccur, K, d, L.Kp, L.dp, dtype, ws_ptr<uint16_t>(ws, L.cs),
-                                  ws_ptr<float>(ws, L.cn), cused, st) != cudaSuccess)
+                                  ws_ptr<float>(ws, L.cn), cused, ws_ptr<uint16_t>(ws, L.caug),
+                                  st) != cudaSuccess)
             return fail(FK_ERR_CUDA);
         if (!rec()) return fail(FK_ERR_CUDA);
         if ((s = run_assign(planes, nplanes, lda, N, d, K, L, ws, labels, nullptr, nullptr,

@@ -14,6 +14,7 @@ namespace fk {
 constexpr int kBM = 128;  // rows of X per tile (one TMEM lane per row)
 constexpr int kBN = 256;  // centroids per tile (fp32 accumulator columns)
 constexpr int kBK = 64;   // bf16 elements per 128-byte swizzle row
+constexpr int kAug = 16;  // bf16 columns of the norm-folding K step (32-byte rows)
 
 // ----------------------------------------------------------------- sort tiling
 constexpr int kSortThreads = 256;
@@ -91,7 +92,7 @@ inline UpdPlan upd_plan(int64_t N, int d) {
 struct WsLayout {
     size_t err = 0, obj = 0, xn = 0, xs = 0, xnorm = 0, cs = 0, cn = 0, cused = 0,
            calt = 0, keys0 = 0, keys1 = 0, vals0 = 0, vals1 = 0, hist = 0, dtot = 0,
-           pieces = 0, pkeys = 0, piecesb = 0, pkeysb = 0, jpart = 0, jdev = 0, cnt = 0,
+           caug = 0, pieces = 0, pkeys = 0, piecesb = 0, pkeysb = 0, jpart = 0, jdev = 0, cnt = 0,
            off = 0, total = 0;
     int64_t dp = 0, Kp = 0;
     int xplanes = 0;  // bf16 planes of X prepared in the workspace (0, 1 or 2)
@@ -121,6 +122,7 @@ inline WsLayout ws_layout(int64_t N, int d, int K, fk_dtype dtype, fk_metric met
     L.xnorm = take(sizeof(float) * N);
     L.cs = take(sizeof(uint16_t) * L.cplanes * L.Kp * L.dp);
     L.cn = take(sizeof(float) * L.Kp);
+    L.caug = take(sizeof(uint16_t) * L.Kp * kAug);
     L.cused = take(sizeof(float) * K * d);
     L.calt = take(sizeof(float) * K * d);
     L.keys0 = take(sizeof(int32_t) * N);
@@ -156,6 +158,7 @@ struct AssignArgs {
     int64_t lda;           // row stride of an X plane, elements
     const void *b_planes;  // bf16 centroid planes [cplanes][Kp][dp], scaled by -2
     const float *cn;       // [Kp], +inf beyond K
+    const void *caug;      // [Kp][16] bf16: ||c||^2 as hi + mid + lo, then zeros
     int64_t N;
     int d, dp, K, Kp;
     int32_t *labels;
@@ -175,7 +178,7 @@ cudaError_t launch_xnorm_bf16(const uint16_t *X, int64_t N, int d, float *xnorm,
                               cudaStream_t st);
 cudaError_t launch_prep_centroids(const float *C, int K, int d, int64_t Kp, int64_t dp,
                                   fk_dtype dtype, uint16_t *planes, float *cn, float *cused,
-                                  cudaStream_t st);
+                                  uint16_t *caug, cudaStream_t st);
 cudaError_t launch_centroid_norms(const float *C, int K, int d, fk_dtype dtype, float *cn,
                                   cudaStream_t st);
 cudaError_t launch_assign(const AssignArgs &a, cudaStream_t st);

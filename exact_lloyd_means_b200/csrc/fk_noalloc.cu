@@ -4,9 +4,9 @@
 // framework's memory manager (which owns every byte of device memory and forbids
 // cudaMalloc behind its back), and latency-critical paths where cudaMalloc/cudaFree would
 // implicitly synchronise the device.  For them this entry point takes its scratch (the
-// error words, the centroid operand planes and norms, and the bf16 planes of X when the
-// points need splitting or padding) from one file-scope device array of fixed size,
-// instead of from a caller-provided workspace.  The array is part of the library image:
+// error words, the centroid operand planes, norms and norm pieces, and the bf16 planes of
+// X when the points need splitting or padding) from one file-scope device array of fixed
+// size, instead of from a caller-provided workspace.  The array is part of the library image:
 // every GPU that loads libfk holds it until the process exits.
 #include <mutex>
 
@@ -69,6 +69,7 @@ extern "C" FK_API fk_status fk_assign_noalloc(const void *X, fk_dtype dtype, int
     const size_t o_err = take(o, 256);
     const size_t o_cs = take(o, sizeof(uint16_t) * cplanes * Kp * dp);
     const size_t o_cn = take(o, sizeof(float) * Kp);
+    const size_t o_ca = take(o, sizeof(uint16_t) * Kp * kAug);
     const size_t o_xs = take(o, sizeof(uint16_t) * xplanes * N * dp);
     if (o > kStaticScratchBytes) return FK_ERR_WORKSPACE;  // beyond the static maximum
 
@@ -87,11 +88,12 @@ extern "C" FK_API fk_status fk_assign_noalloc(const void *X, fk_dtype dtype, int
     uint32_t *err = reinterpret_cast<uint32_t *>(sc + o_err);
     uint16_t *cs = reinterpret_cast<uint16_t *>(sc + o_cs);
     float *cn = reinterpret_cast<float *>(sc + o_cn);
+    uint16_t *caug = reinterpret_cast<uint16_t *>(sc + o_ca);
     uint16_t *xs = reinterpret_cast<uint16_t *>(sc + o_xs);
 
     // the array keeps the previous call's contents: the error words must start at zero
     if (cudaMemsetAsync(err, 0, 2 * sizeof(uint32_t), st) != cudaSuccess) return FK_ERR_CUDA;
-    if (launch_prep_centroids(C, K, d, Kp, dp, dtype, cs, cn, nullptr, st) != cudaSuccess)
+    if (launch_prep_centroids(C, K, d, Kp, dp, dtype, cs, cn, nullptr, caug, st) != cudaSuccess)
         return FK_ERR_CUDA;
     AssignArgs a{};
     if (dtype == FK_F32) {
@@ -114,6 +116,7 @@ extern "C" FK_API fk_status fk_assign_noalloc(const void *X, fk_dtype dtype, int
     }
     a.b_planes = cs;
     a.cn = cn;
+    a.caug = caug;
     a.N = N;
     a.d = d;
     a.dp = static_cast<int>(dp);

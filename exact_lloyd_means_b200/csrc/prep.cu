@@ -6,8 +6,11 @@
 //               hi*lo' reproduce x.c to about 3 * 2^-16 relative (fp32 emulation).
 //  * prep_centroids: the same split of each centroid, scaled by -2 (exact in bf16), so the
 //               MMA accumulates -2 x.c directly; cn[k] = ||c_k||^2 (fp64 accumulation of
-//               the values the MMA consumes, rounded once); padding centroids get
-//               cn = +inf and zero planes so they can never win the argmin.
+//               the values the MMA consumes, rounded once to fp32); caug[k] = the three
+//               bf16 pieces hi + mid + lo that sum exactly to that fp32 value (then zeros),
+//               which one extra K = 16 MMA step against constant (1, 1, 1, 0, ...) columns
+//               of X folds into the accumulator.  Padding centroids get cn = +inf, a
+//               largest-finite bf16 first piece and zero planes, so they never win.
 //  * normalize: cosine mode (LEANN FlashLib guide, "距离度量只有 squared L2如何支持 mips /
 //               cosine"): x / ||x|| with a zero norm replaced by 1; the norm and the
 //               quotient are computed in fp64 and rounded once to fp32.
@@ -131,7 +134,8 @@ __global__ void normalize_kernel(const float *__restrict__ X, float *__restrict_
 // widened to fp32, i.e. exactly what the MMA sees.
 __global__ void prep_centroids_kernel(const float *__restrict__ C, int K, int d, int64_t Kp,
                                       int64_t dp, int two_planes, uint16_t *__restrict__ planes,
-                                      float *__restrict__ cn, float *__restrict__ cused) {
+                                      float *__restrict__ cn, float *__restrict__ cused,
+                                      uint16_t *__restrict__ caug) {
     const int lane = threadIdx.x & 31;
     const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
     const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
@@ -155,7 +159,20 @@ __global__ void prep_centroids_kernel(const float *__restrict__ C, int K, int d,
             }
         }
         s = warp_sum_d(s);
-        if (lane == 0) cn[k] = k < K ? static_cast<float>(s) : __int_as_float(0x7f800000);
+        const float c2 = static_cast<float>(s);
+        if (lane == 0) cn[k] = k < K ? c2 : __int_as_float(0x7f800000);
+        if (caug != nullptr && lane < kAug) {
+            // exact split: hi captures the top 8 bits, mid the next 8, lo the rest (a
+            // multiple of the fp32 ulp with at most 8 significant bits)
+            const uint16_t h = bf16_bits(c2);
+            const float r1 = c2 - bf16_val(h);
+            const uint16_t m = bf16_bits(r1);
+            const uint16_t l = bf16_bits(r1 - bf16_val(m));
+            uint16_t v = 0;
+            if (k < K) v = lane == 0 ? h : (lane == 1 ? m : (lane == 2 ? l : 0));
+            else v = lane == 0 ? static_cast<uint16_t>(0x7f7f) : 0;  // largest finite bf16
+            caug[k * kAug + lane] = v;
+        }
     }
 }
 
@@ -215,9 +232,9 @@ cudaError_t launch_xnorm_bf16(const uint16_t *X, int64_t N, int d, float *xnorm,
 
 cudaError_t launch_prep_centroids(const float *C, int K, int d, int64_t Kp, int64_t dp,
                                   fk_dtype dtype, uint16_t *planes, float *cn, float *cused,
-                                  cudaStream_t st) {
+                                  uint16_t *caug, cudaStream_t st) {
     prep_centroids_kernel<<<grid_for_warps(Kp, 256), 256, 0, st>>>(
-        C, K, d, Kp, dp, dtype == FK_F32 ? 1 : 0, planes, cn, cused);
+        C, K, d, Kp, dp, dtype == FK_F32 ? 1 : 0, planes, cn, cused, caug);
     note_launch();
     return cudaGetLastError();
 }
