@@ -280,18 +280,23 @@ def fk_arm(args, spec, rank, world, dist):
     assign_ms = acc["ms_assign"] / n_assign
     flops = 2.0 * spec.n * spec.k * spec.d
     achieved = flops / (assign_ms / 1e3) / 1e12
+    # The assign launches run at the clocks the power cap allows for their own (partial)
+    # tensor load, above the clock of the seconds-long cuBLAS loop behind the sustained
+    # figure, so the burst figure is the honest denominator; both are reported.
+    div = 3.0 if spec.dtype == "f32" else 1.0
+    peak = peaks["bf16"] / div
+    peak_sus = peaks["bf16_sustained"] / div
     if spec.dtype == "f32":
-        peak = peaks["bf16_sustained"] / 3.0
-        peak_note = ("fp32 products as 3 bf16 tensor-core products: measured sustained bf16 "
-                     f"dense {peaks['bf16_sustained']} TFLOP/s / 3 ({peaks['source']})")
+        peak_note = ("fp32 products as 3 bf16 tensor-core products: measured bf16 dense peak "
+                     f"{peaks['bf16']} TFLOP/s (burst) / 3 ({peaks['source']})")
     else:
-        peak = peaks["bf16_sustained"]
-        peak_note = f"measured sustained bf16 dense TFLOP/s ({peaks['source']})"
+        peak_note = f"measured bf16 dense peak {peaks['bf16']} TFLOP/s, burst ({peaks['source']})"
     trec = assign_traffic_record()
     roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
             "frac": achieved / peak, "traffic": trec["bytes_per_launch"] if trec else None,
-            "kernel": "assign_kernel (tcgen05)", "algorithmic_flops_per_launch": flops,
-            "avg_launch_ms": assign_ms, "peak_note": peak_note}
+            "kernel": "assign (tcgen05)", "algorithmic_flops_per_launch": flops,
+            "avg_launch_ms": assign_ms, "peak_note": peak_note,
+            "frac_of_sustained": achieved / peak_sus}
     upd_ms = (acc["ms_sort"] + acc["ms_update"]) / n_assign
     e_bytes = 4 if spec.dtype == "f32" else 2
     upd_bytes = spec.n * spec.d * e_bytes + 24.0 * spec.n

@@ -136,7 +136,7 @@ fk_status run_update(const void *Xp, fk_dtype dtype, int64_t N, int d, int K,
                               C_new, counts, ws_ptr<double>(ws, L.pieces),
                               ws_ptr<int32_t>(ws, L.pkeys), ws_ptr<double>(ws, L.piecesb),
                               ws_ptr<int32_t>(ws, L.pkeysb), ws_ptr<double>(ws, L.jpart),
-                              objective, st));
+                              objective, ws_ptr<uint32_t>(ws, L.err), st));
     return FK_OK;
 }
 
@@ -351,7 +351,8 @@ fk_status fk_lloyd(const void *X, fk_dtype dtype, int64_t N, int d, int K, fk_me
                           dtype == FK_F32 ? Ccur : cused, Cnext, cnt,
                           ws_ptr<double>(ws, L.pieces), ws_ptr<int32_t>(ws, L.pkeys),
                           ws_ptr<double>(ws, L.piecesb), ws_ptr<int32_t>(ws, L.pkeysb),
-                          ws_ptr<double>(ws, L.jpart), obj + (t % kObjRing), st) != cudaSuccess)
+                          ws_ptr<double>(ws, L.jpart), obj + (t % kObjRing),
+                          ws_ptr<uint32_t>(ws, L.err), st) != cudaSuccess)
             return fail(FK_ERR_CUDA);
         if (!rec()) return fail(FK_ERR_CUDA);
         float *tmp = Ccur;

@@ -23,7 +23,8 @@ constexpr int kSortTile = kSortThreads * kSortItems;  // keys per block
 constexpr int kSortMaxBits = 11;                      // digit width bound: 2048 bins
 
 // ----------------------------------------------------------------- update tiling
-constexpr int kUpdWarps = 8;          // warps per block of the level-1 kernel
+constexpr int kUpdWarps = 8;          // warps per block of the update kernels
+constexpr int kUpdGroup = 16;         // units of one combine level per unit of the next
 constexpr int kUpdMinRows = 32;       // smallest chunk of sorted positions per warp
 constexpr int kUpdMaxRows = 256;      // largest chunk
 constexpr int64_t kUpdTargetWarps = 148 * 64;  // enough warps to cover the GPU twice
@@ -134,7 +135,7 @@ inline WsLayout ws_layout(int64_t N, int d, int K, fk_dtype dtype, fk_metric met
     L.dtot = take(sizeof(uint32_t) * bins);
     L.pieces = take(sizeof(double) * L.up.nwarps * 2 * L.up.dcov);
     L.pkeys = take(sizeof(int32_t) * L.up.nwarps * 2);
-    const int64_t units2 = ceil_div(L.up.nwarps, 64) + 1;
+    const int64_t units2 = ceil_div(L.up.nwarps, kUpdGroup) + 1;
     L.piecesb = take(sizeof(double) * units2 * 2 * L.up.dcov);
     L.pkeysb = take(sizeof(int32_t) * units2 * 2);
     L.jpart = take(sizeof(double) * L.up.nwarps * L.up.ncolblk);
@@ -192,7 +193,7 @@ cudaError_t launch_update(const void *X, fk_dtype dtype, int64_t N, int d, int K
                           const int32_t *offsets, const float *C_old, const float *C_used,
                           float *C_new, int32_t *counts, double *pieces_a, int32_t *pkeys_a,
                           double *pieces_b, int32_t *pkeys_b, double *jpart,
-                          double *objective, cudaStream_t st);
+                          double *objective, uint32_t *err, cudaStream_t st);
 
 int device_sm_count();
 

@@ -28,11 +28,12 @@
 #include <cuda_bf16.h>
 
 #include "fk_common.cuh"
+#include "ptx_sm100.cuh"
 
 namespace fk {
 namespace {
 
-constexpr int kGroup = 64;  // units of level L-1 per unit of level L
+constexpr int kGroup = kUpdGroup;  // units of level L-1 per unit of level L
 
 // Write the mean of a finished cluster: C_new[k][col..col+3] = acc / cnt.
 __device__ __forceinline__ void store_mean(float *C_new, int64_t k, int d, int col,
@@ -53,17 +54,226 @@ __device__ __forceinline__ void store_piece(double *dst, const double (&acc)[4])
 
 // Level 1.  A warp owns sorted positions [w*R, w*R + R) and the 128 columns of block
 // blockIdx.y (lane l holds columns 4l .. 4l+3).  The warp first stages the R cluster ids
-// and row ids of its chunk in shared memory (one coalesced read), so row fetches never
-// wait on an index load; rows are then fetched B at a time (B = 8 fp32 / 16 bf16 rows,
-// 16 / 8 bytes per lane per row) with the next batch in flight while the current one is
-// added.  When a batch lies in one cluster its rows are first added pairwise in fp32 (a
-// fixed tree) and the batch sum is added to the fp64 accumulator once; otherwise rows are
-// added one by one in fp64.  The objective term (x - c_used)^2 of a row is formed in fp32
-// and accumulated in fp64.
+// and row ids of its chunk in shared memory (one coalesced read).  Rows are then gathered
+// with 1-D bulk copies (one 128-column slice of one row per lane, 512 bytes for fp32 and
+// 256 for bf16) into a ring of kRowRing batches of B rows (B = 8 fp32 / 16 bf16) in
+// shared memory, each batch completing on its own mbarrier, so four batches are in flight
+// per warp without holding any registers.  When a batch lies in one cluster its rows are
+// first added pairwise in fp32 (a fixed tree) and the batch sum is added to the fp64
+// accumulator once; otherwise rows are added one by one in fp64.  The objective term
+// (x - c_used)^2 of a row is formed in fp32 and accumulated in fp64.
+constexpr int kRowRing = 4;        // batches in flight per warp
+constexpr int kRowWarps = 4;       // warps per block of the level-1 kernel
+constexpr int kRowBatchBytes = 4096;  // 8 fp32 rows or 16 bf16 rows of 128 columns
+
 template <bool BF16>
 struct RowVec;
 template <>
 struct RowVec<false> {
+    static constexpr int kBatch = 8;
+    static constexpr int kSlice = 512;  // bytes of a 128-column slice
+    __device__ static void load(const uint8_t *p, float (&f)[4]) {
+        const float4 v = *reinterpret_cast<const float4 *>(p);
+        f[0] = v.x;
+        f[1] = v.y;
+        f[2] = v.z;
+        f[3] = v.w;
+    }
+};
+template <>
+struct RowVec<true> {
+    static constexpr int kBatch = 16;
+    static constexpr int kSlice = 256;
+    __device__ static void load(const uint8_t *p, float (&f)[4]) {
+        const uint2 u = *reinterpret_cast<const uint2 *>(p);
+        f[0] = __uint_as_float(u.x << 16);
+        f[1] = __uint_as_float(u.x & 0xffff0000u);
+        f[2] = __uint_as_float(u.y << 16);
+        f[3] = __uint_as_float(u.y & 0xffff0000u);
+    }
+};
+
+constexpr size_t kRowSmem = size_t(kRowWarps) * kRowRing * kRowBatchBytes;  // dynamic part
+
+template <bool BF16>
+__global__ void __launch_bounds__(kRowWarps * 32, 3)
+    seg_rows_kernel(const void *__restrict__ X, int64_t N, int d, int R, int64_t nwarps,
+                    int dcov, const int32_t *__restrict__ skeys,
+                    const int32_t *__restrict__ perm, const int32_t *__restrict__ offsets,
+                    const float *__restrict__ C_used, float *__restrict__ C_new,
+                    double *__restrict__ pieces, int32_t *__restrict__ pkeys,
+                    double *__restrict__ jpart, uint32_t *__restrict__ err) {
+    using RV = RowVec<BF16>;
+    constexpr int B = RV::kBatch;
+    constexpr int SL = RV::kSlice;
+    constexpr int E = BF16 ? 2 : 4;
+    constexpr uint64_t kWaitNs = 2000000000ull;
+    extern __shared__ __align__(128) uint8_t s_rows_all[];  // [warp][ring][B][SL]
+    __shared__ int32_t s_key[kRowWarps][kUpdMaxRows];
+    __shared__ int32_t s_row[kRowWarps][kUpdMaxRows];
+    __shared__ __align__(8) uint64_t s_bar[kRowWarps][kRowRing];
+    const int lane = threadIdx.x & 31;
+    const int wib = threadIdx.x >> 5;
+    const int64_t w = static_cast<int64_t>(blockIdx.x) * kRowWarps + wib;
+    if (w >= nwarps) return;
+    const int cb = blockIdx.y;
+    const int col = cb * 128 + lane * 4;
+    const bool colv = col < d;
+    const int col0 = cb * 128;
+    const uint32_t slice = static_cast<uint32_t>((d - col0 < 128 ? d - col0 : 128) * E);
+    const int64_t p0 = w * R;
+    const int n = static_cast<int>((p0 + R < N ? p0 + R : N) - p0);
+    const int64_t p1 = p0 + n;
+    int32_t *sk = s_key[wib];
+    int32_t *si = s_row[wib];
+    uint64_t *bar = s_bar[wib];
+    uint8_t *rows = s_rows_all + static_cast<size_t>(wib) * kRowRing * kRowBatchBytes;
+    if (lane < kRowRing) ptx::mbar_init(&bar[lane], 1);
+    ptx::fence_mbar_init();
+    for (int j = lane; j < n; j += 32) {
+        sk[j] = skeys[p0 + j];
+        si[j] = perm[p0 + j];
+    }
+    __syncwarp();
+
+    const uint8_t *Xb = static_cast<const uint8_t *>(X);
+    // Gather the rows of the batch starting at sorted position b into ring slot `slot`.
+    auto issue = [&](int b, int slot) {
+        if (b >= n) return;
+        const int nb = n - b < B ? n - b : B;
+        if (lane == 0) ptx::mbar_arrive_expect_tx(&bar[slot], nb * slice);
+        __syncwarp();
+        if (lane < nb)
+            ptx::bulk_load(rows + slot * kRowBatchBytes + lane * SL,
+                           Xb + (static_cast<int64_t>(si[b + lane]) * d + col0) * E, slice,
+                           &bar[slot]);
+    };
+
+    double acc[4] = {0.0, 0.0, 0.0, 0.0};
+    float cu[4] = {0.f, 0.f, 0.f, 0.f};
+    double jacc = 0.0;
+    int cur = -1, first = -1, slot1 = -1;
+    bool ok = true;
+
+    auto flush = [&](int k) {
+        const int64_t lo = offsets[k], hi = offsets[k + 1];
+        if (lo >= p0 && hi <= p1) {
+            if (colv) store_mean(C_new, k, d, col, acc, static_cast<double>(hi - lo));
+        } else {
+            const int slot = (k == first) ? 0 : 1;
+            if (slot == 1) slot1 = k;
+            store_piece(pieces + (w * 2 + slot) * static_cast<int64_t>(dcov) + col, acc);
+        }
+    };
+    auto start = [&](int k) {
+        if (cur >= 0) flush(cur);
+        if (cur < 0) first = k;
+        cur = k;
+        acc[0] = acc[1] = acc[2] = acc[3] = 0.0;
+        if (colv) {
+            const float4 c = *reinterpret_cast<const float4 *>(C_used + int64_t(k) * d + col);
+            cu[0] = c.x;
+            cu[1] = c.y;
+            cu[2] = c.z;
+            cu[3] = c.w;
+        }
+    };
+
+    for (int i = 0; i < kRowRing; ++i) issue(i * B, i);
+    int it = 0;
+    for (int b = 0; b < n; b += B, ++it) {
+        const int slot = it % kRowRing;
+        uint32_t got = 1;
+        if (lane == 0) got = ptx::mbar_wait(&bar[slot], (it / kRowRing) & 1u, nullptr, kWaitNs);
+        if (!__shfl_sync(0xffffffffu, got, 0)) {
+            if (lane == 0) err[0] = kErrTimeout;
+            ok = false;
+            break;
+        }
+        const uint8_t *base = rows + slot * kRowBatchBytes + lane * (4 * E);
+        const int nb = n - b < B ? n - b : B;
+        const int kf = sk[b], kl = sk[b + nb - 1];
+        if (kf == kl) {
+            // one cluster for the whole batch (positions are sorted by cluster id)
+            if (kf != cur) start(kf);
+            float xs[B][4];
+            float jr[B];
+#pragma unroll
+            for (int j = 0; j < B; ++j) {
+                if (j < nb && colv) {
+                    RV::load(base + j * SL, xs[j]);
+                } else {
+                    xs[j][0] = xs[j][1] = xs[j][2] = xs[j][3] = 0.f;
+                }
+                float t = 0.f;
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float df = j < nb ? xs[j][e] - cu[e] : 0.f;
+                    t = fmaf(df, df, t);
+                }
+                jr[j] = t;
+            }
+#pragma unroll
+            for (int h = B / 2; h > 0; h >>= 1) {
+#pragma unroll
+                for (int j = 0; j < h; ++j) {
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) xs[j][e] += xs[j + h][e];
+                    jr[j] += jr[j + h];
+                }
+            }
+#pragma unroll
+            for (int e = 0; e < 4; ++e) acc[e] += static_cast<double>(xs[0][e]);
+            jacc += static_cast<double>(jr[0]);
+        } else {
+            for (int j = 0; j < nb; ++j) {
+                const int k = sk[b + j];
+                if (k != cur) start(k);
+                float x[4] = {0.f, 0.f, 0.f, 0.f};
+                if (colv) RV::load(base + j * SL, x);
+                float t = 0.f;
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    acc[e] += static_cast<double>(x[e]);
+                    const float df = x[e] - cu[e];
+                    t = fmaf(df, df, t);
+                }
+                jacc += static_cast<double>(t);
+            }
+        }
+        ptx::fence_proxy_async_smem();  // this lane's reads of the slot precede the refill
+        __syncwarp();                   // every lane has read the slot before it is refilled
+        issue(b + kRowRing * B, slot);
+    }
+    if (!ok) {
+        // let the (at most kRowRing) copies still outstanding land before the warp leaves
+        for (int i2 = it; i2 < it + kRowRing && i2 * B < n; ++i2) {
+            if (lane == 0)
+                ptx::mbar_wait(&bar[i2 % kRowRing], (i2 / kRowRing) & 1u, nullptr, kWaitNs);
+        }
+        return;
+    }
+    if (cur >= 0) flush(cur);
+    if (cb == 0 && lane == 0) {
+        // slot 0 holds the first cluster if it was not finished here; slot 1 the last
+        const int64_t lo = offsets[first], hi = offsets[first + 1];
+        const bool first_done = lo >= p0 && hi <= p1;
+        pkeys[w * 2 + 0] = first_done ? -1 : first;
+        pkeys[w * 2 + 1] = slot1;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) jacc += __shfl_xor_sync(0xffffffffu, jacc, o);
+    if (lane == 0) jpart[static_cast<int64_t>(cb) * nwarps + w] = jacc;
+}
+
+// Level 1, register-gather form, used for bf16 rows: a 128-column slice of a bf16 row is
+// only 256 bytes, too small for one bulk copy per row to pay off.  Lanes load their 8 bytes
+// of each row directly, B = 16 rows per batch, with the next batch in flight in registers
+// while the current one is added; the arithmetic is that of seg_rows_kernel.
+template <bool BF16>
+struct RegRowVec;
+template <>
+struct RegRowVec<false> {
     using T = float4;
     static constexpr int kBatch = 8;
     __device__ static void unpack(const float4 &v, float (&f)[4]) {
@@ -75,7 +285,7 @@ struct RowVec<false> {
     __device__ static float4 zero() { return make_float4(0.f, 0.f, 0.f, 0.f); }
 };
 template <>
-struct RowVec<true> {
+struct RegRowVec<true> {
     using T = uint2;
     static constexpr int kBatch = 16;
     __device__ static void unpack(const uint2 &u, float (&f)[4]) {
@@ -89,13 +299,13 @@ struct RowVec<true> {
 
 template <bool BF16>
 __global__ void __launch_bounds__(kUpdWarps * 32, 2)
-    seg_rows_kernel(const void *__restrict__ X, int64_t N, int d, int R, int64_t nwarps,
+    seg_rows_regs_kernel(const void *__restrict__ X, int64_t N, int d, int R, int64_t nwarps,
                     int dcov, const int32_t *__restrict__ skeys,
                     const int32_t *__restrict__ perm, const int32_t *__restrict__ offsets,
                     const float *__restrict__ C_used, float *__restrict__ C_new,
                     double *__restrict__ pieces, int32_t *__restrict__ pkeys,
                     double *__restrict__ jpart) {
-    using RV = RowVec<BF16>;
+    using RV = RegRowVec<BF16>;
     using V = typename RV::T;
     constexpr int B = RV::kBatch;
     __shared__ int32_t s_key[kUpdWarps][kUpdMaxRows];
@@ -342,18 +552,30 @@ __global__ void __launch_bounds__(1024)
 cudaError_t run_levels(const void *X, bool bf16, int64_t N, int d, const UpdPlan &up,
                        const int32_t *skeys, const int32_t *perm, const int32_t *offsets,
                        const float *C_used, float *C_new, double *pa, int32_t *ka,
-                       double *pb, int32_t *kb, double *jpart, cudaStream_t st) {
-    const dim3 block(kUpdWarps * 32);
-    dim3 grid(static_cast<unsigned>(ceil_div(up.nwarps, kUpdWarps)), up.ncolblk);
+                       double *pb, int32_t *kb, double *jpart, uint32_t *err,
+                       cudaStream_t st) {
+    static bool attr = false;
+    if (!attr) {
+        cudaFuncSetAttribute(seg_rows_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(kRowSmem));
+        cudaFuncSetAttribute(seg_rows_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(kRowSmem));
+        attr = true;
+    }
+    const dim3 rblock(kRowWarps * 32);
+    dim3 rgrid(static_cast<unsigned>(ceil_div(up.nwarps, kRowWarps)), up.ncolblk);
     if (bf16)
-        seg_rows_kernel<true><<<grid, block, 0, st>>>(X, N, d, up.rows, up.nwarps, up.dcov,
-                                                      skeys, perm, offsets, C_used, C_new, pa,
-                                                      ka, jpart);
+        seg_rows_regs_kernel<true><<<dim3(static_cast<unsigned>(ceil_div(up.nwarps, kUpdWarps)),
+                                          up.ncolblk),
+                                     dim3(kUpdWarps * 32), 0, st>>>(
+            X, N, d, up.rows, up.nwarps, up.dcov, skeys, perm, offsets, C_used, C_new, pa, ka,
+            jpart);
     else
-        seg_rows_kernel<false><<<grid, block, 0, st>>>(X, N, d, up.rows, up.nwarps, up.dcov,
-                                                       skeys, perm, offsets, C_used, C_new, pa,
-                                                       ka, jpart);
+        seg_rows_kernel<false><<<rgrid, rblock, kRowSmem, st>>>(
+            X, N, d, up.rows, up.nwarps, up.dcov, skeys, perm, offsets, C_used, C_new, pa, ka,
+            jpart, err);
     note_launch();
+    const dim3 block(kUpdWarps * 32);
     int64_t units = up.nwarps;
     int64_t span = up.rows;
     double *pin = pa, *pout = pb;
@@ -383,10 +605,10 @@ cudaError_t launch_update(const void *X, fk_dtype dtype, int64_t N, int d, int K
                           const int32_t *offsets, const float *C_old, const float *C_used,
                           float *C_new, int32_t *counts, double *pieces_a, int32_t *pkeys_a,
                           double *pieces_b, int32_t *pkeys_b, double *jpart,
-                          double *objective, cudaStream_t st) {
+                          double *objective, uint32_t *err, cudaStream_t st) {
     const bool bf16 = dtype == FK_BF16;
     cudaError_t e = run_levels(X, bf16, N, d, up, skeys, perm, offsets, C_used, C_new,
-                               pieces_a, pkeys_a, pieces_b, pkeys_b, jpart, st);
+                               pieces_a, pkeys_a, pieces_b, pkeys_b, jpart, err, st);
     if (e != cudaSuccess) return e;
     int64_t fgrid = ceil_div(K, 8);
     const int64_t cap = static_cast<int64_t>(device_sm_count()) * 16;
