@@ -10,8 +10,10 @@ Default workload: N = 1,000,000 points, d = 768, K = 4096, fp32, cosine, 20 iter
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
 
-Under torchrun every rank runs its own independent copy of the workload (its own seed), so
-per-GPU work is fixed (weak scaling); the whole-job value divides all ranks' points x
+Under torchrun (N > 1 ranks) the run is data-parallel: every rank holds N points of its own
+(its own seed; per-GPU work is fixed, weak scaling), the centroids are replicated from
+rank 0, and each iteration exchanges per-cluster sums and counts with NCCL all_gather
+(exact_lloyd_means_b200.dist).  The whole-job value divides all ranks' points x
 iterations by the slowest rank's device time.
 """
 from __future__ import annotations
@@ -65,9 +67,9 @@ def load_peaks():
     return {"hbm_gbs": 6650.0, "bf16": 1590.0, "bf16_sustained": 1400.0, "source": "fallback"}
 
 
-def assign_traffic_record():
+def assign_traffic_record(workload):
     """DRAM bytes per assign launch from a committed ncu summary, if it was taken on the
-    current kernel source (else None)."""
+    current kernel source and for this workload (else None)."""
     path = os.path.join(ROOT, "profiles", "assign_traffic.json")
     src = os.path.join(ROOT, "exact_lloyd_means_b200", "csrc", "assign_sm100.cu")
     if not os.path.exists(path):
@@ -75,7 +77,7 @@ def assign_traffic_record():
     with open(path) as f:
         rec = json.load(f)
     h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
-    return rec if rec.get("kernel_sha") == h else None
+    return rec if rec.get("kernel_sha") == h and rec.get("workload") == workload else None
 
 
 class ClockSampler:
@@ -218,26 +220,47 @@ def fk_arm(args, spec, rank, world, dist):
 
     dev = torch.device("cuda", torch.cuda.current_device())
     niter = args.niter or spec.niter
+    sharded = world > 1
+    # weak scaling: every rank holds spec.n points of its own (own seed); one k-means
+    # problem over all world * spec.n points when sharded
     seed = spec.seed + rank
     X, _, _ = gaussian_mixture(spec.n, spec.d, spec.k, centers=spec.centers, sigma=spec.sigma,
                                weights=spec.weights, zipf_s=spec.zipf_s, dtype=spec.dtype,
                                seed=seed, device=dev)
     C0 = X[init_indices(spec.n, spec.k, seed, device=dev)].float().contiguous()
+    if sharded:
+        dist.broadcast(C0, src=0)  # replicated initial centroids: rank 0's choice
     C = torch.empty_like(C0)
     labels = torch.empty(spec.n, dtype=torch.int32, device=dev)
     counts = torch.empty(spec.k, dtype=torch.int32, device=dev)
-    ws = fk.workspace(spec.n, spec.d, spec.k, X.dtype, spec.metric, device=dev)
+    if sharded:
+        from exact_lloyd_means_b200.dist import gpu_ops, lloyd_sharded
+        ops = gpu_ops(spec.n, spec.d, spec.k, X.dtype, dev)
+        Xn = torch.empty_like(X) if spec.metric == "cosine" else None
+    else:
+        ws = fk.workspace(spec.n, spec.d, spec.k, X.dtype, spec.metric, device=dev)
     torch.cuda.synchronize()
+
+    def run(Xin, acc):
+        """One complete k-means run from raw points and C (in place)."""
+        if not sharded:
+            objs, tm = fk.fk_lloyd(Xin, C, niter, labels, ws, metric=spec.metric,
+                                   counts=counts, timing=acc is not None)
+            if acc is not None:
+                for k in ("ms_setup", "ms_prep", "ms_assign", "ms_sort", "ms_update"):
+                    acc[k] = acc.get(k, 0.0) + tm[k]
+            return objs
+        Xp = Xin
+        if spec.metric == "cosine":  # normalise once per run, as fk_lloyd does
+            fk.fk_normalize_rows(Xin, Xn)
+            fk.fk_normalize_rows(C, C)
+            Xp = Xn
+        objs, _ = lloyd_sharded(Xp, C, niter, ops, timing=acc)
+        return objs
 
     def step(acc):
         C.copy_(C0)
-        objs, tm = fk.fk_lloyd(X, C, niter, labels, ws, metric=spec.metric, counts=counts,
-                               timing=True)
-        if acc is not None:
-            for k in ("ms_setup", "ms_prep", "ms_assign", "ms_sort", "ms_update"):
-                acc[k] = acc.get(k, 0.0) + tm[k]
-            acc["launches"] = acc.get("launches", 0) + tm["launches"]
-        return objs
+        return run(X, acc)
 
     for _ in range(args.warmup):
         step(None)
@@ -254,6 +277,7 @@ def fk_arm(args, spec, rank, world, dist):
     if dist:
         dist.barrier()
     torch.cuda.synchronize()
+    launches0 = fk.launch_count()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record()
@@ -261,6 +285,7 @@ def fk_arm(args, spec, rank, world, dist):
         objs = step(acc)
     e1.record()
     torch.cuda.synchronize()
+    launches = fk.launch_count() - launches0
     if dist:
         dist.barrier()
     clocks = sampler.stop()
@@ -291,17 +316,22 @@ def fk_arm(args, spec, rank, world, dist):
                      f"{peaks['bf16']} TFLOP/s (burst) / 3 ({peaks['source']})")
     else:
         peak_note = f"measured bf16 dense peak {peaks['bf16']} TFLOP/s, burst ({peaks['source']})"
-    trec = assign_traffic_record()
+    trec = assign_traffic_record(spec.name)
     roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
             "frac": achieved / peak, "traffic": trec["bytes_per_launch"] if trec else None,
             "kernel": "assign (tcgen05)", "algorithmic_flops_per_launch": flops,
             "avg_launch_ms": assign_ms, "peak_note": peak_note,
             "frac_of_sustained": achieved / peak_sus}
-    upd_ms = (acc["ms_sort"] + acc["ms_update"]) / n_assign
+    if sharded:  # the library's sort + update run inside fk_update_partial
+        upd_ms = acc["ms_partial"] / n_assign
+        phases = {k: acc[k] / args.steps for k in ("ms_assign", "ms_partial", "ms_exchange",
+                                                    "ms_finalize")}
+    else:
+        upd_ms = (acc["ms_sort"] + acc["ms_update"]) / n_assign
+        phases = {k: acc[k] / args.steps for k in ("ms_setup", "ms_prep", "ms_assign",
+                                                    "ms_sort", "ms_update")}
     e_bytes = 4 if spec.dtype == "f32" else 2
     upd_bytes = spec.n * spec.d * e_bytes + 24.0 * spec.n
-    phases = {k: acc[k] / args.steps for k in ("ms_setup", "ms_prep", "ms_assign",
-                                                "ms_sort", "ms_update")}
 
     out = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
@@ -313,7 +343,8 @@ def fk_arm(args, spec, rank, world, dist):
            "dtype": spec.dtype, "data": "synthetic",
            "config": {"workload": spec.name, "N": spec.n, "d": spec.d, "K": spec.k,
                       "metric": spec.metric, "niter_per_step": niter,
-                      "parallelism": f"replica x{world}",
+                      "parallelism": f"dp{world}" if sharded else "single GPU",
+                      "points_per_rank": spec.n,
                       "l2": f"inputs larger than L2 (X = {spec.n * spec.d * e_bytes / 1e9:.2f}"
                             " GB per rank)"},
            "roofline": roof,
@@ -322,7 +353,7 @@ def fk_arm(args, spec, rank, world, dist):
                           "frac": upd_bytes / (upd_ms / 1e3) / 1e9 / peaks["hbm_gbs"],
                           "avg_ms": upd_ms},
            "phase_ms_per_step": phases,
-           "gpu_launches": acc["launches"], "final_objective": objs[-1],
+           "gpu_launches": launches, "final_objective": objs[-1],
            "clocks": clocks}
 
     # end to end through the public API with host buffers
@@ -339,8 +370,9 @@ def fk_arm(args, spec, rank, world, dist):
         def e2e_step():
             Xd.copy_(Xh, non_blocking=True)
             C.copy_(C0h, non_blocking=True)
-            fk.fk_lloyd(Xd, C, niter, labels, ws, metric=spec.metric)
-            labh.copy_(labels, non_blocking=True)
+            run(Xd, None)
+            if not sharded:
+                labh.copy_(labels, non_blocking=True)
             Ch.copy_(C, non_blocking=True)
             torch.cuda.synchronize()
 
@@ -362,7 +394,8 @@ def fk_arm(args, spec, rank, world, dist):
             ems = t.item()
         out["e2e"] = {"value": spec.n * niter * ke * world / (ems / 1e3), "unit": UNIT,
                       "h2d_bytes_per_step": X.numel() * X.element_size() + C0.numel() * 4,
-                      "d2h_bytes_per_step": spec.n * 4 + C0.numel() * 4 + niter * 8,
+                      "d2h_bytes_per_step": (0 if sharded else spec.n * 4) + C0.numel() * 4
+                      + niter * 8,
                       "steps": ke}
         del Xh, Xd
 
@@ -400,7 +433,7 @@ def main():
         import torch.distributed as tdist
         local = int(os.environ.get("LOCAL_RANK", "0"))
         torch.cuda.set_device(local)
-        tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600))
+        tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=180))
         dist = tdist
     fk_arm(args, spec, rank, world, dist)
     if dist:

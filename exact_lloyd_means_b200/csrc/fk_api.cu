@@ -42,10 +42,13 @@ fk_status check_device() {
 
 bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
-fk_status validate_shape(int64_t N, int d, int K, fk_dtype dtype, fk_metric metric) {
+fk_status validate_shape(int64_t N, int d, int K, fk_dtype dtype, fk_metric metric,
+                         bool planes_ok = false) {
     if (N < 1 || N > 2147483647LL - 1) return FK_ERR_INVALID_ARG;
     if (d < 1 || K < 1 || K > N) return FK_ERR_INVALID_ARG;
-    if (dtype != FK_F32 && dtype != FK_BF16) return FK_ERR_UNSUPPORTED;
+    if (dtype == FK_BF16X2 && !planes_ok) return FK_ERR_UNSUPPORTED;
+    if (dtype != FK_F32 && dtype != FK_BF16 && dtype != FK_BF16X2) return FK_ERR_UNSUPPORTED;
+    if (dtype == FK_BF16X2 && metric != FK_L2) return FK_ERR_UNSUPPORTED;
     if (metric != FK_L2 && metric != FK_COSINE) return FK_ERR_UNSUPPORTED;
     if (dtype == FK_F32 && d % 4 != 0) return FK_ERR_UNSUPPORTED;
     if (dtype == FK_BF16 && d % 8 != 0) return FK_ERR_UNSUPPORTED;
@@ -75,6 +78,12 @@ fk_status prepare_x(const void *Xp, fk_dtype dtype, int64_t N, int d, const WsLa
                     void *ws, float *xnorm, cudaStream_t st, const void **planes,
                     int *nplanes, int64_t *lda) {
     uint16_t *xs = ws_ptr<uint16_t>(ws, L.xs);
+    if (dtype == FK_BF16X2) {  // already split by fk_split_points
+        *planes = Xp;
+        *nplanes = 2;
+        *lda = L.dp;
+        return FK_OK;
+    }
     if (dtype == FK_F32) {
         FK_TRY_CUDA(launch_split_x(static_cast<const float *>(Xp), N, d, L.dp, xs, xs + N * L.dp,
                                    xnorm, st));
@@ -125,7 +134,8 @@ fk_status run_assign(const void *planes, int nplanes, int64_t lda, int64_t N, in
 fk_status run_update(const void *Xp, fk_dtype dtype, int64_t N, int d, int K,
                      const WsLayout &L, void *ws, const int32_t *labels, const float *C_old,
                      const float *C_used, float *C_new, int32_t *counts, int32_t *offsets,
-                     int32_t *perm_out, double *objective, cudaStream_t st) {
+                     int32_t *perm_out, double *objective, double *sums_out,
+                     cudaStream_t st) {
     const int32_t *skeys = nullptr, *perm = nullptr;
     FK_TRY_CUDA(launch_sort_csr(labels, N, K, L.sp, ws_ptr<int32_t>(ws, L.keys0),
                                 ws_ptr<int32_t>(ws, L.keys1), ws_ptr<int32_t>(ws, L.vals0),
@@ -136,7 +146,7 @@ fk_status run_update(const void *Xp, fk_dtype dtype, int64_t N, int d, int K,
                               C_new, counts, ws_ptr<double>(ws, L.pieces),
                               ws_ptr<int32_t>(ws, L.pkeys), ws_ptr<double>(ws, L.piecesb),
                               ws_ptr<int32_t>(ws, L.pkeysb), ws_ptr<double>(ws, L.jpart),
-                              objective, ws_ptr<uint32_t>(ws, L.err), st));
+                              objective, ws_ptr<uint32_t>(ws, L.err), sums_out, st));
     return FK_OK;
 }
 
@@ -187,10 +197,12 @@ const char *fk_status_string(fk_status s) {
 
 int fk_version(void) { return 1; }
 
+int64_t fk_launch_count(void) { return g_launches; }
+
 fk_status fk_workspace_size(int64_t N, int d, int K, fk_dtype dtype, fk_metric metric,
                             size_t *bytes) {
     if (!bytes) return FK_ERR_INVALID_ARG;
-    fk_status s = validate_shape(N, d, K, dtype, metric);
+    fk_status s = validate_shape(N, d, K, dtype, metric, true);
     if (s != FK_OK) return s;
     const size_t a = ws_layout(N, d, K, dtype, metric).total;
     const size_t b = ws_layout(N, d, K, dtype, FK_L2).total;
@@ -209,6 +221,17 @@ fk_status fk_normalize_rows(const float *X_in, float *X_out, int64_t N, int d,
     return FK_OK;
 }
 
+fk_status fk_split_points(const float *X, int64_t N, int d, void *planes, fk_stream_t stream) {
+    if (N < 1 || d < 1 || !X || !planes) return FK_ERR_INVALID_ARG;
+    if (d % 4 != 0 || !aligned(X, 16) || !aligned(planes, 16)) return FK_ERR_UNSUPPORTED;
+    fk_status s = check_device();
+    if (s != FK_OK) return s;
+    const int64_t dp = round_up(d, kBK);
+    uint16_t *p = static_cast<uint16_t *>(planes);
+    FK_TRY_CUDA(launch_split_x(X, N, d, dp, p, p + N * dp, nullptr, stream));
+    return FK_OK;
+}
+
 fk_status fk_centroid_norms(const float *C, int K, int d, fk_dtype dtype, float *cn,
                             fk_stream_t stream) {
     if (K < 1 || d < 1 || !C || !cn) return FK_ERR_INVALID_ARG;
@@ -222,7 +245,8 @@ fk_status fk_centroid_norms(const float *C, int K, int d, fk_dtype dtype, float 
 fk_status fk_assign(const void *X, fk_dtype dtype, int64_t N, int d, const float *C, int K,
                     int32_t *labels, float *mind, void *ws, size_t ws_bytes,
                     fk_stream_t stream) {
-    fk_status s = validate_shape(N, d, K, dtype, FK_L2);
+    fk_status s = validate_shape(N, d, K, dtype, FK_L2, true);
+    if (s == FK_OK && dtype == FK_BF16X2 && mind) return FK_ERR_UNSUPPORTED;
     if (s != FK_OK) return s;
     if (!X || !C || !labels) return FK_ERR_INVALID_ARG;
     if (!aligned(X, 16) || !aligned(C, 4) || !aligned(labels, 4) || (mind && !aligned(mind, 4)))
@@ -268,7 +292,7 @@ fk_status fk_update(const void *X, fk_dtype dtype, int64_t N, int d, int K,
         C_used = ws_ptr<float>(ws, L.cused);
     }
     return run_update(X, dtype, N, d, K, L, ws, labels, C_old, C_used, C_new, counts, offsets,
-                      perm, objective, st);
+                      perm, objective, nullptr, st);
 }
 
 fk_status fk_lloyd(const void *X, fk_dtype dtype, int64_t N, int d, int K, fk_metric metric,
@@ -352,7 +376,7 @@ fk_status fk_lloyd(const void *X, fk_dtype dtype, int64_t N, int d, int K, fk_me
                           ws_ptr<double>(ws, L.pieces), ws_ptr<int32_t>(ws, L.pkeys),
                           ws_ptr<double>(ws, L.piecesb), ws_ptr<int32_t>(ws, L.pkeysb),
                           ws_ptr<double>(ws, L.jpart), obj + (t % kObjRing),
-                          ws_ptr<uint32_t>(ws, L.err), st) != cudaSuccess)
+                          ws_ptr<uint32_t>(ws, L.err), nullptr, st) != cudaSuccess)
             return fail(FK_ERR_CUDA);
         if (!rec()) return fail(FK_ERR_CUDA);
         float *tmp = Ccur;
@@ -395,6 +419,48 @@ fk_status fk_lloyd(const void *X, fk_dtype dtype, int64_t N, int d, int K, fk_me
     }
     cleanup();
     return static_cast<fk_status>(code);
+}
+
+fk_status fk_update_partial(const void *X, fk_dtype dtype, int64_t N, int d, int K,
+                            const int32_t *labels, const float *C_old, double *sums,
+                            int32_t *counts, int32_t *offsets, double *objective, void *ws,
+                            size_t ws_bytes, fk_stream_t stream) {
+    fk_status s = validate_shape(N, d, K, dtype, FK_L2);
+    if (s != FK_OK) return s;
+    if (!X || !labels || !C_old || !sums || !counts || !offsets) return FK_ERR_INVALID_ARG;
+    if (!aligned(X, 16) || !aligned(C_old, 16) || !aligned(sums, 16) || !aligned(labels, 4) ||
+        !aligned(counts, 4) || !aligned(offsets, 4) || (objective && !aligned(objective, 8)))
+        return FK_ERR_UNSUPPORTED;
+    const WsLayout L = ws_layout(N, d, K, dtype, FK_L2);
+    if ((s = check_ws(ws, ws_bytes, L)) != FK_OK) return s;
+    if ((s = check_device()) != FK_OK) return s;
+    cudaStream_t st = stream;
+    const float *C_used = C_old;
+    if (dtype == FK_BF16) {
+        FK_TRY_CUDA(launch_prep_centroids(C_old, K, d, L.Kp, L.dp, dtype,
+                                          ws_ptr<uint16_t>(ws, L.cs), ws_ptr<float>(ws, L.cn),
+                                          ws_ptr<float>(ws, L.cused), nullptr, st));
+        C_used = ws_ptr<float>(ws, L.cused);
+    }
+    return run_update(X, dtype, N, d, K, L, ws, labels, C_old, C_used, nullptr, counts,
+                      offsets, nullptr, objective, sums, st);
+}
+
+fk_status fk_finalize_shards(const double *sums, const int64_t *counts_w,
+                             const double *objectives_w, int W, int K, int d,
+                             const float *C_old, float *C_new, int64_t *counts,
+                             double *objective, fk_stream_t stream) {
+    if (W < 1 || K < 1 || d < 1 || !sums || !counts_w || !C_old || !C_new)
+        return FK_ERR_INVALID_ARG;
+    if ((objective && !objectives_w) || static_cast<int64_t>(K) * d > 2147483647LL)
+        return FK_ERR_INVALID_ARG;
+    const size_t cbytes = sizeof(float) * static_cast<size_t>(K) * d;
+    if (overlap(C_old, cbytes, C_new, cbytes)) return FK_ERR_INVALID_ARG;
+    fk_status s = check_device();
+    if (s != FK_OK) return s;
+    FK_TRY_CUDA(launch_finalize_shards(sums, counts_w, objectives_w, W, K, d, C_old, C_new,
+                                       counts, objective, stream));
+    return FK_OK;
 }
 
 fk_status fk_get_device_error(void *ws, size_t ws_bytes, int *code, fk_stream_t stream) {

@@ -106,8 +106,8 @@ inline WsLayout ws_layout(int64_t N, int d, int K, fk_dtype dtype, fk_metric met
     WsLayout L;
     L.dp = round_up(d, kBK);
     L.Kp = round_up(K, kBN);
-    L.cplanes = dtype == FK_F32 ? 2 : 1;
-    L.xplanes = dtype == FK_F32 ? 2 : ((d % kBK) != 0 ? 1 : 0);
+    L.cplanes = dtype == FK_BF16 ? 1 : 2;
+    L.xplanes = dtype == FK_F32 ? 2 : ((dtype == FK_BF16 && (d % kBK) != 0) ? 1 : 0);
     L.sp = sort_plan(N, K);
     L.up = upd_plan(N, d);
     size_t o = 0;
@@ -193,7 +193,11 @@ cudaError_t launch_update(const void *X, fk_dtype dtype, int64_t N, int d, int K
                           const int32_t *offsets, const float *C_old, const float *C_used,
                           float *C_new, int32_t *counts, double *pieces_a, int32_t *pkeys_a,
                           double *pieces_b, int32_t *pkeys_b, double *jpart,
-                          double *objective, uint32_t *err, cudaStream_t st);
+                          double *objective, uint32_t *err, double *sums_out,
+                          cudaStream_t st);
+cudaError_t launch_finalize_shards(const double *sums, const int64_t *cnts, const double *objs,
+                                   int W, int K, int d, const float *C_old, float *C_new,
+                                   int64_t *counts, double *objective, cudaStream_t st);
 
 int device_sm_count();
 

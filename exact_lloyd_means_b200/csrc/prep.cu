@@ -234,7 +234,7 @@ cudaError_t launch_prep_centroids(const float *C, int K, int d, int64_t Kp, int6
                                   fk_dtype dtype, uint16_t *planes, float *cn, float *cused,
                                   uint16_t *caug, cudaStream_t st) {
     prep_centroids_kernel<<<grid_for_warps(Kp, 256), 256, 0, st>>>(
-        C, K, d, Kp, dp, dtype == FK_F32 ? 1 : 0, planes, cn, cused, caug);
+        C, K, d, Kp, dp, dtype == FK_BF16 ? 0 : 1, planes, cn, cused, caug);
     note_launch();
     return cudaGetLastError();
 }

@@ -46,6 +46,19 @@ __device__ __forceinline__ void store_mean(float *C_new, int64_t k, int d, int c
     *reinterpret_cast<float4 *>(C_new + k * d + col) = o;
 }
 
+// A finished cluster: its mean into C_new (fp32), or, when sums_out is given (a shard of a
+// data-parallel run), its fp64 sum into sums_out for a later combine across shards.
+__device__ __forceinline__ void store_done(float *C_new, double *sums_out, int64_t k, int d,
+                                          int col, const double (&acc)[4], double cnt) {
+    if (sums_out) {
+        double2 *q = reinterpret_cast<double2 *>(sums_out + k * d + col);
+        q[0] = make_double2(acc[0], acc[1]);
+        q[1] = make_double2(acc[2], acc[3]);
+    } else {
+        store_mean(C_new, k, d, col, acc, cnt);
+    }
+}
+
 __device__ __forceinline__ void store_piece(double *dst, const double (&acc)[4]) {
     double2 *q = reinterpret_cast<double2 *>(dst);
     q[0] = make_double2(acc[0], acc[1]);
@@ -101,8 +114,9 @@ __global__ void __launch_bounds__(kRowWarps * 32, 3)
                     int dcov, const int32_t *__restrict__ skeys,
                     const int32_t *__restrict__ perm, const int32_t *__restrict__ offsets,
                     const float *__restrict__ C_used, float *__restrict__ C_new,
-                    double *__restrict__ pieces, int32_t *__restrict__ pkeys,
-                    double *__restrict__ jpart, uint32_t *__restrict__ err) {
+                    double *__restrict__ sums_out, double *__restrict__ pieces,
+                    int32_t *__restrict__ pkeys, double *__restrict__ jpart,
+                    uint32_t *__restrict__ err) {
     using RV = RowVec<BF16>;
     constexpr int B = RV::kBatch;
     constexpr int SL = RV::kSlice;
@@ -158,7 +172,7 @@ __global__ void __launch_bounds__(kRowWarps * 32, 3)
     auto flush = [&](int k) {
         const int64_t lo = offsets[k], hi = offsets[k + 1];
         if (lo >= p0 && hi <= p1) {
-            if (colv) store_mean(C_new, k, d, col, acc, static_cast<double>(hi - lo));
+            if (colv) store_done(C_new, sums_out, k, d, col, acc, static_cast<double>(hi - lo));
         } else {
             const int slot = (k == first) ? 0 : 1;
             if (slot == 1) slot1 = k;
@@ -303,8 +317,8 @@ __global__ void __launch_bounds__(kUpdWarps * 32, 2)
                     int dcov, const int32_t *__restrict__ skeys,
                     const int32_t *__restrict__ perm, const int32_t *__restrict__ offsets,
                     const float *__restrict__ C_used, float *__restrict__ C_new,
-                    double *__restrict__ pieces, int32_t *__restrict__ pkeys,
-                    double *__restrict__ jpart) {
+                    double *__restrict__ sums_out, double *__restrict__ pieces,
+                    int32_t *__restrict__ pkeys, double *__restrict__ jpart) {
     using RV = RegRowVec<BF16>;
     using V = typename RV::T;
     constexpr int B = RV::kBatch;
@@ -337,7 +351,7 @@ __global__ void __launch_bounds__(kUpdWarps * 32, 2)
     auto flush = [&](int k) {
         const int64_t lo = offsets[k], hi = offsets[k + 1];
         if (lo >= p0 && hi <= p1) {
-            if (colv) store_mean(C_new, k, d, col, acc, static_cast<double>(hi - lo));
+            if (colv) store_done(C_new, sums_out, k, d, col, acc, static_cast<double>(hi - lo));
         } else {
             const int slot = (k == first) ? 0 : 1;
             if (slot == 1) slot1 = k;
@@ -447,7 +461,8 @@ __global__ void __launch_bounds__(kUpdWarps * 32)
     seg_pieces_kernel(const double *__restrict__ pin, const int32_t *__restrict__ kin,
                       int64_t nslots_in, double *__restrict__ pout,
                       int32_t *__restrict__ kout, int64_t nunits, int64_t span, int d,
-                      int dcov, const int32_t *__restrict__ offsets, float *__restrict__ C_new) {
+                      int dcov, const int32_t *__restrict__ offsets, float *__restrict__ C_new,
+                      double *__restrict__ sums_out) {
     constexpr int S = 2 * kGroup;
     constexpr int B = 8;
     __shared__ int32_t s_key[kUpdWarps][S];
@@ -472,7 +487,7 @@ __global__ void __launch_bounds__(kUpdWarps * 32)
         const bool done = (lo / span) == ((hi - 1) / span);
         if (k == first) first_done = done;
         if (done) {
-            if (col < d) store_mean(C_new, k, d, col, acc, static_cast<double>(hi - lo));
+            if (col < d) store_done(C_new, sums_out, k, d, col, acc, static_cast<double>(hi - lo));
         } else {
             const int slot = (k == first) ? 0 : 1;
             if (slot == 1) slot1 = k;
@@ -519,18 +534,57 @@ __global__ void __launch_bounds__(kUpdWarps * 32)
     }
 }
 
-// counts[k] = offsets[k+1] - offsets[k]; an empty cluster keeps C_old bit for bit.
+// counts[k] = offsets[k+1] - offsets[k]; an empty cluster keeps C_old bit for bit (or, for
+// a shard's partial sums, gets a zero sum).
 __global__ void finalize_kernel(const int32_t *__restrict__ offsets, int K, int d,
                                 const float *__restrict__ C_old, float *__restrict__ C_new,
-                                int32_t *__restrict__ counts) {
+                                int32_t *__restrict__ counts, double *__restrict__ sums_out) {
     const int lane = threadIdx.x & 31;
     const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
     const int64_t nw = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
     for (int64_t k = warp; k < K; k += nw) {
         const int32_t c = offsets[k + 1] - offsets[k];
         if (lane == 0 && counts) counts[k] = c;
-        if (c == 0)
-            for (int j = lane; j < d; j += 32) C_new[k * d + j] = C_old[k * d + j];
+        if (c == 0) {
+            if (sums_out)
+                for (int j = lane; j < d; j += 32) sums_out[k * d + j] = 0.0;
+            else
+                for (int j = lane; j < d; j += 32) C_new[k * d + j] = C_old[k * d + j];
+        }
+    }
+}
+
+// Combine W shards of a data-parallel iteration, in shard order: c_k = (sum_w S_wk) /
+// (sum_w n_wk) in fp64, rounded once to fp32, or C_old[k] bit for bit when no shard holds
+// a point of cluster k; counts[k] = sum_w n_wk; *objective = sum_w J_w (shard order).
+__global__ void finalize_shards_kernel(const double *__restrict__ sums,
+                                       const int64_t *__restrict__ cnts,
+                                       const double *__restrict__ objs, int W, int K, int d,
+                                       const float *__restrict__ C_old, float *__restrict__ C_new,
+                                       int64_t *__restrict__ counts,
+                                       double *__restrict__ objective) {
+    const int lane = threadIdx.x & 31;
+    const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+    const int64_t nw = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+    if (warp == 0 && lane == 0 && objective) {
+        double j = 0.0;
+        for (int w = 0; w < W; ++w) j += objs[w];
+        *objective = j;
+    }
+    const int64_t KD = static_cast<int64_t>(K) * d;
+    for (int64_t k = warp; k < K; k += nw) {
+        int64_t c = 0;
+        for (int w = 0; w < W; ++w) c += cnts[w * static_cast<int64_t>(K) + k];
+        if (lane == 0 && counts) counts[k] = c;
+        for (int j = lane; j < d; j += 32) {
+            if (c == 0) {
+                C_new[k * d + j] = C_old[k * d + j];
+            } else {
+                double acc = 0.0;
+                for (int w = 0; w < W; ++w) acc += sums[w * KD + k * d + j];
+                C_new[k * d + j] = static_cast<float>(acc / static_cast<double>(c));
+            }
+        }
     }
 }
 
@@ -551,7 +605,8 @@ __global__ void __launch_bounds__(1024)
 
 cudaError_t run_levels(const void *X, bool bf16, int64_t N, int d, const UpdPlan &up,
                        const int32_t *skeys, const int32_t *perm, const int32_t *offsets,
-                       const float *C_used, float *C_new, double *pa, int32_t *ka,
+                       const float *C_used, float *C_new, double *sums_out, double *pa,
+                       int32_t *ka,
                        double *pb, int32_t *kb, double *jpart, uint32_t *err,
                        cudaStream_t st) {
     static bool attr = false;
@@ -568,12 +623,12 @@ cudaError_t run_levels(const void *X, bool bf16, int64_t N, int d, const UpdPlan
         seg_rows_regs_kernel<true><<<dim3(static_cast<unsigned>(ceil_div(up.nwarps, kUpdWarps)),
                                           up.ncolblk),
                                      dim3(kUpdWarps * 32), 0, st>>>(
-            X, N, d, up.rows, up.nwarps, up.dcov, skeys, perm, offsets, C_used, C_new, pa, ka,
-            jpart);
+            X, N, d, up.rows, up.nwarps, up.dcov, skeys, perm, offsets, C_used, C_new, sums_out,
+            pa, ka, jpart);
     else
         seg_rows_kernel<false><<<rgrid, rblock, kRowSmem, st>>>(
-            X, N, d, up.rows, up.nwarps, up.dcov, skeys, perm, offsets, C_used, C_new, pa, ka,
-            jpart, err);
+            X, N, d, up.rows, up.nwarps, up.dcov, skeys, perm, offsets, C_used, C_new, sums_out,
+            pa, ka, jpart, err);
     note_launch();
     const dim3 block(kUpdWarps * 32);
     int64_t units = up.nwarps;
@@ -585,7 +640,7 @@ cudaError_t run_levels(const void *X, bool bf16, int64_t N, int d, const UpdPlan
         span *= kGroup;
         dim3 g2(static_cast<unsigned>(ceil_div(nunits, kUpdWarps)), up.ncolblk);
         seg_pieces_kernel<<<g2, block, 0, st>>>(pin, kin, units * 2, pout, kout, nunits, span, d,
-                                                up.dcov, offsets, C_new);
+                                                up.dcov, offsets, C_new, sums_out);
         note_launch();
         units = nunits;
         double *tp = pin;
@@ -605,21 +660,34 @@ cudaError_t launch_update(const void *X, fk_dtype dtype, int64_t N, int d, int K
                           const int32_t *offsets, const float *C_old, const float *C_used,
                           float *C_new, int32_t *counts, double *pieces_a, int32_t *pkeys_a,
                           double *pieces_b, int32_t *pkeys_b, double *jpart,
-                          double *objective, uint32_t *err, cudaStream_t st) {
+                          double *objective, uint32_t *err, double *sums_out,
+                          cudaStream_t st) {
     const bool bf16 = dtype == FK_BF16;
     cudaError_t e = run_levels(X, bf16, N, d, up, skeys, perm, offsets, C_used, C_new,
-                               pieces_a, pkeys_a, pieces_b, pkeys_b, jpart, err, st);
+                               sums_out, pieces_a, pkeys_a, pieces_b, pkeys_b, jpart, err, st);
     if (e != cudaSuccess) return e;
     int64_t fgrid = ceil_div(K, 8);
     const int64_t cap = static_cast<int64_t>(device_sm_count()) * 16;
     if (fgrid > cap) fgrid = cap;
     finalize_kernel<<<static_cast<unsigned>(fgrid), 256, 0, st>>>(offsets, K, d, C_old, C_new,
-                                                                   counts);
+                                                                   counts, sums_out);
     note_launch();
     if (objective) {
         objective_kernel<<<1, 1024, 0, st>>>(jpart, up.nwarps * up.ncolblk, objective);
         note_launch();
     }
+    return cudaGetLastError();
+}
+
+cudaError_t launch_finalize_shards(const double *sums, const int64_t *cnts, const double *objs,
+                                   int W, int K, int d, const float *C_old, float *C_new,
+                                   int64_t *counts, double *objective, cudaStream_t st) {
+    int64_t g = ceil_div(K, 8);
+    const int64_t cap = static_cast<int64_t>(device_sm_count()) * 16;
+    if (g > cap) g = cap;
+    finalize_shards_kernel<<<static_cast<unsigned>(g < 1 ? 1 : g), 256, 0, st>>>(
+        sums, cnts, objs, W, K, d, C_old, C_new, counts, objective);
+    note_launch();
     return cudaGetLastError();
 }
 

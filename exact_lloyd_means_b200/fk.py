@@ -18,7 +18,7 @@ LIB_PATH = os.path.join(_HERE, "libfk.so")
 
 FK_OK, FK_ERR_INVALID_ARG, FK_ERR_UNSUPPORTED, FK_ERR_WORKSPACE = 0, 1, 2, 3
 FK_ERR_CUDA, FK_ERR_TIMEOUT, FK_ERR_DEVICE = 4, 5, 6
-FK_F32, FK_BF16 = 0, 1
+FK_F32, FK_BF16, FK_BF16X2 = 0, 1, 2
 FK_L2, FK_COSINE = 0, 1
 
 if not os.path.exists(LIB_PATH):
@@ -49,8 +49,10 @@ def _sig(name, args, res=ctypes.c_int):
 _lib.fk_status_string.argtypes = [ctypes.c_int]
 _lib.fk_status_string.restype = ctypes.c_char_p
 _sig("fk_version", [])
+_sig("fk_launch_count", [], ctypes.c_int64)
 _sig("fk_workspace_size", [_i64, _int, _int, _int, _int, ctypes.POINTER(_sz)])
 _sig("fk_normalize_rows", [_vp, _vp, _i64, _int, _vp])
+_sig("fk_split_points", [_vp, _i64, _int, _vp, _vp])
 _sig("fk_centroid_norms", [_vp, _int, _int, _int, _vp, _vp])
 _sig("fk_assign", [_vp, _int, _i64, _int, _vp, _int, _vp, _vp, _vp, _sz, _vp])
 _sig("fk_update", [_vp, _int, _i64, _int, _int, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
@@ -60,10 +62,15 @@ _sig("fk_lloyd", [_vp, _int, _i64, _int, _int, _int, _int, _vp, _vp, _vp, _vp,
 _sig("fk_get_device_error", [_vp, _sz, ctypes.POINTER(ctypes.c_int), _vp])
 _sig("fk_selftest_timeout", [_vp, _sz, ctypes.c_uint64, _vp])
 _sig("fk_assign_noalloc", [_vp, _int, _i64, _int, _vp, _int, _vp, _vp])
+_sig("fk_update_partial", [_vp, _int, _i64, _int, _int, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz,
+                           _vp])
+_sig("fk_finalize_shards", [_vp, _vp, _vp, _int, _int, _int, _vp, _vp, _vp, _vp, _vp])
 
 EXPORTED = ["fk_status_string", "fk_version", "fk_workspace_size", "fk_normalize_rows",
             "fk_centroid_norms", "fk_assign", "fk_update", "fk_lloyd",
-            "fk_get_device_error", "fk_selftest_timeout", "fk_assign_noalloc"]
+            "fk_get_device_error", "fk_selftest_timeout", "fk_assign_noalloc",
+            "fk_update_partial", "fk_finalize_shards", "fk_split_points",
+            "fk_launch_count"]
 
 # Bytes of the static device array fk_assign_noalloc takes its scratch from.
 NOALLOC_SCRATCH_BYTES = 8 << 20
@@ -86,6 +93,11 @@ def status_string(status: int) -> str:
 
 def version() -> int:
     return _lib.fk_version()
+
+
+def launch_count() -> int:
+    """Kernels libfk has launched from this host thread so far."""
+    return _lib.fk_launch_count()
 
 
 def _dtype_code(t: torch.Tensor) -> int:
@@ -162,11 +174,42 @@ def fk_centroid_norms(C: torch.Tensor, cn: torch.Tensor, dtype=torch.float32, st
            "fk_centroid_norms")
 
 
-def fk_assign(X: torch.Tensor, C: torch.Tensor, labels: torch.Tensor, ws: torch.Tensor,
+class SplitPoints:
+    """fp32 points already split into bf16 hi/lo planes by fk_split_points ([2, N, d_p]
+    bf16, d_p = d rounded up to 64).  fk_assign takes it in place of the fp32 tensor
+    (dtype FK_BF16X2) and skips its per-call split."""
+
+    def __init__(self, planes: torch.Tensor, N: int, d: int):
+        self.planes, self.N, self.d = planes, N, d
+
+    @property
+    def shape(self):
+        return (self.N, self.d)
+
+
+def fk_split_points(X: torch.Tensor, out: torch.Tensor | None = None,
+                    stream=None) -> SplitPoints:
+    """Split fp32 points into bf16 hi/lo planes once; `out` ([2, N, d_p] bf16) is
+    allocated when not given."""
+    N, d = X.shape
+    dp = (d + 63) // 64 * 64
+    if out is None:
+        out = torch.empty(2, N, dp, dtype=torch.bfloat16, device=X.device)
+    _check(_lib.fk_split_points(_dev(X, "X", torch.float32), N, d,
+                                _dev(out, "out", torch.bfloat16, (2, N, dp)),
+                                _stream(stream)), "fk_split_points")
+    return SplitPoints(out, N, d)
+
+
+def fk_assign(X, C: torch.Tensor, labels: torch.Tensor, ws: torch.Tensor,
               mind: torch.Tensor | None = None, stream=None):
     N, d = X.shape
     K = C.shape[0]
-    _check(_lib.fk_assign(_dev(X, "X"), _dtype_code(X), N, d,
+    if isinstance(X, SplitPoints):
+        xptr, code = _dev(X.planes, "X.planes", torch.bfloat16), FK_BF16X2
+    else:
+        xptr, code = _dev(X, "X"), _dtype_code(X)
+    _check(_lib.fk_assign(xptr, code, N, d,
                           _dev(C, "C", torch.float32, (K, d)), K,
                           _dev(labels, "labels", torch.int32, (N,)),
                           _opt(mind, "mind", torch.float32, (N,)),
@@ -236,3 +279,36 @@ def fk_assign_noalloc(X: torch.Tensor, C: torch.Tensor, labels: torch.Tensor, st
                                   _dev(C, "C", torch.float32, (K, d)), K,
                                   _dev(labels, "labels", torch.int32, (N,)), _stream(stream)),
            "fk_assign_noalloc")
+
+
+def fk_update_partial(X: torch.Tensor, labels: torch.Tensor, C_old: torch.Tensor,
+                      sums: torch.Tensor, counts: torch.Tensor, offsets: torch.Tensor,
+                      ws: torch.Tensor, objective: torch.Tensor | None = None, stream=None):
+    """One shard's fp64 per-cluster sums, counts, CSR offsets and objective."""
+    N, d = X.shape
+    K = C_old.shape[0]
+    _check(_lib.fk_update_partial(_dev(X, "X"), _dtype_code(X), N, d, K,
+                                  _dev(labels, "labels", torch.int32, (N,)),
+                                  _dev(C_old, "C_old", torch.float32, (K, d)),
+                                  _dev(sums, "sums", torch.float64, (K, d)),
+                                  _dev(counts, "counts", torch.int32, (K,)),
+                                  _dev(offsets, "offsets", torch.int32, (K + 1,)),
+                                  _opt(objective, "objective", torch.float64, (1,)),
+                                  _dev(ws, "ws", torch.uint8), ws.numel(), _stream(stream)),
+           "fk_update_partial")
+
+
+def fk_finalize_shards(sums: torch.Tensor, counts_w: torch.Tensor, C_old: torch.Tensor,
+                       C_new: torch.Tensor, objectives_w: torch.Tensor | None = None,
+                       counts: torch.Tensor | None = None,
+                       objective: torch.Tensor | None = None, stream=None):
+    """Combine W gathered shards ([W][K][d] sums, [W][K] int64 counts) in shard order."""
+    W, K, d = sums.shape
+    _check(_lib.fk_finalize_shards(_dev(sums, "sums", torch.float64),
+                                   _dev(counts_w, "counts_w", torch.int64, (W, K)),
+                                   _opt(objectives_w, "objectives_w", torch.float64, (W,)),
+                                   W, K, d, _dev(C_old, "C_old", torch.float32, (K, d)),
+                                   _dev(C_new, "C_new", torch.float32, (K, d)),
+                                   _opt(counts, "counts", torch.int64, (K,)),
+                                   _opt(objective, "objective", torch.float64, (1,)),
+                                   _stream(stream)), "fk_finalize_shards")

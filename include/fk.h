@@ -74,9 +74,11 @@ typedef enum fk_status {
 } fk_status;
 
 typedef enum fk_dtype {
-    FK_F32 = 0,  /* fp32 points; products emulated to fp32 accuracy with three bf16
-                    tensor-core products (hi*hi + lo*hi + hi*lo)                      */
-    FK_BF16 = 1  /* bf16 points; bf16 tensor-core products (exact), fp32 accumulation  */
+    FK_F32 = 0,   /* fp32 points; products emulated to fp32 accuracy with three bf16
+                     tensor-core products (hi*hi + lo*hi + hi*lo)                     */
+    FK_BF16 = 1,  /* bf16 points; bf16 tensor-core products (exact), fp32 accumulation */
+    FK_BF16X2 = 2 /* fp32 points given already split by fk_split_points: two bf16 planes
+                     [2][N][roundup(d,64)] (hi, then lo); fk_assign only             */
 } fk_dtype;
 
 typedef enum fk_metric {
@@ -102,6 +104,10 @@ FK_API const char *fk_status_string(fk_status s);
 /* Library ABI version (incremented on any signature change). */
 FK_API int fk_version(void);
 
+/* Number of kernels this library has launched from the calling host thread since it was
+ * loaded (every entry point counts its own launches).  Host-only; for accounting. */
+FK_API int64_t fk_launch_count(void);
+
 /* Bytes of workspace that fk_assign, fk_update and fk_lloyd need for this problem
  * (any of them; the largest need).  Host-only, synchronous.  `bytes` is a host pointer. */
 FK_API fk_status fk_workspace_size(int64_t N, int d, int K, fk_dtype dtype, fk_metric metric,
@@ -113,6 +119,14 @@ FK_API fk_status fk_workspace_size(int64_t N, int d, int K, fk_dtype dtype, fk_m
  * fp32.  fp32 only; X_out may equal X_in (in place).  N x d row-major. */
 FK_API fk_status fk_normalize_rows(const float *X_in, float *X_out, int64_t N, int d,
                             fk_stream_t stream);
+
+/* Split fp32 points once for repeated assignment (the first step of fk_assign for
+ * FK_F32): planes = [2][N][d_p] bf16 with d_p = roundup(d, 64), hi = RN_bf16(x), lo =
+ * RN_bf16(x - hi), zero padding.  `planes` (device, 16-byte aligned, 4*N*d_p bytes) can
+ * then be passed to fk_assign as X with dtype FK_BF16X2, skipping the per-call split.
+ * fp32 only (d % 4 == 0, X 16-byte aligned). */
+FK_API fk_status fk_split_points(const float *X, int64_t N, int d, void *planes,
+                                 fk_stream_t stream);
 
 /* Centroid norms: cn[k] = sum_j c_kj^2 over the values the tensor cores consume (the
  * fp32 centroids for FK_F32, their bf16 rounding for FK_BF16), accumulated in fp64 and
@@ -128,7 +142,9 @@ FK_API fk_status fk_centroid_norms(const float *C, int K, int d, fk_dtype dtype,
  * bf16).  labels: N int32.  The N x K distance matrix is never stored: a tcgen05 kernel
  * keeps one 128 x 256 fp32 tile in tensor memory and a running min/argmin per row.
  * For FK_F32 each call first splits X into bf16 hi/lo planes inside `ws` (one extra
- * pass over X; fk_lloyd does this once per call instead of once per iteration). */
+ * pass over X; fk_lloyd does this once per call instead of once per iteration); callers
+ * that assign the same points repeatedly split once with fk_split_points and pass the
+ * planes with FK_BF16X2. */
 FK_API fk_status fk_assign(const void *X, fk_dtype dtype, int64_t N, int d, const float *C,
                     int K, int32_t *labels, float *mind, void *ws, size_t ws_bytes,
                     fk_stream_t stream);
@@ -167,6 +183,29 @@ FK_API fk_status fk_lloyd(const void *X, fk_dtype dtype, int64_t N, int d, int K
                    fk_metric metric, int niter, float *C, int32_t *labels,
                    int32_t *counts, int32_t *offsets, double *objective_host,
                    fk_timing *timing, void *ws, size_t ws_bytes, fk_stream_t stream);
+
+/* Data-parallel Lloyd over shards of X (one call per shard, typically one per GPU; X
+ * rows split, centroids replicated).  Same steps as fk_update, but instead of centroids
+ * the shard's per-cluster sums are returned for a combine across shards:
+ *   sums      K x d fp64 (device): sum of the shard's points with label k (zeros when none)
+ *   counts    K int32: points of the shard per cluster; offsets: the shard's CSR (K+1)
+ *   objective fp64 (device, optional): sum over the shard of ||x_i - c_used[l_i]||^2
+ * The sums are accumulated in fp64 in the fixed order of fk_update. */
+FK_API fk_status fk_update_partial(const void *X, fk_dtype dtype, int64_t N, int d, int K,
+                                   const int32_t *labels, const float *C_old, double *sums,
+                                   int32_t *counts, int32_t *offsets, double *objective,
+                                   void *ws, size_t ws_bytes, fk_stream_t stream);
+
+/* Combine W shards gathered side by side (device arrays): sums [W][K][d] fp64, counts_w
+ * [W][K] int64, objectives_w [W] fp64 (may be NULL with objective NULL).  In shard order,
+ * in fp64: C_new[k] = (sum_w sums[w][k]) / (sum_w counts_w[w][k]) rounded once to fp32, or
+ * C_old[k] bit for bit when every count is 0; counts[k] (int64, optional) = sum_w counts;
+ * *objective (optional) = sum_w objectives_w[w].  The order is fixed, so every rank that
+ * runs it on the same gathered data gets the same bits. */
+FK_API fk_status fk_finalize_shards(const double *sums, const int64_t *counts_w,
+                                    const double *objectives_w, int W, int K, int d,
+                                    const float *C_old, float *C_new, int64_t *counts,
+                                    double *objective, fk_stream_t stream);
 
 /* Scratch held by fk_assign_noalloc: one static device array of this many bytes. */
 #define FK_NOALLOC_SCRATCH_BYTES (8u << 20)

@@ -91,3 +91,26 @@ def test_binding_rejects_cpu_tensors(fk):
     with pytest.raises(ValueError):
         fk.fk_assign(X, torch.zeros(2, 8), torch.zeros(10, dtype=torch.int32),
                      torch.zeros(256, dtype=torch.uint8))
+
+
+def test_pre_split_dtype_is_assign_only(fk):
+    lib = fk._lib
+    n32 = fk.fk_workspace_size(4096, 100, 64, fk.FK_F32, "l2")
+    nx2 = fk.fk_workspace_size(4096, 100, 64, fk.FK_BF16X2, "l2")
+    assert nx2 < n32  # no room for the planes of X: the caller holds them
+    with pytest.raises(fk.FkError) as e:
+        fk.fk_workspace_size(4096, 100, 64, fk.FK_BF16X2, "cosine")
+    assert e.value.status == fk.FK_ERR_UNSUPPORTED
+    big = 1 << 30
+    assert lib.fk_lloyd(256, fk.FK_BF16X2, 100, 8, 4, 0, 1, 256, 256, None, None, None, None,
+                        256, big, None) == fk.FK_ERR_UNSUPPORTED
+    assert lib.fk_update(256, fk.FK_BF16X2, 100, 8, 4, 256, 4096, 8192, 256, 256, None, None,
+                         256, big, None) == fk.FK_ERR_UNSUPPORTED
+    assert lib.fk_update_partial(256, fk.FK_BF16X2, 100, 8, 4, 256, 256, 256, 256, 256, None,
+                                 256, big, None) == fk.FK_ERR_UNSUPPORTED
+    # the pre-split form has no point norms, so no distances are returned
+    assert lib.fk_assign(256, fk.FK_BF16X2, 100, 8, 256, 4, 256, 512, 256, big, None) == \
+        fk.FK_ERR_UNSUPPORTED
+    assert lib.fk_split_points(None, 100, 8, 256, None) == fk.FK_ERR_INVALID_ARG
+    assert lib.fk_split_points(256, 100, 6, 256, None) == fk.FK_ERR_UNSUPPORTED
+    assert lib.fk_split_points(8, 100, 8, 256, None) == fk.FK_ERR_UNSUPPORTED

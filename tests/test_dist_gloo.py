@@ -1,0 +1,107 @@
+"""The data-parallel (N > 1 ranks) path on CPU: two gloo ranks, each holding half of the
+points, run exact_lloyd_means_b200.dist.lloyd_sharded with stand-in local steps (the fp64
+oracle for the assignment, per-cluster sums for the partial update, and a rank-order
+combine rounded once to fp32 like the GPU's).  The result must equal the single-process
+oracle Lloyd on all the points: the exchange (gather order, combine, counts, objective)
+is what is under test."""
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _data():
+    from synth import gaussian_mixture, init_indices
+    X, _, _ = gaussian_mixture(3001, 16, 7, centers="normal", sigma=0.4, seed=5)
+    C0 = X[init_indices(3001, 7, 5)].clone()
+    return X, C0
+
+
+def _stand_in_ops():
+    import oracle
+    from exact_lloyd_means_b200.dist import LocalOps
+
+    def assign(X, C):
+        lab, _, _ = oracle.assign(X.numpy(), C.numpy())
+        return torch.from_numpy(lab)
+
+    def partial(X, lab, C):
+        K, d = C.shape
+        Xd = X.double().numpy()
+        lab = lab.numpy()
+        sums = np.zeros((K, d))
+        for k in range(K):
+            sums[k] = Xd[lab == k].sum(axis=0)
+        cnt = np.bincount(lab, minlength=K).astype(np.int64)
+        obj = oracle.objective(Xd, C.double().numpy(), lab)
+        return (torch.from_numpy(sums), torch.from_numpy(cnt),
+                torch.tensor([obj], dtype=torch.float64))
+
+    def finalize(sums_w, counts_w, objs_w, C_old):
+        S = torch.zeros_like(sums_w[0])
+        n = torch.zeros_like(counts_w[0])
+        for w in range(sums_w.shape[0]):  # rank order
+            S += sums_w[w]
+            n += counts_w[w]
+        C_new = C_old.clone()
+        nz = n > 0
+        C_new[nz] = (S[nz] / n[nz].double()[:, None]).float()
+        return C_new, n, objs_w.sum().reshape(1)
+
+    return LocalOps(assign, partial, finalize)
+
+
+def _rank(rank, world, port, niter, out):
+    os.environ["OMP_NUM_THREADS"] = "1"
+    import sys
+    sys.path.insert(0, ROOT)
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank,
+                            world_size=world)
+    from exact_lloyd_means_b200.dist import lloyd_sharded
+    X, C0 = _data()
+    bounds = np.linspace(0, X.shape[0], world + 1).astype(int)
+    Xl = X[bounds[rank]:bounds[rank + 1]].contiguous()
+    C = C0.clone()
+    objs, counts = lloyd_sharded(Xl, C, niter, _stand_in_ops())
+    out.put((rank, C.numpy(), objs, counts.numpy()))
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2])
+def test_sharded_lloyd_equals_single_process_oracle(world):
+    import oracle
+    niter = 4
+    ctx = mp.get_context("spawn")
+    out = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank, args=(r, world, port, niter, out)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = [out.get(timeout=180) for _ in range(world)]
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    res.sort(key=lambda t: t[0])
+    X, C0 = _data()
+    ref = oracle.lloyd(X.numpy(), C0.numpy(), niter)
+    for rank, C, objs, counts in res:
+        # every rank holds the same centroids: the oracle's, up to the order of fp64 sums
+        scale = np.abs(ref["C_next"][-1]).max(axis=1, keepdims=True)
+        assert (np.abs(C - ref["C_next"][-1]) <= 1e-6 * scale).all()
+        for t in range(niter):
+            assert abs(objs[t] - ref["J"][t]) <= 1e-9 * ref["J"][t]
+        assert (counts == ref["counts"][-1]).all()
+    assert np.array_equal(res[0][1], res[1][1])  # bit-identical across ranks

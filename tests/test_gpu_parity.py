@@ -242,3 +242,98 @@ def test_device_error_paths_without_fault():
     assert m2.fk_get_device_error(ws) == m2.FK_ERR_DEVICE
     lab2, _ = gpu_assign(Xg, C0.to(DEV))  # still works
     assert (lab2 >= 0).all()
+
+
+def test_update_partial_and_shard_finalize_match_fk_update():
+    """Two shards through fk_update_partial + fk_finalize_shards give fk_update's result
+    on all the points (same fp64 sums, combined in shard order)."""
+    m = fk()
+    X, C0, comp = _mixture(30000, 128, 300, seed=21, centers="normal", sigma=0.3)
+    Xg = X.to(DEV)
+    lab = comp.to(DEV)
+    K, d = 300, 128
+    full = gpu_update(Xg, comp.numpy(), C0.to(DEV), want_perm=False)
+    sums_w = torch.empty(2, K, d, dtype=torch.float64, device=DEV)
+    cnt_w = torch.empty(2, K, dtype=torch.int64, device=DEV)
+    obj_w = torch.empty(2, dtype=torch.float64, device=DEV)
+    for w, (a, b) in enumerate([(0, 13001), (13001, 30000)]):
+        ws = m.workspace(b - a, d, K, torch.float32, "l2")
+        cnt = torch.empty(K, dtype=torch.int32, device=DEV)
+        off = torch.empty(K + 1, dtype=torch.int32, device=DEV)
+        obj = torch.empty(1, dtype=torch.float64, device=DEV)
+        m.fk_update_partial(Xg[a:b].contiguous(), lab[a:b].contiguous(), C0.to(DEV),
+                            sums_w[w], cnt, off, ws, objective=obj)
+        cnt_w[w] = cnt.to(torch.int64)
+        obj_w[w] = obj[0]
+    C_new = torch.empty(K, d, device=DEV)
+    counts = torch.empty(K, dtype=torch.int64, device=DEV)
+    objective = torch.empty(1, dtype=torch.float64, device=DEV)
+    m.fk_finalize_shards(sums_w, cnt_w, C0.to(DEV), C_new, objectives_w=obj_w, counts=counts,
+                         objective=objective)
+    assert (counts.cpu().numpy() == full["counts"]).all()
+    assert centroid_rel_err(C_new.cpu().numpy(), full["C_new"]) <= 1e-6
+    # The objective's per-row terms are fp32 and are summed in fp32 within a batch of at most
+    # 16 rows before going to fp64. Shard boundaries move those batches, so the two sums
+    # can differ by up to 16 fp32 roundings of the objective's size (16 * 2^-24 < 1e-6).
+    assert abs(objective.item() - full["J"]) <= 1e-6 * full["J"]
+
+
+def test_lloyd_sharded_one_rank_equals_fk_lloyd():
+    """The data-parallel loop on one NCCL rank reproduces fk_lloyd bit for bit."""
+    import os
+    import socket
+    import torch.distributed as dist
+    from exact_lloyd_means_b200.dist import gpu_ops, lloyd_sharded
+    m = fk()
+    X, C0, _ = _mixture(40000, 128, 200, seed=22, centers="normal", sigma=0.3)
+    Xg = X.to(DEV)
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{port}", rank=0,
+                            world_size=1)
+    try:
+        C1 = C0.to(DEV).clone()
+        objs1, counts1 = lloyd_sharded(Xg, C1, 4, gpu_ops(40000, 128, 200,
+                                                            torch.float32, DEV))
+    finally:
+        dist.destroy_process_group()
+    C2 = C0.to(DEV).clone()
+    labels = torch.empty(40000, dtype=torch.int32, device=DEV)
+    counts2 = torch.empty(200, dtype=torch.int32, device=DEV)
+    objs2, _ = m.fk_lloyd(Xg, C2, 4, labels, m.workspace(40000, 128, 200), counts=counts2)
+    assert torch.equal(C1, C2)
+    assert objs1 == objs2
+    assert torch.equal(counts1.cpu(), counts2.cpu().to(torch.int64))
+
+
+@pytest.mark.parametrize("N,d", [(1000, 64), (4097, 100), (300, 768)])
+def test_split_points_planes_are_rounded_hi_lo(N, d):
+    """fk_split_points: hi = RN_bf16(x), lo = RN_bf16(x - hi), zero padding to d_p = 64k,
+    compared with PyTorch's own round-to-nearest-even casts."""
+    m = fk()
+    g = torch.Generator().manual_seed(N + d)
+    X = torch.randn(N, d, generator=g) * torch.logspace(-3, 3, d)
+    sp = m.fk_split_points(X.to(DEV))
+    P = sp.planes.cpu()
+    dp = (d + 63) // 64 * 64
+    assert tuple(P.shape) == (2, N, dp)
+    hi = X.to(torch.bfloat16)
+    lo = (X - hi.float()).to(torch.bfloat16)
+    assert torch.equal(P[0, :, :d].view(torch.int16), hi.view(torch.int16))
+    assert torch.equal(P[1, :, :d].view(torch.int16), lo.view(torch.int16))
+    assert not P[:, :, d:].float().any()
+
+
+@pytest.mark.parametrize("N,d,K", [(20000, 128, 300), (5000, 768, 1000), (3001, 64, 37)])
+def test_assign_pre_split_points_equals_fp32_assign(N, d, K):
+    """fk_assign on fk_split_points planes (FK_BF16X2) gives the fp32 call's labels."""
+    m = fk()
+    X, C0, _ = _mixture(N, d, K, seed=N + K, centers="normal", sigma=0.3)
+    Xg, Cg = X.to(DEV), C0.to(DEV)
+    ws = m.workspace(N, d, K)
+    l1 = torch.empty(N, dtype=torch.int32, device=DEV)
+    l2 = torch.empty(N, dtype=torch.int32, device=DEV)
+    m.fk_assign(Xg, Cg, l1, ws)
+    m.fk_assign(m.fk_split_points(Xg), Cg, l2, ws)
+    assert torch.equal(l1, l2)
