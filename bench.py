@@ -48,6 +48,9 @@ def parse():
     p.add_argument("--n", type=int, default=None,
                    help="override N (smaller cases for profiling captures)")
     p.add_argument("--impl", default="fk", choices=["fk", "reference"])
+    p.add_argument("--dp", action="store_true",
+                   help="run the data-parallel loop (exact_lloyd_means_b200.dist) even on "
+                        "one rank")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=12.0)
@@ -220,7 +223,7 @@ def fk_arm(args, spec, rank, world, dist):
 
     dev = torch.device("cuda", torch.cuda.current_device())
     niter = args.niter or spec.niter
-    sharded = world > 1
+    sharded = world > 1 or args.dp
     # weak scaling: every rank holds spec.n points of its own (own seed); one k-means
     # problem over all world * spec.n points when sharded
     seed = spec.seed + rank
@@ -228,7 +231,7 @@ def fk_arm(args, spec, rank, world, dist):
                                weights=spec.weights, zipf_s=spec.zipf_s, dtype=spec.dtype,
                                seed=seed, device=dev)
     C0 = X[init_indices(spec.n, spec.k, seed, device=dev)].float().contiguous()
-    if sharded:
+    if world > 1:
         dist.broadcast(C0, src=0)  # replicated initial centroids: rank 0's choice
     C = torch.empty_like(C0)
     labels = torch.empty(spec.n, dtype=torch.int32, device=dev)
@@ -427,12 +430,21 @@ def main():
         return
     import torch
     dist = None
-    if world > 1:
+    if world > 1 or args.dp:
         import datetime
 
         import torch.distributed as tdist
+        # NCCL prints its version banner on stdout when NCCL_DEBUG=VERSION; the bench's
+        # stdout carries exactly one JSON line, so keep library banners off it
+        if os.environ.get("NCCL_DEBUG", "").upper() == "VERSION":
+            os.environ["NCCL_DEBUG"] = "WARN"
         local = int(os.environ.get("LOCAL_RANK", "0"))
         torch.cuda.set_device(local)
+        if world == 1:  # --dp on one process: a one-rank group
+            os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+            os.environ.setdefault("MASTER_PORT", "29517")
+            os.environ.setdefault("RANK", "0")
+            os.environ.setdefault("WORLD_SIZE", "1")
         tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=180))
         dist = tdist
     fk_arm(args, spec, rank, world, dist)

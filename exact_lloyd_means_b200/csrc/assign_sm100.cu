@@ -679,8 +679,7 @@ __global__ void __launch_bounds__(PairCfg<NP, RES>::kThreads, 1)
                     for (int nt = 0; nt < ntiles && ok; ++nt, ++titer) {
                         const uint32_t acc = titer & 1u;
                         const uint32_t aphase = (titer >> 1) & 1u;
-                        if (!ptx::mbar_wait_cluster(&tempty[acc], aphase ^ 1u, abort_flag,
-                                                    wait_ns)) {
+                        if (!ptx::mbar_wait(&tempty[acc], aphase ^ 1u, abort_flag, wait_ns)) {
                             raise_timeout(abort_flag, err);
                             ok = false;
                             break;

@@ -77,34 +77,6 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity,
     }
 }
 
-// Bounded wait with cluster-scope acquire (for barriers that receive arrivals from the
-// peer CTA of a cluster pair).
-__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t *bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-
-__device__ __forceinline__ bool mbar_wait_cluster(uint64_t *bar, uint32_t parity,
-                                                  const volatile uint32_t *abort,
-                                                  uint64_t limit_ns) {
-    if (mbar_try_wait_cluster(bar, parity)) return true;
-    const uint64_t t0 = globaltimer_ns();
-    for (uint32_t it = 1;; ++it) {
-        if (mbar_try_wait_cluster(bar, parity)) return true;
-        if ((it & 15u) == 0) {
-            if (abort != nullptr && *abort) return false;
-            if (globaltimer_ns() - t0 > limit_ns) return false;
-        }
-    }
-}
-
 // ---------------------------------------------------------------- clusters (CTA pairs)
 
 __device__ __forceinline__ uint32_t cluster_ctarank() {
@@ -121,11 +93,14 @@ __device__ __forceinline__ uint32_t mapa_shared(uint32_t saddr, uint32_t rank) {
     return r;
 }
 
-// Arrive (release at cluster scope) on an mbarrier given by its shared::cluster address,
-// possibly in the peer CTA.
+// Arrive on an mbarrier given by its shared::cluster address, possibly in the peer CTA,
+// with the default (release, CTA-scope) semantics.  Used to hand a consumed accumulator
+// back to the MMA issuer: the arriving thread's tensor-memory loads have already completed
+// (tcgen05.wait::ld) and are ordered by tcgen05.fence::before_thread_sync, and it has no
+// memory writes the waiter needs, so no cluster-scope release (a full memory barrier on
+// every arrive) is required.
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
-    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(
-                     cluster_addr)
+    asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
                  : "memory");
 }
 
