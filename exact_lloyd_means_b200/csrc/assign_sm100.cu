@@ -95,6 +95,28 @@ __device__ __forceinline__ void init_aug_a(uint8_t *aaug, int r) {
 }
 
 // Minimum of 64 values with three-input mins: 21 + 7 + 3 + 1 instructions.
+// Width of the screening window for one row: twice a bound E on |v~ - v|, where
+// v = ||c||^2 - 2 x.c is exact and v~ is what the single-product pass accumulates from
+// bf16 x~ = RN(x) and c~ = RN(c) (each within a relative 2^-8 of its value; u = 2^-8):
+//   operand rounding   |sum x~c~ - sum xc| <= (2u + u^2) sum |x_j||c_j| <= (2u + u^2)|x||c|,
+//                      doubled by the factor -2;
+//   accumulation       each of the dp/16 + 1 MMA steps adds 16 exact products to the fp32
+//                      accumulator; assume up to 17 units of 2^-23 of the largest partial
+//                      value, which is at most ||c||^2 + 2|x||c| (with margin);
+//   norm               ||c||^2 rounded once to fp32 (2^-24 relative).
+// If k* is the true argmin, v~(k*) <= v(k*) + E <= v(k) + E <= v~(k) + 2E for every k, so
+// k* lies within 2E of the screened minimum.  ||c|| is bounded by cmax = max_k ||c_k||.
+// The result carries a 1% margin for the rounding of this expression itself.
+__device__ __forceinline__ float screen_window(float xnorm2, float cmax2, int dp) {
+    const float xn = sqrtf(xnorm2), cm = sqrtf(cmax2);
+    const float u = 0.00390625f;
+    const float prod = 2.f * (2.f * u + u * u) * xn * cm;
+    const float accum = static_cast<float>(dp / 16 + 1) * 17.f * 1.1920929e-7f *
+                        (cmax2 + 2.f * xn * cm) * 1.01f;
+    const float norm = 5.9604645e-8f * cmax2;
+    return 2.f * (prod + accum + norm) * 1.01f;
+}
+
 __device__ __forceinline__ float min64(const float (&v)[64]) {
     float t[22];
 #pragma unroll
@@ -109,6 +131,38 @@ __device__ __forceinline__ float min64(const float (&v)[64]) {
     return ptx::fmin3(a, b, fminf(u[6], u[7]));
 }
 
+// Screening helpers.  The smallest published running minimum of this row's column groups
+// in the current row block (entries [g * kBM] for g = 0..3, tagged with the row block),
+// and `own` (this group's own minimum).
+__device__ __forceinline__ float scr_global_min(const uint64_t *pub_row, uint32_t tag,
+                                                float own) {
+    float gm = own;
+#pragma unroll
+    for (int o = 0; o < 4; ++o) {
+        const uint64_t p = ptx::ld_relaxed_u64(pub_row + o * kBM);
+        if (static_cast<uint32_t>(p >> 32) == tag)
+            gm = fminf(gm, __uint_as_float(static_cast<uint32_t>(p)));
+    }
+    return gm;
+}
+
+// Append the columns base + bit of `mask` to the (up to four) candidates c0..c3.
+__device__ __forceinline__ void scr_emit(uint64_t mask, int base, int &cnt, int &c0, int &c1,
+                                         int &c2, int &c3, bool &over) {
+    for (; mask != 0ull && !over; mask &= mask - 1ull) {
+        const int col = base + __ffsll(static_cast<long long>(mask)) - 1;
+        if (cnt < 4) {
+            c3 = c2;
+            c2 = c1;
+            c1 = c0;
+            c0 = col;
+            ++cnt;
+        } else {
+            over = true;
+        }
+    }
+}
+
 template <int NP, bool RES>
 __global__ void __launch_bounds__(AsgCfg<NP, RES>::kThreads, 1)
     assign_kernel(const __grid_constant__ CUtensorMap tmA0,
@@ -118,9 +172,14 @@ __global__ void __launch_bounds__(AsgCfg<NP, RES>::kThreads, 1)
                   const __grid_constant__ CUtensorMap tmC,
                   int64_t N, int nkc, int ntiles, int64_t nmb, int32_t *__restrict__ labels,
                   float *__restrict__ best_out, const float *__restrict__ xnorm,
-                  float *__restrict__ mind, uint32_t *__restrict__ err, uint64_t wait_ns) {
+                  float *__restrict__ mind, uint32_t *__restrict__ err, uint64_t wait_ns,
+                  const uint32_t *__restrict__ n_dev) {
     using Cfg = AsgCfg<NP, RES>;
     constexpr int S = Cfg::kStages;
+    if (n_dev != nullptr) {  // row count written on the device by an earlier kernel
+        N = *n_dev;
+        nmb = (N + kBM - 1) / kBM;
+    }
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -486,7 +545,7 @@ struct PairCfg {
     static_assert(kSmemBytes <= 232448, "shared memory");
 };
 
-template <int NP, bool RES>
+template <int NP, bool RES, bool SCR>
 __global__ void __launch_bounds__(PairCfg<NP, RES>::kThreads, 1)
     assign_pair_kernel(const __grid_constant__ CUtensorMap tmA0,
                        const __grid_constant__ CUtensorMap tmA1,
@@ -496,10 +555,18 @@ __global__ void __launch_bounds__(PairCfg<NP, RES>::kThreads, 1)
                        int64_t N, int nkc, int ntiles, int64_t nmb,
                        int32_t *__restrict__ labels, float *__restrict__ best_out,
                        const float *__restrict__ xnorm, float *__restrict__ mind,
-                       uint32_t *__restrict__ err, uint64_t wait_ns) {
+                       uint32_t *__restrict__ err, uint64_t wait_ns,
+                       const uint32_t *__restrict__ n_dev, int32_t *__restrict__ cand,
+                       const float *__restrict__ cmax2) {
+    static_assert(!SCR || NP == 1, "screening runs the single-product form");
+    static_assert(PairCfg<NP, RES>::kEpiGroups == 4, "scr_global_min reads four groups");
     using Cfg = PairCfg<NP, RES>;
     constexpr int S = Cfg::kStages;
     constexpr int EC = Cfg::kEpiCols;
+    if (n_dev != nullptr) {  // row count written on the device by an earlier kernel
+        N = *n_dev;
+        nmb = (N + 2 * kBM - 1) / (2 * kBM);
+    }
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -564,6 +631,8 @@ __global__ void __launch_bounds__(PairCfg<NP, RES>::kThreads, 1)
         init_aug_a(aaug, (warp & 3) * 32 + lane);
         ptx::fence_proxy_async_smem();  // visible to the tensor core (async proxy)
     }
+    if (SCR && warp >= 2)  // published minima start with a tag no row block carries
+        reinterpret_cast<uint64_t *>(red_v)[(warp - 2) * 32 + lane] = ~0ull;
     ptx::tc_fence_before();
     __syncthreads();
     ptx::cluster_sync();  // barriers of both CTAs initialised, tensor memory allocated
@@ -748,11 +817,42 @@ __global__ void __launch_bounds__(PairCfg<NP, RES>::kThreads, 1)
         const int g = (warp - 2) >> 2;
         const int q = warp & 3;
         const int r = q * 32 + lane;
+        const float cm2 = SCR ? *cmax2 : 0.f;
+        // screening: each group publishes its running minimum per row, tagged with the row
+        // block, so every group can window against the minimum over all 256 columns of
+        // the tiles seen so far.  A value read while its writer is a tile ahead or behind
+        // is still some group's minimum over real columns of this row, so the window it
+        // gives can only be wider than the exact one (never narrower).
+        uint64_t *pub = reinterpret_cast<uint64_t *>(red_v);  // [kEpiGroups][kBM]
         uint32_t titer = 0, mbi = 0;
         bool ok = true;
+        // ||x||^2 of this thread's row in the next row block, loaded a block ahead so the
+        // window is ready when the block starts
+        float xn_next = 0.f;
+        if (SCR) {
+            const int64_t row0 = pair * 2 * kBM + static_cast<int64_t>(rank) * kBM + r;
+            if (pair < nmb && row0 < N) xn_next = xnorm[row0];
+        }
         for (int64_t mb = pair; mb < nmb && ok; mb += npairs, ++mbi) {
+            const int64_t row = mb * 2 * kBM + static_cast<int64_t>(rank) * kBM + r;
             float best = __int_as_float(0x7f800000);
             int bestk = 0;
+            // screening state: the window width; up to three kept tiles, each with its
+            // minimum over this group's columns (+inf = free slot), its index and the mask
+            // of its columns inside the window when it was kept; and the smallest minimum
+            // of a tile dropped for lack of room (the row overflows if that tile is still
+            // inside the final window)
+            float W = 0.f;
+            float em0 = __int_as_float(0x7f800000), em1 = em0, em2 = em0, lost = em0;
+            int et0 = 0, et1 = 0, et2 = 0;
+            uint32_t el0 = 0, eh0 = 0, el1 = 0, eh1 = 0, el2 = 0, eh2 = 0;
+            bool over = false;
+            const uint32_t tag = static_cast<uint32_t>(mb);
+            if (SCR) {
+                W = screen_window(xn_next, cm2, nkc * kBK);
+                const int64_t rn = row + npairs * 2 * kBM;
+                xn_next = (mb + npairs < nmb && rn < N) ? xnorm[rn] : 0.f;
+            }
             for (int nt = 0; nt < ntiles; ++nt, ++titer) {
                 const uint32_t acc = titer & 1u;
                 const uint32_t aphase = (titer >> 1) & 1u;
@@ -772,7 +872,49 @@ __global__ void __launch_bounds__(PairCfg<NP, RES>::kThreads, 1)
                 __syncwarp();
                 if (lane == 0) ptx::mbar_arrive_cluster(tempty_c + acc * 8);  // consumed
                 const float m = min64(v);
-                if (m < best) {
+                if (SCR) {
+                    float gm = scr_global_min(pub + r, tag, best);
+                    if (m <= gm + W) {  // this tile has columns inside the window
+                        if (m < best) {
+                            best = m;
+                            ptx::st_relaxed_u64(pub + g * kBM + r,
+                                                (static_cast<uint64_t>(tag) << 32) |
+                                                    __float_as_uint(m));
+                        }
+                        gm = fminf(gm, m);
+                        const float T = fminf(gm + W, kScreenMax);
+                        uint32_t lo = 0u, hi = 0u;
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) {
+                            lo |= (v[j] <= T ? 1u : 0u) << j;
+                            hi |= (v[32 + j] <= T ? 1u : 0u) << j;
+                        }
+                        const float inf = __int_as_float(0x7f800000);
+                        if (em0 > T) em0 = inf;  // kept tiles that left the window for good
+                        if (em1 > T) em1 = inf;
+                        if (em2 > T) em2 = inf;
+                        if ((lo | hi) != 0u) {
+                            if (em0 == inf) {
+                                em0 = m; et0 = nt; el0 = lo; eh0 = hi;
+                            } else if (em1 == inf) {
+                                em1 = m; et1 = nt; el1 = lo; eh1 = hi;
+                            } else if (em2 == inf) {
+                                em2 = m; et2 = nt; el2 = lo; eh2 = hi;
+                            } else if (m >= em0 && m >= em1 && m >= em2) {
+                                lost = fminf(lost, m);  // keep the three smallest minima
+                            } else if (em0 >= em1 && em0 >= em2) {
+                                lost = fminf(lost, em0);
+                                em0 = m; et0 = nt; el0 = lo; eh0 = hi;
+                            } else if (em1 >= em2) {
+                                lost = fminf(lost, em1);
+                                em1 = m; et1 = nt; el1 = lo; eh1 = hi;
+                            } else {
+                                lost = fminf(lost, em2);
+                                em2 = m; et2 = nt; el2 = lo; eh2 = hi;
+                            }
+                        }
+                    }
+                } else if (m < best) {
                     int idx = 0;
 #pragma unroll
                     for (int j = EC - 1; j >= 0; --j)
@@ -782,6 +924,29 @@ __global__ void __launch_bounds__(PairCfg<NP, RES>::kThreads, 1)
                 }
             }
             if (!ok) break;
+            if (SCR) {
+                // candidates of this row among this group's columns: every column of a kept
+                // tile whose minimum is still inside the final window (up to four)
+                const float T = fminf(scr_global_min(pub + r, tag, best) + W, kScreenMax);
+                if (lost <= T) over = true;  // a dropped tile may hold a candidate
+                int32_t c0 = -1, c1 = -1, c2 = -1, c3 = -1;
+                int cnt = 0;
+                if (em0 <= T)
+                    scr_emit((static_cast<uint64_t>(eh0) << 32) | el0, et0 * kBN + g * EC, cnt,
+                             c0, c1, c2, c3, over);
+                if (em1 <= T)
+                    scr_emit((static_cast<uint64_t>(eh1) << 32) | el1, et1 * kBN + g * EC, cnt,
+                             c0, c1, c2, c3, over);
+                if (em2 <= T)
+                    scr_emit((static_cast<uint64_t>(eh2) << 32) | el2, et2 * kBN + g * EC, cnt,
+                             c0, c1, c2, c3, over);
+                if (row < N) {
+                    const int4 o = over ? make_int4(kCandOverflow, -1, -1, -1)
+                                        : make_int4(c0, c1, c2, c3);
+                    *reinterpret_cast<int4 *>(cand + row * kCandPerRow + g * 4) = o;
+                }
+                continue;
+            }
             const uint32_t slot = mbi & 1u;
             const uint32_t spar = (mbi >> 1) & 1u;
             if (g > 0) {
@@ -809,7 +974,6 @@ __global__ void __launch_bounds__(PairCfg<NP, RES>::kThreads, 1)
                     }
                 }
                 ptx::mbar_arrive(&redempty[slot]);
-                const int64_t row = mb * 2 * kBM + static_cast<int64_t>(rank) * kBM + r;
                 if (row < N) {
                     labels[row] = bestk;
                     if (best_out) best_out[row] = best;
@@ -887,12 +1051,12 @@ cudaError_t launch_assign_cfg(const AssignArgs &a, const CUtensorMap (&tA)[2],
     assign_kernel<NP, RES><<<grid, Cfg::kThreads, Cfg::kSmemBytes, st>>>(
         tA[0], tA[1], tB[0], tB[1], tC, a.N, static_cast<int>(a.dp / kBK),
         static_cast<int>(a.Kp / kBN), nmb, a.labels, a.best, a.xnorm, a.mind, a.err,
-        a.wait_ns);
+        a.wait_ns, a.n_dev);
     note_launch();
     return cudaGetLastError();
 }
 
-template <int NP, bool RES>
+template <int NP, bool RES, bool SCR>
 cudaError_t launch_assign_pair_cfg(const AssignArgs &a, const CUtensorMap (&tA)[2],
                                    const CUtensorMap (&tB)[2], const CUtensorMap &tC,
                                    int max_pairs, cudaStream_t st) {
@@ -911,24 +1075,24 @@ cudaError_t launch_assign_pair_cfg(const AssignArgs &a, const CUtensorMap (&tA)[
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, assign_pair_kernel<NP, RES>, tA[0], tA[1], tB[0],
-                                       tB[1], tC, a.N, static_cast<int>(a.dp / kBK),
-                                       static_cast<int>(a.Kp / kBN), nmb, a.labels, a.best,
-                                       a.xnorm, a.mind, a.err, a.wait_ns);
+    cudaError_t e = cudaLaunchKernelEx(
+        &cfg, assign_pair_kernel<NP, RES, SCR>, tA[0], tA[1], tB[0], tB[1], tC, a.N,
+        static_cast<int>(a.dp / kBK), static_cast<int>(a.Kp / kBN), nmb, a.labels, a.best,
+        a.xnorm, a.mind, a.err, a.wait_ns, a.n_dev, a.cand, a.cmax2);
     note_launch();
     return e;
 }
 
 // Largest number of CTA pairs of this configuration that can be resident at once (the
 // persistent grid must not exceed it, or part of it would wait for a second wave).
-template <int NP, bool RES>
+template <int NP, bool RES, bool SCR>
 int max_resident_pairs() {
     using Cfg = PairCfg<NP, RES>;
     static int cached[64] = {0};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
     if (cached[dev]) return cached[dev];
-    if (cudaFuncSetAttribute(assign_pair_kernel<NP, RES>,
+    if (cudaFuncSetAttribute(assign_pair_kernel<NP, RES, SCR>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                              Cfg::kSmemBytes) != cudaSuccess)
         return 0;
@@ -944,16 +1108,30 @@ int max_resident_pairs() {
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, assign_pair_kernel<NP, RES>, &cfg) != cudaSuccess)
+    if (cudaOccupancyMaxActiveClusters(&n, assign_pair_kernel<NP, RES, SCR>, &cfg) !=
+        cudaSuccess)
         n = 0;
     cached[dev] = n;
     return n;
 }
 
-template <int NP>
+// X block resident in shared memory when it fits (d <= 128) and, for the fp32 emulation
+// (one X buffer, so a short gap at each new block), when the sweep over the centroid tiles
+// is long enough to hide that gap.
+inline bool resident_x(int NP, int dp, int Kp) {
+    const int nkc = dp / kBK;
+    const int ntiles = Kp / kBN;
+    return nkc <= 2 && (NP == 1 || ntiles >= 16);
+}
+
+// CTA pairs (M = 256 per MMA) once there are enough 256-row blocks to fill the GPU.
+inline bool pair_rows(int64_t N) { return N >= int64_t(2 * kBM) * device_sm_count() / 2; }
+
+template <int NP, bool SCR>
 cudaError_t launch_assign_pair(const AssignArgs &a, cudaStream_t st, bool res, bool *done) {
     *done = false;
-    const int mp = res ? max_resident_pairs<NP, true>() : max_resident_pairs<NP, false>();
+    const int mp = res ? max_resident_pairs<NP, true, SCR>()
+                       : max_resident_pairs<NP, false, SCR>();
     if (mp <= 0) return cudaSuccess;  // pairs cannot be scheduled: use the single-CTA form
     CUtensorMap tA[2], tB[2];
     const uint16_t *ap = static_cast<const uint16_t *>(a.a_planes);
@@ -972,12 +1150,18 @@ cudaError_t launch_assign_pair(const AssignArgs &a, cudaStream_t st, bool res, b
     CUtensorMap tC;
     if (!make_tmap(&tC, a.caug, a.Kp, kAug, kAug, kBN / 2, kAug)) return cudaErrorInvalidValue;
     *done = true;
-    return res ? launch_assign_pair_cfg<NP, true>(a, tA, tB, tC, mp, st)
-               : launch_assign_pair_cfg<NP, false>(a, tA, tB, tC, mp, st);
+    return res ? launch_assign_pair_cfg<NP, true, SCR>(a, tA, tB, tC, mp, st)
+               : launch_assign_pair_cfg<NP, false, SCR>(a, tA, tB, tC, mp, st);
 }
 
 template <int NP>
 cudaError_t launch_assign_np(const AssignArgs &a, cudaStream_t st) {
+    const bool res = resident_x(NP, a.dp, a.Kp);
+    if (pair_rows(a.N)) {
+        bool done = false;
+        const cudaError_t e = launch_assign_pair<NP, false>(a, st, res, &done);
+        if (done || e != cudaSuccess) return e;
+    }
     CUtensorMap tA[2], tB[2];
     const uint16_t *ap = static_cast<const uint16_t *>(a.a_planes);
     const uint16_t *bp = static_cast<const uint16_t *>(a.b_planes);
@@ -992,18 +1176,6 @@ cudaError_t launch_assign_np(const AssignArgs &a, cudaStream_t st) {
         tA[1] = tA[0];
         tB[1] = tB[0];
     }
-    // X block resident in shared memory when it fits (d <= 128) and, for the fp32
-    // emulation (one X buffer, so a short gap at each new block), when the sweep over
-    // the centroid tiles is long enough to hide that gap.
-    const int nkc = a.dp / kBK;
-    const int ntiles = a.Kp / kBN;
-    const bool res = nkc <= 2 && (NP == 1 || ntiles >= 16);
-    // CTA pairs (M = 256 per MMA) once there are enough 256-row blocks to fill the GPU
-    if (a.N >= int64_t(2 * kBM) * device_sm_count() / 2) {
-        bool done = false;
-        const cudaError_t e = launch_assign_pair<NP>(a, st, res, &done);
-        if (done || e != cudaSuccess) return e;
-    }
     CUtensorMap tC;
     if (!make_tmap(&tC, a.caug, a.Kp, kAug, kAug, kBN, kAug)) return cudaErrorInvalidValue;
     if (res) return launch_assign_cfg<NP, true>(a, tA, tB, tC, st);
@@ -1014,7 +1186,21 @@ cudaError_t launch_assign_np(const AssignArgs &a, cudaStream_t st) {
 
 cudaError_t launch_assign(const AssignArgs &a, cudaStream_t st) {
     if (a.N <= 0) return cudaSuccess;
+    if (a.cand != nullptr) {  // the screening pass exists only in the CTA-pair form
+        if (a.a_nplanes != 1 || !assign_can_screen(a.N, a.dp, a.Kp))
+            return cudaErrorNotSupported;
+        bool done = false;
+        const cudaError_t e =
+            launch_assign_pair<1, true>(a, st, resident_x(1, a.dp, a.Kp), &done);
+        return e != cudaSuccess ? e : (done ? cudaSuccess : cudaErrorNotSupported);
+    }
     return a.a_nplanes == 2 ? launch_assign_np<2>(a, st) : launch_assign_np<1>(a, st);
+}
+
+bool assign_can_screen(int64_t N, int dp, int Kp) {
+    if (!pair_rows(N)) return false;
+    return resident_x(1, dp, Kp) ? max_resident_pairs<1, true, true>() > 0
+                                 : max_resident_pairs<1, false, true>() > 0;
 }
 
 }  // namespace fk

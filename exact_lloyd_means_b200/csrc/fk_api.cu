@@ -73,15 +73,21 @@ bool overlap(const void *a, size_t an, const void *b, size_t bn) {
     } while (0)
 
 // The operand X planes the assign kernel reads, prepared from the (possibly normalised)
-// points.  Returns the planes pointer, plane count and row stride.
+// points.  Returns the planes pointer, plane count and row stride.  `xnorm` receives
+// ||x||^2 per row when given; for pre-split points the norms already follow the planes and
+// *xnorm_ready points at them.
 fk_status prepare_x(const void *Xp, fk_dtype dtype, int64_t N, int d, const WsLayout &L,
                     void *ws, float *xnorm, cudaStream_t st, const void **planes,
-                    int *nplanes, int64_t *lda) {
+                    int *nplanes, int64_t *lda, const float **xnorm_ready = nullptr) {
     uint16_t *xs = ws_ptr<uint16_t>(ws, L.xs);
+    if (xnorm_ready) *xnorm_ready = xnorm;
     if (dtype == FK_BF16X2) {  // already split by fk_split_points
         *planes = Xp;
         *nplanes = 2;
         *lda = L.dp;
+        if (xnorm_ready)
+            *xnorm_ready = reinterpret_cast<const float *>(static_cast<const uint16_t *>(Xp) +
+                                                           2 * N * L.dp);
         return FK_OK;
     }
     if (dtype == FK_F32) {
@@ -106,9 +112,16 @@ fk_status prepare_x(const void *Xp, fk_dtype dtype, int64_t N, int d, const WsLa
     return FK_OK;
 }
 
+// Assignment from prepared planes.  Two-plane (fp32) problems large enough for the CTA-pair
+// kernel take the screened route (single product, exact re-ranking, three products for the
+// rows that need them); it needs ||x||^2 in `xnorm`, the centroids C (fp32, the values the
+// planes were made from) and, when available, the fp32 points X32 for the re-ranking.
 fk_status run_assign(const void *planes, int nplanes, int64_t lda, int64_t N, int d, int K,
                      const WsLayout &L, void *ws, int32_t *labels, const float *xnorm,
-                     float *mind, cudaStream_t st) {
+                     float *mind, cudaStream_t st, const float *X32 = nullptr,
+                     const float *C = nullptr, bool allow_screen = true,
+                     bool *screened = nullptr) {
+    if (screened) *screened = false;
     AssignArgs a{};
     a.a_planes = planes;
     a.a_nplanes = nplanes;
@@ -127,6 +140,20 @@ fk_status run_assign(const void *planes, int nplanes, int64_t lda, int64_t N, in
     a.mind = mind;
     a.err = ws_ptr<uint32_t>(ws, L.err);
     a.wait_ns = kDefaultWaitNs;
+    if (allow_screen && nplanes == 2 && L.dp >= kScreenMinD && C != nullptr &&
+        xnorm != nullptr && lda == L.dp && d % 4 == 0 && aligned(C, 16) &&
+        (X32 == nullptr || aligned(X32, 16)) && assign_can_screen(N, a.dp, a.Kp)) {
+        ScreenBufs sb;
+        sb.cand = ws_ptr<int32_t>(ws, L.cand);
+        sb.nfb = ws_ptr<uint32_t>(ws, L.nfb);
+        sb.fbrows = ws_ptr<int32_t>(ws, L.fbrows);
+        sb.fblab = ws_ptr<int32_t>(ws, L.fblab);
+        sb.xsfb = ws_ptr<uint16_t>(ws, L.xsfb);
+        sb.cmax2 = ws_ptr<float>(ws, L.cmax2);
+        FK_TRY_CUDA(launch_assign_screened(a, X32, C, sb, st));
+        if (screened) *screened = true;
+        return FK_OK;
+    }
     FK_TRY_CUDA(launch_assign(a, st));
     return FK_OK;
 }
@@ -228,7 +255,8 @@ fk_status fk_split_points(const float *X, int64_t N, int d, void *planes, fk_str
     if (s != FK_OK) return s;
     const int64_t dp = round_up(d, kBK);
     uint16_t *p = static_cast<uint16_t *>(planes);
-    FK_TRY_CUDA(launch_split_x(X, N, d, dp, p, p + N * dp, nullptr, stream));
+    float *norms = reinterpret_cast<float *>(p + 2 * N * dp);
+    FK_TRY_CUDA(launch_split_x(X, N, d, dp, p, p + N * dp, norms, stream));
     return FK_OK;
 }
 
@@ -246,7 +274,6 @@ fk_status fk_assign(const void *X, fk_dtype dtype, int64_t N, int d, const float
                     int32_t *labels, float *mind, void *ws, size_t ws_bytes,
                     fk_stream_t stream) {
     fk_status s = validate_shape(N, d, K, dtype, FK_L2, true);
-    if (s == FK_OK && dtype == FK_BF16X2 && mind) return FK_ERR_UNSUPPORTED;
     if (s != FK_OK) return s;
     if (!X || !C || !labels) return FK_ERR_INVALID_ARG;
     if (!aligned(X, 16) || !aligned(C, 4) || !aligned(labels, 4) || (mind && !aligned(mind, 4)))
@@ -258,13 +285,18 @@ fk_status fk_assign(const void *X, fk_dtype dtype, int64_t N, int d, const float
     FK_TRY_CUDA(launch_prep_centroids(C, K, d, L.Kp, L.dp, dtype, ws_ptr<uint16_t>(ws, L.cs),
                                       ws_ptr<float>(ws, L.cn), ws_ptr<float>(ws, L.cused),
                                       ws_ptr<uint16_t>(ws, L.caug), st));
-    float *xnorm = mind ? ws_ptr<float>(ws, L.xnorm) : nullptr;
+    // ||x||^2 per row: for the distances of `mind`, and for the screening window of fp32
+    // points (the split computes it in the same pass)
+    float *xnorm = (mind || dtype == FK_F32) ? ws_ptr<float>(ws, L.xnorm) : nullptr;
     const void *planes = nullptr;
+    const float *xn = nullptr;
     int nplanes = 0;
     int64_t lda = 0;
-    if ((s = prepare_x(X, dtype, N, d, L, ws, xnorm, st, &planes, &nplanes, &lda)) != FK_OK)
+    if ((s = prepare_x(X, dtype, N, d, L, ws, xnorm, st, &planes, &nplanes, &lda, &xn)) !=
+        FK_OK)
         return s;
-    return run_assign(planes, nplanes, lda, N, d, K, L, ws, labels, xnorm, mind, st);
+    return run_assign(planes, nplanes, lda, N, d, K, L, ws, labels, xn, mind, st,
+                      dtype == FK_F32 ? static_cast<const float *>(X) : nullptr, C);
 }
 
 fk_status fk_update(const void *X, fk_dtype dtype, int64_t N, int d, int K,
@@ -342,8 +374,10 @@ fk_status fk_lloyd(const void *X, fk_dtype dtype, int64_t N, int d, int K, fk_me
     const void *planes = nullptr;
     int nplanes = 0;
     int64_t lda = 0;
+    // fp32 points: ||x||^2 per row for the screening window, computed by the split
+    float *xnorm = dtype == FK_F32 ? ws_ptr<float>(ws, L.xnorm) : nullptr;
     if (niter > 0 &&
-        (s = prepare_x(Xp, dtype, N, d, L, ws, nullptr, st, &planes, &nplanes, &lda)) != FK_OK)
+        (s = prepare_x(Xp, dtype, N, d, L, ws, xnorm, st, &planes, &nplanes, &lda)) != FK_OK)
         return fail(s);
     if (!rec()) return fail(FK_ERR_CUDA);
 
@@ -353,15 +387,28 @@ fk_status fk_lloyd(const void *X, fk_dtype dtype, int64_t N, int d, int K, fk_me
     double *obj = ws_ptr<double>(ws, L.obj);
     float *cused = ws_ptr<float>(ws, L.cused);
     int copied = 0;
+    bool allow_screen = true;
     for (int t = 0; t < niter; ++t) {
         if (launch_prep_centroids(Ccur, K, d, L.Kp, L.dp, dtype, ws_ptr<uint16_t>(ws, L.cs),
                                   ws_ptr<float>(ws, L.cn), cused, ws_ptr<uint16_t>(ws, L.caug),
                                   st) != cudaSuccess)
             return fail(FK_ERR_CUDA);
         if (!rec()) return fail(FK_ERR_CUDA);
-        if ((s = run_assign(planes, nplanes, lda, N, d, K, L, ws, labels, nullptr, nullptr,
-                            st)) != FK_OK)
+        bool screened = false;
+        if ((s = run_assign(planes, nplanes, lda, N, d, K, L, ws, labels, xnorm, nullptr, st,
+                            dtype == FK_F32 ? static_cast<const float *>(Xp) : nullptr, Ccur,
+                            allow_screen, &screened)) != FK_OK)
             return fail(s);
+        if (screened && t == 0 && niter > 1) {
+            // one look (a single host synchronisation per call) at how many rows needed
+            // the three-product pass; if too many, the plain three-product pass is cheaper
+            uint32_t nfb = 0;
+            if (cudaMemcpyAsync(&nfb, ws_ptr<uint32_t>(ws, L.nfb), sizeof(nfb),
+                                cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+                cudaStreamSynchronize(st) != cudaSuccess)
+                return fail(FK_ERR_CUDA);
+            allow_screen = static_cast<int64_t>(nfb) * kScreenMaxFallback <= N;
+        }
         if (!rec()) return fail(FK_ERR_CUDA);
         const int32_t *skeys = nullptr, *perm = nullptr;
         if (launch_sort_csr(labels, N, K, L.sp, ws_ptr<int32_t>(ws, L.keys0),

@@ -29,6 +29,25 @@ constexpr int kUpdMinRows = 32;       // smallest chunk of sorted positions per 
 constexpr int kUpdMaxRows = 256;      // largest chunk
 constexpr int64_t kUpdTargetWarps = 148 * 64;  // enough warps to cover the GPU twice
 
+// ----------------------------------------------------------------- screening (fp32)
+// The single-product pass writes, per row, four candidate columns for each of the four
+// column groups of a tile (unused slots -1; a group that ran out of room writes
+// kCandOverflow in its first slot and the row goes to the three-product pass).
+constexpr int kCandPerRow = 16;
+constexpr int32_t kCandOverflow = -2;
+// Screened values at or above this are never candidates: padding centroids (whose first
+// norm piece is the largest finite bf16, about 3.39e38) lie above it, and real data whose
+// ||c||^2 + 2|x.c| reaches it is outside the supported range.
+constexpr float kScreenMax = 1e38f;
+// Screening pays where the three-product pass is long per tile: from d = 256 on.  Below,
+// a tile of 256 centroids is so short (9 single-product MMA steps at d = 128) that the
+// candidate bookkeeping in the epilogue, not the tensor cores, sets the pace.
+constexpr int kScreenMinD = 256;
+// fk_lloyd stops screening for the rest of a call when more than 1/kScreenMaxFallback of
+// the rows needed the three-product pass in its first iteration (mixtures whose heavy
+// components hold many nearly equidistant centroids).
+constexpr int kScreenMaxFallback = 4;
+
 // Objective slots kept on the device by fk_lloyd before a copy to the host.
 constexpr int kObjRing = 4096;
 
@@ -94,7 +113,8 @@ struct WsLayout {
     size_t err = 0, obj = 0, xn = 0, xs = 0, xnorm = 0, cs = 0, cn = 0, cused = 0,
            calt = 0, keys0 = 0, keys1 = 0, vals0 = 0, vals1 = 0, hist = 0, dtot = 0,
            caug = 0, pieces = 0, pkeys = 0, piecesb = 0, pkeysb = 0, jpart = 0, jdev = 0, cnt = 0,
-           off = 0, total = 0;
+           off = 0, cand = 0, nfb = 0, fbrows = 0, fblab = 0, xsfb = 0, cmax2 = 0,
+           total = 0;
     int64_t dp = 0, Kp = 0;
     int xplanes = 0;  // bf16 planes of X prepared in the workspace (0, 1 or 2)
     int cplanes = 0;  // bf16 planes of the centroids (1 or 2)
@@ -142,6 +162,15 @@ inline WsLayout ws_layout(int64_t N, int d, int K, fk_dtype dtype, fk_metric met
     L.jdev = take(sizeof(double) * 2);
     L.cnt = take(sizeof(int32_t) * K);
     L.off = take(sizeof(int32_t) * (K + 1));
+    // screened assignment of fp32 points (single bf16 product, exact re-ranking, and the
+    // three-product pass for rows whose candidates did not fit)
+    const bool screen = dtype == FK_F32 || dtype == FK_BF16X2;
+    L.cand = take(screen ? sizeof(int32_t) * kCandPerRow * N : 0);
+    L.nfb = take(screen ? 256 : 0);
+    L.fbrows = take(screen ? sizeof(int32_t) * N : 0);
+    L.fblab = take(screen ? sizeof(int32_t) * N : 0);
+    L.xsfb = take(screen ? sizeof(uint16_t) * 2 * N * L.dp : 0);
+    L.cmax2 = take(screen ? 256 : 0);
     L.total = o;
     return L;
 }
@@ -168,6 +197,9 @@ struct AssignArgs {
     float *mind;           // optional [N]
     uint32_t *err;         // workspace error words
     uint64_t wait_ns;      // bound on every mbarrier wait inside the kernel
+    const uint32_t *n_dev; // optional: row count read on the device (N bounds the maps)
+    int32_t *cand;         // screening pass: [N][kCandPerRow] candidates instead of labels
+    const float *cmax2;    // screening pass: device max_k ||c_k||^2
 };
 
 cudaError_t launch_split_x(const float *X, int64_t N, int d, int64_t dp, uint16_t *hi,
@@ -183,6 +215,22 @@ cudaError_t launch_prep_centroids(const float *C, int K, int d, int64_t Kp, int6
 cudaError_t launch_centroid_norms(const float *C, int K, int d, fk_dtype dtype, float *cn,
                                   cudaStream_t st);
 cudaError_t launch_assign(const AssignArgs &a, cudaStream_t st);
+bool assign_can_screen(int64_t N, int dp, int Kp);
+
+// Screened fp32 assignment (screen.cu): the single-product pass over plane 0 of `a`'s X
+// planes, exact re-ranking of the candidates, and the three-product pass over the rows
+// whose candidates did not fit.  `a` describes the two-plane (hi, lo) problem; X32 is the
+// fp32 points (or null: re-rank from hi + lo).
+struct ScreenBufs {
+    int32_t *cand;     // [N][kCandPerRow]
+    uint32_t *nfb;     // [1] rows sent to the three-product pass
+    int32_t *fbrows;   // [N]
+    int32_t *fblab;    // [N]
+    uint16_t *xsfb;    // [2][N][dp]
+    float *cmax2;      // [1]
+};
+cudaError_t launch_assign_screened(const AssignArgs &a, const float *X32, const float *C,
+                                   const ScreenBufs &sb, cudaStream_t st);
 cudaError_t launch_sort_csr(const int32_t *labels, int64_t N, int K, const SortPlan &sp,
                             int32_t *keys0, int32_t *keys1, int32_t *vals0, int32_t *vals1,
                             int32_t *perm_out, uint32_t *hist, uint32_t *dtot,

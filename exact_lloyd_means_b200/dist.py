@@ -47,9 +47,7 @@ def gpu_ops(N: int, d: int, K: int, dtype, device) -> LocalOps:
     instead of on every assignment; the points must not change during the run."""
     from . import fk
     ws = fk.workspace(N, d, K, dtype, "l2", device=device)
-    dp = (d + 63) // 64 * 64
-    planes = (torch.empty(2, N, dp, dtype=torch.bfloat16, device=device)
-              if dtype == torch.float32 else None)
+    planes = fk.split_points_buffer(N, d, device) if dtype == torch.float32 else None
     state = {"x": None, "split": None}
     labels = torch.empty(N, dtype=torch.int32, device=device)
     sums = torch.empty(K, d, dtype=torch.float64, device=device)

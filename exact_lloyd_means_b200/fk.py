@@ -175,28 +175,38 @@ def fk_centroid_norms(C: torch.Tensor, cn: torch.Tensor, dtype=torch.float32, st
 
 
 class SplitPoints:
-    """fp32 points already split into bf16 hi/lo planes by fk_split_points ([2, N, d_p]
-    bf16, d_p = d rounded up to 64).  fk_assign takes it in place of the fp32 tensor
-    (dtype FK_BF16X2) and skips its per-call split."""
+    """fp32 points already split by fk_split_points: one buffer holding the bf16 hi/lo
+    planes ([2, N, d_p] bf16, d_p = d rounded up to 64) followed by ||x||^2 per row ([N]
+    fp32).  fk_assign takes it in place of the fp32 tensor (dtype FK_BF16X2) and skips its
+    per-call split."""
 
-    def __init__(self, planes: torch.Tensor, N: int, d: int):
-        self.planes, self.N, self.d = planes, N, d
+    def __init__(self, buf: torch.Tensor, N: int, d: int):
+        dp = (d + 63) // 64 * 64
+        self.buf, self.N, self.d = buf, N, d
+        self.planes = buf[:2 * N * dp].view(2, N, dp)
+        self.norms = buf[2 * N * dp:].view(torch.float32)
 
     @property
     def shape(self):
         return (self.N, self.d)
 
 
+def split_points_buffer(N: int, d: int, device="cuda") -> torch.Tensor:
+    """A buffer of the size fk_split_points writes (4 N d_p + 4 N bytes, as bf16)."""
+    dp = (d + 63) // 64 * 64
+    return torch.empty(2 * N * dp + 2 * N, dtype=torch.bfloat16, device=device)
+
+
 def fk_split_points(X: torch.Tensor, out: torch.Tensor | None = None,
                     stream=None) -> SplitPoints:
-    """Split fp32 points into bf16 hi/lo planes once; `out` ([2, N, d_p] bf16) is
-    allocated when not given."""
+    """Split fp32 points into bf16 hi/lo planes (and their squared norms) once; `out`
+    (from split_points_buffer) is allocated when not given."""
     N, d = X.shape
     dp = (d + 63) // 64 * 64
     if out is None:
-        out = torch.empty(2, N, dp, dtype=torch.bfloat16, device=X.device)
+        out = split_points_buffer(N, d, X.device)
     _check(_lib.fk_split_points(_dev(X, "X", torch.float32), N, d,
-                                _dev(out, "out", torch.bfloat16, (2, N, dp)),
+                                _dev(out, "out", torch.bfloat16, (2 * N * dp + 2 * N,)),
                                 _stream(stream)), "fk_split_points")
     return SplitPoints(out, N, d)
 
@@ -206,7 +216,7 @@ def fk_assign(X, C: torch.Tensor, labels: torch.Tensor, ws: torch.Tensor,
     N, d = X.shape
     K = C.shape[0]
     if isinstance(X, SplitPoints):
-        xptr, code = _dev(X.planes, "X.planes", torch.bfloat16), FK_BF16X2
+        xptr, code = _dev(X.buf, "X.buf", torch.bfloat16), FK_BF16X2
     else:
         xptr, code = _dev(X, "X"), _dtype_code(X)
     _check(_lib.fk_assign(xptr, code, N, d,

@@ -77,8 +77,8 @@ typedef enum fk_dtype {
     FK_F32 = 0,   /* fp32 points; products emulated to fp32 accuracy with three bf16
                      tensor-core products (hi*hi + lo*hi + hi*lo)                     */
     FK_BF16 = 1,  /* bf16 points; bf16 tensor-core products (exact), fp32 accumulation */
-    FK_BF16X2 = 2 /* fp32 points given already split by fk_split_points: two bf16 planes
-                     [2][N][roundup(d,64)] (hi, then lo); fk_assign only             */
+    FK_BF16X2 = 2 /* fp32 points given already split by fk_split_points (bf16 hi/lo
+                     planes, then ||x||^2 per row); fk_assign only                     */
 } fk_dtype;
 
 typedef enum fk_metric {
@@ -121,10 +121,11 @@ FK_API fk_status fk_normalize_rows(const float *X_in, float *X_out, int64_t N, i
                             fk_stream_t stream);
 
 /* Split fp32 points once for repeated assignment (the first step of fk_assign for
- * FK_F32): planes = [2][N][d_p] bf16 with d_p = roundup(d, 64), hi = RN_bf16(x), lo =
- * RN_bf16(x - hi), zero padding.  `planes` (device, 16-byte aligned, 4*N*d_p bytes) can
- * then be passed to fk_assign as X with dtype FK_BF16X2, skipping the per-call split.
- * fp32 only (d % 4 == 0, X 16-byte aligned). */
+ * FK_F32).  `planes` (device, 16-byte aligned, 4*N*d_p + 4*N bytes, d_p = roundup(d, 64))
+ * receives [2][N][d_p] bf16, hi = RN_bf16(x) then lo = RN_bf16(x - hi), zero padded,
+ * followed by [N] fp32 ||x||^2 (fp64 accumulation, one rounding).  It can then be passed
+ * to fk_assign as X with dtype FK_BF16X2, skipping the per-call split.  fp32 only
+ * (d % 4 == 0, X 16-byte aligned). */
 FK_API fk_status fk_split_points(const float *X, int64_t N, int d, void *planes,
                                  fk_stream_t stream);
 
@@ -136,15 +137,22 @@ FK_API fk_status fk_centroid_norms(const float *C, int K, int d, fk_dtype dtype,
 
 /* Assignment step (Flash-KMeans article, "FlashAssign：把距离矩阵按块切成流水线").
  *   labels[i] = argmin_k ||x_i - c_k||^2, lowest k on exact ties, for i < N.
- *   mind[i]   = ||x_i||^2 + min_k (||c_k||^2 - 2 x_i.c_k)  (expansion form; optional,
- *               pass NULL to skip).
+ *   mind[i]   = min_k ||x_i - c_k||^2 (optional, pass NULL to skip), within
+ *               1e-4 (||x_i||^2 + max_k ||c_k||^2): the re-ranking's fp64
+ *               difference form on the screened route below, else the tensor-core
+ *               expansion ||x||^2 + (||c||^2 - 2 x.c).
  * X: N x d, dtype `dtype`.  C: K x d fp32 (for FK_BF16 the kernel uses C rounded to
  * bf16).  labels: N int32.  The N x K distance matrix is never stored: a tcgen05 kernel
  * keeps one 128 x 256 fp32 tile in tensor memory and a running min/argmin per row.
  * For FK_F32 each call first splits X into bf16 hi/lo planes inside `ws` (one extra
  * pass over X; fk_lloyd does this once per call instead of once per iteration); callers
  * that assign the same points repeatedly split once with fk_split_points and pass the
- * planes with FK_BF16X2. */
+ * planes with FK_BF16X2.
+ * Screened route (fp32 points, N >= 18,944 rows, C 16-byte aligned): one bf16 product
+ * per term finds, for every row, the centroids within a proven bound of the nearest; their
+ * distances (fp64, difference form) pick the label, and rows with more such
+ * centroids than the kernel keeps are assigned by the three-product form.  Labels are the
+ * same as the three-product form's outside the parity tie window. */
 FK_API fk_status fk_assign(const void *X, fk_dtype dtype, int64_t N, int d, const float *C,
                     int K, int32_t *labels, float *mind, void *ws, size_t ws_bytes,
                     fk_stream_t stream);

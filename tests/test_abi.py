@@ -108,9 +108,6 @@ def test_pre_split_dtype_is_assign_only(fk):
                          256, big, None) == fk.FK_ERR_UNSUPPORTED
     assert lib.fk_update_partial(256, fk.FK_BF16X2, 100, 8, 4, 256, 256, 256, 256, 256, None,
                                  256, big, None) == fk.FK_ERR_UNSUPPORTED
-    # the pre-split form has no point norms, so no distances are returned
-    assert lib.fk_assign(256, fk.FK_BF16X2, 100, 8, 256, 4, 256, 512, 256, big, None) == \
-        fk.FK_ERR_UNSUPPORTED
     assert lib.fk_split_points(None, 100, 8, 256, None) == fk.FK_ERR_INVALID_ARG
     assert lib.fk_split_points(256, 100, 6, 256, None) == fk.FK_ERR_UNSUPPORTED
     assert lib.fk_split_points(8, 100, 8, 256, None) == fk.FK_ERR_UNSUPPORTED

@@ -323,6 +323,8 @@ def test_split_points_planes_are_rounded_hi_lo(N, d):
     assert torch.equal(P[0, :, :d].view(torch.int16), hi.view(torch.int16))
     assert torch.equal(P[1, :, :d].view(torch.int16), lo.view(torch.int16))
     assert not P[:, :, d:].float().any()
+    norms = sp.norms.cpu().double()
+    assert torch.allclose(norms, (X.double() ** 2).sum(1), rtol=1e-6, atol=0)
 
 
 @pytest.mark.parametrize("N,d,K", [(20000, 128, 300), (5000, 768, 1000), (3001, 64, 37)])
@@ -337,3 +339,63 @@ def test_assign_pre_split_points_equals_fp32_assign(N, d, K):
     m.fk_assign(Xg, Cg, l1, ws)
     m.fk_assign(m.fk_split_points(Xg), Cg, l2, ws)
     assert torch.equal(l1, l2)
+
+
+# Screened fp32 assignment: for fp32 points with d >= 256 at CTA-pair sizes
+# (N >= 2 * 128 * 148 / 2) the single-product pass keeps the columns inside a proven error window, the candidates
+# are re-ranked exactly, and rows whose candidates do not fit are assigned by the
+# three-product pass.  These cases drive each branch: ordinary mixtures (few candidates),
+# components that received several initial centroids (several candidates), exact
+# duplicates (ties resolved to the lowest index), and a Zipf mixture whose heavy
+# components hold hundreds of nearly equidistant centroids (the overflow path).
+SCREEN_CASES = [
+    ("normal", 40000, 256, 300, "equal", 0.3),
+    ("normal", 30000, 768, 1024, "equal", 0.3),
+    ("uniform", 50001, 320, 4100, "equal", 0.2),
+    ("normal", 40000, 256, 2000, "zipf", 0.15),
+    ("normal", 20000, 1032, 700, "equal", 0.3),
+]
+
+
+@pytest.mark.parametrize("centers,N,d,K,weights,sigma", SCREEN_CASES)
+def test_screened_assign_matches_oracle(centers, N, d, K, weights, sigma):
+    X, comp, _ = gaussian_mixture(N, d, K, centers=centers, sigma=sigma, weights=weights,
+                                  seed=N + K)
+    C0 = X[init_indices(N, K, N + K)].float().contiguous()
+    ref, dmin, d2nd = oracle.assign(X, C0.numpy())
+    ties = oracle.tie_mask(X, C0.numpy(), dmin, d2nd)
+    lab, mind = gpu_assign(X.to(DEV), C0.to(DEV), with_mind=True)
+    assert (lab >= 0).all() and (lab < K).all()
+    assert label_mismatches(lab, ref, ties) == 0, f"ties={int(ties.sum())}"
+    Xd = X.double().numpy()
+    s = (Xd * Xd).sum(1) + (C0.double().numpy() ** 2).sum(1).max()
+    assert (np.abs(mind.astype(np.float64) - dmin) <= 1e-4 * s).all()
+
+
+def test_screened_assign_duplicates_take_lowest_index():
+    """30 distinct centroids, each present 10 times at scattered columns: every row's
+    nearest value is shared by 10 columns, which overflows some column groups; the label
+    must be the lowest of the 10 (bit-identical values), whichever pass decides it."""
+    N, d = 40000, 256
+    X, _, _ = gaussian_mixture(N, d, 30, centers="normal", sigma=0.3, seed=31)
+    base = X[init_indices(N, 30, 31)].float()
+    C = base.repeat(10, 1).contiguous()  # column 30 * r + j is a copy of base[j]
+    lab, _ = gpu_assign(X.to(DEV), C.to(DEV))
+    ref, dmin, d2nd = oracle.assign(X, base.numpy())
+    ties = oracle.tie_mask(X, base.numpy(), dmin, d2nd)
+    assert label_mismatches(lab, ref, ties) == 0  # and so the lowest copy, column < 30
+    assert (lab[~ties] < 30).all()
+
+
+def test_screened_lloyd_lockstep_heavy_components():
+    """Lockstep iterations on a Zipf mixture (many centroids per heavy component)."""
+    X, _, _ = gaussian_mixture(40000, 256, 1500, centers="normal", sigma=0.15,
+                               weights="zipf", seed=33)
+    C0 = X[init_indices(40000, 1500, 33)].float().contiguous()
+    ref = oracle.lloyd(X, C0, 2)
+    Xg = X.to(DEV)
+    C_master = [C0.double().numpy()] + ref["C_next"]
+    for t in range(2):
+        Cm = torch.as_tensor(C_master[t], dtype=torch.float32)
+        lab, _ = gpu_assign(Xg, Cm.to(DEV))
+        assert label_mismatches(lab, ref["labels"][t], ref["ties"][t]) == 0, t
