@@ -120,7 +120,8 @@ fk_status run_assign(const void *planes, int nplanes, int64_t lda, int64_t N, in
                      const WsLayout &L, void *ws, int32_t *labels, const float *xnorm,
                      float *mind, cudaStream_t st, const float *X32 = nullptr,
                      const float *C = nullptr, bool allow_screen = true,
-                     bool *screened = nullptr) {
+                     bool *screened = nullptr, cudaEvent_t ev_mma0 = nullptr,
+                     cudaEvent_t ev_mma1 = nullptr) {
     if (screened) *screened = false;
     AssignArgs a{};
     a.a_planes = planes;
@@ -150,11 +151,13 @@ fk_status run_assign(const void *planes, int nplanes, int64_t lda, int64_t N, in
         sb.fblab = ws_ptr<int32_t>(ws, L.fblab);
         sb.xsfb = ws_ptr<uint16_t>(ws, L.xsfb);
         sb.cmax2 = ws_ptr<float>(ws, L.cmax2);
-        FK_TRY_CUDA(launch_assign_screened(a, X32, C, sb, st));
+        FK_TRY_CUDA(launch_assign_screened(a, X32, C, sb, st, ev_mma0, ev_mma1));
         if (screened) *screened = true;
         return FK_OK;
     }
+    if (ev_mma0) FK_TRY_CUDA(cudaEventRecord(ev_mma0, st));
     FK_TRY_CUDA(launch_assign(a, st));
+    if (ev_mma1) FK_TRY_CUDA(cudaEventRecord(ev_mma1, st));
     return FK_OK;
 }
 
@@ -222,7 +225,7 @@ const char *fk_status_string(fk_status s) {
     return "FK_UNKNOWN_STATUS";
 }
 
-int fk_version(void) { return 1; }
+int fk_version(void) { return 2; }
 
 int64_t fk_launch_count(void) { return g_launches; }
 
@@ -351,8 +354,18 @@ fk_status fk_lloyd(const void *X, fk_dtype dtype, int64_t N, int d, int K, fk_me
         ev.push_back(e);
         return cudaEventRecord(e, st) == cudaSuccess;
     };
+    // events around the main tensor-core kernel of each iteration's assignment
+    std::vector<cudaEvent_t> evm;
+    auto mk = [&](cudaEvent_t *e) -> bool {
+        *e = nullptr;
+        if (!timing) return true;
+        if (cudaEventCreate(e) != cudaSuccess) return false;
+        evm.push_back(*e);
+        return true;
+    };
     auto cleanup = [&]() {
         for (auto e : ev) cudaEventDestroy(e);
+        for (auto e : evm) cudaEventDestroy(e);
     };
     auto fail = [&](fk_status f) {
         cleanup();
@@ -388,6 +401,7 @@ fk_status fk_lloyd(const void *X, fk_dtype dtype, int64_t N, int d, int K, fk_me
     float *cused = ws_ptr<float>(ws, L.cused);
     int copied = 0;
     bool allow_screen = true;
+    int nscreened = 0;
     for (int t = 0; t < niter; ++t) {
         if (launch_prep_centroids(Ccur, K, d, L.Kp, L.dp, dtype, ws_ptr<uint16_t>(ws, L.cs),
                                   ws_ptr<float>(ws, L.cn), cused, ws_ptr<uint16_t>(ws, L.caug),
@@ -395,10 +409,13 @@ fk_status fk_lloyd(const void *X, fk_dtype dtype, int64_t N, int d, int K, fk_me
             return fail(FK_ERR_CUDA);
         if (!rec()) return fail(FK_ERR_CUDA);
         bool screened = false;
+        cudaEvent_t m0 = nullptr, m1 = nullptr;
+        if (!mk(&m0) || !mk(&m1)) return fail(FK_ERR_CUDA);
         if ((s = run_assign(planes, nplanes, lda, N, d, K, L, ws, labels, xnorm, nullptr, st,
                             dtype == FK_F32 ? static_cast<const float *>(Xp) : nullptr, Ccur,
-                            allow_screen, &screened)) != FK_OK)
+                            allow_screen, &screened, m0, m1)) != FK_OK)
             return fail(s);
+        nscreened += screened ? 1 : 0;
         if (screened && t == 0 && niter > 1) {
             // one look (a single host synchronisation per call) at how many rows needed
             // the three-product pass; if too many, the plain three-product pass is cheaper
@@ -463,6 +480,10 @@ fk_status fk_lloyd(const void *X, fk_dtype dtype, int64_t N, int d, int K, fk_me
         }
         timing->iterations = niter;
         timing->launches = static_cast<int>(g_launches - launches0);
+        for (size_t a = 0; a + 1 < evm.size(); a += 2)
+            if (cudaEventElapsedTime(&ms, evm[a], evm[a + 1]) == cudaSuccess)
+                timing->ms_assign_mma += ms;
+        timing->screened = nscreened;
     }
     cleanup();
     return static_cast<fk_status>(code);

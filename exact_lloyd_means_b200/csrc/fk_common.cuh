@@ -230,7 +230,9 @@ struct ScreenBufs {
     float *cmax2;      // [1]
 };
 cudaError_t launch_assign_screened(const AssignArgs &a, const float *X32, const float *C,
-                                   const ScreenBufs &sb, cudaStream_t st);
+                                   const ScreenBufs &sb, cudaStream_t st,
+                                   cudaEvent_t ev_mma0 = nullptr,
+                                   cudaEvent_t ev_mma1 = nullptr);
 cudaError_t launch_sort_csr(const int32_t *labels, int64_t N, int K, const SortPlan &sp,
                             int32_t *keys0, int32_t *keys1, int32_t *vals0, int32_t *vals1,
                             int32_t *perm_out, uint32_t *hist, uint32_t *dtot,

@@ -212,7 +212,8 @@ __global__ void fb_scatter_kernel(const uint32_t *__restrict__ nfb,
 }  // namespace
 
 cudaError_t launch_assign_screened(const AssignArgs &a, const float *X32, const float *C,
-                                   const ScreenBufs &sb, cudaStream_t st) {
+                                   const ScreenBufs &sb, cudaStream_t st, cudaEvent_t ev_mma0,
+                                   cudaEvent_t ev_mma1) {
     const uint16_t *xhi = static_cast<const uint16_t *>(a.a_planes);
     const uint16_t *xlo = xhi + a.N * a.lda;
     window_kernel<<<1, 1024, 0, st>>>(a.cn, a.K, sb.cmax2, sb.nfb);
@@ -227,7 +228,9 @@ cudaError_t launch_assign_screened(const AssignArgs &a, const float *X32, const 
     s1.mind = nullptr;
     s1.best = nullptr;
     s1.n_dev = nullptr;
+    if (ev_mma0 && (e = cudaEventRecord(ev_mma0, st)) != cudaSuccess) return e;
     if ((e = launch_assign(s1, st)) != cudaSuccess) return e;
+    if (ev_mma1 && (e = cudaEventRecord(ev_mma1, st)) != cudaSuccess) return e;
 
     const int64_t rr_blocks = ceil_div(a.N, 8);
     const int rgrid = static_cast<int>(rr_blocks < 148 * 16 ? rr_blocks : 148 * 16);

@@ -36,7 +36,8 @@ class FkTiming(ctypes.Structure):
     _fields_ = [("ms_setup", ctypes.c_double), ("ms_prep", ctypes.c_double),
                 ("ms_assign", ctypes.c_double), ("ms_sort", ctypes.c_double),
                 ("ms_update", ctypes.c_double), ("iterations", ctypes.c_int),
-                ("launches", ctypes.c_int)]
+                ("launches", ctypes.c_int), ("ms_assign_mma", ctypes.c_double),
+                ("screened", ctypes.c_int)]
 
 
 def _sig(name, args, res=ctypes.c_int):

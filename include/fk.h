@@ -91,17 +91,21 @@ typedef enum fk_metric {
 typedef struct fk_timing {
     double ms_setup;   /* once per call: normalisation (cosine) and the fp32 split of X */
     double ms_prep;    /* per iteration: centroid norms and operand preparation        */
-    double ms_assign;  /* per iteration: the fused tensor-core assign kernel           */
+    double ms_assign;  /* per iteration: the whole assignment (every kernel of it)     */
     double ms_sort;    /* per iteration: radix sort of labels -> perm + CSR offsets   */
     double ms_update;  /* per iteration: segmented reduction, combine, finalize, J     */
     int iterations;
     int launches;      /* kernels this call launched (library kernels only)            */
+    double ms_assign_mma; /* per iteration: the main tensor-core kernel of the assignment
+                             alone (the single-product screening pass on the screened
+                             route, else the assign kernel)                           */
+    int screened;      /* iterations that took the screened route                      */
 } fk_timing;
 
 /* Human-readable name of a status code (static string, never NULL). */
 FK_API const char *fk_status_string(fk_status s);
 
-/* Library ABI version (incremented on any signature change). */
+/* Library ABI version (incremented on any signature or struct change). */
 FK_API int fk_version(void);
 
 /* Number of kernels this library has launched from the calling host thread since it was
