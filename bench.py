@@ -175,7 +175,9 @@ def reference_arm(args, spec, rank, world):
 
     import oracle
     from synth import gaussian_mixture, init_indices
-    S = 256 if spec.d * spec.k > 1_000_000 else 4096
+    # a sample large enough that the per-step fixed costs (centroid normalisation and
+    # rounding) are small next to the per-point work, yet about a second of CPU per step
+    S = int(max(256, min(65536, 2e10 // (spec.k * spec.d))))
     n_gen = 2 * max(S, spec.k)
     X, _, _ = gaussian_mixture(n_gen, spec.d, spec.k, centers=spec.centers, sigma=spec.sigma,
                                weights=spec.weights, zipf_s=spec.zipf_s, dtype=spec.dtype,
