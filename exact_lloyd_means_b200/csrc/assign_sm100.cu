@@ -131,34 +131,43 @@ __device__ __forceinline__ float min64(const float (&v)[64]) {
     return ptx::fmin3(a, b, fminf(u[6], u[7]));
 }
 
-// Screening helpers.  The smallest published running minimum of this row's column groups
-// in the current row block (entries [g * kBM] for g = 0..3, tagged with the row block),
-// and `own` (this group's own minimum).
-__device__ __forceinline__ float scr_global_min(const uint64_t *pub_row, uint32_t tag,
-                                                float own) {
-    float gm = own;
+// Screening: add the columns base + bit of `mask` (screened values >= m, the minimum of
+// their chunk) to a row's candidate list.  A free slot holds +inf.  When the list is full,
+// the entry with the largest bound gives way (or the new column, if its bound is the
+// largest) and that bound is remembered in `lost`: the row overflows if it is still inside
+// the final window.
+template <int KS>
+__device__ __forceinline__ void scr_insert(uint32_t mask, int base, float m, float (&lb)[KS],
+                                           int (&cc)[KS], float &lost) {
+    const float inf = __int_as_float(0x7f800000);
+    for (; mask != 0u; mask &= mask - 1u) {
+        const int col = base + __ffs(mask) - 1;
+        bool placed = false;
 #pragma unroll
-    for (int o = 0; o < 4; ++o) {
-        const uint64_t p = ptx::ld_relaxed_u64(pub_row + o * kBM);
-        if (static_cast<uint32_t>(p >> 32) == tag)
-            gm = fminf(gm, __uint_as_float(static_cast<uint32_t>(p)));
-    }
-    return gm;
-}
-
-// Append the columns base + bit of `mask` to the (up to four) candidates c0..c3.
-__device__ __forceinline__ void scr_emit(uint64_t mask, int base, int &cnt, int &c0, int &c1,
-                                         int &c2, int &c3, bool &over) {
-    for (; mask != 0ull && !over; mask &= mask - 1ull) {
-        const int col = base + __ffsll(static_cast<long long>(mask)) - 1;
-        if (cnt < 4) {
-            c3 = c2;
-            c2 = c1;
-            c1 = c0;
-            c0 = col;
-            ++cnt;
+        for (int t = 0; t < KS; ++t) {
+            if (!placed && lb[t] == inf) {
+                lb[t] = m;
+                cc[t] = col;
+                placed = true;
+            }
+        }
+        if (placed) continue;
+        float mx = lb[0];
+#pragma unroll
+        for (int t = 1; t < KS; ++t) mx = fmaxf(mx, lb[t]);
+        if (m < mx) {
+            bool done = false;
+#pragma unroll
+            for (int t = 0; t < KS; ++t) {
+                if (!done && lb[t] == mx) {
+                    lb[t] = m;
+                    cc[t] = col;
+                    done = true;
+                }
+            }
+            lost = fminf(lost, mx);
         } else {
-            over = true;
+            lost = fminf(lost, m);
         }
     }
 }
@@ -515,7 +524,7 @@ __global__ void __launch_bounds__(AsgCfg<NP, RES>::kThreads, 1)
 // complete on the even CTA's barriers, MMA completion is signalled to both CTAs
 // (tcgen05.commit multicast), and both CTAs' epilogues release the accumulator to the
 // even CTA by remote arrive.  No load is multicast.
-template <int NP, bool RES>
+template <int NP, bool RES, int EG = 4>
 struct PairCfg {
     static constexpr int kABytes = kBM * kBK * 2;         // 16 KB: 128 X rows, one chunk
     static constexpr int kBBytes = (kBN / 2) * kBK * 2;   // 16 KB: 128 centroids, one chunk
@@ -531,7 +540,9 @@ struct PairCfg {
     static constexpr int kStages = RES ? (NP == 1 ? 4 : 2) : (NP == 2 ? 3 : 6);
     static constexpr int kDataBytes = kARegion + kStages * kStageBytes;  // 192 KB
     static constexpr int kBarBytes = 512;
-    static constexpr int kEpiGroups = 4;
+    // epilogue warpgroups splitting a tile's columns: 4 for the argmin; 1 for the screening
+    // pass, whose per-row candidate list must see all 256 columns of every tile
+    static constexpr int kEpiGroups = EG;
     static constexpr int kEpiCols = kBN / kEpiGroups;
     static constexpr int kRedBytes = (kEpiGroups - 1) * 2 * kBM * 8;
     static constexpr int kAugA = kBM * kAug * 2;         // 4 KB: constant (1, 1, 1, 0, ...)
@@ -546,7 +557,7 @@ struct PairCfg {
 };
 
 template <int NP, bool RES, bool SCR>
-__global__ void __launch_bounds__(PairCfg<NP, RES>::kThreads, 1)
+__global__ void __launch_bounds__(PairCfg<NP, RES, SCR ? 1 : 4>::kThreads, 1)
     assign_pair_kernel(const __grid_constant__ CUtensorMap tmA0,
                        const __grid_constant__ CUtensorMap tmA1,
                        const __grid_constant__ CUtensorMap tmB0,
@@ -559,8 +570,7 @@ __global__ void __launch_bounds__(PairCfg<NP, RES>::kThreads, 1)
                        const uint32_t *__restrict__ n_dev, int32_t *__restrict__ cand,
                        const float *__restrict__ cmax2) {
     static_assert(!SCR || NP == 1, "screening runs the single-product form");
-    static_assert(PairCfg<NP, RES>::kEpiGroups == 4, "scr_global_min reads four groups");
-    using Cfg = PairCfg<NP, RES>;
+    using Cfg = PairCfg<NP, RES, SCR ? 1 : 4>;
     constexpr int S = Cfg::kStages;
     constexpr int EC = Cfg::kEpiCols;
     if (n_dev != nullptr) {  // row count written on the device by an earlier kernel
@@ -606,8 +616,10 @@ __global__ void __launch_bounds__(PairCfg<NP, RES>::kThreads, 1)
             ptx::mbar_init(&tempty[a], 2 * Cfg::kEpiWarps);
             ptx::mbar_init(&afull[a], 1);
             ptx::mbar_init(&aempty[a], 1);
-            ptx::mbar_init(&redfull[a], (Cfg::kEpiGroups - 1) * kBM);
-            ptx::mbar_init(&redempty[a], kBM);
+            if (Cfg::kEpiGroups > 1) {
+                ptx::mbar_init(&redfull[a], (Cfg::kEpiGroups - 1) * kBM);
+                ptx::mbar_init(&redempty[a], kBM);
+            }
             ptx::mbar_init(&augfull[a], 1);
         }
         ptx::mbar_init(drain, 1);
@@ -631,8 +643,6 @@ __global__ void __launch_bounds__(PairCfg<NP, RES>::kThreads, 1)
         init_aug_a(aaug, (warp & 3) * 32 + lane);
         ptx::fence_proxy_async_smem();  // visible to the tensor core (async proxy)
     }
-    if (SCR && warp >= 2)  // published minima start with a tag no row block carries
-        reinterpret_cast<uint64_t *>(red_v)[(warp - 2) * 32 + lane] = ~0ull;
     ptx::tc_fence_before();
     __syncthreads();
     ptx::cluster_sync();  // barriers of both CTAs initialised, tensor memory allocated
@@ -812,47 +822,112 @@ __global__ void __launch_bounds__(PairCfg<NP, RES>::kThreads, 1)
                 }
             }
         }
+    } else if constexpr (SCR) {
+        // ------------------------------------------------------ screening epilogue (both)
+        // One warpgroup owns all 256 columns of every tile: warp q holds the rows of tensor
+        // memory lanes 32q .. 32q + 31 and reads each tile as four 64-column chunks.  Per
+        // row it keeps the running screened minimum and a list of up to kScreenSlots
+        // candidate columns, each with a lower bound on its screened value (the minimum of
+        // the chunk it came from).
+        const int q = warp & 3;
+        const int r = q * 32 + lane;
+        const float cm2 = *cmax2;
+        const float inf = __int_as_float(0x7f800000);
+        uint32_t titer = 0;
+        bool ok = true;
+        // ||x||^2 of this thread's row in the next row block, loaded a block ahead
+        float xn_next = 0.f;
+        {
+            const int64_t row0 = pair * 2 * kBM + static_cast<int64_t>(rank) * kBM + r;
+            if (pair < nmb && row0 < N) xn_next = xnorm[row0];
+        }
+        for (int64_t mb = pair; mb < nmb && ok; mb += npairs) {
+            const int64_t row = mb * 2 * kBM + static_cast<int64_t>(rank) * kBM + r;
+            const float W = screen_window(xn_next, cm2, nkc * kBK);
+            {
+                const int64_t rn = row + npairs * 2 * kBM;
+                xn_next = (mb + npairs < nmb && rn < N) ? xnorm[rn] : 0.f;
+            }
+            float best = inf, lost = inf;
+            float lb[kScreenSlots];
+            int cc[kScreenSlots];
+#pragma unroll
+            for (int t = 0; t < kScreenSlots; ++t) {
+                lb[t] = inf;
+                cc[t] = -1;
+            }
+            for (int nt = 0; nt < ntiles; ++nt, ++titer) {
+                const uint32_t acc = titer & 1u;
+                const uint32_t aphase = (titer >> 1) & 1u;
+                if (!warp_wait(&tfull[acc], aphase, abort_flag, wait_ns)) {
+                    if (lane == 0) raise_timeout(abort_flag, err);
+                    ok = false;
+                    break;
+                }
+                ptx::tc_fence_after();
+                const uint32_t tb = tmem + (static_cast<uint32_t>(q * 32) << 16) + acc * kBN;
+#pragma unroll 1
+                for (int c4 = 0; c4 < kBN / 64; ++c4) {
+                    __syncwarp();
+                    float v[64];  // ||c||^2 - 2 x~.c~ for 64 columns
+                    ptx::tmem_ld64_sync(tb + c4 * 64, v);
+                    if (c4 == kBN / 64 - 1) {  // the whole tile is in registers: release it
+                        ptx::tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) ptx::mbar_arrive_cluster(tempty_c + acc * 8);
+                    }
+                    const float m = min64(v);
+                    if (m <= best + W) {  // this chunk has columns inside the window
+                        if (m < best) {
+                            best = m;
+                            const float T0 = fminf(best + W, kScreenMax);
+#pragma unroll
+                            for (int t = 0; t < kScreenSlots; ++t)
+                                if (lb[t] > T0) lb[t] = inf;  // left the window for good
+                        }
+                        const float T = fminf(best + W, kScreenMax);
+                        uint32_t lo = 0u, hi = 0u;
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) {
+                            lo |= (v[j] <= T ? 1u : 0u) << j;
+                            hi |= (v[32 + j] <= T ? 1u : 0u) << j;
+                        }
+                        const int base = nt * kBN + c4 * 64;
+                        scr_insert(lo, base, m, lb, cc, lost);
+                        scr_insert(hi, base + 32, m, lb, cc, lost);
+                    }
+                }
+            }
+            if (!ok) break;
+            // candidates: every kept column whose chunk minimum is inside the final window;
+            // the row overflows if a column dropped for lack of room could still be inside
+            const float T = fminf(best + W, kScreenMax);
+            const bool over = lost <= T;
+            if (row < N) {
+                int4 *dst = reinterpret_cast<int4 *>(cand + row * kCandPerRow);
+#pragma unroll
+                for (int t4 = 0; t4 < kScreenSlots / 4; ++t4) {
+                    int4 o;
+                    o.x = lb[4 * t4 + 0] <= T ? cc[4 * t4 + 0] : -1;
+                    o.y = lb[4 * t4 + 1] <= T ? cc[4 * t4 + 1] : -1;
+                    o.z = lb[4 * t4 + 2] <= T ? cc[4 * t4 + 2] : -1;
+                    o.w = lb[4 * t4 + 3] <= T ? cc[4 * t4 + 3] : -1;
+                    if (t4 == 0 && over) o.x = kCandOverflow;
+                    dst[t4] = o;
+                }
+            }
+        }
     } else {
         // ------------------------------------------------------------ epilogue (both)
         const int g = (warp - 2) >> 2;
         const int q = warp & 3;
         const int r = q * 32 + lane;
-        const float cm2 = SCR ? *cmax2 : 0.f;
-        // screening: each group publishes its running minimum per row, tagged with the row
-        // block, so every group can window against the minimum over all 256 columns of
-        // the tiles seen so far.  A value read while its writer is a tile ahead or behind
-        // is still some group's minimum over real columns of this row, so the window it
-        // gives can only be wider than the exact one (never narrower).
-        uint64_t *pub = reinterpret_cast<uint64_t *>(red_v);  // [kEpiGroups][kBM]
         uint32_t titer = 0, mbi = 0;
         bool ok = true;
-        // ||x||^2 of this thread's row in the next row block, loaded a block ahead so the
-        // window is ready when the block starts
-        float xn_next = 0.f;
-        if (SCR) {
-            const int64_t row0 = pair * 2 * kBM + static_cast<int64_t>(rank) * kBM + r;
-            if (pair < nmb && row0 < N) xn_next = xnorm[row0];
-        }
         for (int64_t mb = pair; mb < nmb && ok; mb += npairs, ++mbi) {
             const int64_t row = mb * 2 * kBM + static_cast<int64_t>(rank) * kBM + r;
             float best = __int_as_float(0x7f800000);
             int bestk = 0;
-            // screening state: the window width; up to three kept tiles, each with its
-            // minimum over this group's columns (+inf = free slot), its index and the mask
-            // of its columns inside the window when it was kept; and the smallest minimum
-            // of a tile dropped for lack of room (the row overflows if that tile is still
-            // inside the final window)
-            float W = 0.f;
-            float em0 = __int_as_float(0x7f800000), em1 = em0, em2 = em0, lost = em0;
-            int et0 = 0, et1 = 0, et2 = 0;
-            uint32_t el0 = 0, eh0 = 0, el1 = 0, eh1 = 0, el2 = 0, eh2 = 0;
-            bool over = false;
-            const uint32_t tag = static_cast<uint32_t>(mb);
-            if (SCR) {
-                W = screen_window(xn_next, cm2, nkc * kBK);
-                const int64_t rn = row + npairs * 2 * kBM;
-                xn_next = (mb + npairs < nmb && rn < N) ? xnorm[rn] : 0.f;
-            }
             for (int nt = 0; nt < ntiles; ++nt, ++titer) {
                 const uint32_t acc = titer & 1u;
                 const uint32_t aphase = (titer >> 1) & 1u;
@@ -872,49 +947,7 @@ __global__ void __launch_bounds__(PairCfg<NP, RES>::kThreads, 1)
                 __syncwarp();
                 if (lane == 0) ptx::mbar_arrive_cluster(tempty_c + acc * 8);  // consumed
                 const float m = min64(v);
-                if (SCR) {
-                    float gm = scr_global_min(pub + r, tag, best);
-                    if (m <= gm + W) {  // this tile has columns inside the window
-                        if (m < best) {
-                            best = m;
-                            ptx::st_relaxed_u64(pub + g * kBM + r,
-                                                (static_cast<uint64_t>(tag) << 32) |
-                                                    __float_as_uint(m));
-                        }
-                        gm = fminf(gm, m);
-                        const float T = fminf(gm + W, kScreenMax);
-                        uint32_t lo = 0u, hi = 0u;
-#pragma unroll
-                        for (int j = 0; j < 32; ++j) {
-                            lo |= (v[j] <= T ? 1u : 0u) << j;
-                            hi |= (v[32 + j] <= T ? 1u : 0u) << j;
-                        }
-                        const float inf = __int_as_float(0x7f800000);
-                        if (em0 > T) em0 = inf;  // kept tiles that left the window for good
-                        if (em1 > T) em1 = inf;
-                        if (em2 > T) em2 = inf;
-                        if ((lo | hi) != 0u) {
-                            if (em0 == inf) {
-                                em0 = m; et0 = nt; el0 = lo; eh0 = hi;
-                            } else if (em1 == inf) {
-                                em1 = m; et1 = nt; el1 = lo; eh1 = hi;
-                            } else if (em2 == inf) {
-                                em2 = m; et2 = nt; el2 = lo; eh2 = hi;
-                            } else if (m >= em0 && m >= em1 && m >= em2) {
-                                lost = fminf(lost, m);  // keep the three smallest minima
-                            } else if (em0 >= em1 && em0 >= em2) {
-                                lost = fminf(lost, em0);
-                                em0 = m; et0 = nt; el0 = lo; eh0 = hi;
-                            } else if (em1 >= em2) {
-                                lost = fminf(lost, em1);
-                                em1 = m; et1 = nt; el1 = lo; eh1 = hi;
-                            } else {
-                                lost = fminf(lost, em2);
-                                em2 = m; et2 = nt; el2 = lo; eh2 = hi;
-                            }
-                        }
-                    }
-                } else if (m < best) {
+                if (m < best) {
                     int idx = 0;
 #pragma unroll
                     for (int j = EC - 1; j >= 0; --j)
@@ -924,29 +957,6 @@ __global__ void __launch_bounds__(PairCfg<NP, RES>::kThreads, 1)
                 }
             }
             if (!ok) break;
-            if (SCR) {
-                // candidates of this row among this group's columns: every column of a kept
-                // tile whose minimum is still inside the final window (up to four)
-                const float T = fminf(scr_global_min(pub + r, tag, best) + W, kScreenMax);
-                if (lost <= T) over = true;  // a dropped tile may hold a candidate
-                int32_t c0 = -1, c1 = -1, c2 = -1, c3 = -1;
-                int cnt = 0;
-                if (em0 <= T)
-                    scr_emit((static_cast<uint64_t>(eh0) << 32) | el0, et0 * kBN + g * EC, cnt,
-                             c0, c1, c2, c3, over);
-                if (em1 <= T)
-                    scr_emit((static_cast<uint64_t>(eh1) << 32) | el1, et1 * kBN + g * EC, cnt,
-                             c0, c1, c2, c3, over);
-                if (em2 <= T)
-                    scr_emit((static_cast<uint64_t>(eh2) << 32) | el2, et2 * kBN + g * EC, cnt,
-                             c0, c1, c2, c3, over);
-                if (row < N) {
-                    const int4 o = over ? make_int4(kCandOverflow, -1, -1, -1)
-                                        : make_int4(c0, c1, c2, c3);
-                    *reinterpret_cast<int4 *>(cand + row * kCandPerRow + g * 4) = o;
-                }
-                continue;
-            }
             const uint32_t slot = mbi & 1u;
             const uint32_t spar = (mbi >> 1) & 1u;
             if (g > 0) {
@@ -1060,7 +1070,7 @@ template <int NP, bool RES, bool SCR>
 cudaError_t launch_assign_pair_cfg(const AssignArgs &a, const CUtensorMap (&tA)[2],
                                    const CUtensorMap (&tB)[2], const CUtensorMap &tC,
                                    int max_pairs, cudaStream_t st) {
-    using Cfg = PairCfg<NP, RES>;
+    using Cfg = PairCfg<NP, RES, SCR ? 1 : 4>;
     const int64_t nmb = ceil_div(a.N, 2 * kBM);
     const int pairs = static_cast<int>(nmb < max_pairs ? nmb : max_pairs);
     cudaLaunchConfig_t cfg = {};
@@ -1087,7 +1097,7 @@ cudaError_t launch_assign_pair_cfg(const AssignArgs &a, const CUtensorMap (&tA)[
 // persistent grid must not exceed it, or part of it would wait for a second wave).
 template <int NP, bool RES, bool SCR>
 int max_resident_pairs() {
-    using Cfg = PairCfg<NP, RES>;
+    using Cfg = PairCfg<NP, RES, SCR ? 1 : 4>;
     static int cached[64] = {0};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;

@@ -30,10 +30,11 @@ constexpr int kUpdMaxRows = 256;      // largest chunk
 constexpr int64_t kUpdTargetWarps = 148 * 64;  // enough warps to cover the GPU twice
 
 // ----------------------------------------------------------------- screening (fp32)
-// The single-product pass writes, per row, four candidate columns for each of the four
-// column groups of a tile (unused slots -1; a group that ran out of room writes
-// kCandOverflow in its first slot and the row goes to the three-product pass).
+// The single-product pass writes, per row, up to kCandPerRow candidate columns (unused
+// slots -1; a row whose list ran out of room has kCandOverflow in its first slot and goes
+// to the three-product pass).
 constexpr int kCandPerRow = 16;
+constexpr int kScreenSlots = kCandPerRow;  // candidate columns the screening pass keeps
 constexpr int32_t kCandOverflow = -2;
 // Screened values at or above this are never candidates: padding centroids (whose first
 // norm piece is the largest finite bf16, about 3.39e38) lie above it, and real data whose

@@ -338,16 +338,5 @@ __device__ __forceinline__ float fmin3(float a, float b, float c) {
     return r;
 }
 
-// 64-bit shared-memory load and store with relaxed CTA-scope semantics: single-copy
-// atomic, so a reader sees either the old or the new 64-bit value, never a mix.
-__device__ __forceinline__ void st_relaxed_u64(uint64_t *p, uint64_t v) {
-    asm volatile("st.relaxed.cta.shared.b64 [%0], %1;" ::"r"(smem_u32(p)), "l"(v) : "memory");
-}
-__device__ __forceinline__ uint64_t ld_relaxed_u64(const uint64_t *p) {
-    uint64_t v;
-    asm volatile("ld.relaxed.cta.shared.b64 %0, [%1];" : "=l"(v) : "r"(smem_u32(p)) : "memory");
-    return v;
-}
-
 }  // namespace ptx
 }  // namespace fk
