@@ -133,9 +133,9 @@ __device__ __forceinline__ float min64(const float (&v)[64]) {
 
 // Screening: add the columns base + bit of `mask` (screened values >= m, the minimum of
 // their chunk) to a row's candidate list.  A free slot holds +inf.  When the list is full,
-// the entry with the largest bound gives way (or the new column, if its bound is the
-// largest) and that bound is remembered in `lost`: the row overflows if it is still inside
-// the final window.
+// the entry with the largest bound gives way (or the new column, if its bound is not
+// smaller) and the smallest bound ever dropped is kept in `lost`: the row overflows if it
+// is still inside the final window.
 template <int KS>
 __device__ __forceinline__ void scr_insert(uint32_t mask, int base, float m, float (&lb)[KS],
                                            int (&cc)[KS], float &lost) {
@@ -155,20 +155,20 @@ __device__ __forceinline__ void scr_insert(uint32_t mask, int base, float m, flo
         float mx = lb[0];
 #pragma unroll
         for (int t = 1; t < KS; ++t) mx = fmaxf(mx, lb[t]);
-        if (m < mx) {
-            bool done = false;
-#pragma unroll
-            for (int t = 0; t < KS; ++t) {
-                if (!done && lb[t] == mx) {
-                    lb[t] = m;
-                    cc[t] = col;
-                    done = true;
-                }
-            }
-            lost = fminf(lost, mx);
-        } else {
-            lost = fminf(lost, m);
+        if (!(m < mx)) {  // full of bounds <= m: every remaining column of the chunk
+            lost = fminf(lost, m);  // (same bound m) would be dropped, so drop them at once
+            return;
         }
+        bool done = false;
+#pragma unroll
+        for (int t = 0; t < KS; ++t) {
+            if (!done && lb[t] == mx) {
+                lb[t] = m;
+                cc[t] = col;
+                done = true;
+            }
+        }
+        lost = fminf(lost, mx);
     }
 }
 
@@ -877,7 +877,10 @@ __global__ void __launch_bounds__(PairCfg<NP, RES, SCR ? 1 : 4>::kThreads, 1)
                         if (lane == 0) ptx::mbar_arrive_cluster(tempty_c + acc * 8);
                     }
                     const float m = min64(v);
-                    if (m <= best + W) {  // this chunk has columns inside the window
+                    // a chunk with columns inside the window; a chunk no better than a column
+                    // already dropped cannot matter (if the final window reaches that column
+                    // the row overflows anyway; if not, neither does this chunk)
+                    if (m <= best + W && m < lost) {
                         if (m < best) {
                             best = m;
                             const float T0 = fminf(best + W, kScreenMax);

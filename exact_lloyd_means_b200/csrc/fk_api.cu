@@ -121,7 +121,9 @@ fk_status run_assign(const void *planes, int nplanes, int64_t lda, int64_t N, in
                      float *mind, cudaStream_t st, const float *X32 = nullptr,
                      const float *C = nullptr, bool allow_screen = true,
                      bool *screened = nullptr, cudaEvent_t ev_mma0 = nullptr,
-                     cudaEvent_t ev_mma1 = nullptr) {
+                     cudaEvent_t ev_mma1 = nullptr, int64_t probe_rows = 0) {
+    // probe_rows > 0: only the screening pass and re-ranking over the first probe_rows rows
+    // (if the screened route applies), counting the rows that would need the fallback
     if (screened) *screened = false;
     AssignArgs a{};
     a.a_planes = planes;
@@ -141,7 +143,9 @@ fk_status run_assign(const void *planes, int nplanes, int64_t lda, int64_t N, in
     a.mind = mind;
     a.err = ws_ptr<uint32_t>(ws, L.err);
     a.wait_ns = kDefaultWaitNs;
-    if (allow_screen && nplanes == 2 && L.dp >= kScreenMinD && C != nullptr &&
+    const bool screen_pays =
+        L.dp >= kScreenMinD || static_cast<int64_t>(K) * L.dp >= kScreenMinKD;
+    if (allow_screen && nplanes == 2 && screen_pays && C != nullptr &&
         xnorm != nullptr && lda == L.dp && d % 4 == 0 && aligned(C, 16) &&
         (X32 == nullptr || aligned(X32, 16)) && assign_can_screen(N, a.dp, a.Kp)) {
         ScreenBufs sb;
@@ -151,10 +155,14 @@ fk_status run_assign(const void *planes, int nplanes, int64_t lda, int64_t N, in
         sb.fblab = ws_ptr<int32_t>(ws, L.fblab);
         sb.xsfb = ws_ptr<uint16_t>(ws, L.xsfb);
         sb.cmax2 = ws_ptr<float>(ws, L.cmax2);
-        FK_TRY_CUDA(launch_assign_screened(a, X32, C, sb, st, ev_mma0, ev_mma1));
+        if (probe_rows > 0)
+            FK_TRY_CUDA(launch_screen_probe(a, N < probe_rows ? N : probe_rows, X32, C, sb, st));
+        else
+            FK_TRY_CUDA(launch_assign_screened(a, X32, C, sb, st, ev_mma0, ev_mma1));
         if (screened) *screened = true;
         return FK_OK;
     }
+    if (probe_rows > 0) return FK_OK;
     if (ev_mma0) FK_TRY_CUDA(cudaEventRecord(ev_mma0, st));
     FK_TRY_CUDA(launch_assign(a, st));
     if (ev_mma1) FK_TRY_CUDA(cudaEventRecord(ev_mma1, st));
@@ -392,7 +400,6 @@ fk_status fk_lloyd(const void *X, fk_dtype dtype, int64_t N, int d, int K, fk_me
     if (niter > 0 &&
         (s = prepare_x(Xp, dtype, N, d, L, ws, xnorm, st, &planes, &nplanes, &lda)) != FK_OK)
         return fail(s);
-    if (!rec()) return fail(FK_ERR_CUDA);
 
     float *Ccur = C, *Cnext = ws_ptr<float>(ws, L.calt);
     int32_t *cnt = counts ? counts : ws_ptr<int32_t>(ws, L.cnt);
@@ -402,6 +409,30 @@ fk_status fk_lloyd(const void *X, fk_dtype dtype, int64_t N, int d, int K, fk_me
     int copied = 0;
     bool allow_screen = true;
     int nscreened = 0;
+    if (niter > 0 && dtype == FK_F32) {
+        // Where the screened route applies, try it first on a sample of the rows with the
+        // initial centroids and read how many would need the three-product pass (a single
+        // host synchronisation per call); screen the call only if few would.
+        bool probed = false;
+        if (launch_prep_centroids(Ccur, K, d, L.Kp, L.dp, dtype, ws_ptr<uint16_t>(ws, L.cs),
+                                  ws_ptr<float>(ws, L.cn), cused, ws_ptr<uint16_t>(ws, L.caug),
+                                  st) != cudaSuccess)
+            return fail(FK_ERR_CUDA);
+        if ((s = run_assign(planes, nplanes, lda, N, d, K, L, ws, labels, xnorm, nullptr, st,
+                            static_cast<const float *>(Xp), Ccur, true, &probed, nullptr,
+                            nullptr, kScreenProbeRows)) != FK_OK)
+            return fail(s);
+        if (probed) {
+            uint32_t nfb = 0;
+            if (cudaMemcpyAsync(&nfb, ws_ptr<uint32_t>(ws, L.nfb), sizeof(nfb),
+                                cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+                cudaStreamSynchronize(st) != cudaSuccess)
+                return fail(FK_ERR_CUDA);
+            const int64_t n = N < kScreenProbeRows ? N : kScreenProbeRows;
+            allow_screen = static_cast<int64_t>(nfb) * kScreenMaxFallback <= n;
+        }
+    }
+    if (!rec()) return fail(FK_ERR_CUDA);  // end of the once-per-call setup
     for (int t = 0; t < niter; ++t) {
         if (launch_prep_centroids(Ccur, K, d, L.Kp, L.dp, dtype, ws_ptr<uint16_t>(ws, L.cs),
                                   ws_ptr<float>(ws, L.cn), cused, ws_ptr<uint16_t>(ws, L.caug),
@@ -416,16 +447,6 @@ fk_status fk_lloyd(const void *X, fk_dtype dtype, int64_t N, int d, int K, fk_me
                             allow_screen, &screened, m0, m1)) != FK_OK)
             return fail(s);
         nscreened += screened ? 1 : 0;
-        if (screened && t == 0 && niter > 1) {
-            // one look (a single host synchronisation per call) at how many rows needed
-            // the three-product pass; if too many, the plain three-product pass is cheaper
-            uint32_t nfb = 0;
-            if (cudaMemcpyAsync(&nfb, ws_ptr<uint32_t>(ws, L.nfb), sizeof(nfb),
-                                cudaMemcpyDeviceToHost, st) != cudaSuccess ||
-                cudaStreamSynchronize(st) != cudaSuccess)
-                return fail(FK_ERR_CUDA);
-            allow_screen = static_cast<int64_t>(nfb) * kScreenMaxFallback <= N;
-        }
         if (!rec()) return fail(FK_ERR_CUDA);
         const int32_t *skeys = nullptr, *perm = nullptr;
         if (launch_sort_csr(labels, N, K, L.sp, ws_ptr<int32_t>(ws, L.keys0),

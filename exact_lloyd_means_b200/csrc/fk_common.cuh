@@ -40,14 +40,17 @@ constexpr int32_t kCandOverflow = -2;
 // norm piece is the largest finite bf16, about 3.39e38) lie above it, and real data whose
 // ||c||^2 + 2|x.c| reaches it is outside the supported range.
 constexpr float kScreenMax = 1e38f;
-// Screening pays where the three-product pass is long per tile: from d = 256 on.  Below,
-// a tile of 256 centroids is so short (9 single-product MMA steps at d = 128) that the
-// candidate bookkeeping in the epilogue, not the tensor cores, sets the pace.
+// Screening pays where the tensor-core work per row is large next to its fixed per-row
+// costs (candidate list, re-ranking): from d = 256 on, and below that from K * d = 2^22
+// (measured on B200: d = 128 wins from K = 32768, loses at K <= 8192; d = 192, K = 4096
+// breaks even).
 constexpr int kScreenMinD = 256;
-// fk_lloyd stops screening for the rest of a call when more than 1/kScreenMaxFallback of
-// the rows needed the three-product pass in its first iteration (mixtures whose heavy
-// components hold many nearly equidistant centroids).
+constexpr int64_t kScreenMinKD = int64_t(1) << 22;
+// fk_lloyd screens a call only if, on a sample of kScreenProbeRows rows with the initial
+// centroids, at most 1/kScreenMaxFallback of them would need the three-product pass
+// (mixtures whose heavy components hold many nearly equidistant centroids do not qualify).
 constexpr int kScreenMaxFallback = 4;
+constexpr int64_t kScreenProbeRows = 2 * 128 * 148;
 
 // Objective slots kept on the device by fk_lloyd before a copy to the host.
 constexpr int kObjRing = 4096;
@@ -230,6 +233,10 @@ struct ScreenBufs {
     uint16_t *xsfb;    // [2][N][dp]
     float *cmax2;      // [1]
 };
+// The screening pass and re-ranking over the first n_probe rows, counting in sb.nfb the
+// rows that would need the three-product pass (their labels are not final).
+cudaError_t launch_screen_probe(const AssignArgs &a, int64_t n_probe, const float *X32,
+                                const float *C, const ScreenBufs &sb, cudaStream_t st);
 cudaError_t launch_assign_screened(const AssignArgs &a, const float *X32, const float *C,
                                    const ScreenBufs &sb, cudaStream_t st,
                                    cudaEvent_t ev_mma0 = nullptr,

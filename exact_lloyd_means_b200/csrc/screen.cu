@@ -263,3 +263,33 @@ cudaError_t launch_assign_screened(const AssignArgs &a, const float *X32, const 
 }
 
 }  // namespace fk
+
+namespace fk {
+
+cudaError_t launch_screen_probe(const AssignArgs &a, int64_t n_probe, const float *X32,
+                                const float *C, const ScreenBufs &sb, cudaStream_t st) {
+    // the screening pass and the re-ranking over the first n_probe rows only; the rows
+    // that would need the three-product pass are counted in sb.nfb, not assigned
+    window_kernel<<<1, 1024, 0, st>>>(a.cn, a.K, sb.cmax2, sb.nfb);
+    note_launch();
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    AssignArgs s1 = a;
+    s1.N = n_probe;
+    s1.a_nplanes = 1;
+    s1.cand = sb.cand;
+    s1.cmax2 = sb.cmax2;
+    s1.mind = nullptr;
+    s1.best = nullptr;
+    s1.n_dev = nullptr;
+    if ((e = launch_assign(s1, st)) != cudaSuccess) return e;
+    const uint16_t *xhi = static_cast<const uint16_t *>(a.a_planes);
+    const int64_t rr_blocks = ceil_div(n_probe, 8);
+    const int rgrid = static_cast<int>(rr_blocks < 148 * 16 ? rr_blocks : 148 * 16);
+    rerank_kernel<<<rgrid, 256, 0, st>>>(X32, xhi, xhi + a.N * a.lda, a.lda, C, n_probe, a.d,
+                                         a.K, sb.cand, a.labels, nullptr, sb.nfb, sb.fbrows);
+    note_launch();
+    return cudaGetLastError();
+}
+
+}  // namespace fk

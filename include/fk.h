@@ -89,7 +89,8 @@ typedef enum fk_metric {
 /* Per-phase device time of an fk_lloyd call, summed over its iterations (CUDA events
  * recorded on the caller's stream around each phase). */
 typedef struct fk_timing {
-    double ms_setup;   /* once per call: normalisation (cosine) and the fp32 split of X */
+    double ms_setup;   /* once per call: normalisation (cosine), the fp32 split of X and
+                          the screening probe                                          */
     double ms_prep;    /* per iteration: centroid norms and operand preparation        */
     double ms_assign;  /* per iteration: the whole assignment (every kernel of it)     */
     double ms_sort;    /* per iteration: radix sort of labels -> perm + CSR offsets   */
@@ -152,7 +153,8 @@ FK_API fk_status fk_centroid_norms(const float *C, int K, int d, fk_dtype dtype,
  * pass over X; fk_lloyd does this once per call instead of once per iteration); callers
  * that assign the same points repeatedly split once with fk_split_points and pass the
  * planes with FK_BF16X2.
- * Screened route (fp32 points, N >= 18,944 rows, C 16-byte aligned): one bf16 product
+ * Screened route (fp32 points, N >= 18,944 rows, d >= 256 or K * d >= 2^22, C 16-byte
+ * aligned): one bf16 product
  * per term finds, for every row, the centroids within a proven bound of the nearest; their
  * distances (fp64, difference form) pick the label, and rows with more such
  * centroids than the kernel keeps are assigned by the three-product form.  Labels are the

@@ -341,8 +341,8 @@ def test_assign_pre_split_points_equals_fp32_assign(N, d, K):
     assert torch.equal(l1, l2)
 
 
-# Screened fp32 assignment: for fp32 points with d >= 256 at CTA-pair sizes
-# (N >= 2 * 128 * 148 / 2) the single-product pass keeps the columns inside a proven error window, the candidates
+# Screened fp32 assignment: for fp32 points with d >= 256 or K * d >= 2^22 at CTA-pair
+# sizes (N >= 2 * 128 * 148 / 2) the single-product pass keeps the columns inside a proven error window, the candidates
 # are re-ranked exactly, and rows whose candidates do not fit are assigned by the
 # three-product pass.  These cases drive each branch: ordinary mixtures (few candidates),
 # components that received several initial centroids (several candidates), exact
@@ -354,6 +354,7 @@ SCREEN_CASES = [
     ("uniform", 50001, 320, 4100, "equal", 0.2),
     ("normal", 40000, 256, 2000, "zipf", 0.15),
     ("normal", 20000, 1032, 700, "equal", 0.3),
+    ("normal", 40000, 128, 32768, "equal", 0.25),
 ]
 
 
