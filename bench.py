@@ -382,6 +382,34 @@ def fk_arm(args, spec, rank, world, dist):
            "gpu_launches": launches, "final_objective": objs[-1],
            "clocks": clocks}
 
+    # the inverted lists of the finished clustering (LEANN guide, "工作原理"): CSR offsets,
+    # row ids in cell order and the points gathered in that order; HBM-bound, timed apart
+    # from the Lloyd steps with CUDA events on this stream
+    if not sharded:
+        offs = torch.empty(spec.k + 1, dtype=torch.int32, device=dev)
+        rids = torch.empty(spec.n, dtype=torch.int32, device=dev)
+        Xl = torch.empty_like(X)
+        for _ in range(2):
+            fk.fk_ivf_lists(X, labels, spec.k, offs, rids, ws, X_lists=Xl)
+        torch.cuda.synchronize()
+        g0 = torch.cuda.Event(enable_timing=True)
+        g1 = torch.cuda.Event(enable_timing=True)
+        g0.record()
+        for _ in range(5):
+            fk.fk_ivf_lists(X, labels, spec.k, offs, rids, ws, X_lists=Xl)
+        g1.record()
+        torch.cuda.synchronize()
+        ivf_ms = g0.elapsed_time(g1) / 5
+        # algorithmic bytes: the rows read and written once, plus the sort's label, key and
+        # id traffic (about 20 B per point per radix pass)
+        passes = max(1, -(-max(1, (spec.k - 1).bit_length()) // 11))
+        ivf_bytes = 2.0 * spec.n * spec.d * e_bytes + 20.0 * spec.n * passes
+        out["ivf_lists"] = {"ms": ivf_ms, "achieved_gbs": ivf_bytes / (ivf_ms / 1e3) / 1e9,
+                            "peak_gbs": peaks["hbm_gbs"],
+                            "frac": ivf_bytes / (ivf_ms / 1e3) / 1e9 / peaks["hbm_gbs"],
+                            "algorithmic_bytes": ivf_bytes}
+        del Xl
+
     # end to end through the public API with host buffers
     if not args.no_e2e:
         Xh = torch.empty(X.shape, dtype=X.dtype, pin_memory=True)

@@ -510,6 +510,33 @@ fk_status fk_lloyd(const void *X, fk_dtype dtype, int64_t N, int d, int K, fk_me
     return static_cast<fk_status>(code);
 }
 
+fk_status fk_ivf_lists(const void *X, fk_dtype dtype, int64_t N, int d, int K,
+                       const int32_t *labels, int32_t *offsets, int32_t *row_ids,
+                       void *X_lists, void *ws, size_t ws_bytes, fk_stream_t stream) {
+    fk_status s = validate_shape(N, d, K, dtype, FK_L2);
+    if (s != FK_OK) return s;
+    if (!X || !labels || !offsets || !row_ids) return FK_ERR_INVALID_ARG;
+    const size_t xbytes = static_cast<size_t>(N) * d * (dtype == FK_F32 ? 4 : 2);
+    if (X_lists && overlap(X, xbytes, X_lists, xbytes)) return FK_ERR_INVALID_ARG;
+    if (!aligned(X, 16) || !aligned(labels, 4) || !aligned(offsets, 4) ||
+        !aligned(row_ids, 4) || (X_lists && !aligned(X_lists, 16)))
+        return FK_ERR_UNSUPPORTED;
+    const WsLayout L = ws_layout(N, d, K, dtype, FK_L2);
+    if ((s = check_ws(ws, ws_bytes, L)) != FK_OK) return s;
+    if ((s = check_device()) != FK_OK) return s;
+    cudaStream_t st = stream;
+    const int32_t *skeys = nullptr, *perm = nullptr;
+    FK_TRY_CUDA(launch_sort_csr(labels, N, K, L.sp, ws_ptr<int32_t>(ws, L.keys0),
+                                ws_ptr<int32_t>(ws, L.keys1), ws_ptr<int32_t>(ws, L.vals0),
+                                ws_ptr<int32_t>(ws, L.vals1), row_ids,
+                                ws_ptr<uint32_t>(ws, L.hist), ws_ptr<uint32_t>(ws, L.dtot),
+                                offsets, &skeys, &perm, ws_ptr<uint32_t>(ws, L.err), st));
+    if (X_lists)
+        FK_TRY_CUDA(launch_gather_rows(X, N, static_cast<int64_t>(d) * (dtype == FK_F32 ? 4 : 2),
+                                       row_ids, X_lists, st));
+    return FK_OK;
+}
+
 fk_status fk_update_partial(const void *X, fk_dtype dtype, int64_t N, int d, int K,
                             const int32_t *labels, const float *C_old, double *sums,
                             int32_t *counts, int32_t *offsets, double *objective, void *ws,

@@ -253,6 +253,8 @@ cudaError_t launch_update(const void *X, fk_dtype dtype, int64_t N, int d, int K
                           double *pieces_b, int32_t *pkeys_b, double *jpart,
                           double *objective, uint32_t *err, double *sums_out,
                           cudaStream_t st);
+cudaError_t launch_gather_rows(const void *X, int64_t N, int64_t row_bytes,
+                               const int32_t *row_ids, void *out, cudaStream_t st);
 cudaError_t launch_finalize_shards(const double *sums, const int64_t *cnts, const double *objs,
                                    int W, int K, int d, const float *C_old, float *C_new,
                                    int64_t *counts, double *objective, cudaStream_t st);

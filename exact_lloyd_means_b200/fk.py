@@ -66,12 +66,13 @@ _sig("fk_assign_noalloc", [_vp, _int, _i64, _int, _vp, _int, _vp, _vp])
 _sig("fk_update_partial", [_vp, _int, _i64, _int, _int, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz,
                            _vp])
 _sig("fk_finalize_shards", [_vp, _vp, _vp, _int, _int, _int, _vp, _vp, _vp, _vp, _vp])
+_sig("fk_ivf_lists", [_vp, _int, _i64, _int, _int, _vp, _vp, _vp, _vp, _vp, _sz, _vp])
 
 EXPORTED = ["fk_status_string", "fk_version", "fk_workspace_size", "fk_normalize_rows",
             "fk_centroid_norms", "fk_assign", "fk_update", "fk_lloyd",
             "fk_get_device_error", "fk_selftest_timeout", "fk_assign_noalloc",
             "fk_update_partial", "fk_finalize_shards", "fk_split_points",
-            "fk_launch_count"]
+            "fk_launch_count", "fk_ivf_lists"]
 
 # Bytes of the static device array fk_assign_noalloc takes its scratch from.
 NOALLOC_SCRATCH_BYTES = 8 << 20
@@ -323,3 +324,18 @@ def fk_finalize_shards(sums: torch.Tensor, counts_w: torch.Tensor, C_old: torch.
                                    _opt(counts, "counts", torch.int64, (K,)),
                                    _opt(objective, "objective", torch.float64, (1,)),
                                    _stream(stream)), "fk_finalize_shards")
+
+
+def fk_ivf_lists(X: torch.Tensor, labels: torch.Tensor, K: int, offsets: torch.Tensor,
+                 row_ids: torch.Tensor, ws: torch.Tensor, X_lists: torch.Tensor | None = None,
+                 stream=None):
+    """Inverted lists of a clustering: CSR offsets per cell, row ids in cell order and
+    (optionally) the points gathered in that order."""
+    N, d = X.shape
+    _check(_lib.fk_ivf_lists(_dev(X, "X"), _dtype_code(X), N, d, K,
+                             _dev(labels, "labels", torch.int32, (N,)),
+                             _dev(offsets, "offsets", torch.int32, (K + 1,)),
+                             _dev(row_ids, "row_ids", torch.int32, (N,)),
+                             _opt(X_lists, "X_lists", X.dtype, (N, d)),
+                             _dev(ws, "ws", torch.uint8), ws.numel(), _stream(stream)),
+           "fk_ivf_lists")

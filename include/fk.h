@@ -221,6 +221,20 @@ FK_API fk_status fk_finalize_shards(const double *sums, const int64_t *counts_w,
                                     const float *C_old, float *C_new, int64_t *counts,
                                     double *objective, fk_stream_t stream);
 
+/* Inverted lists of a clustering (LEANN FlashLib guide, "工作原理": an IVF index keeps,
+ * per cell, the ids of its points in CSR form and the points of a cell contiguous).
+ *   offsets[k] .. offsets[k+1] - 1 : the positions of cell k (offsets: K+1 int32)
+ *   row_ids[p] : the point at position p, stable order by (label, index) (N int32)
+ *   X_lists[p] : X[row_ids[p]], same dtype and row length as X (N x d; optional, NULL to
+ *                skip the gather)
+ * X (fp32 or bf16, N x d, 16-byte aligned rows as for fk_update) and labels (values in
+ * [0, K)) are device pointers; so are the outputs, which must not overlap X.  Workspace
+ * as for fk_update.  Asynchronous; a label outside [0, K) is reported by
+ * fk_get_device_error. */
+FK_API fk_status fk_ivf_lists(const void *X, fk_dtype dtype, int64_t N, int d, int K,
+                              const int32_t *labels, int32_t *offsets, int32_t *row_ids,
+                              void *X_lists, void *ws, size_t ws_bytes, fk_stream_t stream);
+
 /* Scratch held by fk_assign_noalloc: one static device array of this many bytes. */
 #define FK_NOALLOC_SCRATCH_BYTES (8u << 20)
 

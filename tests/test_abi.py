@@ -111,3 +111,15 @@ def test_pre_split_dtype_is_assign_only(fk):
     assert lib.fk_split_points(None, 100, 8, 256, None) == fk.FK_ERR_INVALID_ARG
     assert lib.fk_split_points(256, 100, 6, 256, None) == fk.FK_ERR_UNSUPPORTED
     assert lib.fk_split_points(8, 100, 8, 256, None) == fk.FK_ERR_UNSUPPORTED
+
+
+def test_ivf_lists_host_checks(fk):
+    lib = fk._lib
+    big = 1 << 30
+    assert lib.fk_ivf_lists(None, 0, 100, 8, 4, 256, 256, 256, None, 256, big, None) == \
+        fk.FK_ERR_INVALID_ARG
+    # X_lists overlapping X
+    assert lib.fk_ivf_lists(4096, 0, 100, 8, 4, 256, 256, 256, 4096 + 64, 256, big, None) == \
+        fk.FK_ERR_INVALID_ARG
+    assert lib.fk_ivf_lists(4096, 0, 100, 8, 4, 256, 256, 256, None, 256, 10, None) == \
+        fk.FK_ERR_WORKSPACE

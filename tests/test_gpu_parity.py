@@ -400,3 +400,57 @@ def test_screened_lloyd_lockstep_heavy_components():
         Cm = torch.as_tensor(C_master[t], dtype=torch.float32)
         lab, _ = gpu_assign(Xg, Cm.to(DEV))
         assert label_mismatches(lab, ref["labels"][t], ref["ties"][t]) == 0, t
+
+
+def test_screened_lloyd_deterministic_and_resumable():
+    """The screened route gives the same bits run to run (its fallback queue's order
+    varies with scheduling, the labels do not), and 2 + 2 iterations equal 4."""
+    X, _, _ = gaussian_mixture(40000, 256, 600, centers="normal", sigma=0.3, seed=41)
+    C0 = X[init_indices(40000, 600, 41)].float().contiguous()
+    m = fk()
+    Xg = X.to(DEV)
+    ws = m.workspace(40000, 256, 600, torch.float32, "l2")
+
+    def run(C, n):
+        labels = torch.empty(40000, dtype=torch.int32, device=DEV)
+        objs, tm = m.fk_lloyd(Xg, C, n, labels, ws, timing=True)
+        assert tm["screened"] == n  # the screened route was taken
+        return C, labels, objs
+
+    a = run(C0.to(DEV).clone(), 4)
+    b = run(C0.to(DEV).clone(), 4)
+    assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1]) and a[2] == b[2]
+    c = run(C0.to(DEV).clone(), 2)
+    d = run(c[0].clone(), 2)
+    assert torch.equal(d[0], a[0]) and torch.equal(d[1], a[1]) and d[2] == a[2][2:]
+
+
+IVF_CASES = [(1000, 64, 10, "equal"), (70001, 128, 1024, "zipf"), (20000, 768, 300, "equal"),
+             (5000, 8, 1, "equal"), (3000, 1032, 2500, "equal")]
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("N,d,K,weights", IVF_CASES)
+def test_ivf_lists_match_oracle(N, d, K, weights, dtype):
+    """fk_ivf_lists: offsets and row ids bit-exact against the oracle's stable CSR, and the
+    gathered rows bit-exact against X[row_ids] (empty cells included)."""
+    m = fk()
+    X, comp, _ = gaussian_mixture(N, d, K, centers="normal", sigma=0.3, weights=weights,
+                                  dtype=dtype, seed=N + K)
+    lab = comp.numpy().astype(np.int32)
+    _, off_ref, perm_ref = oracle.csr(lab, K)
+    Xg = X.to(DEV)
+    offsets = torch.full((K + 1,), -1, dtype=torch.int32, device=DEV)
+    row_ids = torch.full((N,), -1, dtype=torch.int32, device=DEV)
+    X_lists = torch.empty_like(Xg)
+    ws = m.workspace(N, d, K, Xg.dtype, "l2")
+    m.fk_ivf_lists(Xg, torch.as_tensor(lab).to(DEV), K, offsets, row_ids, ws, X_lists=X_lists)
+    assert m.fk_get_device_error(ws) == m.FK_OK
+    assert (offsets.cpu().numpy() == off_ref).all()
+    assert (row_ids.cpu().numpy() == perm_ref).all()
+    assert torch.equal(X_lists.cpu().view(torch.int16 if dtype == "bf16" else torch.int32),
+                       X[perm_ref].view(torch.int16 if dtype == "bf16" else torch.int32))
+    # without the gather: the same ids
+    row2 = torch.empty_like(row_ids)
+    m.fk_ivf_lists(Xg, torch.as_tensor(lab).to(DEV), K, offsets, row2, ws)
+    assert torch.equal(row2, row_ids)
