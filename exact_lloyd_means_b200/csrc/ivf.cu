@@ -9,19 +9,25 @@
 namespace fk {
 namespace {
 
-// X_lists[i] = X[row_ids[i]]: one warp per row, 16-byte vectors (rows are whole multiples
-// of 16 bytes).  Reads and writes are contiguous within a row; rows are read in cell order.
+// X_lists[i] = X[row_ids[i]]: rows of 16-byte vectors, each copied by a group of G lanes
+// (G = 32, or 16 for rows of at most 16 vectors, so that short rows keep the whole warp
+// busy).  Reads and writes are contiguous within a row; rows are read in cell order.
 __global__ void gather_rows_kernel(const uint4 *__restrict__ X, int64_t N, int vec_per_row,
                                    const int32_t *__restrict__ row_ids,
                                    uint4 *__restrict__ out) {
     const int lane = threadIdx.x & 31;
+    const int G = vec_per_row <= 16 ? 16 : 32;
+    const int rows_per_warp = 32 / G;
+    const int sub = lane % G;
     const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
     const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
-    for (int64_t i = warp; i < N; i += nwarps) {
+    for (int64_t i0 = warp * rows_per_warp; i0 < N; i0 += nwarps * rows_per_warp) {
+        const int64_t i = i0 + lane / G;
+        if (i >= N) continue;
         const int64_t src = row_ids[i];
         const uint4 *s = X + src * vec_per_row;
         uint4 *t = out + i * vec_per_row;
-        for (int v = lane; v < vec_per_row; v += 32) t[v] = s[v];
+        for (int v = sub; v < vec_per_row; v += G) t[v] = s[v];
     }
 }
 

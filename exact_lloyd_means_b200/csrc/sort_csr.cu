@@ -7,16 +7,18 @@
 //
 // A stable least-significant-digit radix sort with digits of up to 11 bits (one pass for
 // K <= 2048, two for K <= 2^22), written without atomics:
-//   upsweep   : each block of 4096 keys counts its digits; every warp keeps a private
-//               histogram in shared memory that only the elected leader of each group of
-//               equal digits (__match_any_sync) updates, so no two lanes write one counter;
+//   upsweep   : each block of 4096 keys counts its digits into per-warp histograms in
+//               shared memory (shared-memory atomic adds: the counts do not depend on
+//               their order);
 //   scan      : one block per digit scans the per-block counts (digit-major order) and
 //               stores the digit total;
-//   downsweep : each block recounts, turns warp counts into exclusive offsets (digits in
-//               order, then blocks in order, then warps in order) and scatters every key
-//               to base + rank, rank = #equal digits before it in the warp (popc of the
-//               match mask below the lane).  Keys are visited in index order, so the sort
-//               is stable and the output is unique.
+//   downsweep : each block recounts, turns warp counts into offsets within its tile
+//               (digits in order, then warps in order), places every key in shared memory
+//               at offset + rank, rank = #equal digits before it in the warp (popc of the
+//               match mask below the lane), then writes each digit's run of the tile to
+//               its global place (digits, then blocks in order) with consecutive threads
+//               on consecutive addresses.  Keys are visited in index order, so the sort is
+//               stable and the output is unique.
 // offsets[k] = first sorted position whose key is >= k, written once per k.
 #include "fk_common.cuh"
 
@@ -32,29 +34,43 @@ __device__ __forceinline__ uint32_t lanemask_lt() {
 }
 
 // Check labels (first pass) and count digits of one 4096-key tile into per-warp
-// histograms wh[kWarps][bins].
+// histograms wh[kWarps][bins].  Each thread reads 16 consecutive keys with 16-byte loads
+// and adds them with shared-memory atomics: counts do not depend on the order of the
+// additions, so the result is the same on every run.
 __device__ __forceinline__ void count_tile(const int32_t *__restrict__ keys, int64_t n,
                                            int64_t tile0, int shift, uint32_t mask, int K,
                                            uint32_t *__restrict__ err, int check,
                                            uint32_t *wh, int bins) {
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int warp = threadIdx.x >> 5;
     uint32_t *h = wh + warp * bins;
-    const int64_t base = tile0 + static_cast<int64_t>(warp) * (32 * kSortItems);
-    for (int step = 0; step < kSortItems; ++step) {
-        const int64_t idx = base + step * 32 + lane;
-        const bool valid = idx < n;
-        int key = valid ? keys[idx] : 0;
-        if (check && valid && (key < 0 || key >= K)) {
-            err[1] = 1u;
-            key = key < 0 ? 0 : K - 1;
+    const int64_t start = tile0 + static_cast<int64_t>(threadIdx.x) * kSortItems;
+    // labels need only 4-byte alignment: 16-byte loads only from a 16-byte aligned array
+    // (start is a multiple of 16 keys, so then every load below is aligned)
+    const bool vec = (reinterpret_cast<uintptr_t>(keys) & 15u) == 0u;
+#pragma unroll
+    for (int j = 0; j < kSortItems; j += 4) {
+        const int64_t idx = start + j;
+        int k4[4];
+        if (vec && idx + 3 < n) {
+            const int4 v = *reinterpret_cast<const int4 *>(keys + idx);
+            k4[0] = v.x;
+            k4[1] = v.y;
+            k4[2] = v.z;
+            k4[3] = v.w;
+        } else {
+#pragma unroll
+            for (int t = 0; t < 4; ++t) k4[t] = idx + t < n ? keys[idx + t] : -1;
         }
-        const uint32_t digit = (static_cast<uint32_t>(key) >> shift) & mask;
-        const uint32_t vmask = __ballot_sync(0xffffffffu, valid);
-        if (valid) {
-            const uint32_t peers = __match_any_sync(vmask, digit);
-            if (lane == __ffs(peers) - 1) h[digit] += __popc(peers);
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+            if (idx + t >= n) continue;
+            int key = k4[t];
+            if (key < 0 || key >= K) {
+                if (check) err[1] = 1u;
+                key = key < 0 ? 0 : K - 1;
+            }
+            atomicAdd(&h[(static_cast<uint32_t>(key) >> shift) & mask], 1u);
         }
-        __syncwarp();
     }
 }
 
@@ -124,6 +140,38 @@ __global__ void __launch_bounds__(1024)
     if (threadIdx.x == 0) dtot[blockIdx.x] = total;
 }
 
+// Exclusive scan of cnt[0..bins) into out[0..bins) by one block: every thread sums a
+// contiguous run of entries, one thread scans the run totals, then the runs are filled in.
+__device__ __forceinline__ void block_scan_bins(const uint32_t *cnt, uint32_t *out, int bins,
+                                                uint32_t *part) {
+    const int per = (bins + kSortThreads - 1) / kSortThreads;
+    const int lo = threadIdx.x * per;
+    const int hi = lo + per < bins ? lo + per : bins;
+    uint32_t s = 0;
+    for (int b = lo; b < hi; ++b) s += cnt[b];
+    part[threadIdx.x] = s;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        uint32_t run = 0;
+        for (int t = 0; t < kSortThreads; ++t) {
+            const uint32_t v = part[t];
+            part[t] = run;
+            run += v;
+        }
+    }
+    __syncthreads();
+    uint32_t run = part[threadIdx.x];
+    for (int b = lo; b < hi; ++b) {
+        const uint32_t v = cnt[b];
+        out[b] = run;
+        run += v;
+    }
+    __syncthreads();
+}
+
+// Scatter one 4096-key tile: the keys are first placed in shared memory in digit order
+// (stable: warps, then steps, then lanes follow the index order), then each digit's run is
+// written to its global place with consecutive threads writing consecutive addresses.
 __global__ void __launch_bounds__(kSortThreads)
     downsweep_kernel(const int32_t *__restrict__ kin, const int32_t *__restrict__ vin,
                      int32_t *__restrict__ kout, int32_t *__restrict__ vout, int64_t n,
@@ -132,43 +180,33 @@ __global__ void __launch_bounds__(kSortThreads)
     extern __shared__ uint32_t sm[];
     const int bins = 1 << bits;
     const uint32_t mask = bins - 1;
-    uint32_t *wh = sm;                   // [kWarps][bins]
-    uint32_t *dbase = sm + kWarps * bins;  // [bins] exclusive scan of digit totals
+    uint32_t *wh = sm;                      // [kWarps][bins] counts, then local offsets
+    uint32_t *lstart = wh + kWarps * bins;  // [bins] this tile's digit starts (local)
+    uint32_t *gstart = lstart + bins;       // [bins] where this tile's digit run goes
+    uint32_t *bcnt = gstart + bins;         // [bins] scratch
+    int32_t *skey = reinterpret_cast<int32_t *>(bcnt + bins);  // [kSortTile]
+    int32_t *sval = skey + kSortTile;                           // [kSortTile]
     __shared__ uint32_t part[kSortThreads];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     for (int i = threadIdx.x; i < kWarps * bins; i += blockDim.x) wh[i] = 0;
-    // digit bases: thread t scans a contiguous run of digits, then the runs are combined
-    {
-        const int per = (bins + kSortThreads - 1) / kSortThreads;
-        const int lo = threadIdx.x * per;
-        const int hi = lo + per < bins ? lo + per : bins;
-        uint32_t s = 0;
-        for (int b = lo; b < hi; ++b) s += dtot[b];
-        part[threadIdx.x] = s;
-        __syncthreads();
-        if (threadIdx.x == 0) {
-            uint32_t run = 0;
-            for (int t = 0; t < kSortThreads; ++t) {
-                const uint32_t v = part[t];
-                part[t] = run;
-                run += v;
-            }
-        }
-        __syncthreads();
-        uint32_t run = part[threadIdx.x];
-        for (int b = lo; b < hi; ++b) {
-            dbase[b] = run;
-            run += dtot[b];
-        }
-    }
-    __syncthreads();
+    // global digit bases: exclusive scan of the digit totals
+    block_scan_bins(dtot, gstart, bins, part);
+    for (int b = threadIdx.x; b < bins; b += blockDim.x)
+        gstart[b] += hist[static_cast<int64_t>(b) * nblocks + blockIdx.x];
 
     const int64_t tile0 = static_cast<int64_t>(blockIdx.x) * kSortTile;
     count_tile(kin, n, tile0, shift, mask, K, nullptr, 0, wh, bins);
     __syncthreads();
     for (int b = threadIdx.x; b < bins; b += blockDim.x) {
-        uint32_t run = dbase[b] + hist[static_cast<int64_t>(b) * nblocks + blockIdx.x];
+        uint32_t t = 0;
+        for (int w = 0; w < kWarps; ++w) t += wh[w * bins + b];
+        bcnt[b] = t;
+    }
+    __syncthreads();
+    block_scan_bins(bcnt, lstart, bins, part);
+    for (int b = threadIdx.x; b < bins; b += blockDim.x) {
+        uint32_t run = lstart[b];
         for (int w = 0; w < kWarps; ++w) {
             const uint32_t t = wh[w * bins + b];
             wh[w * bins + b] = run;
@@ -199,10 +237,21 @@ __global__ void __launch_bounds__(kSortThreads)
         __syncwarp();
         if (valid) {
             if (lane == __ffs(peers) - 1) h[digit] += __popc(peers);
-            kout[pos] = key;
-            vout[pos] = val;
+            skey[pos] = key;
+            sval[pos] = val;
         }
         __syncwarp();
+    }
+    __syncthreads();
+
+    const int64_t left = n - tile0;
+    const int cnt = static_cast<int>(left < kSortTile ? left : kSortTile);
+    for (int i = threadIdx.x; i < cnt; i += blockDim.x) {
+        const int32_t key = skey[i];
+        const uint32_t digit = (static_cast<uint32_t>(key) >> shift) & mask;
+        const int64_t g = static_cast<int64_t>(gstart[digit]) + (i - static_cast<int>(lstart[digit]));
+        kout[g] = key;
+        vout[g] = sval[i];
     }
 }
 
@@ -253,7 +302,8 @@ cudaError_t launch_sort_csr(const int32_t *labels, int64_t N, int K, const SortP
     } else {
         const int bins = 1 << sp.bits;
         const size_t up_smem = sizeof(uint32_t) * kWarps * bins;
-        const size_t dn_smem = sizeof(uint32_t) * (kWarps + 1) * bins;
+        const size_t dn_smem =
+            sizeof(uint32_t) * ((kWarps + 3) * bins) + sizeof(int32_t) * 2 * kSortTile;
         static bool attr = false;
         if (!attr) {
             const int maxb = 1 << kSortMaxBits;
@@ -261,7 +311,8 @@ cudaError_t launch_sort_csr(const int32_t *labels, int64_t N, int K, const SortP
                                  static_cast<int>(sizeof(uint32_t) * kWarps * maxb));
             cudaFuncSetAttribute(downsweep_kernel,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 static_cast<int>(sizeof(uint32_t) * (kWarps + 1) * maxb));
+                                 static_cast<int>(sizeof(uint32_t) * (kWarps + 3) * maxb +
+                                                  sizeof(int32_t) * 2 * kSortTile));
             attr = true;
         }
         const int32_t *kin = labels;
