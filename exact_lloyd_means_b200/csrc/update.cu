@@ -282,7 +282,8 @@ __global__ void __launch_bounds__(kRowWarps * 32, 3)
 
 // Level 1, register-gather form, used for bf16 rows: a 128-column slice of a bf16 row is
 // only 256 bytes, too small for one bulk copy per row to pay off.  Lanes load their 8 bytes
-// of each row directly, B = 16 rows per batch, with the next batch in flight in registers
+// of each row directly, B = 8 rows per batch (three blocks per SM: more warps with smaller
+// batches measured faster), with the next batch in flight in registers
 // while the current one is added; the arithmetic is that of seg_rows_kernel.
 template <bool BF16>
 struct RegRowVec;
@@ -301,7 +302,7 @@ struct RegRowVec<false> {
 template <>
 struct RegRowVec<true> {
     using T = uint2;
-    static constexpr int kBatch = 16;
+    static constexpr int kBatch = 8;
     __device__ static void unpack(const uint2 &u, float (&f)[4]) {
         f[0] = __uint_as_float(u.x << 16);
         f[1] = __uint_as_float(u.x & 0xffff0000u);
@@ -312,7 +313,7 @@ struct RegRowVec<true> {
 };
 
 template <bool BF16>
-__global__ void __launch_bounds__(kUpdWarps * 32, 2)
+__global__ void __launch_bounds__(kUpdWarps * 32, 3)
     seg_rows_regs_kernel(const void *__restrict__ X, int64_t N, int d, int R, int64_t nwarps,
                     int dcov, const int32_t *__restrict__ skeys,
                     const int32_t *__restrict__ perm, const int32_t *__restrict__ offsets,
