@@ -458,24 +458,21 @@ __global__ void __launch_bounds__(kUpdWarps * 32, 3)
 // each), one 128-column block per grid.y.  `span` = sorted positions covered by one unit
 // of THIS level.  The group's slot keys are staged in shared memory first and the pieces
 // are read 8 slots at a time, so the loop is not a chain of dependent loads.
-__global__ void __launch_bounds__(kUpdWarps * 32)
-    seg_pieces_kernel(const double *__restrict__ pin, const int32_t *__restrict__ kin,
-                      int64_t nslots_in, double *__restrict__ pout,
-                      int32_t *__restrict__ kout, int64_t nunits, int64_t span, int d,
-                      int dcov, const int32_t *__restrict__ offsets, float *__restrict__ C_new,
-                      double *__restrict__ sums_out) {
+// One warp: unit u of a combine level, column block cb; sk = the warp's shared key slots.
+__device__ __forceinline__ void pieces_unit(const double *__restrict__ pin,
+                                            const int32_t *__restrict__ kin, int64_t nslots_in,
+                                            double *__restrict__ pout,
+                                            int32_t *__restrict__ kout, int64_t u, int cb,
+                                            int64_t span, int d, int dcov,
+                                            const int32_t *__restrict__ offsets,
+                                            float *__restrict__ C_new,
+                                            double *__restrict__ sums_out, int32_t *sk) {
     constexpr int S = 2 * kGroup;
     constexpr int B = 8;
-    __shared__ int32_t s_key[kUpdWarps][S];
     const int lane = threadIdx.x & 31;
-    const int wib = threadIdx.x >> 5;
-    const int64_t u = static_cast<int64_t>(blockIdx.x) * kUpdWarps + wib;
-    if (u >= nunits) return;
-    const int cb = blockIdx.y;
     const int col = cb * 128 + lane * 4;
     const int64_t s0 = u * S;
     const int ns = static_cast<int>((s0 + S < nslots_in ? s0 + S : nslots_in) - s0);
-    int32_t *sk = s_key[wib];
     for (int j = lane; j < ns; j += 32) sk[j] = kin[s0 + j];
     __syncwarp();
 
@@ -535,24 +532,18 @@ __global__ void __launch_bounds__(kUpdWarps * 32)
     }
 }
 
-// counts[k] = offsets[k+1] - offsets[k]; an empty cluster keeps C_old bit for bit (or, for
-// a shard's partial sums, gets a zero sum).
-__global__ void finalize_kernel(const int32_t *__restrict__ offsets, int K, int d,
-                                const float *__restrict__ C_old, float *__restrict__ C_new,
-                                int32_t *__restrict__ counts, double *__restrict__ sums_out) {
-    const int lane = threadIdx.x & 31;
-    const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-    const int64_t nw = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
-    for (int64_t k = warp; k < K; k += nw) {
-        const int32_t c = offsets[k + 1] - offsets[k];
-        if (lane == 0 && counts) counts[k] = c;
-        if (c == 0) {
-            if (sums_out)
-                for (int j = lane; j < d; j += 32) sums_out[k * d + j] = 0.0;
-            else
-                for (int j = lane; j < d; j += 32) C_new[k * d + j] = C_old[k * d + j];
-        }
-    }
+__global__ void __launch_bounds__(kUpdWarps * 32)
+    seg_pieces_kernel(const double *__restrict__ pin, const int32_t *__restrict__ kin,
+                      int64_t nslots_in, double *__restrict__ pout,
+                      int32_t *__restrict__ kout, int64_t nunits, int64_t span, int d,
+                      int dcov, const int32_t *__restrict__ offsets, float *__restrict__ C_new,
+                      double *__restrict__ sums_out) {
+    __shared__ int32_t s_key[kUpdWarps][2 * kGroup];
+    const int wib = threadIdx.x >> 5;
+    const int64_t u = static_cast<int64_t>(blockIdx.x) * kUpdWarps + wib;
+    if (u >= nunits) return;
+    pieces_unit(pin, kin, nslots_in, pout, kout, u, blockIdx.y, span, d, dcov, offsets, C_new,
+                sums_out, s_key[wib]);
 }
 
 // Combine W shards of a data-parallel iteration, in shard order: c_k = (sum_w S_wk) /
@@ -589,27 +580,75 @@ __global__ void finalize_shards_kernel(const double *__restrict__ sums,
     }
 }
 
-// One block sums n partials: thread t adds t, t+1024, ... in order, then a fixed tree.
-__global__ void __launch_bounds__(1024)
-    objective_kernel(const double *__restrict__ part, int64_t n, double *__restrict__ out) {
-    __shared__ double sh[1024];
-    double s = 0.0;
-    for (int64_t i = threadIdx.x; i < n; i += 1024) s += part[i];
-    sh[threadIdx.x] = s;
-    __syncthreads();
-    for (int o = 512; o > 0; o >>= 1) {
-        if (threadIdx.x < o) sh[threadIdx.x] += sh[threadIdx.x + o];
+// The update's tail steps in one launch.  Block 0 sums the n objective partials (thread t
+// adds t, t + 256, ... in order, then a fixed tree).  Blocks 1 .. nfin run the last combine
+// level (one unit; warp 0 of block 1 + cb handles column block cb).  The other blocks
+// finalize: counts[k] = offsets[k+1] - offsets[k], an empty cluster keeps C_old bit for
+// bit (or, for a shard's partial sums, gets a zero sum).  The combine writes only clusters
+// that hold points and the finalize only empty ones, so the blocks touch disjoint rows.
+__global__ void __launch_bounds__(256)
+    finalize_objective_kernel(const int32_t *__restrict__ offsets, int K, int d,
+                              const float *__restrict__ C_old, float *__restrict__ C_new,
+                              int32_t *__restrict__ counts, double *__restrict__ sums_out,
+                              const double *__restrict__ part, int64_t n,
+                              double *__restrict__ objective, int nfin,
+                              const double *__restrict__ pin, const int32_t *__restrict__ kin,
+                              int64_t nslots, double *__restrict__ pout,
+                              int32_t *__restrict__ kout, int64_t span, int dcov) {
+    if (blockIdx.x == 0) {
+        if (objective == nullptr) return;
+        __shared__ double sh[256];
+        double s = 0.0;
+        for (int64_t i = threadIdx.x; i < n; i += 256) s += part[i];
+        sh[threadIdx.x] = s;
         __syncthreads();
+        for (int o = 128; o > 0; o >>= 1) {
+            if (threadIdx.x < o) sh[threadIdx.x] += sh[threadIdx.x + o];
+            __syncthreads();
+        }
+        if (threadIdx.x == 0) *objective = sh[0];
+        return;
     }
-    if (threadIdx.x == 0) *out = sh[0];
+    if (static_cast<int>(blockIdx.x) <= nfin) {
+        __shared__ int32_t s_key[2 * kGroup];
+        if (threadIdx.x < 32)
+            pieces_unit(pin, kin, nslots, pout, kout, 0, static_cast<int>(blockIdx.x) - 1, span,
+                        d, dcov, offsets, C_new, sums_out, s_key);
+        return;
+    }
+    const int lane = threadIdx.x & 31;
+    const int64_t warp =
+        (static_cast<int64_t>(blockIdx.x - 1 - nfin) * blockDim.x + threadIdx.x) >> 5;
+    const int64_t nw = (static_cast<int64_t>(gridDim.x - 1 - nfin) * blockDim.x) >> 5;
+    for (int64_t k = warp; k < K; k += nw) {
+        const int32_t c = offsets[k + 1] - offsets[k];
+        if (lane == 0 && counts) counts[k] = c;
+        if (c == 0) {
+            if (sums_out)
+                for (int j = lane; j < d; j += 32) sums_out[k * d + j] = 0.0;
+            else
+                for (int j = lane; j < d; j += 32) C_new[k * d + j] = C_old[k * d + j];
+        }
+    }
 }
+
+// The last combine level (a single unit), left for the update's tail launch.
+struct FinalLevel {
+    bool pending = false;
+    const double *pin = nullptr;
+    const int32_t *kin = nullptr;
+    int64_t nslots = 0;
+    double *pout = nullptr;
+    int32_t *kout = nullptr;
+    int64_t span = 0;
+};
 
 cudaError_t run_levels(const void *X, bool bf16, int64_t N, int d, const UpdPlan &up,
                        const int32_t *skeys, const int32_t *perm, const int32_t *offsets,
                        const float *C_used, float *C_new, double *sums_out, double *pa,
                        int32_t *ka,
                        double *pb, int32_t *kb, double *jpart, uint32_t *err,
-                       cudaStream_t st) {
+                       cudaStream_t st, FinalLevel *final_level) {
     static bool attr = false;
     if (!attr) {
         cudaFuncSetAttribute(seg_rows_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -639,6 +678,16 @@ cudaError_t run_levels(const void *X, bool bf16, int64_t N, int d, const UpdPlan
     while (units > 1) {
         const int64_t nunits = ceil_div(units, kGroup);
         span *= kGroup;
+        if (nunits == 1) {  // the last level runs inside the tail launch
+            final_level->pending = true;
+            final_level->pin = pin;
+            final_level->kin = kin;
+            final_level->nslots = units * 2;
+            final_level->pout = pout;
+            final_level->kout = kout;
+            final_level->span = span;
+            break;
+        }
         dim3 g2(static_cast<unsigned>(ceil_div(nunits, kUpdWarps)), up.ncolblk);
         seg_pieces_kernel<<<g2, block, 0, st>>>(pin, kin, units * 2, pout, kout, nunits, span, d,
                                                 up.dcov, offsets, C_new, sums_out);
@@ -664,19 +713,21 @@ cudaError_t launch_update(const void *X, fk_dtype dtype, int64_t N, int d, int K
                           double *objective, uint32_t *err, double *sums_out,
                           cudaStream_t st) {
     const bool bf16 = dtype == FK_BF16;
+    FinalLevel fl;
     cudaError_t e = run_levels(X, bf16, N, d, up, skeys, perm, offsets, C_used, C_new,
-                               sums_out, pieces_a, pkeys_a, pieces_b, pkeys_b, jpart, err, st);
+                               sums_out, pieces_a, pkeys_a, pieces_b, pkeys_b, jpart, err, st,
+                               &fl);
     if (e != cudaSuccess) return e;
+    // the update's tail in one launch: the objective (block 0), the last combine level (one
+    // block per 128-column block) and the empty clusters (the remaining blocks)
     int64_t fgrid = ceil_div(K, 8);
     const int64_t cap = static_cast<int64_t>(device_sm_count()) * 16;
     if (fgrid > cap) fgrid = cap;
-    finalize_kernel<<<static_cast<unsigned>(fgrid), 256, 0, st>>>(offsets, K, d, C_old, C_new,
-                                                                   counts, sums_out);
+    const int nfin = fl.pending ? up.ncolblk : 0;
+    finalize_objective_kernel<<<static_cast<unsigned>(1 + nfin + fgrid), 256, 0, st>>>(
+        offsets, K, d, C_old, C_new, counts, sums_out, jpart, up.nwarps * up.ncolblk,
+        objective, nfin, fl.pin, fl.kin, fl.nslots, fl.pout, fl.kout, fl.span, up.dcov);
     note_launch();
-    if (objective) {
-        objective_kernel<<<1, 1024, 0, st>>>(jpart, up.nwarps * up.ncolblk, objective);
-        note_launch();
-    }
     return cudaGetLastError();
 }
 
