@@ -20,7 +20,9 @@ constexpr int kAug = 16;  // bf16 columns of the norm-folding K step (32-byte ro
 constexpr int kSortThreads = 256;
 constexpr int kSortItems = 16;
 constexpr int kSortTile = kSortThreads * kSortItems;  // keys per block
-constexpr int kSortMaxBits = 11;                      // digit width bound: 2048 bins
+// digit width bound: 256 bins (a tile's per-digit bookkeeping grows with the bins, so two
+// narrow passes beat one wide one from about 1024 bins)
+constexpr int kSortMaxBits = 8;
 
 // ----------------------------------------------------------------- update tiling
 constexpr int kUpdWarps = 8;          // warps per block of the update kernels

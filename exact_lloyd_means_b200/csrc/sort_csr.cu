@@ -5,8 +5,8 @@
 // points can be read contiguously; LEANN FlashLib guide, section "工作原理": the coarse
 // quantizer's output is CSR offsets plus cell-ordered row ids.
 //
-// A stable least-significant-digit radix sort with digits of up to 11 bits (one pass for
-// K <= 2048, two for K <= 2^22), written without atomics:
+// A stable least-significant-digit radix sort with digits of up to 8 bits (one pass for
+// K <= 256, two for K <= 65536, three beyond), whose ranks need no atomics:
 //   upsweep   : each block of 4096 keys counts its digits into per-warp histograms in
 //               shared memory (shared-memory atomic adds: the counts do not depend on
 //               their order);
@@ -141,26 +141,35 @@ __global__ void __launch_bounds__(1024)
 }
 
 // Exclusive scan of cnt[0..bins) into out[0..bins) by one block: every thread sums a
-// contiguous run of entries, one thread scans the run totals, then the runs are filled in.
+// contiguous run of entries, the run totals are scanned with warp shuffles (each warp,
+// then the eight warp totals), then the runs are filled in.
 __device__ __forceinline__ void block_scan_bins(const uint32_t *cnt, uint32_t *out, int bins,
                                                 uint32_t *part) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int per = (bins + kSortThreads - 1) / kSortThreads;
     const int lo = threadIdx.x * per;
     const int hi = lo + per < bins ? lo + per : bins;
     uint32_t s = 0;
     for (int b = lo; b < hi; ++b) s += cnt[b];
-    part[threadIdx.x] = s;
+    uint32_t x = s;  // inclusive scan within the warp
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+    }
+    if (lane == 31) part[warp] = x;
     __syncthreads();
-    if (threadIdx.x == 0) {
-        uint32_t run = 0;
-        for (int t = 0; t < kSortThreads; ++t) {
-            const uint32_t v = part[t];
-            part[t] = run;
-            run += v;
+    if (warp == 0) {
+        uint32_t t = lane < kWarps ? part[lane] : 0u;
+#pragma unroll
+        for (int o = 1; o < kWarps; o <<= 1) {
+            const uint32_t y = __shfl_up_sync(0xffffffffu, t, o);
+            if (lane >= o) t += y;
         }
+        if (lane < kWarps) part[kWarps + lane] = t;  // inclusive warp totals
     }
     __syncthreads();
-    uint32_t run = part[threadIdx.x];
+    uint32_t run = (warp == 0 ? 0u : part[kWarps + warp - 1]) + x - s;
     for (int b = lo; b < hi; ++b) {
         const uint32_t v = cnt[b];
         out[b] = run;
