@@ -51,6 +51,9 @@ def parse():
     p.add_argument("--dp", action="store_true",
                    help="run the data-parallel loop (exact_lloyd_means_b200.dist) even on "
                         "one rank")
+    p.add_argument("--streamed", type=int, default=0, metavar="CHUNK_ROWS",
+                   help="keep X in pinned host memory and stream it every iteration in "
+                        "chunks of this many rows (fk_lloyd_streamed, the out-of-core mode)")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=12.0)
@@ -466,6 +469,87 @@ def fk_arm(args, spec, rank, world, dist):
         print(json.dumps(out), flush=True)
 
 
+def streamed_arm(args, spec, rank, world, dist):
+    """X in pinned host memory, streamed every iteration (fk_lloyd_streamed).  One process,
+    one GPU: the step is a complete k-means run; the value is points x iterations per second
+    of device time, with the host-to-device rate it needed beside it."""
+    import torch
+
+    from exact_lloyd_means_b200 import fk
+    from synth import gaussian_mixture, init_indices
+    if world != 1:
+        raise SystemExit("--streamed runs on one GPU")
+    dev = torch.device("cuda", torch.cuda.current_device())
+    niter = args.niter or spec.niter
+    tdt = torch.bfloat16 if spec.dtype == "bf16" else torch.float32
+    e_bytes = 2 if spec.dtype == "bf16" else 4
+    Xh = torch.empty((spec.n, spec.d), dtype=tdt, pin_memory=True)
+    # generate on the device in slices and park them in pinned host memory
+    X, _, _ = gaussian_mixture(spec.n, spec.d, spec.k, centers=spec.centers, sigma=spec.sigma,
+                               weights=spec.weights, zipf_s=spec.zipf_s, dtype=spec.dtype,
+                               seed=spec.seed, device=dev)
+    C0 = X[init_indices(spec.n, spec.k, spec.seed, device=dev)].float().contiguous()
+    Xh.copy_(X)
+    del X
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    # the pinned host-to-device copy rate of this box, for context
+    probe = torch.empty(1 << 28, dtype=torch.uint8, pin_memory=True)
+    probe_d = torch.empty_like(probe, device=dev)
+    h0, h1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    probe_d.copy_(probe, non_blocking=True)
+    h0.record()
+    for _ in range(4):
+        probe_d.copy_(probe, non_blocking=True)
+    h1.record()
+    torch.cuda.synchronize()
+    h2d_gbs = 4 * probe.numel() / (h0.elapsed_time(h1) / 1e3) / 1e9
+    del probe, probe_d
+    chunk = args.streamed
+    ws = fk.streamed_workspace(chunk, spec.d, spec.k, tdt, spec.metric, device=dev)
+    C = torch.empty_like(C0)
+
+    def step():
+        C.copy_(C0)
+        return fk.fk_lloyd_streamed(Xh, C, niter, ws, chunk, metric=spec.metric)
+
+    for _ in range(args.warmup):
+        step()
+    uuid = None
+    try:
+        uuid = torch.cuda.get_device_properties(dev).uuid
+    except Exception:
+        pass
+    sampler = ClockSampler(uuid)
+    sampler.start()
+    time.sleep(0.4)
+    torch.cuda.synchronize()
+    launches0 = fk.launch_count()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        objs = step()
+    e1.record()
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    ms = e0.elapsed_time(e1)
+    value = spec.n * niter * args.steps / (ms / 1e3)
+    need = spec.n * spec.d * e_bytes * niter * args.steps / (ms / 1e3) / 1e9
+    print(json.dumps({
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": spec.dtype, "data": "synthetic",
+        "config": {"workload": spec.name, "N": spec.n, "d": spec.d, "K": spec.k,
+                   "metric": spec.metric, "niter_per_step": niter, "mode": "streamed",
+                   "chunk_rows": chunk,
+                   "l2": "X streamed from pinned host memory every iteration"},
+        "streamed": {"h2d_gbs_used": need, "h2d_gbs_measured": h2d_gbs,
+                     "frac_of_h2d": need / h2d_gbs,
+                     "x_host_gb": spec.n * spec.d * e_bytes / 1e9},
+        "gpu_launches": fk.launch_count() - launches0, "final_objective": objs[-1],
+        "clocks": clocks}), flush=True)
+
+
 def main():
     args = parse()
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -498,7 +582,10 @@ def main():
             os.environ.setdefault("WORLD_SIZE", "1")
         tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=180))
         dist = tdist
-    fk_arm(args, spec, rank, world, dist)
+    if args.streamed:
+        streamed_arm(args, spec, rank, world, dist)
+    else:
+        fk_arm(args, spec, rank, world, dist)
     if dist:
         dist.barrier()
         dist.destroy_process_group()

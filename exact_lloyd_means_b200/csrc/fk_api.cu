@@ -199,6 +199,41 @@ fk_status read_err(void *ws, const WsLayout &L, cudaStream_t st, bool clear, int
     return FK_OK;
 }
 
+// Workspace of fk_lloyd_streamed: the per-chunk workspace (an fk_assign / fk_update
+// workspace for chunk_rows points, L2), then two chunk buffers of points and labels, one
+// chunk's partial sums, counts, offsets and objective, the iteration's running totals, the
+// objectives of every iteration and the alternate centroids.
+struct StreamLayout {
+    WsLayout L;  // per-chunk workspace, at offset 0
+    size_t xbuf[2] = {0, 0}, lab[2] = {0, 0}, sums = 0, cnt = 0, off = 0, objc = 0,
+           sums_tot = 0, cnt_tot = 0, obj_tot = 0, calt = 0, total = 0;
+};
+
+StreamLayout stream_layout(int64_t chunk, int d, int K, fk_dtype dtype) {
+    StreamLayout S;
+    S.L = ws_layout(chunk, d, K, dtype, FK_L2);
+    size_t o = S.L.total;
+    auto take = [&](size_t bytes) {
+        size_t at = o;
+        o += static_cast<size_t>(round_up(static_cast<int64_t>(bytes > 0 ? bytes : 1), 256));
+        return at;
+    };
+    const size_t e = dtype == FK_F32 ? 4 : 2;
+    const size_t KD = static_cast<size_t>(K) * d;
+    for (int b = 0; b < 2; ++b) S.xbuf[b] = take(e * chunk * d);
+    for (int b = 0; b < 2; ++b) S.lab[b] = take(sizeof(int32_t) * chunk);
+    S.sums = take(sizeof(double) * KD);
+    S.cnt = take(sizeof(int32_t) * K);
+    S.off = take(sizeof(int32_t) * (K + 1));
+    S.objc = take(sizeof(double));
+    S.sums_tot = take(sizeof(double) * KD);
+    S.cnt_tot = take(sizeof(int64_t) * K);
+    S.obj_tot = take(sizeof(double) * kObjRing);
+    S.calt = take(sizeof(float) * KD);
+    S.total = o;
+    return S;
+}
+
 // A kernel whose mbarrier is never arrived on: its bounded wait must expire and record
 // a timeout in the workspace error word (exercises the failure path without a fault).
 __global__ void wait_selftest_kernel(uint32_t *err, uint64_t limit_ns) {
@@ -560,6 +595,180 @@ fk_status fk_update_partial(const void *X, fk_dtype dtype, int64_t N, int d, int
     }
     return run_update(X, dtype, N, d, K, L, ws, labels, C_old, C_used, nullptr, counts,
                       offsets, nullptr, objective, sums, st);
+}
+
+fk_status fk_streamed_workspace_size(int64_t chunk_rows, int d, int K, fk_dtype dtype,
+                                     fk_metric metric, size_t *bytes) {
+    if (!bytes) return FK_ERR_INVALID_ARG;
+    fk_status s = validate_shape(chunk_rows, d, K, dtype, metric);
+    if (s != FK_OK) return s;
+    *bytes = stream_layout(chunk_rows, d, K, dtype).total;
+    return FK_OK;
+}
+
+fk_status fk_lloyd_streamed(const void *X_host, fk_dtype dtype, int64_t N, int d, int K,
+                            fk_metric metric, int niter, float *C, int32_t *labels_host,
+                            double *objective_host, int64_t chunk_rows, void *ws,
+                            size_t ws_bytes, fk_stream_t stream) {
+    fk_status s = validate_shape(N, d, K, dtype, metric);
+    if (s != FK_OK) return s;
+    if (!X_host || !C || niter < 0 || niter > kObjRing || chunk_rows < 1)
+        return FK_ERR_INVALID_ARG;
+    if (chunk_rows > N) chunk_rows = N;
+    if (chunk_rows < K) return FK_ERR_INVALID_ARG;
+    if (!aligned(C, 16)) return FK_ERR_UNSUPPORTED;
+    const StreamLayout S = stream_layout(chunk_rows, d, K, dtype);
+    if (ws == nullptr || !aligned(ws, 256) || ws_bytes < S.total) return FK_ERR_WORKSPACE;
+    if ((s = check_device()) != FK_OK) return s;
+    const WsLayout &L = S.L;
+    cudaStream_t st = stream;
+
+    // the copy stream, its events, and their release on every exit
+    cudaStream_t cs = nullptr;
+    cudaEvent_t ev[5] = {nullptr, nullptr, nullptr, nullptr, nullptr};
+    auto cleanup = [&]() {
+        for (auto e : ev)
+            if (e) cudaEventDestroy(e);
+        if (cs) cudaStreamDestroy(cs);
+    };
+    auto fail = [&](fk_status f) {
+        if (cs) cudaStreamSynchronize(cs);
+        cleanup();
+        return f;
+    };
+    if (cudaStreamCreateWithFlags(&cs, cudaStreamNonBlocking) != cudaSuccess) return FK_ERR_CUDA;
+    for (auto &e : ev)
+        if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess)
+            return fail(FK_ERR_CUDA);
+    cudaEvent_t *copied = ev, *done = ev + 2, entry = ev[4];
+    // nothing on the copy stream may start before the caller's earlier work on `stream`
+    if (cudaEventRecord(entry, st) != cudaSuccess || cudaStreamWaitEvent(cs, entry, 0) != cudaSuccess)
+        return fail(FK_ERR_CUDA);
+
+    const size_t row_bytes = static_cast<size_t>(d) * (dtype == FK_F32 ? 4 : 2);
+    const size_t KD = static_cast<size_t>(K) * d;
+    const int64_t nchunks = ceil_div(N, chunk_rows);
+    const char *Xh = static_cast<const char *>(X_host);
+    double *sums = ws_ptr<double>(ws, S.sums), *sums_tot = ws_ptr<double>(ws, S.sums_tot);
+    int32_t *cnt = ws_ptr<int32_t>(ws, S.cnt), *off = ws_ptr<int32_t>(ws, S.off);
+    int64_t *cnt_tot = ws_ptr<int64_t>(ws, S.cnt_tot);
+    double *objc = ws_ptr<double>(ws, S.objc), *obj_tot = ws_ptr<double>(ws, S.obj_tot);
+    float *xnorm = dtype == FK_F32 ? ws_ptr<float>(ws, L.xnorm) : nullptr;
+    float *cused = ws_ptr<float>(ws, L.cused);
+    auto rows_of = [&](int64_t c) { return N - c * chunk_rows < chunk_rows ? N - c * chunk_rows : chunk_rows; };
+
+    if (cudaMemsetAsync(ws_ptr<uint32_t>(ws, L.err), 0, 2 * sizeof(uint32_t), st) != cudaSuccess)
+        return fail(FK_ERR_CUDA);
+    if (metric == FK_COSINE && launch_normalize(C, C, K, d, st) != cudaSuccess)
+        return fail(FK_ERR_CUDA);
+    float *Ccur = C, *Cnext = ws_ptr<float>(ws, S.calt);
+    int64_t pend[2] = {-1, -1};  // chunk whose labels wait in lab[slot] for the host copy
+    bool allow_screen = true, probed = false;
+    int64_t g = 0;
+    for (int t = 0; t < niter; ++t) {
+        if (cudaMemsetAsync(sums_tot, 0, sizeof(double) * KD, st) != cudaSuccess ||
+            cudaMemsetAsync(cnt_tot, 0, sizeof(int64_t) * K, st) != cudaSuccess ||
+            cudaMemsetAsync(obj_tot + t, 0, sizeof(double), st) != cudaSuccess)
+            return fail(FK_ERR_CUDA);
+        if (launch_prep_centroids(Ccur, K, d, L.Kp, L.dp, dtype, ws_ptr<uint16_t>(ws, L.cs),
+                                  ws_ptr<float>(ws, L.cn), cused, ws_ptr<uint16_t>(ws, L.caug),
+                                  st) != cudaSuccess)
+            return fail(FK_ERR_CUDA);
+        for (int64_t c = 0; c < nchunks; ++c, ++g) {
+            const int slot = static_cast<int>(g & 1);
+            const int64_t rows = rows_of(c);
+            void *xb = ws_ptr<void>(ws, S.xbuf[slot]);
+            int32_t *lab = ws_ptr<int32_t>(ws, S.lab[slot]);
+            // copy stream: once the chunk two back is done with this slot, hand its labels
+            // to the host (last iteration) and bring in this chunk's points
+            if (g >= 2 && cudaStreamWaitEvent(cs, done[slot], 0) != cudaSuccess)
+                return fail(FK_ERR_CUDA);
+            if (pend[slot] >= 0) {
+                if (cudaMemcpyAsync(labels_host + pend[slot] * chunk_rows, lab,
+                                    sizeof(int32_t) * rows_of(pend[slot]),
+                                    cudaMemcpyDeviceToHost, cs) != cudaSuccess)
+                    return fail(FK_ERR_CUDA);
+                pend[slot] = -1;
+            }
+            if (cudaMemcpyAsync(xb, Xh + c * chunk_rows * row_bytes, rows * row_bytes,
+                                cudaMemcpyHostToDevice, cs) != cudaSuccess ||
+                cudaEventRecord(copied[slot], cs) != cudaSuccess ||
+                cudaStreamWaitEvent(st, copied[slot], 0) != cudaSuccess)
+                return fail(FK_ERR_CUDA);
+            // compute stream: normalise (cosine), assign, partial update, add to the totals
+            if (metric == FK_COSINE &&
+                launch_normalize(static_cast<float *>(xb), static_cast<float *>(xb), rows, d,
+                                 st) != cudaSuccess)
+                return fail(FK_ERR_CUDA);
+            const void *planes = nullptr;
+            const float *xn = nullptr;
+            int nplanes = 0;
+            int64_t lda = 0;
+            if ((s = prepare_x(xb, dtype, rows, d, L, ws, xnorm, st, &planes, &nplanes, &lda,
+                               &xn)) != FK_OK)
+                return fail(s);
+            const float *X32 = dtype == FK_F32 ? static_cast<const float *>(xb) : nullptr;
+            if (!probed && dtype == FK_F32) {
+                // the screening probe of fk_lloyd, on the first chunk
+                probed = true;
+                bool p = false;
+                if ((s = run_assign(planes, nplanes, lda, rows, d, K, L, ws, lab, xn, nullptr,
+                                    st, X32, Ccur, true, &p, nullptr, nullptr,
+                                    kScreenProbeRows)) != FK_OK)
+                    return fail(s);
+                if (p) {
+                    uint32_t nfb = 0;
+                    if (cudaMemcpyAsync(&nfb, ws_ptr<uint32_t>(ws, L.nfb), sizeof(nfb),
+                                        cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+                        cudaStreamSynchronize(st) != cudaSuccess)
+                        return fail(FK_ERR_CUDA);
+                    const int64_t n = rows < kScreenProbeRows ? rows : kScreenProbeRows;
+                    allow_screen = static_cast<int64_t>(nfb) * kScreenMaxFallback <= n;
+                }
+            }
+            if ((s = run_assign(planes, nplanes, lda, rows, d, K, L, ws, lab, xn, nullptr, st,
+                                X32, Ccur, allow_screen)) != FK_OK)
+                return fail(s);
+            if ((s = run_update(xb, dtype, rows, d, K, L, ws, lab, Ccur,
+                                dtype == FK_BF16 ? cused : Ccur, nullptr, cnt, off, nullptr,
+                                objc, sums, st)) != FK_OK)
+                return fail(s);
+            if (launch_accumulate_chunk(sums_tot, sums, static_cast<int64_t>(KD), cnt_tot, cnt,
+                                        K, obj_tot + t, objc, st) != cudaSuccess ||
+                cudaEventRecord(done[slot], st) != cudaSuccess)
+                return fail(FK_ERR_CUDA);
+            if (labels_host && t == niter - 1) pend[slot] = c;
+        }
+        // new centroids from the iteration's totals (an empty cluster keeps its centroid)
+        if (launch_finalize_shards(sums_tot, cnt_tot, nullptr, 1, K, d, Ccur, Cnext, nullptr,
+                                   nullptr, st) != cudaSuccess)
+            return fail(FK_ERR_CUDA);
+        float *tmp = Ccur;
+        Ccur = Cnext;
+        Cnext = tmp;
+    }
+    for (int k = 0; k < 2; ++k) {  // the last labels still waiting for their host copy
+        const int slot = static_cast<int>((g + k) & 1);
+        if (pend[slot] < 0) continue;
+        if (cudaStreamWaitEvent(cs, done[slot], 0) != cudaSuccess ||
+            cudaMemcpyAsync(labels_host + pend[slot] * chunk_rows,
+                            ws_ptr<int32_t>(ws, S.lab[slot]),
+                            sizeof(int32_t) * rows_of(pend[slot]), cudaMemcpyDeviceToHost,
+                            cs) != cudaSuccess)
+            return fail(FK_ERR_CUDA);
+    }
+    if (Ccur != C && cudaMemcpyAsync(C, Ccur, sizeof(float) * KD, cudaMemcpyDeviceToDevice,
+                                     st) != cudaSuccess)
+        return fail(FK_ERR_CUDA);
+    if (objective_host && niter > 0 &&
+        cudaMemcpyAsync(objective_host, obj_tot, sizeof(double) * niter,
+                        cudaMemcpyDeviceToHost, st) != cudaSuccess)
+        return fail(FK_ERR_CUDA);
+    if (cudaStreamSynchronize(cs) != cudaSuccess) return fail(FK_ERR_CUDA);
+    int code = FK_OK;
+    if (read_err(ws, L, st, true, &code) != FK_OK) return fail(FK_ERR_CUDA);
+    cleanup();
+    return static_cast<fk_status>(code);
 }
 
 fk_status fk_finalize_shards(const double *sums, const int64_t *counts_w,

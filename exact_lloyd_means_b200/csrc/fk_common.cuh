@@ -257,6 +257,9 @@ cudaError_t launch_update(const void *X, fk_dtype dtype, int64_t N, int d, int K
                           cudaStream_t st);
 cudaError_t launch_gather_rows(const void *X, int64_t N, int64_t row_bytes,
                                const int32_t *row_ids, void *out, cudaStream_t st);
+cudaError_t launch_accumulate_chunk(double *tot, const double *part, int64_t KD,
+                                    int64_t *cnt_tot, const int32_t *cnt, int K,
+                                    double *obj_tot, const double *obj, cudaStream_t st);
 cudaError_t launch_finalize_shards(const double *sums, const int64_t *cnts, const double *objs,
                                    int W, int K, int d, const float *C_old, float *C_new,
                                    int64_t *counts, double *objective, cudaStream_t st);

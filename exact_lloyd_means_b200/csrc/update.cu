@@ -731,6 +731,36 @@ cudaError_t launch_update(const void *X, fk_dtype dtype, int64_t N, int d, int K
     return cudaGetLastError();
 }
 
+namespace {
+
+// Running totals of a streamed iteration: tot += one chunk's sums, counts and objective
+// (the chunks are added in their order, so the totals do not depend on scheduling).
+__global__ void accumulate_chunk_kernel(double *__restrict__ tot, const double *__restrict__ part,
+                                        int64_t KD, int64_t *__restrict__ cnt_tot,
+                                        const int32_t *__restrict__ cnt, int K,
+                                        double *__restrict__ obj_tot,
+                                        const double *__restrict__ obj) {
+    const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+    const int64_t t0 = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    for (int64_t i = t0; i < KD; i += stride) tot[i] += part[i];
+    for (int64_t k = t0; k < K; k += stride) cnt_tot[k] += cnt[k];
+    if (t0 == 0) *obj_tot += *obj;
+}
+
+}  // namespace
+
+cudaError_t launch_accumulate_chunk(double *tot, const double *part, int64_t KD,
+                                    int64_t *cnt_tot, const int32_t *cnt, int K,
+                                    double *obj_tot, const double *obj, cudaStream_t st) {
+    int64_t g = ceil_div(KD, 256);
+    const int64_t cap = static_cast<int64_t>(device_sm_count()) * 8;
+    if (g > cap) g = cap;
+    accumulate_chunk_kernel<<<static_cast<unsigned>(g < 1 ? 1 : g), 256, 0, st>>>(
+        tot, part, KD, cnt_tot, cnt, K, obj_tot, obj);
+    note_launch();
+    return cudaGetLastError();
+}
+
 cudaError_t launch_finalize_shards(const double *sums, const int64_t *cnts, const double *objs,
                                    int W, int K, int d, const float *C_old, float *C_new,
                                    int64_t *counts, double *objective, cudaStream_t st) {

@@ -67,12 +67,16 @@ _sig("fk_update_partial", [_vp, _int, _i64, _int, _int, _vp, _vp, _vp, _vp, _vp,
                            _vp])
 _sig("fk_finalize_shards", [_vp, _vp, _vp, _int, _int, _int, _vp, _vp, _vp, _vp, _vp])
 _sig("fk_ivf_lists", [_vp, _int, _i64, _int, _int, _vp, _vp, _vp, _vp, _vp, _sz, _vp])
+_sig("fk_lloyd_streamed", [_vp, _int, _i64, _int, _int, _int, _int, _vp, _vp,
+                           ctypes.POINTER(ctypes.c_double), _i64, _vp, _sz, _vp])
+_sig("fk_streamed_workspace_size", [_i64, _int, _int, _int, _int, ctypes.POINTER(_sz)])
 
 EXPORTED = ["fk_status_string", "fk_version", "fk_workspace_size", "fk_normalize_rows",
             "fk_centroid_norms", "fk_assign", "fk_update", "fk_lloyd",
             "fk_get_device_error", "fk_selftest_timeout", "fk_assign_noalloc",
             "fk_update_partial", "fk_finalize_shards", "fk_split_points",
-            "fk_launch_count", "fk_ivf_lists"]
+            "fk_launch_count", "fk_ivf_lists", "fk_lloyd_streamed",
+            "fk_streamed_workspace_size"]
 
 # Bytes of the static device array fk_assign_noalloc takes its scratch from.
 NOALLOC_SCRATCH_BYTES = 8 << 20
@@ -339,3 +343,38 @@ def fk_ivf_lists(X: torch.Tensor, labels: torch.Tensor, K: int, offsets: torch.T
                              _opt(X_lists, "X_lists", X.dtype, (N, d)),
                              _dev(ws, "ws", torch.uint8), ws.numel(), _stream(stream)),
            "fk_ivf_lists")
+
+
+def streamed_workspace(chunk_rows: int, d: int, K: int, dtype=torch.float32, metric="l2",
+                       device="cuda"):
+    """A workspace tensor for fk_lloyd_streamed with this chunk size."""
+    code = FK_F32 if dtype == torch.float32 else FK_BF16
+    out = _sz(0)
+    _check(_lib.fk_streamed_workspace_size(chunk_rows, d, K, code, _metric_code(metric),
+                                           ctypes.byref(out)), "fk_streamed_workspace_size")
+    return torch.zeros(out.value, dtype=torch.uint8, device=device)
+
+
+def fk_lloyd_streamed(X_host: torch.Tensor, C: torch.Tensor, niter: int, ws: torch.Tensor,
+                      chunk_rows: int, metric="l2", labels: torch.Tensor | None = None,
+                      stream=None):
+    """Lloyd's iterations over points in host memory (pin them for overlap), streamed in
+    chunks.  C (device) is updated in place; returns the objectives; `labels` (host int32)
+    receives the last iteration's labels."""
+    if X_host.device.type != "cpu" or not X_host.is_contiguous():
+        raise ValueError("X_host must be a contiguous CPU tensor")
+    N, d = X_host.shape
+    K = C.shape[0]
+    obj = (ctypes.c_double * max(niter, 1))()
+    lab_ptr = None
+    if labels is not None:
+        if labels.device.type != "cpu" or labels.dtype != torch.int32 or \
+                tuple(labels.shape) != (N,) or not labels.is_contiguous():
+            raise ValueError("labels must be a contiguous CPU int32 tensor of N entries")
+        lab_ptr = labels.data_ptr()
+    _check(_lib.fk_lloyd_streamed(X_host.data_ptr(), _dtype_code(X_host), N, d, K,
+                                  _metric_code(metric), niter,
+                                  _dev(C, "C", torch.float32, (K, d)), lab_ptr, obj,
+                                  chunk_rows, _dev(ws, "ws", torch.uint8), ws.numel(),
+                                  _stream(stream)), "fk_lloyd_streamed")
+    return [obj[i] for i in range(niter)]

@@ -221,6 +221,32 @@ FK_API fk_status fk_finalize_shards(const double *sums, const int64_t *counts_w,
                                     const float *C_old, float *C_new, int64_t *counts,
                                     double *objective, fk_stream_t stream);
 
+/* Lloyd's iterations over points held in HOST memory (the out-of-core mode of the
+ * Flash-KMeans article: the data set can exceed the GPU's memory).  Each iteration streams
+ * X from the host in chunks of chunk_rows rows: while one chunk is assigned and reduced on
+ * `stream`, the next is copied in on a second stream (double buffering).  Every chunk's
+ * fp64 per-cluster sums, counts and objective share are added to the iteration's totals in
+ * chunk order, then the centroids are formed once (an empty cluster keeps its centroid).
+ * The result is deterministic; it equals fk_lloyd's up to the order of the fp64 sums.
+ *   X_host        : N x d points (fp32 or bf16), host memory; page-locked (pinned) memory
+ *                   lets the copies overlap the compute
+ *   C             : K x d fp32, device: initial centroids in, final centroids out
+ *   labels_host   : optional N int32, host: labels of the last iteration
+ *   objective_host: optional niter doubles, host: objective of every iteration
+ *   chunk_rows    : rows per chunk (>= K; clamped to N); the workspace holds two chunks
+ * Same metric semantics as fk_lloyd (cosine: each chunk and the initial C normalised).
+ * niter <= 4096.  Synchronous: returns after the last copy has landed. */
+FK_API fk_status fk_lloyd_streamed(const void *X_host, fk_dtype dtype, int64_t N, int d,
+                                   int K, fk_metric metric, int niter, float *C,
+                                   int32_t *labels_host, double *objective_host,
+                                   int64_t chunk_rows, void *ws, size_t ws_bytes,
+                                   fk_stream_t stream);
+
+/* Workspace bytes of fk_lloyd_streamed for this chunk size (the per-chunk workspace of
+ * fk_assign / fk_update, two chunk buffers, and K x d fp64 sums twice). */
+FK_API fk_status fk_streamed_workspace_size(int64_t chunk_rows, int d, int K, fk_dtype dtype,
+                                            fk_metric metric, size_t *bytes);
+
 /* Inverted lists of a clustering (LEANN FlashLib guide, "工作原理": an IVF index keeps,
  * per cell, the ids of its points in CSR form and the points of a cell contiguous).
  *   offsets[k] .. offsets[k+1] - 1 : the positions of cell k (offsets: K+1 int32)

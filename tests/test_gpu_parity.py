@@ -454,3 +454,39 @@ def test_ivf_lists_match_oracle(N, d, K, weights, dtype):
     row2 = torch.empty_like(row_ids)
     m.fk_ivf_lists(Xg, torch.as_tensor(lab).to(DEV), K, offsets, row2, ws)
     assert torch.equal(row2, row_ids)
+
+
+@pytest.mark.parametrize("dtype,metric,d", [("f32", "l2", 128), ("f32", "cosine", 256),
+                                            ("bf16", "l2", 128), ("f32", "l2", 768)])
+def test_lloyd_streamed_matches_oracle_and_fk_lloyd(dtype, metric, d):
+    """fk_lloyd_streamed (points in pinned host memory, 4 chunks with a ragged last one)
+    against the oracle on the first iteration (labels outside ties, centroids, objective)
+    and against fk_lloyd on the same data (objectives and centroids)."""
+    m = fk()
+    N, K = 150001, 500
+    X, _, _ = gaussian_mixture(N, d, K, centers="normal", sigma=0.3, dtype=dtype, seed=51)
+    C0 = X[init_indices(N, K, 51)].float().contiguous()
+    prec = "bf16" if dtype == "bf16" else "f32"
+    ref = oracle.lloyd(X, C0, 1, metric=metric, precision=prec)
+    Xh = torch.empty(X.shape, dtype=X.dtype, pin_memory=True)
+    Xh.copy_(X)
+    labels = torch.empty(N, dtype=torch.int32, pin_memory=True)
+    tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
+    ws = m.streamed_workspace(40000, d, K, tdt, metric)
+    C = C0.to(DEV).clone()
+    objs = m.fk_lloyd_streamed(Xh, C, 1, ws, 40000, metric=metric, labels=labels)
+    lab = labels.numpy()
+    assert label_mismatches(lab, ref["labels"][0], ref["ties"][0]) == 0
+    assert abs(objs[0] - ref["J"][0]) <= OBJECTIVE_TOL * ref["J"][0]
+    if not ref["ties"][0].any():
+        assert centroid_rel_err(C.cpu().numpy(), ref["C_next"][0]) <= CENTROID_TOL
+    # three iterations against fk_lloyd on the device copy
+    C1 = C0.to(DEV).clone()
+    objs1 = m.fk_lloyd_streamed(Xh, C1, 3, ws, 40000, metric=metric)
+    C2 = C0.to(DEV).clone()
+    lab2 = torch.empty(N, dtype=torch.int32, device=DEV)
+    objs2, _ = m.fk_lloyd(X.to(DEV), C2, 3, lab2, m.workspace(N, d, K, tdt, metric),
+                          metric=metric)
+    for a, b in zip(objs1, objs2):
+        assert abs(a - b) <= 1e-6 * b
+    assert centroid_rel_err(C1.cpu().numpy(), C2.cpu().numpy()) <= 1e-5
