@@ -65,19 +65,19 @@ __device__ __forceinline__ void store_piece(double *dst, const double (&acc)[4])
     q[1] = make_double2(acc[2], acc[3]);
 }
 
-// Level 1.  A warp owns sorted positions [w*R, w*R + R) and the 128 columns of block
-// blockIdx.y (lane l holds columns 4l .. 4l+3).  The warp first stages the R cluster ids
-// and row ids of its chunk in shared memory (one coalesced read).  Rows are then gathered
-// with 1-D bulk copies (one 128-column slice of one row per lane, 512 bytes for fp32 and
-// 256 for bf16) into a ring of kRowRing batches of B rows (B = 8 fp32 / 16 bf16) in
-// shared memory, each batch completing on its own mbarrier, so four batches are in flight
-// per warp without holding any registers.  When a batch lies in one cluster its rows are
+// Level 1 for fp32 points (bf16 points use seg_rows_regs_kernel below).  A warp owns
+// sorted positions [w*R, w*R + R) and the 128 columns of block blockIdx.y (lane l holds
+// columns 4l .. 4l+3).  The warp first stages the R cluster ids and row ids of its chunk in
+// shared memory (one coalesced read).  Rows are then gathered with 1-D bulk copies (one
+// 512-byte 128-column slice of one row per lane) into a ring of kRowRing batches of B = 8
+// rows in shared memory, each batch completing on its own mbarrier, so four batches are in
+// flight per warp without holding any registers.  When a batch lies in one cluster its rows are
 // first added pairwise in fp32 (a fixed tree) and the batch sum is added to the fp64
 // accumulator once; otherwise rows are added one by one in fp64.  The objective term
 // (x - c_used)^2 of a row is formed in fp32 and accumulated in fp64.
 constexpr int kRowRing = 4;        // batches in flight per warp
 constexpr int kRowWarps = 4;       // warps per block of the level-1 kernel
-constexpr int kRowBatchBytes = 4096;  // 8 fp32 rows or 16 bf16 rows of 128 columns
+constexpr int kRowBatchBytes = 4096;  // 8 fp32 rows of 128 columns
 
 template <bool BF16>
 struct RowVec;
@@ -93,19 +93,6 @@ struct RowVec<false> {
         f[3] = v.w;
     }
 };
-template <>
-struct RowVec<true> {
-    static constexpr int kBatch = 16;
-    static constexpr int kSlice = 256;
-    __device__ static void load(const uint8_t *p, float (&f)[4]) {
-        const uint2 u = *reinterpret_cast<const uint2 *>(p);
-        f[0] = __uint_as_float(u.x << 16);
-        f[1] = __uint_as_float(u.x & 0xffff0000u);
-        f[2] = __uint_as_float(u.y << 16);
-        f[3] = __uint_as_float(u.y & 0xffff0000u);
-    }
-};
-
 constexpr size_t kRowSmem = size_t(kRowWarps) * kRowRing * kRowBatchBytes;  // dynamic part
 
 template <bool BF16>
@@ -287,18 +274,6 @@ __global__ void __launch_bounds__(kRowWarps * 32, 3)
 // while the current one is added; the arithmetic is that of seg_rows_kernel.
 template <bool BF16>
 struct RegRowVec;
-template <>
-struct RegRowVec<false> {
-    using T = float4;
-    static constexpr int kBatch = 8;
-    __device__ static void unpack(const float4 &v, float (&f)[4]) {
-        f[0] = v.x;
-        f[1] = v.y;
-        f[2] = v.z;
-        f[3] = v.w;
-    }
-    __device__ static float4 zero() { return make_float4(0.f, 0.f, 0.f, 0.f); }
-};
 template <>
 struct RegRowVec<true> {
     using T = uint2;
@@ -651,8 +626,6 @@ cudaError_t run_levels(const void *X, bool bf16, int64_t N, int d, const UpdPlan
                        cudaStream_t st, FinalLevel *final_level) {
     static bool attr = false;
     if (!attr) {
-        cudaFuncSetAttribute(seg_rows_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(kRowSmem));
         cudaFuncSetAttribute(seg_rows_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(kRowSmem));
         attr = true;
