@@ -490,3 +490,31 @@ def test_lloyd_streamed_matches_oracle_and_fk_lloyd(dtype, metric, d):
     for a, b in zip(objs1, objs2):
         assert abs(a - b) <= 1e-6 * b
     assert centroid_rel_err(C1.cpu().numpy(), C2.cpu().numpy()) <= 1e-5
+
+
+@pytest.mark.parametrize("case", ["threshold_rows", "ragged_d", "k_equals_n", "zero_rows"])
+def test_screened_assign_edge_cases(case):
+    """Screened-route edges: N exactly at the CTA-pair threshold (2 * 128 * 148 / 2 rows),
+    d not a multiple of 64 (padded operand columns), K = N (every point its own centroid,
+    256-column tiles full of near-ties), and all-zero rows (every centroid at distance
+    ||c||^2: ties resolved to the lowest index of the smallest norm)."""
+    g = torch.Generator().manual_seed(61)
+    if case == "threshold_rows":
+        X, _, _ = gaussian_mixture(18944, 256, 300, centers="normal", sigma=0.3, seed=61)
+        C = X[init_indices(18944, 300, 61)].float().contiguous()
+    elif case == "ragged_d":
+        X, _, _ = gaussian_mixture(30001, 260, 700, centers="normal", sigma=0.3, seed=62)
+        C = X[init_indices(30001, 700, 62)].float().contiguous()
+    elif case == "k_equals_n":
+        X, _, _ = gaussian_mixture(20000, 256, 20000, centers="normal", sigma=0.3, seed=63)
+        C = X.clone()
+    else:
+        X, _, _ = gaussian_mixture(20000, 256, 400, centers="normal", sigma=0.3, seed=64)
+        X[::7] = 0.0
+        C = X[init_indices(20000, 400, 64)].float().contiguous()
+    ref, dmin, d2nd = oracle.assign(X, C.numpy())
+    ties = oracle.tie_mask(X, C.numpy(), dmin, d2nd)
+    lab, _ = gpu_assign(X.to(DEV), C.to(DEV))
+    assert label_mismatches(lab, ref, ties) == 0, f"ties={int(ties.sum())}"
+    if case == "k_equals_n":
+        assert (lab == np.arange(20000)).all()
