@@ -46,6 +46,10 @@ def lib():
         L.orc_csr.restype = ctypes.c_int
         L.orc_update.argtypes = [_dp, ctypes.c_int64, ctypes.c_int, _ip, _dp,
                                  ctypes.c_int, _dp]
+        L.orc_ivf_search.argtypes = [_dp, ctypes.c_int64, ctypes.c_int, _dp, ctypes.c_int,
+                                     _dp, ctypes.c_int64, _ip, ctypes.c_int, ctypes.c_int,
+                                     _ip, _ip, _dp]
+        L.orc_ivf_search.restype = ctypes.c_int
         _lib = L
     return _lib
 
@@ -125,6 +129,33 @@ def update(X, labels, C_old) -> np.ndarray:
     lib().orc_update(_ptr(X, _dp), n, d, _ptr(labels, _ip), _ptr(C_old, _dp), K,
                      _ptr(C_new, _dp))
     return C_new
+
+
+def ivf_search(Q, C, X, labels, nprobe: int, k: int):
+    """IVF-Flat search in fp64 (ivf_search_oracle.c): for every query, the nprobe cells
+    with the nearest centroids (ascending (distance, cell)), then the k nearest points of
+    those cells (ascending (distance, point index); missing slots -1 / +inf).
+
+    Returns (probes int32 [nq, nprobe], ids int32 [nq, k], dist fp64 [nq, k]).  `labels`
+    gives every point's cell; X is in the original point order.
+    """
+    Q = _f64(Q)
+    C = _f64(C)
+    X = _f64(X)
+    labels = np.ascontiguousarray(labels, dtype=np.int32)
+    nq, d = Q.shape
+    nlist = C.shape[0]
+    n = X.shape[0]
+    assert C.shape[1] == d and X.shape[1] == d and labels.shape == (n,)
+    probes = np.empty((nq, nprobe), dtype=np.int32)
+    ids = np.empty((nq, k), dtype=np.int32)
+    dist = np.empty((nq, k), dtype=np.float64)
+    rc = lib().orc_ivf_search(_ptr(Q, _dp), nq, d, _ptr(C, _dp), nlist, _ptr(X, _dp), n,
+                              _ptr(labels, _ip), nprobe, k, _ptr(probes, _ip),
+                              _ptr(ids, _ip), _ptr(dist, _dp))
+    if rc != 0:
+        raise ValueError("ivf_search: label outside [0, nlist) or nprobe/k out of range")
+    return probes, ids, dist
 
 
 def tie_mask(X, C, dmin, d2nd, tau: float = TIE_TAU) -> np.ndarray:

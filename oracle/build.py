@@ -7,7 +7,7 @@ import subprocess
 import sys
 
 HERE = os.path.dirname(os.path.abspath(__file__))
-SRC = os.path.join(HERE, "lloyd_oracle.c")
+SRCS = [os.path.join(HERE, "lloyd_oracle.c"), os.path.join(HERE, "ivf_search_oracle.c")]
 OUT_DIR = os.path.join(HERE, "_build")
 LIB = os.path.join(OUT_DIR, "liboracle.so")
 
@@ -15,12 +15,12 @@ LIB = os.path.join(OUT_DIR, "liboracle.so")
 def build(force: bool = False) -> str:
     """Build liboracle.so if it is missing or older than its source; return its path."""
     if (not force and os.path.exists(LIB)
-            and os.path.getmtime(LIB) >= os.path.getmtime(SRC)):
+            and all(os.path.getmtime(LIB) >= os.path.getmtime(s) for s in SRCS)):
         return LIB
     os.makedirs(OUT_DIR, exist_ok=True)
     tmp = LIB + f".tmp{os.getpid()}"
     cmd = ["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c99",
-           "-fno-fast-math", "-ffp-contract=off", SRC, "-o", tmp, "-lm"]
+           "-fno-fast-math", "-ffp-contract=off", *SRCS, "-o", tmp, "-lm"]
     subprocess.run(cmd, check=True)
     os.replace(tmp, LIB)
     return LIB

@@ -260,3 +260,123 @@ def test_round_bf16_is_nearest_even():
     ulp = 2.0 ** -7  # bf16 spacing on [1, 2)
     v = np.array([1 + ulp / 2, 1 + 1.5 * ulp, 1 + 0.75 * ulp, -(1 + ulp / 2)])
     assert oracle.round_bf16(v).tolist() == [1.0, 1 + 2 * ulp, 1 + ulp, -1.0]
+
+
+# --------------------------------------------------------------------------- IVF-Flat search
+
+
+def _sq_loop(u, v):
+    # sequential fp64 sum (the builtin sum() of floats is compensated since Python 3.12)
+    s = 0.0
+    for a, b in zip(u, v):
+        s += (a - b) * (a - b)
+    return s
+
+
+def _search_python_loops(Q, C, X, labels, nprobe, k):
+    """Brute force in pure Python on tiny inputs: sorted() over (distance, index) tuples."""
+    probes, ids, dist = [], [], []
+    for q in Q.tolist():
+        cd = [(_sq_loop(q, c), j) for j, c in enumerate(C.tolist())]
+        cells = [j for _, j in sorted(cd)[:nprobe]]
+        cand = [(_sq_loop(q, x), i) for i, x in enumerate(X.tolist()) if labels[i] in cells]
+        best = sorted(cand)[:k]
+        probes.append(cells)
+        ids.append([i for _, i in best] + [-1] * (k - len(best)))
+        dist.append([v for v, _ in best] + [np.inf] * (k - len(best)))
+    return np.array(probes), np.array(ids), np.array(dist)
+
+
+def test_ivf_search_golden_hand_derived():
+    g = json.load(open(os.path.join(GOLDEN, "ivf_search_hand.json")))
+    C, X = np.array(g["C"]), np.array(g["X"])
+    labels = np.array(g["labels"], dtype=np.int32)
+    for case in g["cases"]:
+        probes, ids, dist = oracle.ivf_search(np.array(case["Q"]), C, X, labels,
+                                              case["nprobe"], case["k"])
+        assert probes.tolist() == case["probes"]
+        assert ids.tolist() == case["ids"]
+        want = np.array([[np.inf if v is None else v for v in row] for row in case["dist"]])
+        assert np.array_equal(dist, want)
+
+
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_ivf_search_matches_python_brute_force(seed):
+    r = _rng(40 + seed)
+    X = np.round(r.normal(size=(70, 3)), 1)   # one decimal: exact ties occur
+    C = np.round(r.normal(size=(6, 3)), 1)
+    Q = np.round(r.normal(size=(9, 3)), 1)
+    labels = r.integers(0, 6, size=70).astype(np.int32)
+    for nprobe, k in ((1, 3), (2, 5), (6, 7), (3, 40)):
+        got = oracle.ivf_search(Q, C, X, labels, nprobe, k)
+        want = _search_python_loops(Q, C, X, labels, nprobe, k)
+        for a, b in zip(got, want):
+            assert np.array_equal(a, b)
+
+
+def test_ivf_search_all_cells_is_exact_knn():
+    """nprobe = nlist probes every cell: the result is the exact k-nearest-neighbour list of
+    scikit-learn's brute-force search."""
+    from sklearn.neighbors import NearestNeighbors
+    r = _rng(50)
+    X = r.normal(size=(3000, 16))
+    C = X[:40].copy()
+    labels, _, _ = oracle.assign(X, C)
+    Q = r.normal(size=(25, 16))
+    _, ids, dist = oracle.ivf_search(Q, C, X, labels, 40, 10)
+    nn = NearestNeighbors(n_neighbors=10, algorithm="brute").fit(X)
+    d_ref, i_ref = nn.kneighbors(Q)
+    assert np.array_equal(ids, i_ref)
+    np.testing.assert_allclose(dist, d_ref ** 2, rtol=1e-10)
+
+
+def test_ivf_probes_are_nearest_centroids_by_cdist():
+    from scipy.spatial.distance import cdist
+    r = _rng(51)
+    C = r.normal(size=(64, 12))
+    X = r.normal(size=(500, 12))
+    labels = r.integers(0, 64, size=500).astype(np.int32)
+    Q = r.normal(size=(30, 12))
+    probes, _, _ = oracle.ivf_search(Q, C, X, labels, 9, 1)
+    D = cdist(Q, C, "sqeuclidean")
+    want = np.argsort(D, axis=1, kind="stable")[:, :9]
+    assert np.array_equal(probes, want)
+
+
+def test_ivf_search_self_query_finds_itself():
+    """With labels from the assignment against the same centroids, a point used as a query
+    probes its own cell first and is its own nearest neighbour at distance 0."""
+    r = _rng(52)
+    X = r.normal(size=(800, 10))
+    C = X[r.choice(800, 20, replace=False)]
+    labels, _, _ = oracle.assign(X, C)
+    sel = r.choice(800, 40, replace=False)
+    probes, ids, dist = oracle.ivf_search(X[sel], C, X, labels, 1, 3)
+    assert np.array_equal(probes[:, 0], labels[sel])
+    assert np.array_equal(ids[:, 0], sel)
+    assert np.all(dist[:, 0] == 0.0)
+    assert np.all(np.diff(dist, axis=1) >= 0)
+
+
+def test_ivf_search_kth_distance_non_increasing_in_nprobe():
+    r = _rng(53)
+    X = r.normal(size=(2000, 8))
+    C = r.normal(size=(32, 8))
+    labels, _, _ = oracle.assign(X, C)
+    Q = r.normal(size=(20, 8))
+    prev = None
+    for nprobe in (1, 2, 4, 8, 16, 32):
+        probes, _, dist = oracle.ivf_search(Q, C, X, labels, nprobe, 5)
+        if prev is not None:
+            assert np.all(dist[:, -1] <= prev[1][:, -1])
+            assert np.array_equal(probes[:, :prev[0].shape[1]], prev[0])  # nested probe lists
+        prev = (probes, dist)
+
+
+def test_ivf_search_rejects_bad_arguments():
+    X = np.zeros((4, 2))
+    C = np.zeros((2, 2))
+    with pytest.raises(ValueError):
+        oracle.ivf_search(X, C, X, np.array([0, 1, 2, 0], dtype=np.int32), 1, 1)
+    with pytest.raises(ValueError):
+        oracle.ivf_search(X, C, X, np.zeros(4, dtype=np.int32), 3, 1)
