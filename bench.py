@@ -54,6 +54,13 @@ def parse():
     p.add_argument("--streamed", type=int, default=0, metavar="CHUNK_ROWS",
                    help="keep X in pinned host memory and stream it every iteration in "
                         "chunks of this many rows (fk_lloyd_streamed, the out-of-core mode)")
+    p.add_argument("--search", type=int, default=0, metavar="NPROBE",
+                   help="IVF-Flat search instead of k-means: build the index of the workload "
+                        "(its Lloyd run, then the cell lists), then time searches of a "
+                        "batch of --queries queries probing NPROBE cells for --topk "
+                        "neighbours (fk_ivf_search)")
+    p.add_argument("--queries", type=int, default=10000)
+    p.add_argument("--topk", type=int, default=10)
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=12.0)
@@ -550,6 +557,241 @@ def streamed_arm(args, spec, rank, world, dist):
         "clocks": clocks}), flush=True)
 
 
+SEARCH_UNIT = "queries/s"
+
+
+def search_metric(nprobe, k):
+    return f"queries/sec of IVF-Flat search (nprobe {nprobe}, top-{k}) on 1 B200"
+
+
+def fp64_peak_tflops(peaks_path=None):
+    """fp64 FMA peak of the B200 from its unit counts and clock: 148 SMs x 64 fp64 FMA lanes
+    per SM per clock x 2 flops x the maximum SM clock (1965 MHz unless MEASURED_PEAKS.json
+    records another)."""
+    mhz = 1965.0
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            mhz = float(json.load(f).get("sm_max_mhz", mhz))
+    return 148 * 64 * 2 * mhz * 1e6 / 1e12, mhz
+
+
+def search_cpu_sample(spec, seconds, nq_cap, rank_seed=0):
+    """The oracle's IVF-Flat search timed on this host's cores over a bounded query sample.
+    The index it searches is the workload's mixture components as cells (the oracle cannot
+    run the 20-iteration build of a million points in bounded time); cells of the same
+    sizes make the same amount of work.  Returns (queries/s, threads, description, step)."""
+    import numpy as np
+
+    import oracle
+    from synth import gaussian_mixture, mixture_queries
+    X, comp, cen = gaussian_mixture(spec.n, spec.d, spec.k, centers=spec.centers,
+                                    sigma=spec.sigma, weights=spec.weights,
+                                    zipf_s=spec.zipf_s, dtype="f32", seed=spec.seed)
+    labels = comp.numpy().astype(np.int32)
+    Xd = oracle.normalize_rows(X) if spec.metric == "cosine" else oracle._f64(X)
+    Cd = oracle.normalize_rows(cen) if spec.metric == "cosine" else oracle._f64(cen)
+    del X
+    Q = mixture_queries(nq_cap, spec.d, spec.k, centers=spec.centers, sigma=spec.sigma,
+                        weights=spec.weights, zipf_s=spec.zipf_s, seed=spec.seed,
+                        stream=1 + rank_seed)
+    Qd = oracle.normalize_rows(Q) if spec.metric == "cosine" else oracle._f64(Q)
+
+    def one(S, nprobe, k):
+        t0 = time.perf_counter()
+        oracle.ivf_search(Qd[:S], Cd, Xd, labels, nprobe, k)
+        return time.perf_counter() - t0
+
+    return Qd, one
+
+
+def search_arm(args, spec, rank, world, dist):
+    """IVF-Flat search over the index of the workload (LEANN guide, "性能对比": 1M x 768,
+    nlist 4096, top-10, an nprobe sweep).  Each rank builds the same index (fk_lloyd, then
+    fk_ivf_lists and fk_ivf_norms) and searches its own batch of queries: replicas, weak
+    scaling.  A step is one fk_ivf_search call over the batch (cosine: with the query
+    normalisation)."""
+    import torch
+
+    from exact_lloyd_means_b200 import fk
+    from synth import gaussian_mixture, init_indices, mixture_queries
+
+    dev = torch.device("cuda", torch.cuda.current_device())
+    nprobe, k, nq = args.search, args.topk, args.queries
+    X, _, _ = gaussian_mixture(spec.n, spec.d, spec.k, centers=spec.centers, sigma=spec.sigma,
+                               weights=spec.weights, zipf_s=spec.zipf_s, dtype="f32",
+                               seed=spec.seed, device=dev)
+    C0 = X[init_indices(spec.n, spec.k, spec.seed, device=dev)].float().contiguous()
+    index = fk.IvfFlatIndex.build(X, C0, args.niter or spec.niter, metric=spec.metric)
+    del X
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    Q = mixture_queries(nq, spec.d, spec.k, centers=spec.centers, sigma=spec.sigma,
+                        weights=spec.weights, zipf_s=spec.zipf_s, seed=spec.seed,
+                        stream=1 + rank, device=dev)
+    ws = fk.ivf_search_workspace(nq, spec.d, spec.k, spec.n, nprobe, k, device=dev)
+    D = torch.empty((nq, k), dtype=torch.float32, device=dev)
+    I = torch.empty((nq, k), dtype=torch.int32, device=dev)
+    P = torch.empty((nq, nprobe), dtype=torch.int32, device=dev)
+
+    def step(Qin, timing=None):
+        index.search(Qin, k, nprobe, ws=ws, distances=D, ids=I, probes=P, timing=timing)
+
+    for _ in range(args.warmup):
+        step(Q)
+    torch.cuda.synchronize()
+    # work of one step: (query, point) distance evaluations of the fine pass
+    sizes = (index.offsets[1:] - index.offsets[:-1]).long()
+    evals = int(sizes[P.long()].sum().item())
+    fine_flops = 2.0 * spec.d * evals
+    coarse_flops = 2.0 * spec.d * nq * spec.k
+
+    uuid = None
+    try:
+        uuid = torch.cuda.get_device_properties(dev).uuid
+    except Exception:
+        pass
+    sampler = ClockSampler(uuid)
+    sampler.start()
+    time.sleep(0.4)
+    acc = {}
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    launches0 = fk.launch_count()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        tm = {}
+        step(Q, tm)
+        for key, v in tm.items():
+            acc[key] = acc.get(key, 0.0) + v
+    e1.record()
+    torch.cuda.synchronize()
+    launches = fk.launch_count() - launches0
+    if dist:
+        dist.barrier()
+    clocks = sampler.stop()
+    ms = e0.elapsed_time(e1)
+    if dist:
+        t = torch.tensor([ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = t.item()
+    value = nq * args.steps * world / (ms / 1e3)
+    phases = {key: v / args.steps for key, v in acc.items()}
+    peak, mhz = fp64_peak_tflops()
+    fine_tf = fine_flops / (phases["ms_fine"] / 1e3) / 1e12
+    coarse_tf = coarse_flops / (phases["ms_coarse"] / 1e3) / 1e12
+    out = {"metric": search_metric(nprobe, k), "value": value, "unit": SEARCH_UNIT,
+           "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+           "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
+           "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+           "config": {"workload": f"ivf_search_{spec.n}x{spec.d}_nlist{spec.k}_nq{nq}"
+                                  f"_nprobe{nprobe}_k{k}_{spec.metric}",
+                      "N": spec.n, "d": spec.d, "nlist": spec.k, "queries": nq,
+                      "nprobe": nprobe, "k": k, "metric": spec.metric,
+                      "index": f"fk_lloyd {args.niter or spec.niter} iterations + "
+                               "fk_ivf_lists + fk_ivf_norms, built before timing",
+                      "l2": "cell-ordered points (N x d fp32) larger than L2; no flush"},
+           "roofline": {"bound": "alu", "achieved": fine_tf, "peak": peak,
+                        "unit": "TFLOP/s", "frac": fine_tf / peak, "traffic": None,
+                        "kernel": "ivf_tile_kernel<true> (fine pass, fp64 FMA)",
+                        "flops_per_launch": fine_flops, "avg_ms": phases["ms_fine"],
+                        "peak_basis": f"148 SMs x 64 fp64 FMA/clk x 2 x {mhz:.0f} MHz"},
+           "coarse": {"achieved_tflops": coarse_tf, "frac": coarse_tf / peak,
+                      "flops": coarse_flops, "avg_ms": phases["ms_coarse"]},
+           "distance_evals_per_query": evals / nq,
+           "phase_ms_per_step": phases, "gpu_launches": launches, "clocks": clocks}
+
+    if not args.no_e2e:
+        Qh = torch.empty(Q.shape, dtype=torch.float32, pin_memory=True)
+        Qh.copy_(Q)
+        Dh = torch.empty(D.shape, dtype=torch.float32, pin_memory=True)
+        Ih = torch.empty(I.shape, dtype=torch.int32, pin_memory=True)
+        Qd = torch.empty_like(Q)
+        ke = max(1, args.steps)
+
+        def e2e_step():
+            Qd.copy_(Qh, non_blocking=True)
+            step(Qd)
+            Dh.copy_(D, non_blocking=True)
+            Ih.copy_(I, non_blocking=True)
+            torch.cuda.synchronize()
+
+        e2e_step()
+        if dist:
+            dist.barrier()
+        torch.cuda.synchronize()
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        f0.record()
+        for _ in range(ke):
+            e2e_step()
+        f1.record()
+        torch.cuda.synchronize()
+        ems = f0.elapsed_time(f1)
+        if dist:
+            t = torch.tensor([ems], device=dev, dtype=torch.float64)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ems = t.item()
+        out["e2e"] = {"value": nq * ke * world / (ems / 1e3), "unit": SEARCH_UNIT,
+                      "h2d_bytes_per_step": Q.numel() * 4,
+                      "d2h_bytes_per_step": D.numel() * 4 + I.numel() * 4, "steps": ke}
+
+    if not args.no_cpu_baseline and world == 1 and rank == 0:
+        import oracle
+        Qd, one = search_cpu_sample(spec, args.cpu_seconds, nq)
+        S = 16
+        t = one(S, nprobe, k)
+        while t < 1.0 and S < nq:
+            S = min(nq, S * 4)
+            t = one(S, nprobe, k)
+        S2 = int(min(nq, max(S, S * args.cpu_seconds / max(t, 1e-9))))
+        t2 = one(S2, nprobe, k)
+        out["cpu_baseline"] = {"value": S2 / t2, "unit": SEARCH_UNIT,
+                               "cores": oracle.threads(), "kind": "oracle",
+                               "sample": f"oracle IVF-Flat search of {S2} queries over the "
+                                         "workload's mixture components as cells",
+                               "host_nproc": os.cpu_count()}
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+
+
+def search_reference_arm(args, spec, rank, world):
+    """The oracle's IVF-Flat search timed on the host as the reference arm: each step
+    searches a bounded sample of the query batch."""
+    if rank != 0:
+        return
+    import oracle
+    nprobe, k = args.search, args.topk
+    Qd, one = search_cpu_sample(spec, args.cpu_seconds, args.queries)
+    S = 16
+    t = one(S, nprobe, k)
+    while t < 0.5 and S < args.queries:
+        S = min(args.queries, S * 2)
+        t = one(S, nprobe, k)
+    for _ in range(args.warmup):
+        one(S, nprobe, k)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        one(S, nprobe, k)
+    dt = time.perf_counter() - t0
+    value = S * args.steps / dt
+    sample = (f"oracle IVF-Flat search of {S} of the {args.queries} queries per step, over "
+              "the workload's mixture components as cells")
+    print(json.dumps({
+        "impl": "reference", "metric": search_metric(nprobe, k), "value": value,
+        "unit": SEARCH_UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": dt * 1e3 / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": f"ivf_search_{spec.n}x{spec.d}_nlist{spec.k}_nq{args.queries}"
+                               f"_nprobe{nprobe}_k{k}_{spec.metric}",
+                   "sample_queries": S},
+        "cpu_baseline": {"value": value, "unit": SEARCH_UNIT, "cores": oracle.threads(),
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": SEARCH_UNIT, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0}}), flush=True)
+
+
 def main():
     args = parse()
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -561,7 +803,10 @@ def main():
     if args.n:
         spec = replace(spec, n=args.n, name=spec.name.replace(str(spec.n), str(args.n)))
     if args.impl == "reference":
-        reference_arm(args, spec, rank, world)
+        if args.search:
+            search_reference_arm(args, spec, rank, world)
+        else:
+            reference_arm(args, spec, rank, world)
         return
     import torch
     dist = None
@@ -582,7 +827,9 @@ def main():
             os.environ.setdefault("WORLD_SIZE", "1")
         tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=180))
         dist = tdist
-    if args.streamed:
+    if args.search:
+        search_arm(args, spec, rank, world, dist)
+    elif args.streamed:
         streamed_arm(args, spec, rank, world, dist)
     else:
         fk_arm(args, spec, rank, world, dist)

@@ -248,6 +248,60 @@ __global__ void wait_selftest_kernel(uint32_t *err, uint64_t limit_ns) {
     }
 }
 
+fk_status validate_search(int64_t nq, int d, int nlist, int64_t N, int nprobe, int k) {
+    if (nq < 1 || d < 1 || nlist < 1 || N < 1 || N > 2147483647LL - 1) return FK_ERR_INVALID_ARG;
+    if (nprobe < 1 || nprobe > nlist || nprobe > kSearchMaxProbe) return FK_ERR_INVALID_ARG;
+    if (k < 1 || k > kSearchMaxK) return FK_ERR_INVALID_ARG;
+    if (nq > (2147483647LL - 1) / nprobe) return FK_ERR_INVALID_ARG;
+    if (d % 4 != 0) return FK_ERR_UNSUPPORTED;
+    return FK_OK;
+}
+
+fk_status run_ivf_search(const float *Q, int64_t nq, int d, const float *C, int nlist,
+                         const float *X_lists, const double *X_norms, const int32_t *offsets,
+                         const int32_t *row_ids, int nprobe, int k, float *distances,
+                         int32_t *ids, int32_t *probes, void *ws, const SearchLayout &L,
+                         cudaStream_t st, const cudaEvent_t *ev) {
+    // ev (optional): five events recorded between the phases
+    auto mark = [&](int i) { return !ev || cudaEventRecord(ev[i], st) == cudaSuccess; };
+    if (!mark(0)) return FK_ERR_CUDA;
+    double *qn = ws_ptr<double>(ws, L.qn), *cn = ws_ptr<double>(ws, L.cn);
+    FK_TRY_CUDA(launch_sqnorm_f64(Q, nq, d, qn, st));
+    FK_TRY_CUDA(launch_sqnorm_f64(C, nlist, d, cn, st));
+    // coarse: distances to every centroid, then the nprobe nearest per query
+    int32_t *pr = probes ? probes : ws_ptr<int32_t>(ws, L.probes);
+    double *D = ws_ptr<double>(ws, L.D);
+    for (int64_t q0 = 0; q0 < nq; q0 += L.qbatch) {
+        const int nqb = static_cast<int>(nq - q0 < L.qbatch ? nq - q0 : L.qbatch);
+        FK_TRY_CUDA(launch_ivf_coarse(Q, qn, q0, nqb, d, C, cn, nlist, D, st));
+        FK_TRY_CUDA(launch_ivf_select(D, nullptr, nlist, nqb, nlist, nprobe, pr + q0 * nprobe,
+                                      nullptr, nprobe, st));
+    }
+    if (!mark(1)) return FK_ERR_CUDA;
+    // the (query, probe) pairs in cell order, cut into work items
+    const int32_t *skeys = nullptr, *psorted = nullptr;
+    int32_t *poff = ws_ptr<int32_t>(ws, L.poff);
+    FK_TRY_CUDA(launch_sort_csr(pr, L.P, nlist, L.sp, ws_ptr<int32_t>(ws, L.keys0),
+                                ws_ptr<int32_t>(ws, L.keys1), ws_ptr<int32_t>(ws, L.vals0),
+                                ws_ptr<int32_t>(ws, L.vals1), ws_ptr<int32_t>(ws, L.psorted),
+                                ws_ptr<uint32_t>(ws, L.hist), ws_ptr<uint32_t>(ws, L.dtot), poff,
+                                &skeys, &psorted, ws_ptr<uint32_t>(ws, L.err), st));
+    int2 *items = ws_ptr<int2>(ws, L.items);
+    int *nitems = ws_ptr<int>(ws, L.nitems);
+    FK_TRY_CUDA(launch_ivf_items(poff, nlist, items, nitems, nitems + 1, st));
+    if (!mark(2)) return FK_ERR_CUDA;
+    // fine: per pair, the k nearest points of its cell; then per query the k nearest overall
+    double *Ld = ws_ptr<double>(ws, L.Ld);
+    uint32_t *Li = ws_ptr<uint32_t>(ws, L.Li);
+    FK_TRY_CUDA(launch_ivf_fine(Q, qn, d, X_lists, X_norms, offsets, row_ids, psorted, poff,
+                                items, nitems, nitems + 1, L.max_items, nprobe, k, Ld, Li, st));
+    if (!mark(3)) return FK_ERR_CUDA;
+    const int64_t Lrow = static_cast<int64_t>(nprobe) * k;
+    FK_TRY_CUDA(launch_ivf_select(Ld, Li, Lrow, nq, static_cast<int>(Lrow), k, ids, distances,
+                                  k, st));
+    if (!mark(4)) return FK_ERR_CUDA;
+    return FK_OK;
+}
 }  // namespace
 }  // namespace fk
 
@@ -787,6 +841,74 @@ fk_status fk_finalize_shards(const double *sums, const int64_t *counts_w,
                                        counts, objective, stream));
     return FK_OK;
 }
+
+fk_status fk_ivf_norms(const float *V, int64_t n, int d, double *norms, fk_stream_t stream) {
+    if (!V || !norms || n < 1 || d < 1) return FK_ERR_INVALID_ARG;
+    if (d % 4 != 0 || !aligned(V, 16) || !aligned(norms, 8)) return FK_ERR_UNSUPPORTED;
+    fk_status s = check_device();
+    if (s != FK_OK) return s;
+    FK_TRY_CUDA(launch_sqnorm_f64(V, n, d, norms, stream));
+    return FK_OK;
+}
+
+
+fk_status fk_ivf_search_workspace_size(int64_t nq, int d, int nlist, int64_t N, int nprobe,
+                                       int k, size_t *bytes) {
+    if (!bytes) return FK_ERR_INVALID_ARG;
+    fk_status s = validate_search(nq, d, nlist, N, nprobe, k);
+    if (s != FK_OK) return s;
+    *bytes = search_layout(nq, d, nlist, nprobe, k).total;
+    return FK_OK;
+}
+
+fk_status fk_ivf_search(const float *Q, int64_t nq, int d, const float *C, int nlist,
+                        const float *X_lists, const double *X_norms, const int32_t *offsets,
+                        const int32_t *row_ids, int64_t N, int nprobe, int k,
+                        float *distances, int32_t *ids, int32_t *probes, void *ws,
+                        size_t ws_bytes, fk_search_timing *timing, fk_stream_t stream) {
+    fk_status s = validate_search(nq, d, nlist, N, nprobe, k);
+    if (s != FK_OK) return s;
+    if (!Q || !C || !X_lists || !X_norms || !offsets || !row_ids || !distances || !ids)
+        return FK_ERR_INVALID_ARG;
+    if (!aligned(Q, 16) || !aligned(C, 16) || !aligned(X_lists, 16) || !aligned(X_norms, 8) ||
+        !aligned(offsets, 4) || !aligned(row_ids, 4) || !aligned(distances, 4) ||
+        !aligned(ids, 4) || (probes && !aligned(probes, 4)))
+        return FK_ERR_UNSUPPORTED;
+    const SearchLayout L = search_layout(nq, d, nlist, nprobe, k);
+    if (ws == nullptr || !aligned(ws, 256) || ws_bytes < L.total) return FK_ERR_WORKSPACE;
+    if ((s = check_device()) != FK_OK) return s;
+    cudaStream_t st = stream;
+    cudaEvent_t ev[5] = {};
+    auto destroy = [&]() {
+        for (cudaEvent_t &e : ev)
+            if (e) cudaEventDestroy(e);
+    };
+    if (timing) {
+        for (cudaEvent_t &e : ev)
+            if (cudaEventCreate(&e) != cudaSuccess) {
+                destroy();
+                return FK_ERR_CUDA;
+            }
+    }
+    const fk_status r = run_ivf_search(Q, nq, d, C, nlist, X_lists, X_norms, offsets, row_ids,
+                                       nprobe, k, distances, ids, probes, ws, L, st,
+                                       timing ? ev : nullptr);
+    if (r == FK_OK && timing) {
+        if (cudaStreamSynchronize(st) != cudaSuccess) {
+            destroy();
+            return FK_ERR_CUDA;
+        }
+        float ms[4] = {0, 0, 0, 0};
+        for (int i = 0; i < 4; ++i) cudaEventElapsedTime(&ms[i], ev[i], ev[i + 1]);
+        timing->ms_coarse = ms[0];
+        timing->ms_sort = ms[1];
+        timing->ms_fine = ms[2];
+        timing->ms_merge = ms[3];
+    }
+    destroy();
+    return r;
+}
+
 
 fk_status fk_get_device_error(void *ws, size_t ws_bytes, int *code, fk_stream_t stream) {
     if (!ws || !code || ws_bytes < 256 || !aligned(ws, 256)) return FK_ERR_INVALID_ARG;

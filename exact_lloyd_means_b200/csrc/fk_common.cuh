@@ -264,6 +264,75 @@ cudaError_t launch_finalize_shards(const double *sums, const int64_t *cnts, cons
                                    int W, int K, int d, const float *C_old, float *C_new,
                                    int64_t *counts, double *objective, cudaStream_t st);
 
+// IVF-Flat search (ivf_search.cu).
+cudaError_t launch_sqnorm_f64(const float *V, int64_t n, int d, double *out, cudaStream_t st);
+cudaError_t launch_ivf_coarse(const float *Q, const double *qn, int64_t q0, int nqb, int d,
+                              const float *C, const double *cn, int nlist, double *D,
+                              cudaStream_t st);
+cudaError_t launch_ivf_select(const double *D, const uint32_t *I, int64_t ld, int64_t rows, int L,
+                              int m, int32_t *out_id, float *out_dist, int64_t ldo,
+                              cudaStream_t st);
+cudaError_t launch_ivf_items(const int32_t *pair_off, int nlist, int2 *items, int *nitems,
+                             int *ctr, cudaStream_t st);
+cudaError_t launch_ivf_fine(const float *Q, const double *qn, int d, const float *X_lists,
+                            const double *xn, const int32_t *offsets, const int32_t *row_ids,
+                            const int32_t *pair_sorted, const int32_t *pair_off,
+                            const int2 *items, const int *nitems, int *item_ctr, int64_t max_items,
+                            int nprobe, int k, double *Ld, uint32_t *Li, cudaStream_t st);
+
+// Limits of fk_ivf_search: k is held one rank per lane, nprobe by the selection's sort.
+constexpr int kSearchMaxK = 32;
+constexpr int kSearchMaxProbe = 1024;
+constexpr int kSearchPairsPerItem = 32;
+// Rows of the coarse distance matrix held at once: a query batch of at most this many bytes.
+constexpr int64_t kSearchCoarseBytes = int64_t(512) << 20;
+
+struct SearchLayout {
+    size_t err = 0, qn = 0, cn = 0, D = 0, probes = 0, keys0 = 0, keys1 = 0, vals0 = 0,
+           vals1 = 0, hist = 0, dtot = 0, psorted = 0, poff = 0, items = 0, nitems = 0,
+           Ld = 0, Li = 0, total = 0;
+    int64_t P = 0, qbatch = 0, max_items = 0;
+    SortPlan sp;
+};
+
+inline SearchLayout search_layout(int64_t nq, int d, int nlist, int nprobe, int k) {
+    (void)d;
+    SearchLayout L;
+    L.P = nq * nprobe;
+    int64_t qb = kSearchCoarseBytes / (static_cast<int64_t>(nlist) * 8);
+    qb = qb / 32 * 32;
+    if (qb < 32) qb = 32;
+    L.qbatch = qb < nq ? qb : nq;
+    L.sp = sort_plan(L.P, nlist);
+    L.max_items = nlist + ceil_div(L.P, kSearchPairsPerItem);
+    size_t o = 0;
+    auto take = [&](size_t bytes) {
+        size_t at = o;
+        o += static_cast<size_t>(round_up(static_cast<int64_t>(bytes > 0 ? bytes : 1), 256));
+        return at;
+    };
+    L.err = take(256);
+    L.qn = take(sizeof(double) * nq);
+    L.cn = take(sizeof(double) * nlist);
+    L.D = take(sizeof(double) * L.qbatch * nlist);
+    L.probes = take(sizeof(int32_t) * L.P);
+    L.keys0 = take(sizeof(int32_t) * L.P);
+    L.keys1 = take(sizeof(int32_t) * L.P);
+    L.vals0 = take(sizeof(int32_t) * L.P);
+    L.vals1 = take(sizeof(int32_t) * L.P);
+    const int64_t bins = int64_t(1) << (L.sp.bits > 0 ? L.sp.bits : 1);
+    L.hist = take(sizeof(uint32_t) * bins * L.sp.nblocks);
+    L.dtot = take(sizeof(uint32_t) * bins);
+    L.psorted = take(sizeof(int32_t) * L.P);
+    L.poff = take(sizeof(int32_t) * (nlist + 1));
+    L.items = take(sizeof(int32_t) * 2 * L.max_items);
+    L.nitems = take(sizeof(int32_t) * 2);
+    L.Ld = take(sizeof(double) * L.P * k);
+    L.Li = take(sizeof(uint32_t) * L.P * k);
+    L.total = o;
+    return L;
+}
+
 int device_sm_count();
 
 // Kernels launched by this host thread since the last reset (fk_lloyd reports it).

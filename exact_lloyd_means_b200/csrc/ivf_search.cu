@@ -1,0 +1,663 @@
+// ivf_search.cu -- IVF-Flat search over the inverted lists of a finished clustering.
+//
+// LEANN FlashLib guide: an IVF-Flat index fitted on a corpus answers the k nearest
+// neighbours of a batch of queries (section "什么是 FlashLib 后端"); its cells are the coarse
+// k-means clusters, stored cell-contiguous with row ids and CSR offsets (section "工作原理");
+// a query probes nprobe cells (sections "nlist 与 nprobe 的推导规则", "参数速查"); the only
+// distance is squared L2 (section "距离度量只有 squared L2").
+//
+// One search call, per batch of queries:
+//   1. fp64 norms of the queries and centroids (the points' norms come with the index);
+//   2. coarse: the fp64 distance of every query to every centroid (tile kernel, COARSE
+//      mode, written to a query-batch x nlist matrix), then per query the nprobe smallest
+//      by (distance, cell) (radix select);
+//   3. the (query, probe) pairs sorted by cell with the same stable LSD sort as the update,
+//      cut into work items of up to 32 pairs of one cell;
+//   4. fine: for every item, the fp64 distances of its queries to every point of its cell
+//      (tile kernel, FINE mode), keeping per pair the k smallest by (distance, point id)
+//      in registers;
+//   5. per query, the k smallest of its nprobe pair lists (radix select).
+//
+// Every distance is ||q||^2 + ||v||^2 - 2 q.v in fp64: products of two fp32 values are exact
+// in fp64, the dot product accumulates with fp64 FMAs in dimension order, and the norms are
+// fp64 sums of squares.  The result differs from the difference form sum_j (q_j - v_j)^2 by
+// rounding at the 1e-16 relative level of the norms, so the selections agree with an fp64
+// evaluation except between candidates that close.  Selections use the strict total order
+// (distance, id): the k smallest entries form a unique set, whatever order they were seen in.
+#include <cmath>
+
+#include "fk_common.cuh"
+
+namespace fk {
+namespace {
+
+constexpr unsigned kFull = 0xffffffffu;
+
+// ---------------------------------------------------------------- fp64 tile geometry
+// A tile is 32 queries x 128 vectors; 4 warps, warp w owns queries 8w..8w+7 and lane l
+// owns vectors l, l+32, l+64, l+96.  Dimensions are staged in chunks of 32, converted to
+// fp64 once at staging.  The vector rows in shared memory are 34 doubles long: a
+// quarter-warp's 16-byte reads at one dimension then fall on distinct banks.
+constexpr int kTQ = 32;
+constexpr int kTV = 128;
+constexpr int kTD = 32;
+constexpr int kVS = kTD + 2;
+constexpr int kTThreads = 128;
+
+struct TileSmem {
+    double q[kTQ * kTD];  // [query][dim]
+    double v[kTV * kVS];  // [vector][dim], padded rows
+};
+
+// Registers of one staged chunk: 8 float4 of vectors and 2 of queries per thread.
+struct Stage {
+    float4 v[8];
+    float4 q[2];
+};
+
+__device__ __forceinline__ bool before(double da, uint32_t ia, double db, uint32_t ib) {
+    return da < db || (da == db && ia < ib);
+}
+
+// Element f of a chunk (f = tid + 128 r): row f / 8, float4 column f % 8.  A row's 128-byte
+// piece is read by 8 consecutive lanes.
+__device__ __forceinline__ void stage_load(Stage &s, const float *V, int nv, const float *qrow0,
+                                           const float *qrow1, int d, int j0, int tid) {
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+        const int f = tid + kTThreads * r;
+        const int row = f >> 3;
+        const int j = j0 + (f & 7) * 4;
+        s.v[r] = (row < nv && j < d)
+                     ? __ldg(reinterpret_cast<const float4 *>(V + static_cast<int64_t>(row) * d + j))
+                     : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    const int j = j0 + (tid & 7) * 4;
+    s.q[0] = (qrow0 && j < d) ? __ldg(reinterpret_cast<const float4 *>(qrow0 + j))
+                              : make_float4(0.f, 0.f, 0.f, 0.f);
+    s.q[1] = (qrow1 && j < d) ? __ldg(reinterpret_cast<const float4 *>(qrow1 + j))
+                              : make_float4(0.f, 0.f, 0.f, 0.f);
+}
+
+__device__ __forceinline__ void put4(double *p, float4 x) {
+    reinterpret_cast<double2 *>(p)[0] = make_double2(x.x, x.y);
+    reinterpret_cast<double2 *>(p)[1] = make_double2(x.z, x.w);
+}
+
+__device__ __forceinline__ void stage_store(const Stage &s, TileSmem &sm, int tid) {
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+        const int f = tid + kTThreads * r;
+        put4(sm.v + (f >> 3) * kVS + (f & 7) * 4, s.v[r]);
+    }
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+        const int f = tid + kTThreads * r;
+        put4(sm.q + (f >> 3) * kTD + (f & 7) * 4, s.q[r]);
+    }
+}
+
+// acc[a][i] += sum over the chunk's dimensions of q[8w + a][j] * v[l + 32 i][j], in
+// dimension order.
+__device__ __forceinline__ void tile_fma(const TileSmem &sm, int warp, int lane,
+                                         double (&acc)[8][4]) {
+    const double *qb = sm.q + warp * 8 * kTD;
+    const double *vb = sm.v + lane * kVS;
+#pragma unroll 2
+    for (int j = 0; j < kTD; j += 2) {
+        double2 vv[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            vv[i] = *reinterpret_cast<const double2 *>(vb + i * 32 * kVS + j);
+#pragma unroll
+        for (int a = 0; a < 8; ++a) {
+            const double2 qq = *reinterpret_cast<const double2 *>(qb + a * kTD + j);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                acc[a][i] = fma(qq.x, vv[i].x, acc[a][i]);
+                acc[a][i] = fma(qq.y, vv[i].y, acc[a][i]);
+            }
+        }
+    }
+}
+
+struct TileArgs {
+    const float *Q;       // [nq][d] queries
+    const double *qn;     // [nq] ||q||^2
+    const float *V;       // COARSE: centroids [nlist][d]; FINE: cell-contiguous points [N][d]
+    const double *vn;     // ||v||^2 of the rows of V
+    int d;
+    // COARSE
+    int64_t q0;           // first query of the batch
+    int nqb;              // queries in the batch
+    int nv;               // centroids
+    int vchunk;           // centroids per work item (a multiple of kTV)
+    int nvchunks;
+    double *D;            // [nqb][nv]
+    // FINE
+    const int32_t *offsets;      // [nlist + 1] cell starts in V
+    const int32_t *row_ids;      // [N] original index of every row of V
+    const int32_t *pair_sorted;  // pairs (q * nprobe + t) in cell order
+    const int32_t *pair_off;     // [nlist + 1] first sorted position of every cell
+    const int2 *items;           // (cell, first sorted position)
+    const int *nitems;
+    int *item_ctr;               // zero at launch
+    int nprobe, k;
+    double *Ld;                  // [nq * nprobe][k]
+    uint32_t *Li;
+};
+
+// COARSE: blockIdx.x = query block * nvchunks + centroid chunk; writes distances.
+// FINE: persistent blocks take work items from a counter; writes per-pair top-k lists.
+// Padding ids of a pair list are 0x80000000 | (t * k + rank), unique within a query, above
+// every point id and recognised as "no point" by the final selection.
+template <bool FINE>
+__global__ void __launch_bounds__(kTThreads, 3) ivf_tile_kernel(TileArgs a) {
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    TileSmem &sm = *reinterpret_cast<TileSmem *>(smem_raw);
+    __shared__ int s_item;
+    __shared__ int s_pair[kTQ];
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int d = a.d;
+
+    for (int round = 0;; ++round) {
+        int item;
+        if (FINE) {
+            if (tid == 0) s_item = atomicAdd(a.item_ctr, 1);
+            __syncthreads();
+            item = s_item;
+            if (item >= *a.nitems) return;
+        } else {
+            if (round > 0) return;
+            item = blockIdx.x;
+        }
+        int nq_i;
+        int64_t vbeg, vend, q_first = 0;
+        if (FINE) {
+            const int2 it = a.items[item];
+            nq_i = min(kTQ, a.pair_off[it.x + 1] - it.y);
+            vbeg = a.offsets[it.x];
+            vend = a.offsets[it.x + 1];
+            if (tid < kTQ) s_pair[tid] = tid < nq_i ? a.pair_sorted[it.y + tid] : 0;
+        } else {
+            const int qb = item / a.nvchunks, vc = item % a.nvchunks;
+            q_first = static_cast<int64_t>(qb) * kTQ;
+            nq_i = static_cast<int>(min(static_cast<int64_t>(kTQ), a.nqb - q_first));
+            vbeg = static_cast<int64_t>(vc) * a.vchunk;
+            vend = min(vbeg + a.vchunk, static_cast<int64_t>(a.nv));
+        }
+        __syncthreads();
+
+        auto query_of = [&](int qi) -> int64_t {
+            return FINE ? static_cast<int64_t>(s_pair[qi] / a.nprobe) : a.q0 + q_first + qi;
+        };
+        const int sq0 = tid >> 3, sq1 = (tid + kTThreads) >> 3;  // query rows this thread stages
+        const float *qrow0 = sq0 < nq_i ? a.Q + query_of(sq0) * d : nullptr;
+        const float *qrow1 = sq1 < nq_i ? a.Q + query_of(sq1) * d : nullptr;
+
+        // per-pair top-k lists: lane r holds rank r of each of the warp's 8 queries
+        double ld[8];
+        uint32_t li[8];
+#pragma unroll
+        for (int q8 = 0; q8 < 8; ++q8) {
+            ld[q8] = INFINITY;
+            li[q8] = 0xffffffffu;
+            if (FINE) {
+                const int qi = warp * 8 + q8;
+                if (qi < nq_i && lane < a.k)
+                    li[q8] = 0x80000000u |
+                             static_cast<uint32_t>((s_pair[qi] % a.nprobe) * a.k + lane);
+            }
+        }
+
+        for (int64_t v0 = vbeg; v0 < vend; v0 += kTV) {
+            const int nv_t = static_cast<int>(min(static_cast<int64_t>(kTV), vend - v0));
+            const float *Vt = a.V + v0 * d;
+            double acc[8][4];
+#pragma unroll
+            for (int q8 = 0; q8 < 8; ++q8)
+#pragma unroll
+                for (int i = 0; i < 4; ++i) acc[q8][i] = 0.0;
+            Stage st;
+            stage_load(st, Vt, nv_t, qrow0, qrow1, d, 0, tid);
+            for (int j0 = 0; j0 < d; j0 += kTD) {
+                __syncthreads();  // the previous chunk's readers are done
+                stage_store(st, sm, tid);
+                __syncthreads();
+                if (j0 + kTD < d) stage_load(st, Vt, nv_t, qrow0, qrow1, d, j0 + kTD, tid);
+                tile_fma(sm, warp, lane, acc);
+            }
+
+            double vn_i[4];
+            uint32_t id_i[4];
+            bool ok_i[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int vl = lane + 32 * i;
+                ok_i[i] = vl < nv_t;
+                vn_i[i] = ok_i[i] ? a.vn[v0 + vl] : 0.0;
+                id_i[i] = FINE ? (ok_i[i] ? static_cast<uint32_t>(a.row_ids[v0 + vl]) : 0u)
+                               : static_cast<uint32_t>(v0 + vl);
+            }
+#pragma unroll
+            for (int q8 = 0; q8 < 8; ++q8) {
+                const int qi = warp * 8 + q8;
+                if (qi >= nq_i) continue;  // warp-uniform
+                const double qn = a.qn[query_of(qi)];
+                if (!FINE) {
+                    double *Drow = a.D + (q_first + qi) * static_cast<int64_t>(a.nv);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i)
+                        if (ok_i[i]) Drow[v0 + lane + 32 * i] = fma(-2.0, acc[q8][i], qn + vn_i[i]);
+                } else {
+                    double td = __shfl_sync(kFull, ld[q8], a.k - 1);
+                    uint32_t ti = __shfl_sync(kFull, li[q8], a.k - 1);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const double cd = fma(-2.0, acc[q8][i], qn + vn_i[i]);
+                        const uint32_t ci = id_i[i];
+                        bool pend = ok_i[i] && before(cd, ci, td, ti);
+                        unsigned m = __ballot_sync(kFull, pend);
+                        while (m) {
+                            const int src = __ffs(m) - 1;
+                            const double xd = __shfl_sync(kFull, cd, src);
+                            const uint32_t xi = __shfl_sync(kFull, ci, src);
+                            const int pos = __popc(__ballot_sync(
+                                kFull, lane < a.k && before(ld[q8], li[q8], xd, xi)));
+                            const double ud = __shfl_up_sync(kFull, ld[q8], 1);
+                            const uint32_t ui = __shfl_up_sync(kFull, li[q8], 1);
+                            if (lane == pos) {
+                                ld[q8] = xd;
+                                li[q8] = xi;
+                            } else if (lane > pos && lane < a.k) {
+                                ld[q8] = ud;
+                                li[q8] = ui;
+                            }
+                            td = __shfl_sync(kFull, ld[q8], a.k - 1);
+                            ti = __shfl_sync(kFull, li[q8], a.k - 1);
+                            if (lane == src) pend = false;
+                            pend = pend && before(cd, ci, td, ti);
+                            m = __ballot_sync(kFull, pend);
+                        }
+                    }
+                }
+            }
+        }
+
+        if (FINE) {
+#pragma unroll
+            for (int q8 = 0; q8 < 8; ++q8) {
+                const int qi = warp * 8 + q8;
+                if (qi < nq_i && lane < a.k) {
+                    const int64_t at = static_cast<int64_t>(s_pair[qi]) * a.k + lane;
+                    a.Ld[at] = ld[q8];
+                    a.Li[at] = li[q8];
+                }
+            }
+        }
+    }
+}
+
+// ---------------------------------------------------------------- row selection
+// Per row (one block each): the m smallest entries by (distance, id), output in ascending
+// order.  The m-th smallest 96-bit key (order-preserving distance bits, then id) is found
+// digit by digit, 8 bits at a time, with a 256-bin histogram of the entries that still
+// match the decided digits; the search stops as soon as every entry of the chosen bin is
+// inside the first m.  The selected entries are then gathered and sorted (bitonic).
+constexpr int kSelThreads = 256;
+constexpr int kSelMaxM = 1024;   // largest m
+constexpr int kSelCache = 8192;  // rows up to this length are staged in shared memory
+
+__device__ __forceinline__ uint64_t order_key(double x) {
+    const uint64_t u = static_cast<uint64_t>(__double_as_longlong(x));
+    return (u >> 63) ? ~u : (u | 0x8000000000000000ull);
+}
+
+__device__ __forceinline__ double key_value(uint64_t k) {
+    const uint64_t u = (k >> 63) ? (k & 0x7fffffffffffffffull) : ~k;
+    return __longlong_as_double(static_cast<long long>(u));
+}
+
+struct SelArgs {
+    const double *D;    // [rows][ld] distances
+    const uint32_t *I;  // [rows][ld] ids, or null: the id of entry j is j
+    int64_t ld;
+    int L, m;
+    int32_t *out_id;    // [rows][ldo]; ids with bit 31 set are written as -1
+    float *out_dist;    // optional [rows][ldo]; +inf for those
+    int64_t ldo;
+};
+
+template <bool CACHE>
+__global__ void __launch_bounds__(kSelThreads) select_rows_kernel(SelArgs a) {
+    extern __shared__ __align__(16) unsigned char sel_raw[];
+    uint64_t *ck = reinterpret_cast<uint64_t *>(sel_raw);
+    uint32_t *ci = reinterpret_cast<uint32_t *>(sel_raw + sizeof(uint64_t) * (CACHE ? a.L : 0));
+    __shared__ uint32_t hist[256];
+    __shared__ uint64_t sel_k[kSelMaxM];
+    __shared__ uint32_t sel_i[kSelMaxM];
+    __shared__ uint64_t s_phi;
+    __shared__ uint32_t s_plo;
+    __shared__ int s_r, s_done, s_cnt;
+
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int64_t row = blockIdx.x;
+    const double *drow = a.D + row * a.ld;
+    const uint32_t *irow = a.I ? a.I + row * a.ld : nullptr;
+    const int L = a.L, m = a.m;
+    const int Lpad = (L + kSelThreads - 1) / kSelThreads * kSelThreads;
+
+    if (CACHE) {
+        for (int j = tid; j < L; j += kSelThreads) {
+            ck[j] = order_key(drow[j]);
+            ci[j] = irow ? irow[j] : static_cast<uint32_t>(j);
+        }
+    }
+    if (tid == 0) {
+        s_phi = 0;
+        s_plo = 0;
+        s_r = m - 1;
+        s_done = 0;
+        s_cnt = 0;
+    }
+    auto load = [&](int j, uint64_t &kh, uint32_t &kl) {
+        if (CACHE) {
+            kh = ck[j];
+            kl = ci[j];
+        } else {
+            kh = order_key(drow[j]);
+            kl = irow ? irow[j] : static_cast<uint32_t>(j);
+        }
+    };
+    auto hi_mask = [](int b) -> uint64_t { return b >= 8 ? ~0ull : (b == 0 ? 0ull : ~0ull << (64 - 8 * b)); };
+    auto lo_mask = [](int b) -> uint32_t { return b <= 8 ? 0u : ~0u << (32 - 8 * (b - 8)); };
+
+    int b = 0;
+    while (b < 12) {
+        hist[tid] = 0;
+        __syncthreads();
+        const uint64_t phi = s_phi, mhi = hi_mask(b);
+        const uint32_t plo = s_plo, mlo = lo_mask(b);
+        for (int j = tid; j < Lpad; j += kSelThreads) {
+            uint64_t kh = 0;
+            uint32_t kl = 0;
+            const bool valid = j < L;
+            if (valid) load(j, kh, kl);
+            const bool match = valid && (kh & mhi) == phi && (kl & mlo) == plo;
+            int dig = b < 8 ? static_cast<int>((kh >> (56 - 8 * b)) & 255u)
+                            : static_cast<int>((kl >> (24 - 8 * (b - 8))) & 255u);
+            dig = match ? dig : 256;
+            const unsigned peers = __match_any_sync(kFull, dig);
+            if (match && lane == __ffs(peers) - 1) atomicAdd(&hist[dig], __popc(peers));
+        }
+        __syncthreads();
+        if (warp == 0) {
+            uint32_t h[8], sum = 0;
+#pragma unroll
+            for (int t = 0; t < 8; ++t) {
+                h[t] = hist[lane * 8 + t];
+                sum += h[t];
+            }
+            uint32_t incl = sum;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const uint32_t y = __shfl_up_sync(kFull, incl, o);
+                if (lane >= o) incl += y;
+            }
+            const uint32_t excl = incl - sum;
+            const uint32_t r = static_cast<uint32_t>(s_r);
+            if (excl <= r && r < incl) {
+                uint32_t c = excl;
+#pragma unroll
+                for (int t = 0; t < 8; ++t) {
+                    if (r >= c && r < c + h[t]) {
+                        const uint32_t bin = lane * 8 + t;
+                        if (b < 8)
+                            s_phi = phi | (static_cast<uint64_t>(bin) << (56 - 8 * b));
+                        else
+                            s_plo = plo | (bin << (24 - 8 * (b - 8)));
+                        s_r = static_cast<int>(r - c);
+                        s_done = (r - c + 1 == h[t]) ? 1 : 0;
+                    }
+                    c += h[t];
+                }
+            }
+        }
+        __syncthreads();
+        ++b;
+        if (s_done) break;
+    }
+
+    // every entry whose first b digits are at most the decided prefix is selected: exactly m
+    {
+        const uint64_t phi = s_phi, mhi = hi_mask(b);
+        const uint32_t plo = s_plo, mlo = lo_mask(b);
+        for (int j = tid; j < L; j += kSelThreads) {
+            uint64_t kh;
+            uint32_t kl;
+            load(j, kh, kl);
+            const uint64_t th = kh & mhi;
+            const uint32_t tl = kl & mlo;
+            if (th < phi || (th == phi && tl <= plo)) {
+                const int at = atomicAdd(&s_cnt, 1);
+                if (at < kSelMaxM) {
+                    sel_k[at] = kh;
+                    sel_i[at] = kl;
+                }
+            }
+        }
+    }
+    int M = 1;
+    while (M < m) M <<= 1;
+    __syncthreads();
+    for (int t = m + tid; t < M; t += kSelThreads) {
+        sel_k[t] = ~0ull;
+        sel_i[t] = ~0u;
+    }
+    __syncthreads();
+    for (int size = 2; size <= M; size <<= 1) {
+        for (int stride = size >> 1; stride > 0; stride >>= 1) {
+            for (int t = tid; t < (M >> 1); t += kSelThreads) {
+                const int lo = 2 * t - (t & (stride - 1));
+                const int hi = lo + stride;
+                const bool up = (lo & size) == 0;
+                const uint64_t ka = sel_k[lo], kb = sel_k[hi];
+                const uint32_t ia = sel_i[lo], ib = sel_i[hi];
+                const bool gt = ka > kb || (ka == kb && ia > ib);
+                if (gt == up) {
+                    sel_k[lo] = kb;
+                    sel_k[hi] = ka;
+                    sel_i[lo] = ib;
+                    sel_i[hi] = ia;
+                }
+            }
+            __syncthreads();
+        }
+    }
+    for (int t = tid; t < m; t += kSelThreads) {
+        const uint32_t id = sel_i[t];
+        const bool pad = (id & 0x80000000u) != 0;
+        a.out_id[row * a.ldo + t] = pad ? -1 : static_cast<int32_t>(id);
+        if (a.out_dist)
+            a.out_dist[row * a.ldo + t] =
+                pad ? INFINITY : static_cast<float>(fmax(key_value(sel_k[t]), 0.0));
+    }
+}
+
+// ---------------------------------------------------------------- small kernels
+// ||v||^2 in fp64, a warp per row: lane partial sums over float4 columns, then a fixed
+// butterfly.
+__global__ void sqnorm_f64_kernel(const float *__restrict__ V, int64_t n, int d,
+                                  double *__restrict__ out) {
+    const int lane = threadIdx.x & 31;
+    const int64_t w0 = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+    const int64_t nw = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+    for (int64_t r = w0; r < n; r += nw) {
+        const float *x = V + r * d;
+        double s = 0.0;
+        for (int j = lane * 4; j < d; j += 128) {
+            const float4 v = __ldg(reinterpret_cast<const float4 *>(x + j));
+            s = fma(static_cast<double>(v.x), static_cast<double>(v.x), s);
+            s = fma(static_cast<double>(v.y), static_cast<double>(v.y), s);
+            s = fma(static_cast<double>(v.z), static_cast<double>(v.z), s);
+            s = fma(static_cast<double>(v.w), static_cast<double>(v.w), s);
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(kFull, s, o);
+        if (lane == 0) out[r] = s;
+    }
+}
+
+// Work items of the fine pass: a cell probed by n pairs gives ceil(n / 32) items, in cell
+// order.  One block; cells in rounds of 1024 with a running base.
+__global__ void __launch_bounds__(1024) build_items_kernel(const int32_t *__restrict__ pair_off,
+                                                           int nlist, int2 *__restrict__ items,
+                                                           int *nitems, int *ctr) {
+    __shared__ int wsum[32];
+    __shared__ int s_base;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    if (tid == 0) s_base = 0;
+    __syncthreads();
+    for (int c0 = 0; c0 < nlist; c0 += 1024) {
+        const int c = c0 + tid;
+        const int start = c < nlist ? pair_off[c] : 0;
+        const int cnt = c < nlist ? (pair_off[c + 1] - start + kTQ - 1) / kTQ : 0;
+        int incl = cnt;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(kFull, incl, o);
+            if (lane >= o) incl += y;
+        }
+        if (lane == 31) wsum[warp] = incl;
+        __syncthreads();
+        if (warp == 0) {
+            int w = wsum[lane];
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(kFull, w, o);
+                if (lane >= o) w += y;
+            }
+            wsum[lane] = w;  // inclusive
+        }
+        __syncthreads();
+        const int base = s_base + (warp ? wsum[warp - 1] : 0) + incl - cnt;
+        for (int t = 0; t < cnt; ++t) items[base + t] = make_int2(c, start + t * kTQ);
+        __syncthreads();
+        if (tid == 0) s_base += wsum[31];
+        __syncthreads();
+    }
+    if (tid == 0) {
+        *nitems = s_base;
+        *ctr = 0;
+    }
+}
+
+}  // namespace
+
+// ---------------------------------------------------------------- host side
+size_t ivf_tile_smem() { return sizeof(TileSmem); }
+
+cudaError_t launch_sqnorm_f64(const float *V, int64_t n, int d, double *out, cudaStream_t st) {
+    if (n <= 0) return cudaSuccess;
+    const int64_t blocks = ceil_div(n, 8);
+    const int grid = static_cast<int>(blocks < 148 * 16 ? blocks : 148 * 16);
+    sqnorm_f64_kernel<<<grid, 256, 0, st>>>(V, n, d, out);
+    note_launch();
+    return cudaGetLastError();
+}
+
+cudaError_t launch_ivf_coarse(const float *Q, const double *qn, int64_t q0, int nqb, int d,
+                              const float *C, const double *cn, int nlist, double *D,
+                              cudaStream_t st) {
+    TileArgs a{};
+    a.Q = Q;
+    a.qn = qn;
+    a.V = C;
+    a.vn = cn;
+    a.d = d;
+    a.q0 = q0;
+    a.nqb = nqb;
+    a.nv = nlist;
+    a.D = D;
+    const int64_t qblocks = ceil_div(nqb, kTQ);
+    // enough items for about four waves of three blocks per SM
+    const int64_t want = static_cast<int64_t>(device_sm_count()) * 3 * 4;
+    int64_t chunks = ceil_div(want, qblocks);
+    const int64_t maxchunks = ceil_div(nlist, kTV);
+    if (chunks > maxchunks) chunks = maxchunks;
+    if (chunks < 1) chunks = 1;
+    a.vchunk = static_cast<int>(round_up(ceil_div(nlist, chunks), kTV));
+    a.nvchunks = static_cast<int>(ceil_div(nlist, a.vchunk));
+    const int64_t grid = qblocks * a.nvchunks;
+    ivf_tile_kernel<false><<<static_cast<unsigned>(grid), kTThreads, sizeof(TileSmem), st>>>(a);
+    note_launch();
+    return cudaGetLastError();
+}
+
+cudaError_t launch_ivf_select(const double *D, const uint32_t *I, int64_t ld, int64_t rows, int L,
+                              int m, int32_t *out_id, float *out_dist, int64_t ldo,
+                              cudaStream_t st) {
+    if (rows <= 0) return cudaSuccess;
+    SelArgs a{D, I, ld, L, m, out_id, out_dist, ldo};
+    if (L <= kSelCache) {
+        const size_t smem = static_cast<size_t>(L) * (sizeof(uint64_t) + sizeof(uint32_t));
+        static bool attr = false;
+        if (!attr) {
+            cudaFuncSetAttribute(select_rows_kernel<true>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(kSelCache * (sizeof(uint64_t) + sizeof(uint32_t))));
+            attr = true;
+        }
+        select_rows_kernel<true><<<static_cast<unsigned>(rows), kSelThreads, smem, st>>>(a);
+    } else {
+        select_rows_kernel<false><<<static_cast<unsigned>(rows), kSelThreads, 0, st>>>(a);
+    }
+    note_launch();
+    return cudaGetLastError();
+}
+
+cudaError_t launch_ivf_items(const int32_t *pair_off, int nlist, int2 *items, int *nitems,
+                             int *ctr, cudaStream_t st) {
+    build_items_kernel<<<1, 1024, 0, st>>>(pair_off, nlist, items, nitems, ctr);
+    note_launch();
+    return cudaGetLastError();
+}
+
+cudaError_t launch_ivf_fine(const float *Q, const double *qn, int d, const float *X_lists,
+                            const double *xn, const int32_t *offsets, const int32_t *row_ids,
+                            const int32_t *pair_sorted, const int32_t *pair_off,
+                            const int2 *items, const int *nitems, int *item_ctr, int64_t max_items,
+                            int nprobe, int k, double *Ld, uint32_t *Li, cudaStream_t st) {
+    TileArgs a{};
+    a.Q = Q;
+    a.qn = qn;
+    a.V = X_lists;
+    a.vn = xn;
+    a.d = d;
+    a.offsets = offsets;
+    a.row_ids = row_ids;
+    a.pair_sorted = pair_sorted;
+    a.pair_off = pair_off;
+    a.items = items;
+    a.nitems = nitems;
+    a.item_ctr = item_ctr;
+    a.nprobe = nprobe;
+    a.k = k;
+    a.Ld = Ld;
+    a.Li = Li;
+    static int occ = 0;
+    if (occ == 0) {
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, ivf_tile_kernel<true>, kTThreads,
+                                                          sizeof(TileSmem)) != cudaSuccess ||
+            occ < 1)
+            occ = 1;
+    }
+    int64_t grid = static_cast<int64_t>(device_sm_count()) * occ;
+    if (grid > max_items) grid = max_items;
+    if (grid < 1) grid = 1;
+    ivf_tile_kernel<true><<<static_cast<unsigned>(grid), kTThreads, sizeof(TileSmem), st>>>(a);
+    note_launch();
+    return cudaGetLastError();
+}
+
+}  // namespace fk

@@ -40,6 +40,11 @@ class FkTiming(ctypes.Structure):
                 ("screened", ctypes.c_int)]
 
 
+class FkSearchTiming(ctypes.Structure):
+    _fields_ = [("ms_coarse", ctypes.c_double), ("ms_sort", ctypes.c_double),
+                ("ms_fine", ctypes.c_double), ("ms_merge", ctypes.c_double)]
+
+
 def _sig(name, args, res=ctypes.c_int):
     f = getattr(_lib, name)
     f.argtypes = args
@@ -70,13 +75,18 @@ _sig("fk_ivf_lists", [_vp, _int, _i64, _int, _int, _vp, _vp, _vp, _vp, _vp, _sz,
 _sig("fk_lloyd_streamed", [_vp, _int, _i64, _int, _int, _int, _int, _vp, _vp,
                            ctypes.POINTER(ctypes.c_double), _i64, _vp, _sz, _vp])
 _sig("fk_streamed_workspace_size", [_i64, _int, _int, _int, _int, ctypes.POINTER(_sz)])
+_sig("fk_ivf_norms", [_vp, _i64, _int, _vp, _vp])
+_sig("fk_ivf_search_workspace_size", [_i64, _int, _int, _i64, _int, _int, ctypes.POINTER(_sz)])
+_sig("fk_ivf_search", [_vp, _i64, _int, _vp, _int, _vp, _vp, _vp, _vp, _i64, _int, _int, _vp,
+                       _vp, _vp, _vp, _sz, ctypes.POINTER(FkSearchTiming), _vp])
 
 EXPORTED = ["fk_status_string", "fk_version", "fk_workspace_size", "fk_normalize_rows",
             "fk_centroid_norms", "fk_assign", "fk_update", "fk_lloyd",
             "fk_get_device_error", "fk_selftest_timeout", "fk_assign_noalloc",
             "fk_update_partial", "fk_finalize_shards", "fk_split_points",
             "fk_launch_count", "fk_ivf_lists", "fk_lloyd_streamed",
-            "fk_streamed_workspace_size"]
+            "fk_streamed_workspace_size", "fk_ivf_norms", "fk_ivf_search_workspace_size",
+            "fk_ivf_search"]
 
 # Bytes of the static device array fk_assign_noalloc takes its scratch from.
 NOALLOC_SCRATCH_BYTES = 8 << 20
@@ -378,3 +388,103 @@ def fk_lloyd_streamed(X_host: torch.Tensor, C: torch.Tensor, niter: int, ws: tor
                                   chunk_rows, _dev(ws, "ws", torch.uint8), ws.numel(),
                                   _stream(stream)), "fk_lloyd_streamed")
     return [obj[i] for i in range(niter)]
+
+
+def fk_ivf_norms(V: torch.Tensor, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """fp64 squared norms of the fp32 rows of V (for fk_ivf_search: V = X_lists)."""
+    n, d = V.shape
+    if out is None:
+        out = torch.empty(n, dtype=torch.float64, device=V.device)
+    _check(_lib.fk_ivf_norms(_dev(V, "V", torch.float32), n, d,
+                             _dev(out, "out", torch.float64, (n,)), _stream(stream)),
+           "fk_ivf_norms")
+    return out
+
+
+def ivf_search_workspace(nq: int, d: int, nlist: int, N: int, nprobe: int, k: int,
+                         device="cuda") -> torch.Tensor:
+    out = _sz(0)
+    _check(_lib.fk_ivf_search_workspace_size(nq, d, nlist, N, nprobe, k, ctypes.byref(out)),
+           "fk_ivf_search_workspace_size")
+    return torch.empty(out.value, dtype=torch.uint8, device=device)
+
+
+def fk_ivf_search(Q: torch.Tensor, C: torch.Tensor, X_lists: torch.Tensor,
+                  X_norms: torch.Tensor, offsets: torch.Tensor, row_ids: torch.Tensor,
+                  nprobe: int, k: int, ws: torch.Tensor | None = None,
+                  distances: torch.Tensor | None = None, ids: torch.Tensor | None = None,
+                  probes: torch.Tensor | None = None, timing: dict | None = None,
+                  stream=None):
+    """IVF-Flat search: returns (distances fp32 [nq, k], ids int32 [nq, k]); `probes`
+    (int32 [nq, nprobe]) receives the probed cells when given.  A `timing` dict receives
+    the per-phase device times in ms (the call then synchronises its stream)."""
+    nq, d = Q.shape
+    nlist = C.shape[0]
+    N = X_lists.shape[0]
+    if ws is None:
+        ws = ivf_search_workspace(nq, d, nlist, N, nprobe, k, Q.device)
+    if distances is None:
+        distances = torch.empty((nq, k), dtype=torch.float32, device=Q.device)
+    if ids is None:
+        ids = torch.empty((nq, k), dtype=torch.int32, device=Q.device)
+    tm = FkSearchTiming() if timing is not None else None
+    _check(_lib.fk_ivf_search(_dev(Q, "Q", torch.float32), nq, d,
+                              _dev(C, "C", torch.float32, (nlist, d)), nlist,
+                              _dev(X_lists, "X_lists", torch.float32, (N, d)),
+                              _dev(X_norms, "X_norms", torch.float64, (N,)),
+                              _dev(offsets, "offsets", torch.int32, (nlist + 1,)),
+                              _dev(row_ids, "row_ids", torch.int32, (N,)), N, nprobe, k,
+                              _dev(distances, "distances", torch.float32, (nq, k)),
+                              _dev(ids, "ids", torch.int32, (nq, k)),
+                              _opt(probes, "probes", torch.int32, (nq, nprobe)),
+                              _dev(ws, "ws", torch.uint8), ws.numel(),
+                              ctypes.byref(tm) if tm is not None else None, _stream(stream)),
+           "fk_ivf_search")
+    if tm is not None:
+        timing.update({f: getattr(tm, f) for f, _ in FkSearchTiming._fields_})
+    return distances, ids
+
+
+class IvfFlatIndex:
+    """An IVF-Flat index: centroids, cell-contiguous points with their original ids, CSR
+    offsets and fp64 norms.  `build` and `search` only sequence libfk calls
+    (fk_normalize_rows, fk_lloyd, fk_ivf_lists, fk_ivf_norms, fk_ivf_search)."""
+
+    def __init__(self, C, X_lists, X_norms, offsets, row_ids, metric="l2"):
+        self.C, self.X_lists, self.X_norms = C, X_lists, X_norms
+        self.offsets, self.row_ids, self.metric = offsets, row_ids, metric
+
+    @classmethod
+    def build(cls, X: torch.Tensor, C0: torch.Tensor, niter: int, metric="l2", stream=None):
+        """Cluster X (fp32, N x d) from the initial centroids C0 with niter Lloyd iterations
+        and lay out the cells.  metric "cosine" L2-normalises X and C0 first."""
+        N, d = X.shape
+        K = C0.shape[0]
+        C = C0.clone()
+        if metric == "cosine":
+            Xn = torch.empty_like(X)
+            fk_normalize_rows(X, Xn, stream)
+            fk_normalize_rows(C0, C, stream)
+            X = Xn
+        labels = torch.empty(N, dtype=torch.int32, device=X.device)
+        ws = workspace(N, d, K, X.dtype, "l2", X.device)
+        fk_lloyd(X, C, niter, labels, ws, "l2", stream=stream)
+        offsets = torch.empty(K + 1, dtype=torch.int32, device=X.device)
+        row_ids = torch.empty(N, dtype=torch.int32, device=X.device)
+        X_lists = torch.empty_like(X)
+        fk_ivf_lists(X, labels, K, offsets, row_ids, ws, X_lists, stream)
+        del ws
+        X_norms = fk_ivf_norms(X_lists, stream=stream)
+        return cls(C, X_lists, X_norms, offsets, row_ids, metric)
+
+    def search(self, Q: torch.Tensor, k: int, nprobe: int, ws=None, distances=None,
+               ids=None, probes=None, timing=None, stream=None):
+        """(distances, ids) of the k nearest indexed points of every query, probing nprobe
+        cells; a cosine index L2-normalises the queries first."""
+        if self.metric == "cosine":
+            Qn = torch.empty_like(Q)
+            fk_normalize_rows(Q, Qn, stream)
+            Q = Qn
+        return fk_ivf_search(Q, self.C, self.X_lists, self.X_norms, self.offsets,
+                             self.row_ids, nprobe, k, ws=ws, distances=distances, ids=ids,
+                             probes=probes, timing=timing, stream=stream)

@@ -261,6 +261,61 @@ FK_API fk_status fk_ivf_lists(const void *X, fk_dtype dtype, int64_t N, int d, i
                               const int32_t *labels, int32_t *offsets, int32_t *row_ids,
                               void *X_lists, void *ws, size_t ws_bytes, fk_stream_t stream);
 
+/* Squared norms in fp64 for IVF-Flat search: norms[i] = sum_j V[i][j]^2 of the fp32 rows
+ * (each square exact in fp64, summed in fp64).  V: n x d fp32, device, 16-byte aligned,
+ * d % 4 == 0.  norms: n doubles, device.  Asynchronous on `stream`.  For fk_ivf_search
+ * this is computed once per index over X_lists, in list order. */
+FK_API fk_status fk_ivf_norms(const float *V, int64_t n, int d, double *norms,
+                              fk_stream_t stream);
+
+/* Workspace bytes of fk_ivf_search for these sizes. */
+FK_API fk_status fk_ivf_search_workspace_size(int64_t nq, int d, int nlist, int64_t N,
+                                              int nprobe, int k, size_t *bytes);
+
+/* IVF-Flat search (LEANN FlashLib guide: "什么是 FlashLib 后端" -- k nearest neighbours of
+ * a batch of queries; "工作原理" -- cells are the coarse k-means clusters, cell-contiguous
+ * with row ids and CSR offsets; "nlist 与 nprobe 的推导规则" -- nprobe cells probed per
+ * query; "距离度量只有 squared L2" -- squared L2, with cosine / inner product served by
+ * L2-normalising both sides first, which the caller does with fk_normalize_rows).
+ *
+ * For each query q (row of Q):
+ *   probes[q][0..nprobe)  the nprobe cells whose centroids are nearest to q, ascending by
+ *                         (distance, cell);
+ *   ids[q][0..k)          the k points of those cells nearest to q, ascending by
+ *                         (distance, original index), as original indices (row_ids);
+ *   distances[q][0..k)    their squared L2 distances (fp32 rounding of an fp64 value,
+ *                         clamped at 0); slots beyond the number of candidates hold id -1
+ *                         and distance +inf.
+ * Distances are evaluated in fp64 as ||q||^2 + ||x||^2 - 2 q.x; the selections agree with
+ * an exact fp64 evaluation except between candidates whose fp64 distances differ by the
+ * rounding of that expression (about 1e-16 of the squared norms).
+ *
+ * Inputs (device pointers, read only): Q nq x d fp32; C nlist x d fp32 centroids; X_lists
+ * N x d fp32, the points in cell order (fk_ivf_lists); X_norms N doubles, fk_ivf_norms of
+ * X_lists; offsets nlist + 1 int32 (offsets[0] = 0, offsets[nlist] = N, non-decreasing);
+ * row_ids N int32 (fk_ivf_lists).  Outputs (device): distances nq x k fp32, ids nq x k
+ * int32, probes nq x nprobe int32 or NULL (then kept in the workspace).
+ * Requirements: d % 4 == 0; Q, C, X_lists 16-byte aligned; 1 <= nprobe <= min(nlist,
+ * 1024); 1 <= k <= 32; nq * nprobe < 2^31; N < 2^31; finite inputs.  Violations return
+ * FK_ERR_INVALID_ARG (sizes, null pointers) or FK_ERR_UNSUPPORTED (alignment, d % 4).
+ * Asynchronous on `stream`; the workspace (fk_ivf_search_workspace_size, 256-byte aligned)
+ * must stay untouched until the call's work on the stream is done.  `timing` (host, may be
+ * NULL): when given, CUDA events on `stream` time each phase and the call synchronises the
+ * stream before it returns, to fill it in. */
+typedef struct fk_search_timing {
+    double ms_coarse; /* query and centroid norms, coarse distances, probe selection */
+    double ms_sort;   /* (query, probe) pairs sorted by cell, work items */
+    double ms_fine;   /* the fine distance kernel (per-pair k nearest) */
+    double ms_merge;  /* the per-query selection of the k nearest */
+} fk_search_timing;
+
+FK_API fk_status fk_ivf_search(const float *Q, int64_t nq, int d, const float *C, int nlist,
+                               const float *X_lists, const double *X_norms,
+                               const int32_t *offsets, const int32_t *row_ids, int64_t N,
+                               int nprobe, int k, float *distances, int32_t *ids,
+                               int32_t *probes, void *ws, size_t ws_bytes,
+                               fk_search_timing *timing, fk_stream_t stream);
+
 /* Scratch held by fk_assign_noalloc: one static device array of this many bytes. */
 #define FK_NOALLOC_SCRATCH_BYTES (8u << 20)
 

@@ -12,7 +12,7 @@ guide's "性能对比" section, and the d=128, K=32768 shape of the Flash-KMeans
 headline run scaled to one GPU.
 """
 from .mixture import (CONFIGS, IVF, LARGE, MID, TINY, ZIPF, MixtureSpec, gaussian_mixture,
-                      init_indices, make_config)
+                      init_indices, make_config, mixture_queries)
 
 __all__ = ["CONFIGS", "TINY", "IVF", "MID", "ZIPF", "LARGE", "MixtureSpec", "make_config",
-           "gaussian_mixture", "init_indices"]
+           "gaussian_mixture", "init_indices", "mixture_queries"]

@@ -24,6 +24,7 @@ import torch
 
 # Stream ids for the independent generators derived from one seed.
 _S_CENTERS, _S_COMP, _S_NOISE, _S_INIT = 11, 23, 37, 41
+_S_QCOMP, _S_QNOISE = 53, 67  # query draws (offset by 1000 * query stream)
 
 
 @dataclass(frozen=True)
@@ -76,15 +77,25 @@ def gaussian_mixture(n: int, d: int, n_comp: int, *, centers: str = "normal",
     """Return (X [n, d] fp32 or bf16, comp [n] int32 component ids, centers [n_comp, d]
     fp32), all on `device`."""
     device = torch.device(device)
+    cen = _centers(d, n_comp, centers, seed, device)
+
+    X, comp = _draw_points(n, d, cen, sigma, weights, zipf_s, dtype,
+                           _gen(device, seed, _S_COMP), _gen(device, seed, _S_NOISE),
+                           device, chunk_rows)
+    return X, comp, cen
+
+
+def _centers(d: int, n_comp: int, centers: str, seed: int, device) -> torch.Tensor:
     gc = _gen(device, seed, _S_CENTERS)
     if centers == "uniform":
-        cen = torch.rand(n_comp, d, generator=gc, device=device) * 2.0 - 1.0
-    elif centers == "normal":
-        cen = torch.randn(n_comp, d, generator=gc, device=device)
-    else:
-        raise ValueError(centers)
+        return torch.rand(n_comp, d, generator=gc, device=device) * 2.0 - 1.0
+    if centers == "normal":
+        return torch.randn(n_comp, d, generator=gc, device=device)
+    raise ValueError(centers)
 
-    gk = _gen(device, seed, _S_COMP)
+
+def _draw_points(n, d, cen, sigma, weights, zipf_s, dtype, gk, gn, device, chunk_rows):
+    n_comp = cen.shape[0]
     if weights == "equal":
         comp = torch.randint(0, n_comp, (n,), generator=gk, device=device,
                              dtype=torch.int64)
@@ -96,15 +107,26 @@ def gaussian_mixture(n: int, d: int, n_comp: int, *, centers: str = "normal",
         comp = torch.searchsorted(cdf, u, right=True).clamp_(max=n_comp - 1)
     else:
         raise ValueError(weights)
-
-    gn = _gen(device, seed, _S_NOISE)
     X = torch.empty(n, d, dtype=_torch_dtype(dtype), device=device)
     for r0 in range(0, n, chunk_rows):
         r1 = min(n, r0 + chunk_rows)
         noise = torch.randn(r1 - r0, d, generator=gn, device=device)
         X[r0:r1] = (cen[comp[r0:r1]] + sigma * noise).to(X.dtype)
         del noise
-    return X, comp.to(torch.int32), cen
+    return X, comp.to(torch.int32)
+
+
+def mixture_queries(nq: int, d: int, n_comp: int, *, centers: str = "normal",
+                    sigma: float = 0.1, weights: str = "equal", zipf_s: float = 1.2,
+                    seed: int = 0, stream: int = 0, device="cpu") -> torch.Tensor:
+    """nq fp32 queries from the same mixture as gaussian_mixture(..., seed=seed) (same
+    centers, fresh component and noise draws); `stream` selects independent query sets."""
+    device = torch.device(device)
+    cen = _centers(d, n_comp, centers, seed, device)
+    Q, _ = _draw_points(nq, d, cen, sigma, weights, zipf_s, "f32",
+                        _gen(device, seed, _S_QCOMP + 1000 * stream),
+                        _gen(device, seed, _S_QNOISE + 1000 * stream), device, 1 << 22)
+    return Q
 
 
 def init_indices(n: int, k: int, seed: int = 0, device="cpu") -> torch.Tensor:

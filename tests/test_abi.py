@@ -123,3 +123,34 @@ def test_ivf_lists_host_checks(fk):
         fk.FK_ERR_INVALID_ARG
     assert lib.fk_ivf_lists(4096, 0, 100, 8, 4, 256, 256, 256, None, 256, 10, None) == \
         fk.FK_ERR_WORKSPACE
+
+
+def test_ivf_search_host_checks(fk):
+    lib = fk._lib
+    big = 1 << 30
+    ok = dict(Q=256, nq=10, d=8, C=256, nlist=4, Xl=256, Xn=256, off=256, rid=256, N=100,
+              nprobe=2, k=3, dist=256, ids=256, probes=None, ws=256, wsb=big)
+
+    def call(**kw):
+        a = dict(ok, **kw)
+        return lib.fk_ivf_search(a["Q"], a["nq"], a["d"], a["C"], a["nlist"], a["Xl"], a["Xn"],
+                                 a["off"], a["rid"], a["N"], a["nprobe"], a["k"], a["dist"],
+                                 a["ids"], a["probes"], a["ws"], a["wsb"], None, None)
+
+    for bad in (dict(nprobe=5), dict(nprobe=0), dict(k=0), dict(k=33), dict(nq=0),
+                dict(N=0), dict(Q=None), dict(Xn=None), dict(ids=None),
+                dict(nq=1 << 30, nprobe=4)):
+        assert call(**bad) == fk.FK_ERR_INVALID_ARG, bad
+    for bad in (dict(d=6), dict(Q=8), dict(Xl=264), dict(probes=258)):
+        assert call(**bad) == fk.FK_ERR_UNSUPPORTED, bad
+    assert call(wsb=10) == fk.FK_ERR_WORKSPACE
+    assert call(ws=None) == fk.FK_ERR_WORKSPACE
+    assert lib.fk_ivf_norms(None, 10, 8, 256, None) == fk.FK_ERR_INVALID_ARG
+    assert lib.fk_ivf_norms(256, 10, 6, 256, None) == fk.FK_ERR_UNSUPPORTED
+    with pytest.raises(fk.FkError) as e:
+        fk.ivf_search_workspace(10, 8, 4, 100, 5, 3, device="cpu")
+    assert e.value.status == fk.FK_ERR_INVALID_ARG
+    # the workspace grows with the queries' pairs and the coarse batch
+    s1 = fk.ivf_search_workspace(1000, 8, 64, 100, 8, 10, device="meta").numel()
+    s2 = fk.ivf_search_workspace(2000, 8, 64, 100, 8, 10, device="meta").numel()
+    assert s2 > s1 > 1000 * 8 * 10 * 12

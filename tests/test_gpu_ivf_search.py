@@ -1,0 +1,210 @@
+"""GPU parity of fk_ivf_search (IVF-Flat search) against the fp64 oracle.
+
+The index is laid out on the GPU by fk_ivf_lists / fk_ivf_norms from labels that come from
+the generator or the oracle, never from the GPU.  Parity rule: probes and ids equal the
+oracle's; where a row differs, the GPU's selection must be an equally valid one in fp64
+(its oracle distances equal the oracle's sorted list within NEAR of the squared norms: the
+rounding of the fp64 expansion the kernels evaluate), and such rows must stay rare.
+Distances are the fp32 rounding of an fp64 value: within 2^-23 relative (plus NEAR of the
+norms, absolute) of the oracle's.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from synth import gaussian_mixture, init_indices, mixture_queries
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda:0"
+NEAR = 1e-12  # relative to ||q||^2 + max ||x||^2
+
+
+def fk():
+    from exact_lloyd_means_b200 import fk as m
+    return m
+
+
+def _index(X, labels, nlist):
+    m = fk()
+    N, d = X.shape
+    Xg = X.to(DEV)
+    offsets = torch.empty(nlist + 1, dtype=torch.int32, device=DEV)
+    row_ids = torch.empty(N, dtype=torch.int32, device=DEV)
+    X_lists = torch.empty_like(Xg)
+    ws = m.workspace(N, d, nlist, Xg.dtype, "l2")
+    m.fk_ivf_lists(Xg, torch.as_tensor(labels).to(DEV), nlist, offsets, row_ids, ws,
+                   X_lists=X_lists)
+    assert m.fk_get_device_error(ws) == m.FK_OK
+    return X_lists, m.fk_ivf_norms(X_lists), offsets, row_ids
+
+
+def _search(Q, C, idx, nprobe, k):
+    m = fk()
+    X_lists, X_norms, offsets, row_ids = idx
+    nq = Q.shape[0]
+    probes = torch.full((nq, nprobe), -7, dtype=torch.int32, device=DEV)
+    dist, ids = m.fk_ivf_search(Q.to(DEV), C.to(DEV), X_lists, X_norms, offsets, row_ids,
+                                nprobe, k, probes=probes)
+    torch.cuda.synchronize()
+    return probes.cpu().numpy(), ids.cpu().numpy(), dist.cpu().numpy()
+
+
+def _sqd(A, B):
+    """fp64 difference-form squared distances of the rows of A to the rows of B."""
+    A = np.asarray(A, dtype=np.float64)
+    B = np.asarray(B, dtype=np.float64)
+    return ((A[:, None, :] - B[None, :, :]) ** 2).sum(axis=2)
+
+
+def check_search(Q, C, X, got, ref, max_bad_frac=0.01):
+    probes, ids, dist = got
+    rp, ri, rd = ref
+    Q64, X64, C64 = (np.asarray(a, dtype=np.float64) for a in (Q, X, C))
+    scale = (Q64 ** 2).sum(1) + max((X64 ** 2).sum(1).max(), (C64 ** 2).sum(1).max())
+    bad = 0
+    for r in np.nonzero((probes != rp).any(axis=1))[0]:
+        bad += 1
+        dc = _sqd(Q64[r:r + 1], C64)[0]
+        assert np.allclose(np.sort(dc[probes[r]]), np.sort(dc[rp[r]]), rtol=0,
+                           atol=NEAR * scale[r]), f"query {r}: probes {probes[r]} vs {rp[r]}"
+    for r in np.nonzero((ids != ri).any(axis=1))[0]:
+        bad += 1
+        real = ids[r] >= 0
+        assert (real == (ri[r] >= 0)).all(), f"query {r}: padding differs"
+        dg = _sqd(Q64[r:r + 1], X64[ids[r][real]])[0]
+        assert np.allclose(dg, rd[r][real], rtol=0, atol=NEAR * scale[r]), \
+            f"query {r}: ids {ids[r]} vs {ri[r]}"
+    assert bad <= max_bad_frac * len(Q64) + 0.5, f"{bad} rows differ"
+    fin = np.isfinite(rd)
+    assert np.array_equal(np.isfinite(dist), fin)
+    assert np.array_equal(ids[~fin], np.full((~fin).sum(), -1))
+    err = np.abs(dist[fin].astype(np.float64) - rd[fin])
+    tol = 2.0 ** -23 * np.abs(rd[fin]) + NEAR * np.broadcast_to(scale[:, None], rd.shape)[fin]
+    assert (err <= tol).all(), float((err - tol).max())
+    return bad
+
+
+CASES = [
+    # N, d, nlist, nq, nprobe, k, weights, labels
+    (20000, 64, 64, 100, 4, 10, "equal", "assign"),
+    (30011, 100, 97, 77, 7, 32, "equal", "assign"),     # ragged d, nq and tiles
+    (50000, 768, 256, 64, 16, 10, "equal", "assign"),   # the guide's d
+    (4000, 128, 50, 33, 50, 5, "equal", "assign"),      # nprobe = nlist: exact kNN
+    (2000, 16, 40, 40, 1, 1, "equal", "assign"),
+    (60000, 32, 100, 300, 8, 10, "zipf", "comp"),       # cells of thousands, many items/cell
+    (3000, 24, 300, 50, 3, 20, "equal", "comp"),        # tiny cells: padded lists
+]
+
+
+@pytest.mark.parametrize("N,d,nlist,nq,nprobe,k,weights,labels_from", CASES)
+def test_ivf_search_matches_oracle(N, d, nlist, nq, nprobe, k, weights, labels_from):
+    X, comp, _ = gaussian_mixture(N, d, nlist, centers="normal", sigma=0.4, weights=weights,
+                                  seed=N + d)
+    C = X[init_indices(N, nlist, N + d)].float().contiguous()
+    if labels_from == "assign":
+        labels, _, _ = oracle.assign(X, C)
+    else:
+        labels = comp.numpy().astype(np.int32)
+    Q = mixture_queries(nq, d, nlist, centers="normal", sigma=0.4, weights=weights,
+                        seed=N + d, stream=1)
+    got = _search(Q, C, _index(X, labels, nlist), nprobe, k)
+    ref = oracle.ivf_search(Q, C, X, labels, nprobe, k)
+    check_search(Q, C, X, got, ref)
+
+
+def test_ivf_search_empty_cells_and_few_candidates():
+    """Centroids with no points (probed and returning nothing) and fewer candidates than
+    k: padded slots are -1 / +inf, exactly as the oracle's."""
+    N, d, K = 500, 32, 20
+    X, comp, _ = gaussian_mixture(N, d, K, centers="normal", sigma=0.2, seed=7)
+    labels = comp.numpy().astype(np.int32)
+    extra = torch.randn(12, d, generator=torch.Generator().manual_seed(3))
+    C = torch.cat([X[init_indices(N, K, 7)].float(), extra]).contiguous()
+    nlist = C.shape[0]
+    Q = torch.cat([extra[:4] + 0.01, mixture_queries(40, d, K, sigma=0.2, seed=7, stream=1)])
+    for nprobe, k in ((1, 32), (3, 32), (nlist, 8)):
+        got = _search(Q, C, _index(X, labels, nlist), nprobe, k)
+        ref = oracle.ivf_search(Q, C, X, labels, nprobe, k)
+        assert (ref[1] == -1).any() or nprobe == nlist
+        check_search(Q, C, X, got, ref, max_bad_frac=0.0)
+
+
+def test_ivf_search_duplicates_and_self_queries():
+    """Exact duplicate points tie at every query: the lower original index comes first.
+    Queries that are data points find themselves at distance 0."""
+    N, d, K = 6000, 48, 30
+    X, comp, _ = gaussian_mixture(N, d, K, centers="normal", sigma=0.3, seed=9)
+    X[N // 2:N // 2 + 200] = X[100:300]   # 200 duplicated rows
+    C = X[init_indices(N, K, 9)].float().contiguous()
+    labels, _, _ = oracle.assign(X, C)
+    sel = np.r_[np.arange(100, 140), np.arange(4000, 4030)]
+    Q = X[sel].clone()
+    got = _search(Q, C, _index(X, labels, K), 2, 6)
+    ref = oracle.ivf_search(Q, C, X, labels, 2, 6)
+    check_search(Q, C, X, got, ref, max_bad_frac=0.0)
+    ids = got[1]
+    assert (ids[:, 0] == sel).all()
+    assert (ids[:40, 1] == sel[:40] + N // 2 - 100).all()   # the duplicate, second
+
+
+def test_ivf_search_built_index_exhaustive_is_exact_knn():
+    """IvfFlatIndex.build (GPU Lloyd, cosine) then search with every cell probed: the result
+    is the exact k nearest neighbours of the normalised corpus, whatever the partition."""
+    m = fk()
+    N, d, K = 40000, 96, 64
+    X, _, _ = gaussian_mixture(N, d, K, centers="normal", sigma=0.5, seed=11)
+    C0 = X[init_indices(N, K, 11)].float().contiguous()
+    index = m.IvfFlatIndex.build(X.to(DEV), C0.to(DEV), 5, metric="cosine")
+    Q = mixture_queries(64, d, K, sigma=0.5, seed=11, stream=2)
+    dist, ids = index.search(Q.to(DEV), 10, K)
+    torch.cuda.synchronize()
+    Xn = oracle.normalize_rows(X)
+    Qn = oracle.normalize_rows(Q)
+    # one cell holding every point: the oracle's search is then the brute-force kNN
+    _, ri, rd = oracle.ivf_search(Qn, Xn[:1], Xn, np.zeros(N, dtype=np.int32), 1, 10)
+    ids = ids.cpu().numpy()
+    assert (ids == ri).mean() > 0.999
+    np.testing.assert_allclose(dist.cpu().numpy(), rd, rtol=1e-6, atol=1e-6)
+
+
+def test_ivf_search_deterministic_and_batched_coarse():
+    """Two calls give the same bits; a query set larger than one coarse batch (nlist large
+    enough that the coarse matrix is cut) gives the same answers as per-batch calls."""
+    m = fk()
+    N, d, K = 70000, 16, 20000
+    X, comp, _ = gaussian_mixture(N, d, 4000, centers="normal", sigma=0.3, seed=13)
+    C = X[init_indices(N, K, 13)].float().contiguous()
+    labels = torch.randint(0, K, (N,), generator=torch.Generator().manual_seed(5)).numpy()
+    labels = labels.astype(np.int32)
+    idx = _index(X, labels, K)
+    nq = 4000   # coarse batch: 512 MiB / (20000 * 8 B) = 3328 rows -> two batches
+    Q = mixture_queries(nq, d, 4000, sigma=0.3, seed=13, stream=3)
+    a = _search(Q, C, idx, 5, 7)
+    b = _search(Q, C, idx, 5, 7)
+    for x, y in zip(a, b):
+        assert np.array_equal(x, y)
+    c = [_search(Q[i:i + 1000], C, idx, 5, 7) for i in range(0, nq, 1000)]
+    for t in range(3):
+        assert np.array_equal(a[t], np.concatenate([z[t] for z in c]))
+    sub = np.arange(0, nq, 97)
+    ref = oracle.ivf_search(Q[sub], C, X, labels, 5, 7)
+    check_search(Q[sub], C, X, tuple(x[sub] for x in a), ref)
+
+
+def test_ivf_search_argument_errors():
+    m = fk()
+    N, d, K = 1000, 16, 10
+    X, comp, _ = gaussian_mixture(N, d, K, seed=17)
+    C = X[:K].contiguous().to(DEV)
+    idx = _index(X, comp.numpy().astype(np.int32), K)
+    Q = X[:5].to(DEV)
+    for nprobe, k in ((K + 1, 3), (0, 3), (2, 0), (2, 33)):
+        with pytest.raises(m.FkError) as e:
+            m.fk_ivf_search(Q, C, *idx, nprobe, k)
+        assert e.value.status == m.FK_ERR_INVALID_ARG
+    ws = m.ivf_search_workspace(5, d, K, N, 2, 3)
+    with pytest.raises(m.FkError) as e:
+        m.fk_ivf_search(Q, C, *idx, 2, 3, ws=ws[:1024])
+    assert e.value.status == m.FK_ERR_WORKSPACE
