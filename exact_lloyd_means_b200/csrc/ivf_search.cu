@@ -34,19 +34,28 @@ namespace {
 constexpr unsigned kFull = 0xffffffffu;
 
 // ---------------------------------------------------------------- fp64 tile geometry
-// A tile is 32 queries x 128 vectors; 4 warps, warp w owns queries 8w..8w+7 and lane l
-// owns vectors l, l+32, l+64, l+96.  Dimensions are staged in chunks of 32, converted to
-// fp64 once at staging.  The vector rows in shared memory are 34 doubles long: a
-// quarter-warp's 16-byte reads at one dimension then fall on distinct banks.
+// A tile is 32 queries x 128 vectors, 4 warps.  The dot products run on the fp64 tensor
+// instruction mma.m8n8k4 (8 queries x 8 vectors x 4 dimensions per instruction): warp w
+// covers queries 16 (w >> 1) .. +15 (two 8-row blocks) and vectors 64 (w & 1) .. +63 (eight
+// 8-column blocks), so per 4 dimensions it loads 2 + 8 operand fragments for 16 products.
+// Blocks of 8 queries or vectors beyond the item's count are skipped.  Dimensions are
+// staged in chunks of 32, converted to fp64 once at staging, in rows of 36 doubles: the
+// fragment reads (8 rows x 4 consecutive dimensions per instruction) then hit 32 distinct
+// banks.  After the last chunk the accumulators go through shared memory (rows of 136
+// doubles, over the vector buffer) so that each warp reads whole rows of 128 products.
 constexpr int kTQ = 32;
 constexpr int kTV = 128;
 constexpr int kTD = 32;
-constexpr int kVS = kTD + 2;
+constexpr int kS = kTD + 4;
+constexpr int kDS = kTV + 8;
 constexpr int kTThreads = 128;
 
 struct TileSmem {
-    double q[kTQ * kTD];  // [query][dim]
-    double v[kTV * kVS];  // [vector][dim], padded rows
+    double q[kTQ * kS];  // [query][dim]
+    union {
+        double v[kTV * kS];    // [vector][dim]
+        double dot[kTQ * kDS];  // [query][vector]: the tile's dot products
+    };
 };
 
 // Registers of one staged chunk: 8 float4 of vectors and 2 of queries per thread.
@@ -88,34 +97,42 @@ __device__ __forceinline__ void stage_store(const Stage &s, TileSmem &sm, int ti
 #pragma unroll
     for (int r = 0; r < 8; ++r) {
         const int f = tid + kTThreads * r;
-        put4(sm.v + (f >> 3) * kVS + (f & 7) * 4, s.v[r]);
+        put4(sm.v + (f >> 3) * kS + (f & 7) * 4, s.v[r]);
     }
 #pragma unroll
     for (int r = 0; r < 2; ++r) {
         const int f = tid + kTThreads * r;
-        put4(sm.q + (f >> 3) * kTD + (f & 7) * 4, s.q[r]);
+        put4(sm.q + (f >> 3) * kS + (f & 7) * 4, s.q[r]);
     }
 }
 
-// acc[a][i] += sum over the chunk's dimensions of q[8w + a][j] * v[l + 32 i][j], in
-// dimension order.
-__device__ __forceinline__ void tile_fma(const TileSmem &sm, int warp, int lane,
-                                         double (&acc)[8][4]) {
-    const double *qb = sm.q + warp * 8 * kTD;
-    const double *vb = sm.v + lane * kVS;
-#pragma unroll 2
-    for (int j = 0; j < kTD; j += 2) {
-        double2 vv[4];
+// D (8 x 8) += A (8 x 4) B (4 x 8) in fp64.  Fragments: this lane holds A[g][t] and B[t][g]
+// and accumulates D[g][2t], D[g][2t + 1], with g = lane / 4 and t = lane % 4.
+__device__ __forceinline__ void dmma(double &d0, double &d1, double a, double b) {
+    asm("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0,%1}, {%2}, {%3}, {%0,%1};"
+        : "+d"(d0), "+d"(d1)
+        : "d"(a), "d"(b));
+}
+
+// acc[a][n] += the chunk's dot products of query block (2 wq + a) with vector block
+// (8 wp + n), for the mact query blocks and nact vector blocks this warp has.
+__device__ __forceinline__ void tile_mma(const TileSmem &sm, int wq, int wp, int lane, int mact,
+                                         int nact, double (&acc)[2][8][2]) {
+    const int g = lane >> 2, t = lane & 3;
+    const double *qa = sm.q + (wq * 16 + g) * kS + t;
+    const double *vb = sm.v + (wp * 64 + g) * kS + t;
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
-            vv[i] = *reinterpret_cast<const double2 *>(vb + i * 32 * kVS + j);
+    for (int ks = 0; ks < kTD / 4; ++ks) {
+        const double a0 = qa[ks * 4];
+        const double a1 = qa[8 * kS + ks * 4];
+        double b[8];
 #pragma unroll
-        for (int a = 0; a < 8; ++a) {
-            const double2 qq = *reinterpret_cast<const double2 *>(qb + a * kTD + j);
+        for (int n = 0; n < 8; ++n) b[n] = vb[n * 8 * kS + ks * 4];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                acc[a][i] = fma(qq.x, vv[i].x, acc[a][i]);
-                acc[a][i] = fma(qq.y, vv[i].y, acc[a][i]);
+        for (int n = 0; n < 8; ++n) {
+            if (n < nact) {
+                dmma(acc[0][n][0], acc[0][n][1], a0, b[n]);
+                if (mact > 1) dmma(acc[1][n][0], acc[1][n][1], a1, b[n]);
             }
         }
     }
@@ -213,20 +230,37 @@ __global__ void __launch_bounds__(kTThreads, 3) ivf_tile_kernel(TileArgs a) {
         for (int64_t v0 = vbeg; v0 < vend; v0 += kTV) {
             const int nv_t = static_cast<int>(min(static_cast<int64_t>(kTV), vend - v0));
             const float *Vt = a.V + v0 * d;
-            double acc[8][4];
+            // this warp's blocks of 8 queries (of 2) and of 8 vectors (of 8) that hold data
+            const int wq = warp >> 1, wp = warp & 1;
+            const int mact = max(0, min(2, (nq_i + 7) / 8 - 2 * wq));
+            const int nact = max(0, min(8, (nv_t + 7) / 8 - 8 * wp));
+            double acc[2][8][2];
 #pragma unroll
-            for (int q8 = 0; q8 < 8; ++q8)
+            for (int a2 = 0; a2 < 2; ++a2)
 #pragma unroll
-                for (int i = 0; i < 4; ++i) acc[q8][i] = 0.0;
+                for (int n = 0; n < 8; ++n) acc[a2][n][0] = acc[a2][n][1] = 0.0;
             Stage st;
             stage_load(st, Vt, nv_t, qrow0, qrow1, d, 0, tid);
             for (int j0 = 0; j0 < d; j0 += kTD) {
-                __syncthreads();  // the previous chunk's readers are done
+                __syncthreads();  // the previous chunk's (or tile's) readers are done
                 stage_store(st, sm, tid);
                 __syncthreads();
                 if (j0 + kTD < d) stage_load(st, Vt, nv_t, qrow0, qrow1, d, j0 + kTD, tid);
-                tile_fma(sm, warp, lane, acc);
+                if (mact > 0) tile_mma(sm, wq, wp, lane, mact, nact, acc);
             }
+            __syncthreads();  // the dot-product rows overwrite the vector buffer
+            {
+                const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+                for (int a2 = 0; a2 < 2; ++a2)
+#pragma unroll
+                    for (int n = 0; n < 8; ++n)
+                        if (a2 < mact && n < nact)
+                            *reinterpret_cast<double2 *>(
+                                sm.dot + (wq * 16 + a2 * 8 + g) * kDS + wp * 64 + n * 8 + 2 * t) =
+                                make_double2(acc[a2][n][0], acc[a2][n][1]);
+            }
+            __syncthreads();
 
             double vn_i[4];
             uint32_t id_i[4];
@@ -248,13 +282,15 @@ __global__ void __launch_bounds__(kTThreads, 3) ivf_tile_kernel(TileArgs a) {
                     double *Drow = a.D + (q_first + qi) * static_cast<int64_t>(a.nv);
 #pragma unroll
                     for (int i = 0; i < 4; ++i)
-                        if (ok_i[i]) Drow[v0 + lane + 32 * i] = fma(-2.0, acc[q8][i], qn + vn_i[i]);
+                        if (ok_i[i])
+                            Drow[v0 + lane + 32 * i] =
+                                fma(-2.0, sm.dot[qi * kDS + lane + 32 * i], qn + vn_i[i]);
                 } else {
                     double td = __shfl_sync(kFull, ld[q8], a.k - 1);
                     uint32_t ti = __shfl_sync(kFull, li[q8], a.k - 1);
 #pragma unroll
                     for (int i = 0; i < 4; ++i) {
-                        const double cd = fma(-2.0, acc[q8][i], qn + vn_i[i]);
+                        const double cd = fma(-2.0, sm.dot[qi * kDS + lane + 32 * i], qn + vn_i[i]);
                         const uint32_t ci = id_i[i];
                         bool pend = ok_i[i] && before(cd, ci, td, ti);
                         unsigned m = __ballot_sync(kFull, pend);
