@@ -38,72 +38,70 @@ constexpr unsigned kFull = 0xffffffffu;
 // instruction mma.m8n8k4 (8 queries x 8 vectors x 4 dimensions per instruction): warp w
 // covers queries 16 (w >> 1) .. +15 (two 8-row blocks) and vectors 64 (w & 1) .. +63 (eight
 // 8-column blocks), so per 4 dimensions it loads 2 + 8 operand fragments for 16 products.
-// Blocks of 8 queries or vectors beyond the item's count are skipped.  Dimensions are
-// staged in chunks of 32, converted to fp64 once at staging, in rows of 36 doubles: the
-// fragment reads (8 rows x 4 consecutive dimensions per instruction) then hit 32 distinct
-// banks.  After the last chunk the accumulators go through shared memory (rows of 136
-// doubles, over the vector buffer) so that each warp reads whole rows of 128 products.
+// Blocks of 8 queries or vectors beyond the item's count are skipped.
+// Dimensions are staged in chunks of 32 fp32 values per row, copied global -> shared with
+// cp.async into two alternating stages (the next chunk lands while this one is used), in
+// rows of 36 floats: a fragment read (8 rows x 4 consecutive dimensions) then hits 32
+// distinct banks.  Each fragment value is widened to fp64 (exactly) as it is read.  After
+// the last chunk the accumulators go through shared memory (rows of 136 doubles, over the
+// stages) so that each warp reads whole rows of 128 products.
 constexpr int kTQ = 32;
 constexpr int kTV = 128;
 constexpr int kTD = 32;
 constexpr int kS = kTD + 4;
 constexpr int kDS = kTV + 8;
 constexpr int kTThreads = 128;
+constexpr int kStages = 2;
 
-struct TileSmem {
-    double q[kTQ * kS];  // [query][dim]
-    union {
-        double v[kTV * kS];    // [vector][dim]
-        double dot[kTQ * kDS];  // [query][vector]: the tile's dot products
-    };
+struct StageBuf {
+    float q[kTQ * kS];  // [query][dim]
+    float v[kTV * kS];  // [vector][dim]
 };
 
-// Registers of one staged chunk: 8 float4 of vectors and 2 of queries per thread.
-struct Stage {
-    float4 v[8];
-    float4 q[2];
+struct TileSmem {
+    union {
+        StageBuf st[kStages];
+        double dot[kTQ * kDS];  // [query][vector]: the tile's dot products
+    };
 };
 
 __device__ __forceinline__ bool before(double da, uint32_t ia, double db, uint32_t ib) {
     return da < db || (da == db && ia < ib);
 }
 
-// Element f of a chunk (f = tid + 128 r): row f / 8, float4 column f % 8.  A row's 128-byte
-// piece is read by 8 consecutive lanes.
-__device__ __forceinline__ void stage_load(Stage &s, const float *V, int nv, const float *qrow0,
-                                           const float *qrow1, int d, int j0, int tid) {
+// 16-byte global -> shared copy; src_bytes = 0 fills zeros without reading.
+__device__ __forceinline__ void cp_async16(void *smem, const void *gmem, int src_bytes) {
+    const uint32_t sa = static_cast<uint32_t>(__cvta_generic_to_shared(smem));
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(sa), "l"(gmem),
+                 "r"(src_bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// Copy chunk j0 .. j0 + 31 of the tile's vectors (rows 0 .. nv - 1 of V) and queries into
+// a stage: element f = tid + 128 r is row f / 8, 16-byte column f % 8, so a row's 128-byte
+// piece is read by 8 consecutive lanes.  Rows past the data and columns past d are zeros.
+__device__ __forceinline__ void stage_issue(StageBuf &sb, const float *V, int nv,
+                                            const float *qrow0, const float *qrow1, int d,
+                                            int j0, int tid) {
 #pragma unroll
     for (int r = 0; r < 8; ++r) {
         const int f = tid + kTThreads * r;
         const int row = f >> 3;
         const int j = j0 + (f & 7) * 4;
-        s.v[r] = (row < nv && j < d)
-                     ? __ldg(reinterpret_cast<const float4 *>(V + static_cast<int64_t>(row) * d + j))
-                     : make_float4(0.f, 0.f, 0.f, 0.f);
+        const bool ok = row < nv && j < d;
+        cp_async16(sb.v + row * kS + (f & 7) * 4, ok ? V + static_cast<int64_t>(row) * d + j : V,
+                   ok ? 16 : 0);
     }
     const int j = j0 + (tid & 7) * 4;
-    s.q[0] = (qrow0 && j < d) ? __ldg(reinterpret_cast<const float4 *>(qrow0 + j))
-                              : make_float4(0.f, 0.f, 0.f, 0.f);
-    s.q[1] = (qrow1 && j < d) ? __ldg(reinterpret_cast<const float4 *>(qrow1 + j))
-                              : make_float4(0.f, 0.f, 0.f, 0.f);
-}
-
-__device__ __forceinline__ void put4(double *p, float4 x) {
-    reinterpret_cast<double2 *>(p)[0] = make_double2(x.x, x.y);
-    reinterpret_cast<double2 *>(p)[1] = make_double2(x.z, x.w);
-}
-
-__device__ __forceinline__ void stage_store(const Stage &s, TileSmem &sm, int tid) {
-#pragma unroll
-    for (int r = 0; r < 8; ++r) {
-        const int f = tid + kTThreads * r;
-        put4(sm.v + (f >> 3) * kS + (f & 7) * 4, s.v[r]);
-    }
-#pragma unroll
-    for (int r = 0; r < 2; ++r) {
-        const int f = tid + kTThreads * r;
-        put4(sm.q + (f >> 3) * kS + (f & 7) * 4, s.q[r]);
-    }
+    const int qr0 = tid >> 3, qr1 = (tid + kTThreads) >> 3;
+    const bool ok0 = qrow0 && j < d, ok1 = qrow1 && j < d;
+    cp_async16(sb.q + qr0 * kS + (tid & 7) * 4, ok0 ? qrow0 + j : V, ok0 ? 16 : 0);
+    cp_async16(sb.q + qr1 * kS + (tid & 7) * 4, ok1 ? qrow1 + j : V, ok1 ? 16 : 0);
 }
 
 // D (8 x 8) += A (8 x 4) B (4 x 8) in fp64.  Fragments: this lane holds A[g][t] and B[t][g]
@@ -116,11 +114,11 @@ __device__ __forceinline__ void dmma(double &d0, double &d1, double a, double b)
 
 // acc[a][n] += the chunk's dot products of query block (2 wq + a) with vector block
 // (8 wp + n), for the mact query blocks and nact vector blocks this warp has.
-__device__ __forceinline__ void tile_mma(const TileSmem &sm, int wq, int wp, int lane, int mact,
+__device__ __forceinline__ void tile_mma(const StageBuf &sb, int wq, int wp, int lane, int mact,
                                          int nact, double (&acc)[2][8][2]) {
     const int g = lane >> 2, t = lane & 3;
-    const double *qa = sm.q + (wq * 16 + g) * kS + t;
-    const double *vb = sm.v + (wp * 64 + g) * kS + t;
+    const float *qa = sb.q + (wq * 16 + g) * kS + t;
+    const float *vb = sb.v + (wp * 64 + g) * kS + t;
 #pragma unroll
     for (int ks = 0; ks < kTD / 4; ++ks) {
         const double a0 = qa[ks * 4];
@@ -169,7 +167,7 @@ struct TileArgs {
 // Padding ids of a pair list are 0x80000000 | (t * k + rank), unique within a query, above
 // every point id and recognised as "no point" by the final selection.
 template <bool FINE>
-__global__ void __launch_bounds__(kTThreads, 3) ivf_tile_kernel(TileArgs a) {
+__global__ void __launch_bounds__(kTThreads, 4) ivf_tile_kernel(TileArgs a) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     TileSmem &sm = *reinterpret_cast<TileSmem *>(smem_raw);
     __shared__ int s_item;
@@ -239,17 +237,23 @@ __global__ void __launch_bounds__(kTThreads, 3) ivf_tile_kernel(TileArgs a) {
             for (int a2 = 0; a2 < 2; ++a2)
 #pragma unroll
                 for (int n = 0; n < 8; ++n) acc[a2][n][0] = acc[a2][n][1] = 0.0;
-            Stage st;
-            stage_load(st, Vt, nv_t, qrow0, qrow1, d, 0, tid);
-            for (int j0 = 0; j0 < d; j0 += kTD) {
-                __syncthreads();  // the previous chunk's (or tile's) readers are done
-                stage_store(st, sm, tid);
-                __syncthreads();
-                if (j0 + kTD < d) stage_load(st, Vt, nv_t, qrow0, qrow1, d, j0 + kTD, tid);
-                if (mact > 0) tile_mma(sm, wq, wp, lane, mact, nact, acc);
+            const int nch = (d + kTD - 1) / kTD;
+            __syncthreads();  // the previous tile's readers of the dot rows are done
+            stage_issue(sm.st[0], Vt, nv_t, qrow0, qrow1, d, 0, tid);
+            cp_async_commit();
+            for (int c = 0; c < nch; ++c) {
+                if (c + 1 < nch) {
+                    stage_issue(sm.st[(c + 1) & 1], Vt, nv_t, qrow0, qrow1, d, (c + 1) * kTD, tid);
+                    cp_async_commit();
+                    cp_async_wait<1>();
+                } else {
+                    cp_async_wait<0>();
+                }
+                __syncthreads();  // chunk c is in shared memory for every thread
+                if (mact > 0) tile_mma(sm.st[c & 1], wq, wp, lane, mact, nact, acc);
+                __syncthreads();  // stage (c & 1) is free for chunk c + 2
             }
-            __syncthreads();  // the dot-product rows overwrite the vector buffer
-            {
+            {  // the dot-product rows overwrite the stages (every reader passed the last barrier)
                 const int g = lane >> 2, t = lane & 3;
 #pragma unroll
                 for (int a2 = 0; a2 < 2; ++a2)
