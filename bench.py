@@ -47,6 +47,9 @@ def parse():
     p.add_argument("--niter", type=int, default=None)
     p.add_argument("--n", type=int, default=None,
                    help="override N (smaller cases for profiling captures)")
+    p.add_argument("--k", type=int, default=None,
+                   help="override K, the number of clusters (cells); with --n, a small case "
+                        "of the same points per cell for profiling captures")
     p.add_argument("--impl", default="fk", choices=["fk", "reference"])
     p.add_argument("--dp", action="store_true",
                    help="run the data-parallel loop (exact_lloyd_means_b200.dist) even on "
@@ -802,6 +805,8 @@ def main():
     spec = CONFIGS[args.workload]
     if args.n:
         spec = replace(spec, n=args.n, name=spec.name.replace(str(spec.n), str(args.n)))
+    if args.k:
+        spec = replace(spec, k=args.k, name=spec.name.replace(f"k{spec.k}", f"k{args.k}"))
     if args.impl == "reference":
         if args.search:
             search_reference_arm(args, spec, rank, world)
