@@ -390,6 +390,7 @@ def fk_arm(args, spec, rank, world, dist):
            "update_hbm": {"achieved_gbs": upd_bytes / (upd_ms / 1e3) / 1e9,
                           "peak_gbs": peaks["hbm_gbs"],
                           "frac": upd_bytes / (upd_ms / 1e3) / 1e9 / peaks["hbm_gbs"],
+                          "frac_of_8tbs_spec": upd_bytes / (upd_ms / 1e3) / 1e9 / 8000.0,
                           "avg_ms": upd_ms},
            "phase_ms_per_step": phases,
            "gpu_launches": launches, "final_objective": objs[-1],
@@ -701,8 +702,14 @@ def search_arm(args, spec, rank, world, dist):
                         "kernel": "ivf_tile_kernel<true> (fine pass, fp64 FMA)",
                         "flops_per_launch": fine_flops, "avg_ms": phases["ms_fine"],
                         "peak_basis": f"148 SMs x 64 fp64 FMA/clk x 2 x {mhz:.0f} MHz"},
-           "coarse": {"achieved_tflops": coarse_tf, "frac": coarse_tf / peak,
-                      "flops": coarse_flops, "avg_ms": phases["ms_coarse"]},
+           "coarse": {"path": "tensor-core screening + fp64 re-ranking"
+                              if phases.get("screened_coarse") else "fp64",
+                      "useful_tflops": coarse_tf, "flops": coarse_flops,
+                      "avg_ms": phases["ms_coarse"],
+                      "frac": coarse_tf / (load_peaks()["bf16"] if phases.get("screened_coarse")
+                                           else peak),
+                      "frac_of": "measured bf16 burst peak" if phases.get("screened_coarse")
+                                 else "fp64 peak"},
            "distance_evals_per_query": evals / nq,
            "phase_ms_per_step": phases, "gpu_launches": launches, "clocks": clocks}
 

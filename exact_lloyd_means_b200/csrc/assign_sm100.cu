@@ -95,27 +95,6 @@ __device__ __forceinline__ void init_aug_a(uint8_t *aaug, int r) {
 }
 
 // Minimum of 64 values with three-input mins: 21 + 7 + 3 + 1 instructions.
-// Width of the screening window for one row: twice a bound E on |v~ - v|, where
-// v = ||c||^2 - 2 x.c is exact and v~ is what the single-product pass accumulates from
-// bf16 x~ = RN(x) and c~ = RN(c) (each within a relative 2^-8 of its value; u = 2^-8):
-//   operand rounding   |sum x~c~ - sum xc| <= (2u + u^2) sum |x_j||c_j| <= (2u + u^2)|x||c|,
-//                      doubled by the factor -2;
-//   accumulation       each of the dp/16 + 1 MMA steps adds 16 exact products to the fp32
-//                      accumulator; assume up to 17 units of 2^-23 of the largest partial
-//                      value, which is at most ||c||^2 + 2|x||c| (with margin);
-//   norm               ||c||^2 rounded once to fp32 (2^-24 relative).
-// If k* is the true argmin, v~(k*) <= v(k*) + E <= v(k) + E <= v~(k) + 2E for every k, so
-// k* lies within 2E of the screened minimum.  ||c|| is bounded by cmax = max_k ||c_k||.
-// The result carries a 1% margin for the rounding of this expression itself.
-__device__ __forceinline__ float screen_window(float xnorm2, float cmax2, int dp) {
-    const float xn = sqrtf(xnorm2), cm = sqrtf(cmax2);
-    const float u = 0.00390625f;
-    const float prod = 2.f * (2.f * u + u * u) * xn * cm;
-    const float accum = static_cast<float>(dp / 16 + 1) * 17.f * 1.1920929e-7f *
-                        (cmax2 + 2.f * xn * cm) * 1.01f;
-    const float norm = 5.9604645e-8f * cmax2;
-    return 2.f * (prod + accum + norm) * 1.01f;
-}
 
 __device__ __forceinline__ float min64(const float (&v)[64]) {
     float t[22];
@@ -568,7 +547,8 @@ __global__ void __launch_bounds__(PairCfg<NP, RES, SCR ? 1 : 4>::kThreads, 1)
                        const float *__restrict__ xnorm, float *__restrict__ mind,
                        uint32_t *__restrict__ err, uint64_t wait_ns,
                        const uint32_t *__restrict__ n_dev, int32_t *__restrict__ cand,
-                       const float *__restrict__ cmax2) {
+                       const float *__restrict__ cmax2, float *__restrict__ dump,
+                       int64_t ldd) {
     static_assert(!SCR || NP == 1, "screening runs the single-product form");
     using Cfg = PairCfg<NP, RES, SCR ? 1 : 4>;
     constexpr int S = Cfg::kStages;
@@ -876,6 +856,17 @@ __global__ void __launch_bounds__(PairCfg<NP, RES, SCR ? 1 : 4>::kThreads, 1)
                         __syncwarp();
                         if (lane == 0) ptx::mbar_arrive_cluster(tempty_c + acc * 8);
                     }
+                    if (dump != nullptr) {  // every screened value goes out: no candidates
+                        if (row < N) {
+                            float4 *dst = reinterpret_cast<float4 *>(
+                                dump + row * ldd + static_cast<int64_t>(nt) * kBN + c4 * 64);
+#pragma unroll
+                            for (int j = 0; j < 16; ++j)
+                                dst[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2],
+                                                     v[4 * j + 3]);
+                        }
+                        continue;
+                    }
                     const float m = min64(v);
                     // a chunk with columns inside the window; a chunk no better than a column
                     // already dropped cannot matter (if the final window reaches that column
@@ -902,6 +893,7 @@ __global__ void __launch_bounds__(PairCfg<NP, RES, SCR ? 1 : 4>::kThreads, 1)
                 }
             }
             if (!ok) break;
+            if (dump != nullptr) continue;
             // candidates: every kept column whose chunk minimum is inside the final window;
             // the row overflows if a column dropped for lack of room could still be inside
             const float T = fminf(best + W, kScreenMax);
@@ -1091,7 +1083,7 @@ cudaError_t launch_assign_pair_cfg(const AssignArgs &a, const CUtensorMap (&tA)[
     cudaError_t e = cudaLaunchKernelEx(
         &cfg, assign_pair_kernel<NP, RES, SCR>, tA[0], tA[1], tB[0], tB[1], tC, a.N,
         static_cast<int>(a.dp / kBK), static_cast<int>(a.Kp / kBN), nmb, a.labels, a.best,
-        a.xnorm, a.mind, a.err, a.wait_ns, a.n_dev, a.cand, a.cmax2);
+        a.xnorm, a.mind, a.err, a.wait_ns, a.n_dev, a.cand, a.cmax2, a.dump, a.ldd);
     note_launch();
     return e;
 }
@@ -1199,8 +1191,8 @@ cudaError_t launch_assign_np(const AssignArgs &a, cudaStream_t st) {
 
 cudaError_t launch_assign(const AssignArgs &a, cudaStream_t st) {
     if (a.N <= 0) return cudaSuccess;
-    if (a.cand != nullptr) {  // the screening pass exists only in the CTA-pair form
-        if (a.a_nplanes != 1 || !assign_can_screen(a.N, a.dp, a.Kp))
+    if (a.cand != nullptr || a.dump != nullptr) {  // only in the CTA-pair form
+        if (a.a_nplanes != 1 || (a.cand != nullptr && !assign_can_screen(a.N, a.dp, a.Kp)))
             return cudaErrorNotSupported;
         bool done = false;
         const cudaError_t e =
@@ -1212,6 +1204,10 @@ cudaError_t launch_assign(const AssignArgs &a, cudaStream_t st) {
 
 bool assign_can_screen(int64_t N, int dp, int Kp) {
     if (!pair_rows(N)) return false;
+    return assign_can_dump(dp, Kp);
+}
+
+bool assign_can_dump(int dp, int Kp) {
     return resident_x(1, dp, Kp) ? max_resident_pairs<1, true, true>() > 0
                                  : max_resident_pairs<1, false, true>() > 0;
 }

@@ -259,9 +259,9 @@ fk_status validate_search(int64_t nq, int d, int nlist, int64_t N, int nprobe, i
 
 fk_status run_ivf_search(const float *Q, int64_t nq, int d, const float *C, int nlist,
                          const float *X_lists, const double *X_norms, const int32_t *offsets,
-                         const int32_t *row_ids, int nprobe, int k, float *distances,
-                         int32_t *ids, int32_t *probes, void *ws, const SearchLayout &L,
-                         cudaStream_t st, const cudaEvent_t *ev) {
+                         const int32_t *row_ids, int nprobe, int k, bool screen,
+                         float *distances, int32_t *ids, int32_t *probes, void *ws,
+                         const SearchLayout &L, cudaStream_t st, const cudaEvent_t *ev) {
     // ev (optional): five events recorded between the phases
     auto mark = [&](int i) { return !ev || cudaEventRecord(ev[i], st) == cudaSuccess; };
     if (!mark(0)) return FK_ERR_CUDA;
@@ -271,11 +271,48 @@ fk_status run_ivf_search(const float *Q, int64_t nq, int d, const float *C, int 
     // coarse: distances to every centroid, then the nprobe nearest per query
     int32_t *pr = probes ? probes : ws_ptr<int32_t>(ws, L.probes);
     double *D = ws_ptr<double>(ws, L.D);
-    for (int64_t q0 = 0; q0 < nq; q0 += L.qbatch) {
-        const int nqb = static_cast<int>(nq - q0 < L.qbatch ? nq - q0 : L.qbatch);
-        FK_TRY_CUDA(launch_ivf_coarse(Q, qn, q0, nqb, d, C, cn, nlist, D, st));
-        FK_TRY_CUDA(launch_ivf_select(D, nullptr, nlist, nqb, nlist, nprobe, pr + q0 * nprobe,
-                                      nullptr, nprobe, st));
+    if (screen) {
+        // tensor-core screening of every (query, centroid), fp64 re-ranking of the window
+        AssignArgs a{};
+        uint16_t *qh = ws_ptr<uint16_t>(ws, L.qplanes);
+        uint16_t *cpl = ws_ptr<uint16_t>(ws, L.cplanes);
+        float *ccn = ws_ptr<float>(ws, L.ccn), *qxn = ws_ptr<float>(ws, L.qxn);
+        float *cmax2 = ws_ptr<float>(ws, L.cmax2), *Vs = ws_ptr<float>(ws, L.D);
+        FK_TRY_CUDA(launch_prep_centroids(C, nlist, d, L.Kp, L.dp, FK_F32, cpl, ccn,
+                                          ws_ptr<float>(ws, L.cused),
+                                          ws_ptr<uint16_t>(ws, L.caug), st));
+        FK_TRY_CUDA(launch_ivf_cmax(ccn, nlist, cmax2, st));
+        a.a_nplanes = 1;
+        a.lda = L.dp;
+        a.b_planes = cpl;
+        a.cn = ccn;
+        a.caug = ws_ptr<uint16_t>(ws, L.caug);
+        a.d = d;
+        a.dp = static_cast<int>(L.dp);
+        a.K = nlist;
+        a.Kp = static_cast<int>(L.Kp);
+        a.xnorm = qxn;
+        a.err = ws_ptr<uint32_t>(ws, L.err);
+        a.wait_ns = kDefaultWaitNs;
+        a.cmax2 = cmax2;
+        a.dump = Vs;
+        a.ldd = L.Kp;
+        for (int64_t q0 = 0; q0 < nq; q0 += L.qbatch) {
+            const int64_t nqb = nq - q0 < L.qbatch ? nq - q0 : L.qbatch;
+            FK_TRY_CUDA(launch_split_x(Q + q0 * d, nqb, d, L.dp, qh, qh + nqb * L.dp, qxn, st));
+            a.a_planes = qh;
+            a.N = nqb;
+            FK_TRY_CUDA(launch_assign(a, st));
+            FK_TRY_CUDA(launch_ivf_coarse_rerank(Vs, L.Kp, nqb, nlist, nprobe, Q, q0, C, d,
+                                                 static_cast<int>(L.dp), qxn, cmax2, pr, st));
+        }
+    } else {
+        for (int64_t q0 = 0; q0 < nq; q0 += L.qbatch) {
+            const int nqb = static_cast<int>(nq - q0 < L.qbatch ? nq - q0 : L.qbatch);
+            FK_TRY_CUDA(launch_ivf_coarse(Q, qn, q0, nqb, d, C, cn, nlist, D, st));
+            FK_TRY_CUDA(launch_ivf_select(D, nullptr, nlist, nqb, nlist, nprobe,
+                                          pr + q0 * nprobe, nullptr, nprobe, st));
+        }
     }
     if (!mark(1)) return FK_ERR_CUDA;
     // the (query, probe) pairs in cell order, cut into work items
@@ -322,7 +359,7 @@ const char *fk_status_string(fk_status s) {
     return "FK_UNKNOWN_STATUS";
 }
 
-int fk_version(void) { return 2; }
+int fk_version(void) { return 3; }
 
 int64_t fk_launch_count(void) { return g_launches; }
 
@@ -863,7 +900,7 @@ fk_status fk_ivf_search_workspace_size(int64_t nq, int d, int nlist, int64_t N, 
 
 fk_status fk_ivf_search(const float *Q, int64_t nq, int d, const float *C, int nlist,
                         const float *X_lists, const double *X_norms, const int32_t *offsets,
-                        const int32_t *row_ids, int64_t N, int nprobe, int k,
+                        const int32_t *row_ids, int64_t N, int nprobe, int k, int flags,
                         float *distances, int32_t *ids, int32_t *probes, void *ws,
                         size_t ws_bytes, fk_search_timing *timing, fk_stream_t stream) {
     fk_status s = validate_search(nq, d, nlist, N, nprobe, k);
@@ -890,8 +927,11 @@ fk_status fk_ivf_search(const float *Q, int64_t nq, int d, const float *C, int n
                 return FK_ERR_CUDA;
             }
     }
+    const bool screen = (flags & FK_SEARCH_FP64_COARSE) == 0 &&
+                        ivf_coarse_can_screen(nlist, static_cast<int>(L.dp),
+                                              static_cast<int>(L.Kp));
     const fk_status r = run_ivf_search(Q, nq, d, C, nlist, X_lists, X_norms, offsets, row_ids,
-                                       nprobe, k, distances, ids, probes, ws, L, st,
+                                       nprobe, k, screen, distances, ids, probes, ws, L, st,
                                        timing ? ev : nullptr);
     if (r == FK_OK && timing) {
         if (cudaStreamSynchronize(st) != cudaSuccess) {
@@ -904,6 +944,7 @@ fk_status fk_ivf_search(const float *Q, int64_t nq, int d, const float *C, int n
         timing->ms_sort = ms[1];
         timing->ms_fine = ms[2];
         timing->ms_merge = ms[3];
+        timing->screened_coarse = screen ? 1 : 0;
     }
     destroy();
     return r;

@@ -54,6 +54,31 @@ constexpr int64_t kScreenMinKD = int64_t(1) << 22;
 constexpr int kScreenMaxFallback = 4;
 constexpr int64_t kScreenProbeRows = 2 * 128 * 148;
 
+// Width of the screening window for one row: twice a bound E on |v~ - v|, where
+// v = ||c||^2 - 2 x.c is exact and v~ is what the single-product pass accumulates from
+// bf16 x~ = RN(x) and c~ = RN(c) (each within a relative 2^-8 of its value; u = 2^-8):
+//   operand rounding   |sum x~c~ - sum xc| <= (2u + u^2) sum |x_j||c_j| <= (2u + u^2)|x||c|,
+//                      doubled by the factor -2;
+//   accumulation       each of the dp/16 + 1 MMA steps adds 16 exact products to the fp32
+//                      accumulator; assume up to 17 units of 2^-23 of the largest partial
+//                      value, which is at most ||c||^2 + 2|x||c| (with margin);
+//   norm               ||c||^2 rounded once to fp32 (2^-24 relative).
+// If k* is the true argmin, v~(k*) <= v(k*) + E <= v(k) + E <= v~(k) + 2E for every k, so
+// k* lies within 2E of the screened minimum.  Likewise, if T~ is the m-th smallest
+// screened value, the m columns with the smallest screened values have v <= T~ + E, so
+// the m-th smallest exact value is at most T~ + E and every column among the m exact
+// smallest has v~ <= T~ + 2E.  ||c|| is bounded by cmax = max_k ||c_k||.
+// The result carries a 1% margin for the rounding of this expression itself.
+__device__ __forceinline__ float screen_window(float xnorm2, float cmax2, int dp) {
+    const float xn = sqrtf(xnorm2), cm = sqrtf(cmax2);
+    const float u = 0.00390625f;
+    const float prod = 2.f * (2.f * u + u * u) * xn * cm;
+    const float accum = static_cast<float>(dp / 16 + 1) * 17.f * 1.1920929e-7f *
+                        (cmax2 + 2.f * xn * cm) * 1.01f;
+    const float norm = 5.9604645e-8f * cmax2;
+    return 2.f * (prod + accum + norm) * 1.01f;
+}
+
 // Objective slots kept on the device by fk_lloyd before a copy to the host.
 constexpr int kObjRing = 4096;
 
@@ -206,6 +231,9 @@ struct AssignArgs {
     const uint32_t *n_dev; // optional: row count read on the device (N bounds the maps)
     int32_t *cand;         // screening pass: [N][kCandPerRow] candidates instead of labels
     const float *cmax2;    // screening pass: device max_k ||c_k||^2
+    float *dump;           // single-product pass that writes every screened value instead:
+                           // dump[row * ldd + col] = ||c||^2 - 2 x~.c~ for col < Kp
+    int64_t ldd;
 };
 
 cudaError_t launch_split_x(const float *X, int64_t N, int d, int64_t dp, uint16_t *hi,
@@ -222,6 +250,9 @@ cudaError_t launch_centroid_norms(const float *C, int K, int d, fk_dtype dtype, 
                                   cudaStream_t st);
 cudaError_t launch_assign(const AssignArgs &a, cudaStream_t st);
 bool assign_can_screen(int64_t N, int dp, int Kp);
+// The single-product pass with every screened value written out (AssignArgs::dump) can run
+// for this shape (any number of rows).
+bool assign_can_dump(int dp, int Kp);
 
 // Screened fp32 assignment (screen.cu): the single-product pass over plane 0 of `a`'s X
 // planes, exact re-ranking of the candidates, and the three-product pass over the rows
@@ -274,6 +305,15 @@ cudaError_t launch_ivf_select(const double *D, const uint32_t *I, int64_t ld, in
                               cudaStream_t st);
 cudaError_t launch_ivf_items(const int32_t *pair_off, int nlist, int2 *items, int *nitems,
                              int *ctr, cudaStream_t st);
+// The screened coarse pass: the assignment kernel's single-product pass writes every
+// screened value (AssignArgs::dump), then the candidates within the window above the
+// nprobe-th are re-ranked in fp64 (ivf_search.cu).
+bool ivf_coarse_can_screen(int nlist, int dp, int Kp);
+cudaError_t launch_ivf_cmax(const float *cn, int K, float *out, cudaStream_t st);
+cudaError_t launch_ivf_coarse_rerank(const float *Vs, int64_t ldv, int64_t rows, int L, int m,
+                                     const float *Q, int64_t q0, const float *C, int d, int dp,
+                                     const float *xnorm, const float *cmax2, int32_t *probes,
+                                     cudaStream_t st);
 cudaError_t launch_ivf_fine(const float *Q, const double *qn, int d, const float *X_lists,
                             const double *xn, const int32_t *offsets, const int32_t *row_ids,
                             const int32_t *pair_sorted, const int32_t *pair_off,
@@ -290,15 +330,17 @@ constexpr int64_t kSearchCoarseBytes = int64_t(512) << 20;
 struct SearchLayout {
     size_t err = 0, qn = 0, cn = 0, D = 0, probes = 0, keys0 = 0, keys1 = 0, vals0 = 0,
            vals1 = 0, hist = 0, dtot = 0, psorted = 0, poff = 0, items = 0, nitems = 0,
-           Ld = 0, Li = 0, total = 0;
-    int64_t P = 0, qbatch = 0, max_items = 0;
+           Ld = 0, Li = 0, qplanes = 0, qxn = 0, cplanes = 0, ccn = 0, cused = 0, caug = 0,
+           cmax2 = 0, total = 0;
+    int64_t P = 0, qbatch = 0, max_items = 0, dp = 0, Kp = 0;
     SortPlan sp;
 };
 
 inline SearchLayout search_layout(int64_t nq, int d, int nlist, int nprobe, int k) {
-    (void)d;
     SearchLayout L;
     L.P = nq * nprobe;
+    L.dp = round_up(d, kBK);
+    L.Kp = round_up(nlist, kBN);
     int64_t qb = kSearchCoarseBytes / (static_cast<int64_t>(nlist) * 8);
     qb = qb / 32 * 32;
     if (qb < 32) qb = 32;
@@ -314,7 +356,10 @@ inline SearchLayout search_layout(int64_t nq, int d, int nlist, int nprobe, int 
     L.err = take(256);
     L.qn = take(sizeof(double) * nq);
     L.cn = take(sizeof(double) * nlist);
-    L.D = take(sizeof(double) * L.qbatch * nlist);
+    // fp64 coarse distances, or the screened values (fp32, rows of Kp) of a batch
+    const int64_t dbytes = sizeof(double) * L.qbatch * nlist;
+    const int64_t sbytes = sizeof(float) * L.qbatch * L.Kp;
+    L.D = take(static_cast<size_t>(dbytes > sbytes ? dbytes : sbytes));
     L.probes = take(sizeof(int32_t) * L.P);
     L.keys0 = take(sizeof(int32_t) * L.P);
     L.keys1 = take(sizeof(int32_t) * L.P);
@@ -329,6 +374,14 @@ inline SearchLayout search_layout(int64_t nq, int d, int nlist, int nprobe, int 
     L.nitems = take(sizeof(int32_t) * 2);
     L.Ld = take(sizeof(double) * L.P * k);
     L.Li = take(sizeof(uint32_t) * L.P * k);
+    // screened coarse pass: bf16 planes of a query batch and of the centroids
+    L.qplanes = take(sizeof(uint16_t) * 2 * L.qbatch * L.dp);
+    L.qxn = take(sizeof(float) * L.qbatch);
+    L.cplanes = take(sizeof(uint16_t) * 2 * L.Kp * L.dp);
+    L.ccn = take(sizeof(float) * L.Kp);
+    L.cused = take(sizeof(float) * nlist * d);
+    L.caug = take(sizeof(uint16_t) * L.Kp * kAug);
+    L.cmax2 = take(256);
     L.total = o;
     return L;
 }

@@ -242,17 +242,17 @@ __global__ void __launch_bounds__(kTThreads, 4) ivf_tile_kernel(TileArgs a) {
             stage_issue(sm.st[0], Vt, nv_t, qrow0, qrow1, d, 0, tid);
             cp_async_commit();
             for (int c = 0; c < nch; ++c) {
+                cp_async_wait<0>();  // chunk c, the only copy in flight, has landed
+                // ... for every thread, and every warp is done with chunk c - 1, whose
+                // stage the next copy overwrites
+                __syncthreads();
                 if (c + 1 < nch) {
                     stage_issue(sm.st[(c + 1) & 1], Vt, nv_t, qrow0, qrow1, d, (c + 1) * kTD, tid);
                     cp_async_commit();
-                    cp_async_wait<1>();
-                } else {
-                    cp_async_wait<0>();
                 }
-                __syncthreads();  // chunk c is in shared memory for every thread
                 if (mact > 0) tile_mma(sm.st[c & 1], wq, wp, lane, mact, nact, acc);
-                __syncthreads();  // stage (c & 1) is free for chunk c + 2
             }
+            __syncthreads();  // every warp is done with the last stage
             {  // the dot-product rows overwrite the stages (every reader passed the last barrier)
                 const int g = lane >> 2, t = lane & 3;
 #pragma unroll
@@ -340,13 +340,23 @@ __global__ void __launch_bounds__(kTThreads, 4) ivf_tile_kernel(TileArgs a) {
 
 // ---------------------------------------------------------------- row selection
 // Per row (one block each): the m smallest entries by (distance, id), output in ascending
-// order.  The m-th smallest 96-bit key (order-preserving distance bits, then id) is found
-// digit by digit, 8 bits at a time, with a 256-bin histogram of the entries that still
-// match the decided digits; the search stops as soon as every entry of the chosen bin is
-// inside the first m.  The selected entries are then gathered and sorted (bitonic).
+// order.
+// Rows of up to kSelCache entries are staged in shared memory and go through a histogram:
+// the fp32 rounding of each distance is mapped linearly onto kSelBins bins between the
+// row's smallest and largest finite values (a non-decreasing map of the distance), the bin
+// holding the m-th entry is found with a prefix sum, and every entry in it or below is a
+// candidate: no entry above it can be among the m smallest.  The candidates (at least m,
+// usually a few more) are sorted by (distance, id) and the first m kept.
+// A row whose candidates would not fit (many equal distances), and every row too long to
+// stage, takes the radix path instead: the m-th smallest 96-bit key (order-preserving
+// distance bits, then id) is found digit by digit, 8 bits at a time, with a 256-bin
+// histogram of the entries that still match the decided digits, stopping as soon as every
+// entry of the chosen bin is inside the first m; exactly m entries are gathered.
 constexpr int kSelThreads = 256;
-constexpr int kSelMaxM = 1024;   // largest m
-constexpr int kSelCache = 8192;  // rows up to this length are staged in shared memory
+constexpr int kSelMaxM = 1024;     // largest m
+constexpr int kSelCache = 8192;    // rows up to this length are staged in shared memory
+constexpr int kSelBins = 2048;     // histogram bins of the staged path
+constexpr int kSelMaxCand = 2048;  // candidates the staged path sorts
 
 __device__ __forceinline__ uint64_t order_key(double x) {
     const uint64_t u = static_cast<uint64_t>(__double_as_longlong(x));
@@ -373,12 +383,14 @@ __global__ void __launch_bounds__(kSelThreads) select_rows_kernel(SelArgs a) {
     extern __shared__ __align__(16) unsigned char sel_raw[];
     uint64_t *ck = reinterpret_cast<uint64_t *>(sel_raw);
     uint32_t *ci = reinterpret_cast<uint32_t *>(sel_raw + sizeof(uint64_t) * (CACHE ? a.L : 0));
-    __shared__ uint32_t hist[256];
-    __shared__ uint64_t sel_k[kSelMaxM];
-    __shared__ uint32_t sel_i[kSelMaxM];
+    __shared__ uint32_t hist[kSelBins];  // the radix path uses the first 256
+    __shared__ uint64_t sel_k[kSelMaxCand];
+    __shared__ uint32_t sel_i[kSelMaxCand];
+    __shared__ float s_min[kSelThreads / 32], s_max[kSelThreads / 32];
+    __shared__ uint32_t s_wsum[kSelThreads / 32];
     __shared__ uint64_t s_phi;
     __shared__ uint32_t s_plo;
-    __shared__ int s_r, s_done, s_cnt;
+    __shared__ int s_r, s_done, s_cnt, s_bstar, s_ncand;
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int64_t row = blockIdx.x;
@@ -387,18 +399,112 @@ __global__ void __launch_bounds__(kSelThreads) select_rows_kernel(SelArgs a) {
     const int L = a.L, m = a.m;
     const int Lpad = (L + kSelThreads - 1) / kSelThreads * kSelThreads;
 
-    if (CACHE) {
-        for (int j = tid; j < L; j += kSelThreads) {
-            ck[j] = order_key(drow[j]);
-            ci[j] = irow ? irow[j] : static_cast<uint32_t>(j);
-        }
-    }
     if (tid == 0) {
         s_phi = 0;
         s_plo = 0;
         s_r = m - 1;
         s_done = 0;
         s_cnt = 0;
+        s_ncand = kSelMaxCand + 1;
+    }
+    int n_sel = -1;  // candidates gathered into sel_k / sel_i
+    if (CACHE) {
+        float lmin = INFINITY, lmax = -INFINITY;
+        // eight loads in flight per thread before any is used
+        constexpr int kU = 8;
+        for (int j0 = tid; j0 < L; j0 += kSelThreads * kU) {
+            double x[kU];
+            uint32_t id[kU];
+#pragma unroll
+            for (int u = 0; u < kU; ++u) {
+                const int j = j0 + u * kSelThreads;
+                x[u] = j < L ? drow[j] : 0.0;
+                id[u] = (j < L && irow) ? irow[j] : static_cast<uint32_t>(j);
+            }
+#pragma unroll
+            for (int u = 0; u < kU; ++u) {
+                const int j = j0 + u * kSelThreads;
+                if (j < L) {
+                    ck[j] = order_key(x[u]);
+                    ci[j] = id[u];
+                    const float fx = static_cast<float>(x[u]);
+                    if (fx < INFINITY) {
+                        lmin = fminf(lmin, fx);
+                        lmax = fmaxf(lmax, fx);
+                    }
+                }
+            }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            lmin = fminf(lmin, __shfl_xor_sync(kFull, lmin, o));
+            lmax = fmaxf(lmax, __shfl_xor_sync(kFull, lmax, o));
+        }
+        if (lane == 0) {
+            s_min[warp] = lmin;
+            s_max[warp] = lmax;
+        }
+        for (int t = tid; t < kSelBins; t += kSelThreads) hist[t] = 0;
+        __syncthreads();
+        float fmn = s_min[0], fmx = s_max[0];
+#pragma unroll
+        for (int w = 1; w < kSelThreads / 32; ++w) {
+            fmn = fminf(fmn, s_min[w]);
+            fmx = fmaxf(fmx, s_max[w]);
+        }
+        const float scale = fmx > fmn ? static_cast<float>(kSelBins - 1) / (fmx - fmn) : 0.f;
+        auto bin_of = [&](uint64_t k) -> int {
+            const float fx = static_cast<float>(key_value(k));
+            if (!(fx < fmx)) return kSelBins - 1;  // the largest finite value and +inf
+            const int bq = static_cast<int>((fx - fmn) * scale);
+            return bq < 0 ? 0 : (bq > kSelBins - 1 ? kSelBins - 1 : bq);
+        };
+        for (int j = tid; j < L; j += kSelThreads) atomicAdd(&hist[bin_of(ck[j])], 1u);
+        __syncthreads();
+        // prefix over the bins: thread t owns bins 8t .. 8t + 7
+        constexpr int kPer = kSelBins / kSelThreads;
+        uint32_t h[kPer], sum = 0;
+#pragma unroll
+        for (int t = 0; t < kPer; ++t) {
+            h[t] = hist[tid * kPer + t];
+            sum += h[t];
+        }
+        uint32_t incl = sum;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t y = __shfl_up_sync(kFull, incl, o);
+            if (lane >= o) incl += y;
+        }
+        if (lane == 31) s_wsum[warp] = incl;
+        __syncthreads();
+        uint32_t base = 0;
+        for (int w = 0; w < warp; ++w) base += s_wsum[w];
+        uint32_t c = base + incl - sum;  // entries in bins below 8 tid
+        const uint32_t need = static_cast<uint32_t>(m);
+        if (c < need && need <= c + sum) {
+#pragma unroll
+            for (int t = 0; t < kPer; ++t) {
+                if (c < need && need <= c + h[t]) {
+                    s_bstar = tid * kPer + t;
+                    s_ncand = static_cast<int>(c + h[t]);
+                }
+                c += h[t];
+            }
+        }
+        __syncthreads();
+        if (s_ncand <= kSelMaxCand) {
+            const int bstar = s_bstar;
+            for (int j = tid; j < L; j += kSelThreads) {
+                const uint64_t kh = ck[j];
+                if (bin_of(kh) <= bstar) {
+                    const int at = atomicAdd(&s_cnt, 1);
+                    sel_k[at] = kh;
+                    sel_i[at] = ci[j];
+                }
+            }
+            n_sel = s_ncand;
+        }
+        __syncthreads();
     }
     auto load = [&](int j, uint64_t &kh, uint32_t &kl) {
         if (CACHE) {
@@ -409,67 +515,67 @@ __global__ void __launch_bounds__(kSelThreads) select_rows_kernel(SelArgs a) {
             kl = irow ? irow[j] : static_cast<uint32_t>(j);
         }
     };
-    auto hi_mask = [](int b) -> uint64_t { return b >= 8 ? ~0ull : (b == 0 ? 0ull : ~0ull << (64 - 8 * b)); };
-    auto lo_mask = [](int b) -> uint32_t { return b <= 8 ? 0u : ~0u << (32 - 8 * (b - 8)); };
-
-    int b = 0;
-    while (b < 12) {
-        hist[tid] = 0;
-        __syncthreads();
-        const uint64_t phi = s_phi, mhi = hi_mask(b);
-        const uint32_t plo = s_plo, mlo = lo_mask(b);
-        for (int j = tid; j < Lpad; j += kSelThreads) {
-            uint64_t kh = 0;
-            uint32_t kl = 0;
-            const bool valid = j < L;
-            if (valid) load(j, kh, kl);
-            const bool match = valid && (kh & mhi) == phi && (kl & mlo) == plo;
-            int dig = b < 8 ? static_cast<int>((kh >> (56 - 8 * b)) & 255u)
-                            : static_cast<int>((kl >> (24 - 8 * (b - 8))) & 255u);
-            dig = match ? dig : 256;
-            const unsigned peers = __match_any_sync(kFull, dig);
-            if (match && lane == __ffs(peers) - 1) atomicAdd(&hist[dig], __popc(peers));
-        }
-        __syncthreads();
-        if (warp == 0) {
-            uint32_t h[8], sum = 0;
-#pragma unroll
-            for (int t = 0; t < 8; ++t) {
-                h[t] = hist[lane * 8 + t];
-                sum += h[t];
+    if (n_sel < 0) {
+        auto hi_mask = [](int b) -> uint64_t {
+            return b >= 8 ? ~0ull : (b == 0 ? 0ull : ~0ull << (64 - 8 * b));
+        };
+        auto lo_mask = [](int b) -> uint32_t { return b <= 8 ? 0u : ~0u << (32 - 8 * (b - 8)); };
+        int b = 0;
+        while (b < 12) {
+            hist[tid] = 0;
+            __syncthreads();
+            const uint64_t phi = s_phi, mhi = hi_mask(b);
+            const uint32_t plo = s_plo, mlo = lo_mask(b);
+            for (int j = tid; j < Lpad; j += kSelThreads) {
+                uint64_t kh = 0;
+                uint32_t kl = 0;
+                const bool valid = j < L;
+                if (valid) load(j, kh, kl);
+                const bool match = valid && (kh & mhi) == phi && (kl & mlo) == plo;
+                int dig = b < 8 ? static_cast<int>((kh >> (56 - 8 * b)) & 255u)
+                                : static_cast<int>((kl >> (24 - 8 * (b - 8))) & 255u);
+                dig = match ? dig : 256;
+                const unsigned peers = __match_any_sync(kFull, dig);
+                if (match && lane == __ffs(peers) - 1) atomicAdd(&hist[dig], __popc(peers));
             }
-            uint32_t incl = sum;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const uint32_t y = __shfl_up_sync(kFull, incl, o);
-                if (lane >= o) incl += y;
-            }
-            const uint32_t excl = incl - sum;
-            const uint32_t r = static_cast<uint32_t>(s_r);
-            if (excl <= r && r < incl) {
-                uint32_t c = excl;
+            __syncthreads();
+            if (warp == 0) {
+                uint32_t h[8], sum = 0;
 #pragma unroll
                 for (int t = 0; t < 8; ++t) {
-                    if (r >= c && r < c + h[t]) {
-                        const uint32_t bin = lane * 8 + t;
-                        if (b < 8)
-                            s_phi = phi | (static_cast<uint64_t>(bin) << (56 - 8 * b));
-                        else
-                            s_plo = plo | (bin << (24 - 8 * (b - 8)));
-                        s_r = static_cast<int>(r - c);
-                        s_done = (r - c + 1 == h[t]) ? 1 : 0;
+                    h[t] = hist[lane * 8 + t];
+                    sum += h[t];
+                }
+                uint32_t incl = sum;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const uint32_t y = __shfl_up_sync(kFull, incl, o);
+                    if (lane >= o) incl += y;
+                }
+                const uint32_t excl = incl - sum;
+                const uint32_t r = static_cast<uint32_t>(s_r);
+                if (excl <= r && r < incl) {
+                    uint32_t c = excl;
+#pragma unroll
+                    for (int t = 0; t < 8; ++t) {
+                        if (r >= c && r < c + h[t]) {
+                            const uint32_t bin = lane * 8 + t;
+                            if (b < 8)
+                                s_phi = phi | (static_cast<uint64_t>(bin) << (56 - 8 * b));
+                            else
+                                s_plo = plo | (bin << (24 - 8 * (b - 8)));
+                            s_r = static_cast<int>(r - c);
+                            s_done = (r - c + 1 == h[t]) ? 1 : 0;
+                        }
+                        c += h[t];
                     }
-                    c += h[t];
                 }
             }
+            __syncthreads();
+            ++b;
+            if (s_done) break;
         }
-        __syncthreads();
-        ++b;
-        if (s_done) break;
-    }
-
-    // every entry whose first b digits are at most the decided prefix is selected: exactly m
-    {
+        // every entry whose first b digits are at most the decided prefix: exactly m
         const uint64_t phi = s_phi, mhi = hi_mask(b);
         const uint32_t plo = s_plo, mlo = lo_mask(b);
         for (int j = tid; j < L; j += kSelThreads) {
@@ -480,17 +586,18 @@ __global__ void __launch_bounds__(kSelThreads) select_rows_kernel(SelArgs a) {
             const uint32_t tl = kl & mlo;
             if (th < phi || (th == phi && tl <= plo)) {
                 const int at = atomicAdd(&s_cnt, 1);
-                if (at < kSelMaxM) {
+                if (at < kSelMaxCand) {
                     sel_k[at] = kh;
                     sel_i[at] = kl;
                 }
             }
         }
+        n_sel = m;
     }
     int M = 1;
-    while (M < m) M <<= 1;
+    while (M < n_sel) M <<= 1;
     __syncthreads();
-    for (int t = m + tid; t < M; t += kSelThreads) {
+    for (int t = n_sel + tid; t < M; t += kSelThreads) {
         sel_k[t] = ~0ull;
         sel_i[t] = ~0u;
     }
@@ -521,6 +628,215 @@ __global__ void __launch_bounds__(kSelThreads) select_rows_kernel(SelArgs a) {
         if (a.out_dist)
             a.out_dist[row * a.ldo + t] =
                 pad ? INFINITY : static_cast<float>(fmax(key_value(sel_k[t]), 0.0));
+    }
+}
+
+// ---------------------------------------------------------------- screened coarse pass
+// The coarse distances as a dense product on the tensor cores: the single-product pass of
+// the assignment kernel (one bf16 product per term, norms folded in exactly) writes the
+// screened value v~ = ||c||^2 - 2 q~.c~ of every (query, centroid), each within E of the
+// exact ||c||^2 - 2 q.c (screen_window).  Per query, if T~ is the nprobe-th smallest
+// screened value, every centroid among the nprobe nearest has v~ <= T~ + 2E; those
+// candidates are re-ranked exactly (fp64, difference form) and the nprobe smallest by
+// (distance, cell) kept.  The same probes as the fp64 coarse pass, for a fraction of the
+// work; only the candidates (typically a few more than nprobe) see fp64 arithmetic.
+constexpr int kCoarseThreads = 256;
+constexpr int kCoarseMaxL = 8192;  // centroids a block stages
+
+struct CoarseArgs {
+    const float *V;        // [rows][ldv] screened values of the batch
+    int64_t ldv;
+    int L, m;              // centroids, probes
+    const float *Q;        // fp32 queries; row q0 + r is the block's
+    int64_t q0;
+    const float *C;        // fp32 centroids [L][d]
+    int d, dp;             // dimension, and the padded width the screening pass ran over
+    const float *xnorm;    // [nq] ||q||^2 (fp32) the window is derived from
+    const float *cmax2;    // max_k ||c_k||^2
+    int32_t *probes;       // [nq][m]
+};
+
+__device__ __forceinline__ uint32_t fkey(float x) {
+    const uint32_t u = __float_as_uint(x);
+    return (u >> 31) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float fkey_value(uint32_t k) {
+    return __uint_as_float((k >> 31) ? (k & 0x7fffffffu) : ~k);
+}
+
+__global__ void __launch_bounds__(kCoarseThreads) coarse_rerank_kernel(CoarseArgs a) {
+    extern __shared__ __align__(16) unsigned char co_raw[];
+    int P = 1;
+    while (P < a.L) P <<= 1;
+    double *cd = reinterpret_cast<double *>(co_raw);               // [P] candidate distances
+    uint32_t *cid = reinterpret_cast<uint32_t *>(cd + P);          // [P] candidate cells
+    uint32_t *key = cid + P;                                       // [L] screened-value keys
+    __shared__ uint32_t hist[kSelBins];
+    __shared__ float s_min[kCoarseThreads / 32], s_max[kCoarseThreads / 32];
+    __shared__ uint32_t s_wsum[kCoarseThreads / 32];
+    __shared__ int s_bstar, s_n;
+    __shared__ uint32_t s_tmax;
+
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int64_t r = blockIdx.x;
+    const int64_t q = a.q0 + r;
+    const float *vrow = a.V + r * a.ldv;
+    const int L = a.L, m = a.m;
+    if (tid == 0) {
+        s_n = 0;
+        s_tmax = 0u;
+    }
+    for (int t = tid; t < kSelBins; t += kCoarseThreads) hist[t] = 0;
+
+    // 1. the row's screened values, as order keys, and their range
+    float lmin = INFINITY, lmax = -INFINITY;
+    constexpr int kU = 8;
+    for (int j0 = tid; j0 < L; j0 += kCoarseThreads * kU) {
+        float x[kU];
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+            const int j = j0 + u * kCoarseThreads;
+            x[u] = j < L ? vrow[j] : 0.f;
+        }
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+            const int j = j0 + u * kCoarseThreads;
+            if (j < L) {
+                key[j] = fkey(x[u]);
+                lmin = fminf(lmin, x[u]);
+                lmax = fmaxf(lmax, x[u]);
+            }
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        lmin = fminf(lmin, __shfl_xor_sync(kFull, lmin, o));
+        lmax = fmaxf(lmax, __shfl_xor_sync(kFull, lmax, o));
+    }
+    if (lane == 0) {
+        s_min[warp] = lmin;
+        s_max[warp] = lmax;
+    }
+    __syncthreads();
+    float fmn = s_min[0], fmx = s_max[0];
+#pragma unroll
+    for (int w = 1; w < kCoarseThreads / 32; ++w) {
+        fmn = fminf(fmn, s_min[w]);
+        fmx = fmaxf(fmx, s_max[w]);
+    }
+    const float scale = fmx > fmn ? static_cast<float>(kSelBins - 1) / (fmx - fmn) : 0.f;
+    auto bin_of = [&](uint32_t k) -> int {
+        const float x = fkey_value(k);
+        if (!(x < fmx)) return kSelBins - 1;
+        const int b = static_cast<int>((x - fmn) * scale);
+        return b < 0 ? 0 : (b > kSelBins - 1 ? kSelBins - 1 : b);
+    };
+    // 2. histogram; the bin holding the m-th smallest value
+    for (int j = tid; j < L; j += kCoarseThreads) atomicAdd(&hist[bin_of(key[j])], 1u);
+    __syncthreads();
+    constexpr int kPer = kSelBins / kCoarseThreads;
+    uint32_t h[kPer], sum = 0;
+#pragma unroll
+    for (int t = 0; t < kPer; ++t) {
+        h[t] = hist[tid * kPer + t];
+        sum += h[t];
+    }
+    uint32_t incl = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(kFull, incl, o);
+        if (lane >= o) incl += y;
+    }
+    if (lane == 31) s_wsum[warp] = incl;
+    __syncthreads();
+    {
+        uint32_t c = incl - sum;
+        for (int w = 0; w < warp; ++w) c += s_wsum[w];
+        const uint32_t need = static_cast<uint32_t>(m);
+        if (c < need && need <= c + sum) {
+#pragma unroll
+            for (int t = 0; t < kPer; ++t) {
+                if (c < need && need <= c + h[t]) s_bstar = tid * kPer + t;
+                c += h[t];
+            }
+        }
+    }
+    __syncthreads();
+    // 3. T~ <= the largest value in that bin; candidates within the window above it
+    const int bstar = s_bstar;
+    for (int j = tid; j < L; j += kCoarseThreads)
+        if (bin_of(key[j]) == bstar) atomicMax(&s_tmax, key[j]);
+    __syncthreads();
+    const float W = screen_window(a.xnorm[q], *a.cmax2, a.dp);
+    const uint32_t kthr = fkey(fkey_value(s_tmax) + W);
+    for (int j = tid; j < L; j += kCoarseThreads)
+        if (key[j] <= kthr) cid[atomicAdd(&s_n, 1)] = static_cast<uint32_t>(j);
+    __syncthreads();
+    const int n = s_n;
+    // 4. exact fp64 distance of each candidate, a warp each: fixed lane split, fixed tree
+    const float *qv = a.Q + q * a.d;
+    for (int t = warp; t < n; t += kCoarseThreads / 32) {
+        const float *cv = a.C + static_cast<int64_t>(cid[t]) * a.d;
+        double acc = 0.0;
+        for (int j = lane * 4; j < a.d; j += 128) {
+            const float4 x = __ldg(reinterpret_cast<const float4 *>(qv + j));
+            const float4 y = __ldg(reinterpret_cast<const float4 *>(cv + j));
+            const double e0 = static_cast<double>(x.x) - y.x, e1 = static_cast<double>(x.y) - y.y;
+            const double e2 = static_cast<double>(x.z) - y.z, e3 = static_cast<double>(x.w) - y.w;
+            acc = fma(e0, e0, acc);
+            acc = fma(e1, e1, acc);
+            acc = fma(e2, e2, acc);
+            acc = fma(e3, e3, acc);
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(kFull, acc, o);
+        if (lane == 0) cd[t] = acc;
+    }
+    // 5. sort the candidates by (distance, cell) and keep the first m
+    int M = 1;
+    while (M < n) M <<= 1;
+    for (int t = n + tid; t < M; t += kCoarseThreads) {
+        cd[t] = INFINITY;
+        cid[t] = ~0u;
+    }
+    __syncthreads();
+    for (int size = 2; size <= M; size <<= 1) {
+        for (int stride = size >> 1; stride > 0; stride >>= 1) {
+            for (int t = tid; t < (M >> 1); t += kCoarseThreads) {
+                const int lo = 2 * t - (t & (stride - 1));
+                const int hi = lo + stride;
+                const bool up = (lo & size) == 0;
+                const double da = cd[lo], db = cd[hi];
+                const uint32_t ia = cid[lo], ib = cid[hi];
+                const bool gt = da > db || (da == db && ia > ib);
+                if (gt == up) {
+                    cd[lo] = db;
+                    cd[hi] = da;
+                    cid[lo] = ib;
+                    cid[hi] = ia;
+                }
+            }
+            __syncthreads();
+        }
+    }
+    for (int t = tid; t < m; t += kCoarseThreads)
+        a.probes[q * m + t] = static_cast<int32_t>(cid[t]);
+}
+
+// max_k ||c_k||^2 over the real centroids (one block).
+__global__ void cmax_kernel(const float *__restrict__ cn, int K, float *__restrict__ out) {
+    __shared__ float red[32];
+    float mx = 0.f;
+    for (int k = threadIdx.x; k < K; k += blockDim.x) mx = fmaxf(mx, cn[k]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, o));
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = mx;
+    __syncthreads();
+    if (threadIdx.x < 32) {
+        mx = threadIdx.x < (blockDim.x >> 5) ? red[threadIdx.x] : 0.f;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, o));
+        if (threadIdx.x == 0) *out = mx;
     }
 }
 
@@ -652,6 +968,37 @@ cudaError_t launch_ivf_select(const double *D, const uint32_t *I, int64_t ld, in
     } else {
         select_rows_kernel<false><<<static_cast<unsigned>(rows), kSelThreads, 0, st>>>(a);
     }
+    note_launch();
+    return cudaGetLastError();
+}
+
+bool ivf_coarse_can_screen(int nlist, int dp, int Kp) {
+    return nlist <= kCoarseMaxL && assign_can_dump(dp, Kp);
+}
+
+cudaError_t launch_ivf_cmax(const float *cn, int K, float *out, cudaStream_t st) {
+    cmax_kernel<<<1, 1024, 0, st>>>(cn, K, out);
+    note_launch();
+    return cudaGetLastError();
+}
+
+cudaError_t launch_ivf_coarse_rerank(const float *Vs, int64_t ldv, int64_t rows, int L, int m,
+                                     const float *Q, int64_t q0, const float *C, int d, int dp,
+                                     const float *xnorm, const float *cmax2, int32_t *probes,
+                                     cudaStream_t st) {
+    if (rows <= 0) return cudaSuccess;
+    CoarseArgs a{Vs, ldv, L, m, Q, q0, C, d, dp, xnorm, cmax2, probes};
+    int P = 1;
+    while (P < L) P <<= 1;
+    const size_t smem = static_cast<size_t>(P) * (sizeof(double) + sizeof(uint32_t)) +
+                        static_cast<size_t>(L) * sizeof(uint32_t);
+    static bool attr = false;
+    if (!attr) {
+        cudaFuncSetAttribute(coarse_rerank_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(kCoarseMaxL * (sizeof(double) + 2 * sizeof(uint32_t))));
+        attr = true;
+    }
+    coarse_rerank_kernel<<<static_cast<unsigned>(rows), kCoarseThreads, smem, st>>>(a);
     note_launch();
     return cudaGetLastError();
 }

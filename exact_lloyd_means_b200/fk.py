@@ -42,7 +42,11 @@ class FkTiming(ctypes.Structure):
 
 class FkSearchTiming(ctypes.Structure):
     _fields_ = [("ms_coarse", ctypes.c_double), ("ms_sort", ctypes.c_double),
-                ("ms_fine", ctypes.c_double), ("ms_merge", ctypes.c_double)]
+                ("ms_fine", ctypes.c_double), ("ms_merge", ctypes.c_double),
+                ("screened_coarse", ctypes.c_int)]
+
+
+FK_SEARCH_FP64_COARSE = 1
 
 
 def _sig(name, args, res=ctypes.c_int):
@@ -77,8 +81,8 @@ _sig("fk_lloyd_streamed", [_vp, _int, _i64, _int, _int, _int, _int, _vp, _vp,
 _sig("fk_streamed_workspace_size", [_i64, _int, _int, _int, _int, ctypes.POINTER(_sz)])
 _sig("fk_ivf_norms", [_vp, _i64, _int, _vp, _vp])
 _sig("fk_ivf_search_workspace_size", [_i64, _int, _int, _i64, _int, _int, ctypes.POINTER(_sz)])
-_sig("fk_ivf_search", [_vp, _i64, _int, _vp, _int, _vp, _vp, _vp, _vp, _i64, _int, _int, _vp,
-                       _vp, _vp, _vp, _sz, ctypes.POINTER(FkSearchTiming), _vp])
+_sig("fk_ivf_search", [_vp, _i64, _int, _vp, _int, _vp, _vp, _vp, _vp, _i64, _int, _int, _int,
+                       _vp, _vp, _vp, _vp, _sz, ctypes.POINTER(FkSearchTiming), _vp])
 
 EXPORTED = ["fk_status_string", "fk_version", "fk_workspace_size", "fk_normalize_rows",
             "fk_centroid_norms", "fk_assign", "fk_update", "fk_lloyd",
@@ -414,10 +418,11 @@ def fk_ivf_search(Q: torch.Tensor, C: torch.Tensor, X_lists: torch.Tensor,
                   nprobe: int, k: int, ws: torch.Tensor | None = None,
                   distances: torch.Tensor | None = None, ids: torch.Tensor | None = None,
                   probes: torch.Tensor | None = None, timing: dict | None = None,
-                  stream=None):
+                  fp64_coarse: bool = False, stream=None):
     """IVF-Flat search: returns (distances fp32 [nq, k], ids int32 [nq, k]); `probes`
     (int32 [nq, nprobe]) receives the probed cells when given.  A `timing` dict receives
-    the per-phase device times in ms (the call then synchronises its stream)."""
+    the per-phase device times in ms (the call then synchronises its stream).
+    fp64_coarse computes every coarse distance in fp64 (FK_SEARCH_FP64_COARSE)."""
     nq, d = Q.shape
     nlist = C.shape[0]
     N = X_lists.shape[0]
@@ -434,6 +439,7 @@ def fk_ivf_search(Q: torch.Tensor, C: torch.Tensor, X_lists: torch.Tensor,
                               _dev(X_norms, "X_norms", torch.float64, (N,)),
                               _dev(offsets, "offsets", torch.int32, (nlist + 1,)),
                               _dev(row_ids, "row_ids", torch.int32, (N,)), N, nprobe, k,
+                              FK_SEARCH_FP64_COARSE if fp64_coarse else 0,
                               _dev(distances, "distances", torch.float32, (nq, k)),
                               _dev(ids, "ids", torch.int32, (nq, k)),
                               _opt(probes, "probes", torch.int32, (nq, nprobe)),
@@ -478,7 +484,7 @@ class IvfFlatIndex:
         return cls(C, X_lists, X_norms, offsets, row_ids, metric)
 
     def search(self, Q: torch.Tensor, k: int, nprobe: int, ws=None, distances=None,
-               ids=None, probes=None, timing=None, stream=None):
+               ids=None, probes=None, timing=None, fp64_coarse=False, stream=None):
         """(distances, ids) of the k nearest indexed points of every query, probing nprobe
         cells; a cosine index L2-normalises the queries first."""
         if self.metric == "cosine":
@@ -487,4 +493,5 @@ class IvfFlatIndex:
             Q = Qn
         return fk_ivf_search(Q, self.C, self.X_lists, self.X_norms, self.offsets,
                              self.row_ids, nprobe, k, ws=ws, distances=distances, ids=ids,
-                             probes=probes, timing=timing, stream=stream)
+                             probes=probes, timing=timing, fp64_coarse=fp64_coarse,
+                             stream=stream)

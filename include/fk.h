@@ -289,6 +289,11 @@ FK_API fk_status fk_ivf_search_workspace_size(int64_t nq, int d, int nlist, int6
  * Distances are evaluated in fp64 as ||q||^2 + ||x||^2 - 2 q.x; the selections agree with
  * an exact fp64 evaluation except between candidates whose fp64 distances differ by the
  * rounding of that expression (about 1e-16 of the squared norms).
+ * Coarse pass: by default (flags 0, nlist <= 8192) the query-centroid products run on the
+ * tensor cores with one bf16 product per term; every centroid within a proven error window
+ * of the nprobe-th screened value is then re-ranked in fp64 (difference form), so the
+ * probes are those of the fp64 evaluation.  FK_SEARCH_FP64_COARSE computes every coarse
+ * distance in fp64 instead (same probes, more work).
  *
  * Inputs (device pointers, read only): Q nq x d fp32; C nlist x d fp32 centroids; X_lists
  * N x d fp32, the points in cell order (fk_ivf_lists); X_norms N doubles, fk_ivf_norms of
@@ -307,12 +312,16 @@ typedef struct fk_search_timing {
     double ms_sort;   /* (query, probe) pairs sorted by cell, work items */
     double ms_fine;   /* the fine distance kernel (per-pair k nearest) */
     double ms_merge;  /* the per-query selection of the k nearest */
+    int screened_coarse; /* 1 when the coarse pass ran on the tensor cores (see flags) */
 } fk_search_timing;
+
+/* fk_ivf_search flags. */
+#define FK_SEARCH_FP64_COARSE 1 /* every coarse distance in fp64 (no tensor-core screening) */
 
 FK_API fk_status fk_ivf_search(const float *Q, int64_t nq, int d, const float *C, int nlist,
                                const float *X_lists, const double *X_norms,
                                const int32_t *offsets, const int32_t *row_ids, int64_t N,
-                               int nprobe, int k, float *distances, int32_t *ids,
+                               int nprobe, int k, int flags, float *distances, int32_t *ids,
                                int32_t *probes, void *ws, size_t ws_bytes,
                                fk_search_timing *timing, fk_stream_t stream);
 

@@ -129,12 +129,13 @@ def test_ivf_search_host_checks(fk):
     lib = fk._lib
     big = 1 << 30
     ok = dict(Q=256, nq=10, d=8, C=256, nlist=4, Xl=256, Xn=256, off=256, rid=256, N=100,
-              nprobe=2, k=3, dist=256, ids=256, probes=None, ws=256, wsb=big)
+              nprobe=2, k=3, flags=0, dist=256, ids=256, probes=None, ws=256, wsb=big)
 
     def call(**kw):
         a = dict(ok, **kw)
         return lib.fk_ivf_search(a["Q"], a["nq"], a["d"], a["C"], a["nlist"], a["Xl"], a["Xn"],
-                                 a["off"], a["rid"], a["N"], a["nprobe"], a["k"], a["dist"],
+                                 a["off"], a["rid"], a["N"], a["nprobe"], a["k"], a["flags"],
+                                 a["dist"],
                                  a["ids"], a["probes"], a["ws"], a["wsb"], None, None)
 
     for bad in (dict(nprobe=5), dict(nprobe=0), dict(k=0), dict(k=33), dict(nq=0),

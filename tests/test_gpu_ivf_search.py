@@ -40,13 +40,14 @@ def _index(X, labels, nlist):
     return X_lists, m.fk_ivf_norms(X_lists), offsets, row_ids
 
 
-def _search(Q, C, idx, nprobe, k):
+def _search(Q, C, idx, nprobe, k, fp64_coarse=False, timing=None):
     m = fk()
     X_lists, X_norms, offsets, row_ids = idx
     nq = Q.shape[0]
     probes = torch.full((nq, nprobe), -7, dtype=torch.int32, device=DEV)
     dist, ids = m.fk_ivf_search(Q.to(DEV), C.to(DEV), X_lists, X_norms, offsets, row_ids,
-                                nprobe, k, probes=probes)
+                                nprobe, k, probes=probes, fp64_coarse=fp64_coarse,
+                                timing=timing)
     torch.cuda.synchronize()
     return probes.cpu().numpy(), ids.cpu().numpy(), dist.cpu().numpy()
 
@@ -98,8 +99,9 @@ CASES = [
 ]
 
 
+@pytest.mark.parametrize("coarse", ["screened", "fp64"])
 @pytest.mark.parametrize("N,d,nlist,nq,nprobe,k,weights,labels_from", CASES)
-def test_ivf_search_matches_oracle(N, d, nlist, nq, nprobe, k, weights, labels_from):
+def test_ivf_search_matches_oracle(N, d, nlist, nq, nprobe, k, weights, labels_from, coarse):
     X, comp, _ = gaussian_mixture(N, d, nlist, centers="normal", sigma=0.4, weights=weights,
                                   seed=N + d)
     C = X[init_indices(N, nlist, N + d)].float().contiguous()
@@ -109,7 +111,10 @@ def test_ivf_search_matches_oracle(N, d, nlist, nq, nprobe, k, weights, labels_f
         labels = comp.numpy().astype(np.int32)
     Q = mixture_queries(nq, d, nlist, centers="normal", sigma=0.4, weights=weights,
                         seed=N + d, stream=1)
-    got = _search(Q, C, _index(X, labels, nlist), nprobe, k)
+    tm = {}
+    got = _search(Q, C, _index(X, labels, nlist), nprobe, k, fp64_coarse=coarse == "fp64",
+                  timing=tm)
+    assert tm["screened_coarse"] == (1 if coarse == "screened" else 0)
     ref = oracle.ivf_search(Q, C, X, labels, nprobe, k)
     check_search(Q, C, X, got, ref)
 
@@ -125,10 +130,11 @@ def test_ivf_search_empty_cells_and_few_candidates():
     nlist = C.shape[0]
     Q = torch.cat([extra[:4] + 0.01, mixture_queries(40, d, K, sigma=0.2, seed=7, stream=1)])
     for nprobe, k in ((1, 32), (3, 32), (nlist, 8)):
-        got = _search(Q, C, _index(X, labels, nlist), nprobe, k)
         ref = oracle.ivf_search(Q, C, X, labels, nprobe, k)
         assert (ref[1] == -1).any() or nprobe == nlist
-        check_search(Q, C, X, got, ref, max_bad_frac=0.0)
+        for f64 in (False, True):
+            got = _search(Q, C, _index(X, labels, nlist), nprobe, k, fp64_coarse=f64)
+            check_search(Q, C, X, got, ref, max_bad_frac=0.0)
 
 
 def test_ivf_search_duplicates_and_self_queries():
@@ -208,3 +214,45 @@ def test_ivf_search_argument_errors():
     with pytest.raises(m.FkError) as e:
         m.fk_ivf_search(Q, C, *idx, 2, 3, ws=ws[:1024])
     assert e.value.status == m.FK_ERR_WORKSPACE
+
+
+def test_ivf_search_equal_centroid_distances():
+    """Thousands of identical centroids: every coarse distance of a query ties, so one
+    histogram bin holds more entries than the staged selection sorts and the radix path
+    decides; the probes are the lowest cell indices, as in the oracle."""
+    N, d, nlist = 4000, 16, 3000
+    X, _, _ = gaussian_mixture(N, d, 10, centers="normal", sigma=0.3, seed=21)
+    C = X[:1].expand(nlist, d).contiguous()
+    labels = (np.arange(N) % nlist).astype(np.int32)
+    Q = mixture_queries(40, d, 10, sigma=0.3, seed=21, stream=1)
+    for nprobe, k in ((5, 4), (700, 32)):
+        ref = oracle.ivf_search(Q, C, X, labels, nprobe, k)
+        for f64 in (False, True):
+            got = _search(Q, C, _index(X, labels, nlist), nprobe, k, fp64_coarse=f64)
+            assert (got[0] == np.arange(nprobe)).all()
+            check_search(Q, C, X, got, ref, max_bad_frac=0.0)
+
+
+def test_ivf_search_coarse_paths_agree_and_large_nlist_uses_fp64():
+    """The screened and the fp64 coarse pass give the same probes and results bit for bit
+    on a cosine workload at the guide's d; above 8192 cells the fp64 pass runs."""
+    N, d, K = 60000, 768, 512
+    X, _, _ = gaussian_mixture(N, d, K, centers="normal", sigma=0.3, seed=23)
+    Xn = torch.nn.functional.normalize(X, dim=1)
+    labels = torch.randint(0, K, (N,), generator=torch.Generator().manual_seed(2)).numpy()
+    idx = _index(Xn, labels.astype(np.int32), K)
+    C = Xn[init_indices(N, K, 23)].contiguous()
+    Q = torch.nn.functional.normalize(mixture_queries(1000, d, K, sigma=0.3, seed=23,
+                                                      stream=1), dim=1)
+    for nprobe in (1, 16, 128):
+        ta, tb = {}, {}
+        a = _search(Q, C, idx, nprobe, 10, timing=ta)
+        b = _search(Q, C, idx, nprobe, 10, fp64_coarse=True, timing=tb)
+        assert ta["screened_coarse"] == 1 and tb["screened_coarse"] == 0
+        assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
+        assert np.array_equal(a[2], b[2])
+    tm = {}
+    Cbig = Xn[init_indices(N, 9000, 24)].contiguous()
+    lab = torch.randint(0, 9000, (N,), generator=torch.Generator().manual_seed(3)).numpy()
+    _search(Q[:50], Cbig, _index(Xn, lab.astype(np.int32), 9000), 4, 5, timing=tm)
+    assert tm["screened_coarse"] == 0
