@@ -697,11 +697,23 @@ def search_arm(args, spec, rank, world, dist):
                       "index": f"fk_lloyd {args.niter or spec.niter} iterations + "
                                "fk_ivf_lists + fk_ivf_norms, built before timing",
                       "l2": "cell-ordered points (N x d fp32) larger than L2; no flush"},
-           "roofline": {"bound": "alu", "achieved": fine_tf, "peak": peak,
-                        "unit": "TFLOP/s", "frac": fine_tf / peak, "traffic": None,
-                        "kernel": "ivf_tile_kernel<true> (fine pass, fp64 FMA)",
-                        "flops_per_launch": fine_flops, "avg_ms": phases["ms_fine"],
-                        "peak_basis": f"148 SMs x 64 fp64 FMA/clk x 2 x {mhz:.0f} MHz"},
+           "roofline": ({"bound": "tensor", "achieved": fine_tf,
+                         "peak": load_peaks()["bf16"] / 3, "unit": "TFLOP/s",
+                         "frac": fine_tf / (load_peaks()["bf16"] / 3), "traffic": None,
+                         "kernel": "ivf_fine_scr_kernel (fine pass: three bf16 products per "
+                                   "term on mma.m16n8k16, fp32 accumulation)",
+                         "flops_per_launch": fine_flops, "avg_ms": phases["ms_fine"],
+                         "peak_basis": "measured bf16 burst peak / 3 (a third of the tensor "
+                                       "work is useful); mma.m16n8k16 bf16 measured alone "
+                                       "at 550 TFLOP/s on this GPU"}
+                        if phases.get("screened_fine") else
+                        {"bound": "alu", "achieved": fine_tf, "peak": peak,
+                         "unit": "TFLOP/s", "frac": fine_tf / peak, "traffic": None,
+                         "kernel": "ivf_tile_kernel<true> (fine pass, fp64 mma.m8n8k4)",
+                         "flops_per_launch": fine_flops, "avg_ms": phases["ms_fine"],
+                         "peak_basis": f"148 SMs x 64 fp64 FMA/clk x 2 x {mhz:.0f} MHz"}),
+           "fine_path": "tensor-core screening (three bf16 products) + fp64 re-ranking"
+                        if phases.get("screened_fine") else "fp64",
            "coarse": {"path": "tensor-core screening + fp64 re-ranking"
                               if phases.get("screened_coarse") else "fp64",
                       "useful_tflops": coarse_tf, "flops": coarse_flops,

@@ -258,10 +258,11 @@ fk_status validate_search(int64_t nq, int d, int nlist, int64_t N, int nprobe, i
 }
 
 fk_status run_ivf_search(const float *Q, int64_t nq, int d, const float *C, int nlist,
-                         const float *X_lists, const double *X_norms, const int32_t *offsets,
-                         const int32_t *row_ids, int nprobe, int k, bool screen,
-                         float *distances, int32_t *ids, int32_t *probes, void *ws,
-                         const SearchLayout &L, cudaStream_t st, const cudaEvent_t *ev) {
+                         const float *X_lists, const double *X_norms, const void *X_planes,
+                         const int32_t *offsets, const int32_t *row_ids, int64_t N, int nprobe,
+                         int k, bool screen, bool screen_fine, float *distances, int32_t *ids,
+                         int32_t *probes, void *ws, const SearchLayout &L, cudaStream_t st,
+                         const cudaEvent_t *ev) {
     // ev (optional): five events recorded between the phases
     auto mark = [&](int i) { return !ev || cudaEventRecord(ev[i], st) == cudaSuccess; };
     if (!mark(0)) return FK_ERR_CUDA;
@@ -271,12 +272,15 @@ fk_status run_ivf_search(const float *Q, int64_t nq, int d, const float *C, int 
     // coarse: distances to every centroid, then the nprobe nearest per query
     int32_t *pr = probes ? probes : ws_ptr<int32_t>(ws, L.probes);
     double *D = ws_ptr<double>(ws, L.D);
+    uint16_t *qh = ws_ptr<uint16_t>(ws, L.qplanes);
+    float *qxn = ws_ptr<float>(ws, L.qxn);
+    if (screen || screen_fine)  // bf16 hi / lo planes of every query, and ||q||^2
+        FK_TRY_CUDA(launch_split_x(Q, nq, d, L.dp, qh, qh + nq * L.dp, qxn, st));
     if (screen) {
         // tensor-core screening of every (query, centroid), fp64 re-ranking of the window
         AssignArgs a{};
-        uint16_t *qh = ws_ptr<uint16_t>(ws, L.qplanes);
         uint16_t *cpl = ws_ptr<uint16_t>(ws, L.cplanes);
-        float *ccn = ws_ptr<float>(ws, L.ccn), *qxn = ws_ptr<float>(ws, L.qxn);
+        float *ccn = ws_ptr<float>(ws, L.ccn);
         float *cmax2 = ws_ptr<float>(ws, L.cmax2), *Vs = ws_ptr<float>(ws, L.D);
         FK_TRY_CUDA(launch_prep_centroids(C, nlist, d, L.Kp, L.dp, FK_F32, cpl, ccn,
                                           ws_ptr<float>(ws, L.cused),
@@ -291,7 +295,6 @@ fk_status run_ivf_search(const float *Q, int64_t nq, int d, const float *C, int 
         a.dp = static_cast<int>(L.dp);
         a.K = nlist;
         a.Kp = static_cast<int>(L.Kp);
-        a.xnorm = qxn;
         a.err = ws_ptr<uint32_t>(ws, L.err);
         a.wait_ns = kDefaultWaitNs;
         a.cmax2 = cmax2;
@@ -299,12 +302,13 @@ fk_status run_ivf_search(const float *Q, int64_t nq, int d, const float *C, int 
         a.ldd = L.Kp;
         for (int64_t q0 = 0; q0 < nq; q0 += L.qbatch) {
             const int64_t nqb = nq - q0 < L.qbatch ? nq - q0 : L.qbatch;
-            FK_TRY_CUDA(launch_split_x(Q + q0 * d, nqb, d, L.dp, qh, qh + nqb * L.dp, qxn, st));
-            a.a_planes = qh;
+            a.a_planes = qh + q0 * L.dp;  // rows q0 .. of the hi plane
+            a.xnorm = qxn + q0;
             a.N = nqb;
             FK_TRY_CUDA(launch_assign(a, st));
             FK_TRY_CUDA(launch_ivf_coarse_rerank(Vs, L.Kp, nqb, nlist, nprobe, Q, q0, C, d,
-                                                 static_cast<int>(L.dp), qxn, cmax2, pr, st));
+                                                 static_cast<int>(L.dp), qxn + q0, cmax2, pr,
+                                                 st));
         }
     } else {
         for (int64_t q0 = 0; q0 < nq; q0 += L.qbatch) {
@@ -327,15 +331,36 @@ fk_status run_ivf_search(const float *Q, int64_t nq, int d, const float *C, int 
     int *nitems = ws_ptr<int>(ws, L.nitems);
     FK_TRY_CUDA(launch_ivf_items(poff, nlist, items, nitems, nitems + 1, st));
     if (!mark(2)) return FK_ERR_CUDA;
-    // fine: per pair, the k nearest points of its cell; then per query the k nearest overall
-    double *Ld = ws_ptr<double>(ws, L.Ld);
-    uint32_t *Li = ws_ptr<uint32_t>(ws, L.Li);
-    FK_TRY_CUDA(launch_ivf_fine(Q, qn, d, X_lists, X_norms, offsets, row_ids, psorted, poff,
-                                items, nitems, nitems + 1, L.max_items, nprobe, k, Ld, Li, st));
-    if (!mark(3)) return FK_ERR_CUDA;
-    const int64_t Lrow = static_cast<int64_t>(nprobe) * k;
-    FK_TRY_CUDA(launch_ivf_select(Ld, Li, Lrow, nq, static_cast<int>(Lrow), k, ids, distances,
-                                  k, st));
+    if (screen_fine) {
+        // per pair the 32 smallest screened distances; per query the window re-ranked in
+        // fp64; the queries whose lists may have dropped a candidate, exactly
+        float *Sv = ws_ptr<float>(ws, L.Sv), *Slost = ws_ptr<float>(ws, L.Slost);
+        uint32_t *Sp = ws_ptr<uint32_t>(ws, L.Sp);
+        int32_t *fb = ws_ptr<int32_t>(ws, L.fb);
+        float *xmax2 = ws_ptr<float>(ws, L.xmax2);
+        const uint16_t *Xp = static_cast<const uint16_t *>(X_planes);
+        FK_TRY_CUDA(launch_ivf_fine_scr(qh, nq, Xp, N, static_cast<int>(L.dp), qn, X_norms,
+                                        offsets, psorted, poff, items, nitems, nitems + 1,
+                                        L.max_items, nprobe, Sv, Sp, Slost, st));
+        if (!mark(3)) return FK_ERR_CUDA;
+        FK_TRY_CUDA(launch_max_norm(X_norms, N, xmax2, st));
+        FK_TRY_CUDA(launch_ivf_query_rerank(Sv, Sp, Slost, nq, nprobe, k, Q, X_lists, d,
+                                            static_cast<int>(L.dp), qn, xmax2, row_ids,
+                                            distances, ids, fb, st));
+        FK_TRY_CUDA(launch_ivf_fallback(fb, pr, nq, nprobe, k, Q, X_lists, d, offsets, row_ids,
+                                        distances, ids, st));
+    } else {
+        // fine: per pair, the k nearest points of its cell; then per query the k nearest
+        double *Ld = ws_ptr<double>(ws, L.Ld);
+        uint32_t *Li = ws_ptr<uint32_t>(ws, L.Li);
+        FK_TRY_CUDA(launch_ivf_fine(Q, qn, d, X_lists, X_norms, offsets, row_ids, psorted, poff,
+                                    items, nitems, nitems + 1, L.max_items, nprobe, k, Ld, Li,
+                                    st));
+        if (!mark(3)) return FK_ERR_CUDA;
+        const int64_t Lrow = static_cast<int64_t>(nprobe) * k;
+        FK_TRY_CUDA(launch_ivf_select(Ld, Li, Lrow, nq, static_cast<int>(Lrow), k, ids,
+                                      distances, k, st));
+    }
     if (!mark(4)) return FK_ERR_CUDA;
     return FK_OK;
 }
@@ -899,8 +924,9 @@ fk_status fk_ivf_search_workspace_size(int64_t nq, int d, int nlist, int64_t N, 
 }
 
 fk_status fk_ivf_search(const float *Q, int64_t nq, int d, const float *C, int nlist,
-                        const float *X_lists, const double *X_norms, const int32_t *offsets,
-                        const int32_t *row_ids, int64_t N, int nprobe, int k, int flags,
+                        const float *X_lists, const double *X_norms, const void *X_planes,
+                        const int32_t *offsets, const int32_t *row_ids, int64_t N, int nprobe,
+                        int k, int flags,
                         float *distances, int32_t *ids, int32_t *probes, void *ws,
                         size_t ws_bytes, fk_search_timing *timing, fk_stream_t stream) {
     fk_status s = validate_search(nq, d, nlist, N, nprobe, k);
@@ -909,7 +935,8 @@ fk_status fk_ivf_search(const float *Q, int64_t nq, int d, const float *C, int n
         return FK_ERR_INVALID_ARG;
     if (!aligned(Q, 16) || !aligned(C, 16) || !aligned(X_lists, 16) || !aligned(X_norms, 8) ||
         !aligned(offsets, 4) || !aligned(row_ids, 4) || !aligned(distances, 4) ||
-        !aligned(ids, 4) || (probes && !aligned(probes, 4)))
+        !aligned(ids, 4) || (probes && !aligned(probes, 4)) ||
+        (X_planes && !aligned(X_planes, 16)))
         return FK_ERR_UNSUPPORTED;
     const SearchLayout L = search_layout(nq, d, nlist, nprobe, k);
     if (ws == nullptr || !aligned(ws, 256) || ws_bytes < L.total) return FK_ERR_WORKSPACE;
@@ -930,14 +957,27 @@ fk_status fk_ivf_search(const float *Q, int64_t nq, int d, const float *C, int n
     const bool screen = (flags & FK_SEARCH_FP64_COARSE) == 0 &&
                         ivf_coarse_can_screen(nlist, static_cast<int>(L.dp),
                                               static_cast<int>(L.Kp));
-    const fk_status r = run_ivf_search(Q, nq, d, C, nlist, X_lists, X_norms, offsets, row_ids,
-                                       nprobe, k, screen, distances, ids, probes, ws, L, st,
-                                       timing ? ev : nullptr);
+    const bool screen_fine = X_planes != nullptr && (flags & FK_SEARCH_FP64_FINE) == 0 &&
+                             k <= kSearchScrMaxK && nprobe <= kSearchScrMaxProbe;
+    const fk_status r = run_ivf_search(Q, nq, d, C, nlist, X_lists, X_norms, X_planes, offsets,
+                                       row_ids, N, nprobe, k, screen, screen_fine, distances,
+                                       ids, probes, ws, L, st, timing ? ev : nullptr);
     if (r == FK_OK && timing) {
+        int nfb = 0;
+        if (screen_fine) {  // the flagged-query count sits in the word after the max norm
+            int *cnt = ws_ptr<int>(ws, L.xmax2) + 1;
+            if (launch_count_flags(ws_ptr<int32_t>(ws, L.fb), nq, cnt, st) != cudaSuccess ||
+                cudaMemcpyAsync(&nfb, cnt, sizeof(int), cudaMemcpyDeviceToHost, st) !=
+                    cudaSuccess) {
+                destroy();
+                return FK_ERR_CUDA;
+            }
+        }
         if (cudaStreamSynchronize(st) != cudaSuccess) {
             destroy();
             return FK_ERR_CUDA;
         }
+        timing->fallback_queries = nfb;
         float ms[4] = {0, 0, 0, 0};
         for (int i = 0; i < 4; ++i) cudaEventElapsedTime(&ms[i], ev[i], ev[i + 1]);
         timing->ms_coarse = ms[0];
@@ -945,6 +985,7 @@ fk_status fk_ivf_search(const float *Q, int64_t nq, int d, const float *C, int n
         timing->ms_fine = ms[2];
         timing->ms_merge = ms[3];
         timing->screened_coarse = screen ? 1 : 0;
+        timing->screened_fine = screen_fine ? 1 : 0;
     }
     destroy();
     return r;

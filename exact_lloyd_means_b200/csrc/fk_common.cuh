@@ -320,9 +320,37 @@ cudaError_t launch_ivf_fine(const float *Q, const double *qn, int d, const float
                             const int2 *items, const int *nitems, int *item_ctr, int64_t max_items,
                             int nprobe, int k, double *Ld, uint32_t *Li, cudaStream_t st);
 
+// The screened fine pass (ivf_search.cu): bf16 three-product screening per (query, point),
+// per-pair lists of the 32 smallest screened distances, a per-query merge that re-ranks the
+// window in fp64, and an exact fallback for the queries whose lists may have dropped a
+// point of their top-k.
+cudaError_t launch_ivf_fine_scr(const uint16_t *Qp, int64_t nq, const uint16_t *Xp, int64_t N,
+                                int dp, const double *qn, const double *xn,
+                                const int32_t *offsets, const int32_t *pair_sorted,
+                                const int32_t *pair_off, const int2 *items, const int *nitems,
+                                int *item_ctr, int64_t max_items, int nprobe, float *Sv,
+                                uint32_t *Sp, float *Slost, cudaStream_t st);
+cudaError_t launch_ivf_query_rerank(const float *Sv, const uint32_t *Sp, const float *Slost,
+                                    int64_t nq, int nprobe, int k, const float *Q,
+                                    const float *X, int d, int dp, const double *qn,
+                                    const float *xmax2, const int32_t *row_ids,
+                                    float *out_dist, int32_t *out_id, int32_t *fallback,
+                                    cudaStream_t st);
+cudaError_t launch_ivf_fallback(const int32_t *fallback, const int32_t *probes, int64_t nq,
+                                int nprobe, int k, const float *Q, const float *X, int d,
+                                const int32_t *offsets, const int32_t *row_ids, float *out_dist,
+                                int32_t *out_id, cudaStream_t st);
+cudaError_t launch_max_norm(const double *xn, int64_t n, float *out, cudaStream_t st);
+cudaError_t launch_count_flags(const int32_t *f, int64_t n, int *out, cudaStream_t st);
+
 // Limits of fk_ivf_search: k is held one rank per lane, nprobe by the selection's sort.
 constexpr int kSearchMaxK = 32;
 constexpr int kSearchMaxProbe = 1024;
+// The screened fine pass: k up to half a pair list (the rest is slack against dropping a
+// point of the top-k), and a query's nprobe lists staged in shared memory at once.
+constexpr int kSearchScrMaxK = 16;
+constexpr int kSearchScrMaxProbe = 256;
+constexpr int kSearchScrList = 32;
 constexpr int kSearchPairsPerItem = 32;
 // Rows of the coarse distance matrix held at once: a query batch of at most this many bytes.
 constexpr int64_t kSearchCoarseBytes = int64_t(512) << 20;
@@ -331,7 +359,7 @@ struct SearchLayout {
     size_t err = 0, qn = 0, cn = 0, D = 0, probes = 0, keys0 = 0, keys1 = 0, vals0 = 0,
            vals1 = 0, hist = 0, dtot = 0, psorted = 0, poff = 0, items = 0, nitems = 0,
            Ld = 0, Li = 0, qplanes = 0, qxn = 0, cplanes = 0, ccn = 0, cused = 0, caug = 0,
-           cmax2 = 0, total = 0;
+           cmax2 = 0, Sv = 0, Sp = 0, Slost = 0, fb = 0, xmax2 = 0, total = 0;
     int64_t P = 0, qbatch = 0, max_items = 0, dp = 0, Kp = 0;
     SortPlan sp;
 };
@@ -374,14 +402,21 @@ inline SearchLayout search_layout(int64_t nq, int d, int nlist, int nprobe, int 
     L.nitems = take(sizeof(int32_t) * 2);
     L.Ld = take(sizeof(double) * L.P * k);
     L.Li = take(sizeof(uint32_t) * L.P * k);
-    // screened coarse pass: bf16 planes of a query batch and of the centroids
-    L.qplanes = take(sizeof(uint16_t) * 2 * L.qbatch * L.dp);
-    L.qxn = take(sizeof(float) * L.qbatch);
+    // screened passes: bf16 planes of the queries and of the centroids
+    L.qplanes = take(sizeof(uint16_t) * 2 * nq * L.dp);
+    L.qxn = take(sizeof(float) * nq);
     L.cplanes = take(sizeof(uint16_t) * 2 * L.Kp * L.dp);
     L.ccn = take(sizeof(float) * L.Kp);
     L.cused = take(sizeof(float) * nlist * d);
     L.caug = take(sizeof(uint16_t) * L.Kp * kAug);
     L.cmax2 = take(256);
+    // screened fine pass: per-pair lists, per-query fallback flags, the largest point norm
+    const bool scr_fine = k <= kSearchScrMaxK && nprobe <= kSearchScrMaxProbe;
+    L.Sv = take(scr_fine ? sizeof(float) * L.P * kSearchScrList : 0);
+    L.Sp = take(scr_fine ? sizeof(uint32_t) * L.P * kSearchScrList : 0);
+    L.Slost = take(scr_fine ? sizeof(float) * L.P : 0);
+    L.fb = take(scr_fine ? sizeof(int32_t) * nq : 0);
+    L.xmax2 = take(256);
     L.total = o;
     return L;
 }

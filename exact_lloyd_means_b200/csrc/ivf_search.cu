@@ -353,7 +353,6 @@ __global__ void __launch_bounds__(kTThreads, 4) ivf_tile_kernel(TileArgs a) {
 // histogram of the entries that still match the decided digits, stopping as soon as every
 // entry of the chosen bin is inside the first m; exactly m entries are gathered.
 constexpr int kSelThreads = 256;
-constexpr int kSelMaxM = 1024;     // largest m
 constexpr int kSelCache = 8192;    // rows up to this length are staged in shared memory
 constexpr int kSelBins = 2048;     // histogram bins of the staged path
 constexpr int kSelMaxCand = 2048;  // candidates the staged path sorts
@@ -840,6 +839,646 @@ __global__ void cmax_kernel(const float *__restrict__ cn, int K, float *__restri
     }
 }
 
+// ---------------------------------------------------------------- screened fine pass
+// The fine products on the tensor cores.  Each (query, point) dot product is taken as three
+// bf16 products of the RN-bf16 split x = hi + lo (+ a residual below 2^-16 |x|) of both
+// sides, hi.hi + hi.lo + lo.hi, accumulated in fp32 by mma.m16n8k16; the screened distance
+// s~ = ||q||^2 + ||x||^2 - 2 q.x~ (rounded to fp32) is within E(q) of the exact one
+// (fine_window_coeffs).  Per pair a lane-held list keeps the kScrList smallest s~ with the points'
+// positions, and the smallest s~ it dropped ("lost").  query_rerank_kernel merges a query's
+// lists: every point of the exact top-k has s~ within 2E of the k-th smallest s~, so
+// re-ranking those entries in fp64 gives the exact result -- unless a pair dropped an
+// entry inside that window, which sends the query to fallback_kernel.
+// Tile: 128 points x 32 queries; warp w owns points 32w .. 32w + 31 (two 16-row blocks)
+// and all four 8-query blocks.  bf16 chunks of 32 dimensions of both planes arrive by
+// cp.async in two stages, rows of 40 elements (80 bytes: the 8 rows an ldmatrix reads
+// fall on distinct banks).
+constexpr int kScrList = kSearchScrList;  // entries per pair list, one per lane
+constexpr int kBS = kTD + 8;   // bf16 row stride of the stages
+constexpr int kDSF = kTV + 4;  // fp32 row stride of the dot-product rows
+
+struct StageB {
+    uint16_t vh[kTV * kBS], vl[kTV * kBS];  // points: hi, lo
+    uint16_t qh[kTQ * kBS], ql[kTQ * kBS];  // queries: hi, lo
+};
+
+struct FineSmem {
+    union {
+        StageB st[2];
+        float dot[kTQ * kDSF];  // [query][point]
+    };
+};
+
+struct FineArgs {
+    const uint16_t *Qp;        // [2][nq][dp] bf16 planes of the queries
+    int64_t nq;
+    const uint16_t *Xp;        // [2][N][dp] bf16 planes of the cell-ordered points
+    int64_t N;
+    int dp;
+    const double *qn, *xn;     // fp64 squared norms
+    const int32_t *offsets, *pair_sorted, *pair_off;
+    const int2 *items;
+    const int *nitems;
+    int *item_ctr;
+    int nprobe;
+    float *Sv;                 // [P][kScrList] screened values, ascending
+    uint32_t *Sp;              // [P][kScrList] point positions (0xffffffff: no point)
+    float *Slost;              // [P]
+};
+
+__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], const void *p) {
+    const uint32_t a = static_cast<uint32_t>(__cvta_generic_to_shared(p));
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(a)
+                 : "memory");
+}
+
+// C (16 x 8, fp32) += A (16 x 16, bf16, row) B (16 x 8, bf16, col).  This lane holds
+// A[g][2t..], A[g+8][2t..], A[g][2t+8..], A[g+8][2t+8..], B[2t..][g], B[2t+8..][g] and
+// C[g][2t], C[g][2t+1], C[g+8][2t], C[g+8][2t+1], with g = lane / 4, t = lane % 4.
+__device__ __forceinline__ void hmma(float (&c)[4], const uint32_t (&a)[4], uint32_t b0,
+                                     uint32_t b1) {
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, "
+        "{%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// Chunk j0 .. j0 + 31 of both planes of the tile's points (rows 0 .. nv - 1 from v0) and
+// of the item's queries: thread t copies 16-byte piece t % 4 of point rows t / 4 + 32 r
+// and of query row t / 4.  Rows past the data are zeros.
+__device__ __forceinline__ void stage_issue_b(StageB &sb, const uint16_t *Xh, const uint16_t *Xl,
+                                              int64_t v0, int nv, int dp, const uint16_t *qh,
+                                              const uint16_t *ql, int j0, int tid) {
+    const int c16 = tid & 3;
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+        const int row = (tid >> 2) + 32 * r;
+        const bool ok = row < nv;
+        const int64_t off = ok ? (v0 + row) * dp + j0 + c16 * 8 : 0;
+        cp_async16(sb.vh + row * kBS + c16 * 8, Xh + off, ok ? 16 : 0);
+        cp_async16(sb.vl + row * kBS + c16 * 8, Xl + off, ok ? 16 : 0);
+    }
+    const int qr = tid >> 2;
+    cp_async16(sb.qh + qr * kBS + c16 * 8, qh ? qh + j0 + c16 * 8 : Xh, qh ? 16 : 0);
+    cp_async16(sb.ql + qr * kBS + c16 * 8, ql ? ql + j0 + c16 * 8 : Xh, ql ? 16 : 0);
+}
+
+// acc[m][n] += the chunk's three-product dot products of point block (2 warp + m) with
+// query block n, for the mact point blocks and nact query blocks that hold data.
+__device__ __forceinline__ void fine_mma(const StageB &sb, int warp, int lane, int mact,
+                                         int nact, float (&acc)[2][4][4]) {
+    const int i = lane >> 3, r = lane & 7;
+#pragma unroll
+    for (int ks = 0; ks < kTD / 16; ++ks) {
+        uint32_t bh[2][4], bl[2][4];
+#pragma unroll
+        for (int np = 0; np < 2; ++np) {
+            if (2 * np < nact) {
+                const int q = np * 16 + (i >> 1) * 8 + r;
+                const int col = ks * 16 + (i & 1) * 8;
+                ldsm_x4(bh[np], sb.qh + q * kBS + col);
+                ldsm_x4(bl[np], sb.ql + q * kBS + col);
+            }
+        }
+#pragma unroll
+        for (int m = 0; m < 2; ++m) {
+            if (m < mact) {
+                const int p = warp * 32 + m * 16 + (i & 1) * 8 + r;
+                const int col = ks * 16 + (i >> 1) * 8;
+                uint32_t ah[4], al[4];
+                ldsm_x4(ah, sb.vh + p * kBS + col);
+                ldsm_x4(al, sb.vl + p * kBS + col);
+#pragma unroll
+                for (int n = 0; n < 4; ++n) {
+                    if (n < nact) {
+                        const int o = (n & 1) * 2;
+                        hmma(acc[m][n], ah, bh[n >> 1][o], bh[n >> 1][o + 1]);
+                        hmma(acc[m][n], ah, bl[n >> 1][o], bl[n >> 1][o + 1]);
+                        hmma(acc[m][n], al, bh[n >> 1][o], bh[n >> 1][o + 1]);
+                    }
+                }
+            }
+        }
+    }
+}
+
+__device__ __forceinline__ bool before_f(float a, uint32_t pa, float b, uint32_t pb) {
+    return a < b || (a == b && pa < pb);
+}
+
+__global__ void __launch_bounds__(kTThreads, 4) ivf_fine_scr_kernel(FineArgs a) {
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    FineSmem &sm = *reinterpret_cast<FineSmem *>(smem_raw);
+    __shared__ int s_item;
+    __shared__ int s_pair[kTQ];
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int dp = a.dp;
+    const uint16_t *Xh = a.Xp, *Xl = a.Xp + a.N * dp;
+    const uint16_t *Qh = a.Qp, *Ql = a.Qp + a.nq * dp;
+
+    for (;;) {
+        if (tid == 0) s_item = atomicAdd(a.item_ctr, 1);
+        __syncthreads();
+        const int item = s_item;
+        if (item >= *a.nitems) return;
+        const int2 it = a.items[item];
+        const int nq_i = min(kTQ, a.pair_off[it.x + 1] - it.y);
+        const int64_t vbeg = a.offsets[it.x], vend = a.offsets[it.x + 1];
+        if (tid < kTQ) s_pair[tid] = tid < nq_i ? a.pair_sorted[it.y + tid] : 0;
+        __syncthreads();
+
+        const int sq = tid >> 2;  // the query row this thread stages
+        const int64_t qrow = sq < nq_i ? static_cast<int64_t>(s_pair[sq] / a.nprobe) * dp : -1;
+        const uint16_t *qh = qrow >= 0 ? Qh + qrow : nullptr;
+        const uint16_t *ql = qrow >= 0 ? Ql + qrow : nullptr;
+        const int nact = (nq_i + 7) >> 3;
+
+        // per-pair lists: lane r holds rank r of each of the warp's 8 queries
+        float lv[8], lost[8];
+        uint32_t lp[8];
+#pragma unroll
+        for (int q8 = 0; q8 < 8; ++q8) {
+            lv[q8] = INFINITY;
+            lp[q8] = 0xffffffffu;
+            lost[q8] = INFINITY;
+        }
+
+        for (int64_t v0 = vbeg; v0 < vend; v0 += kTV) {
+            const int nv_t = static_cast<int>(min(static_cast<int64_t>(kTV), vend - v0));
+            const int mact = max(0, min(2, (nv_t + 15) / 16 - 2 * warp));
+            float acc[2][4][4];
+#pragma unroll
+            for (int m = 0; m < 2; ++m)
+#pragma unroll
+                for (int n = 0; n < 4; ++n)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) acc[m][n][e] = 0.f;
+            const int nch = dp / kTD;
+            __syncthreads();  // the previous tile's readers of the dot rows are done
+            stage_issue_b(sm.st[0], Xh, Xl, v0, nv_t, dp, qh, ql, 0, tid);
+            cp_async_commit();
+            for (int c = 0; c < nch; ++c) {
+                cp_async_wait<0>();
+                __syncthreads();  // chunk c landed everywhere; chunk c - 1's stage is free
+                if (c + 1 < nch) {
+                    stage_issue_b(sm.st[(c + 1) & 1], Xh, Xl, v0, nv_t, dp, qh, ql,
+                                  (c + 1) * kTD, tid);
+                    cp_async_commit();
+                }
+                if (mact > 0) fine_mma(sm.st[c & 1], warp, lane, mact, nact, acc);
+            }
+            __syncthreads();  // every warp is done with the last stage
+            {
+                const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+                for (int m = 0; m < 2; ++m)
+#pragma unroll
+                    for (int n = 0; n < 4; ++n)
+                        if (m < mact && n < nact) {
+                            const int p = warp * 32 + m * 16 + g, q = n * 8 + 2 * t;
+                            sm.dot[q * kDSF + p] = acc[m][n][0];
+                            sm.dot[(q + 1) * kDSF + p] = acc[m][n][1];
+                            sm.dot[q * kDSF + p + 8] = acc[m][n][2];
+                            sm.dot[(q + 1) * kDSF + p + 8] = acc[m][n][3];
+                        }
+            }
+            __syncthreads();
+
+            double xn_i[4];
+            bool ok_i[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int vl = lane + 32 * i;
+                ok_i[i] = vl < nv_t;
+                xn_i[i] = ok_i[i] ? a.xn[v0 + vl] : 0.0;
+            }
+#pragma unroll
+            for (int q8 = 0; q8 < 8; ++q8) {
+                const int qi = warp * 8 + q8;
+                if (qi >= nq_i) continue;  // warp-uniform
+                const double qn = a.qn[s_pair[qi] / a.nprobe];
+                float tv = __shfl_sync(kFull, lv[q8], kScrList - 1);
+                uint32_t tp = __shfl_sync(kFull, lp[q8], kScrList - 1);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const float cv = ok_i[i] ? static_cast<float>(fma(
+                                                   -2.0, static_cast<double>(sm.dot[qi * kDSF + lane + 32 * i]),
+                                                   qn + xn_i[i]))
+                                             : INFINITY;
+                    const uint32_t cp = static_cast<uint32_t>(v0 + lane + 32 * i);
+                    bool pend = ok_i[i] && before_f(cv, cp, tv, tp);
+                    if (ok_i[i] && !pend) lost[q8] = fminf(lost[q8], cv);
+                    unsigned m = __ballot_sync(kFull, pend);
+                    while (m) {
+                        const int src = __ffs(m) - 1;
+                        const float xv = __shfl_sync(kFull, cv, src);
+                        const uint32_t xp = __shfl_sync(kFull, cp, src);
+                        const int pos = __popc(__ballot_sync(kFull, before_f(lv[q8], lp[q8], xv, xp)));
+                        // the last entry leaves a full list: it joins the dropped values
+                        if (lane == kScrList - 1 && lp[q8] != 0xffffffffu)
+                            lost[q8] = fminf(lost[q8], lv[q8]);
+                        const float uv = __shfl_up_sync(kFull, lv[q8], 1);
+                        const uint32_t up = __shfl_up_sync(kFull, lp[q8], 1);
+                        if (lane == pos) {
+                            lv[q8] = xv;
+                            lp[q8] = xp;
+                        } else if (lane > pos) {
+                            lv[q8] = uv;
+                            lp[q8] = up;
+                        }
+                        tv = __shfl_sync(kFull, lv[q8], kScrList - 1);
+                        tp = __shfl_sync(kFull, lp[q8], kScrList - 1);
+                        if (lane == src) pend = false;
+                        if (pend && !before_f(cv, cp, tv, tp)) {
+                            pend = false;
+                            lost[q8] = fminf(lost[q8], cv);
+                        }
+                        m = __ballot_sync(kFull, pend);
+                    }
+                }
+            }
+        }
+
+#pragma unroll
+        for (int q8 = 0; q8 < 8; ++q8) {
+            const int qi = warp * 8 + q8;
+            if (qi >= nq_i) continue;
+            float lo = lost[q8];
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) lo = fminf(lo, __shfl_xor_sync(kFull, lo, o));
+            const int64_t pr = s_pair[qi];
+            a.Sv[pr * kScrList + lane] = lv[q8];
+            a.Sp[pr * kScrList + lane] = lp[q8];
+            if (lane == 0) a.Slost[pr] = lo;
+        }
+    }
+}
+
+// Per query (one block): the nprobe pair lists merged.  T~ bounds the k-th smallest screened
+// value from above (the largest value of the histogram bin holding it); every point of the
+// exact top-k has s~ <= T~ + W, W = 2 E(q).  If a pair dropped a value at or below that,
+// its list may lack such a point: the query is flagged for fallback_kernel.  Otherwise the
+// entries up to T~ + W are re-ranked exactly (fp64, difference form; a warp per entry) and
+// the k smallest by (distance, original id) written.
+constexpr int kQThreads = 256;
+
+struct QueryArgs {
+    const float *Sv;
+    const uint32_t *Sp;
+    const float *Slost;
+    int nprobe, k;
+    const float *Q, *X;        // fp32 queries [nq][d] and cell-ordered points [N][d]
+    int d;
+    const double *qn;          // fp64 ||q||^2
+    const float *xmax2;        // max ||x||^2 over the points
+    float ce_dot;              // |s~ - s| <= ce_dot ||q|| ||x|| + ce_round (||q||^2 + ||x||^2)
+    float ce_round;
+    const int32_t *row_ids;
+    float *out_dist;
+    int32_t *out_id;
+    int32_t *fallback;         // [nq]: 1 for queries left to fallback_kernel
+};
+
+__device__ __forceinline__ double exact_sq_dist(const float *q, const float *x, int d, int lane) {
+    double acc = 0.0;
+    for (int j = lane * 4; j < d; j += 128) {
+        const float4 u = __ldg(reinterpret_cast<const float4 *>(q + j));
+        const float4 v = __ldg(reinterpret_cast<const float4 *>(x + j));
+        const double e0 = static_cast<double>(u.x) - v.x, e1 = static_cast<double>(u.y) - v.y;
+        const double e2 = static_cast<double>(u.z) - v.z, e3 = static_cast<double>(u.w) - v.w;
+        acc = fma(e0, e0, acc);
+        acc = fma(e1, e1, acc);
+        acc = fma(e2, e2, acc);
+        acc = fma(e3, e3, acc);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(kFull, acc, o);
+    return acc;
+}
+
+__global__ void __launch_bounds__(kQThreads) query_rerank_kernel(QueryArgs a) {
+    extern __shared__ __align__(16) unsigned char qr_raw[];
+    const int L = a.nprobe * kScrList;
+    int P2 = 1;
+    while (P2 < L) P2 <<= 1;
+    double *cd = reinterpret_cast<double *>(qr_raw);           // [P2] candidate distances
+    uint32_t *cid = reinterpret_cast<uint32_t *>(cd + P2);     // [P2] candidate ids
+    uint32_t *cpos = cid + P2;                                 // [P2] candidate positions
+    uint32_t *key = cpos + P2;                                 // [L] screened-value keys
+    __shared__ uint32_t hist[kSelBins];
+    __shared__ float s_min[kQThreads / 32], s_max[kQThreads / 32];
+    __shared__ uint32_t s_wsum[kQThreads / 32];
+    __shared__ int s_bstar, s_n, s_over, s_cbelow, s_nb;
+    __shared__ uint32_t s_tmax, s_tk;
+
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int64_t q = blockIdx.x;
+    const float *sv = a.Sv + q * L;
+    const uint32_t *sp = a.Sp + q * L;
+    const int k = a.k;
+    if (tid == 0) {
+        s_n = 0;
+        s_nb = 0;
+        s_tmax = 0u;
+        s_over = 0;
+    }
+    for (int t = tid; t < kSelBins; t += kQThreads) hist[t] = 0;
+    float lmin = INFINITY, lmax = -INFINITY;
+    for (int j = tid; j < L; j += kQThreads) {
+        const float v = sv[j];
+        key[j] = fkey(v);
+        if (v < INFINITY) {
+            lmin = fminf(lmin, v);
+            lmax = fmaxf(lmax, v);
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        lmin = fminf(lmin, __shfl_xor_sync(kFull, lmin, o));
+        lmax = fmaxf(lmax, __shfl_xor_sync(kFull, lmax, o));
+    }
+    if (lane == 0) {
+        s_min[warp] = lmin;
+        s_max[warp] = lmax;
+    }
+    __syncthreads();
+    float fmn = s_min[0], fmx = s_max[0];
+#pragma unroll
+    for (int w = 1; w < kQThreads / 32; ++w) {
+        fmn = fminf(fmn, s_min[w]);
+        fmx = fmaxf(fmx, s_max[w]);
+    }
+    const float scale = fmx > fmn ? static_cast<float>(kSelBins - 1) / (fmx - fmn) : 0.f;
+    auto bin_of = [&](uint32_t kk) -> int {
+        const float x = fkey_value(kk);
+        if (!(x < fmx)) return kSelBins - 1;
+        const int b = static_cast<int>((x - fmn) * scale);
+        return b < 0 ? 0 : (b > kSelBins - 1 ? kSelBins - 1 : b);
+    };
+    for (int j = tid; j < L; j += kQThreads) atomicAdd(&hist[bin_of(key[j])], 1u);
+    __syncthreads();
+    constexpr int kPer = kSelBins / kQThreads;
+    uint32_t h[kPer], sum = 0;
+#pragma unroll
+    for (int t = 0; t < kPer; ++t) {
+        h[t] = hist[tid * kPer + t];
+        sum += h[t];
+    }
+    uint32_t incl = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(kFull, incl, o);
+        if (lane >= o) incl += y;
+    }
+    if (lane == 31) s_wsum[warp] = incl;
+    __syncthreads();
+    {
+        uint32_t c = incl - sum;
+        for (int w = 0; w < warp; ++w) c += s_wsum[w];
+        const uint32_t need = static_cast<uint32_t>(k);
+        if (c < need && need <= c + sum) {
+#pragma unroll
+            for (int t = 0; t < kPer; ++t) {
+                if (c < need && need <= c + h[t]) {
+                    s_bstar = tid * kPer + t;
+                    s_cbelow = static_cast<int>(c);
+                }
+                c += h[t];
+            }
+        }
+    }
+    __syncthreads();
+    // T~: the k-th smallest screened value, ranked exactly among the entries of its bin
+    // (or, for a bin of more than kQRank entries, the bin's largest value: an upper bound)
+    constexpr int kQRank = 1024;
+    const int bstar = s_bstar;
+    for (int j = tid; j < L; j += kQThreads)
+        if (bin_of(key[j]) == bstar) {
+            const int at = atomicAdd(&s_nb, 1);
+            if (at < kQRank && at < P2) {  // the candidate buffers are free until later
+                cid[at] = key[j];
+                cpos[at] = static_cast<uint32_t>(j);
+            }
+            atomicMax(&s_tmax, key[j]);
+        }
+    __syncthreads();
+    const int nb = s_nb;
+    if (nb > kQRank || nb > P2) {
+        if (tid == 0) s_tk = s_tmax;
+    } else {
+        const int want = k - 1 - s_cbelow;  // 0-based rank inside the bin
+        for (int u = tid; u < nb; u += kQThreads) {
+            const uint32_t ku = cid[u], ju = cpos[u];
+            int rank = 0;
+            for (int v = 0; v < nb; ++v)
+                rank += (cid[v] < ku || (cid[v] == ku && cpos[v] < ju)) ? 1 : 0;
+            if (rank == want) s_tk = ku;
+        }
+    }
+    __syncthreads();
+    const double qn = a.qn[q];
+    const float xm2 = *a.xmax2;
+    const float E = a.ce_dot * sqrtf(static_cast<float>(qn) * xm2) +
+                    a.ce_round * (static_cast<float>(qn) + xm2);
+    const float thr = fkey_value(s_tk) + 2.f * E;  // +inf when fewer than k points exist
+    const uint32_t kthr = fkey(thr);
+    for (int t = tid; t < a.nprobe; t += kQThreads)
+        if (a.Slost[q * a.nprobe + t] < INFINITY && a.Slost[q * a.nprobe + t] <= thr) s_over = 1;
+    __syncthreads();  // the ranking's use of the candidate buffers is over
+    for (int j = tid; j < L; j += kQThreads)
+        if (key[j] <= kthr && sp[j] != 0xffffffffu) cpos[atomicAdd(&s_n, 1)] = sp[j];
+    __syncthreads();
+    if (s_over) {
+        if (tid == 0) a.fallback[q] = 1;
+        return;
+    }
+    if (tid == 0) a.fallback[q] = 0;
+    const int n = s_n;
+    const float *qv = a.Q + q * a.d;
+    for (int t = warp; t < n; t += kQThreads / 32) {
+        const uint32_t pos = cpos[t];
+        const double e = exact_sq_dist(qv, a.X + static_cast<int64_t>(pos) * a.d, a.d, lane);
+        if (lane == 0) {
+            cd[t] = e;
+            cid[t] = static_cast<uint32_t>(a.row_ids[pos]);
+        }
+    }
+    int M = 1;
+    while (M < n) M <<= 1;
+    for (int t = n + tid; t < M; t += kQThreads) {
+        cd[t] = INFINITY;
+        cid[t] = ~0u;
+    }
+    __syncthreads();
+    for (int size = 2; size <= M; size <<= 1) {
+        for (int stride = size >> 1; stride > 0; stride >>= 1) {
+            for (int t = tid; t < (M >> 1); t += kQThreads) {
+                const int lo = 2 * t - (t & (stride - 1));
+                const int hi = lo + stride;
+                const bool up = (lo & size) == 0;
+                const double da = cd[lo], db = cd[hi];
+                const uint32_t ia = cid[lo], ib = cid[hi];
+                const bool gt = da > db || (da == db && ia > ib);
+                if (gt == up) {
+                    cd[lo] = db;
+                    cd[hi] = da;
+                    cid[lo] = ib;
+                    cid[hi] = ia;
+                }
+            }
+            __syncthreads();
+        }
+    }
+    for (int t = tid; t < k; t += kQThreads) {
+        const bool real = t < n;
+        a.out_id[q * k + t] = real ? static_cast<int32_t>(cid[t]) : -1;
+        a.out_dist[q * k + t] = real ? static_cast<float>(cd[t]) : INFINITY;
+    }
+}
+
+// Queries whose pair lists may have dropped a point of their top-k: the exact k nearest
+// over every point of the probed cells.  Each lane takes a whole point (fp64, difference
+// form, in dimension order), so a warp streams 32 rows at once; each warp keeps a
+// lane-held list, and the eight lists are merged.  Rarely taken (many points whose
+// screened distances fall within 2E of one another in one cell).
+struct FallbackArgs {
+    const int32_t *fallback;
+    const int32_t *probes;
+    int nprobe, k;
+    const float *Q, *X;
+    int d;
+    const int32_t *offsets, *row_ids;
+    float *out_dist;
+    int32_t *out_id;
+};
+
+__global__ void __launch_bounds__(kQThreads) fallback_kernel(FallbackArgs a) {
+    __shared__ double s_d[kQThreads];
+    __shared__ uint32_t s_i[kQThreads];
+    const int64_t q = blockIdx.x;
+    if (a.fallback[q] == 0) return;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int k = a.k, d = a.d;
+    const float *qv = a.Q + q * d;
+    double ld = INFINITY;
+    uint32_t li = 0xffffffffu;
+    double td = INFINITY;
+    uint32_t ti = 0xffffffffu;
+    for (int t = 0; t < a.nprobe; ++t) {
+        const int cell = a.probes[q * a.nprobe + t];
+        const int e = a.offsets[cell + 1];
+        for (int p0 = a.offsets[cell] + warp * 32; p0 < e; p0 += kQThreads) {
+            const int pos = p0 + lane;
+            const bool ok = pos < e;
+            double cd = INFINITY;
+            uint32_t ci = 0xffffffffu;
+            if (ok) {
+                const float *xv = a.X + static_cast<int64_t>(pos) * d;
+                double acc = 0.0;
+                for (int j = 0; j < d; j += 4) {
+                    const float4 u = __ldg(reinterpret_cast<const float4 *>(qv + j));
+                    const float4 v = __ldg(reinterpret_cast<const float4 *>(xv + j));
+                    const double e0 = static_cast<double>(u.x) - v.x;
+                    const double e1 = static_cast<double>(u.y) - v.y;
+                    const double e2 = static_cast<double>(u.z) - v.z;
+                    const double e3 = static_cast<double>(u.w) - v.w;
+                    acc = fma(e0, e0, acc);
+                    acc = fma(e1, e1, acc);
+                    acc = fma(e2, e2, acc);
+                    acc = fma(e3, e3, acc);
+                }
+                cd = acc;
+                ci = static_cast<uint32_t>(a.row_ids[pos]);
+            }
+            bool pend = ok && before(cd, ci, td, ti);
+            unsigned m = __ballot_sync(kFull, pend);
+            while (m) {
+                const int src = __ffs(m) - 1;
+                const double xd = __shfl_sync(kFull, cd, src);
+                const uint32_t xi = __shfl_sync(kFull, ci, src);
+                const int at = __popc(__ballot_sync(kFull, lane < k && before(ld, li, xd, xi)));
+                const double ud = __shfl_up_sync(kFull, ld, 1);
+                const uint32_t ui = __shfl_up_sync(kFull, li, 1);
+                if (lane == at) {
+                    ld = xd;
+                    li = xi;
+                } else if (lane > at && lane < k) {
+                    ld = ud;
+                    li = ui;
+                }
+                td = __shfl_sync(kFull, ld, k - 1);
+                ti = __shfl_sync(kFull, li, k - 1);
+                if (lane == src) pend = false;
+                pend = pend && before(cd, ci, td, ti);
+                m = __ballot_sync(kFull, pend);
+            }
+        }
+    }
+    s_d[tid] = lane < k ? ld : INFINITY;
+    s_i[tid] = lane < k ? li : 0xffffffffu;
+    __syncthreads();
+    for (int size = 2; size <= kQThreads; size <<= 1) {
+        for (int stride = size >> 1; stride > 0; stride >>= 1) {
+            for (int t = tid; t < kQThreads / 2; t += kQThreads) {
+                const int lo = 2 * t - (t & (stride - 1));
+                const int hi = lo + stride;
+                const bool up = (lo & size) == 0;
+                const double da = s_d[lo], db = s_d[hi];
+                const uint32_t ia = s_i[lo], ib = s_i[hi];
+                const bool gt = da > db || (da == db && ia > ib);
+                if (gt == up) {
+                    s_d[lo] = db;
+                    s_d[hi] = da;
+                    s_i[lo] = ib;
+                    s_i[hi] = ia;
+                }
+            }
+            __syncthreads();
+        }
+    }
+    for (int t = tid; t < k; t += kQThreads) {
+        const bool real = s_i[t] != 0xffffffffu;
+        a.out_id[q * k + t] = real ? static_cast<int32_t>(s_i[t]) : -1;
+        a.out_dist[q * k + t] = real ? static_cast<float>(s_d[t]) : INFINITY;
+    }
+}
+
+// Number of flagged queries (one block), for the caller's diagnostics.
+__global__ void count_flags_kernel(const int32_t *__restrict__ f, int64_t n, int *__restrict__ out) {
+    __shared__ int red[32];
+    int c = 0;
+    for (int64_t i = threadIdx.x; i < n; i += blockDim.x) c += f[i] != 0;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(kFull, c, o);
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = c;
+    __syncthreads();
+    if (threadIdx.x < 32) {
+        c = threadIdx.x < (blockDim.x >> 5) ? red[threadIdx.x] : 0;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(kFull, c, o);
+        if (threadIdx.x == 0) *out = c;
+    }
+}
+
+// max_i ||x_i||^2 of fp64 norms, rounded up to fp32 (one block).
+__global__ void max_norm_kernel(const double *__restrict__ xn, int64_t n, float *__restrict__ out) {
+    __shared__ double red[32];
+    double mx = 0.0;
+    for (int64_t i = threadIdx.x; i < n; i += blockDim.x) mx = fmax(mx, xn[i]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mx = fmax(mx, __shfl_xor_sync(kFull, mx, o));
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = mx;
+    __syncthreads();
+    if (threadIdx.x < 32) {
+        mx = threadIdx.x < (blockDim.x >> 5) ? red[threadIdx.x] : 0.0;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) mx = fmax(mx, __shfl_xor_sync(kFull, mx, o));
+        if (threadIdx.x == 0) *out = __double2float_ru(mx);
+    }
+}
+
 // ---------------------------------------------------------------- small kernels
 // ||v||^2 in fp64, a warp per row: lane partial sums over float4 columns, then a fixed
 // butterfly.
@@ -999,6 +1638,106 @@ cudaError_t launch_ivf_coarse_rerank(const float *Vs, int64_t ldv, int64_t rows,
         attr = true;
     }
     coarse_rerank_kernel<<<static_cast<unsigned>(rows), kCoarseThreads, smem, st>>>(a);
+    note_launch();
+    return cudaGetLastError();
+}
+
+cudaError_t launch_ivf_fine_scr(const uint16_t *Qp, int64_t nq, const uint16_t *Xp, int64_t N,
+                                int dp, const double *qn, const double *xn,
+                                const int32_t *offsets, const int32_t *pair_sorted,
+                                const int32_t *pair_off, const int2 *items, const int *nitems,
+                                int *item_ctr, int64_t max_items, int nprobe, float *Sv,
+                                uint32_t *Sp, float *Slost, cudaStream_t st) {
+    FineArgs a{Qp, nq, Xp, N, dp, qn, xn, offsets, pair_sorted, pair_off, items, nitems,
+               item_ctr, nprobe, Sv, Sp, Slost};
+    static int occ = 0;
+    if (occ == 0) {
+        cudaFuncSetAttribute(ivf_fine_scr_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(sizeof(FineSmem)));
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, ivf_fine_scr_kernel, kTThreads,
+                                                          sizeof(FineSmem)) != cudaSuccess ||
+            occ < 1)
+            occ = 1;
+    }
+    int64_t grid = static_cast<int64_t>(device_sm_count()) * occ;
+    if (grid > max_items) grid = max_items;
+    if (grid < 1) grid = 1;
+    ivf_fine_scr_kernel<<<static_cast<unsigned>(grid), kTThreads, sizeof(FineSmem), st>>>(a);
+    note_launch();
+    return cudaGetLastError();
+}
+
+// Window coefficients of the screened fine pass for rows padded to dp: with u = 2^-8 (bf16
+// rounding), the three products miss at most 3.1 u^2 sum |q_j||x_j| <= 3.1 u^2 |q||x|; the
+// 3 dp / 16 mma steps add at most 17 units of 2^-23 of a partial sum bounded by
+// 1.02 |q||x| each; the factor 2 of -2 q.x; the fp32 rounding of s~ at most 2^-23
+// (||q||^2 + ||x||^2); a 1% margin on both.
+void fine_window_coeffs(int dp, float *ce_dot, float *ce_round) {
+    const double u = 1.0 / 256.0;
+    const double e_dot = 3.1 * u * u + 3.0 * (dp / 16) * 17.0 * std::ldexp(1.0, -23) * 1.02;
+    *ce_dot = static_cast<float>(2.0 * e_dot * 1.01);
+    *ce_round = static_cast<float>(std::ldexp(1.0, -23) * 1.01);
+}
+
+cudaError_t launch_ivf_query_rerank(const float *Sv, const uint32_t *Sp, const float *Slost,
+                                    int64_t nq, int nprobe, int k, const float *Q,
+                                    const float *X, int d, int dp, const double *qn,
+                                    const float *xmax2, const int32_t *row_ids,
+                                    float *out_dist, int32_t *out_id, int32_t *fallback,
+                                    cudaStream_t st) {
+    if (nq <= 0) return cudaSuccess;
+    QueryArgs a{};
+    a.Sv = Sv;
+    a.Sp = Sp;
+    a.Slost = Slost;
+    a.nprobe = nprobe;
+    a.k = k;
+    a.Q = Q;
+    a.X = X;
+    a.d = d;
+    a.qn = qn;
+    a.xmax2 = xmax2;
+    fine_window_coeffs(dp, &a.ce_dot, &a.ce_round);
+    a.row_ids = row_ids;
+    a.out_dist = out_dist;
+    a.out_id = out_id;
+    a.fallback = fallback;
+    const int L = nprobe * kScrList;
+    int P2 = 1;
+    while (P2 < L) P2 <<= 1;
+    const size_t smem = static_cast<size_t>(P2) * (sizeof(double) + 2 * sizeof(uint32_t)) +
+                        static_cast<size_t>(L) * sizeof(uint32_t);
+    static bool attr = false;
+    if (!attr) {
+        cudaFuncSetAttribute(query_rerank_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(kSearchScrMaxProbe * kScrList *
+                                              (sizeof(double) + 3 * sizeof(uint32_t))));
+        attr = true;
+    }
+    query_rerank_kernel<<<static_cast<unsigned>(nq), kQThreads, smem, st>>>(a);
+    note_launch();
+    return cudaGetLastError();
+}
+
+cudaError_t launch_ivf_fallback(const int32_t *fallback, const int32_t *probes, int64_t nq,
+                                int nprobe, int k, const float *Q, const float *X, int d,
+                                const int32_t *offsets, const int32_t *row_ids, float *out_dist,
+                                int32_t *out_id, cudaStream_t st) {
+    if (nq <= 0) return cudaSuccess;
+    FallbackArgs a{fallback, probes, nprobe, k, Q, X, d, offsets, row_ids, out_dist, out_id};
+    fallback_kernel<<<static_cast<unsigned>(nq), kQThreads, 0, st>>>(a);
+    note_launch();
+    return cudaGetLastError();
+}
+
+cudaError_t launch_count_flags(const int32_t *f, int64_t n, int *out, cudaStream_t st) {
+    count_flags_kernel<<<1, 1024, 0, st>>>(f, n, out);
+    note_launch();
+    return cudaGetLastError();
+}
+
+cudaError_t launch_max_norm(const double *xn, int64_t n, float *out, cudaStream_t st) {
+    max_norm_kernel<<<1, 1024, 0, st>>>(xn, n, out);
     note_launch();
     return cudaGetLastError();
 }

@@ -43,10 +43,11 @@ class FkTiming(ctypes.Structure):
 class FkSearchTiming(ctypes.Structure):
     _fields_ = [("ms_coarse", ctypes.c_double), ("ms_sort", ctypes.c_double),
                 ("ms_fine", ctypes.c_double), ("ms_merge", ctypes.c_double),
-                ("screened_coarse", ctypes.c_int)]
+                ("screened_coarse", ctypes.c_int), ("screened_fine", ctypes.c_int),
+                ("fallback_queries", ctypes.c_int)]
 
 
-FK_SEARCH_FP64_COARSE = 1
+FK_SEARCH_FP64_COARSE, FK_SEARCH_FP64_FINE = 1, 2
 
 
 def _sig(name, args, res=ctypes.c_int):
@@ -81,8 +82,8 @@ _sig("fk_lloyd_streamed", [_vp, _int, _i64, _int, _int, _int, _int, _vp, _vp,
 _sig("fk_streamed_workspace_size", [_i64, _int, _int, _int, _int, ctypes.POINTER(_sz)])
 _sig("fk_ivf_norms", [_vp, _i64, _int, _vp, _vp])
 _sig("fk_ivf_search_workspace_size", [_i64, _int, _int, _i64, _int, _int, ctypes.POINTER(_sz)])
-_sig("fk_ivf_search", [_vp, _i64, _int, _vp, _int, _vp, _vp, _vp, _vp, _i64, _int, _int, _int,
-                       _vp, _vp, _vp, _vp, _sz, ctypes.POINTER(FkSearchTiming), _vp])
+_sig("fk_ivf_search", [_vp, _i64, _int, _vp, _int, _vp, _vp, _vp, _vp, _vp, _i64, _int, _int,
+                       _int, _vp, _vp, _vp, _vp, _sz, ctypes.POINTER(FkSearchTiming), _vp])
 
 EXPORTED = ["fk_status_string", "fk_version", "fk_workspace_size", "fk_normalize_rows",
             "fk_centroid_norms", "fk_assign", "fk_update", "fk_lloyd",
@@ -418,11 +419,14 @@ def fk_ivf_search(Q: torch.Tensor, C: torch.Tensor, X_lists: torch.Tensor,
                   nprobe: int, k: int, ws: torch.Tensor | None = None,
                   distances: torch.Tensor | None = None, ids: torch.Tensor | None = None,
                   probes: torch.Tensor | None = None, timing: dict | None = None,
-                  fp64_coarse: bool = False, stream=None):
+                  fp64_coarse: bool = False, X_planes=None, fp64_fine: bool = False,
+                  stream=None):
     """IVF-Flat search: returns (distances fp32 [nq, k], ids int32 [nq, k]); `probes`
     (int32 [nq, nprobe]) receives the probed cells when given.  A `timing` dict receives
     the per-phase device times in ms (the call then synchronises its stream).
-    fp64_coarse computes every coarse distance in fp64 (FK_SEARCH_FP64_COARSE)."""
+    X_planes: fk_split_points of X_lists (a SplitPoints or its buffer), which enables the
+    tensor-core fine pass.  fp64_coarse / fp64_fine compute every coarse / fine distance
+    in fp64 (FK_SEARCH_FP64_COARSE / FK_SEARCH_FP64_FINE)."""
     nq, d = Q.shape
     nlist = C.shape[0]
     N = X_lists.shape[0]
@@ -433,13 +437,21 @@ def fk_ivf_search(Q: torch.Tensor, C: torch.Tensor, X_lists: torch.Tensor,
     if ids is None:
         ids = torch.empty((nq, k), dtype=torch.int32, device=Q.device)
     tm = FkSearchTiming() if timing is not None else None
+    if isinstance(X_planes, SplitPoints):
+        if X_planes.N != N or X_planes.d != d:
+            raise ValueError("X_planes must split X_lists")
+        X_planes = X_planes.buf
+    dp = (d + 63) // 64 * 64
+    planes_ptr = _opt(X_planes, "X_planes", torch.bfloat16, (2 * N * dp + 2 * N,))
+    flags = (FK_SEARCH_FP64_COARSE if fp64_coarse else 0) | \
+        (FK_SEARCH_FP64_FINE if fp64_fine else 0)
     _check(_lib.fk_ivf_search(_dev(Q, "Q", torch.float32), nq, d,
                               _dev(C, "C", torch.float32, (nlist, d)), nlist,
                               _dev(X_lists, "X_lists", torch.float32, (N, d)),
-                              _dev(X_norms, "X_norms", torch.float64, (N,)),
+                              _dev(X_norms, "X_norms", torch.float64, (N,)), planes_ptr,
                               _dev(offsets, "offsets", torch.int32, (nlist + 1,)),
                               _dev(row_ids, "row_ids", torch.int32, (N,)), N, nprobe, k,
-                              FK_SEARCH_FP64_COARSE if fp64_coarse else 0,
+                              flags,
                               _dev(distances, "distances", torch.float32, (nq, k)),
                               _dev(ids, "ids", torch.int32, (nq, k)),
                               _opt(probes, "probes", torch.int32, (nq, nprobe)),
@@ -453,12 +465,14 @@ def fk_ivf_search(Q: torch.Tensor, C: torch.Tensor, X_lists: torch.Tensor,
 
 class IvfFlatIndex:
     """An IVF-Flat index: centroids, cell-contiguous points with their original ids, CSR
-    offsets and fp64 norms.  `build` and `search` only sequence libfk calls
-    (fk_normalize_rows, fk_lloyd, fk_ivf_lists, fk_ivf_norms, fk_ivf_search)."""
+    offsets, fp64 norms and the bf16 planes of the points (for the tensor-core fine pass).
+    `build` and `search` only sequence libfk calls (fk_normalize_rows, fk_lloyd,
+    fk_ivf_lists, fk_ivf_norms, fk_split_points, fk_ivf_search)."""
 
-    def __init__(self, C, X_lists, X_norms, offsets, row_ids, metric="l2"):
+    def __init__(self, C, X_lists, X_norms, offsets, row_ids, metric="l2", X_planes=None):
         self.C, self.X_lists, self.X_norms = C, X_lists, X_norms
         self.offsets, self.row_ids, self.metric = offsets, row_ids, metric
+        self.X_planes = X_planes
 
     @classmethod
     def build(cls, X: torch.Tensor, C0: torch.Tensor, niter: int, metric="l2", stream=None):
@@ -481,10 +495,12 @@ class IvfFlatIndex:
         fk_ivf_lists(X, labels, K, offsets, row_ids, ws, X_lists, stream)
         del ws
         X_norms = fk_ivf_norms(X_lists, stream=stream)
-        return cls(C, X_lists, X_norms, offsets, row_ids, metric)
+        X_planes = fk_split_points(X_lists, stream=stream)
+        return cls(C, X_lists, X_norms, offsets, row_ids, metric, X_planes)
 
     def search(self, Q: torch.Tensor, k: int, nprobe: int, ws=None, distances=None,
-               ids=None, probes=None, timing=None, fp64_coarse=False, stream=None):
+               ids=None, probes=None, timing=None, fp64_coarse=False, fp64_fine=False,
+               stream=None):
         """(distances, ids) of the k nearest indexed points of every query, probing nprobe
         cells; a cosine index L2-normalises the queries first."""
         if self.metric == "cosine":
@@ -494,4 +510,4 @@ class IvfFlatIndex:
         return fk_ivf_search(Q, self.C, self.X_lists, self.X_norms, self.offsets,
                              self.row_ids, nprobe, k, ws=ws, distances=distances, ids=ids,
                              probes=probes, timing=timing, fp64_coarse=fp64_coarse,
-                             stream=stream)
+                             X_planes=self.X_planes, fp64_fine=fp64_fine, stream=stream)

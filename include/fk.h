@@ -294,10 +294,18 @@ FK_API fk_status fk_ivf_search_workspace_size(int64_t nq, int d, int nlist, int6
  * of the nprobe-th screened value is then re-ranked in fp64 (difference form), so the
  * probes are those of the fp64 evaluation.  FK_SEARCH_FP64_COARSE computes every coarse
  * distance in fp64 instead (same probes, more work).
+ * Fine pass: with X_planes given (fk_split_points of X_lists), k <= 16 and nprobe <= 256,
+ * each (query, point) product is screened on the tensor cores (three bf16 products, fp32
+ * accumulation); per query, the points within a proven window of the k-th screened
+ * distance are re-ranked in fp64 (difference form), and a query whose per-cell candidate
+ * lists may have dropped one is recomputed exactly over its probed cells.  Otherwise, or
+ * with FK_SEARCH_FP64_FINE, every fine distance is fp64.
  *
  * Inputs (device pointers, read only): Q nq x d fp32; C nlist x d fp32 centroids; X_lists
  * N x d fp32, the points in cell order (fk_ivf_lists); X_norms N doubles, fk_ivf_norms of
- * X_lists; offsets nlist + 1 int32 (offsets[0] = 0, offsets[nlist] = N, non-decreasing);
+ * X_lists; X_planes NULL or the 4 N d_p + 4 N bytes that fk_split_points writes for
+ * X_lists (16-byte aligned); offsets nlist + 1 int32 (offsets[0] = 0, offsets[nlist] = N,
+ * non-decreasing);
  * row_ids N int32 (fk_ivf_lists).  Outputs (device): distances nq x k fp32, ids nq x k
  * int32, probes nq x nprobe int32 or NULL (then kept in the workspace).
  * Requirements: d % 4 == 0; Q, C, X_lists 16-byte aligned; 1 <= nprobe <= min(nlist,
@@ -310,18 +318,23 @@ FK_API fk_status fk_ivf_search_workspace_size(int64_t nq, int d, int nlist, int6
 typedef struct fk_search_timing {
     double ms_coarse; /* query and centroid norms, coarse distances, probe selection */
     double ms_sort;   /* (query, probe) pairs sorted by cell, work items */
-    double ms_fine;   /* the fine distance kernel (per-pair k nearest) */
-    double ms_merge;  /* the per-query selection of the k nearest */
+    double ms_fine;   /* the fine distance kernel (per-pair candidate lists) */
+    double ms_merge;  /* the per-query selection (and exact re-ranking) of the k nearest */
     int screened_coarse; /* 1 when the coarse pass ran on the tensor cores (see flags) */
+    int screened_fine;   /* 1 when the fine pass ran on the tensor cores (see flags)   */
+    int fallback_queries; /* screened fine pass: queries recomputed exactly over their
+                             probed cells (their candidate lists may have dropped a point) */
 } fk_search_timing;
 
 /* fk_ivf_search flags. */
 #define FK_SEARCH_FP64_COARSE 1 /* every coarse distance in fp64 (no tensor-core screening) */
+#define FK_SEARCH_FP64_FINE 2   /* every fine distance in fp64 (no tensor-core screening)   */
 
 FK_API fk_status fk_ivf_search(const float *Q, int64_t nq, int d, const float *C, int nlist,
                                const float *X_lists, const double *X_norms,
-                               const int32_t *offsets, const int32_t *row_ids, int64_t N,
-                               int nprobe, int k, int flags, float *distances, int32_t *ids,
+                               const void *X_planes, const int32_t *offsets,
+                               const int32_t *row_ids, int64_t N, int nprobe, int k,
+                               int flags, float *distances, int32_t *ids,
                                int32_t *probes, void *ws, size_t ws_bytes,
                                fk_search_timing *timing, fk_stream_t stream);
 

@@ -37,19 +37,22 @@ def _index(X, labels, nlist):
     m.fk_ivf_lists(Xg, torch.as_tensor(labels).to(DEV), nlist, offsets, row_ids, ws,
                    X_lists=X_lists)
     assert m.fk_get_device_error(ws) == m.FK_OK
-    return X_lists, m.fk_ivf_norms(X_lists), offsets, row_ids
+    return X_lists, m.fk_ivf_norms(X_lists), offsets, row_ids, m.fk_split_points(X_lists)
 
 
-def _search(Q, C, idx, nprobe, k, fp64_coarse=False, timing=None):
+def _search(Q, C, idx, nprobe, k, fp64_coarse=False, fp64_fine=False, timing=None):
     m = fk()
-    X_lists, X_norms, offsets, row_ids = idx
+    X_lists, X_norms, offsets, row_ids, planes = idx
     nq = Q.shape[0]
     probes = torch.full((nq, nprobe), -7, dtype=torch.int32, device=DEV)
     dist, ids = m.fk_ivf_search(Q.to(DEV), C.to(DEV), X_lists, X_norms, offsets, row_ids,
                                 nprobe, k, probes=probes, fp64_coarse=fp64_coarse,
-                                timing=timing)
+                                X_planes=planes, fp64_fine=fp64_fine, timing=timing)
     torch.cuda.synchronize()
     return probes.cpu().numpy(), ids.cpu().numpy(), dist.cpu().numpy()
+
+
+MODES = [(False, False), (True, False), (False, True), (True, True)]  # fp64 coarse, fp64 fine
 
 
 def _sqd(A, B):
@@ -99,9 +102,8 @@ CASES = [
 ]
 
 
-@pytest.mark.parametrize("coarse", ["screened", "fp64"])
 @pytest.mark.parametrize("N,d,nlist,nq,nprobe,k,weights,labels_from", CASES)
-def test_ivf_search_matches_oracle(N, d, nlist, nq, nprobe, k, weights, labels_from, coarse):
+def test_ivf_search_matches_oracle(N, d, nlist, nq, nprobe, k, weights, labels_from):
     X, comp, _ = gaussian_mixture(N, d, nlist, centers="normal", sigma=0.4, weights=weights,
                                   seed=N + d)
     C = X[init_indices(N, nlist, N + d)].float().contiguous()
@@ -111,12 +113,14 @@ def test_ivf_search_matches_oracle(N, d, nlist, nq, nprobe, k, weights, labels_f
         labels = comp.numpy().astype(np.int32)
     Q = mixture_queries(nq, d, nlist, centers="normal", sigma=0.4, weights=weights,
                         seed=N + d, stream=1)
-    tm = {}
-    got = _search(Q, C, _index(X, labels, nlist), nprobe, k, fp64_coarse=coarse == "fp64",
-                  timing=tm)
-    assert tm["screened_coarse"] == (1 if coarse == "screened" else 0)
     ref = oracle.ivf_search(Q, C, X, labels, nprobe, k)
-    check_search(Q, C, X, got, ref)
+    idx = _index(X, labels, nlist)
+    for f64c, f64f in MODES:
+        tm = {}
+        got = _search(Q, C, idx, nprobe, k, fp64_coarse=f64c, fp64_fine=f64f, timing=tm)
+        assert tm["screened_coarse"] == (0 if f64c else 1)
+        assert tm["screened_fine"] == (0 if (f64f or k > 16) else 1)
+        check_search(Q, C, X, got, ref)
 
 
 def test_ivf_search_empty_cells_and_few_candidates():
@@ -132,8 +136,9 @@ def test_ivf_search_empty_cells_and_few_candidates():
     for nprobe, k in ((1, 32), (3, 32), (nlist, 8)):
         ref = oracle.ivf_search(Q, C, X, labels, nprobe, k)
         assert (ref[1] == -1).any() or nprobe == nlist
-        for f64 in (False, True):
-            got = _search(Q, C, _index(X, labels, nlist), nprobe, k, fp64_coarse=f64)
+        idx = _index(X, labels, nlist)
+        for f64c, f64f in MODES:
+            got = _search(Q, C, idx, nprobe, k, fp64_coarse=f64c, fp64_fine=f64f)
             check_search(Q, C, X, got, ref, max_bad_frac=0.0)
 
 
@@ -147,12 +152,14 @@ def test_ivf_search_duplicates_and_self_queries():
     labels, _, _ = oracle.assign(X, C)
     sel = np.r_[np.arange(100, 140), np.arange(4000, 4030)]
     Q = X[sel].clone()
-    got = _search(Q, C, _index(X, labels, K), 2, 6)
     ref = oracle.ivf_search(Q, C, X, labels, 2, 6)
-    check_search(Q, C, X, got, ref, max_bad_frac=0.0)
-    ids = got[1]
-    assert (ids[:, 0] == sel).all()
-    assert (ids[:40, 1] == sel[:40] + N // 2 - 100).all()   # the duplicate, second
+    idx = _index(X, labels, K)
+    for f64c, f64f in MODES:
+        got = _search(Q, C, idx, 2, 6, fp64_coarse=f64c, fp64_fine=f64f)
+        check_search(Q, C, X, got, ref, max_bad_frac=0.0)
+        ids = got[1]
+        assert (ids[:, 0] == sel).all()
+        assert (ids[:40, 1] == sel[:40] + N // 2 - 100).all()   # the duplicate, second
 
 
 def test_ivf_search_built_index_exhaustive_is_exact_knn():
@@ -208,11 +215,11 @@ def test_ivf_search_argument_errors():
     Q = X[:5].to(DEV)
     for nprobe, k in ((K + 1, 3), (0, 3), (2, 0), (2, 33)):
         with pytest.raises(m.FkError) as e:
-            m.fk_ivf_search(Q, C, *idx, nprobe, k)
+            m.fk_ivf_search(Q, C, *idx[:4], nprobe, k)
         assert e.value.status == m.FK_ERR_INVALID_ARG
     ws = m.ivf_search_workspace(5, d, K, N, 2, 3)
     with pytest.raises(m.FkError) as e:
-        m.fk_ivf_search(Q, C, *idx, 2, 3, ws=ws[:1024])
+        m.fk_ivf_search(Q, C, *idx[:4], 2, 3, ws=ws[:1024])
     assert e.value.status == m.FK_ERR_WORKSPACE
 
 
@@ -225,10 +232,11 @@ def test_ivf_search_equal_centroid_distances():
     C = X[:1].expand(nlist, d).contiguous()
     labels = (np.arange(N) % nlist).astype(np.int32)
     Q = mixture_queries(40, d, 10, sigma=0.3, seed=21, stream=1)
+    idx = _index(X, labels, nlist)
     for nprobe, k in ((5, 4), (700, 32)):
         ref = oracle.ivf_search(Q, C, X, labels, nprobe, k)
         for f64 in (False, True):
-            got = _search(Q, C, _index(X, labels, nlist), nprobe, k, fp64_coarse=f64)
+            got = _search(Q, C, idx, nprobe, k, fp64_coarse=f64)
             assert (got[0] == np.arange(nprobe)).all()
             check_search(Q, C, X, got, ref, max_bad_frac=0.0)
 
@@ -256,3 +264,24 @@ def test_ivf_search_coarse_paths_agree_and_large_nlist_uses_fp64():
     lab = torch.randint(0, 9000, (N,), generator=torch.Generator().manual_seed(3)).numpy()
     _search(Q[:50], Cbig, _index(Xn, lab.astype(np.int32), 9000), 4, 5, timing=tm)
     assert tm["screened_coarse"] == 0
+
+
+def test_ivf_search_screened_fine_fallback_on_tied_candidates():
+    """100 copies of one point in a cell tie at every query, so a pair list (32 entries)
+    drops copies inside the re-ranking window and the query is recomputed exactly: the
+    lowest original indices of the copies come first, as in the oracle."""
+    N, d, K = 5000, 64, 20
+    X, comp, _ = gaussian_mixture(N, d, K, centers="normal", sigma=0.3, seed=29)
+    dup = np.arange(1000, 1100)
+    X[dup] = X[7].clone()
+    C = X[init_indices(N, K, 29)].float().contiguous()
+    labels, _, _ = oracle.assign(X, C)
+    Q = torch.cat([X[7:8] + 0.01, mixture_queries(30, d, K, sigma=0.3, seed=29, stream=1)])
+    idx = _index(X, labels, K)
+    for k in (10, 16):
+        ref = oracle.ivf_search(Q, C, X, labels, 3, k)
+        tm = {}
+        got = _search(Q, C, idx, 3, k, timing=tm)
+        assert tm["screened_fine"] == 1 and tm["fallback_queries"] >= 1
+        check_search(Q, C, X, got, ref, max_bad_frac=0.0)
+        assert (got[1][0] == np.r_[7, dup][:k]).all()
