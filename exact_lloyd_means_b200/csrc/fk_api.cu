@@ -259,7 +259,7 @@ fk_status validate_search(int64_t nq, int d, int nlist, int64_t N, int nprobe, i
 
 fk_status run_ivf_search(const float *Q, int64_t nq, int d, const float *C, int nlist,
                          const float *X_lists, const double *X_norms, const void *X_planes,
-                         const int32_t *offsets, const int32_t *row_ids, int64_t N, int nprobe,
+                         const float *cell_radius, const int32_t *offsets, const int32_t *row_ids, int64_t N, int nprobe,
                          int k, bool screen, bool screen_fine, float *distances, int32_t *ids,
                          int32_t *probes, void *ws, const SearchLayout &L, cudaStream_t st,
                          const cudaEvent_t *ev) {
@@ -339,14 +339,18 @@ fk_status run_ivf_search(const float *Q, int64_t nq, int d, const float *C, int 
         int32_t *fb = ws_ptr<int32_t>(ws, L.fb);
         float *xmax2 = ws_ptr<float>(ws, L.xmax2);
         const uint16_t *Xp = static_cast<const uint16_t *>(X_planes);
+        float *cut = cell_radius ? ws_ptr<float>(ws, L.ubound) : nullptr;
+        FK_TRY_CUDA(launch_max_norm(X_norms, N, xmax2, st));
+        if (cut)
+            FK_TRY_CUDA(launch_query_cut(Q, C, pr, offsets, cell_radius, qn, xmax2,
+                                         static_cast<int>(L.dp), nq, nprobe, k, d, cut, st));
         FK_TRY_CUDA(launch_ivf_fine_scr(qh, nq, Xp, N, static_cast<int>(L.dp), qn, X_norms,
                                         offsets, psorted, poff, items, nitems, nitems + 1,
-                                        L.max_items, nprobe, Sv, Sp, Slost, st));
+                                        L.max_items, nprobe, Sv, Sp, Slost, cut, st));
         if (!mark(3)) return FK_ERR_CUDA;
-        FK_TRY_CUDA(launch_max_norm(X_norms, N, xmax2, st));
         FK_TRY_CUDA(launch_ivf_query_rerank(Sv, Sp, Slost, nq, nprobe, k, Q, X_lists, d,
                                             static_cast<int>(L.dp), qn, xmax2, row_ids,
-                                            distances, ids, fb, st));
+                                            distances, ids, fb, cut, st));
         FK_TRY_CUDA(launch_ivf_fallback(fb, pr, nq, nprobe, k, Q, X_lists, d, offsets, row_ids,
                                         distances, ids, st));
     } else {
@@ -914,6 +918,18 @@ fk_status fk_ivf_norms(const float *V, int64_t n, int d, double *norms, fk_strea
 }
 
 
+fk_status fk_ivf_radii(const float *C, int nlist, const float *X_lists, const int32_t *offsets,
+                       int d, float *radius, fk_stream_t stream) {
+    if (!C || !X_lists || !offsets || !radius || nlist < 1 || d < 1) return FK_ERR_INVALID_ARG;
+    if (d % 4 != 0 || !aligned(C, 16) || !aligned(X_lists, 16) || !aligned(offsets, 4) ||
+        !aligned(radius, 4))
+        return FK_ERR_UNSUPPORTED;
+    fk_status s = check_device();
+    if (s != FK_OK) return s;
+    FK_TRY_CUDA(launch_cell_radius(C, nlist, X_lists, offsets, d, radius, stream));
+    return FK_OK;
+}
+
 fk_status fk_ivf_search_workspace_size(int64_t nq, int d, int nlist, int64_t N, int nprobe,
                                        int k, size_t *bytes) {
     if (!bytes) return FK_ERR_INVALID_ARG;
@@ -925,7 +941,7 @@ fk_status fk_ivf_search_workspace_size(int64_t nq, int d, int nlist, int64_t N, 
 
 fk_status fk_ivf_search(const float *Q, int64_t nq, int d, const float *C, int nlist,
                         const float *X_lists, const double *X_norms, const void *X_planes,
-                        const int32_t *offsets, const int32_t *row_ids, int64_t N, int nprobe,
+                        const float *cell_radius, const int32_t *offsets, const int32_t *row_ids, int64_t N, int nprobe,
                         int k, int flags,
                         float *distances, int32_t *ids, int32_t *probes, void *ws,
                         size_t ws_bytes, fk_search_timing *timing, fk_stream_t stream) {
@@ -936,7 +952,7 @@ fk_status fk_ivf_search(const float *Q, int64_t nq, int d, const float *C, int n
     if (!aligned(Q, 16) || !aligned(C, 16) || !aligned(X_lists, 16) || !aligned(X_norms, 8) ||
         !aligned(offsets, 4) || !aligned(row_ids, 4) || !aligned(distances, 4) ||
         !aligned(ids, 4) || (probes && !aligned(probes, 4)) ||
-        (X_planes && !aligned(X_planes, 16)))
+        (X_planes && !aligned(X_planes, 16)) || (cell_radius && !aligned(cell_radius, 4)))
         return FK_ERR_UNSUPPORTED;
     const SearchLayout L = search_layout(nq, d, nlist, nprobe, k);
     if (ws == nullptr || !aligned(ws, 256) || ws_bytes < L.total) return FK_ERR_WORKSPACE;
@@ -959,9 +975,10 @@ fk_status fk_ivf_search(const float *Q, int64_t nq, int d, const float *C, int n
                                               static_cast<int>(L.Kp));
     const bool screen_fine = X_planes != nullptr && (flags & FK_SEARCH_FP64_FINE) == 0 &&
                              k <= kSearchScrMaxK && nprobe <= kSearchScrMaxProbe;
-    const fk_status r = run_ivf_search(Q, nq, d, C, nlist, X_lists, X_norms, X_planes, offsets,
-                                       row_ids, N, nprobe, k, screen, screen_fine, distances,
-                                       ids, probes, ws, L, st, timing ? ev : nullptr);
+    const fk_status r = run_ivf_search(Q, nq, d, C, nlist, X_lists, X_norms, X_planes,
+                                       cell_radius, offsets, row_ids, N, nprobe, k, screen,
+                                       screen_fine, distances, ids, probes, ws, L, st,
+                                       timing ? ev : nullptr);
     if (r == FK_OK && timing) {
         int nfb = 0;
         if (screen_fine) {  // the flagged-query count sits in the word after the max norm

@@ -329,19 +329,26 @@ cudaError_t launch_ivf_fine_scr(const uint16_t *Qp, int64_t nq, const uint16_t *
                                 const int32_t *offsets, const int32_t *pair_sorted,
                                 const int32_t *pair_off, const int2 *items, const int *nitems,
                                 int *item_ctr, int64_t max_items, int nprobe, float *Sv,
-                                uint32_t *Sp, float *Slost, cudaStream_t st);
+                                uint32_t *Sp, float *Slost, const float *cut, cudaStream_t st);
 cudaError_t launch_ivf_query_rerank(const float *Sv, const uint32_t *Sp, const float *Slost,
                                     int64_t nq, int nprobe, int k, const float *Q,
                                     const float *X, int d, int dp, const double *qn,
                                     const float *xmax2, const int32_t *row_ids,
                                     float *out_dist, int32_t *out_id, int32_t *fallback,
-                                    cudaStream_t st);
+                                    const float *cut, cudaStream_t st);
 cudaError_t launch_ivf_fallback(const int32_t *fallback, const int32_t *probes, int64_t nq,
                                 int nprobe, int k, const float *Q, const float *X, int d,
                                 const int32_t *offsets, const int32_t *row_ids, float *out_dist,
                                 int32_t *out_id, cudaStream_t st);
 cudaError_t launch_max_norm(const double *xn, int64_t n, float *out, cudaStream_t st);
 cudaError_t launch_count_flags(const int32_t *f, int64_t n, int *out, cudaStream_t st);
+// Cell radii of an index, and per query a cut on the fine pass's screened distances.
+cudaError_t launch_cell_radius(const float *C, int nlist, const float *X, const int32_t *offsets,
+                               int d, float *radius, cudaStream_t st);
+cudaError_t launch_query_cut(const float *Q, const float *C, const int32_t *probes,
+                             const int32_t *offsets, const float *radius, const double *qn,
+                             const float *xmax2, int dp, int64_t nq, int nprobe, int k, int d,
+                             float *cut, cudaStream_t st);
 
 // Limits of fk_ivf_search: k is held one rank per lane, nprobe by the selection's sort.
 constexpr int kSearchMaxK = 32;
@@ -359,7 +366,7 @@ struct SearchLayout {
     size_t err = 0, qn = 0, cn = 0, D = 0, probes = 0, keys0 = 0, keys1 = 0, vals0 = 0,
            vals1 = 0, hist = 0, dtot = 0, psorted = 0, poff = 0, items = 0, nitems = 0,
            Ld = 0, Li = 0, qplanes = 0, qxn = 0, cplanes = 0, ccn = 0, cused = 0, caug = 0,
-           cmax2 = 0, Sv = 0, Sp = 0, Slost = 0, fb = 0, xmax2 = 0, total = 0;
+           cmax2 = 0, Sv = 0, Sp = 0, Slost = 0, fb = 0, ubound = 0, xmax2 = 0, total = 0;
     int64_t P = 0, qbatch = 0, max_items = 0, dp = 0, Kp = 0;
     SortPlan sp;
 };
@@ -416,6 +423,7 @@ inline SearchLayout search_layout(int64_t nq, int d, int nlist, int nprobe, int 
     L.Sp = take(scr_fine ? sizeof(uint32_t) * L.P * kSearchScrList : 0);
     L.Slost = take(scr_fine ? sizeof(float) * L.P : 0);
     L.fb = take(scr_fine ? sizeof(int32_t) * nq : 0);
+    L.ubound = take(scr_fine ? sizeof(float) * nq : 0);
     L.xmax2 = take(256);
     L.total = o;
     return L;

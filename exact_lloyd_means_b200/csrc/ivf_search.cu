@@ -852,10 +852,13 @@ __global__ void cmax_kernel(const float *__restrict__ cn, int K, float *__restri
 // Tile: 128 points x 32 queries; warp w owns points 32w .. 32w + 31 (two 16-row blocks)
 // and all four 8-query blocks.  bf16 chunks of 32 dimensions of both planes arrive by
 // cp.async in two stages, rows of 40 elements (80 bytes: the 8 rows an ldmatrix reads
-// fall on distinct banks).
+// fall on distinct banks).  Measured on B200: a 4-stage pipeline (2 blocks per SM) and an
+// XOR-swizzled unpadded layout were both slower than this (4 blocks per SM).
 constexpr int kScrList = kSearchScrList;  // entries per pair list, one per lane
-constexpr int kBS = kTD + 8;   // bf16 row stride of the stages
+constexpr int kBS = kTD + 8;   // bf16 row stride of a stage: 80 bytes, so the 8 rows an
+                               // ldmatrix reads fall on distinct banks
 constexpr int kDSF = kTV + 4;  // fp32 row stride of the dot-product rows
+constexpr int kFineStages = 2; // chunks in flight: one behind the one in use
 
 struct StageB {
     uint16_t vh[kTV * kBS], vl[kTV * kBS];  // points: hi, lo
@@ -864,10 +867,13 @@ struct StageB {
 
 struct FineSmem {
     union {
-        StageB st[2];
+        StageB st[kFineStages];
         float dot[kTQ * kDSF];  // [query][point]
     };
 };
+
+// Element offset of 16-byte piece `piece` of stage row `row`.
+__device__ __forceinline__ int swz(int row, int piece) { return row * kBS + (piece << 3); }
 
 struct FineArgs {
     const uint16_t *Qp;        // [2][nq][dp] bf16 planes of the queries
@@ -884,6 +890,7 @@ struct FineArgs {
     float *Sv;                 // [P][kScrList] screened values, ascending
     uint32_t *Sp;              // [P][kScrList] point positions (0xffffffff: no point)
     float *Slost;              // [P]
+    const float *cut;          // optional [nq]: screened values above it are dropped uncounted
 };
 
 __device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], const void *p) {
@@ -917,12 +924,12 @@ __device__ __forceinline__ void stage_issue_b(StageB &sb, const uint16_t *Xh, co
         const int row = (tid >> 2) + 32 * r;
         const bool ok = row < nv;
         const int64_t off = ok ? (v0 + row) * dp + j0 + c16 * 8 : 0;
-        cp_async16(sb.vh + row * kBS + c16 * 8, Xh + off, ok ? 16 : 0);
-        cp_async16(sb.vl + row * kBS + c16 * 8, Xl + off, ok ? 16 : 0);
+        cp_async16(sb.vh + swz(row, c16), Xh + off, ok ? 16 : 0);
+        cp_async16(sb.vl + swz(row, c16), Xl + off, ok ? 16 : 0);
     }
     const int qr = tid >> 2;
-    cp_async16(sb.qh + qr * kBS + c16 * 8, qh ? qh + j0 + c16 * 8 : Xh, qh ? 16 : 0);
-    cp_async16(sb.ql + qr * kBS + c16 * 8, ql ? ql + j0 + c16 * 8 : Xh, ql ? 16 : 0);
+    cp_async16(sb.qh + swz(qr, c16), qh ? qh + j0 + c16 * 8 : Xh, qh ? 16 : 0);
+    cp_async16(sb.ql + swz(qr, c16), ql ? ql + j0 + c16 * 8 : Xh, ql ? 16 : 0);
 }
 
 // acc[m][n] += the chunk's three-product dot products of point block (2 warp + m) with
@@ -937,26 +944,34 @@ __device__ __forceinline__ void fine_mma(const StageB &sb, int warp, int lane, i
         for (int np = 0; np < 2; ++np) {
             if (2 * np < nact) {
                 const int q = np * 16 + (i >> 1) * 8 + r;
-                const int col = ks * 16 + (i & 1) * 8;
-                ldsm_x4(bh[np], sb.qh + q * kBS + col);
-                ldsm_x4(bl[np], sb.ql + q * kBS + col);
+                const int piece = ks * 2 + (i & 1);
+                ldsm_x4(bh[np], sb.qh + swz(q, piece));
+                ldsm_x4(bl[np], sb.ql + swz(q, piece));
             }
         }
+        uint32_t ah[2][4], al[2][4];
 #pragma unroll
         for (int m = 0; m < 2; ++m) {
             if (m < mact) {
                 const int p = warp * 32 + m * 16 + (i & 1) * 8 + r;
-                const int col = ks * 16 + (i >> 1) * 8;
-                uint32_t ah[4], al[4];
-                ldsm_x4(ah, sb.vh + p * kBS + col);
-                ldsm_x4(al, sb.vl + p * kBS + col);
+                const int piece = ks * 2 + (i >> 1);
+                ldsm_x4(ah[m], sb.vh + swz(p, piece));
+                ldsm_x4(al[m], sb.vl + swz(p, piece));
+            }
+        }
+        // one product at a time over all eight accumulators, so that consecutive
+        // instructions do not wait on one another
+#pragma unroll
+        for (int prod = 0; prod < 3; ++prod) {
+#pragma unroll
+            for (int m = 0; m < 2; ++m) {
 #pragma unroll
                 for (int n = 0; n < 4; ++n) {
-                    if (n < nact) {
+                    if (m < mact && n < nact) {
                         const int o = (n & 1) * 2;
-                        hmma(acc[m][n], ah, bh[n >> 1][o], bh[n >> 1][o + 1]);
-                        hmma(acc[m][n], ah, bl[n >> 1][o], bl[n >> 1][o + 1]);
-                        hmma(acc[m][n], al, bh[n >> 1][o], bh[n >> 1][o + 1]);
+                        const uint32_t(&aa)[4] = prod == 2 ? al[m] : ah[m];
+                        const uint32_t *bb = prod == 1 ? bl[n >> 1] : bh[n >> 1];
+                        hmma(acc[m][n], aa, bb[o], bb[o + 1]);
                     }
                 }
             }
@@ -973,6 +988,8 @@ __global__ void __launch_bounds__(kTThreads, 4) ivf_fine_scr_kernel(FineArgs a) 
     FineSmem &sm = *reinterpret_cast<FineSmem *>(smem_raw);
     __shared__ int s_item;
     __shared__ int s_pair[kTQ];
+    __shared__ double s_qn[kTQ];
+    __shared__ float s_cut[kTQ];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int dp = a.dp;
     const uint16_t *Xh = a.Xp, *Xl = a.Xp + a.N * dp;
@@ -986,7 +1003,13 @@ __global__ void __launch_bounds__(kTThreads, 4) ivf_fine_scr_kernel(FineArgs a) 
         const int2 it = a.items[item];
         const int nq_i = min(kTQ, a.pair_off[it.x + 1] - it.y);
         const int64_t vbeg = a.offsets[it.x], vend = a.offsets[it.x + 1];
-        if (tid < kTQ) s_pair[tid] = tid < nq_i ? a.pair_sorted[it.y + tid] : 0;
+        if (tid < kTQ) {
+            const int pr = tid < nq_i ? a.pair_sorted[it.y + tid] : 0;
+            s_pair[tid] = pr;
+            const int64_t qg = pr / a.nprobe;
+            s_qn[tid] = tid < nq_i ? a.qn[qg] : 0.0;
+            s_cut[tid] = (tid < nq_i && a.cut) ? a.cut[qg] : INFINITY;
+        }
         __syncthreads();
 
         const int sq = tid >> 2;  // the query row this thread stages
@@ -1017,18 +1040,25 @@ __global__ void __launch_bounds__(kTThreads, 4) ivf_fine_scr_kernel(FineArgs a) 
                     for (int e = 0; e < 4; ++e) acc[m][n][e] = 0.f;
             const int nch = dp / kTD;
             __syncthreads();  // the previous tile's readers of the dot rows are done
-            stage_issue_b(sm.st[0], Xh, Xl, v0, nv_t, dp, qh, ql, 0, tid);
-            cp_async_commit();
-            for (int c = 0; c < nch; ++c) {
-                cp_async_wait<0>();
-                __syncthreads();  // chunk c landed everywhere; chunk c - 1's stage is free
-                if (c + 1 < nch) {
-                    stage_issue_b(sm.st[(c + 1) & 1], Xh, Xl, v0, nv_t, dp, qh, ql,
-                                  (c + 1) * kTD, tid);
-                    cp_async_commit();
-                }
-                if (mact > 0) fine_mma(sm.st[c & 1], warp, lane, mact, nact, acc);
+#pragma unroll
+            for (int c = 0; c < kFineStages - 1; ++c) {  // every commit makes one group
+                if (c < nch)
+                    stage_issue_b(sm.st[c], Xh, Xl, v0, nv_t, dp, qh, ql, c * kTD, tid);
+                cp_async_commit();
             }
+            for (int c = 0; c < nch; ++c) {
+                cp_async_wait<kFineStages - 2>();  // chunk c has landed for this thread
+                // ... for every thread, and every warp is done with chunk c - 1, whose stage
+                // the copy below refills
+                __syncthreads();
+                const int cn = c + kFineStages - 1;
+                if (cn < nch)
+                    stage_issue_b(sm.st[cn % kFineStages], Xh, Xl, v0, nv_t, dp, qh, ql, cn * kTD,
+                                  tid);
+                cp_async_commit();
+                if (mact > 0) fine_mma(sm.st[c % kFineStages], warp, lane, mact, nact, acc);
+            }
+            cp_async_wait<0>();
             __syncthreads();  // every warp is done with the last stage
             {
                 const int g = lane >> 2, t = lane & 3;
@@ -1058,7 +1088,8 @@ __global__ void __launch_bounds__(kTThreads, 4) ivf_fine_scr_kernel(FineArgs a) 
             for (int q8 = 0; q8 < 8; ++q8) {
                 const int qi = warp * 8 + q8;
                 if (qi >= nq_i) continue;  // warp-uniform
-                const double qn = a.qn[s_pair[qi] / a.nprobe];
+                const double qn = s_qn[qi];
+                const float cut = s_cut[qi];
                 float tv = __shfl_sync(kFull, lv[q8], kScrList - 1);
                 uint32_t tp = __shfl_sync(kFull, lp[q8], kScrList - 1);
 #pragma unroll
@@ -1068,8 +1099,9 @@ __global__ void __launch_bounds__(kTThreads, 4) ivf_fine_scr_kernel(FineArgs a) 
                                                    qn + xn_i[i]))
                                              : INFINITY;
                     const uint32_t cp = static_cast<uint32_t>(v0 + lane + 32 * i);
-                    bool pend = ok_i[i] && before_f(cv, cp, tv, tp);
-                    if (ok_i[i] && !pend) lost[q8] = fminf(lost[q8], cv);
+                    const bool in = ok_i[i] && cv <= cut;  // else outside every window
+                    bool pend = in && before_f(cv, cp, tv, tp);
+                    if (in && !pend) lost[q8] = fminf(lost[q8], cv);
                     unsigned m = __ballot_sync(kFull, pend);
                     while (m) {
                         const int src = __ffs(m) - 1;
@@ -1139,6 +1171,7 @@ struct QueryArgs {
     float *out_dist;
     int32_t *out_id;
     int32_t *fallback;         // [nq]: 1 for queries left to fallback_kernel
+    const float *cut;          // optional [nq]: the fine pass's cut (query_cut_kernel)
 };
 
 __device__ __forceinline__ double exact_sq_dist(const float *q, const float *x, int d, int lane) {
@@ -1286,6 +1319,7 @@ __global__ void __launch_bounds__(kQThreads) query_rerank_kernel(QueryArgs a) {
     const uint32_t kthr = fkey(thr);
     for (int t = tid; t < a.nprobe; t += kQThreads)
         if (a.Slost[q * a.nprobe + t] < INFINITY && a.Slost[q * a.nprobe + t] <= thr) s_over = 1;
+    if (tid == 0 && a.cut && !(thr <= a.cut[q])) s_over = 1;  // the cut dropped values uncounted
     __syncthreads();  // the ranking's use of the candidate buffers is over
     for (int j = tid; j < L; j += kQThreads)
         if (key[j] <= kthr && sp[j] != 0xffffffffu) cpos[atomicAdd(&s_n, 1)] = sp[j];
@@ -1445,6 +1479,59 @@ __global__ void __launch_bounds__(kQThreads) fallback_kernel(FallbackArgs a) {
     }
 }
 
+// Cell radii: radius[c] >= max over the points x of cell c of ||x - c||, one block per
+// cell, a warp per point (fp64 difference form), rounded up to fp32 with a relative
+// margin far above the fp64 rounding; 0 for an empty cell.
+__global__ void __launch_bounds__(256) cell_radius_kernel(const float *__restrict__ C,
+                                                          const float *__restrict__ X,
+                                                          const int32_t *__restrict__ offsets,
+                                                          int d, float *__restrict__ radius) {
+    __shared__ double red[8];
+    const int c = blockIdx.x;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const float *cv = C + static_cast<int64_t>(c) * d;
+    double mx = 0.0;
+    for (int p = offsets[c] + warp; p < offsets[c + 1]; p += 8)
+        mx = fmax(mx, exact_sq_dist(cv, X + static_cast<int64_t>(p) * d, d, lane));
+    if (lane == 0) red[warp] = mx;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        for (int w = 1; w < 8; ++w) mx = fmax(mx, red[w]);
+        radius[c] = __double2float_ru(sqrt(mx) * (1.0 + 1e-9));
+    }
+}
+
+// Per query, a cut on the screened distances of the fine pass.  Every probed cell with at
+// least k points holds k points within (sqrt(D_c) + r_c)^2 of the query (D_c its fp64
+// squared distance to the centroid), so the smallest such value U bounds the query's k-th
+// smallest exact distance, and the k-th smallest screened value T~ <= U + E.  An entry
+// above cut = U + 3.1 E is therefore above T~ + 2E, outside the re-ranking window: the
+// fine pass drops it without counting it, and the merge sends the query to the exact
+// fallback should its own window ever reach past the cut.  +inf when no probed cell has k
+// points.  A warp per query.
+__global__ void __launch_bounds__(256) query_cut_kernel(
+    const float *__restrict__ Q, const float *__restrict__ C, const int32_t *__restrict__ probes,
+    const int32_t *__restrict__ offsets, const float *__restrict__ radius,
+    const double *__restrict__ qn, const float *__restrict__ xmax2, float ce_dot,
+    float ce_round, int64_t nq, int nprobe, int k, int d, float *__restrict__ cut) {
+    const int lane = threadIdx.x & 31;
+    const int64_t q = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+    if (q >= nq) return;
+    double u = INFINITY;
+    for (int t = 0; t < nprobe; ++t) {
+        const int c = probes[q * nprobe + t];
+        if (offsets[c + 1] - offsets[c] < k) continue;
+        const double D = exact_sq_dist(Q + q * d, C + static_cast<int64_t>(c) * d, d, lane);
+        const double r = sqrt(D) * (1.0 + 1e-9) + static_cast<double>(radius[c]);
+        u = fmin(u, r * r * (1.0 + 1e-9));
+    }
+    if (lane == 0) {
+        const float xm2 = *xmax2, qf = static_cast<float>(qn[q]);
+        const float E = ce_dot * sqrtf(qf * xm2) + ce_round * (qf + xm2);
+        cut[q] = __fadd_ru(__double2float_ru(u), 3.1f * E);
+    }
+}
+
 // Number of flagged queries (one block), for the caller's diagnostics.
 __global__ void count_flags_kernel(const int32_t *__restrict__ f, int64_t n, int *__restrict__ out) {
     __shared__ int red[32];
@@ -1550,6 +1637,8 @@ __global__ void __launch_bounds__(1024) build_items_kernel(const int32_t *__rest
 }  // namespace
 
 // ---------------------------------------------------------------- host side
+void fine_window_coeffs(int dp, float *ce_dot, float *ce_round);
+
 size_t ivf_tile_smem() { return sizeof(TileSmem); }
 
 cudaError_t launch_sqnorm_f64(const float *V, int64_t n, int d, double *out, cudaStream_t st) {
@@ -1647,9 +1736,9 @@ cudaError_t launch_ivf_fine_scr(const uint16_t *Qp, int64_t nq, const uint16_t *
                                 const int32_t *offsets, const int32_t *pair_sorted,
                                 const int32_t *pair_off, const int2 *items, const int *nitems,
                                 int *item_ctr, int64_t max_items, int nprobe, float *Sv,
-                                uint32_t *Sp, float *Slost, cudaStream_t st) {
+                                uint32_t *Sp, float *Slost, const float *cut, cudaStream_t st) {
     FineArgs a{Qp, nq, Xp, N, dp, qn, xn, offsets, pair_sorted, pair_off, items, nitems,
-               item_ctr, nprobe, Sv, Sp, Slost};
+               item_ctr, nprobe, Sv, Sp, Slost, cut};
     static int occ = 0;
     if (occ == 0) {
         cudaFuncSetAttribute(ivf_fine_scr_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -1684,9 +1773,10 @@ cudaError_t launch_ivf_query_rerank(const float *Sv, const uint32_t *Sp, const f
                                     const float *X, int d, int dp, const double *qn,
                                     const float *xmax2, const int32_t *row_ids,
                                     float *out_dist, int32_t *out_id, int32_t *fallback,
-                                    cudaStream_t st) {
+                                    const float *cut, cudaStream_t st) {
     if (nq <= 0) return cudaSuccess;
     QueryArgs a{};
+    a.cut = cut;
     a.Sv = Sv;
     a.Sp = Sp;
     a.Slost = Slost;
@@ -1726,6 +1816,27 @@ cudaError_t launch_ivf_fallback(const int32_t *fallback, const int32_t *probes, 
     if (nq <= 0) return cudaSuccess;
     FallbackArgs a{fallback, probes, nprobe, k, Q, X, d, offsets, row_ids, out_dist, out_id};
     fallback_kernel<<<static_cast<unsigned>(nq), kQThreads, 0, st>>>(a);
+    note_launch();
+    return cudaGetLastError();
+}
+
+cudaError_t launch_cell_radius(const float *C, int nlist, const float *X, const int32_t *offsets,
+                               int d, float *radius, cudaStream_t st) {
+    cell_radius_kernel<<<nlist, 256, 0, st>>>(C, X, offsets, d, radius);
+    note_launch();
+    return cudaGetLastError();
+}
+
+cudaError_t launch_query_cut(const float *Q, const float *C, const int32_t *probes,
+                             const int32_t *offsets, const float *radius, const double *qn,
+                             const float *xmax2, int dp, int64_t nq, int nprobe, int k, int d,
+                             float *cut, cudaStream_t st) {
+    if (nq <= 0) return cudaSuccess;
+    float ce_dot, ce_round;
+    fine_window_coeffs(dp, &ce_dot, &ce_round);
+    const int64_t blocks = ceil_div(nq, 8);
+    query_cut_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(
+        Q, C, probes, offsets, radius, qn, xmax2, ce_dot, ce_round, nq, nprobe, k, d, cut);
     note_launch();
     return cudaGetLastError();
 }

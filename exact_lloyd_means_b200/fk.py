@@ -82,8 +82,10 @@ _sig("fk_lloyd_streamed", [_vp, _int, _i64, _int, _int, _int, _int, _vp, _vp,
 _sig("fk_streamed_workspace_size", [_i64, _int, _int, _int, _int, ctypes.POINTER(_sz)])
 _sig("fk_ivf_norms", [_vp, _i64, _int, _vp, _vp])
 _sig("fk_ivf_search_workspace_size", [_i64, _int, _int, _i64, _int, _int, ctypes.POINTER(_sz)])
-_sig("fk_ivf_search", [_vp, _i64, _int, _vp, _int, _vp, _vp, _vp, _vp, _vp, _i64, _int, _int,
-                       _int, _vp, _vp, _vp, _vp, _sz, ctypes.POINTER(FkSearchTiming), _vp])
+_sig("fk_ivf_search", [_vp, _i64, _int, _vp, _int, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _int,
+                       _int, _int, _vp, _vp, _vp, _vp, _sz, ctypes.POINTER(FkSearchTiming),
+                       _vp])
+_sig("fk_ivf_radii", [_vp, _int, _vp, _vp, _int, _vp, _vp])
 
 EXPORTED = ["fk_status_string", "fk_version", "fk_workspace_size", "fk_normalize_rows",
             "fk_centroid_norms", "fk_assign", "fk_update", "fk_lloyd",
@@ -91,7 +93,7 @@ EXPORTED = ["fk_status_string", "fk_version", "fk_workspace_size", "fk_normalize
             "fk_update_partial", "fk_finalize_shards", "fk_split_points",
             "fk_launch_count", "fk_ivf_lists", "fk_lloyd_streamed",
             "fk_streamed_workspace_size", "fk_ivf_norms", "fk_ivf_search_workspace_size",
-            "fk_ivf_search"]
+            "fk_ivf_search", "fk_ivf_radii"]
 
 # Bytes of the static device array fk_assign_noalloc takes its scratch from.
 NOALLOC_SCRATCH_BYTES = 8 << 20
@@ -420,12 +422,13 @@ def fk_ivf_search(Q: torch.Tensor, C: torch.Tensor, X_lists: torch.Tensor,
                   distances: torch.Tensor | None = None, ids: torch.Tensor | None = None,
                   probes: torch.Tensor | None = None, timing: dict | None = None,
                   fp64_coarse: bool = False, X_planes=None, fp64_fine: bool = False,
-                  stream=None):
+                  cell_radius: torch.Tensor | None = None, stream=None):
     """IVF-Flat search: returns (distances fp32 [nq, k], ids int32 [nq, k]); `probes`
     (int32 [nq, nprobe]) receives the probed cells when given.  A `timing` dict receives
     the per-phase device times in ms (the call then synchronises its stream).
     X_planes: fk_split_points of X_lists (a SplitPoints or its buffer), which enables the
-    tensor-core fine pass.  fp64_coarse / fp64_fine compute every coarse / fine distance
+    tensor-core fine pass; cell_radius: fk_ivf_radii of the index, which lets that pass
+    skip the points that cannot be among a query's k nearest.  fp64_coarse / fp64_fine compute every coarse / fine distance
     in fp64 (FK_SEARCH_FP64_COARSE / FK_SEARCH_FP64_FINE)."""
     nq, d = Q.shape
     nlist = C.shape[0]
@@ -449,6 +452,7 @@ def fk_ivf_search(Q: torch.Tensor, C: torch.Tensor, X_lists: torch.Tensor,
                               _dev(C, "C", torch.float32, (nlist, d)), nlist,
                               _dev(X_lists, "X_lists", torch.float32, (N, d)),
                               _dev(X_norms, "X_norms", torch.float64, (N,)), planes_ptr,
+                              _opt(cell_radius, "cell_radius", torch.float32, (nlist,)),
                               _dev(offsets, "offsets", torch.int32, (nlist + 1,)),
                               _dev(row_ids, "row_ids", torch.int32, (N,)), N, nprobe, k,
                               flags,
@@ -463,16 +467,32 @@ def fk_ivf_search(Q: torch.Tensor, C: torch.Tensor, X_lists: torch.Tensor,
     return distances, ids
 
 
+def fk_ivf_radii(C: torch.Tensor, X_lists: torch.Tensor, offsets: torch.Tensor,
+                 out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Per cell, an upper bound on the distance of its points to its centroid."""
+    nlist, d = C.shape
+    if out is None:
+        out = torch.empty(nlist, dtype=torch.float32, device=C.device)
+    _check(_lib.fk_ivf_radii(_dev(C, "C", torch.float32), nlist,
+                             _dev(X_lists, "X_lists", torch.float32),
+                             _dev(offsets, "offsets", torch.int32, (nlist + 1,)), d,
+                             _dev(out, "out", torch.float32, (nlist,)), _stream(stream)),
+           "fk_ivf_radii")
+    return out
+
+
 class IvfFlatIndex:
     """An IVF-Flat index: centroids, cell-contiguous points with their original ids, CSR
-    offsets, fp64 norms and the bf16 planes of the points (for the tensor-core fine pass).
-    `build` and `search` only sequence libfk calls (fk_normalize_rows, fk_lloyd,
-    fk_ivf_lists, fk_ivf_norms, fk_split_points, fk_ivf_search)."""
+    offsets, fp64 norms, and for the tensor-core fine pass the bf16 planes of the points
+    and the cell radii.  `build` and `search` only sequence libfk calls
+    (fk_normalize_rows, fk_lloyd, fk_ivf_lists, fk_ivf_norms, fk_split_points,
+    fk_ivf_radii, fk_ivf_search)."""
 
-    def __init__(self, C, X_lists, X_norms, offsets, row_ids, metric="l2", X_planes=None):
+    def __init__(self, C, X_lists, X_norms, offsets, row_ids, metric="l2", X_planes=None,
+                 cell_radius=None):
         self.C, self.X_lists, self.X_norms = C, X_lists, X_norms
         self.offsets, self.row_ids, self.metric = offsets, row_ids, metric
-        self.X_planes = X_planes
+        self.X_planes, self.cell_radius = X_planes, cell_radius
 
     @classmethod
     def build(cls, X: torch.Tensor, C0: torch.Tensor, niter: int, metric="l2", stream=None):
@@ -496,7 +516,8 @@ class IvfFlatIndex:
         del ws
         X_norms = fk_ivf_norms(X_lists, stream=stream)
         X_planes = fk_split_points(X_lists, stream=stream)
-        return cls(C, X_lists, X_norms, offsets, row_ids, metric, X_planes)
+        radius = fk_ivf_radii(C, X_lists, offsets, stream=stream)
+        return cls(C, X_lists, X_norms, offsets, row_ids, metric, X_planes, radius)
 
     def search(self, Q: torch.Tensor, k: int, nprobe: int, ws=None, distances=None,
                ids=None, probes=None, timing=None, fp64_coarse=False, fp64_fine=False,
@@ -510,4 +531,5 @@ class IvfFlatIndex:
         return fk_ivf_search(Q, self.C, self.X_lists, self.X_norms, self.offsets,
                              self.row_ids, nprobe, k, ws=ws, distances=distances, ids=ids,
                              probes=probes, timing=timing, fp64_coarse=fp64_coarse,
-                             X_planes=self.X_planes, fp64_fine=fp64_fine, stream=stream)
+                             X_planes=self.X_planes, fp64_fine=fp64_fine,
+                             cell_radius=self.cell_radius, stream=stream)

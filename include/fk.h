@@ -268,6 +268,15 @@ FK_API fk_status fk_ivf_lists(const void *X, fk_dtype dtype, int64_t N, int d, i
 FK_API fk_status fk_ivf_norms(const float *V, int64_t n, int d, double *norms,
                               fk_stream_t stream);
 
+/* Cell radii for IVF-Flat search: radius[c] >= max over the points x of cell c of
+ * ||x - C[c]|| (fp64 distances, rounded up to fp32 with a relative margin), 0 for an empty
+ * cell.  C nlist x d fp32, X_lists N x d fp32 in cell order, offsets nlist + 1 int32
+ * (fk_ivf_lists), radius nlist floats; all device; d % 4 == 0, C and X_lists 16-byte
+ * aligned.  Computed once per index; fk_ivf_search uses it to skip, in its screened fine
+ * pass, the points that cannot be among a query's k nearest. */
+FK_API fk_status fk_ivf_radii(const float *C, int nlist, const float *X_lists,
+                              const int32_t *offsets, int d, float *radius, fk_stream_t stream);
+
 /* Workspace bytes of fk_ivf_search for these sizes. */
 FK_API fk_status fk_ivf_search_workspace_size(int64_t nq, int d, int nlist, int64_t N,
                                               int nprobe, int k, size_t *bytes);
@@ -304,7 +313,9 @@ FK_API fk_status fk_ivf_search_workspace_size(int64_t nq, int d, int nlist, int6
  * Inputs (device pointers, read only): Q nq x d fp32; C nlist x d fp32 centroids; X_lists
  * N x d fp32, the points in cell order (fk_ivf_lists); X_norms N doubles, fk_ivf_norms of
  * X_lists; X_planes NULL or the 4 N d_p + 4 N bytes that fk_split_points writes for
- * X_lists (16-byte aligned); offsets nlist + 1 int32 (offsets[0] = 0, offsets[nlist] = N,
+ * X_lists (16-byte aligned); cell_radius NULL or fk_ivf_radii of (C, X_lists) (with the
+ * screened fine pass, each query then skips the points farther than a bound on its k-th
+ * nearest that the nearest probed cells give); offsets nlist + 1 int32 (offsets[0] = 0, offsets[nlist] = N,
  * non-decreasing);
  * row_ids N int32 (fk_ivf_lists).  Outputs (device): distances nq x k fp32, ids nq x k
  * int32, probes nq x nprobe int32 or NULL (then kept in the workspace).
@@ -332,7 +343,8 @@ typedef struct fk_search_timing {
 
 FK_API fk_status fk_ivf_search(const float *Q, int64_t nq, int d, const float *C, int nlist,
                                const float *X_lists, const double *X_norms,
-                               const void *X_planes, const int32_t *offsets,
+                               const void *X_planes, const float *cell_radius,
+                               const int32_t *offsets,
                                const int32_t *row_ids, int64_t N, int nprobe, int k,
                                int flags, float *distances, int32_t *ids,
                                int32_t *probes, void *ws, size_t ws_bytes,

@@ -128,14 +128,14 @@ def test_ivf_lists_host_checks(fk):
 def test_ivf_search_host_checks(fk):
     lib = fk._lib
     big = 1 << 30
-    ok = dict(Q=256, nq=10, d=8, C=256, nlist=4, Xl=256, Xn=256, Xp=None, off=256, rid=256,
-              N=100,
+    ok = dict(Q=256, nq=10, d=8, C=256, nlist=4, Xl=256, Xn=256, Xp=None, rad=None, off=256,
+              rid=256, N=100,
               nprobe=2, k=3, flags=0, dist=256, ids=256, probes=None, ws=256, wsb=big)
 
     def call(**kw):
         a = dict(ok, **kw)
         return lib.fk_ivf_search(a["Q"], a["nq"], a["d"], a["C"], a["nlist"], a["Xl"], a["Xn"],
-                                 a["Xp"], a["off"], a["rid"], a["N"], a["nprobe"], a["k"], a["flags"],
+                                 a["Xp"], a["rad"], a["off"], a["rid"], a["N"], a["nprobe"], a["k"], a["flags"],
                                  a["dist"],
                                  a["ids"], a["probes"], a["ws"], a["wsb"], None, None)
 
@@ -143,11 +143,14 @@ def test_ivf_search_host_checks(fk):
                 dict(N=0), dict(Q=None), dict(Xn=None), dict(ids=None),
                 dict(nq=1 << 30, nprobe=4)):
         assert call(**bad) == fk.FK_ERR_INVALID_ARG, bad
-    for bad in (dict(d=6), dict(Q=8), dict(Xl=264), dict(probes=258), dict(Xp=264)):
+    for bad in (dict(d=6), dict(Q=8), dict(Xl=264), dict(probes=258), dict(Xp=264),
+                dict(rad=258)):
         assert call(**bad) == fk.FK_ERR_UNSUPPORTED, bad
     assert call(wsb=10) == fk.FK_ERR_WORKSPACE
     assert call(ws=None) == fk.FK_ERR_WORKSPACE
     assert lib.fk_ivf_norms(None, 10, 8, 256, None) == fk.FK_ERR_INVALID_ARG
+    assert lib.fk_ivf_radii(None, 4, 256, 256, 8, 256, None) == fk.FK_ERR_INVALID_ARG
+    assert lib.fk_ivf_radii(256, 4, 256, 256, 6, 256, None) == fk.FK_ERR_UNSUPPORTED
     assert lib.fk_ivf_norms(256, 10, 6, 256, None) == fk.FK_ERR_UNSUPPORTED
     with pytest.raises(fk.FkError) as e:
         fk.ivf_search_workspace(10, 8, 4, 100, 5, 3, device="cpu")

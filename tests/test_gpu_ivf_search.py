@@ -40,19 +40,25 @@ def _index(X, labels, nlist):
     return X_lists, m.fk_ivf_norms(X_lists), offsets, row_ids, m.fk_split_points(X_lists)
 
 
-def _search(Q, C, idx, nprobe, k, fp64_coarse=False, fp64_fine=False, timing=None):
+def _search(Q, C, idx, nprobe, k, fp64_coarse=False, fp64_fine=False, timing=None,
+            radius=True):
     m = fk()
     X_lists, X_norms, offsets, row_ids, planes = idx
     nq = Q.shape[0]
+    Cd = C.to(DEV)
+    rad = m.fk_ivf_radii(Cd, X_lists, offsets) if radius else None
     probes = torch.full((nq, nprobe), -7, dtype=torch.int32, device=DEV)
-    dist, ids = m.fk_ivf_search(Q.to(DEV), C.to(DEV), X_lists, X_norms, offsets, row_ids,
+    dist, ids = m.fk_ivf_search(Q.to(DEV), Cd, X_lists, X_norms, offsets, row_ids,
                                 nprobe, k, probes=probes, fp64_coarse=fp64_coarse,
-                                X_planes=planes, fp64_fine=fp64_fine, timing=timing)
+                                X_planes=planes, fp64_fine=fp64_fine, timing=timing,
+                                cell_radius=rad)
     torch.cuda.synchronize()
     return probes.cpu().numpy(), ids.cpu().numpy(), dist.cpu().numpy()
 
 
-MODES = [(False, False), (True, False), (False, True), (True, True)]  # fp64 coarse, fp64 fine
+# (fp64 coarse, fp64 fine, cell radii)
+MODES = [(False, False, True), (True, False, True), (False, True, True), (True, True, True),
+         (False, False, False)]
 
 
 def _sqd(A, B):
@@ -115,9 +121,10 @@ def test_ivf_search_matches_oracle(N, d, nlist, nq, nprobe, k, weights, labels_f
                         seed=N + d, stream=1)
     ref = oracle.ivf_search(Q, C, X, labels, nprobe, k)
     idx = _index(X, labels, nlist)
-    for f64c, f64f in MODES:
+    for f64c, f64f, rad in MODES:
         tm = {}
-        got = _search(Q, C, idx, nprobe, k, fp64_coarse=f64c, fp64_fine=f64f, timing=tm)
+        got = _search(Q, C, idx, nprobe, k, fp64_coarse=f64c, fp64_fine=f64f, timing=tm,
+                      radius=rad)
         assert tm["screened_coarse"] == (0 if f64c else 1)
         assert tm["screened_fine"] == (0 if (f64f or k > 16) else 1)
         check_search(Q, C, X, got, ref)
@@ -137,8 +144,8 @@ def test_ivf_search_empty_cells_and_few_candidates():
         ref = oracle.ivf_search(Q, C, X, labels, nprobe, k)
         assert (ref[1] == -1).any() or nprobe == nlist
         idx = _index(X, labels, nlist)
-        for f64c, f64f in MODES:
-            got = _search(Q, C, idx, nprobe, k, fp64_coarse=f64c, fp64_fine=f64f)
+        for f64c, f64f, rad in MODES:
+            got = _search(Q, C, idx, nprobe, k, fp64_coarse=f64c, fp64_fine=f64f, radius=rad)
             check_search(Q, C, X, got, ref, max_bad_frac=0.0)
 
 
@@ -154,8 +161,8 @@ def test_ivf_search_duplicates_and_self_queries():
     Q = X[sel].clone()
     ref = oracle.ivf_search(Q, C, X, labels, 2, 6)
     idx = _index(X, labels, K)
-    for f64c, f64f in MODES:
-        got = _search(Q, C, idx, 2, 6, fp64_coarse=f64c, fp64_fine=f64f)
+    for f64c, f64f, rad in MODES:
+        got = _search(Q, C, idx, 2, 6, fp64_coarse=f64c, fp64_fine=f64f, radius=rad)
         check_search(Q, C, X, got, ref, max_bad_frac=0.0)
         ids = got[1]
         assert (ids[:, 0] == sel).all()
@@ -285,3 +292,23 @@ def test_ivf_search_screened_fine_fallback_on_tied_candidates():
         assert tm["screened_fine"] == 1 and tm["fallback_queries"] >= 1
         check_search(Q, C, X, got, ref, max_bad_frac=0.0)
         assert (got[1][0] == np.r_[7, dup][:k]).all()
+
+
+def test_ivf_radii_bound_every_cell():
+    """fk_ivf_radii: each radius is at least the largest distance of a cell's points to its
+    centroid (fp64 on the CPU), and within fp32 rounding of it; empty cells give 0."""
+    m = fk()
+    N, d, K = 20000, 48, 64
+    X, comp, _ = gaussian_mixture(N, d, K - 3, centers="normal", sigma=0.4, seed=31)
+    labels = comp.numpy().astype(np.int32)          # cells K-3 .. K-1 stay empty
+    C = torch.randn(K, d, generator=torch.Generator().manual_seed(4))
+    idx = _index(X, labels, K)
+    rad = m.fk_ivf_radii(C.to(DEV), idx[0], idx[2]).cpu().numpy().astype(np.float64)
+    X64, C64 = X.double().numpy(), C.double().numpy()
+    for c in range(K):
+        pts = X64[labels == c]
+        if len(pts) == 0:
+            assert rad[c] == 0.0
+            continue
+        r = np.sqrt(((pts - C64[c]) ** 2).sum(1).max())
+        assert r <= rad[c] <= r * (1 + 1e-6)
