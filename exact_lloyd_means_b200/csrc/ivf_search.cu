@@ -69,6 +69,26 @@ __device__ __forceinline__ bool before(double da, uint32_t ia, double db, uint32
     return da < db || (da == db && ia < ib);
 }
 
+// Exact squared distance of two fp32 rows in fp64 (difference form), a warp cooperating:
+// lane l sums the columns 4l .. 4l + 3 (mod 128) in order, then a fixed butterfly; every
+// lane returns the same value.
+__device__ __forceinline__ double exact_sq_dist(const float *q, const float *x, int d, int lane) {
+    double acc = 0.0;
+    for (int j = lane * 4; j < d; j += 128) {
+        const float4 u = __ldg(reinterpret_cast<const float4 *>(q + j));
+        const float4 v = __ldg(reinterpret_cast<const float4 *>(x + j));
+        const double e0 = static_cast<double>(u.x) - v.x, e1 = static_cast<double>(u.y) - v.y;
+        const double e2 = static_cast<double>(u.z) - v.z, e3 = static_cast<double>(u.w) - v.w;
+        acc = fma(e0, e0, acc);
+        acc = fma(e1, e1, acc);
+        acc = fma(e2, e2, acc);
+        acc = fma(e3, e3, acc);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(kFull, acc, o);
+    return acc;
+}
+
 // 16-byte global -> shared copy; src_bytes = 0 fills zeros without reading.
 __device__ __forceinline__ void cp_async16(void *smem, const void *gmem, int src_bytes) {
     const uint32_t sa = static_cast<uint32_t>(__cvta_generic_to_shared(smem));
@@ -773,23 +793,12 @@ __global__ void __launch_bounds__(kCoarseThreads) coarse_rerank_kernel(CoarseArg
     __syncthreads();
     const int n = s_n;
     // 4. exact fp64 distance of each candidate, a warp each: fixed lane split, fixed tree
+    // (coalesced 512-byte reads of the L2-resident centroid rows; measured faster than a
+    // lane per candidate)
     const float *qv = a.Q + q * a.d;
     for (int t = warp; t < n; t += kCoarseThreads / 32) {
-        const float *cv = a.C + static_cast<int64_t>(cid[t]) * a.d;
-        double acc = 0.0;
-        for (int j = lane * 4; j < a.d; j += 128) {
-            const float4 x = __ldg(reinterpret_cast<const float4 *>(qv + j));
-            const float4 y = __ldg(reinterpret_cast<const float4 *>(cv + j));
-            const double e0 = static_cast<double>(x.x) - y.x, e1 = static_cast<double>(x.y) - y.y;
-            const double e2 = static_cast<double>(x.z) - y.z, e3 = static_cast<double>(x.w) - y.w;
-            acc = fma(e0, e0, acc);
-            acc = fma(e1, e1, acc);
-            acc = fma(e2, e2, acc);
-            acc = fma(e3, e3, acc);
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(kFull, acc, o);
-        if (lane == 0) cd[t] = acc;
+        const double e = exact_sq_dist(qv, a.C + static_cast<int64_t>(cid[t]) * a.d, a.d, lane);
+        if (lane == 0) cd[t] = e;
     }
     // 5. sort the candidates by (distance, cell) and keep the first m
     int M = 1;
@@ -1174,22 +1183,6 @@ struct QueryArgs {
     const float *cut;          // optional [nq]: the fine pass's cut (query_cut_kernel)
 };
 
-__device__ __forceinline__ double exact_sq_dist(const float *q, const float *x, int d, int lane) {
-    double acc = 0.0;
-    for (int j = lane * 4; j < d; j += 128) {
-        const float4 u = __ldg(reinterpret_cast<const float4 *>(q + j));
-        const float4 v = __ldg(reinterpret_cast<const float4 *>(x + j));
-        const double e0 = static_cast<double>(u.x) - v.x, e1 = static_cast<double>(u.y) - v.y;
-        const double e2 = static_cast<double>(u.z) - v.z, e3 = static_cast<double>(u.w) - v.w;
-        acc = fma(e0, e0, acc);
-        acc = fma(e1, e1, acc);
-        acc = fma(e2, e2, acc);
-        acc = fma(e3, e3, acc);
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(kFull, acc, o);
-    return acc;
-}
 
 __global__ void __launch_bounds__(kQThreads) query_rerank_kernel(QueryArgs a) {
     extern __shared__ __align__(16) unsigned char qr_raw[];
@@ -1549,11 +1542,15 @@ __global__ void count_flags_kernel(const int32_t *__restrict__ f, int64_t n, int
     }
 }
 
-// max_i ||x_i||^2 of fp64 norms, rounded up to fp32 (one block).
-__global__ void max_norm_kernel(const double *__restrict__ xn, int64_t n, float *__restrict__ out) {
+// max_i ||x_i||^2 of fp64 norms, rounded up to fp32: block maxima combined by an integer
+// max on the bits (non-negative floats order as their bit patterns; *out starts at 0).
+__global__ void max_norm_kernel(const double *__restrict__ xn, int64_t n,
+                                uint32_t *__restrict__ out) {
     __shared__ double red[32];
     double mx = 0.0;
-    for (int64_t i = threadIdx.x; i < n; i += blockDim.x) mx = fmax(mx, xn[i]);
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+         i += static_cast<int64_t>(gridDim.x) * blockDim.x)
+        mx = fmax(mx, xn[i]);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) mx = fmax(mx, __shfl_xor_sync(kFull, mx, o));
     if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = mx;
@@ -1562,7 +1559,7 @@ __global__ void max_norm_kernel(const double *__restrict__ xn, int64_t n, float 
         mx = threadIdx.x < (blockDim.x >> 5) ? red[threadIdx.x] : 0.0;
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) mx = fmax(mx, __shfl_xor_sync(kFull, mx, o));
-        if (threadIdx.x == 0) *out = __double2float_ru(mx);
+        if (threadIdx.x == 0) atomicMax(out, __float_as_uint(__double2float_ru(mx)));
     }
 }
 
@@ -1848,7 +1845,11 @@ cudaError_t launch_count_flags(const int32_t *f, int64_t n, int *out, cudaStream
 }
 
 cudaError_t launch_max_norm(const double *xn, int64_t n, float *out, cudaStream_t st) {
-    max_norm_kernel<<<1, 1024, 0, st>>>(xn, n, out);
+    cudaError_t e = cudaMemsetAsync(out, 0, sizeof(float), st);
+    if (e != cudaSuccess) return e;
+    const int64_t blocks = ceil_div(n, 1024);
+    const int grid = static_cast<int>(blocks < 148 * 4 ? (blocks < 1 ? 1 : blocks) : 148 * 4);
+    max_norm_kernel<<<grid, 1024, 0, st>>>(xn, n, reinterpret_cast<uint32_t *>(out));
     note_launch();
     return cudaGetLastError();
 }
