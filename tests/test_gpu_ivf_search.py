@@ -312,3 +312,27 @@ def test_ivf_radii_bound_every_cell():
             continue
         r = np.sqrt(((pts - C64[c]) ** 2).sum(1).max())
         assert r <= rad[c] <= r * (1 + 1e-6)
+
+
+@pytest.mark.parametrize("seed", range(12))
+def test_ivf_search_random_shapes(seed):
+    """Seeded random shapes: small and odd d, nlist down to 1, cells of every size, k up to
+    32, nprobe up to nlist; every path against the oracle."""
+    r = np.random.default_rng(1000 + seed)
+    d = int(r.choice([4, 8, 12, 36, 64, 100, 132]))
+    nlist = int(r.choice([1, 2, 7, 33, 100]))
+    N = int(r.integers(max(nlist, 20), 3000))
+    nq = int(r.integers(1, 70))
+    k = int(r.integers(1, 33))
+    nprobe = int(r.integers(1, nlist + 1))
+    X, _, _ = gaussian_mixture(N, d, max(nlist, 2), centers="normal", sigma=float(r.uniform(0.05, 1.0)),
+                               weights=str(r.choice(["equal", "zipf"])), seed=seed)
+    C = X[init_indices(N, nlist, seed)].float().contiguous()
+    labels = (oracle.assign(X, C)[0] if r.random() < 0.5 else
+              r.integers(0, nlist, N).astype(np.int32))
+    Q = mixture_queries(nq, d, max(nlist, 2), seed=seed, stream=3)
+    ref = oracle.ivf_search(Q, C, X, labels, nprobe, k)
+    idx = _index(X, labels, nlist)
+    for f64c, f64f, rad in MODES:
+        got = _search(Q, C, idx, nprobe, k, fp64_coarse=f64c, fp64_fine=f64f, radius=rad)
+        check_search(Q, C, X, got, ref, max_bad_frac=0.05)
