@@ -1,8 +1,11 @@
 // fk_api.cu -- the extern "C" boundary of libfk: argument validation, workspace carving,
 // stream plumbing and the Lloyd loop.  Every arithmetic step runs in the kernels of
 // prep.cu, assign_sm100.cu, sort_csr.cu and update.cu; this file only launches them.
+#include <cstdlib>
 #include <cstring>
 #include <vector>
+
+#include <nvtx3/nvToolsExt.h>
 
 #include "fk_common.cuh"
 #include "ptx_sm100.cuh"
@@ -25,6 +28,32 @@ int device_sm_count() {
 namespace {
 
 constexpr uint64_t kDefaultWaitNs = 2000000000ull;  // 2 s bound on any in-kernel wait
+
+// NVTX range for the phases of a call (visible to profilers that record NVTX; without
+// one attached the calls cost a branch).
+struct NvtxRange {
+    explicit NvtxRange(const char *name) { nvtxRangePushA(name); }
+    ~NvtxRange() { nvtxRangePop(); }
+    NvtxRange(const NvtxRange &) = delete;
+    NvtxRange &operator=(const NvtxRange &) = delete;
+};
+
+// Host-side fault injection for tests of the error paths, chosen by the environment
+// variable FK_FAULT when the library is first used: "workspace" makes every workspace
+// check fail (FK_ERR_WORKSPACE); "launch" makes fk_assign, fk_update, fk_lloyd and
+// fk_ivf_search fail as a failed launch would (FK_ERR_CUDA), before any device work.
+// Nothing is injected on the device.
+enum Fault { kFaultNone = 0, kFaultWorkspace = 1, kFaultLaunch = 2 };
+Fault injected_fault() {
+    static const Fault f = [] {
+        const char *e = std::getenv("FK_FAULT");
+        if (!e) return kFaultNone;
+        if (std::strcmp(e, "workspace") == 0) return kFaultWorkspace;
+        if (std::strcmp(e, "launch") == 0) return kFaultLaunch;
+        return kFaultNone;
+    }();
+    return f;
+}
 
 fk_status check_device() {
     static int verdict[64] = {0};  // 0 unknown, 1 ok, 2 unsupported
@@ -59,6 +88,7 @@ fk_status validate_shape(int64_t N, int d, int K, fk_dtype dtype, fk_metric metr
 
 fk_status check_ws(void *ws, size_t ws_bytes, const WsLayout &L) {
     if (ws == nullptr || !aligned(ws, 256) || ws_bytes < L.total) return FK_ERR_WORKSPACE;
+    if (injected_fault() == kFaultWorkspace) return FK_ERR_WORKSPACE;
     return FK_OK;
 }
 
@@ -388,7 +418,7 @@ const char *fk_status_string(fk_status s) {
     return "FK_UNKNOWN_STATUS";
 }
 
-int fk_version(void) { return 3; }
+int fk_version(void) { return 4; }
 
 int64_t fk_launch_count(void) { return g_launches; }
 
@@ -447,6 +477,7 @@ fk_status fk_assign(const void *X, fk_dtype dtype, int64_t N, int d, const float
     const WsLayout L = ws_layout(N, d, K, dtype, FK_L2);
     if ((s = check_ws(ws, ws_bytes, L)) != FK_OK) return s;
     if ((s = check_device()) != FK_OK) return s;
+    if (injected_fault() == kFaultLaunch) return FK_ERR_CUDA;
     cudaStream_t st = stream;
     FK_TRY_CUDA(launch_prep_centroids(C, K, d, L.Kp, L.dp, dtype, ws_ptr<uint16_t>(ws, L.cs),
                                       ws_ptr<float>(ws, L.cn), ws_ptr<float>(ws, L.cused),
@@ -481,6 +512,7 @@ fk_status fk_update(const void *X, fk_dtype dtype, int64_t N, int d, int K,
     const WsLayout L = ws_layout(N, d, K, dtype, FK_L2);
     if ((s = check_ws(ws, ws_bytes, L)) != FK_OK) return s;
     if ((s = check_device()) != FK_OK) return s;
+    if (injected_fault() == kFaultLaunch) return FK_ERR_CUDA;
     cudaStream_t st = stream;
     const float *C_used = C_old;
     if (dtype == FK_BF16) {
@@ -506,6 +538,7 @@ fk_status fk_lloyd(const void *X, fk_dtype dtype, int64_t N, int d, int K, fk_me
     const WsLayout L = ws_layout(N, d, K, dtype, metric);
     if ((s = check_ws(ws, ws_bytes, L)) != FK_OK) return s;
     if ((s = check_device()) != FK_OK) return s;
+    if (injected_fault() == kFaultLaunch) return FK_ERR_CUDA;
     cudaStream_t st = stream;
 
     // events: [0] start, [1] after setup, then 4 per iteration
@@ -535,6 +568,7 @@ fk_status fk_lloyd(const void *X, fk_dtype dtype, int64_t N, int d, int K, fk_me
         return f;
     };
 
+    NvtxRange call_range("fk_lloyd");
     if (cudaMemsetAsync(ws_ptr<uint32_t>(ws, L.err), 0, 2 * sizeof(uint32_t), st) != cudaSuccess)
         return FK_ERR_CUDA;
     const long launches0 = g_launches;
@@ -564,6 +598,7 @@ fk_status fk_lloyd(const void *X, fk_dtype dtype, int64_t N, int d, int K, fk_me
     int copied = 0;
     bool allow_screen = true;
     int nscreened = 0;
+    bool last_screened = false;
     if (niter > 0 && dtype == FK_F32) {
         // Where the screened route applies, try it first on a sample of the rows with the
         // initial centroids and read how many would need the three-product pass (a single
@@ -589,6 +624,7 @@ fk_status fk_lloyd(const void *X, fk_dtype dtype, int64_t N, int d, int K, fk_me
     }
     if (!rec()) return fail(FK_ERR_CUDA);  // end of the once-per-call setup
     for (int t = 0; t < niter; ++t) {
+        NvtxRange iter_range("fk_lloyd iteration");
         if (launch_prep_centroids(Ccur, K, d, L.Kp, L.dp, dtype, ws_ptr<uint16_t>(ws, L.cs),
                                   ws_ptr<float>(ws, L.cn), cused, ws_ptr<uint16_t>(ws, L.caug),
                                   st) != cudaSuccess)
@@ -602,22 +638,32 @@ fk_status fk_lloyd(const void *X, fk_dtype dtype, int64_t N, int d, int K, fk_me
                             allow_screen, &screened, m0, m1)) != FK_OK)
             return fail(s);
         nscreened += screened ? 1 : 0;
+        last_screened = screened;
         if (!rec()) return fail(FK_ERR_CUDA);
+        nvtxRangePushA("sort + update");
         const int32_t *skeys = nullptr, *perm = nullptr;
         if (launch_sort_csr(labels, N, K, L.sp, ws_ptr<int32_t>(ws, L.keys0),
                             ws_ptr<int32_t>(ws, L.keys1), ws_ptr<int32_t>(ws, L.vals0),
                             ws_ptr<int32_t>(ws, L.vals1), nullptr,
                             ws_ptr<uint32_t>(ws, L.hist), ws_ptr<uint32_t>(ws, L.dtot), off,
-                            &skeys, &perm, ws_ptr<uint32_t>(ws, L.err), st) != cudaSuccess)
+                            &skeys, &perm, ws_ptr<uint32_t>(ws, L.err), st) != cudaSuccess) {
+            nvtxRangePop();
             return fail(FK_ERR_CUDA);
-        if (!rec()) return fail(FK_ERR_CUDA);
+        }
+        if (!rec()) {
+            nvtxRangePop();
+            return fail(FK_ERR_CUDA);
+        }
         if (launch_update(Xp, dtype, N, d, K, L.up, skeys, perm, off, Ccur,
                           dtype == FK_F32 ? Ccur : cused, Cnext, cnt,
                           ws_ptr<double>(ws, L.pieces), ws_ptr<int32_t>(ws, L.pkeys),
                           ws_ptr<double>(ws, L.piecesb), ws_ptr<int32_t>(ws, L.pkeysb),
                           ws_ptr<double>(ws, L.jpart), obj + (t % kObjRing),
-                          ws_ptr<uint32_t>(ws, L.err), nullptr, st) != cudaSuccess)
+                          ws_ptr<uint32_t>(ws, L.err), nullptr, st) != cudaSuccess) {
+            nvtxRangePop();
             return fail(FK_ERR_CUDA);
+        }
+        nvtxRangePop();
         if (!rec()) return fail(FK_ERR_CUDA);
         float *tmp = Ccur;
         Ccur = Cnext;
@@ -638,11 +684,28 @@ fk_status fk_lloyd(const void *X, fk_dtype dtype, int64_t N, int d, int K, fk_me
         cudaMemcpyAsync(objective_host + copied, obj, sizeof(double) * (niter - copied),
                         cudaMemcpyDeviceToHost, st) != cudaSuccess)
         return fail(FK_ERR_CUDA);
+    // last-iteration statistics (timing only): words 4, 5 of the error block get the
+    // empty-cluster count and the largest cluster
+    uint32_t stats[3] = {0, 0, 0};
+    if (timing && niter > 0) {
+        uint32_t *sw = ws_ptr<uint32_t>(ws, L.err) + 4;
+        if (launch_cluster_stats(cnt, K, sw, st) != cudaSuccess ||
+            cudaMemcpyAsync(stats, sw, 2 * sizeof(uint32_t), cudaMemcpyDeviceToHost, st) !=
+                cudaSuccess)
+            return fail(FK_ERR_CUDA);
+        if (last_screened &&
+            cudaMemcpyAsync(stats + 2, ws_ptr<uint32_t>(ws, L.nfb), sizeof(uint32_t),
+                            cudaMemcpyDeviceToHost, st) != cudaSuccess)
+            return fail(FK_ERR_CUDA);
+    }
     int code = FK_OK;
     if (read_err(ws, L, st, true, &code) != FK_OK) return fail(FK_ERR_CUDA);
     if (timing && ev.size() >= 2) {
         float ms = 0.f;
         std::memset(timing, 0, sizeof(*timing));
+        timing->empty_clusters = static_cast<int>(stats[0]);
+        timing->max_cluster = static_cast<int>(stats[1]);
+        timing->fallback_rows = static_cast<int>(stats[2]);
         cudaEventElapsedTime(&ms, ev[0], ev[1]);
         timing->ms_setup = ms;
         double *slot[4] = {&timing->ms_prep, &timing->ms_assign, &timing->ms_sort,
@@ -956,7 +1019,9 @@ fk_status fk_ivf_search(const float *Q, int64_t nq, int d, const float *C, int n
         return FK_ERR_UNSUPPORTED;
     const SearchLayout L = search_layout(nq, d, nlist, nprobe, k);
     if (ws == nullptr || !aligned(ws, 256) || ws_bytes < L.total) return FK_ERR_WORKSPACE;
+    if (injected_fault() == kFaultWorkspace) return FK_ERR_WORKSPACE;
     if ((s = check_device()) != FK_OK) return s;
+    if (injected_fault() == kFaultLaunch) return FK_ERR_CUDA;
     cudaStream_t st = stream;
     cudaEvent_t ev[5] = {};
     auto destroy = [&]() {
@@ -975,6 +1040,7 @@ fk_status fk_ivf_search(const float *Q, int64_t nq, int d, const float *C, int n
                                               static_cast<int>(L.Kp));
     const bool screen_fine = X_planes != nullptr && (flags & FK_SEARCH_FP64_FINE) == 0 &&
                              k <= kSearchScrMaxK && nprobe <= kSearchScrMaxProbe;
+    NvtxRange call_range("fk_ivf_search");
     const fk_status r = run_ivf_search(Q, nq, d, C, nlist, X_lists, X_norms, X_planes,
                                        cell_radius, offsets, row_ids, N, nprobe, k, screen,
                                        screen_fine, distances, ids, probes, ws, L, st,

@@ -429,6 +429,9 @@ inline SearchLayout search_layout(int64_t nq, int d, int nlist, int nprobe, int 
     return L;
 }
 
+// Empty clusters and the largest cluster of counts[K], written to out[0], out[1].
+cudaError_t launch_cluster_stats(const int32_t *counts, int K, uint32_t *out, cudaStream_t st);
+
 int device_sm_count();
 
 // Kernels launched by this host thread since the last reset (fk_lloyd reports it).

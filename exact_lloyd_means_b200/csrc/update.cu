@@ -746,4 +746,42 @@ cudaError_t launch_finalize_shards(const double *sums, const int64_t *cnts, cons
     return cudaGetLastError();
 }
 
+namespace {
+// Empty clusters and the largest cluster of a count array (one block).
+__global__ void cluster_stats_kernel(const int32_t *__restrict__ counts, int K,
+                                     uint32_t *__restrict__ out) {
+    __shared__ uint32_t e_red[32], m_red[32];
+    uint32_t empty = 0, mx = 0;
+    for (int k = threadIdx.x; k < K; k += blockDim.x) {
+        const uint32_t c = static_cast<uint32_t>(counts[k]);
+        empty += c == 0u;
+        mx = c > mx ? c : mx;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        empty += __shfl_xor_sync(0xffffffffu, empty, o);
+        mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    }
+    if ((threadIdx.x & 31) == 0) {
+        e_red[threadIdx.x >> 5] = empty;
+        m_red[threadIdx.x >> 5] = mx;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        for (int w = 1; w < static_cast<int>(blockDim.x >> 5); ++w) {
+            empty += e_red[w];
+            mx = max(mx, m_red[w]);
+        }
+        out[0] = empty;
+        out[1] = mx;
+    }
+}
+}  // namespace
+
+cudaError_t launch_cluster_stats(const int32_t *counts, int K, uint32_t *out, cudaStream_t st) {
+    cluster_stats_kernel<<<1, 1024, 0, st>>>(counts, K, out);
+    note_launch();
+    return cudaGetLastError();
+}
+
 }  // namespace fk

@@ -37,7 +37,8 @@ class FkTiming(ctypes.Structure):
                 ("ms_assign", ctypes.c_double), ("ms_sort", ctypes.c_double),
                 ("ms_update", ctypes.c_double), ("iterations", ctypes.c_int),
                 ("launches", ctypes.c_int), ("ms_assign_mma", ctypes.c_double),
-                ("screened", ctypes.c_int)]
+                ("screened", ctypes.c_int), ("empty_clusters", ctypes.c_int),
+                ("max_cluster", ctypes.c_int), ("fallback_rows", ctypes.c_int)]
 
 
 class FkSearchTiming(ctypes.Structure):

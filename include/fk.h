@@ -101,6 +101,11 @@ typedef struct fk_timing {
                              alone (the single-product screening pass on the screened
                              route, else the assign kernel)                           */
     int screened;      /* iterations that took the screened route                      */
+    int empty_clusters; /* last iteration: clusters that received no point (kept their
+                           previous centroid)                                           */
+    int max_cluster;    /* last iteration: points in the largest cluster                */
+    int fallback_rows;  /* last iteration, screened route: rows sent to the three-product
+                           pass (0 when the iteration was not screened)                 */
 } fk_timing;
 
 /* Human-readable name of a status code (static string, never NULL). */

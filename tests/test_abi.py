@@ -159,3 +159,24 @@ def test_ivf_search_host_checks(fk):
     s1 = fk.ivf_search_workspace(1000, 8, 64, 100, 8, 10, device="meta").numel()
     s2 = fk.ivf_search_workspace(2000, 8, 64, 100, 8, 10, device="meta").numel()
     assert s2 > s1 > 1000 * 8 * 10 * 12
+
+
+def test_fault_injection_workspace_needs_no_device(fk):
+    """FK_FAULT=workspace (read when the library is first used, so in a child process):
+    every workspace check fails with FK_ERR_WORKSPACE, before any device work."""
+    import subprocess
+    import sys
+    code = (
+        "import ctypes, sys\n"
+        f"sys.path.insert(0, {ROOT!r})\n"
+        "from exact_lloyd_means_b200 import fk\n"
+        "lib = fk._lib\n"
+        "r1 = lib.fk_assign(16, 0, 100, 8, 16, 4, 16, None, 256, 1 << 30, None)\n"
+        "r2 = lib.fk_lloyd(16, 0, 100, 8, 4, 0, 1, 16, 16, None, None, None, None, 256, 1 << 30, None)\n"
+        "print(r1, r2)\n")
+    env = dict(os.environ, FK_FAULT="workspace")
+    out = subprocess.run([sys.executable, "-c", code], env=env, capture_output=True, text=True,
+                         timeout=300)
+    assert out.returncode == 0, out.stderr
+    r1, r2 = (int(x) for x in out.stdout.split())
+    assert r1 == fk.FK_ERR_WORKSPACE and r2 == fk.FK_ERR_WORKSPACE

@@ -8,6 +8,8 @@ Parity rules (written here, applied in every test):
   objective  relative error <= 1e-5.
 Inputs reach the GPU from the generator or from the oracle (lockstep); nothing computed on
 the GPU is ever handed to the oracle."""
+import os
+
 import numpy as np
 import pytest
 import torch
@@ -518,3 +520,52 @@ def test_screened_assign_edge_cases(case):
     assert label_mismatches(lab, ref, ties) == 0, f"ties={int(ties.sum())}"
     if case == "k_equals_n":
         assert (lab == np.arange(20000)).all()
+
+
+def test_fk_lloyd_reports_cluster_statistics():
+    """fk_timing's last-iteration statistics: empty clusters and the largest cluster agree
+    with the returned counts; the screened route's fallback count is within [0, N]."""
+    m = fk()
+    N, d, K = 40000, 256, 300
+    X, _, _ = gaussian_mixture(N, d, 200, centers="normal", sigma=0.3, seed=61)
+    C0 = X[init_indices(N, K, 61)].float().contiguous()
+    C0[:5] = 1e3  # far away: these clusters stay empty
+    Xg, C = X.to(DEV), C0.to(DEV)
+    labels = torch.empty(N, dtype=torch.int32, device=DEV)
+    counts = torch.empty(K, dtype=torch.int32, device=DEV)
+    ws = m.workspace(N, d, K, torch.float32, "l2")
+    _, tm = m.fk_lloyd(Xg, C, 3, labels, ws, counts=counts, timing=True)
+    c = counts.cpu().numpy()
+    assert tm["empty_clusters"] == int((c == 0).sum()) >= 5
+    assert tm["max_cluster"] == int(c.max())
+    assert 0 <= tm["fallback_rows"] <= N
+    assert tm["screened"] in (0, 3)
+    if tm["screened"] == 0:
+        assert tm["fallback_rows"] == 0
+
+
+def test_fault_injection_launch_fails_before_device_work():
+    """FK_FAULT=launch (in a child process): fk_lloyd and fk_ivf_search return FK_ERR_CUDA
+    and launch nothing."""
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    code = (
+        "import sys, torch\n"
+        f"sys.path.insert(0, {root!r})\n"
+        "from exact_lloyd_means_b200 import fk\n"
+        "X = torch.randn(4096, 64, device='cuda'); C = X[:16].clone()\n"
+        "lab = torch.empty(4096, dtype=torch.int32, device='cuda')\n"
+        "ws = fk.workspace(4096, 64, 16)\n"
+        "n0 = fk.launch_count()\n"
+        "try:\n"
+        "    fk.fk_lloyd(X, C, 2, lab, ws)\n"
+        "    print('no error')\n"
+        "except fk.FkError as e:\n"
+        "    print(e.status, fk.launch_count() - n0)\n")
+    env = dict(os.environ, FK_FAULT="launch")
+    out = subprocess.run([sys.executable, "-c", code], env=env, capture_output=True, text=True,
+                         timeout=600)
+    assert out.returncode == 0, out.stderr
+    status, launched = (int(x) for x in out.stdout.split())
+    assert status == fk().FK_ERR_CUDA and launched == 0
