@@ -78,6 +78,8 @@ __global__ void __launch_bounds__(kSortThreads)
     upsweep_kernel(const int32_t *__restrict__ keys, int64_t n, int shift, int bits, int K,
                    uint32_t *__restrict__ hist, int64_t nblocks, uint32_t *__restrict__ err,
                    int check) {
+    pdl_wait();
+    pdl_trigger();
     extern __shared__ uint32_t wh[];
     const int bins = 1 << bits;
     for (int i = threadIdx.x; i < kWarps * bins; i += blockDim.x) wh[i] = 0;
@@ -123,6 +125,8 @@ __device__ __forceinline__ uint32_t block_exclusive_scan_1024(uint32_t v, uint32
 // One block (1024 threads) per digit: exclusive scan of hist[b][0..nblocks).
 __global__ void __launch_bounds__(1024)
     scan_rows_kernel(uint32_t *__restrict__ hist, int64_t nblocks, uint32_t *__restrict__ dtot) {
+    pdl_wait();
+    pdl_trigger();
     __shared__ uint32_t sh[64];
     uint32_t *row = hist + static_cast<int64_t>(blockIdx.x) * nblocks;
     const int64_t per = (nblocks + blockDim.x - 1) / blockDim.x;
@@ -186,6 +190,8 @@ __global__ void __launch_bounds__(kSortThreads)
                      int32_t *__restrict__ kout, int32_t *__restrict__ vout, int64_t n,
                      int shift, int bits, int K, const uint32_t *__restrict__ hist,
                      const uint32_t *__restrict__ dtot, int64_t nblocks) {
+    pdl_wait();
+    pdl_trigger();
     extern __shared__ uint32_t sm[];
     const int bins = 1 << bits;
     const uint32_t mask = bins - 1;
@@ -268,6 +274,8 @@ __global__ void __launch_bounds__(kSortThreads)
 __global__ void single_cluster_kernel(const int32_t *__restrict__ labels, int64_t n,
                                       int32_t *__restrict__ kout, int32_t *__restrict__ vout,
                                       uint32_t *__restrict__ err) {
+    pdl_wait();
+    pdl_trigger();
     for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
          i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
         if (labels[i] != 0) err[1] = 1u;
@@ -280,6 +288,8 @@ __global__ void single_cluster_kernel(const int32_t *__restrict__ labels, int64_
 // every k in (skeys[i-1], skeys[i]], so each entry is written exactly once.
 __global__ void csr_offsets_kernel(const int32_t *__restrict__ skeys, int64_t n, int K,
                                    int32_t *__restrict__ offsets) {
+    pdl_wait();
+    pdl_trigger();
     for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i <= n;
          i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
         const int prev = i == 0 ? -1 : skeys[i - 1];
@@ -304,7 +314,8 @@ cudaError_t launch_sort_csr(const int32_t *labels, int64_t N, int K, const SortP
                             const int32_t **perm, uint32_t *err, cudaStream_t st) {
     if (sp.passes == 0) {
         int32_t *vo = perm_out ? perm_out : vals0;
-        single_cluster_kernel<<<grid_cap(N, 256), 256, 0, st>>>(labels, N, keys0, vo, err);
+        launch_pdl(single_cluster_kernel, dim3(grid_cap(N, 256)), dim3(256), 0, st, labels, N,
+                   keys0, vo, err);
         note_launch();
         *sorted_keys = keys0;
         *perm = vo;
@@ -330,14 +341,16 @@ cudaError_t launch_sort_csr(const int32_t *labels, int64_t N, int K, const SortP
         int32_t *vb[2] = {vals0, vals1};
         for (int p = 0; p < sp.passes; ++p) {
             const int shift = p * sp.bits;
-            upsweep_kernel<<<static_cast<unsigned>(sp.nblocks), kSortThreads, up_smem, st>>>(
-                kin, N, shift, sp.bits, K, hist, sp.nblocks, err, p == 0 ? 1 : 0);
+            launch_pdl(upsweep_kernel, dim3(static_cast<unsigned>(sp.nblocks)), dim3(kSortThreads),
+                       up_smem, st, kin, N, shift, sp.bits, K, hist, sp.nblocks, err,
+                       p == 0 ? 1 : 0);
             note_launch();
-            scan_rows_kernel<<<bins, 1024, 0, st>>>(hist, sp.nblocks, dtot);
+            launch_pdl(scan_rows_kernel, dim3(bins), dim3(1024), 0, st, hist, sp.nblocks, dtot);
             note_launch();
             int32_t *vo = (p == sp.passes - 1 && perm_out) ? perm_out : vb[p & 1];
-            downsweep_kernel<<<static_cast<unsigned>(sp.nblocks), kSortThreads, dn_smem, st>>>(
-                kin, vin, kb[p & 1], vo, N, shift, sp.bits, K, hist, dtot, sp.nblocks);
+            launch_pdl(downsweep_kernel, dim3(static_cast<unsigned>(sp.nblocks)),
+                       dim3(kSortThreads), dn_smem, st, kin, vin, kb[p & 1], vo, N, shift,
+                       sp.bits, K, hist, dtot, sp.nblocks);
             note_launch();
             kin = kb[p & 1];
             vin = vo;
@@ -345,7 +358,8 @@ cudaError_t launch_sort_csr(const int32_t *labels, int64_t N, int K, const SortP
         *sorted_keys = kin;
         *perm = vin;
     }
-    csr_offsets_kernel<<<grid_cap(N + 1, 256), 256, 0, st>>>(*sorted_keys, N, K, offsets);
+    launch_pdl(csr_offsets_kernel, dim3(grid_cap(N + 1, 256)), dim3(256), 0, st, *sorted_keys, N,
+               K, offsets);
     note_launch();
     return cudaGetLastError();
 }

@@ -104,6 +104,8 @@ __global__ void __launch_bounds__(kRowWarps * 32, 3)
                     double *__restrict__ sums_out, double *__restrict__ pieces,
                     int32_t *__restrict__ pkeys, double *__restrict__ jpart,
                     uint32_t *__restrict__ err) {
+    pdl_wait();
+    pdl_trigger();
     using RV = RowVec<BF16>;
     constexpr int B = RV::kBatch;
     constexpr int SL = RV::kSlice;
@@ -295,6 +297,8 @@ __global__ void __launch_bounds__(kUpdWarps * 32, 3)
                     const float *__restrict__ C_used, float *__restrict__ C_new,
                     double *__restrict__ sums_out, double *__restrict__ pieces,
                     int32_t *__restrict__ pkeys, double *__restrict__ jpart) {
+    pdl_wait();
+    pdl_trigger();
     using RV = RegRowVec<BF16>;
     using V = typename RV::T;
     constexpr int B = RV::kBatch;
@@ -513,6 +517,8 @@ __global__ void __launch_bounds__(kUpdWarps * 32)
                       int32_t *__restrict__ kout, int64_t nunits, int64_t span, int d,
                       int dcov, const int32_t *__restrict__ offsets, float *__restrict__ C_new,
                       double *__restrict__ sums_out) {
+    pdl_wait();
+    pdl_trigger();
     __shared__ int32_t s_key[kUpdWarps][2 * kGroup];
     const int wib = threadIdx.x >> 5;
     const int64_t u = static_cast<int64_t>(blockIdx.x) * kUpdWarps + wib;
@@ -570,6 +576,8 @@ __global__ void __launch_bounds__(256)
                               const double *__restrict__ pin, const int32_t *__restrict__ kin,
                               int64_t nslots, double *__restrict__ pout,
                               int32_t *__restrict__ kout, int64_t span, int dcov) {
+    pdl_wait();
+    pdl_trigger();
     if (blockIdx.x == 0) {
         if (objective == nullptr) return;
         __shared__ double sh[256];
@@ -633,15 +641,14 @@ cudaError_t run_levels(const void *X, bool bf16, int64_t N, int d, const UpdPlan
     const dim3 rblock(kRowWarps * 32);
     dim3 rgrid(static_cast<unsigned>(ceil_div(up.nwarps, kRowWarps)), up.ncolblk);
     if (bf16)
-        seg_rows_regs_kernel<true><<<dim3(static_cast<unsigned>(ceil_div(up.nwarps, kUpdWarps)),
-                                          up.ncolblk),
-                                     dim3(kUpdWarps * 32), 0, st>>>(
-            X, N, d, up.rows, up.nwarps, up.dcov, skeys, perm, offsets, C_used, C_new, sums_out,
-            pa, ka, jpart);
+        launch_pdl(seg_rows_regs_kernel<true>,
+                   dim3(static_cast<unsigned>(ceil_div(up.nwarps, kUpdWarps)), up.ncolblk),
+                   dim3(kUpdWarps * 32), 0, st, X, N, d, up.rows, up.nwarps, up.dcov, skeys, perm,
+                   offsets, C_used, C_new, sums_out, pa, ka, jpart);
     else
-        seg_rows_kernel<false><<<rgrid, rblock, kRowSmem, st>>>(
-            X, N, d, up.rows, up.nwarps, up.dcov, skeys, perm, offsets, C_used, C_new, sums_out,
-            pa, ka, jpart, err);
+        launch_pdl(seg_rows_kernel<false>, rgrid, rblock, kRowSmem, st, X, N, d, up.rows,
+                   up.nwarps, up.dcov, skeys, perm, offsets, C_used, C_new, sums_out, pa, ka,
+                   jpart, err);
     note_launch();
     const dim3 block(kUpdWarps * 32);
     int64_t units = up.nwarps;
@@ -662,8 +669,8 @@ cudaError_t run_levels(const void *X, bool bf16, int64_t N, int d, const UpdPlan
             break;
         }
         dim3 g2(static_cast<unsigned>(ceil_div(nunits, kUpdWarps)), up.ncolblk);
-        seg_pieces_kernel<<<g2, block, 0, st>>>(pin, kin, units * 2, pout, kout, nunits, span, d,
-                                                up.dcov, offsets, C_new, sums_out);
+        launch_pdl(seg_pieces_kernel, g2, block, 0, st, pin, kin, units * 2, pout, kout, nunits,
+                   span, d, up.dcov, offsets, C_new, sums_out);
         note_launch();
         units = nunits;
         double *tp = pin;
@@ -697,9 +704,10 @@ cudaError_t launch_update(const void *X, fk_dtype dtype, int64_t N, int d, int K
     const int64_t cap = static_cast<int64_t>(device_sm_count()) * 16;
     if (fgrid > cap) fgrid = cap;
     const int nfin = fl.pending ? up.ncolblk : 0;
-    finalize_objective_kernel<<<static_cast<unsigned>(1 + nfin + fgrid), 256, 0, st>>>(
-        offsets, K, d, C_old, C_new, counts, sums_out, jpart, up.nwarps * up.ncolblk,
-        objective, nfin, fl.pin, fl.kin, fl.nslots, fl.pout, fl.kout, fl.span, up.dcov);
+    launch_pdl(finalize_objective_kernel, dim3(static_cast<unsigned>(1 + nfin + fgrid)),
+               dim3(256), 0, st, offsets, K, d, C_old, C_new, counts, sums_out, jpart,
+               up.nwarps * up.ncolblk, objective, nfin, fl.pin, fl.kin, fl.nslots, fl.pout,
+               fl.kout, fl.span, up.dcov);
     note_launch();
     return cudaGetLastError();
 }
