@@ -436,8 +436,11 @@ __global__ void __launch_bounds__(kUpdWarps * 32, 3)
 // Level L >= 2: one warp per group of kGroup units of the previous level (2 piece slots
 // each), one 128-column block per grid.y.  `span` = sorted positions covered by one unit
 // of THIS level.  The group's slot keys are staged in shared memory first and the pieces
-// are read 8 slots at a time, so the loop is not a chain of dependent loads.
-// One warp: unit u of a combine level, column block cb; sk = the warp's shared key slots.
+// are read 8 slots at a time, so the loop is not a chain of dependent loads.  The CSR
+// bounds of every slot's cluster are staged with the keys, so finishing a cluster waits on
+// no global load.
+// One warp: unit u of a combine level, column block cb; sk = the warp's shared key slots,
+// sb = their clusters' [lo, hi) sorted positions.
 __device__ __forceinline__ void pieces_unit(const double *__restrict__ pin,
                                             const int32_t *__restrict__ kin, int64_t nslots_in,
                                             double *__restrict__ pout,
@@ -445,22 +448,27 @@ __device__ __forceinline__ void pieces_unit(const double *__restrict__ pin,
                                             int64_t span, int d, int dcov,
                                             const int32_t *__restrict__ offsets,
                                             float *__restrict__ C_new,
-                                            double *__restrict__ sums_out, int32_t *sk) {
+                                            double *__restrict__ sums_out, int32_t *sk,
+                                            int2 *sb) {
     constexpr int S = 2 * kGroup;
     constexpr int B = 8;
     const int lane = threadIdx.x & 31;
     const int col = cb * 128 + lane * 4;
     const int64_t s0 = u * S;
     const int ns = static_cast<int>((s0 + S < nslots_in ? s0 + S : nslots_in) - s0);
-    for (int j = lane; j < ns; j += 32) sk[j] = kin[s0 + j];
+    for (int j = lane; j < ns; j += 32) {
+        const int k = kin[s0 + j];
+        sk[j] = k;
+        if (k >= 0) sb[j] = make_int2(offsets[k], offsets[k + 1]);
+    }
     __syncwarp();
 
     double acc[4] = {0.0, 0.0, 0.0, 0.0};
-    int cur = -1, first = -1, slot1 = -1;
+    int cur = -1, curq = -1, first = -1, slot1 = -1;
     bool first_done = false;
 
     auto flush = [&](int k) {
-        const int64_t lo = offsets[k], hi = offsets[k + 1];
+        const int64_t lo = sb[curq].x, hi = sb[curq].y;
         const bool done = (lo / span) == ((hi - 1) / span);
         if (k == first) first_done = done;
         if (done) {
@@ -496,6 +504,7 @@ __device__ __forceinline__ void pieces_unit(const double *__restrict__ pin,
                 if (cur >= 0) flush(cur);
                 if (cur < 0) first = k;
                 cur = k;
+                curq = q;
                 acc[0] = acc[1] = acc[2] = acc[3] = 0.0;
             }
             acc[0] += va[j].x;
@@ -520,11 +529,12 @@ __global__ void __launch_bounds__(kUpdWarps * 32)
     pdl_wait();
     pdl_trigger();
     __shared__ int32_t s_key[kUpdWarps][2 * kGroup];
+    __shared__ int2 s_bnd[kUpdWarps][2 * kGroup];
     const int wib = threadIdx.x >> 5;
     const int64_t u = static_cast<int64_t>(blockIdx.x) * kUpdWarps + wib;
     if (u >= nunits) return;
     pieces_unit(pin, kin, nslots_in, pout, kout, u, blockIdx.y, span, d, dcov, offsets, C_new,
-                sums_out, s_key[wib]);
+                sums_out, s_key[wib], s_bnd[wib]);
 }
 
 // Combine W shards of a data-parallel iteration, in shard order: c_k = (sum_w S_wk) /
@@ -581,8 +591,18 @@ __global__ void __launch_bounds__(256)
     if (blockIdx.x == 0) {
         if (objective == nullptr) return;
         __shared__ double sh[256];
+        // each thread adds its strided entries in index order; eight loads are issued
+        // before the eight additions so the loop is not a chain of dependent loads
         double s = 0.0;
-        for (int64_t i = threadIdx.x; i < n; i += 256) s += part[i];
+        int64_t i = threadIdx.x;
+        for (; i + 7 * 256 < n; i += 8 * 256) {
+            double v[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) v[j] = part[i + j * 256];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) s += v[j];
+        }
+        for (; i < n; i += 256) s += part[i];
         sh[threadIdx.x] = s;
         __syncthreads();
         for (int o = 128; o > 0; o >>= 1) {
@@ -594,9 +614,10 @@ __global__ void __launch_bounds__(256)
     }
     if (static_cast<int>(blockIdx.x) <= nfin) {
         __shared__ int32_t s_key[2 * kGroup];
+        __shared__ int2 s_bnd[2 * kGroup];
         if (threadIdx.x < 32)
             pieces_unit(pin, kin, nslots, pout, kout, 0, static_cast<int>(blockIdx.x) - 1, span,
-                        d, dcov, offsets, C_new, sums_out, s_key);
+                        d, dcov, offsets, C_new, sums_out, s_key, s_bnd);
         return;
     }
     const int lane = threadIdx.x & 31;
