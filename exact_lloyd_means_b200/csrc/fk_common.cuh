@@ -19,8 +19,12 @@ constexpr int kAug = 16;  // bf16 columns of the norm-folding K step (32-byte ro
 
 // ----------------------------------------------------------------- sort tiling
 constexpr int kSortThreads = 256;
-constexpr int kSortItems = 16;
-constexpr int kSortTile = kSortThreads * kSortItems;  // keys per block
+constexpr int kSortItems = 16;      // keys per thread of a large-input tile
+constexpr int kSortItemsSmall = 4;  // keys per thread when the input is small
+constexpr int kSortTile = kSortThreads * kSortItems;  // keys per block (the largest tile)
+// Inputs up to this size use the small tile: four times the blocks, each with a quarter of
+// the serial work, which is what bounds a sort whose tiles all fit on the GPU at once.
+constexpr int64_t kSortSmallN = int64_t(1) << 22;
 // digit width bound: 256 bins (a tile's per-digit bookkeeping grows with the bins, so two
 // narrow passes beat one wide one from about 1024 bins)
 constexpr int kSortMaxBits = 8;
@@ -131,6 +135,7 @@ struct SortPlan {
     int nbits = 0;
     int passes = 0;
     int bits = 0;  // digit width per pass (last pass may use fewer significant bits)
+    int items = kSortItems;  // keys per thread; a block's tile is kSortThreads * items keys
     int64_t nblocks = 0;
 };
 
@@ -139,7 +144,8 @@ inline SortPlan sort_plan(int64_t N, int K) {
     p.nbits = key_bits(K);
     p.passes = p.nbits == 0 ? 0 : static_cast<int>(ceil_div(p.nbits, kSortMaxBits));
     p.bits = p.passes == 0 ? 0 : static_cast<int>(ceil_div(p.nbits, p.passes));
-    p.nblocks = ceil_div(N, kSortTile);
+    p.items = N <= kSortSmallN ? kSortItemsSmall : kSortItems;
+    p.nblocks = ceil_div(N, static_cast<int64_t>(kSortThreads) * p.items);
     return p;
 }
 

@@ -7,9 +7,10 @@
 //
 // A stable least-significant-digit radix sort with digits of up to 8 bits (one pass for
 // K <= 256, two for K <= 65536, three beyond), whose ranks need no atomics:
-//   upsweep   : each block of 4096 keys counts its digits into per-warp histograms in
-//               shared memory (shared-memory atomic adds: the counts do not depend on
-//               their order);
+//   upsweep   : each block of 4096 keys (1024 when the input has at most 4M keys, so that
+//               small sorts run on four times the blocks) counts its digits into per-warp
+//               histograms in shared memory (shared-memory atomic adds: the counts do not
+//               depend on their order);
 //   scan      : one block per digit scans the per-block counts (digit-major order) and
 //               stores the digit total;
 //   downsweep : each block recounts, turns warp counts into offsets within its tile
@@ -33,22 +34,23 @@ __device__ __forceinline__ uint32_t lanemask_lt() {
     return m;
 }
 
-// Check labels (first pass) and count digits of one 4096-key tile into per-warp
-// histograms wh[kWarps][bins].  Each thread reads 16 consecutive keys with 16-byte loads
-// and adds them with shared-memory atomics: counts do not depend on the order of the
-// additions, so the result is the same on every run.
+// Check labels (first pass) and count digits of one tile of kSortThreads * ITEMS keys
+// into per-warp histograms wh[kWarps][bins].  Each thread reads ITEMS consecutive keys
+// with 16-byte loads and adds them with shared-memory atomics: counts do not depend on the
+// order of the additions, so the result is the same on every run.
+template <int ITEMS>
 __device__ __forceinline__ void count_tile(const int32_t *__restrict__ keys, int64_t n,
                                            int64_t tile0, int shift, uint32_t mask, int K,
                                            uint32_t *__restrict__ err, int check,
                                            uint32_t *wh, int bins) {
     const int warp = threadIdx.x >> 5;
     uint32_t *h = wh + warp * bins;
-    const int64_t start = tile0 + static_cast<int64_t>(threadIdx.x) * kSortItems;
+    const int64_t start = tile0 + static_cast<int64_t>(threadIdx.x) * ITEMS;
     // labels need only 4-byte alignment: 16-byte loads only from a 16-byte aligned array
-    // (start is a multiple of 16 keys, so then every load below is aligned)
+    // (start is a multiple of 4 keys, so then every load below is aligned)
     const bool vec = (reinterpret_cast<uintptr_t>(keys) & 15u) == 0u;
 #pragma unroll
-    for (int j = 0; j < kSortItems; j += 4) {
+    for (int j = 0; j < ITEMS; j += 4) {
         const int64_t idx = start + j;
         int k4[4];
         if (vec && idx + 3 < n) {
@@ -74,6 +76,7 @@ __device__ __forceinline__ void count_tile(const int32_t *__restrict__ keys, int
     }
 }
 
+template <int ITEMS>
 __global__ void __launch_bounds__(kSortThreads)
     upsweep_kernel(const int32_t *__restrict__ keys, int64_t n, int shift, int bits, int K,
                    uint32_t *__restrict__ hist, int64_t nblocks, uint32_t *__restrict__ err,
@@ -84,7 +87,8 @@ __global__ void __launch_bounds__(kSortThreads)
     const int bins = 1 << bits;
     for (int i = threadIdx.x; i < kWarps * bins; i += blockDim.x) wh[i] = 0;
     __syncthreads();
-    count_tile(keys, n, static_cast<int64_t>(blockIdx.x) * kSortTile, shift, bins - 1, K, err,
+    count_tile<ITEMS>(keys, n, static_cast<int64_t>(blockIdx.x) * (kSortThreads * ITEMS), shift,
+                      bins - 1, K, err,
                check, wh, bins);
     __syncthreads();
     for (int b = threadIdx.x; b < bins; b += blockDim.x) {
@@ -182,9 +186,10 @@ __device__ __forceinline__ void block_scan_bins(const uint32_t *cnt, uint32_t *o
     __syncthreads();
 }
 
-// Scatter one 4096-key tile: the keys are first placed in shared memory in digit order
+// Scatter one tile of kSortThreads * ITEMS keys: the keys are first placed in shared memory in digit order
 // (stable: warps, then steps, then lanes follow the index order), then each digit's run is
 // written to its global place with consecutive threads writing consecutive addresses.
+template <int ITEMS>
 __global__ void __launch_bounds__(kSortThreads)
     downsweep_kernel(const int32_t *__restrict__ kin, const int32_t *__restrict__ vin,
                      int32_t *__restrict__ kout, int32_t *__restrict__ vout, int64_t n,
@@ -199,8 +204,9 @@ __global__ void __launch_bounds__(kSortThreads)
     uint32_t *lstart = wh + kWarps * bins;  // [bins] this tile's digit starts (local)
     uint32_t *gstart = lstart + bins;       // [bins] where this tile's digit run goes
     uint32_t *bcnt = gstart + bins;         // [bins] scratch
-    int32_t *skey = reinterpret_cast<int32_t *>(bcnt + bins);  // [kSortTile]
-    int32_t *sval = skey + kSortTile;                           // [kSortTile]
+    constexpr int kTile = kSortThreads * ITEMS;
+    int32_t *skey = reinterpret_cast<int32_t *>(bcnt + bins);  // [kTile]
+    int32_t *sval = skey + kTile;                               // [kTile]
     __shared__ uint32_t part[kSortThreads];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -210,8 +216,8 @@ __global__ void __launch_bounds__(kSortThreads)
     for (int b = threadIdx.x; b < bins; b += blockDim.x)
         gstart[b] += hist[static_cast<int64_t>(b) * nblocks + blockIdx.x];
 
-    const int64_t tile0 = static_cast<int64_t>(blockIdx.x) * kSortTile;
-    count_tile(kin, n, tile0, shift, mask, K, nullptr, 0, wh, bins);
+    const int64_t tile0 = static_cast<int64_t>(blockIdx.x) * kTile;
+    count_tile<ITEMS>(kin, n, tile0, shift, mask, K, nullptr, 0, wh, bins);
     __syncthreads();
     for (int b = threadIdx.x; b < bins; b += blockDim.x) {
         uint32_t t = 0;
@@ -232,8 +238,8 @@ __global__ void __launch_bounds__(kSortThreads)
 
     uint32_t *h = wh + warp * bins;
     const uint32_t lt = lanemask_lt();
-    const int64_t base = tile0 + static_cast<int64_t>(warp) * (32 * kSortItems);
-    for (int step = 0; step < kSortItems; ++step) {
+    const int64_t base = tile0 + static_cast<int64_t>(warp) * (32 * ITEMS);
+    for (int step = 0; step < ITEMS; ++step) {
         const int64_t idx = base + step * 32 + lane;
         const bool valid = idx < n;
         int key = 0, val = 0;
@@ -260,7 +266,7 @@ __global__ void __launch_bounds__(kSortThreads)
     __syncthreads();
 
     const int64_t left = n - tile0;
-    const int cnt = static_cast<int>(left < kSortTile ? left : kSortTile);
+    const int cnt = static_cast<int>(left < kTile ? left : kTile);
     for (int i = threadIdx.x; i < cnt; i += blockDim.x) {
         const int32_t key = skey[i];
         const uint32_t digit = (static_cast<uint32_t>(key) >> shift) & mask;
@@ -321,35 +327,42 @@ cudaError_t launch_sort_csr(const int32_t *labels, int64_t N, int K, const SortP
         *perm = vo;
     } else {
         const int bins = 1 << sp.bits;
+        const int tile = kSortThreads * sp.items;
         const size_t up_smem = sizeof(uint32_t) * kWarps * bins;
         const size_t dn_smem =
-            sizeof(uint32_t) * ((kWarps + 3) * bins) + sizeof(int32_t) * 2 * kSortTile;
+            sizeof(uint32_t) * ((kWarps + 3) * bins) + sizeof(int32_t) * 2 * tile;
         static bool attr = false;
         if (!attr) {
-            const int maxb = 1 << kSortMaxBits;
-            cudaFuncSetAttribute(upsweep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 static_cast<int>(sizeof(uint32_t) * kWarps * maxb));
-            cudaFuncSetAttribute(downsweep_kernel,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 static_cast<int>(sizeof(uint32_t) * (kWarps + 3) * maxb +
-                                                  sizeof(int32_t) * 2 * kSortTile));
+            const int up_max = static_cast<int>(sizeof(uint32_t) * kWarps * (1 << kSortMaxBits));
+            const int dn_max = static_cast<int>(sizeof(uint32_t) * (kWarps + 3) * (1 << kSortMaxBits) +
+                                                sizeof(int32_t) * 2 * kSortTile);
+            cudaFuncSetAttribute(upsweep_kernel<kSortItems>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, up_max);
+            cudaFuncSetAttribute(upsweep_kernel<kSortItemsSmall>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, up_max);
+            cudaFuncSetAttribute(downsweep_kernel<kSortItems>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, dn_max);
+            cudaFuncSetAttribute(downsweep_kernel<kSortItemsSmall>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, dn_max);
             attr = true;
         }
+        const bool small = sp.items == kSortItemsSmall;
         const int32_t *kin = labels;
         const int32_t *vin = nullptr;
         int32_t *kb[2] = {keys0, keys1};
         int32_t *vb[2] = {vals0, vals1};
         for (int p = 0; p < sp.passes; ++p) {
             const int shift = p * sp.bits;
-            launch_pdl(upsweep_kernel, dim3(static_cast<unsigned>(sp.nblocks)), dim3(kSortThreads),
-                       up_smem, st, kin, N, shift, sp.bits, K, hist, sp.nblocks, err,
-                       p == 0 ? 1 : 0);
+            const dim3 grid(static_cast<unsigned>(sp.nblocks));
+            launch_pdl(small ? upsweep_kernel<kSortItemsSmall> : upsweep_kernel<kSortItems>, grid,
+                       dim3(kSortThreads), up_smem, st, kin, N, shift, sp.bits, K, hist,
+                       sp.nblocks, err, p == 0 ? 1 : 0);
             note_launch();
             launch_pdl(scan_rows_kernel, dim3(bins), dim3(1024), 0, st, hist, sp.nblocks, dtot);
             note_launch();
             int32_t *vo = (p == sp.passes - 1 && perm_out) ? perm_out : vb[p & 1];
-            launch_pdl(downsweep_kernel, dim3(static_cast<unsigned>(sp.nblocks)),
-                       dim3(kSortThreads), dn_smem, st, kin, vin, kb[p & 1], vo, N, shift,
+            launch_pdl(small ? downsweep_kernel<kSortItemsSmall> : downsweep_kernel<kSortItems>,
+                       grid, dim3(kSortThreads), dn_smem, st, kin, vin, kb[p & 1], vo, N, shift,
                        sp.bits, K, hist, dtot, sp.nblocks);
             note_launch();
             kin = kb[p & 1];
