@@ -34,6 +34,7 @@ namespace fk {
 namespace {
 
 constexpr int kGroup = kUpdGroup;  // units of level L-1 per unit of level L
+static_assert((kGroup & (kGroup - 1)) == 0, "combine spans must stay powers of two");
 
 // Write the mean of a finished cluster: C_new[k][col..col+3] = acc / cnt.
 __device__ __forceinline__ void store_mean(float *C_new, int64_t k, int d, int col,
@@ -452,6 +453,9 @@ __device__ __forceinline__ void pieces_unit(const double *__restrict__ pin,
                                             int2 *sb) {
     constexpr int S = 2 * kGroup;
     constexpr int B = 8;
+    // span is a power of two (a power-of-two row count times powers of kGroup), so the
+    // "same unit" test below is a shift rather than a 64-bit division
+    const int span_log2 = __ffsll(static_cast<long long>(span)) - 1;
     const int lane = threadIdx.x & 31;
     const int col = cb * 128 + lane * 4;
     const int64_t s0 = u * S;
@@ -469,7 +473,7 @@ __device__ __forceinline__ void pieces_unit(const double *__restrict__ pin,
 
     auto flush = [&](int k) {
         const int64_t lo = sb[curq].x, hi = sb[curq].y;
-        const bool done = (lo / span) == ((hi - 1) / span);
+        const bool done = (lo >> span_log2) == ((hi - 1) >> span_log2);
         if (k == first) first_done = done;
         if (done) {
             if (col < d) store_done(C_new, sums_out, k, d, col, acc, static_cast<double>(hi - lo));
