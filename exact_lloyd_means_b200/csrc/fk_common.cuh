@@ -19,7 +19,7 @@ constexpr int kAug = 16;  // bf16 columns of the norm-folding K step (32-byte ro
 
 // ----------------------------------------------------------------- sort tiling
 constexpr int kSortThreads = 256;
-constexpr int kSortItems = 16;      // keys per thread of a large-input tile
+constexpr int kSortItems = 8;       // keys per thread of a large-input tile
 constexpr int kSortItemsSmall = 4;  // keys per thread when the input is small
 constexpr int kSortTile = kSortThreads * kSortItems;  // keys per block (the largest tile)
 // Inputs up to this size use the small tile: four times the blocks, each with a quarter of

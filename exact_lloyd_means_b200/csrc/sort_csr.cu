@@ -186,38 +186,81 @@ __device__ __forceinline__ void block_scan_bins(const uint32_t *cnt, uint32_t *o
     __syncthreads();
 }
 
-// Scatter one tile of kSortThreads * ITEMS keys: the keys are first placed in shared memory in digit order
-// (stable: warps, then steps, then lanes follow the index order), then each digit's run is
-// written to its global place with consecutive threads writing consecutive addresses.
+// Scatter one tile of kSortThreads * ITEMS keys.  Every lane holds ITEMS keys (positions
+// base + 32*step + lane of its warp's stretch) and ranks each among the keys of equal digit
+// in its warp, in position order: the peers come from one ballot per digit bit, the rank
+// is the count of earlier peers plus the warp's running count of that digit.  The warps'
+// digit counts then give each warp's base per digit (digits in order, then warps in
+// order), the keys are placed in shared memory at base + rank, and each digit's run is
+// written to its global place with consecutive threads on consecutive addresses.  Ranks
+// follow the index order, so the sort is stable and its output unique.
 template <int ITEMS>
 __global__ void __launch_bounds__(kSortThreads)
     downsweep_kernel(const int32_t *__restrict__ kin, const int32_t *__restrict__ vin,
-                     int32_t *__restrict__ kout, int32_t *__restrict__ vout, int64_t n,
+                     int32_t *__restrict__ kout, int32_t *__restrict__ vout, int64_t n64,
                      int shift, int bits, int K, const uint32_t *__restrict__ hist,
                      const uint32_t *__restrict__ dtot, int64_t nblocks) {
     pdl_wait();
     pdl_trigger();
+    constexpr int kTile = kSortThreads * ITEMS;
     extern __shared__ uint32_t sm[];
     const int bins = 1 << bits;
     const uint32_t mask = bins - 1;
-    uint32_t *wh = sm;                      // [kWarps][bins] counts, then local offsets
+    uint32_t *wh = sm;                      // [kWarps][bins] digit counts, then warp bases
     uint32_t *lstart = wh + kWarps * bins;  // [bins] this tile's digit starts (local)
-    uint32_t *gstart = lstart + bins;       // [bins] where this tile's digit run goes
-    uint32_t *bcnt = gstart + bins;         // [bins] scratch
-    constexpr int kTile = kSortThreads * ITEMS;
+    uint32_t *gofs = lstart + bins;         // [bins] global start minus local start
+    uint32_t *bcnt = gofs + bins;           // [bins] scratch
     int32_t *skey = reinterpret_cast<int32_t *>(bcnt + bins);  // [kTile]
     int32_t *sval = skey + kTile;                               // [kTile]
     __shared__ uint32_t part[kSortThreads];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    // the callers bound n below 2^31, so positions (and a last tile running past n) fit
+    // in 32 unsigned bits
+    const uint32_t n = static_cast<uint32_t>(n64);
+    const uint32_t tile0 = blockIdx.x * static_cast<uint32_t>(kTile);
+    const uint32_t base = tile0 + static_cast<uint32_t>(warp * (32 * ITEMS));
+
+    // this lane's keys and values, loaded up front (-1 marks a position past n)
+    int key[ITEMS], val[ITEMS];
+#pragma unroll
+    for (int step = 0; step < ITEMS; ++step) {
+        const uint32_t idx = base + static_cast<uint32_t>(step * 32 + lane);
+        key[step] = -1;
+        val[step] = 0;
+        if (idx < n) {
+            const int k = kin[idx];
+            key[step] = k < 0 ? 0 : (k >= K ? K - 1 : k);
+            val[step] = vin ? vin[idx] : static_cast<int32_t>(idx);
+        }
+    }
 
     for (int i = threadIdx.x; i < kWarps * bins; i += blockDim.x) wh[i] = 0;
-    // global digit bases: exclusive scan of the digit totals
-    block_scan_bins(dtot, gstart, bins, part);
+    // global digit bases: exclusive scan of the digit totals (its barriers also order the
+    // zeroing above before the counting below)
+    block_scan_bins(dtot, gofs, bins, part);
     for (int b = threadIdx.x; b < bins; b += blockDim.x)
-        gstart[b] += hist[static_cast<int64_t>(b) * nblocks + blockIdx.x];
+        gofs[b] += hist[static_cast<int64_t>(b) * nblocks + blockIdx.x];
 
-    const int64_t tile0 = static_cast<int64_t>(blockIdx.x) * kTile;
-    count_tile<ITEMS>(kin, n, tile0, shift, mask, K, nullptr, 0, wh, bins);
+    uint32_t *h = wh + warp * bins;
+    const uint32_t lt = lanemask_lt();
+    uint32_t rank[ITEMS];
+#pragma unroll
+    for (int step = 0; step < ITEMS; ++step) {
+        const bool valid = key[step] >= 0;
+        const uint32_t digit = (static_cast<uint32_t>(key[step]) >> shift) & mask;
+        uint32_t peers = __ballot_sync(0xffffffffu, valid);
+        for (int b = 0; b < bits; ++b) {
+            const bool on = (digit >> b) & 1u;
+            const uint32_t bal = __ballot_sync(0xffffffffu, on);
+            peers &= on ? bal : ~bal;
+        }
+        uint32_t r = 0;
+        if (valid) r = h[digit] + __popc(peers & lt);
+        __syncwarp();
+        if (valid && lane == __ffs(peers) - 1) h[digit] += __popc(peers);
+        __syncwarp();
+        rank[step] = r;
+    }
     __syncthreads();
     for (int b = threadIdx.x; b < bins; b += blockDim.x) {
         uint32_t t = 0;
@@ -233,45 +276,29 @@ __global__ void __launch_bounds__(kSortThreads)
             wh[w * bins + b] = run;
             run += t;
         }
+        gofs[b] -= lstart[b];  // modulo 2^32: gofs + local position is the global one
     }
     __syncthreads();
-
-    uint32_t *h = wh + warp * bins;
-    const uint32_t lt = lanemask_lt();
-    const int64_t base = tile0 + static_cast<int64_t>(warp) * (32 * ITEMS);
+#pragma unroll
     for (int step = 0; step < ITEMS; ++step) {
-        const int64_t idx = base + step * 32 + lane;
-        const bool valid = idx < n;
-        int key = 0, val = 0;
-        if (valid) {
-            key = kin[idx];
-            key = key < 0 ? 0 : (key >= K ? K - 1 : key);
-            val = vin ? vin[idx] : static_cast<int32_t>(idx);
+        if (key[step] >= 0) {
+            const uint32_t digit = (static_cast<uint32_t>(key[step]) >> shift) & mask;
+            const uint32_t pos = h[digit] + rank[step];
+            skey[pos] = key[step];
+            sval[pos] = val[step];
         }
-        const uint32_t digit = (static_cast<uint32_t>(key) >> shift) & mask;
-        const uint32_t vmask = __ballot_sync(0xffffffffu, valid);
-        uint32_t peers = 0, pos = 0;
-        if (valid) {
-            peers = __match_any_sync(vmask, digit);
-            pos = h[digit] + __popc(peers & lt);
-        }
-        __syncwarp();
-        if (valid) {
-            if (lane == __ffs(peers) - 1) h[digit] += __popc(peers);
-            skey[pos] = key;
-            sval[pos] = val;
-        }
-        __syncwarp();
     }
     __syncthreads();
 
-    const int64_t left = n - tile0;
-    const int cnt = static_cast<int>(left < kTile ? left : kTile);
+    // a plan sized for a larger input (a streamed chunk's capacity) launches blocks whose
+    // tile starts at or past n: they hold no keys and write nothing
+    const int64_t left = static_cast<int64_t>(n) - static_cast<int64_t>(tile0);
+    const int cnt = left <= 0 ? 0 : static_cast<int>(left < kTile ? left : kTile);
     for (int i = threadIdx.x; i < cnt; i += blockDim.x) {
-        const int32_t key = skey[i];
-        const uint32_t digit = (static_cast<uint32_t>(key) >> shift) & mask;
-        const int64_t g = static_cast<int64_t>(gstart[digit]) + (i - static_cast<int>(lstart[digit]));
-        kout[g] = key;
+        const int32_t k = skey[i];
+        const uint32_t digit = (static_cast<uint32_t>(k) >> shift) & mask;
+        const uint32_t g = gofs[digit] + static_cast<uint32_t>(i);
+        kout[g] = k;
         vout[g] = sval[i];
     }
 }

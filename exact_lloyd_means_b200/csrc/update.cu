@@ -13,12 +13,13 @@
 //              contiguous bytes of a row per warp, read as 16-byte vectors across the lanes,
 //              eight rows in flight), adds them in position order in fp64 and,
 //              whenever the cluster id changes, either finishes the cluster (all of it
-//              lies in this chunk: mean = sum / count, rounded once to fp32) or emits a
-//              "piece" (the chunk's first or last cluster, which continues outside).  The
-//              same pass accumulates the objective sum ||x - c_used[label]||^2 in fp64.
-//   level L>1: groups of 64 consecutive units of the previous level are reduced the same
+//              lies in this chunk, which the keys just outside the chunk tell: mean =
+//              sum / count, rounded once to fp32) or emits a "piece" (the chunk's first or
+//              last cluster, which continues outside).  The same pass accumulates the
+//              objective sum ||x - c_used[label]||^2 in fp64.
+//   level L>1: groups of 16 consecutive units of the previous level are reduced the same
 //              way over their pieces, in piece order.  A cluster is finished at the first
-//              level whose unit (R * 64^(L-1) positions) contains all of it, so a
+//              level whose unit (R * 16^(L-1) positions) contains all of it, so a
 //              cluster with millions of points is split over thousands of warps at
 //              level 1 and finished after a few levels with short, parallel sums.
 //   finalize : counts from the CSR offsets; empty clusters copy C_old bit for bit.
@@ -100,7 +101,7 @@ template <bool BF16>
 __global__ void __launch_bounds__(kRowWarps * 32, 3)
     seg_rows_kernel(const void *__restrict__ X, int64_t N, int d, int R, int64_t nwarps,
                     int dcov, const int32_t *__restrict__ skeys,
-                    const int32_t *__restrict__ perm, const int32_t *__restrict__ offsets,
+                    const int32_t *__restrict__ perm,
                     const float *__restrict__ C_used, float *__restrict__ C_new,
                     double *__restrict__ sums_out, double *__restrict__ pieces,
                     int32_t *__restrict__ pkeys, double *__restrict__ jpart,
@@ -138,6 +139,8 @@ __global__ void __launch_bounds__(kRowWarps * 32, 3)
         sk[j] = skeys[p0 + j];
         si[j] = perm[p0 + j];
     }
+    const int k_before = p0 > 0 ? skeys[p0 - 1] : -1;
+    const int k_after = p1 < N ? skeys[p1] : -1;
     __syncwarp();
 
     const uint8_t *Xb = static_cast<const uint8_t *>(X);
@@ -156,13 +159,16 @@ __global__ void __launch_bounds__(kRowWarps * 32, 3)
     double acc[4] = {0.0, 0.0, 0.0, 0.0};
     float cu[4] = {0.f, 0.f, 0.f, 0.f};
     double jacc = 0.0;
-    int cur = -1, first = -1, slot1 = -1;
+    int cur = -1, first = -1, slot1 = -1, ncur = 0;
     bool ok = true;
 
+    // A cluster is finished inside this warp unless it continues from the position before
+    // p0 or into the one at p1 (positions are sorted, so only the first and the last
+    // cluster can); its count is then the rows added here.
+    auto finished = [&](int k) { return k != k_before && k != k_after; };
     auto flush = [&](int k) {
-        const int64_t lo = offsets[k], hi = offsets[k + 1];
-        if (lo >= p0 && hi <= p1) {
-            if (colv) store_done(C_new, sums_out, k, d, col, acc, static_cast<double>(hi - lo));
+        if (finished(k)) {
+            if (colv) store_done(C_new, sums_out, k, d, col, acc, static_cast<double>(ncur));
         } else {
             const int slot = (k == first) ? 0 : 1;
             if (slot == 1) slot1 = k;
@@ -173,6 +179,7 @@ __global__ void __launch_bounds__(kRowWarps * 32, 3)
         if (cur >= 0) flush(cur);
         if (cur < 0) first = k;
         cur = k;
+        ncur = 0;
         acc[0] = acc[1] = acc[2] = acc[3] = 0.0;
         if (colv) {
             const float4 c = *reinterpret_cast<const float4 *>(C_used + int64_t(k) * d + col);
@@ -229,10 +236,12 @@ __global__ void __launch_bounds__(kRowWarps * 32, 3)
 #pragma unroll
             for (int e = 0; e < 4; ++e) acc[e] += static_cast<double>(xs[0][e]);
             jacc += static_cast<double>(jr[0]);
+            ncur += nb;
         } else {
             for (int j = 0; j < nb; ++j) {
                 const int k = sk[b + j];
                 if (k != cur) start(k);
+                ++ncur;
                 float x[4] = {0.f, 0.f, 0.f, 0.f};
                 if (colv) RV::load(base + j * SL, x);
                 float t = 0.f;
@@ -260,9 +269,7 @@ __global__ void __launch_bounds__(kRowWarps * 32, 3)
     if (cur >= 0) flush(cur);
     if (cb == 0 && lane == 0) {
         // slot 0 holds the first cluster if it was not finished here; slot 1 the last
-        const int64_t lo = offsets[first], hi = offsets[first + 1];
-        const bool first_done = lo >= p0 && hi <= p1;
-        pkeys[w * 2 + 0] = first_done ? -1 : first;
+        pkeys[w * 2 + 0] = finished(first) ? -1 : first;
         pkeys[w * 2 + 1] = slot1;
     }
 #pragma unroll
@@ -294,7 +301,7 @@ template <bool BF16>
 __global__ void __launch_bounds__(kUpdWarps * 32, 3)
     seg_rows_regs_kernel(const void *__restrict__ X, int64_t N, int d, int R, int64_t nwarps,
                     int dcov, const int32_t *__restrict__ skeys,
-                    const int32_t *__restrict__ perm, const int32_t *__restrict__ offsets,
+                    const int32_t *__restrict__ perm,
                     const float *__restrict__ C_used, float *__restrict__ C_new,
                     double *__restrict__ sums_out, double *__restrict__ pieces,
                     int32_t *__restrict__ pkeys, double *__restrict__ jpart) {
@@ -321,18 +328,23 @@ __global__ void __launch_bounds__(kUpdWarps * 32, 3)
         sk[j] = skeys[p0 + j];
         si[j] = perm[p0 + j];
     }
+    const int k_before = p0 > 0 ? skeys[p0 - 1] : -1;
+    const int k_after = p1 < N ? skeys[p1] : -1;
     __syncwarp();
 
     const V *Xv = static_cast<const V *>(X);
     double acc[4] = {0.0, 0.0, 0.0, 0.0};
     float cu[4] = {0.f, 0.f, 0.f, 0.f};
     double jacc = 0.0;
-    int cur = -1, first = -1, slot1 = -1;
+    int cur = -1, first = -1, slot1 = -1, ncur = 0;
 
+    // A cluster is finished inside this warp unless it continues from the position before
+    // p0 or into the one at p1 (positions are sorted, so only the first and the last
+    // cluster can); its count is then the rows added here.
+    auto finished = [&](int k) { return k != k_before && k != k_after; };
     auto flush = [&](int k) {
-        const int64_t lo = offsets[k], hi = offsets[k + 1];
-        if (lo >= p0 && hi <= p1) {
-            if (colv) store_done(C_new, sums_out, k, d, col, acc, static_cast<double>(hi - lo));
+        if (finished(k)) {
+            if (colv) store_done(C_new, sums_out, k, d, col, acc, static_cast<double>(ncur));
         } else {
             const int slot = (k == first) ? 0 : 1;
             if (slot == 1) slot1 = k;
@@ -343,6 +355,7 @@ __global__ void __launch_bounds__(kUpdWarps * 32, 3)
         if (cur >= 0) flush(cur);
         if (cur < 0) first = k;
         cur = k;
+        ncur = 0;
         acc[0] = acc[1] = acc[2] = acc[3] = 0.0;
         if (colv) {
             const float4 c = *reinterpret_cast<const float4 *>(C_used + int64_t(k) * d + col);
@@ -391,12 +404,14 @@ __global__ void __launch_bounds__(kUpdWarps * 32, 3)
 #pragma unroll
             for (int e = 0; e < 4; ++e) acc[e] += static_cast<double>(xs[0][e]);
             jacc += static_cast<double>(jr[0]);
+            ncur += nb;
         } else {
 #pragma unroll
             for (int j = 0; j < B; ++j) {
                 if (j < nb) {
                     const int k = sk[b + j];
                     if (k != cur) start(k);
+                    ++ncur;
                     float x[4];
                     RV::unpack(buf[j], x);
                     float t = 0.f;
@@ -424,9 +439,7 @@ __global__ void __launch_bounds__(kUpdWarps * 32, 3)
     if (cur >= 0) flush(cur);
     if (cb == 0 && lane == 0) {
         // slot 0 holds the first cluster if it was not finished here; slot 1 the last
-        const int64_t lo = offsets[first], hi = offsets[first + 1];
-        const bool first_done = lo >= p0 && hi <= p1;
-        pkeys[w * 2 + 0] = first_done ? -1 : first;
+        pkeys[w * 2 + 0] = finished(first) ? -1 : first;
         pkeys[w * 2 + 1] = slot1;
     }
 #pragma unroll
@@ -669,11 +682,11 @@ cudaError_t run_levels(const void *X, bool bf16, int64_t N, int d, const UpdPlan
         launch_pdl(seg_rows_regs_kernel<true>,
                    dim3(static_cast<unsigned>(ceil_div(up.nwarps, kUpdWarps)), up.ncolblk),
                    dim3(kUpdWarps * 32), 0, st, X, N, d, up.rows, up.nwarps, up.dcov, skeys, perm,
-                   offsets, C_used, C_new, sums_out, pa, ka, jpart);
+                   C_used, C_new, sums_out, pa, ka, jpart);
     else
         launch_pdl(seg_rows_kernel<false>, rgrid, rblock, kRowSmem, st, X, N, d, up.rows,
-                   up.nwarps, up.dcov, skeys, perm, offsets, C_used, C_new, sums_out, pa, ka,
-                   jpart, err);
+                   up.nwarps, up.dcov, skeys, perm, C_used, C_new, sums_out, pa, ka, jpart,
+                   err);
     note_launch();
     const dim3 block(kUpdWarps * 32);
     int64_t units = up.nwarps;
