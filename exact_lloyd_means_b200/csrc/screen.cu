@@ -120,8 +120,20 @@ __global__ void rerank_kernel(const float *__restrict__ X32, const uint16_t *__r
     const int q = lane / L, sub = lane % L;
     const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
     const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+    // Most rows need only their candidate slots, so a warp keeps the slots of its next
+    // kPrefetch rows in flight while it handles the current one.
+    constexpr int kPrefetch = 4;
+    auto slots = [&](int64_t r) {
+        return (r < N && lane < kCandPerRow) ? cand[r * kCandPerRow + lane] : -1;
+    };
+    int ring[kPrefetch];
+#pragma unroll
+    for (int t = 0; t < kPrefetch; ++t) ring[t] = slots(warp + t * nwarps);
     for (int64_t i = warp; i < N; i += nwarps) {
-        const int c = lane < kCandPerRow ? cand[i * kCandPerRow + lane] : -1;
+        const int c = ring[0];
+#pragma unroll
+        for (int t = 0; t + 1 < kPrefetch; ++t) ring[t] = ring[t + 1];
+        ring[kPrefetch - 1] = slots(i + kPrefetch * nwarps);
         const bool ovf = __any_sync(0xffffffffu, c == kCandOverflow);
         const uint32_t valid = __ballot_sync(0xffffffffu, c >= 0 && c < K);
         if (ovf || valid == 0u) {
