@@ -22,8 +22,8 @@ constexpr int kSortThreads = 256;
 constexpr int kSortItems = 8;       // keys per thread of a large-input tile
 constexpr int kSortItemsSmall = 4;  // keys per thread when the input is small
 constexpr int kSortTile = kSortThreads * kSortItems;  // keys per block (the largest tile)
-// Inputs up to this size use the small tile: four times the blocks, each with a quarter of
-// the serial work, which is what bounds a sort whose tiles all fit on the GPU at once.
+// Inputs up to this size use the small tile: twice the blocks, each with half the serial
+// work, which is what bounds a sort whose tiles all fit on the GPU at once.
 constexpr int64_t kSortSmallN = int64_t(1) << 22;
 // digit width bound: 256 bins (a tile's per-digit bookkeeping grows with the bins, so two
 // narrow passes beat one wide one from about 1024 bins)

@@ -7,18 +7,19 @@
 //
 // A stable least-significant-digit radix sort with digits of up to 8 bits (one pass for
 // K <= 256, two for K <= 65536, three beyond), whose ranks need no atomics:
-//   upsweep   : each block of 4096 keys (1024 when the input has at most 4M keys, so that
-//               small sorts run on four times the blocks) counts its digits into per-warp
+//   upsweep   : each block of 2048 keys (1024 when the input has at most 4M keys, so that
+//               small sorts run on twice the blocks) counts its digits into per-warp
 //               histograms in shared memory (shared-memory atomic adds: the counts do not
 //               depend on their order);
 //   scan      : one block per digit scans the per-block counts (digit-major order) and
 //               stores the digit total;
-//   downsweep : each block recounts, turns warp counts into offsets within its tile
-//               (digits in order, then warps in order), places every key in shared memory
-//               at offset + rank, rank = #equal digits before it in the warp (popc of the
-//               match mask below the lane), then writes each digit's run of the tile to
-//               its global place (digits, then blocks in order) with consecutive threads
-//               on consecutive addresses.  Keys are visited in index order, so the sort is
+//   downsweep : each lane loads its keys once and ranks each among the equal digits of its
+//               warp (peers from one ballot per digit bit, rank = earlier peers + the
+//               warp's running count); the warps' counts give each warp's base per digit
+//               (digits in order, then warps in order), every key goes to shared memory at
+//               base + rank, and each digit's run of the tile is written to its global
+//               place (digits, then blocks in order) with consecutive threads on
+//               consecutive addresses.  Ranks follow the index order, so the sort is
 //               stable and the output is unique.
 // offsets[k] = first sorted position whose key is >= k, written once per k.
 #include "fk_common.cuh"
