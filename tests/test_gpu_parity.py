@@ -110,6 +110,30 @@ def test_update_single_cluster_is_global_mean():
     assert (g["perm"] == np.arange(50000)).all() and g["offsets"].tolist() == [0, 50000]
 
 
+@pytest.mark.parametrize("K", [256, 300, 65536])
+def test_update_sort_large_input_tiles(K):
+    """Inputs above 4M keys take the radix sort's large tiles (8 keys per thread); N leaves
+    a ragged last tile.  K = 256 sorts in one 8-bit pass, 300 in two 5-bit passes, 65536
+    in two 8-bit passes.  perm, counts and offsets against the oracle's stable CSR (a long
+    run of one label and an empty cluster included), centroids against its means."""
+    N, d = (1 << 22) + 12345, 4
+    rng = np.random.default_rng(K)
+    labels = rng.integers(0, K, N, dtype=np.int32)
+    labels[1000:300000] = 7
+    labels[labels == K - 1] = 0
+    X = torch.randn(N, d, generator=torch.Generator().manual_seed(K))
+    C_old = torch.randn(K, d, generator=torch.Generator().manual_seed(K + 1))
+    counts, offsets, perm = oracle.csr(labels, K)
+    C_ref = oracle.update(X, labels, C_old.numpy())
+    g = gpu_update(X.to(DEV), labels, C_old.to(DEV))
+    assert (g["counts"] == counts).all()
+    assert (g["offsets"] == offsets).all()
+    assert (g["perm"] == perm).all()
+    nonempty = counts > 0
+    assert not nonempty.all()
+    assert centroid_rel_err(g["C_new"][nonempty], C_ref[nonempty]) <= CENTROID_TOL
+
+
 @pytest.mark.parametrize("case", ["tiny_f32", "tiny_bf16", "cosine_768"])
 def test_lockstep_lloyd_matches_oracle(case):
     """Lockstep: each iteration the GPU assigns with the oracle's centroids and updates
