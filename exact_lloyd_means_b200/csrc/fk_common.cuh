@@ -32,7 +32,7 @@ constexpr int kSortMaxBits = 8;
 // ----------------------------------------------------------------- update tiling
 constexpr int kUpdWarps = 8;          // warps per block of the update kernels
 constexpr int kUpdGroup = 16;         // units of one combine level per unit of the next
-constexpr int kUpdMinRows = 32;       // smallest chunk of sorted positions per warp
+constexpr int kUpdMinRows = 64;       // smallest chunk of sorted positions per warp
 constexpr int kUpdMaxRows = 256;      // largest chunk
 constexpr int64_t kUpdTargetWarps = 148 * 64;  // enough warps to cover the GPU twice
 
