@@ -8,7 +8,7 @@
 //
 // B200 design:
 //   level 1  : the sorted order [0, N) is cut into fixed chunks of R positions (a power of
-//              two, 32..256, chosen from N), one per warp and 128-column block, independent
+//              two, 64..256, chosen from N), one per warp and 128-column block, independent
 //              of where clusters start.  A warp gathers its rows through perm (512
 //              contiguous bytes of a row per warp, read as 16-byte vectors across the lanes,
 //              eight rows in flight), adds them in position order in fp64 and,
