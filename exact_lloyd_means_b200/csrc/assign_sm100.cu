@@ -1042,13 +1042,10 @@ cudaError_t launch_assign_cfg(const AssignArgs &a, const CUtensorMap (&tA)[2],
                               const CUtensorMap (&tB)[2], const CUtensorMap &tC,
                               cudaStream_t st) {
     using Cfg = AsgCfg<NP, RES>;
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(assign_kernel<NP, RES>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             Cfg::kSmemBytes);
+    static std::atomic<uint64_t> smem_set{0};
+    {
+        const cudaError_t e = smem_opt_in(assign_kernel<NP, RES>, Cfg::kSmemBytes, smem_set);
         if (e != cudaSuccess) return e;
-        attr_set = true;
     }
     const int64_t nmb = ceil_div(a.N, kBM);
     const int64_t sms = device_sm_count();

@@ -2,6 +2,7 @@
 // and the C-ABI host code of libfk.
 #pragma once
 
+#include <atomic>
 #include <cstddef>
 #include <cstdint>
 #include <utility>
@@ -466,6 +467,21 @@ inline SearchLayout search_layout(int64_t nq, int d, int nlist, int nprobe, int 
 cudaError_t launch_cluster_stats(const int32_t *counts, int K, uint32_t *out, cudaStream_t st);
 
 int device_sm_count();
+
+// Raise a kernel's dynamic shared-memory limit to `bytes` on the current device.  The
+// attribute belongs to the device, so each call site records the devices it has set it
+// on, one bit per ordinal in `done` (ordinals from 64 up set it on every call).
+template <typename Kernel>
+cudaError_t smem_opt_in(Kernel kernel, int bytes, std::atomic<uint64_t> &done) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const uint64_t bit = dev < 64 ? uint64_t(1) << dev : 0;
+    if (bit != 0 && (done.load(std::memory_order_relaxed) & bit) != 0) return cudaSuccess;
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess && bit != 0) done.fetch_or(bit, std::memory_order_relaxed);
+    return e;
+}
 
 // Kernels launched by this host thread since the last reset (fk_lloyd reports it).
 extern thread_local long g_launches;

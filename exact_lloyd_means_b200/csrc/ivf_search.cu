@@ -1682,13 +1682,11 @@ cudaError_t launch_ivf_select(const double *D, const uint32_t *I, int64_t ld, in
     SelArgs a{D, I, ld, L, m, out_id, out_dist, ldo};
     if (L <= kSelCache) {
         const size_t smem = static_cast<size_t>(L) * (sizeof(uint64_t) + sizeof(uint32_t));
-        static bool attr = false;
-        if (!attr) {
-            cudaFuncSetAttribute(select_rows_kernel<true>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 static_cast<int>(kSelCache * (sizeof(uint64_t) + sizeof(uint32_t))));
-            attr = true;
-        }
+        static std::atomic<uint64_t> smem_set{0};
+        const cudaError_t e = smem_opt_in(
+            select_rows_kernel<true>,
+            static_cast<int>(kSelCache * (sizeof(uint64_t) + sizeof(uint32_t))), smem_set);
+        if (e != cudaSuccess) return e;
         select_rows_kernel<true><<<static_cast<unsigned>(rows), kSelThreads, smem, st>>>(a);
     } else {
         select_rows_kernel<false><<<static_cast<unsigned>(rows), kSelThreads, 0, st>>>(a);
@@ -1717,12 +1715,11 @@ cudaError_t launch_ivf_coarse_rerank(const float *Vs, int64_t ldv, int64_t rows,
     while (P < L) P <<= 1;
     const size_t smem = static_cast<size_t>(P) * (sizeof(double) + sizeof(uint32_t)) +
                         static_cast<size_t>(L) * sizeof(uint32_t);
-    static bool attr = false;
-    if (!attr) {
-        cudaFuncSetAttribute(coarse_rerank_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(kCoarseMaxL * (sizeof(double) + 2 * sizeof(uint32_t))));
-        attr = true;
-    }
+    static std::atomic<uint64_t> smem_set{0};
+    const cudaError_t e = smem_opt_in(
+        coarse_rerank_kernel,
+        static_cast<int>(kCoarseMaxL * (sizeof(double) + 2 * sizeof(uint32_t))), smem_set);
+    if (e != cudaSuccess) return e;
     coarse_rerank_kernel<<<static_cast<unsigned>(rows), kCoarseThreads, smem, st>>>(a);
     note_launch();
     return cudaGetLastError();
@@ -1736,10 +1733,12 @@ cudaError_t launch_ivf_fine_scr(const uint16_t *Qp, int64_t nq, const uint16_t *
                                 uint32_t *Sp, float *Slost, const float *cut, cudaStream_t st) {
     FineArgs a{Qp, nq, Xp, N, dp, qn, xn, offsets, pair_sorted, pair_off, items, nitems,
                item_ctr, nprobe, Sv, Sp, Slost, cut};
-    static int occ = 0;
+    static std::atomic<uint64_t> smem_set{0};
+    const cudaError_t e =
+        smem_opt_in(ivf_fine_scr_kernel, static_cast<int>(sizeof(FineSmem)), smem_set);
+    if (e != cudaSuccess) return e;
+    static int occ = 0;  // blocks per SM: the same on every B200
     if (occ == 0) {
-        cudaFuncSetAttribute(ivf_fine_scr_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(sizeof(FineSmem)));
         if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, ivf_fine_scr_kernel, kTThreads,
                                                           sizeof(FineSmem)) != cudaSuccess ||
             occ < 1)
@@ -1794,13 +1793,12 @@ cudaError_t launch_ivf_query_rerank(const float *Sv, const uint32_t *Sp, const f
     while (P2 < L) P2 <<= 1;
     const size_t smem = static_cast<size_t>(P2) * (sizeof(double) + 2 * sizeof(uint32_t)) +
                         static_cast<size_t>(L) * sizeof(uint32_t);
-    static bool attr = false;
-    if (!attr) {
-        cudaFuncSetAttribute(query_rerank_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(kSearchScrMaxProbe * kScrList *
-                                              (sizeof(double) + 3 * sizeof(uint32_t))));
-        attr = true;
-    }
+    static std::atomic<uint64_t> smem_set{0};
+    const cudaError_t e = smem_opt_in(query_rerank_kernel,
+                                      static_cast<int>(kSearchScrMaxProbe * kScrList *
+                                                       (sizeof(double) + 3 * sizeof(uint32_t))),
+                                      smem_set);
+    if (e != cudaSuccess) return e;
     query_rerank_kernel<<<static_cast<unsigned>(nq), kQThreads, smem, st>>>(a);
     note_launch();
     return cudaGetLastError();

@@ -359,21 +359,10 @@ cudaError_t launch_sort_csr(const int32_t *labels, int64_t N, int K, const SortP
         const size_t up_smem = sizeof(uint32_t) * kWarps * bins;
         const size_t dn_smem =
             sizeof(uint32_t) * ((kWarps + 3) * bins) + sizeof(int32_t) * 2 * tile;
-        static bool attr = false;
-        if (!attr) {
-            const int up_max = static_cast<int>(sizeof(uint32_t) * kWarps * (1 << kSortMaxBits));
-            const int dn_max = static_cast<int>(sizeof(uint32_t) * (kWarps + 3) * (1 << kSortMaxBits) +
-                                                sizeof(int32_t) * 2 * kSortTile);
-            cudaFuncSetAttribute(upsweep_kernel<kSortItems>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, up_max);
-            cudaFuncSetAttribute(upsweep_kernel<kSortItemsSmall>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, up_max);
-            cudaFuncSetAttribute(downsweep_kernel<kSortItems>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, dn_max);
-            cudaFuncSetAttribute(downsweep_kernel<kSortItemsSmall>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, dn_max);
-            attr = true;
-        }
+        // the largest tile and digit need 27 KB, under the default 48 KB limit: no opt-in
+        static_assert(sizeof(uint32_t) * (kWarps + 3) * (1 << kSortMaxBits) +
+                              sizeof(int32_t) * 2 * kSortTile <= 48 * 1024,
+                      "sort shared memory above the default limit");
         const bool small = sp.items == kSortItemsSmall;
         const int32_t *kin = labels;
         const int32_t *vin = nullptr;

@@ -670,11 +670,11 @@ cudaError_t run_levels(const void *X, bool bf16, int64_t N, int d, const UpdPlan
                        int32_t *ka,
                        double *pb, int32_t *kb, double *jpart, uint32_t *err,
                        cudaStream_t st, FinalLevel *final_level) {
-    static bool attr = false;
-    if (!attr) {
-        cudaFuncSetAttribute(seg_rows_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(kRowSmem));
-        attr = true;
+    static std::atomic<uint64_t> smem_set{0};
+    {
+        const cudaError_t e =
+            smem_opt_in(seg_rows_kernel<false>, static_cast<int>(kRowSmem), smem_set);
+        if (e != cudaSuccess) return e;
     }
     const dim3 rblock(kRowWarps * 32);
     dim3 rgrid(static_cast<unsigned>(ceil_div(up.nwarps, kRowWarps)), up.ncolblk);
