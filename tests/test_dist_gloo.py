@@ -105,3 +105,66 @@ def test_sharded_lloyd_equals_single_process_oracle(world):
             assert abs(objs[t] - ref["J"][t]) <= 1e-9 * ref["J"][t]
         assert (counts == ref["counts"][-1]).all()
     assert np.array_equal(res[0][1], res[1][1])  # bit-identical across ranks
+
+
+def _failing_rank(rank, world, port, out, mode):
+    """Rank 1 fails in its local step of the second iteration, between exchanges (no
+    collective in flight): mode "raise" leaves (its process ends), mode "stall" stays alive
+    but never reaches the exchange.  Rank 0 carries on into its next exchange."""
+    os.environ["OMP_NUM_THREADS"] = "1"
+    import sys
+    import time
+    from datetime import timedelta
+    sys.path.insert(0, ROOT)
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank,
+                            world_size=world, timeout=timedelta(seconds=10))
+    from exact_lloyd_means_b200.dist import LocalOps, lloyd_sharded
+    X, C0 = _data()
+    bounds = np.linspace(0, X.shape[0], world + 1).astype(int)
+    Xl = X[bounds[rank]:bounds[rank + 1]].contiguous()
+    ops = _stand_in_ops()
+    calls = {"n": 0}
+
+    def assign(Xa, C):
+        calls["n"] += 1
+        if rank == 1 and calls["n"] == 2:
+            if mode == "stall":
+                time.sleep(25.0)
+            raise RuntimeError("injected: rank 1 lost its device")
+        return ops.assign(Xa, C)
+
+    t0 = time.monotonic()
+    try:
+        lloyd_sharded(Xl, C0.clone(), 4, LocalOps(assign, ops.partial, ops.finalize))
+        out.put((rank, "finished", time.monotonic() - t0))
+    except Exception as e:  # noqa: BLE001 - what ended the rank is the result
+        out.put((rank, type(e).__name__ + ": " + str(e)[:120], time.monotonic() - t0))
+    # no destroy_process_group: the peer is gone, and a collective would wait on it
+
+
+@pytest.mark.parametrize("mode", ["raise", "stall"])
+def test_sharded_lloyd_lost_rank_ends_peer_with_error(mode):
+    """Failure detection on the data-parallel path without a GPU: when one rank leaves or
+    stalls between steps, the other's next exchange ends with an error (a closed
+    connection, or the process group's 10 s timeout) instead of waiting for good, and the
+    survivor reports no result."""
+    world = 2
+    ctx = mp.get_context("spawn")
+    out = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_failing_rank, args=(r, world, port, out, mode))
+             for r in range(world)]
+    for p in procs:
+        p.start()
+    res = {}
+    for _ in range(world):
+        rank, what, secs = out.get(timeout=120)
+        res[rank] = (what, secs)
+    for p in procs:
+        p.join(timeout=60)
+        if p.is_alive():
+            p.kill()
+    print(res)
+    assert res[1][0].startswith("RuntimeError: injected")
+    assert res[0][0] != "finished"      # the survivor did not carry on alone
+    assert res[0][1] < 22.0            # it gave up before the stalled peer woke (25 s)
