@@ -31,10 +31,12 @@ TIE_TAU = 1e-4
 
 
 def lib():
-    """Load (building first if needed) the compiled oracle."""
+    """Load (building first if needed) the compiled oracle.  FK_ORACLE_LIB, when set,
+    names another build of the same sources to load instead: the mutation test points the
+    pins at deliberately broken copies with it."""
     global _lib
     if _lib is None:
-        path = _build.build()
+        path = os.environ.get("FK_ORACLE_LIB") or _build.build()
         L = ctypes.CDLL(path)
         L.orc_max_threads.restype = ctypes.c_int
         L.orc_normalize_rows.argtypes = [_dp, ctypes.c_int64, ctypes.c_int]
