@@ -47,6 +47,16 @@ MUTANTS = [
     ("search_pads_with_zero_distance", "ivf_search_oracle.c",
      "dist[q * k + t] = t < klen ? kd[t] : INFINITY;",
      "dist[q * k + t] = t < klen ? kd[t] : 0.0;"),
+    ("search_pads_ids_with_zero", "ivf_search_oracle.c",
+     "ids[q * k + t] = t < klen ? ki[t] : -1;", "ids[q * k + t] = t < klen ? ki[t] : 0;"),
+    ("csr_offsets_not_accumulated", "lloyd_oracle.c",
+     "offsets[k + 1] = offsets[k] + counts[k];", "offsets[k + 1] = counts[k];"),
+    ("distance_in_expanded_form", "lloyd_oracle.c",
+     "        double t = x[j] - c[j];\n        s += t * t;\n",
+     "        s += x[j] * x[j] + c[j] * c[j] - 2.0 * x[j] * c[j];\n"),
+    ("search_distance_in_expanded_form", "ivf_search_oracle.c",
+     "        const double t = a[j] - b[j];\n        s += t * t;\n",
+     "        s += a[j] * a[j] + b[j] * b[j] - 2.0 * a[j] * b[j];\n"),
 ]
 
 

@@ -95,6 +95,28 @@ def test_assign_translation_invariant():
     assert (l0[keep] == l1[keep]).all()
 
 
+def test_distance_is_formed_from_differences():
+    """The squared distance is sum_j (x_j - c_j)^2 formed from the differences (Flash-KMeans
+    article, "它不是银弹，但切中了一个真痛点": squared L2).  On a dyadic grid, a shift of every
+    coordinate by 2^24 is exact in fp64 and so is each difference, so distances, labels, the
+    objective and the search's distances must be bit-identical before and after the shift.
+    Expanding the square (|x|^2 + |c|^2 - 2 x.c) loses about half a unit to cancellation at
+    this offset and fails this."""
+    r = _rng(16)
+    X = np.round(r.normal(size=(200, 8)) * 1024) / 1024
+    C = np.round(r.normal(size=(12, 8)) * 1024) / 1024
+    t = float(2 ** 24)
+    l0, dmin0, d2nd0 = oracle.assign(X, C)
+    l1, dmin1, d2nd1 = oracle.assign(X + t, C + t)
+    assert np.array_equal(dmin0, dmin1) and np.array_equal(d2nd0, d2nd1)
+    assert np.array_equal(l0, l1)
+    assert oracle.objective(X, C, l0) == oracle.objective(X + t, C + t, l0)
+    Q = X[:20]
+    p0, i0, g0 = oracle.ivf_search(Q, C, X, l0, nprobe=3, k=5)
+    p1, i1, g1 = oracle.ivf_search(Q + t, C + t, X + t, l0, nprobe=3, k=5)
+    assert np.array_equal(p0, p1) and np.array_equal(i0, i1) and np.array_equal(g0, g1)
+
+
 def test_tie_mask_definition():
     """A point exactly between two centroids is a tie point; one far from the bisector
     is not."""
