@@ -54,6 +54,18 @@ MUTANTS = [
     ("distance_in_expanded_form", "lloyd_oracle.c",
      "        double t = x[j] - c[j];\n        s += t * t;\n",
      "        s += x[j] * x[j] + c[j] * c[j] - 2.0 * x[j] * c[j];\n"),
+    ("assign_skips_last_centroid", "lloyd_oracle.c",
+     "for (int k = 0; k < K; ++k) {\n            double s = sqdist(",
+     "for (int k = 0; k < K - 1; ++k) {\n            double s = sqdist("),
+    ("objective_against_first_centroid", "lloyd_oracle.c",
+     "per[i] = sqdist(X + i * (int64_t)d, C + (int64_t)labels[i] * d, d);",
+     "per[i] = sqdist(X + i * (int64_t)d, C, d);"),
+    ("normalize_skips_last_column", "lloyd_oracle.c",
+     "for (int j = 0; j < d; ++j) s += x[j] * x[j];",
+     "for (int j = 0; j < d - 1; ++j) s += x[j] * x[j];"),
+    ("search_drops_last_probed_cell", "ivf_search_oracle.c",
+     "for (int t = 0; t < plen; ++t) probed[pi[t]] = 1;",
+     "for (int t = 0; t + 1 < plen; ++t) probed[pi[t]] = 1;"),
     ("search_distance_in_expanded_form", "ivf_search_oracle.c",
      "        const double t = a[j] - b[j];\n        s += t * t;\n",
      "        s += a[j] * a[j] + b[j] * b[j] - 2.0 * a[j] * b[j];\n"),
