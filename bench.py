@@ -178,6 +178,13 @@ def cpu_baseline(X_host, C0_host, metric, precision, seconds):
 # ----------------------------------------------------------------------------- arms
 
 
+def _reference_threads(oracle, world):
+    """Under torchrun (N > 1) only rank 0 runs the reference arm, but torchrun starts every
+    rank with one OpenMP thread: give rank 0 the host's cores back."""
+    if world > 1:
+        oracle.set_threads(len(os.sched_getaffinity(0)))
+
+
 def reference_arm(args, spec, rank, world):
     """The oracle timed on the host as the reference arm: each step is one Lloyd iteration
     over a bounded sample of the workload's points."""
@@ -187,6 +194,7 @@ def reference_arm(args, spec, rank, world):
     import torch
 
     import oracle
+    _reference_threads(oracle, world)
     from synth import gaussian_mixture, init_indices
     # a sample large enough that the per-step fixed costs (centroid normalisation and
     # rounding) are small next to the per-point work, yet about a second of CPU per step
@@ -784,6 +792,7 @@ def search_reference_arm(args, spec, rank, world):
     if rank != 0:
         return
     import oracle
+    _reference_threads(oracle, world)
     nprobe, k = args.search, args.topk
     Qd, one = search_cpu_sample(spec, args.cpu_seconds, args.queries)
     S = 16

@@ -39,6 +39,7 @@ def lib():
         path = os.environ.get("FK_ORACLE_LIB") or _build.build()
         L = ctypes.CDLL(path)
         L.orc_max_threads.restype = ctypes.c_int
+        L.orc_set_threads.argtypes = [ctypes.c_int]
         L.orc_normalize_rows.argtypes = [_dp, ctypes.c_int64, ctypes.c_int]
         L.orc_assign.argtypes = [_dp, ctypes.c_int64, ctypes.c_int, _dp, ctypes.c_int,
                                  _ip, _dp, _dp]
@@ -58,6 +59,12 @@ def lib():
 
 def threads() -> int:
     return lib().orc_max_threads()
+
+
+def set_threads(n: int) -> None:
+    """Threads for the oracle's parallel per-point loops (its results do not depend on
+    the count)."""
+    lib().orc_set_threads(int(n))
 
 
 def _f64(a) -> np.ndarray:

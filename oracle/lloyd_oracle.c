@@ -51,6 +51,15 @@ int orc_max_threads(void) {
 #endif
 }
 
+/* Threads for the parallel loops below (n >= 1); results do not depend on it. */
+void orc_set_threads(int n) {
+#ifdef _OPENMP
+    if (n >= 1) omp_set_num_threads(n);
+#else
+    (void)n;
+#endif
+}
+
 /* x_i <- x_i / ||x_i||, with ||x_i|| replaced by 1 when it is 0 (LEANN FlashLib guide,
  * "距离度量只有 squared L2如何支持 mips / cosine": zero-norm vectors are protected as 1). */
 void orc_normalize_rows(double *X, int64_t n, int d) {
