@@ -247,12 +247,12 @@ def fk_arm(args, spec, rank, world, dist):
     dev = torch.device("cuda", torch.cuda.current_device())
     niter = args.niter or spec.niter
     sharded = world > 1 or args.dp
-    # weak scaling: every rank holds spec.n points of its own (own seed); one k-means
-    # problem over all world * spec.n points when sharded
-    seed = spec.seed + rank
+    # weak scaling: every rank holds spec.n points of its own, drawn from the one mixture
+    # (shard = rank); one k-means problem over all world * spec.n points when sharded
+    seed = spec.seed
     X, _, _ = gaussian_mixture(spec.n, spec.d, spec.k, centers=spec.centers, sigma=spec.sigma,
                                weights=spec.weights, zipf_s=spec.zipf_s, dtype=spec.dtype,
-                               seed=seed, device=dev)
+                               seed=seed, device=dev, shard=rank)
     C0 = X[init_indices(spec.n, spec.k, seed, device=dev)].float().contiguous()
     if world > 1:
         dist.broadcast(C0, src=0)  # replicated initial centroids: rank 0's choice

@@ -73,15 +73,17 @@ def _torch_dtype(dtype: str):
 def gaussian_mixture(n: int, d: int, n_comp: int, *, centers: str = "normal",
                      sigma: float = 0.1, weights: str = "equal", zipf_s: float = 1.2,
                      dtype: str = "f32", seed: int = 0, device="cpu",
-                     chunk_rows: int = 1 << 22):
+                     chunk_rows: int = 1 << 22, shard: int = 0):
     """Return (X [n, d] fp32 or bf16, comp [n] int32 component ids, centers [n_comp, d]
-    fp32), all on `device`."""
+    fp32), all on `device`.  `shard` selects independent component and noise draws from
+    the same mixture (same centers): the points of one data-parallel rank; shard 0 is the
+    plain draw."""
     device = torch.device(device)
     cen = _centers(d, n_comp, centers, seed, device)
 
     X, comp = _draw_points(n, d, cen, sigma, weights, zipf_s, dtype,
-                           _gen(device, seed, _S_COMP), _gen(device, seed, _S_NOISE),
-                           device, chunk_rows)
+                           _gen(device, seed, _S_COMP + 1000 * shard),
+                           _gen(device, seed, _S_NOISE + 1000 * shard), device, chunk_rows)
     return X, comp, cen
 
 

@@ -45,3 +45,17 @@ def test_make_config_shapes():
     spec, X, C0, comp, cen = make_config(TINY, n=4096, k=32)
     assert X.shape == (4096, 128) and C0.shape == (32, 128) and C0.dtype == torch.float32
     assert CONFIGS[LARGE].dtype == "bf16" and CONFIGS[IVF].metric == "cosine"
+
+
+def test_shards_share_the_mixture_and_draw_their_own_points():
+    """A data-parallel rank's points (shard r) come from the same centers with their own
+    component and noise draws; shard 0 is the plain draw."""
+    X0, c0, cen0 = gaussian_mixture(4000, 16, 10, sigma=0.05, seed=3)
+    Xa, ca, cena = gaussian_mixture(4000, 16, 10, sigma=0.05, seed=3, shard=0)
+    X1, c1, cen1 = gaussian_mixture(4000, 16, 10, sigma=0.05, seed=3, shard=1)
+    assert torch.equal(X0, Xa) and torch.equal(c0, ca)
+    assert torch.equal(cen0, cen1)
+    assert not torch.equal(X0, X1) and not torch.equal(c0, c1)
+    # every shard's points sit around the shared centers
+    err = (X1 - cen1[c1.long()]).std()
+    assert abs(float(err) - 0.05) < 0.005
