@@ -1,0 +1,98 @@
+"""Host-side planning of the library, checked on the CPU: the radix sort's digits and
+tiles, the update's chunks, and the workspace layout (exact_lloyd_means_b200/csrc/
+fk_common.cuh).  A small host-only program includes the header, is built with nvcc (no
+GPU needed) and checks the invariants the kernels rely on over a grid of shapes."""
+import os
+import shutil
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+CSRC = os.path.join(ROOT, "exact_lloyd_means_b200", "csrc")
+
+PROGRAM = r"""
+#include "fk_common.cuh"
+#include <cstdio>
+using namespace fk;
+
+static int fails = 0;
+#define CHECK(c)                                                                       \
+    do {                                                                               \
+        if (!(c)) {                                                                    \
+            if (fails < 20)                                                            \
+                std::printf("FAIL %s: N=%lld K=%d d=%d\n", #c, (long long)N, K, d);    \
+            ++fails;                                                                   \
+        }                                                                              \
+    } while (0)
+
+int main() {
+    const long long Ns[] = {1, 2, 255, 256, 1023, 1024, 1025, 65536, 150001, 1 << 20,
+                            4194304, 4194305, 10000000, 16000000, 100000000, 2147483646LL};
+    const int Ks[] = {1, 2, 3, 255, 256, 257, 300, 1024, 4096, 32768, 65535, 65536, 65537,
+                      1 << 20};
+    const int ds[] = {4, 8, 64, 100, 128, 129, 256, 768, 1032};
+    int cases = 0;
+    for (long long N : Ns) {
+        for (int K : Ks) {
+            if (K > N) continue;
+            int d = 0;
+            const SortPlan p = sort_plan(N, K);
+            // digits cover exactly the bits of the largest key, with no empty pass
+            CHECK(K == 1 ? p.nbits == 0 : (1LL << p.nbits) >= K && (1LL << (p.nbits - 1)) < K);
+            CHECK(p.bits <= kSortMaxBits && p.passes * p.bits >= p.nbits);
+            CHECK(p.passes == 0 || (p.passes - 1) * p.bits < p.nbits);
+            // tiles cover [0, N) with no empty block; the last tile's end fits 32 bits
+            const long long tile = (long long)kSortThreads * p.items;
+            CHECK(p.items == (N <= kSortSmallN ? kSortItemsSmall : kSortItems));
+            CHECK(p.nblocks * tile >= N && (p.nblocks - 1) * tile < N);
+            CHECK(p.nblocks * tile <= 0xffffffffLL);
+            for (int dd : ds) {
+                d = dd;
+                const UpdPlan u = upd_plan(N, d);
+                CHECK(u.rows >= kUpdMinRows && u.rows <= kUpdMaxRows);
+                CHECK((u.rows & (u.rows - 1)) == 0);  // combine spans stay powers of two
+                CHECK(u.nwarps * u.rows >= N && (u.nwarps - 1) * u.rows < N);
+                CHECK(u.ncolblk * 128 >= d && (u.ncolblk - 1) * 128 < d);
+                CHECK(u.dcov == u.ncolblk * 128);
+                if (N > 20000000 && d > 128) continue;  // layouts beyond any real device
+                for (int dt = 0; dt < 2; ++dt) {
+                    const fk_dtype dtype = dt ? FK_BF16 : FK_F32;
+                    const WsLayout L = ws_layout(N, d, K, dtype, FK_COSINE);
+                    const size_t offs[] = {L.err, L.obj, L.xn, L.xs, L.xnorm, L.cs, L.cn,
+                                           L.caug, L.cused, L.calt, L.keys0, L.keys1,
+                                           L.vals0, L.vals1, L.hist, L.dtot, L.pieces,
+                                           L.pkeys, L.piecesb, L.pkeysb, L.jpart, L.jdev,
+                                           L.cnt, L.off, L.cand, L.nfb, L.fbrows, L.fblab,
+                                           L.xsfb, L.cmax2};
+                    const int n = sizeof(offs) / sizeof(offs[0]);
+                    for (int i = 0; i < n; ++i) CHECK(offs[i] % 256 == 0);
+                    for (int i = 1; i < n; ++i) CHECK(offs[i] > offs[i - 1]);
+                    CHECK(L.total > offs[n - 1]);
+                    // the sort's histogram and keys, and the combine's buffers, fit
+                    const long long bins = 1LL << (p.bits > 0 ? p.bits : 1);
+                    CHECK(L.dtot - L.hist >= sizeof(uint32_t) * bins * p.nblocks);
+                    CHECK(L.keys1 - L.keys0 >= sizeof(int32_t) * N);
+                    CHECK(L.pkeys - L.pieces >= sizeof(double) * u.nwarps * 2 * u.dcov);
+                    CHECK(L.dp % kBK == 0 && L.dp >= d && L.Kp % kBN == 0 && L.Kp >= K);
+                    ++cases;
+                }
+            }
+        }
+    }
+    std::printf("%d layouts checked, %d failures\n", cases, fails);
+    return fails == 0 ? 0 : 1;
+}
+"""
+
+
+@pytest.mark.skipif(shutil.which("nvcc") is None, reason="nvcc is needed to build the check")
+def test_sort_update_and_workspace_plans(tmp_path):
+    src = tmp_path / "plans.cu"
+    src.write_text(PROGRAM)
+    exe = tmp_path / "plans"
+    subprocess.run(["nvcc", "-std=c++17", "-O1", f"-I{CSRC}", str(src), "-o", str(exe)],
+                   check=True, capture_output=True, text=True)
+    r = subprocess.run([str(exe)], capture_output=True, text=True, timeout=120)
+    print(r.stdout)
+    assert r.returncode == 0, r.stdout
