@@ -1,7 +1,8 @@
 """Host-side planning of the library, checked on the CPU: the radix sort's digits and
-tiles, the update's chunks, and the workspace layout (exact_lloyd_means_b200/csrc/
-fk_common.cuh).  A small host-only program includes the header, is built with nvcc (no
-GPU needed) and checks the invariants the kernels rely on over a grid of shapes."""
+tiles, the update's chunks, and the Lloyd and IVF-Flat search workspace layouts
+(exact_lloyd_means_b200/csrc/fk_common.cuh).  A small host-only program includes the
+header, is built with nvcc (no GPU needed) and checks the invariants the kernels rely on
+over a grid of shapes."""
 import os
 import shutil
 import subprocess
@@ -75,6 +76,47 @@ int main() {
                     CHECK(L.keys1 - L.keys0 >= sizeof(int32_t) * N);
                     CHECK(L.pkeys - L.pieces >= sizeof(double) * u.nwarps * 2 * u.dcov);
                     CHECK(L.dp % kBK == 0 && L.dp >= d && L.Kp % kBN == 0 && L.Kp >= K);
+                    ++cases;
+                }
+            }
+        }
+    }
+    // IVF-Flat search: the workspace for every (queries, cells, probes, k) shape
+    const long long nqs[] = {1, 31, 32, 1000, 10000, 100000};
+    const int nlists[] = {1, 7, 256, 1024, 4096, 16384};
+    const int probes[] = {1, 4, 32, 128, 256, 1024};
+    const int kk[] = {1, 10, 16, 32};
+    for (long long nq : nqs) {
+        for (int nlist : nlists) {
+            for (int nprobe : probes) {
+                if (nprobe > nlist) continue;
+                for (int k : kk) {
+                    long long N = nq;
+                    int K = nlist, d = 768;
+                    const SearchLayout S = search_layout(nq, d, nlist, nprobe, k);
+                    const size_t offs[] = {S.err, S.qn, S.cn, S.D, S.probes, S.keys0, S.keys1,
+                                           S.vals0, S.vals1, S.hist, S.dtot, S.psorted, S.poff,
+                                           S.items, S.nitems, S.Ld, S.Li, S.qplanes, S.qxn,
+                                           S.cplanes, S.ccn, S.cused, S.caug, S.cmax2, S.Sv,
+                                           S.Sp, S.Slost, S.fb};
+                    const int n = sizeof(offs) / sizeof(offs[0]);
+                    for (int i = 0; i < n; ++i) CHECK(offs[i] % 256 == 0);
+                    for (int i = 1; i < n; ++i) CHECK(offs[i] > offs[i - 1]);
+                    CHECK(S.total > offs[n - 1]);
+                    CHECK(S.P == nq * nprobe);
+                    // a coarse batch is a multiple of 32 queries or all of them, and its
+                    // distances (fp64) or screened values (fp32 rows of Kp) fit
+                    CHECK(S.qbatch == nq || S.qbatch % 32 == 0);
+                    CHECK(S.qbatch >= 1 && S.qbatch <= nq);
+                    CHECK(S.probes - S.D >= sizeof(double) * S.qbatch * nlist);
+                    CHECK(S.probes - S.D >= sizeof(float) * S.qbatch * S.Kp);
+                    const long long bins = 1LL << (S.sp.bits > 0 ? S.sp.bits : 1);
+                    CHECK(S.dtot - S.hist >= sizeof(uint32_t) * bins * S.sp.nblocks);
+                    // every pair fits the items: at most one partial item per cell
+                    CHECK(S.max_items >= nlist + (S.P + kSearchPairsPerItem - 1) /
+                                                     kSearchPairsPerItem);
+                    CHECK(S.nitems - S.items >= sizeof(int32_t) * 2 * S.max_items);
+                    CHECK(S.Li - S.Ld >= sizeof(double) * S.P * k);
                     ++cases;
                 }
             }
