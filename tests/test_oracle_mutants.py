@@ -1,13 +1,21 @@
 """The oracle's pins must catch plausible mistakes in the oracle itself.
 
-Each case plants one mistake in a copy of the oracle's C sources (on the CPU, in a temporary
-directory), builds the copy with the oracle's own compiler flags, and runs the pin suite
-(tests/test_oracle_pins.py) against it through FK_ORACLE_LIB.  The pin suite must fail.
-The unchanged copy, built the same way, must pass: that shows the harness itself works.
+C side: each case plants one mistake in a copy of the oracle's C sources (on the CPU, in a
+temporary directory), builds the copy with the oracle's own compiler flags, and runs the
+pin suite (tests/test_oracle_pins.py) against it through FK_ORACLE_LIB.
+
+Python side: each case plants one mistake in a copy of the oracle package (the steps it
+strings together: rounding between iterations, the tie window, the bf16 cast) and runs a
+copy of the pin suite that imports it.
+
+The pin suite must fail for every mistake.  The unchanged copies must pass: that shows the
+harness itself works.
 """
 import os
+import shutil
 import subprocess
 import sys
+from concurrent.futures import ThreadPoolExecutor
 
 import pytest
 
@@ -97,13 +105,85 @@ def _run_pins(lib):
                           cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
 
 
-def test_unchanged_copy_passes_the_pins(tmp_path):
-    r = _run_pins(_build_copy(tmp_path))
+def _run_all(cases, job):
+    """Run job(case) for every case at once (each is its own subprocess); map name ->
+    result, the unchanged copy under None."""
+    workers = max(1, min(8, (os.cpu_count() or 2) // 2))
+    with ThreadPoolExecutor(max_workers=workers) as ex:
+        futs = {(c[0] if c else None): ex.submit(job, c) for c in [None, *cases]}
+        return {name: f.result() for name, f in futs.items()}
+
+
+@pytest.fixture(scope="module")
+def c_results(tmp_path_factory):
+    return _run_all(MUTANTS, lambda m: _run_pins(_build_copy(tmp_path_factory.mktemp("c"), m)))
+
+
+def test_unchanged_copy_passes_the_pins(c_results):
+    r = c_results[None]
     assert r.returncode == 0, r.stdout[-2000:]
 
 
 @pytest.mark.parametrize("mutant", MUTANTS, ids=[m[0] for m in MUTANTS])
-def test_planted_mistake_fails_a_pin(tmp_path, mutant):
-    r = _run_pins(_build_copy(tmp_path, mutant))
+def test_planted_mistake_fails_a_pin(c_results, mutant):
+    r = c_results[mutant[0]]
     # 1: tests ran and at least one failed (not a collection or usage error)
+    assert r.returncode == 1, f"{mutant[0]} survived the pins:\n{r.stdout[-2000:]}"
+
+
+# (name, text in oracle/__init__.py to replace (exactly once), replacement)
+PY_MUTANTS = [
+    ("lloyd_means_not_rounded_to_fp32",
+     "Cnew = round_f32(update(Xd, labels, Cm))", "Cnew = update(Xd, labels, Cm)"),
+    ("lloyd_bf16_assign_unrounded",
+     'Cu = round_bf16(Cm) if precision == "bf16" else Cm', "Cu = Cm"),
+    ("lloyd_objective_against_master",
+     "J = objective(Xd, Cu, labels)", "J = objective(Xd, Cm, labels)"),
+    ("lloyd_cosine_leaves_centroids", "        Cm = normalize_rows(Cm)\n", ""),
+    ("tie_window_uses_smallest_centroid",
+     "(C * C).sum(axis=1).max()", "(C * C).sum(axis=1).min()"),
+    ("bf16_rounding_truncates",
+     "return t.to(torch.bfloat16).double().numpy()",
+     "return (t.view(torch.int32) & -65536).view(torch.float32).double().numpy()"),
+]
+
+
+def _python_copy(tmp_path, mutant=None):
+    shutil.copytree(ORACLE, tmp_path / "oracle",
+                    ignore=shutil.ignore_patterns("_build", "__pycache__"))
+    tests = tmp_path / "tests"
+    tests.mkdir()
+    for name in ("conftest.py", "test_oracle_pins.py"):
+        shutil.copy(os.path.join(ROOT, "tests", name), tests / name)
+    shutil.copytree(os.path.join(ROOT, "tests", "golden"), tests / "golden")
+    if mutant is not None:
+        init = tmp_path / "oracle" / "__init__.py"
+        text = init.read_text()
+        assert text.count(mutant[1]) == 1, f"{mutant[0]}: the planted text must occur once"
+        init.write_text(text.replace(mutant[1], mutant[2]))
+    return str(tmp_path)
+
+
+def _run_copied_pins(cwd):
+    import oracle
+    env = dict(os.environ, FK_ORACLE_LIB=oracle.build.build(), OMP_NUM_THREADS="2")
+    return subprocess.run([sys.executable, "-m", "pytest", "tests/test_oracle_pins.py", "-x",
+                           "-q", "-p", "no:cacheprovider", "-m", "not gpu"],
+                          cwd=cwd, env=env, capture_output=True, text=True, timeout=600)
+
+
+@pytest.fixture(scope="module")
+def py_results(tmp_path_factory):
+    return _run_all(PY_MUTANTS,
+                    lambda m: _run_copied_pins(_python_copy(tmp_path_factory.mktemp("py"), m)))
+
+
+def test_unchanged_python_copy_passes_the_pins(py_results):
+    r = py_results[None]
+    assert r.returncode == 0, r.stdout[-2000:]
+
+
+@pytest.mark.parametrize("mutant", PY_MUTANTS, ids=[m[0] for m in PY_MUTANTS])
+def test_planted_python_mistake_fails_a_pin(py_results, mutant):
+    r = py_results[mutant[0]]
     assert r.returncode == 1, f"{mutant[0]} survived the pins:\n{r.stdout[-2000:]}"

@@ -278,6 +278,48 @@ def test_lloyd_bf16_precision_feeds_rounded_centroids():
     assert (oracle.round_f32(out["C_next"][0]) == out["C_next"][0]).all()
 
 
+def test_lloyd_objective_is_against_the_centroids_used():
+    """J of an iteration is sum_i ||x_i - c_{l_i}||^2 against the centroids that
+    iteration's assignment used: with bf16 centroids, their bf16 roundings, not the fp32
+    master.  Formed here with numpy from the recorded labels; the master gives a J the test
+    can tell apart."""
+    r = _rng(17)
+    X = r.normal(size=(300, 16)).astype(np.float32)
+    out = oracle.lloyd(X, X[:5], 2, precision="bf16")
+    for t in range(2):
+        Cu, lab = out["C_used"][t], out["labels"][t]
+        J_np = float(((out["X"] - Cu[lab]) ** 2).sum())
+        assert abs(out["J"][t] - J_np) <= 1e-12 * J_np
+        master = out["C_next"][t - 1] if t else X[:5].astype(np.float64)
+        J_master = float(((out["X"] - master[lab]) ** 2).sum())
+        assert abs(J_master - J_np) > 1e-9 * J_np
+
+
+def test_lloyd_cosine_normalises_initial_centroids():
+    """Cosine mode L2-normalises the points and the initial centroids (LEANN FlashLib
+    guide, "距离度量只有 squared L2如何支持 mips / cosine"), so the first assignment sees
+    unit-norm centroids (rounded to fp32) and unit-norm points."""
+    r = _rng(18)
+    X = r.normal(size=(100, 8)) * 3.0
+    C0 = X[:4] * np.array([[0.5], [2.0], [7.0], [1.0]])
+    out = oracle.lloyd(X, C0, 1, metric="cosine")
+    assert np.abs(np.linalg.norm(out["C_used"][0], axis=1) - 1.0).max() <= 1e-6
+    assert np.abs(np.linalg.norm(out["X"], axis=1) - 1.0).max() <= 1e-12
+
+
+def test_tie_window_scales_with_the_largest_centroid_norm():
+    """The tie window is tau * (||x||^2 + max_k ||c_k||^2) (the parity rule's reading): a
+    far centroid of large norm widens it for every point.  Here the top-2 gap is 0.04:
+    inside the window with the far centroid (about 1.0), outside it without (about 1e-4)."""
+    C = np.array([[-1.0, 0.0], [1.0, 0.0], [100.0, 0.0]])
+    X = np.array([[0.01, 0.0]])
+    labels, dmin, d2nd = oracle.assign(X, C)
+    assert labels.tolist() == [1]
+    assert oracle.tie_mask(X, C, dmin, d2nd).tolist() == [True]
+    _, dmin2, d2nd2 = oracle.assign(X, C[:2])
+    assert oracle.tie_mask(X, C[:2], dmin2, d2nd2).tolist() == [False]
+
+
 def test_round_bf16_is_nearest_even():
     ulp = 2.0 ** -7  # bf16 spacing on [1, 2)
     v = np.array([1 + ulp / 2, 1 + 1.5 * ulp, 1 + 0.75 * ulp, -(1 + ulp / 2)])
