@@ -180,3 +180,32 @@ def test_fault_injection_workspace_needs_no_device(fk):
     assert out.returncode == 0, out.stderr
     r1, r2 = (int(x) for x in out.stdout.split())
     assert r1 == fk.FK_ERR_WORKSPACE and r2 == fk.FK_ERR_WORKSPACE
+
+
+def test_binding_without_the_library_fails_loudly(tmp_path):
+    """The product path has no CPU fallback: the binding, copied where no libfk.so sits
+    beside it, refuses to import and says how to build the library."""
+    import shutil
+    import subprocess
+    import sys
+    pkg = tmp_path / "exact_lloyd_means_b200"
+    pkg.mkdir()
+    shutil.copy(os.path.join(ROOT, "exact_lloyd_means_b200", "fk.py"), pkg / "fk.py")
+    (pkg / "__init__.py").write_text("")
+    r = subprocess.run([sys.executable, "-c", "import exact_lloyd_means_b200.fk"],
+                       cwd=tmp_path, capture_output=True, text=True, timeout=120)
+    assert r.returncode != 0
+    assert "ImportError" in r.stderr and "build the CUDA library first" in r.stderr
+
+
+def test_product_package_never_imports_the_oracle():
+    """Only tests/, the smoke check and the bench's baseline legs may use oracle/: no module
+    of the product package imports it."""
+    import re
+    pat = re.compile(r"^\s*(import\s+oracle\b|from\s+oracle\b)", re.M)
+    pkg = os.path.join(ROOT, "exact_lloyd_means_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for name in files:
+            if name.endswith(".py"):
+                with open(os.path.join(dirpath, name)) as f:
+                    assert not pat.search(f.read()), os.path.join(dirpath, name)
