@@ -75,7 +75,7 @@ constexpr int64_t kScreenProbeRows = 2 * 128 * 148;
 // the m-th smallest exact value is at most T~ + E and every column among the m exact
 // smallest has v~ <= T~ + 2E.  ||c|| is bounded by cmax = max_k ||c_k||.
 // The result carries a 1% margin for the rounding of this expression itself.
-__device__ __forceinline__ float screen_window(float xnorm2, float cmax2, int dp) {
+__host__ __device__ __forceinline__ float screen_window(float xnorm2, float cmax2, int dp) {
     const float xn = sqrtf(xnorm2), cm = sqrtf(cmax2);
     const float u = 0.00390625f;
     const float prod = 2.f * (2.f * u + u * u) * xn * cm;

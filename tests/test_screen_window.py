@@ -1,0 +1,182 @@
+"""The screened route's window, checked on the CPU against emulated arithmetic.
+
+The single-product screening pass accumulates v~ = ||c||^2 - 2 RN_bf16(x) . RN_bf16(c) in
+fp32 (the squared norm folded in as an exact three-part bf16 split of its fp32 rounding),
+and screen_window() promises E = W / 2 >= |v~ - v| for the exact v = ||c||^2 - 2 x.c.  The
+tensor core's internal accumulation order and rounding are not documented, so a host
+program (built with nvcc, no GPU needed) emulates several: one rounding per 16-product
+MMA step, one per product, round-to-nearest or toward zero, the norm step first or last.
+Every emulation must stay inside E, on random, scaled, aligned, unit-norm and adversarial
+data at the dimensions the route serves (the adversarial case, where every operand rounds
+the same way, must come within a factor 2 of E, so the bound is not loose by more); and
+the exact argmin must lie within W of the screened minimum."""
+import os
+import shutil
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+CSRC = os.path.join(ROOT, "exact_lloyd_means_b200", "csrc")
+
+PROGRAM = r"""
+#include "fk_common.cuh"
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <random>
+#include <vector>
+using namespace fk;
+
+static float bf16_rn(float f) {  // round to nearest even, 8 significant bits
+    uint32_t u;
+    std::memcpy(&u, &f, 4);
+    u += 0x7fffu + ((u >> 16) & 1u);
+    u &= 0xffff0000u;
+    float r;
+    std::memcpy(&r, &u, 4);
+    return r;
+}
+static float to_f32(double v, bool rz) {  // one rounding of an exact value to fp32
+    float f = static_cast<float>(v);
+    if (rz && std::fabs(static_cast<double>(f)) > std::fabs(v))
+        f = std::nextafter(f, 0.0f);
+    return f;
+}
+
+int main() {
+    std::mt19937_64 rng(12345);
+    std::normal_distribution<double> nd(0.0, 1.0);
+    std::uniform_real_distribution<double> ud(-1.0, 1.0);
+    const int dims[] = {256, 384, 768, 1024};
+    const double scales[] = {1e-3, 1.0, 37.0, 1e3};
+    long long checked = 0, bad = 0, argmin_bad = 0;
+    double worst = 0.0, worst_adv = 0.0;  // largest |v~ - v| / E: all kinds, adversarial
+    for (int d : dims) {
+        const int dp = static_cast<int>(round_up(d, kBK));
+        for (double scale : scales) {
+            // kinds: normal, uniform, nearly parallel, unit norm, and adversarial: every
+            // operand just under a bf16 half-unit above a power of two, so all roundings
+            // shrink it by 0.98 u and, with the centroids parallel to x, every product
+            // errs the same way (the operand term of the bound is nearly reached)
+            for (int kind = 0; kind < 5; ++kind) {
+                const int K = 48;
+                std::vector<float> x(d), C(static_cast<size_t>(K) * d);
+                const double p2 = std::ldexp(1.0, std::ilogb(scale));
+                for (int j = 0; j < d; ++j) {
+                    if (kind == 4) {
+                        const double m = (1.0 + 0.49 * std::ldexp(1.0, -7)) *
+                                         std::ldexp(1.0, static_cast<int>(rng() % 5) - 2);
+                        x[j] = static_cast<float>(p2 * ((rng() & 1) ? m : -m));
+                    } else {
+                        x[j] = static_cast<float>(scale * (kind == 1 ? ud(rng) : nd(rng)));
+                    }
+                }
+                for (int k = 0; k < K; ++k)
+                    for (int j = 0; j < d; ++j) {
+                        float &cv = C[static_cast<size_t>(k) * d + j];
+                        if (kind == 4) {
+                            cv = x[j] * static_cast<float>(1 << (k % 4));
+                            continue;
+                        }
+                        double v = kind == 1 ? ud(rng) : nd(rng);
+                        if (kind == 2) v = x[j] / scale + 0.01 * v;  // nearly parallel to x
+                        cv = static_cast<float>(scale * v);
+                    }
+                if (kind == 3) {  // cosine data: unit rows
+                    auto unit = [&](float *r) {
+                        double s = 0.0;
+                        for (int j = 0; j < d; ++j) s += double(r[j]) * r[j];
+                        const double n = std::sqrt(s);
+                        for (int j = 0; j < d; ++j) r[j] = static_cast<float>(r[j] / n);
+                    };
+                    unit(x.data());
+                    for (int k = 0; k < K; ++k) unit(&C[static_cast<size_t>(k) * d]);
+                }
+                double xs = 0.0;
+                for (int j = 0; j < d; ++j) xs += double(x[j]) * x[j];
+                const float xnorm2 = static_cast<float>(xs);
+                std::vector<float> cn(K);
+                float cmax2 = 0.f;
+                for (int k = 0; k < K; ++k) {
+                    double s = 0.0;
+                    for (int j = 0; j < d; ++j) {
+                        const double c = C[static_cast<size_t>(k) * d + j];
+                        s += c * c;
+                    }
+                    cn[k] = static_cast<float>(s);
+                    cmax2 = std::fmax(cmax2, cn[k]);
+                }
+                const float W = screen_window(xnorm2, cmax2, dp);
+                const double E = 0.5 * W;
+                for (int mode = 0; mode < 8; ++mode) {
+                    const bool per_product = mode & 1, rz = (mode >> 1) & 1,
+                               norm_last = (mode >> 2) & 1;
+                    std::vector<double> vt(K), ve(K);
+                    for (int k = 0; k < K; ++k) {
+                        const float *c = &C[static_cast<size_t>(k) * d];
+                        double dot = 0.0, exact_n = 0.0;
+                        for (int j = 0; j < d; ++j) {
+                            dot += double(x[j]) * c[j];
+                            exact_n += double(c[j]) * c[j];
+                        }
+                        ve[k] = exact_n - 2.0 * dot;
+                        // the norm step: exact bf16 split of the fp32 norm, added exactly
+                        const float h = bf16_rn(cn[k]), m = bf16_rn(cn[k] - h),
+                                    l = bf16_rn(cn[k] - h - m);
+                        const double nstep = double(h) + m + l;
+                        float acc = 0.f;
+                        if (!norm_last) acc = to_f32(double(acc) + nstep, rz);
+                        for (int j0 = 0; j0 < dp; j0 += 16) {
+                            double chunk = 0.0;
+                            for (int j = j0; j < j0 + 16; ++j) {
+                                const double p = j < d ? double(bf16_rn(x[j])) *
+                                                             (-2.0 * bf16_rn(c[j]))
+                                                       : 0.0;
+                                if (per_product) acc = to_f32(double(acc) + p, rz);
+                                else chunk += p;  // 16 bf16 products: exact in fp64
+                            }
+                            if (!per_product) acc = to_f32(double(acc) + chunk, rz);
+                        }
+                        if (norm_last) acc = to_f32(double(acc) + nstep, rz);
+                        vt[k] = acc;
+                        const double err = std::fabs(vt[k] - ve[k]);
+                        worst = std::fmax(worst, err / E);
+                        if (kind == 4) worst_adv = std::fmax(worst_adv, err / E);
+                        ++checked;
+                        if (err > E) {
+                            if (bad < 10)
+                                std::printf("FAIL d=%d scale=%g kind=%d mode=%d k=%d: |v~-v|=%g"
+                                            " E=%g\n", d, scale, kind, mode, k, err, E);
+                            ++bad;
+                        }
+                    }
+                    int ke = 0, kt = 0;
+                    for (int k = 1; k < K; ++k) {
+                        if (ve[k] < ve[ke]) ke = k;
+                        if (vt[k] < vt[kt]) kt = k;
+                    }
+                    if (vt[ke] > vt[kt] + W) ++argmin_bad;
+                }
+            }
+        }
+    }
+    std::printf("%lld screened values, worst |v~ - v| / E = %.3f (adversarial %.3f), "
+                "%lld outside E, %lld argmins outside W\n", checked, worst, worst_adv, bad,
+                argmin_bad);
+    // the adversarial inputs come close to the bound: a bound half as wide would fail
+    return (bad == 0 && argmin_bad == 0 && worst_adv > 0.5) ? 0 : 1;
+}
+"""
+
+
+@pytest.mark.skipif(shutil.which("nvcc") is None, reason="nvcc is needed to build the check")
+def test_screen_window_bounds_emulated_screening(tmp_path):
+    src = tmp_path / "window.cu"
+    src.write_text(PROGRAM)
+    exe = tmp_path / "window"
+    subprocess.run(["nvcc", "-std=c++17", "-O2", f"-I{CSRC}", str(src), "-o", str(exe)],
+                   check=True, capture_output=True, text=True)
+    r = subprocess.run([str(exe)], capture_output=True, text=True, timeout=300)
+    print(r.stdout)
+    assert r.returncode == 0, r.stdout
