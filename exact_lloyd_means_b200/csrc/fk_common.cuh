@@ -3,6 +3,7 @@
 #pragma once
 
 #include <atomic>
+#include <cmath>
 #include <cstddef>
 #include <cstdint>
 #include <utility>
@@ -83,6 +84,21 @@ __host__ __device__ __forceinline__ float screen_window(float xnorm2, float cmax
                         (cmax2 + 2.f * xn * cm) * 1.01f;
     const float norm = 5.9604645e-8f * cmax2;
     return 2.f * (prod + accum + norm) * 1.01f;
+}
+
+// Window coefficients of the IVF-Flat search's screened fine pass for rows padded to dp:
+// |s~ - s| <= ce_dot ||q|| ||x|| + ce_round (||q||^2 + ||x||^2), where s = ||q - x||^2 and s~
+// = ||q||^2 + ||x||^2 - 2 q.x~ rounded to fp32, with q.x~ the three bf16 products
+// hi.hi + hi.lo + lo.hi of the RN-bf16 splits v = hi + lo (+ a residual below 2^-16 |v|)
+// accumulated in fp32.  With u = 2^-8 (bf16 rounding), the three products miss at most
+// 3.1 u^2 sum |q_j||x_j| <= 3.1 u^2 |q||x|; the 3 dp / 16 mma steps add at most 17 units of
+// 2^-23 of a partial sum bounded by 1.02 |q||x| each; the factor 2 of -2 q.x; the fp32
+// rounding of s~ at most 2^-23 (||q||^2 + ||x||^2); a 1% margin on both.
+inline void fine_window_coeffs(int dp, float *ce_dot, float *ce_round) {
+    const double u = 1.0 / 256.0;
+    const double e_dot = 3.1 * u * u + 3.0 * (dp / 16) * 17.0 * std::ldexp(1.0, -23) * 1.02;
+    *ce_dot = static_cast<float>(2.0 * e_dot * 1.01);
+    *ce_round = static_cast<float>(std::ldexp(1.0, -23) * 1.01);
 }
 
 // Objective slots kept on the device by fk_lloyd before a copy to the host.

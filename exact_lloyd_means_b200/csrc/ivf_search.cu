@@ -1634,8 +1634,6 @@ __global__ void __launch_bounds__(1024) build_items_kernel(const int32_t *__rest
 }  // namespace
 
 // ---------------------------------------------------------------- host side
-void fine_window_coeffs(int dp, float *ce_dot, float *ce_round);
-
 size_t ivf_tile_smem() { return sizeof(TileSmem); }
 
 cudaError_t launch_sqnorm_f64(const float *V, int64_t n, int d, double *out, cudaStream_t st) {
@@ -1750,18 +1748,6 @@ cudaError_t launch_ivf_fine_scr(const uint16_t *Qp, int64_t nq, const uint16_t *
     ivf_fine_scr_kernel<<<static_cast<unsigned>(grid), kTThreads, sizeof(FineSmem), st>>>(a);
     note_launch();
     return cudaGetLastError();
-}
-
-// Window coefficients of the screened fine pass for rows padded to dp: with u = 2^-8 (bf16
-// rounding), the three products miss at most 3.1 u^2 sum |q_j||x_j| <= 3.1 u^2 |q||x|; the
-// 3 dp / 16 mma steps add at most 17 units of 2^-23 of a partial sum bounded by
-// 1.02 |q||x| each; the factor 2 of -2 q.x; the fp32 rounding of s~ at most 2^-23
-// (||q||^2 + ||x||^2); a 1% margin on both.
-void fine_window_coeffs(int dp, float *ce_dot, float *ce_round) {
-    const double u = 1.0 / 256.0;
-    const double e_dot = 3.1 * u * u + 3.0 * (dp / 16) * 17.0 * std::ldexp(1.0, -23) * 1.02;
-    *ce_dot = static_cast<float>(2.0 * e_dot * 1.01);
-    *ce_round = static_cast<float>(std::ldexp(1.0, -23) * 1.01);
 }
 
 cudaError_t launch_ivf_query_rerank(const float *Sv, const uint32_t *Sp, const float *Slost,

@@ -180,3 +180,144 @@ def test_screen_window_bounds_emulated_screening(tmp_path):
     r = subprocess.run([str(exe)], capture_output=True, text=True, timeout=300)
     print(r.stdout)
     assert r.returncode == 0, r.stdout
+
+
+FINE_PROGRAM = r"""
+#include "fk_common.cuh"
+#include <algorithm>
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <random>
+#include <vector>
+using namespace fk;
+
+static float bf16_rn(float f) {
+    uint32_t u;
+    std::memcpy(&u, &f, 4);
+    u += 0x7fffu + ((u >> 16) & 1u);
+    u &= 0xffff0000u;
+    float r;
+    std::memcpy(&r, &u, 4);
+    return r;
+}
+static float to_f32(double v, bool rz) {
+    float f = static_cast<float>(v);
+    if (rz && std::fabs(static_cast<double>(f)) > std::fabs(v)) f = std::nextafter(f, 0.0f);
+    return f;
+}
+
+int main() {
+    std::mt19937_64 rng(777);
+    std::normal_distribution<double> nd(0.0, 1.0);
+    std::uniform_real_distribution<double> pos(0.0, 1.0);
+    const int dims[] = {64, 128, 768, 1024};
+    const double scales[] = {1e-3, 1.0, 1e3};
+    long long checked = 0, bad = 0, topk_bad = 0;
+    double worst = 0.0, worst_adv = 0.0;
+    for (int d : dims) {
+        const int dp = static_cast<int>(round_up(d, kBK));
+        float ce_dot, ce_round;
+        fine_window_coeffs(dp, &ce_dot, &ce_round);
+        for (double scale : scales) {
+            // kinds: normal; near duplicates of the query; adversarial: every coordinate
+            // positive, so all partial sums grow and one-sided roundings pile up
+            for (int kind = 0; kind < 3; ++kind) {
+                const int M = 64, k = 10;
+                std::vector<float> q(d), X(static_cast<size_t>(M) * d);
+                for (int j = 0; j < d; ++j)
+                    q[j] = static_cast<float>(scale * (kind == 2 ? pos(rng) : nd(rng)));
+                for (int i = 0; i < M; ++i)
+                    for (int j = 0; j < d; ++j) {
+                        double v = kind == 2 ? pos(rng) * scale : nd(rng) * scale;
+                        if (kind == 1) v = q[j] + 1e-3 * scale * nd(rng);
+                        X[static_cast<size_t>(i) * d + j] = static_cast<float>(v);
+                    }
+                double qn = 0.0;
+                for (int j = 0; j < d; ++j) qn += double(q[j]) * q[j];
+                std::vector<double> xn(M, 0.0);
+                double xmax2 = 0.0;
+                for (int i = 0; i < M; ++i) {
+                    for (int j = 0; j < d; ++j) {
+                        const double x = X[static_cast<size_t>(i) * d + j];
+                        xn[i] += x * x;
+                    }
+                    xmax2 = std::max(xmax2, xn[i]);
+                }
+                for (int mode = 0; mode < 4; ++mode) {
+                    const bool per_product = mode & 1, rz = (mode >> 1) & 1;
+                    std::vector<double> st(M), se(M);
+                    for (int i = 0; i < M; ++i) {
+                        const float *x = &X[static_cast<size_t>(i) * d];
+                        double s = 0.0;
+                        for (int j = 0; j < d; ++j) {
+                            const double t = double(q[j]) - x[j];
+                            s += t * t;
+                        }
+                        se[i] = s;
+                        float acc = 0.f;
+                        for (int j0 = 0; j0 < dp; j0 += 16) {
+                            for (int prod = 0; prod < 3; ++prod) {  // hi.hi, hi.lo, lo.hi
+                                double chunk = 0.0;
+                                for (int j = j0; j < j0 + 16 && j < d; ++j) {
+                                    const float qh = bf16_rn(q[j]), ql = bf16_rn(q[j] - qh);
+                                    const float xh = bf16_rn(x[j]), xl = bf16_rn(x[j] - xh);
+                                    const double p = prod == 0 ? double(qh) * xh
+                                                     : prod == 1 ? double(qh) * xl
+                                                                 : double(ql) * xh;
+                                    if (per_product) acc = to_f32(double(acc) + p, rz);
+                                    else chunk += p;
+                                }
+                                if (!per_product) acc = to_f32(double(acc) + chunk, rz);
+                            }
+                        }
+                        st[i] = static_cast<float>(std::fma(-2.0, double(acc), qn + xn[i]));
+                        const double E = ce_dot * std::sqrt(qn * xn[i]) + ce_round * (qn + xn[i]);
+                        const double err = std::fabs(st[i] - se[i]);
+                        worst = std::max(worst, err / E);
+                        if (kind == 2) worst_adv = std::max(worst_adv, err / E);
+                        ++checked;
+                        if (err > E) {
+                            if (bad < 10)
+                                std::printf("FAIL d=%d scale=%g kind=%d mode=%d: |s~-s|=%g E=%g\n",
+                                            d, scale, kind, mode, err, E);
+                            ++bad;
+                        }
+                    }
+                    // every point of the exact top-k lies within 2E (E at the largest
+                    // point norm) of the k-th smallest screened value
+                    std::vector<int> ord(M);
+                    for (int i = 0; i < M; ++i) ord[i] = i;
+                    std::stable_sort(ord.begin(), ord.end(),
+                                     [&](int a, int b) { return se[a] < se[b]; });
+                    std::vector<double> sorted_t(st);
+                    std::sort(sorted_t.begin(), sorted_t.end());
+                    const double Eq = ce_dot * std::sqrt(qn * xmax2) + ce_round * (qn + xmax2);
+                    for (int r = 0; r < k; ++r)
+                        if (st[ord[r]] > sorted_t[k - 1] + 2.0 * Eq) ++topk_bad;
+                }
+            }
+        }
+    }
+    std::printf("%lld screened distances, worst |s~ - s| / E = %.3f (adversarial %.3f), "
+                "%lld outside E, %lld top-k points outside 2E\n", checked, worst, worst_adv,
+                bad, topk_bad);
+    return (bad == 0 && topk_bad == 0) ? 0 : 1;
+}
+"""
+
+
+@pytest.mark.skipif(shutil.which("nvcc") is None, reason="nvcc is needed to build the check")
+def test_search_fine_window_bounds_emulated_three_product_screening(tmp_path):
+    """The IVF-Flat search's fine window (fine_window_coeffs): s~ = ||q||^2 + ||x||^2 - 2 q.x~
+    rounded to fp32, with q.x~ the three bf16 products of the hi/lo splits accumulated in
+    fp32 (per MMA step or per product, to nearest or toward zero), stays within E of the
+    exact squared distance, and the exact top-k lies within 2E of the k-th screened value."""
+    src = tmp_path / "fine_window.cu"
+    src.write_text(FINE_PROGRAM)
+    exe = tmp_path / "fine_window"
+    subprocess.run(["nvcc", "-std=c++17", "-O2", f"-I{CSRC}", str(src), "-o", str(exe)],
+                   check=True, capture_output=True, text=True)
+    r = subprocess.run([str(exe)], capture_output=True, text=True, timeout=300)
+    print(r.stdout)
+    assert r.returncode == 0, r.stdout
