@@ -1188,9 +1188,8 @@ cudaError_t launch_assign_np(const AssignArgs &a, cudaStream_t st) {
 
 cudaError_t launch_assign(const AssignArgs &a, cudaStream_t st) {
     if (a.N <= 0) return cudaSuccess;
-    if (a.cand != nullptr || a.dump != nullptr) {  // only in the CTA-pair form
-        if (a.a_nplanes != 1 || (a.cand != nullptr && !assign_can_screen(a.N, a.dp, a.Kp)))
-            return cudaErrorNotSupported;
+    if (a.cand != nullptr || a.dump != nullptr) {  // only in the CTA-pair form, any N
+        if (a.a_nplanes != 1 || !assign_can_dump(a.dp, a.Kp)) return cudaErrorNotSupported;
         bool done = false;
         const cudaError_t e =
             launch_assign_pair<1, true>(a, st, resident_x(1, a.dp, a.Kp), &done);

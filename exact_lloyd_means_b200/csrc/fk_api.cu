@@ -25,25 +25,8 @@ int device_sm_count() {
     return n;
 }
 
-namespace {
-
-constexpr uint64_t kDefaultWaitNs = 2000000000ull;  // 2 s bound on any in-kernel wait
-
-// NVTX range for the phases of a call (visible to profilers that record NVTX; without
-// one attached the calls cost a branch).
-struct NvtxRange {
-    explicit NvtxRange(const char *name) { nvtxRangePushA(name); }
-    ~NvtxRange() { nvtxRangePop(); }
-    NvtxRange(const NvtxRange &) = delete;
-    NvtxRange &operator=(const NvtxRange &) = delete;
-};
-
-// Host-side fault injection for tests of the error paths, chosen by the environment
-// variable FK_FAULT when the library is first used: "workspace" makes every workspace
-// check fail (FK_ERR_WORKSPACE); "launch" makes fk_assign, fk_update, fk_lloyd and
-// fk_ivf_search fail as a failed launch would (FK_ERR_CUDA), before any device work.
-// Nothing is injected on the device.
-enum Fault { kFaultNone = 0, kFaultWorkspace = 1, kFaultLaunch = 2 };
+// Host-side fault injection, chosen by the environment variable FK_FAULT when the library
+// is first used (see fk_common.cuh).  Nothing is injected on the device.
 Fault injected_fault() {
     static const Fault f = [] {
         const char *e = std::getenv("FK_FAULT");
@@ -72,7 +55,7 @@ fk_status check_device() {
 bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 fk_status validate_shape(int64_t N, int d, int K, fk_dtype dtype, fk_metric metric,
-                         bool planes_ok = false) {
+                         bool planes_ok) {
     if (N < 1 || N > 2147483647LL - 1) return FK_ERR_INVALID_ARG;
     if (d < 1 || K < 1 || K > N) return FK_ERR_INVALID_ARG;
     if (dtype == FK_BF16X2 && !planes_ok) return FK_ERR_UNSUPPORTED;
@@ -85,6 +68,23 @@ fk_status validate_shape(int64_t N, int d, int K, fk_dtype dtype, fk_metric metr
     if (static_cast<int64_t>(K) * d > 2147483647LL) return FK_ERR_UNSUPPORTED;
     return FK_OK;
 }
+
+bool screened_route(int64_t N, int dp, int Kp, int K) {
+    if (dp > kThreeProductMaxDp) return assign_can_dump(dp, Kp);
+    const bool pays = dp >= kScreenMinD || static_cast<int64_t>(K) * dp >= kScreenMinKD;
+    return pays && assign_can_screen(N, dp, Kp);
+}
+
+namespace {
+
+// NVTX range for the phases of a call (visible to profilers that record NVTX; without
+// one attached the calls cost a branch).
+struct NvtxRange {
+    explicit NvtxRange(const char *name) { nvtxRangePushA(name); }
+    ~NvtxRange() { nvtxRangePop(); }
+    NvtxRange(const NvtxRange &) = delete;
+    NvtxRange &operator=(const NvtxRange &) = delete;
+};
 
 fk_status check_ws(void *ws, size_t ws_bytes, const WsLayout &L) {
     if (ws == nullptr || !aligned(ws, 256) || ws_bytes < L.total) return FK_ERR_WORKSPACE;
@@ -173,11 +173,15 @@ fk_status run_assign(const void *planes, int nplanes, int64_t lda, int64_t N, in
     a.mind = mind;
     a.err = ws_ptr<uint32_t>(ws, L.err);
     a.wait_ns = kDefaultWaitNs;
-    const bool screen_pays =
-        L.dp >= kScreenMinD || static_cast<int64_t>(K) * L.dp >= kScreenMinKD;
-    if (allow_screen && nplanes == 2 && screen_pays && C != nullptr &&
-        xnorm != nullptr && lda == L.dp && d % 4 == 0 && aligned(C, 16) &&
-        (X32 == nullptr || aligned(X32, 16)) && assign_can_screen(N, a.dp, a.Kp)) {
+    // beyond kThreeProductMaxDp the three-product form decides no label: screen every call
+    const bool exact_only = nplanes == 2 && L.dp > kThreeProductMaxDp;
+    const bool can_screen = nplanes == 2 && C != nullptr && xnorm != nullptr &&
+                            lda == L.dp && d % 4 == 0 && aligned(C, 16) &&
+                            (X32 == nullptr || aligned(X32, 16));
+    if (exact_only && !can_screen) return FK_ERR_UNSUPPORTED;
+    if (exact_only && probe_rows > 0) return FK_OK;  // nothing to decide: no probe
+    if ((allow_screen || exact_only) && can_screen &&
+        screened_route(N, a.dp, a.Kp, K)) {
         ScreenBufs sb;
         sb.cand = ws_ptr<int32_t>(ws, L.cand);
         sb.nfb = ws_ptr<uint32_t>(ws, L.nfb);
@@ -192,6 +196,7 @@ fk_status run_assign(const void *planes, int nplanes, int64_t lda, int64_t N, in
         if (screened) *screened = true;
         return FK_OK;
     }
+    if (exact_only) return FK_ERR_UNSUPPORTED;  // the pair kernel cannot run on this device
     if (probe_rows > 0) return FK_OK;
     if (ev_mma0) FK_TRY_CUDA(cudaEventRecord(ev_mma0, st));
     FK_TRY_CUDA(launch_assign(a, st));
@@ -494,6 +499,34 @@ fk_status fk_assign(const void *X, fk_dtype dtype, int64_t N, int d, const float
         return s;
     return run_assign(planes, nplanes, lda, N, d, K, L, ws, labels, xn, mind, st,
                       dtype == FK_F32 ? static_cast<const float *>(X) : nullptr, C);
+}
+
+fk_status fk_assign_split(const float *X, const void *planes, int64_t N, int d,
+                          const float *C, int K, int32_t *labels, float *mind, void *ws,
+                          size_t ws_bytes, fk_stream_t stream) {
+    fk_status s = validate_shape(N, d, K, FK_F32, FK_L2);
+    if (s != FK_OK) return s;
+    if (!X || !planes || !C || !labels) return FK_ERR_INVALID_ARG;
+    if (!aligned(X, 16) || !aligned(planes, 16) || !aligned(C, 4) || !aligned(labels, 4) ||
+        (mind && !aligned(mind, 4)))
+        return FK_ERR_UNSUPPORTED;
+    const WsLayout L = ws_layout(N, d, K, FK_BF16X2, FK_L2);
+    if ((s = check_ws(ws, ws_bytes, L)) != FK_OK) return s;
+    if ((s = check_device()) != FK_OK) return s;
+    if (injected_fault() == kFaultLaunch) return FK_ERR_CUDA;
+    cudaStream_t st = stream;
+    FK_TRY_CUDA(launch_prep_centroids(C, K, d, L.Kp, L.dp, FK_F32, ws_ptr<uint16_t>(ws, L.cs),
+                                      ws_ptr<float>(ws, L.cn), ws_ptr<float>(ws, L.cused),
+                                      ws_ptr<uint16_t>(ws, L.caug), st));
+    const void *pl = nullptr;
+    const float *xn = nullptr;
+    int nplanes = 0;
+    int64_t lda = 0;
+    if ((s = prepare_x(planes, FK_BF16X2, N, d, L, ws, nullptr, st, &pl, &nplanes, &lda,
+                       &xn)) != FK_OK)
+        return s;
+    // the planes feed the tensor cores, the fp32 rows the exact re-ranking
+    return run_assign(pl, nplanes, lda, N, d, K, L, ws, labels, xn, mind, st, X, C);
 }
 
 fk_status fk_update(const void *X, fk_dtype dtype, int64_t N, int d, int K,

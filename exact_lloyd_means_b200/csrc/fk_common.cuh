@@ -60,6 +60,15 @@ constexpr int64_t kScreenMinKD = int64_t(1) << 22;
 // (mixtures whose heavy components hold many nearly equidistant centroids do not qualify).
 constexpr int kScreenMaxFallback = 4;
 constexpr int64_t kScreenProbeRows = 2 * 128 * 148;
+// The three-product form (hi.hi + lo.hi + hi.lo in one fp32 accumulator) misses the exact
+// x.c by the dropped lo.lo and residual terms plus its fp32 accumulation.  Emulated under
+// every modelled accumulation order (one rounding per MMA step or per product, to nearest
+// or toward zero), that error stays within half the parity rule's tie window up to a
+// padded depth of 768; beyond it, rounding toward zero after every product reaches 1.55
+// half windows at 1024.  So from d_p > 768 on no label of fp32 points is decided by the
+// three-product form: every call takes the screened route (any N, whatever the probe
+// says), and rows whose candidates overflow get an exact fp64 scan over all centroids.
+constexpr int kThreeProductMaxDp = 768;
 
 // Width of the screening window for one row: twice a bound E on |v~ - v|, where
 // v = ||c||^2 - 2 x.c is exact and v~ is what the single-product pass accumulates from
@@ -103,6 +112,9 @@ inline void fine_window_coeffs(int dp, float *ce_dot, float *ce_round) {
 
 // Objective slots kept on the device by fk_lloyd before a copy to the host.
 constexpr int kObjRing = 4096;
+
+// Bound on every in-kernel wait of a library call (2 s).
+constexpr uint64_t kDefaultWaitNs = 2000000000ull;
 
 // Device error word bits (workspace offset 0).
 constexpr uint32_t kErrTimeout = 1u;
@@ -483,6 +495,29 @@ inline SearchLayout search_layout(int64_t nq, int d, int nlist, int nprobe, int 
 cudaError_t launch_cluster_stats(const int32_t *counts, int K, uint32_t *out, cudaStream_t st);
 
 int device_sm_count();
+
+// Argument and device checks shared by every entry point (fk_api.cu).
+bool aligned(const void *p, size_t a);
+// FK_OK on an sm_100 device, FK_ERR_UNSUPPORTED on any other, FK_ERR_CUDA if it cannot tell.
+fk_status check_device();
+// Shape, dtype and metric rules of the assign / update / Lloyd calls (FK_BF16X2 only
+// where planes_ok).
+fk_status validate_shape(int64_t N, int d, int K, fk_dtype dtype, fk_metric metric,
+                         bool planes_ok = false);
+// Host-side fault injection for tests of the error paths (environment variable FK_FAULT,
+// read when the library is first used): "workspace" fails every workspace check, "launch"
+// fails the computing calls as a failed launch would, before any device work.
+enum Fault { kFaultNone = 0, kFaultWorkspace = 1, kFaultLaunch = 2 };
+Fault injected_fault();
+// Status of the two device error words (word 0: a bounded wait expired; word 1: a label
+// outside [0, K) was met).
+inline fk_status decode_err(const uint32_t (&e)[2]) {
+    return e[0] ? FK_ERR_TIMEOUT : (e[1] ? FK_ERR_DEVICE : FK_OK);
+}
+// Whether fk_assign takes the screened route for two-plane (fp32) points of this shape
+// when its buffers are at hand: always beyond kThreeProductMaxDp, otherwise where
+// screening pays and the CTA-pair kernel has rows enough.
+bool screened_route(int64_t N, int dp, int Kp, int K);
 
 // Raise a kernel's dynamic shared-memory limit to `bytes` on the current device.  The
 // attribute belongs to the device, so each call site records the devices it has set it

@@ -8,8 +8,6 @@
 // X when the points need splitting or padding) from one file-scope device array of fixed
 // size, instead of from a caller-provided workspace.  The array is part of the library image:
 // every GPU that loads libfk holds it until the process exits.
-#include <mutex>
-
 #include "fk_common.cuh"
 
 namespace fk {
@@ -18,25 +16,6 @@ namespace {
 constexpr size_t kStaticScratchBytes = FK_NOALLOC_SCRATCH_BYTES;
 
 __device__ __align__(256) unsigned char g_noalloc_scratch[kStaticScratchBytes];
-
-// Device address of g_noalloc_scratch on the current device.  In host code the array's
-// name is only a host-side stand-in, so the address is looked up once per device with
-// cudaGetSymbolAddress (that device current) and cached.
-fk_status scratch_address(void **out) {
-    static std::mutex mu;
-    static void *addr[64] = {};
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return FK_ERR_CUDA;
-    std::lock_guard<std::mutex> lock(mu);
-    if (addr[dev] == nullptr) {
-        void *p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
-            return FK_ERR_CUDA;
-        addr[dev] = p;
-    }
-    *out = addr[dev];
-    return FK_OK;
-}
 
 size_t take(size_t &o, size_t bytes) {
     const size_t at = o;
@@ -52,14 +31,10 @@ using namespace fk;
 extern "C" FK_API fk_status fk_assign_noalloc(const void *X, fk_dtype dtype, int64_t N, int d,
                                               const float *C, int K, int32_t *labels,
                                               fk_stream_t stream) {
-    if (N < 1 || N > 2147483646LL || d < 1 || K < 1 || K > N) return FK_ERR_INVALID_ARG;
+    fk_status s = validate_shape(N, d, K, dtype, FK_L2);
+    if (s != FK_OK) return s;
     if (!X || !C || !labels) return FK_ERR_INVALID_ARG;
-    if (dtype != FK_F32 && dtype != FK_BF16) return FK_ERR_UNSUPPORTED;
-    if ((dtype == FK_F32 && d % 4 != 0) || (dtype == FK_BF16 && d % 8 != 0))
-        return FK_ERR_UNSUPPORTED;
-    if (reinterpret_cast<uintptr_t>(X) % 16 != 0 || reinterpret_cast<uintptr_t>(C) % 4 != 0 ||
-        reinterpret_cast<uintptr_t>(labels) % 4 != 0)
-        return FK_ERR_UNSUPPORTED;
+    if (!aligned(X, 16) || !aligned(C, 4) || !aligned(labels, 4)) return FK_ERR_UNSUPPORTED;
 
     // scratch layout inside the static array
     const int64_t dp = round_up(d, kBK), Kp = round_up(K, kBN);
@@ -72,17 +47,21 @@ extern "C" FK_API fk_status fk_assign_noalloc(const void *X, fk_dtype dtype, int
     const size_t o_ca = take(o, sizeof(uint16_t) * Kp * kAug);
     const size_t o_xs = take(o, sizeof(uint16_t) * xplanes * N * dp);
     if (o > kStaticScratchBytes) return FK_ERR_WORKSPACE;  // beyond the static maximum
+    if ((s = check_device()) != FK_OK) return s;
+    // fk_assign sends some fp32 problems to the screened route, whose candidate and
+    // re-ranking buffers this array does not hold; those are refused here, so the labels
+    // always come from the same kernel as fk_assign's.  (Every depth beyond 768 is such a
+    // problem; below it, no problem that fits the array has enough rows to be screened.)
+    if (dtype == FK_F32 && screened_route(N, static_cast<int>(dp), static_cast<int>(Kp), K))
+        return FK_ERR_UNSUPPORTED;
+    if (injected_fault() == kFaultLaunch) return FK_ERR_CUDA;
 
-    int major = 0, minor = 0, dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
-        return FK_ERR_CUDA;
-    if (major != 10 || minor != 0) return FK_ERR_UNSUPPORTED;
-
+    // In host code g_noalloc_scratch names a host-side stand-in, not device memory: the
+    // array's address on the current device is looked up on every call (cheap next to the
+    // launches and the synchronisation below), so nothing cached can outlive a context.
     void *base = nullptr;
-    fk_status s = scratch_address(&base);
-    if (s != FK_OK) return s;
+    if (cudaGetSymbolAddress(&base, g_noalloc_scratch) != cudaSuccess || base == nullptr)
+        return FK_ERR_CUDA;
     char *sc = static_cast<char *>(base);
     cudaStream_t st = stream;
     uint32_t *err = reinterpret_cast<uint32_t *>(sc + o_err);
@@ -127,13 +106,13 @@ extern "C" FK_API fk_status fk_assign_noalloc(const void *X, fk_dtype dtype, int
     a.xnorm = nullptr;
     a.mind = nullptr;
     a.err = err;
-    a.wait_ns = 2000000000ull;
+    a.wait_ns = kDefaultWaitNs;
     if (launch_assign(a, st) != cudaSuccess) return FK_ERR_CUDA;
 
-    // synchronous: read the device error words back (no allocation involved)
+    // synchronous: read the device error words back (pageable host memory, no allocation)
     uint32_t e[2] = {0, 0};
     if (cudaMemcpyAsync(e, err, sizeof(e), cudaMemcpyDeviceToHost, st) != cudaSuccess ||
         cudaStreamSynchronize(st) != cudaSuccess)
         return FK_ERR_CUDA;
-    return e[0] ? FK_ERR_TIMEOUT : FK_OK;
+    return decode_err(e);
 }

@@ -14,7 +14,9 @@
 //     centroid index on equal values.
 //  3. Rows whose candidates did not fit in their slots are gathered (fb_gather_kernel) and
 //     assigned by the three-product pass, which reads their count on the device, and the
-//     labels are scattered back (fb_scatter_kernel).
+//     labels are scattered back (fb_scatter_kernel).  Beyond a padded depth of 768, where
+//     the three-product form's error is not shown to stay inside half the tie window,
+//     those rows get an exact fp64 scan over all centroids instead (exact_scan_kernel).
 //
 // Everything stays on the stream: no host synchronisation, no data-dependent launches.
 #include <cuda_bf16.h>
@@ -221,6 +223,52 @@ __global__ void fb_scatter_kernel(const uint32_t *__restrict__ nfb,
     }
 }
 
+// Rows queued by the re-ranking whose labels the three-product pass may not decide (padded
+// depth beyond kThreeProductMaxDp): the exact argmin over all K centroids, each distance in
+// the fp64 difference form of lane_dist2 (the re-ranking's own form at these depths), the
+// lowest index on equal values.  One block per queued row at a time (the count is read on
+// the device); warp w takes centroids w, w + 8, ...
+constexpr int kScanWarps = 8;
+__global__ void __launch_bounds__(kScanWarps * 32)
+    exact_scan_kernel(const uint32_t *__restrict__ nfb, const int32_t *__restrict__ fbrows,
+                      const float *__restrict__ X32, const uint16_t *__restrict__ xhi,
+                      const uint16_t *__restrict__ xlo, int64_t lda,
+                      const float *__restrict__ C, int d, int K, int32_t *__restrict__ labels,
+                      float *__restrict__ mind) {
+    __shared__ double s_best[kScanWarps];
+    __shared__ int s_k[kScanWarps];
+    const int lane = threadIdx.x & 31;
+    const int warp = threadIdx.x >> 5;
+    const int64_t n = *nfb;
+    for (int64_t j = blockIdx.x; j < n; j += gridDim.x) {
+        const int64_t row = fbrows[j];
+        double best = 0.0;
+        int bestk = -1;
+        for (int k = warp; k < K; k += kScanWarps) {
+            const double dk = group_sum(lane_dist2(X32, xhi, xlo, lda, C, d, row, k, lane, 32), 32);
+            if (better(dk, k, best, bestk)) {
+                best = dk;
+                bestk = k;
+            }
+        }
+        if (lane == 0) {
+            s_best[warp] = best;
+            s_k[warp] = bestk;
+        }
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            for (int w = 0; w < kScanWarps; ++w)
+                if (better(s_best[w], s_k[w], best, bestk)) {
+                    best = s_best[w];
+                    bestk = s_k[w];
+                }
+            labels[row] = bestk;
+            if (mind) mind[row] = static_cast<float>(best);
+        }
+        __syncthreads();
+    }
+}
+
 }  // namespace
 
 cudaError_t launch_assign_screened(const AssignArgs &a, const float *X32, const float *C,
@@ -250,6 +298,13 @@ cudaError_t launch_assign_screened(const AssignArgs &a, const float *X32, const 
                                          a.labels, a.mind, sb.nfb, sb.fbrows);
     note_launch();
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
+
+    if (a.dp > kThreeProductMaxDp) {  // overflow rows: exact scan instead of three products
+        exact_scan_kernel<<<device_sm_count() * 8, kScanWarps * 32, 0, st>>>(
+            sb.nfb, sb.fbrows, X32, xhi, xlo, a.lda, C, a.d, a.K, a.labels, a.mind);
+        note_launch();
+        return cudaGetLastError();
+    }
 
     fb_gather_kernel<<<148 * 4, 256, 0, st>>>(sb.nfb, sb.fbrows, xhi, a.lda, a.N, a.dp,
                                               sb.xsfb);

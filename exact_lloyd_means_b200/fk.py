@@ -67,6 +67,7 @@ _sig("fk_normalize_rows", [_vp, _vp, _i64, _int, _vp])
 _sig("fk_split_points", [_vp, _i64, _int, _vp, _vp])
 _sig("fk_centroid_norms", [_vp, _int, _int, _int, _vp, _vp])
 _sig("fk_assign", [_vp, _int, _i64, _int, _vp, _int, _vp, _vp, _vp, _sz, _vp])
+_sig("fk_assign_split", [_vp, _vp, _i64, _int, _vp, _int, _vp, _vp, _vp, _sz, _vp])
 _sig("fk_update", [_vp, _int, _i64, _int, _int, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                    _sz, _vp])
 _sig("fk_lloyd", [_vp, _int, _i64, _int, _int, _int, _int, _vp, _vp, _vp, _vp,
@@ -94,7 +95,7 @@ EXPORTED = ["fk_status_string", "fk_version", "fk_workspace_size", "fk_normalize
             "fk_update_partial", "fk_finalize_shards", "fk_split_points",
             "fk_launch_count", "fk_ivf_lists", "fk_lloyd_streamed",
             "fk_streamed_workspace_size", "fk_ivf_norms", "fk_ivf_search_workspace_size",
-            "fk_ivf_search", "fk_ivf_radii"]
+            "fk_ivf_search", "fk_ivf_radii", "fk_assign_split"]
 
 # Bytes of the static device array fk_assign_noalloc takes its scratch from.
 NOALLOC_SCRATCH_BYTES = 8 << 20
@@ -201,12 +202,13 @@ def fk_centroid_norms(C: torch.Tensor, cn: torch.Tensor, dtype=torch.float32, st
 class SplitPoints:
     """fp32 points already split by fk_split_points: one buffer holding the bf16 hi/lo
     planes ([2, N, d_p] bf16, d_p = d rounded up to 64) followed by ||x||^2 per row ([N]
-    fp32).  fk_assign takes it in place of the fp32 tensor (dtype FK_BF16X2) and skips its
-    per-call split."""
+    fp32).  fk_assign takes it in place of the fp32 tensor and skips its per-call split:
+    with the fp32 rows it was made from (`source`) through fk_assign_split, else as
+    FK_BF16X2 planes alone."""
 
-    def __init__(self, buf: torch.Tensor, N: int, d: int):
+    def __init__(self, buf: torch.Tensor, N: int, d: int, source: torch.Tensor | None = None):
         dp = (d + 63) // 64 * 64
-        self.buf, self.N, self.d = buf, N, d
+        self.buf, self.N, self.d, self.source = buf, N, d, source
         self.planes = buf[:2 * N * dp].view(2, N, dp)
         self.norms = buf[2 * N * dp:].view(torch.float32)
 
@@ -232,13 +234,22 @@ def fk_split_points(X: torch.Tensor, out: torch.Tensor | None = None,
     _check(_lib.fk_split_points(_dev(X, "X", torch.float32), N, d,
                                 _dev(out, "out", torch.bfloat16, (2 * N * dp + 2 * N,)),
                                 _stream(stream)), "fk_split_points")
-    return SplitPoints(out, N, d)
+    return SplitPoints(out, N, d, source=X)
 
 
 def fk_assign(X, C: torch.Tensor, labels: torch.Tensor, ws: torch.Tensor,
               mind: torch.Tensor | None = None, stream=None):
     N, d = X.shape
     K = C.shape[0]
+    if isinstance(X, SplitPoints) and X.source is not None:
+        _check(_lib.fk_assign_split(_dev(X.source, "X.source", torch.float32, (N, d)),
+                                    _dev(X.buf, "X.buf", torch.bfloat16), N, d,
+                                    _dev(C, "C", torch.float32, (K, d)), K,
+                                    _dev(labels, "labels", torch.int32, (N,)),
+                                    _opt(mind, "mind", torch.float32, (N,)),
+                                    _dev(ws, "ws", torch.uint8), ws.numel(), _stream(stream)),
+               "fk_assign_split")
+        return
     if isinstance(X, SplitPoints):
         xptr, code = _dev(X.buf, "X.buf", torch.bfloat16), FK_BF16X2
     else:

@@ -163,10 +163,28 @@ FK_API fk_status fk_centroid_norms(const float *C, int K, int d, fk_dtype dtype,
  * per term finds, for every row, the centroids within a proven bound of the nearest; their
  * distances (fp64, difference form) pick the label, and rows with more such
  * centroids than the kernel keeps are assigned by the three-product form.  Labels are the
- * same as the three-product form's outside the parity tie window. */
+ * same as the three-product form's outside the parity tie window.
+ * Deep fp32 points (d rounded up to 64 above 768): the three-product form's error is not
+ * shown to stay within half the tie window there, so every such call takes the screened
+ * route whatever N, and rows whose candidates overflow are assigned by an exact fp64 scan
+ * over all K centroids instead; C must then be 16-byte aligned (else
+ * FK_ERR_UNSUPPORTED).  With FK_BF16X2 input the re-ranking (and that scan) measures the
+ * distances from hi + lo, which is within 2^-16 |x| of x; fk_assign_split keeps them
+ * exact. */
 FK_API fk_status fk_assign(const void *X, fk_dtype dtype, int64_t N, int d, const float *C,
                     int K, int32_t *labels, float *mind, void *ws, size_t ws_bytes,
                     fk_stream_t stream);
+
+/* fk_assign for fp32 points passed twice: as the rows X (N x d fp32, 16-byte aligned),
+ * which the exact fp64 re-ranking of the screened route reads, and as `planes`, the output
+ * of fk_split_points on that same X, which the tensor cores read.  A caller that assigns
+ * the same points repeatedly (the data-parallel Lloyd) splits them once and still gets
+ * exact re-ranking.  Labels and mind equal fk_assign(X, FK_F32) bit for bit; X and
+ * `planes` must stay unchanged between the split and this call.  Workspace:
+ * fk_workspace_size(N, d, K, FK_BF16X2, FK_L2).  Same errors as fk_assign. */
+FK_API fk_status fk_assign_split(const float *X, const void *planes, int64_t N, int d,
+                                 const float *C, int K, int32_t *labels, float *mind,
+                                 void *ws, size_t ws_bytes, fk_stream_t stream);
 
 /* Update step (Flash-KMeans article, "Sort-Inverse Update：原子操作的另一种解法").
  *   counts[k]  = #{i : labels[i] == k}                         (K int32, required)
@@ -363,7 +381,7 @@ FK_API fk_status fk_ivf_search(const float *Q, int64_t nq, int d, const float *C
  * does not allow cudaMalloc behind its back), or on a latency-critical path where
  * cudaMalloc / cudaFree would implicitly synchronise the device.  The paper has no
  * counterpart; it is an interface variant of the assignment step above, with the same
- * labels (bit for bit) as fk_assign on the same inputs.
+ * labels (bit for bit) as fk_assign on the same inputs, since both run the same kernel.
  *   - Scratch (error words, centroid operand planes and norms, and for FK_F32 -- or
  *     FK_BF16 with d % 64 != 0 -- the bf16 planes of X) lives in one file-scope device
  *     array of FK_NOALLOC_SCRATCH_BYTES (8 MiB) inside libfk; every GPU that loads the
@@ -371,14 +389,18 @@ FK_API fk_status fk_ivf_search(const float *Q, int64_t nq, int d, const float *C
  *   - A problem whose scratch does not fit returns FK_ERR_WORKSPACE before any launch
  *     (roughly: FK_F32 needs 4*N*roundup(d,64) + 4*roundup(K,256)*roundup(d,64) bytes,
  *     FK_BF16 with d % 64 == 0 needs 2*roundup(K,256)*d bytes, plus a few KB).
- *   - The first call on a device looks up the array's device address there
- *     (cudaGetSymbolAddress, with that device current) and caches it; make that first
- *     call before any stream capture.
+ *   - fp32 problems that fk_assign would send to its screened route (every
+ *     roundup(d,64) > 768, and large-N shapes that never fit the array anyway) return
+ *     FK_ERR_UNSUPPORTED: that route needs buffers the array does not hold.
+ *   - Each call looks up the array's address on the current device
+ *     (cudaGetSymbolAddress) and checks the result; nothing about the device is cached.
  *   - Every call shares the one array and it keeps the previous call's contents (the
  *     call clears its error words itself).  Calls whose kernels overlap on the GPU (two
  *     host threads, two streams) race on it: serialise them.
- *   - No mind output.  The call is synchronous: it waits for `stream` and returns
- *     FK_ERR_TIMEOUT if a bounded wait inside the kernel expired. */
+ *   - No mind output.  The call is synchronous: it reads the error words back with a
+ *     device-to-host copy and waits for `stream`, so it cannot be called while `stream`
+ *     is being captured into a CUDA graph.  It returns FK_ERR_TIMEOUT if a bounded wait
+ *     inside the kernel expired and FK_ERR_DEVICE if the kernel met a bad value. */
 FK_API fk_status fk_assign_noalloc(const void *X, fk_dtype dtype, int64_t N, int d,
                                    const float *C, int K, int32_t *labels,
                                    fk_stream_t stream);

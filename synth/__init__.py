@@ -11,8 +11,8 @@ more components than nlist), with the 1M x 768, nlist 4096 coarse-quantizer shap
 guide's "性能对比" section, and the d=128, K=32768 shape of the Flash-KMeans article's
 headline run scaled to one GPU.
 """
-from .mixture import (CONFIGS, IVF, LARGE, MID, TINY, ZIPF, MixtureSpec, gaussian_mixture,
-                      init_indices, make_config, mixture_queries)
+from .mixture import (CONFIGS, IVF, LARGE, MID, TINY, ZIPF, MixtureSpec, adversarial_rows,
+                      gaussian_mixture, init_indices, make_config, mixture_queries)
 
 __all__ = ["CONFIGS", "TINY", "IVF", "MID", "ZIPF", "LARGE", "MixtureSpec", "make_config",
-           "gaussian_mixture", "init_indices", "mixture_queries"]
+           "gaussian_mixture", "init_indices", "mixture_queries", "adversarial_rows"]

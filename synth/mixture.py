@@ -25,6 +25,7 @@ import torch
 # Stream ids for the independent generators derived from one seed.
 _S_CENTERS, _S_COMP, _S_NOISE, _S_INIT = 11, 23, 37, 41
 _S_QCOMP, _S_QNOISE = 53, 67  # query draws (offset by 1000 * query stream)
+_S_ADV = 71  # adversarial rounding rows
 
 
 @dataclass(frozen=True)
@@ -129,6 +130,19 @@ def mixture_queries(nq: int, d: int, n_comp: int, *, centers: str = "normal",
                         _gen(device, seed, _S_QCOMP + 1000 * stream),
                         _gen(device, seed, _S_QNOISE + 1000 * stream), device, 1 << 22)
     return Q
+
+
+def adversarial_rows(n: int, d: int, seed: int = 0) -> torch.Tensor:
+    """n x d fp32 rows built to stress bf16 rounding: every coordinate positive and just
+    under half a bf16 unit above a power of two (2^-2 .. 2^2, drawn per coordinate), with a
+    small seeded jitter that keeps it there (1 + (0.49 +- 0.005) 2^-7 times the power).
+    Rounding such operands to bf16 shrinks each by nearly the same relative amount and
+    every partial sum of their products grows, so roundings pile up one way."""
+    g = torch.Generator().manual_seed(seed * 1_000_003 + _S_ADV)
+    e = torch.randint(-2, 3, (n, d), generator=g).double()
+    jit = (torch.rand(n, d, generator=g, dtype=torch.float64) - 0.5) * 0.01
+    m = 1.0 + (0.49 + jit) * 2.0 ** -7
+    return (m * torch.pow(2.0, e)).float()
 
 
 def init_indices(n: int, k: int, seed: int = 0, device="cpu") -> torch.Tensor:

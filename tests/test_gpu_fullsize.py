@@ -36,16 +36,28 @@ def _rows64(X, idx):
     return X[torch.as_tensor(idx, device=X.device)].double().cpu().numpy()
 
 
+def _oracle_normalized_f32(X, chunk=1 << 17):
+    """The oracle's normalisation of every row, rounded to fp32 (in chunks), as a CPU
+    tensor: an input both sides can share."""
+    out = torch.empty(X.shape, dtype=torch.float32)
+    for r0 in range(0, X.shape[0], chunk):
+        r1 = min(X.shape[0], r0 + chunk)
+        out[r0:r1] = torch.from_numpy(
+            oracle.round_f32(oracle.normalize_rows(X[r0:r1].cpu())).astype(np.float32))
+    return out
+
+
 @pytest.mark.parametrize("cfg", [IVF, MID, ZIPF, LARGE])
 def test_fullsize_assign_sampled_rows(cfg):
     spec, X, _, C0 = _data(cfg)
     m = fk()
     Xa = X
     if spec.metric == "cosine":
+        # the product path normalises the points (fk_normalize_rows); the centroids both
+        # sides assign with are the oracle's normalisation of C0, rounded to fp32
         Xa = torch.empty_like(X)
         m.fk_normalize_rows(X, Xa)
-        C0 = C0.clone()
-        m.fk_normalize_rows(C0, C0)
+        C0 = _oracle_normalized_f32(C0).to("cuda")
     labels = torch.empty(spec.n, dtype=torch.int32, device="cuda")
     ws = m.workspace(spec.n, spec.d, spec.k, X.dtype, "l2")
     m.fk_assign(Xa, C0, labels, ws)
@@ -58,9 +70,7 @@ def test_fullsize_assign_sampled_rows(cfg):
     Xs = _rows64(X, idx)
     C = C0.double().cpu().numpy()
     if spec.metric == "cosine":
-        # the oracle normalises the raw rows itself; the centroids it is given are the
-        # fp32 values the GPU assigned with
-        Xs = oracle.normalize_rows(Xs)
+        Xs = oracle.normalize_rows(Xs)  # the oracle normalises the raw rows itself
     if spec.dtype == "bf16":
         C = oracle.round_bf16(C)
     ref, dmin, d2nd = oracle.assign(Xs, C)
@@ -70,11 +80,16 @@ def test_fullsize_assign_sampled_rows(cfg):
     assert bad == 0
 
 
-@pytest.mark.parametrize("cfg", [MID, ZIPF, LARGE])
+@pytest.mark.parametrize("cfg", [IVF, MID, ZIPF, LARGE])
 def test_fullsize_update_given_labels(cfg):
     spec, X, comp, C0 = _data(cfg)
     m = fk()
     K = spec.k
+    if spec.metric == "cosine":
+        # the update of the cosine workload sees normalised points: both sides take the
+        # oracle's normalisation, rounded to fp32
+        X = _oracle_normalized_f32(X).to("cuda")
+        C0 = _oracle_normalized_f32(C0).to("cuda")
     labels = comp.to("cuda")
     C_new = torch.empty_like(C0)
     counts = torch.empty(K, dtype=torch.int32, device="cuda")

@@ -15,7 +15,7 @@ import pytest
 import torch
 
 import oracle
-from synth import gaussian_mixture, init_indices
+from synth import adversarial_rows, gaussian_mixture, init_indices
 from tests.gpu_helpers import (CENTROID_TOL, OBJECTIVE_TOL, centroid_rel_err, fk, gpu_assign,
                                gpu_update, label_mismatches)
 
@@ -139,8 +139,9 @@ def test_lockstep_lloyd_matches_oracle(case):
     """Lockstep: each iteration the GPU assigns with the oracle's centroids and updates
     with the oracle's labels; every output is compared with the oracle's."""
     if case == "tiny_f32":
+        # the 65,536 x 128, K = 256 workload, all five of its iterations
         X, C0, _ = _mixture(65536, 128, 256, "f32", seed=0, sigma=0.1)
-        niter, prec, metric = 3, "f32", "l2"
+        niter, prec, metric = 5, "f32", "l2"
     elif case == "tiny_bf16":
         X, C0, _ = _mixture(30000, 128, 500, "bf16", seed=1, centers="normal", sigma=0.25)
         niter, prec, metric = 3, "bf16", "l2"
@@ -353,18 +354,118 @@ def test_split_points_planes_are_rounded_hi_lo(N, d):
     assert torch.allclose(norms, (X.double() ** 2).sum(1), rtol=1e-6, atol=0)
 
 
-@pytest.mark.parametrize("N,d,K", [(20000, 128, 300), (5000, 768, 1000), (3001, 64, 37)])
+@pytest.mark.parametrize("N,d,K", [(20000, 128, 300), (5000, 768, 1000), (3001, 64, 37),
+                                   (40000, 256, 300), (20000, 1024, 500)])
 def test_assign_pre_split_points_equals_fp32_assign(N, d, K):
-    """fk_assign on fk_split_points planes (FK_BF16X2) gives the fp32 call's labels."""
+    """fk_assign_split (the fp32 rows plus their fk_split_points planes) gives the fp32
+    call's labels and minimum distances bit for bit, on the three-product route, the
+    screened route (40000 x 256) and the deep route (d = 1024)."""
     m = fk()
     X, C0, _ = _mixture(N, d, K, seed=N + K, centers="normal", sigma=0.3)
     Xg, Cg = X.to(DEV), C0.to(DEV)
     ws = m.workspace(N, d, K)
     l1 = torch.empty(N, dtype=torch.int32, device=DEV)
     l2 = torch.empty(N, dtype=torch.int32, device=DEV)
-    m.fk_assign(Xg, Cg, l1, ws)
-    m.fk_assign(m.fk_split_points(Xg), Cg, l2, ws)
-    assert torch.equal(l1, l2)
+    d1 = torch.empty(N, dtype=torch.float32, device=DEV)
+    d2 = torch.empty(N, dtype=torch.float32, device=DEV)
+    m.fk_assign(Xg, Cg, l1, ws, mind=d1)
+    sp = m.fk_split_points(Xg)
+    assert sp.source is not None  # through fk_assign_split
+    m.fk_assign(sp, Cg, l2, ws, mind=d2)
+    assert torch.equal(l1, l2) and torch.equal(d1, d2)
+
+
+@pytest.mark.parametrize("N,d,K", [(40000, 256, 300), (30000, 768, 1024), (3001, 64, 37)])
+def test_assign_planes_only_matches_oracle(N, d, K):
+    """FK_BF16X2 planes without the fp32 rows: the screened route re-ranks from hi + lo
+    (within 2^-16 |x| of x), which must still match the oracle outside the tie window, at
+    screened shapes (N >= 18,944, d >= 256) and on the three-product route."""
+    m = fk()
+    X, C0, _ = _mixture(N, d, K, seed=N + K + 1, centers="normal", sigma=0.3)
+    sp = m.fk_split_points(X.to(DEV))
+    planes_only = m.SplitPoints(sp.buf, N, d)  # no source rows: dtype FK_BF16X2
+    ref, dmin, d2nd = oracle.assign(X, C0.numpy())
+    ties = oracle.tie_mask(X, C0.numpy(), dmin, d2nd)
+    labels = torch.full((N,), -7, dtype=torch.int32, device=DEV)
+    ws = m.workspace(N, d, K)
+    m.fk_assign(planes_only, C0.to(DEV), labels, ws)
+    assert m.fk_get_device_error(ws) == m.FK_OK
+    lab = labels.cpu().numpy()
+    assert (lab >= 0).all() and (lab < K).all()
+    assert label_mismatches(lab, ref, ties) == 0, f"ties={int(ties.sum())}"
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("K,d", [(1000, 96), (257, 768), (1, 8)])
+def test_centroid_norms_match_oracle(K, d, dtype):
+    """fk_centroid_norms: ||c||^2 of the values the tensor cores consume (bf16-rounded for
+    bf16), against the oracle's fp64 distance of each centroid to the origin, rounded once
+    to fp32: within one fp32 ulp (the two fp64 sums differ only in order)."""
+    m = fk()
+    g = torch.Generator().manual_seed(K + d)
+    C = torch.randn(K, d, generator=g) * torch.logspace(-2, 2, K).unsqueeze(1)
+    cn = torch.full((K,), float("nan"), dtype=torch.float32, device=DEV)
+    m.fk_centroid_norms(C.to(DEV), cn, torch.bfloat16 if dtype == "bf16" else torch.float32)
+    Cref = oracle.round_bf16(C.numpy()) if dtype == "bf16" else C.numpy()
+    _, n2, _ = oracle.assign(Cref, np.zeros((1, d)))  # ||c - 0||^2 in fp64
+    ref = n2.astype(np.float32)
+    got = cn.cpu().numpy()
+    ulp = np.spacing(np.abs(ref))
+    assert (np.abs(got.astype(np.float64) - ref) <= ulp).all()
+
+
+# Deep fp32 points (d rounded up to 64 above 768): no label is decided by the three-product
+# form.  At any N every row is screened and re-ranked in fp64, and rows whose candidates
+# overflow get an exact fp64 scan over all centroids.
+DEEP_CASES = [(6000, 1024, 500, "normal", 0.3), (3001, 1032, 257, "normal", 0.3),
+              (25000, 1024, 2000, "normal", 0.3), (700, 1536, 40, "uniform", 0.2),
+              (200, 832, 1, "normal", 0.3)]
+
+
+@pytest.mark.parametrize("N,d,K,centers,sigma", DEEP_CASES)
+def test_deep_fp32_assign_matches_oracle(N, d, K, centers, sigma):
+    X, _, _ = gaussian_mixture(N, d, K, centers=centers, sigma=sigma, seed=N + d)
+    C0 = X[init_indices(N, K, N + d)].float().contiguous()
+    ref, dmin, d2nd = oracle.assign(X, C0.numpy())
+    ties = oracle.tie_mask(X, C0.numpy(), dmin, d2nd)
+    lab, mind = gpu_assign(X.to(DEV), C0.to(DEV), with_mind=True)
+    assert (lab >= 0).all() and (lab < K).all()
+    assert label_mismatches(lab, ref, ties) == 0, f"ties={int(ties.sum())}"
+    # mind is the fp64 difference form rounded to fp32 on this route
+    assert (np.abs(mind.astype(np.float64) - dmin) <= 2 ** -23 * dmin + 1e-30).all()
+
+
+def test_deep_fp32_overflow_rows_take_the_exact_scan():
+    """d = 1024: 30 distinct centroids, each present 20 times, so every row's nearest
+    value is shared by 20 columns and its 16-slot candidate list overflows: every label
+    comes from the exact fp64 scan, which must pick the lowest of the copies."""
+    N, d = 4000, 1024
+    X, _, _ = gaussian_mixture(N, d, 30, centers="normal", sigma=0.3, seed=77)
+    base = X[init_indices(N, 30, 77)].float()
+    C = base.repeat(20, 1).contiguous()  # column 30 * r + j is a copy of base[j]
+    lab, mind = gpu_assign(X.to(DEV), C.to(DEV), with_mind=True)
+    ref, dmin, d2nd = oracle.assign(X, base.numpy())
+    ties = oracle.tie_mask(X, base.numpy(), dmin, d2nd)
+    assert label_mismatches(lab, ref, ties) == 0
+    assert (lab[~ties] < 30).all()
+    assert (np.abs(mind.astype(np.float64) - dmin) <= 2 ** -23 * dmin + 1e-30).all()
+
+
+@pytest.mark.parametrize("N,d,K", [(40000, 256, 300), (4000, 256, 300), (3000, 1024, 200),
+                                   (20000, 128, 1000)])
+def test_assign_adversarial_roundings_match_oracle(N, d, K):
+    """The near-worst-case operands of the window bounds, on the hardware: the screened
+    route (40000 x 256), the three-product route (4000 x 256 and 20000 x 128) and the deep
+    route (d = 1024) must all match the oracle outside the tie window."""
+    X = adversarial_rows(N, d, seed=N + d + K)
+    C0 = X[init_indices(N, K, 5)].contiguous()
+    C = (C0 * 1.0001).contiguous()  # centroids near, not on, their rows
+    ref, dmin, d2nd = oracle.assign(X, C.numpy())
+    ties = oracle.tie_mask(X, C.numpy(), dmin, d2nd)
+    lab, _ = gpu_assign(X.to(DEV), C.to(DEV))
+    assert (lab >= 0).all() and (lab < K).all()
+    assert label_mismatches(lab, ref, ties) == 0, f"ties={int(ties.sum())}"
+    print(f"adversarial {N}x{d}, K={K}: {int(ties.sum())} tie points")
 
 
 # Screened fp32 assignment: for fp32 points with d >= 256 or K * d >= 2^22 at CTA-pair

@@ -440,9 +440,10 @@ int main() {
                             }
                         }
                         const double err = std::fabs(double(acc) - v);
-                        // truncation after every single product is asserted up to d = 768
-                        // only: at d = 1024 it reaches 1.5 half windows (see below)
-                        if (per_product && rz && d > 768) {
+                        // every model is asserted wherever the library lets the three
+                        // products decide a label (padded depth <= kThreeProductMaxDp);
+                        // beyond it the library never does, so the error is only printed
+                        if (dp > kThreeProductMaxDp) {
                             worst_open = std::max(worst_open, err / half_window);
                             continue;
                         }
@@ -460,9 +461,10 @@ int main() {
             }
         }
     }
-    std::printf("%lld three-product values, worst error / half tie window = %.3f, %lld at or "
-                "beyond it; not asserted: truncation after every product at d = 1024 reaches "
-                "%.3f\n", checked, worst, bad, worst_open);
+    std::printf("%lld three-product values up to d_p = %d, worst error / half tie window = "
+                "%.3f, %lld at or beyond it; beyond d_p = %d (never used there) the worst model "
+                "reaches %.3f\n", checked, kThreeProductMaxDp, worst, bad, kThreeProductMaxDp,
+                worst_open);
     return bad == 0 ? 0 : 1;
 }
 """
@@ -474,10 +476,12 @@ def test_three_product_assignment_stays_inside_half_the_tie_window(tmp_path):
     the norm folded in first, as the kernel does) has an error below half the parity
     rule's tie window, so every point outside the window keeps its exact label.  Emulated
     as above, with normal, nearly parallel and adversarial data (split residuals as large
-    as they get).  Asserted for one rounding per MMA step (to nearest or toward zero) at
-    every d, and for one rounding per product up to d = 768.  Truncating after every
-    single product at d = 1024 is the one model that leaves the half window (about 1.5x);
-    it is printed, not asserted."""
+    as they get).  Every model (one rounding per MMA step or per product, to nearest or
+    toward zero) is asserted at every depth up to the library's kThreeProductMaxDp (768),
+    the deepest at which the three products still decide labels.  Beyond it (d = 1024
+    here) truncation after every single product leaves the half window (about 1.5x); the
+    library then sends every row to the screened route with exact fp64 re-ranking and an
+    exact scan for overflowing rows, so that figure is printed, not asserted."""
     src = tmp_path / "three.cu"
     src.write_text(THREE_PROGRAM)
     exe = tmp_path / "three"
