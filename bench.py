@@ -5,8 +5,11 @@ normalisation once, then assign + sort + update per iteration) over the workload
 synthetic points, starting from the same initial centroids every step.  The metric is
 points x iterations per second for the whole job.
 
-Default workload: N = 1,000,000 points, d = 768, K = 4096, fp32, cosine, 20 iterations
-(the IVF coarse-quantizer build shape of the LEANN FlashLib guide, section "性能对比").
+Default workload: N = 100,000,000 points, d = 128, K = 32,768, bf16 points with fp32
+accumulation and fp32 centroid sums, 3 iterations: the d = 128, K = 32,768 shape of the
+Flash-KMeans article's headline run (opening paragraph: 1e9 points on an H200), scaled to
+one GPU's memory.  --workload selects the others (synth.CONFIGS), e.g. the LEANN FlashLib
+guide's 1M x 768, nlist 4096 coarse-quantizer build (section "性能对比").
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
 
@@ -42,7 +45,7 @@ def parse():
     p.add_argument("--gpus", type=int, default=1)
     p.add_argument("--steps", type=int, default=5)
     p.add_argument("--warmup", type=int, default=3)
-    p.add_argument("--workload", default="ivf_1000000x768_k4096_f32_cosine",
+    p.add_argument("--workload", default="large_100000000x128_k32768_bf16",
                    help="one of synth.CONFIGS")
     p.add_argument("--niter", type=int, default=None)
     p.add_argument("--n", type=int, default=None,
