@@ -26,6 +26,8 @@
 //     bf16 points (NP = 1): one product, exact in fp32.
 //   * every mbarrier wait is bounded; on expiry the CTA raises the abort flag, records
 //     the timeout in the workspace error word and winds down (TMEM is always freed).
+#include <type_traits>
+
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -94,6 +96,19 @@ __device__ __forceinline__ void init_aug_a(uint8_t *aaug, int r) {
     row[1 ^ sw] = zero;
 }
 
+// Calls f(std::integral_constant<int, i>{}) for i = 0 .. n - 1, unrolled at compile time.
+template <int I, int N, typename F>
+__device__ __forceinline__ void static_for_impl(F &&f) {
+    if constexpr (I < N) {
+        f(std::integral_constant<int, I>{});
+        static_for_impl<I + 1, N>(f);
+    }
+}
+template <int N, typename F>
+__device__ __forceinline__ void static_for(F &&f) {
+    static_for_impl<0, N>(f);
+}
+
 // Minimum of 64 values with three-input mins: 21 + 7 + 3 + 1 instructions.
 
 __device__ __forceinline__ float min64(const float (&v)[64]) {
@@ -108,6 +123,42 @@ __device__ __forceinline__ float min64(const float (&v)[64]) {
     const float a = ptx::fmin3(u[0], u[1], u[2]);
     const float b = ptx::fmin3(u[3], u[4], u[5]);
     return ptx::fmin3(a, b, fminf(u[6], u[7]));
+}
+
+// Minimum of 64 values as the minimum of eight groups of eight (their minima in g8): 36
+// three-input mins, a few more than min64, so that the first index of the minimum can be
+// found group by group.
+__device__ __forceinline__ float min64_groups(const float (&v)[64], float (&g8)[8]) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+        g8[i] = ptx::fmin3(ptx::fmin3(v[8 * i], v[8 * i + 1], v[8 * i + 2]),
+                           ptx::fmin3(v[8 * i + 3], v[8 * i + 4], v[8 * i + 5]),
+                           fminf(v[8 * i + 6], v[8 * i + 7]));
+    return ptx::fmin3(ptx::fmin3(g8[0], g8[1], g8[2]), ptx::fmin3(g8[3], g8[4], g8[5]),
+                      fminf(g8[6], g8[7]));
+}
+
+// First column of v equal to m (the minimum), for the lanes with `want`.  Every lane of
+// the warp must call it, together (it votes across the full warp).  The group holding it
+// is the first whose minimum is m; a group's eight columns are scanned only if some lane
+// of the warp needs that group, so a warp in which one row improved pays for one group
+// rather than all 64 columns.
+__device__ __forceinline__ int first_index_of(const float (&v)[64], const float (&g8)[8],
+                                              float m, bool want) {
+    int gi = 7;
+#pragma unroll
+    for (int i = 6; i >= 0; --i) gi = g8[i] == m ? i : gi;
+    int idx = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        if (__any_sync(0xffffffffu, want && gi == i)) {
+            int j = 7;
+#pragma unroll
+            for (int q = 6; q >= 0; --q) j = v[8 * i + q] == m ? q : j;
+            idx = gi == i ? 8 * i + j : idx;
+        }
+    }
+    return idx;
 }
 
 // Screening: add the columns base + bit of `mask` (screened values >= m, the minimum of
@@ -514,25 +565,33 @@ struct PairCfg {
     // resident X: one stage holds all (<= 2) k-chunks of a tile's centroids, so a tile costs
     // one full-wait and one empty-commit; streamed X: one k-chunk of X and centroids
     static constexpr int kStageChunks = RES ? kAChunks : 1;
+    static constexpr int kAugA = kBM * kAug * 2;         // 4 KB: constant (1, 1, 1, 0, ...)
+    static constexpr int kAugB = (kBN / 2) * kAug * 2;   // 4 KB: this CTA's 128 norms
+    // resident X: a stage is one tile, its centroid chunks followed by its norm pieces (so
+    // one barrier covers both); streamed X: a stage is one chunk of X and of the centroids,
+    // and the norm pieces have a ring of kAugSlots slots of their own, each freed by a
+    // commit right after its norm MMA
+    static constexpr int kNormOff = kStageChunks * NP * kBBytes;  // resident X only
     static constexpr int kStageBytes =
-        RES ? kStageChunks * NP * kBBytes : NP * (kABytes + kBBytes);
+        RES ? kNormOff + kAugB : NP * (kABytes + kBBytes);
     static constexpr int kStages = RES ? (NP == 1 ? 4 : 2) : (NP == 2 ? 3 : 6);
-    static constexpr int kDataBytes = kARegion + kStages * kStageBytes;  // 192 KB
+    static constexpr int kDataBytes = kARegion + kStages * kStageBytes;
     static constexpr int kBarBytes = 512;
     // epilogue warpgroups splitting a tile's columns: 4 for the argmin; 1 for the screening
     // pass, whose per-row candidate list must see all 256 columns of every tile
     static constexpr int kEpiGroups = EG;
     static constexpr int kEpiCols = kBN / kEpiGroups;
     static constexpr int kRedBytes = (kEpiGroups - 1) * 2 * kBM * 8;
-    static constexpr int kAugA = kBM * kAug * 2;         // 4 KB: constant (1, 1, 1, 0, ...)
-    static constexpr int kAugB = (kBN / 2) * kAug * 2;   // 4 KB: this CTA's 128 norms
-    static constexpr int kAugRegion = kAugA + 2 * kAugB;
+    static constexpr int kAugSlots = RES ? 0 : 4;
+    static constexpr int kAugRegion = kAugA + kAugSlots * kAugB;
     static constexpr int kSmemBytes = kDataBytes + kAugRegion + kBarBytes + kRedBytes + 1024;
     static constexpr int kEpiWarps = 4 * kEpiGroups;
     static constexpr int kThreads = 64 + kEpiWarps * 32;
     static constexpr int kTmemCols = 2 * kBN;
     static_assert(kStages <= 8, "stage masks");
+    static_assert(kStageBytes % 1024 == 0, "stage bases stay 1024-byte aligned");
     static_assert(kSmemBytes <= 232448, "shared memory");
+    static_assert(8 * (2 * kStages + 12 + 2 * kAugSlots + 1) + 8 <= kBarBytes, "barriers");
 };
 
 template <int NP, bool RES, bool SCR>
@@ -562,7 +621,7 @@ __global__ void __launch_bounds__(PairCfg<NP, RES, SCR ? 1 : 4>::kThreads, 1)
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     uint8_t *ring = smem + Cfg::kARegion;
     uint8_t *aaug = smem + Cfg::kDataBytes;  // constant A block of the norm step
-    uint8_t *baug = aaug + Cfg::kAugA;       // [2][128 rows][32 B]
+    uint8_t *baug = aaug + Cfg::kAugA;       // [kAugSlots][128 rows][32 B]
     uint64_t *full =
         reinterpret_cast<uint64_t *>(smem + Cfg::kDataBytes + Cfg::kAugRegion);  // even CTA
     uint64_t *empty = full + S;
@@ -572,8 +631,9 @@ __global__ void __launch_bounds__(PairCfg<NP, RES, SCR ? 1 : 4>::kThreads, 1)
     uint64_t *aempty = afull + 2;
     uint64_t *redfull = aempty + 2;
     uint64_t *redempty = redfull + 2;
-    uint64_t *augfull = redempty + 2;  // even CTA
-    uint64_t *drain = augfull + 2;
+    uint64_t *augfull = redempty + 2;  // even CTA, [kAugSlots]
+    uint64_t *augempty = augfull + Cfg::kAugSlots;  // both CTAs, [kAugSlots]
+    uint64_t *drain = augempty + Cfg::kAugSlots;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
     volatile uint32_t *abort_flag = tmem_slot + 1;
     float *red_v = reinterpret_cast<float *>(smem + Cfg::kDataBytes + Cfg::kAugRegion +
@@ -600,7 +660,10 @@ __global__ void __launch_bounds__(PairCfg<NP, RES, SCR ? 1 : 4>::kThreads, 1)
                 ptx::mbar_init(&redfull[a], (Cfg::kEpiGroups - 1) * kBM);
                 ptx::mbar_init(&redempty[a], kBM);
             }
+        }
+        for (int a = 0; a < Cfg::kAugSlots; ++a) {
             ptx::mbar_init(&augfull[a], 1);
+            ptx::mbar_init(&augempty[a], 1);
         }
         ptx::mbar_init(drain, 1);
         *abort_flag = 0u;
@@ -662,17 +725,17 @@ __global__ void __launch_bounds__(PairCfg<NP, RES, SCR ? 1 : 4>::kThreads, 1)
                 }
                 for (int nt = 0; nt < ntiles && ok; ++nt, ++titer) {
                     const int crow = nt * kBN + static_cast<int>(rank) * (kBN / 2);
-                    {
-                        // the norm slot is free once the tile two back (same slot) completed
-                        const uint32_t acc = titer & 1u;
-                        const uint32_t aphase = (titer >> 1) & 1u;
-                        if (!ptx::mbar_wait(&tfull[acc], aphase ^ 1u, abort_flag, wait_ns)) {
+                    if constexpr (!RES) {
+                        // the norm slot is free once the norm MMA of its previous tile ran
+                        const uint32_t as = titer % Cfg::kAugSlots;
+                        const uint32_t asp = (titer / Cfg::kAugSlots) & 1u;
+                        if (!ptx::mbar_wait(&augempty[as], asp ^ 1u, abort_flag, wait_ns)) {
                             raise_timeout(abort_flag, err);
                             ok = false;
                             break;
                         }
-                        if (rank == 0) ptx::mbar_arrive_expect_tx(&augfull[acc], 2 * Cfg::kAugB);
-                        ptx::tma_load_2d_pair(baug + acc * Cfg::kAugB, &tmC, augfull_c + acc * 8,
+                        if (rank == 0) ptx::mbar_arrive_expect_tx(&augfull[as], 2 * Cfg::kAugB);
+                        ptx::tma_load_2d_pair(baug + as * Cfg::kAugB, &tmC, augfull_c + as * 8,
                                               0, crow);
                     }
                     for (int kc = 0; kc < nkc; kc += Cfg::kStageChunks) {
@@ -684,12 +747,13 @@ __global__ void __launch_bounds__(PairCfg<NP, RES, SCR ? 1 : 4>::kThreads, 1)
                         const int nch = nkc - kc < Cfg::kStageChunks ? nkc - kc
                                                                      : Cfg::kStageChunks;
                         if (rank == 0)
-                            ptx::mbar_arrive_expect_tx(&full[stage],
-                                                       2 * nch * NP * (RES ? Cfg::kBBytes
-                                                                           : Cfg::kABytes +
-                                                                                 Cfg::kBBytes));
+                            ptx::mbar_arrive_expect_tx(
+                                &full[stage], RES ? 2 * (nch * NP * Cfg::kBBytes + Cfg::kAugB)
+                                                  : 2 * nch * NP * (Cfg::kABytes + Cfg::kBBytes));
                         uint8_t *st = ring + stage * Cfg::kStageBytes;
                         const uint32_t fb = full_c + stage * 8;
+                        if (RES)  // the tile's norm pieces, behind its centroid chunks
+                            ptx::tma_load_2d_pair(st + Cfg::kNormOff, &tmC, fb, 0, crow);
                         for (int c = 0; c < nch; ++c) {
                             uint8_t *sb = st + c * NP * Cfg::kBBytes;
                             if (!RES) {
@@ -722,19 +786,81 @@ __global__ void __launch_bounds__(PairCfg<NP, RES, SCR ? 1 : 4>::kThreads, 1)
                 uint32_t stage = 0, phase = 0, mbi = 0;
                 const uint32_t aaug_s = ptx::smem_u32(aaug);
                 const uint32_t baug_s = ptx::smem_u32(baug);
-                for (int64_t mb = pair; mb < nmb && ok; mb += npairs, ++mbi) {
-                    uint32_t abase = 0, ab = 0;
-                    if (RES) {
-                        ab = mbi % Cfg::kABufs;
-                        const uint32_t apar = (mbi / Cfg::kABufs) & 1u;
-                        if (!ptx::mbar_wait(&afull[ab], apar, abort_flag, wait_ns)) {
-                            raise_timeout(abort_flag, err);
-                            ok = false;
-                            break;
-                        }
+                if constexpr (RES) {
+                    // Resident X: a tile is one stage (its centroid chunks and its norm
+                    // pieces, behind one barrier).  Issuing an MMA blocks while the tensor
+                    // pipe's short queue (about one MMA) is full, so whatever the issuing
+                    // thread does between tiles leaves the pipe idle: the boundary is kept
+                    // short (two commits, non-blocking tests of the next stage and
+                    // accumulator that nearly always pass at once, bounded waits behind
+                    // them) and the MMA sequence is unrolled with its descriptors folded.
+                    // Waiting for the next tile earlier, inside the current tile's MMAs, was
+                    // measured slower: the accumulator is released only while the current
+                    // tile runs.
+                    constexpr int P = NP == 2 ? 3 : 1;           // MMAs per K step
+                    constexpr int kMaxM = Cfg::kAChunks * (kBK / 16) * P;
+                    const int nm = nkc * (kBK / 16) * P;         // data MMAs per tile
+                    auto wait_bar = [&](uint64_t *bar, uint32_t par) -> bool {
+                        if (ptx::mbar_test(bar, par) ||
+                            ptx::mbar_wait(bar, par, abort_flag, wait_ns))
+                            return true;
+                        raise_timeout(abort_flag, err);
+                        return false;
+                    };
+                    // tile ti's stage (the producer's order) and accumulator
+                    auto wait_tile = [&](uint32_t ti, uint32_t stg, uint32_t ph) -> bool {
+                        return wait_bar(&full[stg], ph) &&
+                               wait_bar(&tempty[ti & 1u], ((ti >> 1) & 1u) ^ 1u);
+                    };
+                    auto wait_block = [&](uint32_t bi) -> bool {
+                        return wait_bar(&afull[bi % Cfg::kABufs], (bi / Cfg::kABufs) & 1u);
+                    };
+                    int64_t mb = pair;
+                    int nt = 0;
+                    if (mb < nmb) ok = wait_block(0) && wait_tile(0, 0, 0);
+                    while (ok && mb < nmb) {
                         ptx::tc_fence_after();
-                        abase = ptx::smem_u32(smem + ab * Cfg::kABufBytes);
+                        const uint32_t ab = mbi % Cfg::kABufs;
+                        const uint32_t acc = titer & 1u;
+                        const uint32_t dt = tmem + acc * kBN;
+                        const uint32_t st = ptx::smem_u32(ring + stage * Cfg::kStageBytes);
+                        const uint64_t dA = ptx::sdesc_k_sw128(
+                            ptx::smem_u32(smem + ab * Cfg::kABufBytes));
+                        const uint64_t dB = ptx::sdesc_k_sw128(st);
+                        // D = ||c||^2 (hi + mid + lo against the constant ones)
+                        ptx::mma_bf16_ss_pair(dt, ptx::sdesc_k_sw32(aaug_s),
+                                              ptx::sdesc_k_sw32(st + Cfg::kNormOff), idesc, 0u);
+                        // data MMA i: chunk c, K step ks, product (hi.hi, lo.hi, hi.lo); a
+                        // descriptor's address field advances by bytes / 16
+                        static_for<kMaxM>([&](auto ic) {
+                            constexpr int i = decltype(ic)::value;
+                            constexpr int c = i / ((kBK / 16) * P);
+                            constexpr int ks = (i / P) % (kBK / 16);
+                            constexpr int pa = i % P == 1 ? 1 : 0;
+                            constexpr int pb = i % P == 2 ? 1 : 0;
+                            constexpr uint64_t oa = ((c * NP + pa) * Cfg::kABytes) / 16 + 2 * ks;
+                            constexpr uint64_t ob = ((c * NP + pb) * Cfg::kBBytes) / 16 + 2 * ks;
+                            if (i < nm) ptx::mma_bf16_ss_pair(dt, dA + oa, dB + ob, idesc, 1u);
+                        });
+                        ptx::mma_commit_pair(&empty[stage], 0x3);
+                        ptx::mma_commit_pair(&tfull[acc], 0x3);
+                        // the next tile in this pair's order
+                        if (++nt == ntiles) {
+                            ptx::mma_commit_pair(&aempty[ab], 0x3);  // this X block is done
+                            nt = 0;
+                            mb += npairs;
+                            ++mbi;
+                        }
+                        ++titer;
+                        if (++stage == S) {
+                            stage = 0;
+                            phase ^= 1u;
+                        }
+                        if (mb < nmb)
+                            ok = (nt != 0 || wait_block(mbi)) && wait_tile(titer, stage, phase);
                     }
+                } else {
+                for (int64_t mb = pair; mb < nmb && ok; mb += npairs, ++mbi) {
                     for (int nt = 0; nt < ntiles && ok; ++nt, ++titer) {
                         const uint32_t acc = titer & 1u;
                         const uint32_t aphase = (titer >> 1) & 1u;
@@ -743,7 +869,9 @@ __global__ void __launch_bounds__(PairCfg<NP, RES, SCR ? 1 : 4>::kThreads, 1)
                             ok = false;
                             break;
                         }
-                        if (!ptx::mbar_wait(&augfull[acc], aphase, abort_flag, wait_ns)) {
+                        const uint32_t as = titer % Cfg::kAugSlots;
+                        const uint32_t asp = (titer / Cfg::kAugSlots) & 1u;
+                        if (!ptx::mbar_wait(&augfull[as], asp, abort_flag, wait_ns)) {
                             raise_timeout(abort_flag, err);
                             ok = false;
                             break;
@@ -752,37 +880,32 @@ __global__ void __launch_bounds__(PairCfg<NP, RES, SCR ? 1 : 4>::kThreads, 1)
                         const uint32_t dt = tmem + acc * kBN;
                         // D = ||c||^2 (hi + mid + lo against the constant ones)
                         ptx::mma_bf16_ss_pair(dt, ptx::sdesc_k_sw32(aaug_s),
-                                              ptx::sdesc_k_sw32(baug_s + acc * Cfg::kAugB),
+                                              ptx::sdesc_k_sw32(baug_s + as * Cfg::kAugB),
                                               idesc, 0u);
-                        for (int kc = 0; kc < nkc; kc += Cfg::kStageChunks) {
+                        ptx::mma_commit_pair(&augempty[as], 0x3);  // the slot may be refilled
+                        for (int kc = 0; kc < nkc; ++kc) {  // streamed X: a stage per chunk
                             if (!ptx::mbar_wait(&full[stage], phase, abort_flag, wait_ns)) {
                                 raise_timeout(abort_flag, err);
                                 ok = false;
                                 break;
                             }
                             ptx::tc_fence_after();
-                            const int nch = nkc - kc < Cfg::kStageChunks ? nkc - kc
-                                                                         : Cfg::kStageChunks;
                             const uint32_t st = ptx::smem_u32(ring + stage * Cfg::kStageBytes);
-                            for (int c = 0; c < nch; ++c) {
-                                const uint32_t a0 =
-                                    RES ? abase + ((kc + c) * NP) * Cfg::kABytes : st;
-                                const uint32_t a1 = a0 + Cfg::kABytes;
-                                const uint32_t b0 =
-                                    RES ? st + c * NP * Cfg::kBBytes : st + NP * Cfg::kABytes;
-                                const uint32_t b1 = b0 + Cfg::kBBytes;
-                                const uint64_t da0 = ptx::sdesc_k_sw128(a0);
-                                const uint64_t da1 = ptx::sdesc_k_sw128(a1);
-                                const uint64_t db0 = ptx::sdesc_k_sw128(b0);
-                                const uint64_t db1 = ptx::sdesc_k_sw128(b1);
+                            const uint32_t a0 = st;
+                            const uint32_t a1 = a0 + Cfg::kABytes;
+                            const uint32_t b0 = st + NP * Cfg::kABytes;
+                            const uint32_t b1 = b0 + Cfg::kBBytes;
+                            const uint64_t da0 = ptx::sdesc_k_sw128(a0);
+                            const uint64_t da1 = ptx::sdesc_k_sw128(a1);
+                            const uint64_t db0 = ptx::sdesc_k_sw128(b0);
+                            const uint64_t db1 = ptx::sdesc_k_sw128(b1);
 #pragma unroll
-                                for (int ks = 0; ks < kBK / 16; ++ks) {
-                                    const uint64_t o = 2u * ks;  // +32 bytes along K
-                                    ptx::mma_bf16_ss_pair(dt, da0 + o, db0 + o, idesc, 1u);
-                                    if (NP == 2) {
-                                        ptx::mma_bf16_ss_pair(dt, da1 + o, db0 + o, idesc, 1u);
-                                        ptx::mma_bf16_ss_pair(dt, da0 + o, db1 + o, idesc, 1u);
-                                    }
+                            for (int ks = 0; ks < kBK / 16; ++ks) {
+                                const uint64_t o = 2u * ks;  // +32 bytes along K
+                                ptx::mma_bf16_ss_pair(dt, da0 + o, db0 + o, idesc, 1u);
+                                if (NP == 2) {
+                                    ptx::mma_bf16_ss_pair(dt, da1 + o, db0 + o, idesc, 1u);
+                                    ptx::mma_bf16_ss_pair(dt, da0 + o, db1 + o, idesc, 1u);
                                 }
                             }
                             ptx::mma_commit_pair(&empty[stage], 0x3);
@@ -792,9 +915,9 @@ __global__ void __launch_bounds__(PairCfg<NP, RES, SCR ? 1 : 4>::kThreads, 1)
                             }
                         }
                         if (!ok) break;
-                        ptx::mma_commit_pair(&tfull[acc], 0x3);  // also frees the norm slot
+                        ptx::mma_commit_pair(&tfull[acc], 0x3);
                     }
-                    if (RES && ok) ptx::mma_commit_pair(&aempty[ab], 0x3);
+                }
                 }
                 if (!ok) {
                     ptx::mma_commit_pair(drain, 0x1);
@@ -941,14 +1064,17 @@ __global__ void __launch_bounds__(PairCfg<NP, RES, SCR ? 1 : 4>::kThreads, 1)
                 ptx::tc_fence_before();
                 __syncwarp();
                 if (lane == 0) ptx::mbar_arrive_cluster(tempty_c + acc * 8);  // consumed
-                const float m = min64(v);
-                if (m < best) {
-                    int idx = 0;
-#pragma unroll
-                    for (int j = EC - 1; j >= 0; --j)
-                        if (v[j] == m) idx = j;
-                    best = m;
-                    bestk = colbase + idx;
+                float g8[8];  // minima of the eight groups of eight columns
+                const float m = min64_groups(v, g8);
+                const bool imp = m < best;
+                if (__any_sync(0xffffffffu, imp)) {
+                    // every lane of the warp takes part in the search (it votes across the
+                    // warp); only the lanes whose row improved keep its result
+                    const int idx = first_index_of(v, g8, m, imp);
+                    if (imp) {
+                        best = m;
+                        bestk = colbase + idx;
+                    }
                 }
             }
             if (!ok) break;
