@@ -87,16 +87,19 @@ def load_peaks():
 
 
 def assign_traffic_record(workload):
-    """DRAM bytes per assign launch from a committed ncu summary, if it was taken on the
+    """DRAM bytes per assign launch from a committed ncu summary, if one was taken on the
     current kernel source and for this workload (else None)."""
     path = os.path.join(ROOT, "profiles", "assign_traffic.json")
     src = os.path.join(ROOT, "exact_lloyd_means_b200", "csrc", "assign_sm100.cu")
     if not os.path.exists(path):
         return None
     with open(path) as f:
-        rec = json.load(f)
+        recs = json.load(f).get("records", [])
     h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
-    return rec if rec.get("kernel_sha") == h and rec.get("workload") == workload else None
+    for rec in recs:
+        if rec.get("kernel_sha") == h and rec.get("workload") == workload:
+            return rec
+    return None
 
 
 class ClockSampler:
