@@ -67,7 +67,7 @@ __device__ __forceinline__ void store_piece(double *dst, const double (&acc)[4])
     q[1] = make_double2(acc[2], acc[3]);
 }
 
-// Level 1 for fp32 points (bf16 points use seg_rows_regs_kernel below).  A warp owns
+// Level 1 for fp32 points (bf16 points use seg_rows_cp_kernel below).  A warp owns
 // sorted positions [w*R, w*R + R) and the 128 columns of block blockIdx.y (lane l holds
 // columns 4l .. 4l+3).  The warp first stages the R cluster ids and row ids of its chunk in
 // shared memory (one coalesced read).  Rows are then gathered with 1-D bulk copies (one
@@ -77,16 +77,16 @@ __device__ __forceinline__ void store_piece(double *dst, const double (&acc)[4])
 // first added pairwise in fp32 (a fixed tree) and the batch sum is added to the fp64
 // accumulator once; otherwise rows are added one by one in fp64.  The objective term
 // (x - c_used)^2 of a row is formed in fp32 and accumulated in fp64.
-constexpr int kRowRing = 4;        // batches in flight per warp
 constexpr int kRowWarps = 4;       // warps per block of the level-1 kernel
-constexpr int kRowBatchBytes = 4096;  // 8 fp32 rows of 128 columns
+constexpr int kRowBatchRows = 8;   // rows per batch (one mbarrier each)
 
 template <bool BF16>
 struct RowVec;
 template <>
 struct RowVec<false> {
-    static constexpr int kBatch = 8;
+    static constexpr int kBatch = kRowBatchRows;
     static constexpr int kSlice = 512;  // bytes of a 128-column slice
+    static constexpr int kRing = 4;     // batches in flight per warp: 16 KB
     __device__ static void load(const uint8_t *p, float (&f)[4]) {
         const float4 v = *reinterpret_cast<const float4 *>(p);
         f[0] = v.x;
@@ -95,7 +95,13 @@ struct RowVec<false> {
         f[3] = v.w;
     }
 };
-constexpr size_t kRowSmem = size_t(kRowWarps) * kRowRing * kRowBatchBytes;  // dynamic part
+template <bool BF16>
+constexpr int kRowBatchBytes = kRowBatchRows * RowVec<BF16>::kSlice;
+template <bool BF16>
+constexpr int kRowRing = RowVec<BF16>::kRing;
+// the dynamic shared memory of a block: every warp's ring of batches
+template <bool BF16>
+constexpr size_t kRowSmem = size_t(kRowWarps) * kRowRing<BF16> * kRowBatchBytes<BF16>;
 
 template <bool BF16>
 __global__ void __launch_bounds__(kRowWarps * 32, 3)
@@ -111,12 +117,14 @@ __global__ void __launch_bounds__(kRowWarps * 32, 3)
     using RV = RowVec<BF16>;
     constexpr int B = RV::kBatch;
     constexpr int SL = RV::kSlice;
+    constexpr int kRing = kRowRing<BF16>;
+    constexpr int kBatchBytes = kRowBatchBytes<BF16>;
     constexpr int E = BF16 ? 2 : 4;
     constexpr uint64_t kWaitNs = 2000000000ull;
     extern __shared__ __align__(128) uint8_t s_rows_all[];  // [warp][ring][B][SL]
     __shared__ int32_t s_key[kRowWarps][kUpdMaxRows];
     __shared__ int32_t s_row[kRowWarps][kUpdMaxRows];
-    __shared__ __align__(8) uint64_t s_bar[kRowWarps][kRowRing];
+    __shared__ __align__(8) uint64_t s_bar[kRowWarps][kRing];
     const int lane = threadIdx.x & 31;
     const int wib = threadIdx.x >> 5;
     const int64_t w = static_cast<int64_t>(blockIdx.x) * kRowWarps + wib;
@@ -132,8 +140,8 @@ __global__ void __launch_bounds__(kRowWarps * 32, 3)
     int32_t *sk = s_key[wib];
     int32_t *si = s_row[wib];
     uint64_t *bar = s_bar[wib];
-    uint8_t *rows = s_rows_all + static_cast<size_t>(wib) * kRowRing * kRowBatchBytes;
-    if (lane < kRowRing) ptx::mbar_init(&bar[lane], 1);
+    uint8_t *rows = s_rows_all + static_cast<size_t>(wib) * kRing * kBatchBytes;
+    if (lane < kRing) ptx::mbar_init(&bar[lane], 1);
     ptx::fence_mbar_init();
     for (int j = lane; j < n; j += 32) {
         sk[j] = skeys[p0 + j];
@@ -151,7 +159,7 @@ __global__ void __launch_bounds__(kRowWarps * 32, 3)
         if (lane == 0) ptx::mbar_arrive_expect_tx(&bar[slot], nb * slice);
         __syncwarp();
         if (lane < nb)
-            ptx::bulk_load(rows + slot * kRowBatchBytes + lane * SL,
+            ptx::bulk_load(rows + slot * kBatchBytes + lane * SL,
                            Xb + (static_cast<int64_t>(si[b + lane]) * d + col0) * E, slice,
                            &bar[slot]);
     };
@@ -190,18 +198,18 @@ __global__ void __launch_bounds__(kRowWarps * 32, 3)
         }
     };
 
-    for (int i = 0; i < kRowRing; ++i) issue(i * B, i);
+    for (int i = 0; i < kRing; ++i) issue(i * B, i);
     int it = 0;
     for (int b = 0; b < n; b += B, ++it) {
-        const int slot = it % kRowRing;
+        const int slot = it % kRing;
         uint32_t got = 1;
-        if (lane == 0) got = ptx::mbar_wait(&bar[slot], (it / kRowRing) & 1u, nullptr, kWaitNs);
+        if (lane == 0) got = ptx::mbar_wait(&bar[slot], (it / kRing) & 1u, nullptr, kWaitNs);
         if (!__shfl_sync(0xffffffffu, got, 0)) {
             if (lane == 0) err[0] = kErrTimeout;
             ok = false;
             break;
         }
-        const uint8_t *base = rows + slot * kRowBatchBytes + lane * (4 * E);
+        const uint8_t *base = rows + slot * kBatchBytes + lane * (4 * E);
         const int nb = n - b < B ? n - b : B;
         const int kf = sk[b], kl = sk[b + nb - 1];
         if (kf == kl) {
@@ -256,13 +264,13 @@ __global__ void __launch_bounds__(kRowWarps * 32, 3)
         }
         ptx::fence_proxy_async_smem();  // this lane's reads of the slot precede the refill
         __syncwarp();                   // every lane has read the slot before it is refilled
-        issue(b + kRowRing * B, slot);
+        issue(b + kRing * B, slot);
     }
     if (!ok) {
-        // let the (at most kRowRing) copies still outstanding land before the warp leaves
-        for (int i2 = it; i2 < it + kRowRing && i2 * B < n; ++i2) {
+        // let the (at most kRing) copies still outstanding land before the warp leaves
+        for (int i2 = it; i2 < it + kRing && i2 * B < n; ++i2) {
             if (lane == 0)
-                ptx::mbar_wait(&bar[i2 % kRowRing], (i2 / kRowRing) & 1u, nullptr, kWaitNs);
+                ptx::mbar_wait(&bar[i2 % kRing], (i2 / kRing) & 1u, nullptr, kWaitNs);
         }
         return;
     }
@@ -277,11 +285,7 @@ __global__ void __launch_bounds__(kRowWarps * 32, 3)
     if (lane == 0) jpart[static_cast<int64_t>(cb) * nwarps + w] = jacc;
 }
 
-// Level 1, register-gather form, used for bf16 rows: a 128-column slice of a bf16 row is
-// only 256 bytes, too small for one bulk copy per row to pay off.  Lanes load their 8 bytes
-// of each row directly, B = 8 rows per batch (three blocks per SM: more warps with smaller
-// batches measured faster), with the next batch in flight in registers
-// while the current one is added; the arithmetic is that of seg_rows_kernel.
+// A lane's 8 bytes (four bf16 columns) of a row, unpacked to fp32.
 template <bool BF16>
 struct RegRowVec;
 template <>
@@ -297,33 +301,63 @@ struct RegRowVec<true> {
     __device__ static uint2 zero() { return make_uint2(0u, 0u); }
 };
 
-template <bool BF16>
-__global__ void __launch_bounds__(kUpdWarps * 32, 3)
-    seg_rows_regs_kernel(const void *__restrict__ X, int64_t N, int d, int R, int64_t nwarps,
-                    int dcov, const int32_t *__restrict__ skeys,
-                    const int32_t *__restrict__ perm,
-                    const float *__restrict__ C_used, float *__restrict__ C_new,
-                    double *__restrict__ sums_out, double *__restrict__ pieces,
-                    int32_t *__restrict__ pkeys, double *__restrict__ jpart) {
+// Level 1 for bf16 rows.  A 128-column slice of a bf16 row is only 256 bytes: one bulk copy
+// per row is limited by the copy engine's request rate, and rows loaded into registers
+// (two batches in flight per warp) leave too few bytes in flight.  Here every lane copies
+// 16-byte pieces of the rows with cp.async into a ring of kCpStages stages of kCpRows rows
+// per warp, so kCpStages - 1 stages are in flight without holding registers (measured at
+// 100M rows, K = 32768: sort + update 8.14 -> 7.23 ms against the register form, the same
+// bits).  Each stage is added batch by batch with the arithmetic of seg_rows_kernel.
+constexpr int kCpWarps = 4;    // warps per block
+constexpr int kCpRows = 16;    // rows per stage (two batches of eight)
+constexpr int kCpStages = 3;   // stages per warp (4 and 6 measured slower: fewer blocks fit)
+constexpr int kCpRowBytes = 256;  // a 128-column bf16 slice
+constexpr size_t kCpSmem = size_t(kCpWarps) * kCpStages * kCpRows * kCpRowBytes;  // 48 KB
+
+__device__ __forceinline__ void cp_async16(void *dst, const void *src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(ptx::smem_u32(dst)),
+                 "l"(src)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+    asm volatile("cp.async.commit_group;" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+__global__ void __launch_bounds__(kCpWarps * 32, 4)
+    seg_rows_cp_kernel(const void *__restrict__ X, int64_t N, int d, int R, int64_t nwarps,
+                       int dcov, const int32_t *__restrict__ skeys,
+                       const int32_t *__restrict__ perm, const float *__restrict__ C_used,
+                       float *__restrict__ C_new, double *__restrict__ sums_out,
+                       double *__restrict__ pieces, int32_t *__restrict__ pkeys,
+                       double *__restrict__ jpart) {
     pdl_wait();
     pdl_trigger();
-    using RV = RegRowVec<BF16>;
+    using RV = RegRowVec<true>;
     using V = typename RV::T;
     constexpr int B = RV::kBatch;
-    __shared__ int32_t s_key[kUpdWarps][kUpdMaxRows];
-    __shared__ int32_t s_row[kUpdWarps][kUpdMaxRows];
+    static_assert(kCpRows % B == 0, "a stage is whole batches");
+    extern __shared__ __align__(128) uint8_t s_ring_all[];  // [warp][stage][row][256 B]
+    __shared__ int32_t s_key[kCpWarps][kUpdMaxRows];
+    __shared__ int32_t s_row[kCpWarps][kUpdMaxRows];
     const int lane = threadIdx.x & 31;
     const int wib = threadIdx.x >> 5;
-    const int64_t w = static_cast<int64_t>(blockIdx.x) * kUpdWarps + wib;
+    const int64_t w = static_cast<int64_t>(blockIdx.x) * kCpWarps + wib;
     if (w >= nwarps) return;
     const int cb = blockIdx.y;
     const int col = cb * 128 + lane * 4;
     const bool colv = col < d;
+    const int col0 = cb * 128;
+    const int pieces16 = ((d - col0 < 128 ? d - col0 : 128) * 2) / 16;  // 16-byte pieces
     const int64_t p0 = w * R;
     const int n = static_cast<int>((p0 + R < N ? p0 + R : N) - p0);
     const int64_t p1 = p0 + n;
     int32_t *sk = s_key[wib];
     int32_t *si = s_row[wib];
+    uint8_t *ring = s_ring_all + static_cast<size_t>(wib) * kCpStages * kCpRows * kCpRowBytes;
     for (int j = lane; j < n; j += 32) {
         sk[j] = skeys[p0 + j];
         si[j] = perm[p0 + j];
@@ -332,15 +366,29 @@ __global__ void __launch_bounds__(kUpdWarps * 32, 3)
     const int k_after = p1 < N ? skeys[p1] : -1;
     __syncwarp();
 
-    const V *Xv = static_cast<const V *>(X);
+    const uint8_t *Xb = static_cast<const uint8_t *>(X);
+    // copy the rows of stage g (sorted positions g * kCpRows ..) into its ring slot: lane
+    // l takes pieces l, l + 32, ... of the stage's kCpRows x 16 pieces
+    auto issue = [&](int g) {
+        const int r0 = g * kCpRows;
+        if (r0 < n) {
+            uint8_t *dst = ring + (g % kCpStages) * (kCpRows * kCpRowBytes);
+#pragma unroll
+            for (int t = 0; t < (kCpRows * 16) / 32; ++t) {
+                const int c = lane + 32 * t;
+                const int r = c >> 4, pc = c & 15;
+                if (r0 + r < n && pc < pieces16)
+                    cp_async16(dst + r * kCpRowBytes + pc * 16,
+                               Xb + (static_cast<int64_t>(si[r0 + r]) * d + col0) * 2 + pc * 16);
+            }
+        }
+        cp_async_commit();  // an empty group past the end keeps the count uniform
+    };
+
     double acc[4] = {0.0, 0.0, 0.0, 0.0};
     float cu[4] = {0.f, 0.f, 0.f, 0.f};
     double jacc = 0.0;
     int cur = -1, first = -1, slot1 = -1, ncur = 0;
-
-    // A cluster is finished inside this warp unless it continues from the position before
-    // p0 or into the one at p1 (positions are sorted, so only the first and the last
-    // cluster can); its count is then the rows added here.
     auto finished = [&](int k) { return k != k_before && k != k_after; };
     auto flush = [&](int k) {
         if (finished(k)) {
@@ -365,17 +413,16 @@ __global__ void __launch_bounds__(kUpdWarps * 32, 3)
             cu[3] = c.w;
         }
     };
-    auto issue = [&](int b, V (&buf)[B]) {
-#pragma unroll
-        for (int j = 0; j < B; ++j) {
-            const int q = b + j;
-            buf[j] = (q < n && colv)
-                         ? __ldg(Xv + (static_cast<int64_t>(si[q]) * d + col) / 4)
-                         : RV::zero();
-        }
-    };
-    auto process = [&](int b, const V (&buf)[B]) {
+    // one batch of B rows starting at sorted position b, read from the ring: the same sums
+    // in the same order as the register form
+    auto process = [&](int b, const uint8_t *rows) {
         const int nb = n - b < B ? n - b : B;
+        V buf[B];
+#pragma unroll
+        for (int j = 0; j < B; ++j)
+            buf[j] = (j < nb && colv)
+                         ? *reinterpret_cast<const V *>(rows + j * kCpRowBytes + lane * 8)
+                         : RV::zero();
         const int kf = sk[b], kl = sk[b + nb - 1];
         if (kf == kl) {
             if (kf != cur) start(kf);
@@ -427,18 +474,24 @@ __global__ void __launch_bounds__(kUpdWarps * 32, 3)
         }
     };
 
-    V bufA[B], bufB[B];
-    issue(0, bufA);
-    for (int b = 0; b < n; b += 2 * B) {
-        issue(b + B, bufB);
-        process(b, bufA);
-        if (b + B >= n) break;
-        issue(b + 2 * B, bufA);
-        process(b + B, bufB);
+    const int nstages = (n + kCpRows - 1) / kCpRows;
+#pragma unroll
+    for (int g = 0; g < kCpStages - 1; ++g) issue(g);
+    for (int g = 0; g < nstages; ++g) {
+        issue(g + kCpStages - 1);     // into the slot processed one step ago
+        cp_async_wait<kCpStages - 1>();  // this lane's copies of stage g have landed
+        __syncwarp();                    // and every other lane's
+        const uint8_t *st = ring + (g % kCpStages) * (kCpRows * kCpRowBytes);
+#pragma unroll
+        for (int h = 0; h < kCpRows / B; ++h) {
+            const int b = g * kCpRows + h * B;
+            if (b < n) process(b, st + h * B * kCpRowBytes);
+        }
+        __syncwarp();  // the slot is read by every lane before it is refilled
     }
+    cp_async_wait<0>();
     if (cur >= 0) flush(cur);
     if (cb == 0 && lane == 0) {
-        // slot 0 holds the first cluster if it was not finished here; slot 1 the last
         pkeys[w * 2 + 0] = finished(first) ? -1 : first;
         pkeys[w * 2 + 1] = slot1;
     }
@@ -673,18 +726,24 @@ cudaError_t run_levels(const void *X, bool bf16, int64_t N, int d, const UpdPlan
     static std::atomic<uint64_t> smem_set{0};
     {
         const cudaError_t e =
-            smem_opt_in(seg_rows_kernel<false>, static_cast<int>(kRowSmem), smem_set);
+            smem_opt_in(seg_rows_kernel<false>, static_cast<int>(kRowSmem<false>), smem_set);
         if (e != cudaSuccess) return e;
     }
     const dim3 rblock(kRowWarps * 32);
     dim3 rgrid(static_cast<unsigned>(ceil_div(up.nwarps, kRowWarps)), up.ncolblk);
+    static std::atomic<uint64_t> smem_set_cp{0};
+    {
+        const cudaError_t e =
+            smem_opt_in(seg_rows_cp_kernel, static_cast<int>(kCpSmem), smem_set_cp);
+        if (e != cudaSuccess) return e;
+    }
     if (bf16)
-        launch_pdl(seg_rows_regs_kernel<true>,
-                   dim3(static_cast<unsigned>(ceil_div(up.nwarps, kUpdWarps)), up.ncolblk),
-                   dim3(kUpdWarps * 32), 0, st, X, N, d, up.rows, up.nwarps, up.dcov, skeys, perm,
-                   C_used, C_new, sums_out, pa, ka, jpart);
+        launch_pdl(seg_rows_cp_kernel,
+                   dim3(static_cast<unsigned>(ceil_div(up.nwarps, kCpWarps)), up.ncolblk),
+                   dim3(kCpWarps * 32), kCpSmem, st, X, N, d, up.rows, up.nwarps, up.dcov, skeys,
+                   perm, C_used, C_new, sums_out, pa, ka, jpart);
     else
-        launch_pdl(seg_rows_kernel<false>, rgrid, rblock, kRowSmem, st, X, N, d, up.rows,
+        launch_pdl(seg_rows_kernel<false>, rgrid, rblock, kRowSmem<false>, st, X, N, d, up.rows,
                    up.nwarps, up.dcov, skeys, perm, C_used, C_new, sums_out, pa, ka, jpart,
                    err);
     note_launch();
