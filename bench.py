@@ -38,6 +38,7 @@ UNIT = "points*iter/s"
 # The pages' own figure for the default workload: a 1M x 768, nlist 4096 k-means build
 # (default niter 20) in 10.6 s on an H200 (another machine; context only).
 PAGES_BUILD_RATE = 1_000_000 * 20 / 10.6
+L2_FLUSH_BYTES = 256 << 20  # twice the B200's 126 MB L2
 
 
 def parse():
@@ -45,8 +46,9 @@ def parse():
     p.add_argument("--gpus", type=int, default=1)
     p.add_argument("--steps", type=int, default=5)
     p.add_argument("--warmup", type=int, default=3)
-    p.add_argument("--workload", default="large_100000000x128_k32768_bf16",
-                   help="one of synth.CONFIGS")
+    p.add_argument("--workload", default=None,
+                   help="one of synth.CONFIGS (default: large_100000000x128_k32768_bf16; "
+                        "with --search, ivf_1000000x768_k4096_f32_cosine, the index workload)")
     p.add_argument("--niter", type=int, default=None)
     p.add_argument("--n", type=int, default=None,
                    help="override N (smaller cases for profiling captures)")
@@ -273,11 +275,13 @@ def fk_arm(args, spec, rank, world, dist):
         ws = fk.workspace(spec.n, spec.d, spec.k, X.dtype, spec.metric, device=dev)
     torch.cuda.synchronize()
 
-    def run(Xin, acc):
-        """One complete k-means run from raw points and C (in place)."""
+    def run(Xin, acc, mode=True):
+        """One complete k-means run from raw points and C (in place).  With acc, fk_lloyd's
+        timing is added into it: mode True times every phase, "kernel" only the
+        assignment's tensor-core kernel (two events per iteration)."""
         if not sharded:
             objs, tm = fk.fk_lloyd(Xin, C, niter, labels, ws, metric=spec.metric,
-                                   counts=counts, timing=acc is not None)
+                                   counts=counts, timing=mode if acc is not None else False)
             if acc is not None:
                 for k in ("ms_setup", "ms_prep", "ms_assign", "ms_sort", "ms_update",
                           "ms_assign_mma", "screened"):
@@ -291,9 +295,16 @@ def fk_arm(args, spec, rank, world, dist):
         objs, _ = lloyd_sharded(Xp, C, niter, ops, timing=acc)
         return objs
 
-    def step(acc):
+    def step(acc, mode=True):
         C.copy_(C0)
-        return run(X, acc)
+        return run(X, acc, mode)
+
+    # points smaller than L2 are flushed from it between timed steps (a buffer twice the
+    # L2 written outside the steps' events); larger ones cannot stay in it
+    e_bytes = 4 if spec.dtype == "f32" else 2
+    x_bytes = spec.n * spec.d * e_bytes
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.int32, device=dev) \
+        if x_bytes < L2_FLUSH_BYTES else None
 
     for _ in range(args.warmup):
         step(None)
@@ -311,18 +322,42 @@ def fk_arm(args, spec, rank, world, dist):
         dist.barrier()
     torch.cuda.synchronize()
     launches0 = fk.launch_count()
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for _ in range(args.steps):
-        objs = step(acc)
-    e1.record()
-    torch.cuda.synchronize()
+    # the timed steps time only the assignment kernel (the roofline's launches); the
+    # per-phase breakdown comes from extra steps after the timed region
+    mode = True if sharded else "kernel"
+    if flush is None:
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(args.steps):
+            objs = step(acc, mode)
+        e1.record()
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1)
+    else:
+        marks = []
+        for _ in range(args.steps):
+            flush.fill_(1)
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record()
+            objs = step(acc, mode)
+            b.record()
+            marks.append((a, b))
+        torch.cuda.synchronize()
+        ms = sum(a.elapsed_time(b) for a, b in marks)
     launches = fk.launch_count() - launches0
     if dist:
         dist.barrier()
     clocks = sampler.stop()
-    ms = e0.elapsed_time(e1)
+    pacc, psteps = acc, args.steps
+    if not sharded:  # the phase breakdown, from steps outside the timed region
+        pacc, psteps = {}, max(1, min(args.steps, 3))
+        for _ in range(psteps):
+            if flush is not None:
+                flush.fill_(1)
+            step(pacc)
+        torch.cuda.synchronize()
     if dist:
         t = torch.tensor([ms], device=dev, dtype=torch.float64)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
@@ -337,7 +372,8 @@ def fk_arm(args, spec, rank, world, dist):
     peaks = load_peaks()
     n_assign = niter * args.steps
     flops = 2.0 * spec.n * spec.k * spec.d
-    phase_ms = acc["ms_assign"] / n_assign
+    # the whole assignment phase (every kernel of it), from the phase-timed steps
+    phase_ms = acc["ms_assign"] / n_assign if sharded else pacc["ms_assign"] / (niter * psteps)
     if sharded:
         mma_ms, screened = phase_ms, None
         scr = spec.dtype == "f32" and spec.d >= 256 and spec.n >= 18944
@@ -380,10 +416,12 @@ def fk_arm(args, spec, rank, world, dist):
         phases = {k: acc[k] / args.steps for k in ("ms_assign", "ms_partial", "ms_exchange",
                                                     "ms_finalize")}
     else:
-        upd_ms = (acc["ms_sort"] + acc["ms_update"]) / n_assign
-        phases = {k: acc[k] / args.steps for k in ("ms_setup", "ms_prep", "ms_assign",
-                                                    "ms_sort", "ms_update")}
-    e_bytes = 4 if spec.dtype == "f32" else 2
+        upd_ms = (pacc["ms_sort"] + pacc["ms_update"]) / (niter * psteps)
+        phases = {k: pacc[k] / psteps for k in ("ms_setup", "ms_prep", "ms_assign",
+                                                 "ms_sort", "ms_update")}
+        phases["steps"] = psteps
+        phases["note"] = ("every phase timed with CUDA events in extra steps after the "
+                          "timed region")
     upd_bytes = spec.n * spec.d * e_bytes + 24.0 * spec.n
 
     out = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
@@ -398,8 +436,11 @@ def fk_arm(args, spec, rank, world, dist):
                       "metric": spec.metric, "niter_per_step": niter,
                       "parallelism": f"dp{world}" if sharded else "single GPU",
                       "points_per_rank": spec.n,
-                      "l2": f"inputs larger than L2 (X = {spec.n * spec.d * e_bytes / 1e9:.2f}"
-                            " GB per rank)"},
+                      "l2": (f"inputs larger than L2 (X = {x_bytes / 1e9:.2f} GB per rank)"
+                             if flush is None else
+                             f"X ({x_bytes / 1e9:.3f} GB) smaller than L2: a "
+                             f"{L2_FLUSH_BYTES >> 20} MB buffer written between timed steps,"
+                             " outside their CUDA events")},
            "roofline": roof,
            "update_hbm": {"achieved_gbs": upd_bytes / (upd_ms / 1e3) / 1e9,
                           "peak_gbs": peaks["hbm_gbs"],
@@ -836,6 +877,9 @@ def main():
     from dataclasses import replace
 
     from synth import CONFIGS
+    if args.workload is None:
+        args.workload = ("ivf_1000000x768_k4096_f32_cosine" if args.search
+                         else "large_100000000x128_k32768_bf16")
     spec = CONFIGS[args.workload]
     if args.n:
         spec = replace(spec, n=args.n, name=spec.name.replace(str(spec.n), str(args.n)))

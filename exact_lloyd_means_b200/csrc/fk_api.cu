@@ -54,6 +54,86 @@ fk_status check_device() {
 
 bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
+namespace {
+// The unique id of the calling thread's current CUDA context (0 if there is none or the
+// driver cannot tell).  The per-thread caches below (streams, events, pinned staging,
+// instantiated graphs) belong to the context they were made in: each is tagged with this
+// id and is dropped, not used, once the id changes (a device reset, a new primary
+// context).  Dropped handles are not destroyed: their context is gone with them.
+uint64_t context_id() {
+    using GetCurrent = int (*)(void **);
+    using GetId = int (*)(void *, unsigned long long *);
+    static GetCurrent get_current = nullptr;
+    static GetId get_id = nullptr;
+    static const bool found = [] {
+        void *p = nullptr, *q = nullptr;
+        cudaDriverEntryPointQueryResult r1, r2;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &r1) !=
+                cudaSuccess ||
+            r1 != cudaDriverEntryPointSuccess ||
+            cudaGetDriverEntryPoint("cuCtxGetId", &q, cudaEnableDefault, &r2) != cudaSuccess ||
+            r2 != cudaDriverEntryPointSuccess)
+            return false;
+        get_current = reinterpret_cast<GetCurrent>(p);
+        get_id = reinterpret_cast<GetId>(q);
+        return true;
+    }();
+    void *ctx = nullptr;
+    unsigned long long id = 0;
+    if (!found || get_current(&ctx) != 0 || ctx == nullptr || get_id(ctx, &id) != 0) return 0;
+    return id;
+}
+
+struct SideStream {
+    uint64_t ctx = 0;
+    cudaStream_t s = nullptr;
+    cudaEvent_t fork = nullptr;  // ordering only (no timing)
+    bool used = false;           // forked since the last join
+};
+
+SideStream *side_stream() {
+    thread_local SideStream side[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    const uint64_t ctx = context_id();
+    if (ctx == 0) return nullptr;
+    SideStream &ss = side[dev];
+    if (ss.ctx != ctx) ss = SideStream{};
+    if (!ss.s) {
+        if (cudaStreamCreateWithFlags(&ss.s, cudaStreamNonBlocking) != cudaSuccess ||
+            cudaEventCreateWithFlags(&ss.fork, cudaEventDisableTiming) != cudaSuccess) {
+            ss = SideStream{};
+            return nullptr;
+        }
+        ss.ctx = ctx;
+    }
+    return &ss;
+}
+}  // namespace
+
+cudaError_t record_event(cudaEvent_t e, cudaStream_t st) {
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    cudaError_t r = cudaStreamIsCapturing(st, &cs);
+    if (r != cudaSuccess) return r;
+    if (cs != cudaStreamCaptureStatusActive) return cudaEventRecord(e, st);
+    SideStream *ss = side_stream();
+    if (!ss) return cudaErrorUnknown;
+    if ((r = cudaEventRecord(ss->fork, st)) != cudaSuccess ||
+        (r = cudaStreamWaitEvent(ss->s, ss->fork, 0)) != cudaSuccess)
+        return r;
+    ss->used = true;
+    return cudaEventRecordWithFlags(e, ss->s, cudaEventRecordExternal);
+}
+
+cudaError_t join_side_stream(cudaStream_t st) {
+    SideStream *ss = side_stream();
+    if (!ss) return cudaErrorUnknown;
+    if (!ss->used) return cudaSuccess;
+    ss->used = false;
+    cudaError_t r = cudaEventRecord(ss->fork, ss->s);
+    return r != cudaSuccess ? r : cudaStreamWaitEvent(st, ss->fork, 0);
+}
+
 fk_status validate_shape(int64_t N, int d, int K, fk_dtype dtype, fk_metric metric,
                          bool planes_ok) {
     if (N < 1 || N > 2147483647LL - 1) return FK_ERR_INVALID_ARG;
@@ -198,9 +278,9 @@ fk_status run_assign(const void *planes, int nplanes, int64_t lda, int64_t N, in
     }
     if (exact_only) return FK_ERR_UNSUPPORTED;  // the pair kernel cannot run on this device
     if (probe_rows > 0) return FK_OK;
-    if (ev_mma0) FK_TRY_CUDA(cudaEventRecord(ev_mma0, st));
+    if (ev_mma0) FK_TRY_CUDA(record_event(ev_mma0, st));
     FK_TRY_CUDA(launch_assign(a, st));
-    if (ev_mma1) FK_TRY_CUDA(cudaEventRecord(ev_mma1, st));
+    if (ev_mma1) FK_TRY_CUDA(record_event(ev_mma1, st));
     return FK_OK;
 }
 
@@ -403,6 +483,128 @@ fk_status run_ivf_search(const float *Q, int64_t nq, int d, const float *C, int 
     if (!mark(4)) return FK_ERR_CUDA;
     return FK_OK;
 }
+
+// Timing events, created once per thread and device and reused by every call: each call
+// ends with a synchronisation, so no event is still pending when the next call records it.
+bool pooled_events(size_t n, std::vector<cudaEvent_t> **out) {
+    thread_local std::vector<cudaEvent_t> pools[64];
+    thread_local uint64_t pool_ctx[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
+    const uint64_t ctx = context_id();
+    if (ctx == 0) return false;
+    std::vector<cudaEvent_t> &p = pools[dev];
+    if (pool_ctx[dev] != ctx) {  // events of another context: drop them
+        p.clear();
+        pool_ctx[dev] = ctx;
+    }
+    while (p.size() < n) {
+        cudaEvent_t e;
+        if (cudaEventCreate(&e) != cudaSuccess) return false;
+        p.push_back(e);
+    }
+    *out = &p;
+    return true;
+}
+
+// fk_lloyd's iteration loop as a CUDA graph.  The loop's launches are fixed by the call's
+// arguments and by the screening probe's decision, so a call that repeats the previous call
+// on the same thread (same pointers, sizes, metric, iteration count, timing flag, device and
+// probe decision) captures its loop once and replays it as one graph launch, and later
+// identical calls replay it again.  The graph reads device memory when it runs, so new
+// point or centroid values need no new capture.  FK_LOOP_GRAPH=0 in the environment turns
+// the cache off.
+struct LoopKey {
+    const void *X;
+    float *C;
+    int32_t *labels, *counts, *offsets;
+    void *ws;
+    size_t ws_bytes;
+    int64_t N;
+    int d, K, niter, device;
+    uint64_t ctx;  // the CUDA context the graph belongs to
+    fk_dtype dtype;
+    fk_metric metric;
+    int timing;  // 0 none, 1 kernel only, 2 every phase
+    bool allow_screen;
+    bool operator==(const LoopKey &o) const {
+        return X == o.X && C == o.C && labels == o.labels && counts == o.counts &&
+               offsets == o.offsets && ws == o.ws && ws_bytes == o.ws_bytes && N == o.N &&
+               d == o.d && K == o.K && niter == o.niter && device == o.device && ctx == o.ctx &&
+               dtype == o.dtype && metric == o.metric && timing == o.timing &&
+               allow_screen == o.allow_screen;
+    }
+};
+
+struct LoopGraph {
+    LoopKey key{};
+    cudaGraphExec_t exec = nullptr;
+    std::vector<cudaEvent_t> ev;  // timing: 4 per iteration, then 2 per iteration
+    int nscreened = 0;
+    bool last_screened = false;
+    long launches = 0;  // kernels in the graph
+    uint64_t used = 0;  // exec == nullptr: the capture failed; the call runs eagerly
+};
+
+constexpr size_t kLoopGraphs = 4;
+
+struct LoopGraphCache {
+    bool have_last = false;
+    LoopKey last{};
+    std::vector<LoopGraph> graphs;
+    uint64_t clock = 0;
+    cudaStream_t capture[64] = {};  // one capture stream per device
+    uint64_t capture_ctx[64] = {};   // its context
+};
+
+LoopGraphCache &loop_graphs() {
+    thread_local LoopGraphCache c;
+    return c;
+}
+
+bool loop_graphs_enabled() {
+    static const bool on = [] {
+        const char *e = std::getenv("FK_LOOP_GRAPH");
+        return !(e && std::strcmp(e, "0") == 0);
+    }();
+    return on;
+}
+
+// Pinned host staging for the end of an fk_lloyd call, one per thread and device: the
+// objectives of the iterations since the last ring copy and words 0..6 of the error block
+// (error flags, then the last iteration's statistics), read back by one copy each and one
+// synchronisation.  Pinned, so that the copies can sit in a captured graph.
+struct CallStage {
+    double obj[kObjRing];
+    uint32_t words[8];
+};
+
+CallStage *call_stage() {
+    thread_local CallStage *stages[64] = {};
+    thread_local uint64_t stage_ctx[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    const uint64_t ctx = context_id();
+    if (ctx == 0) return nullptr;
+    if (stage_ctx[dev] != ctx) {  // pinned memory of another context is gone with it
+        stages[dev] = nullptr;
+        stage_ctx[dev] = ctx;
+    }
+    if (!stages[dev]) {
+        void *p = nullptr;
+        if (cudaHostAlloc(&p, sizeof(CallStage), cudaHostAllocDefault) != cudaSuccess)
+            return nullptr;
+        stages[dev] = static_cast<CallStage *>(p);
+    }
+    return stages[dev];
+}
+
+void release(LoopGraph &g) {
+    if (g.exec) cudaGraphExecDestroy(g.exec);
+    for (cudaEvent_t e : g.ev) cudaEventDestroy(e);
+    g.exec = nullptr;
+    g.ev.clear();
+}
 }  // namespace
 }  // namespace fk
 
@@ -574,44 +776,26 @@ fk_status fk_lloyd(const void *X, fk_dtype dtype, int64_t N, int d, int K, fk_me
     if (injected_fault() == kFaultLaunch) return FK_ERR_CUDA;
     cudaStream_t st = stream;
 
-    // events: [0] start, [1] after setup, then 4 per iteration
-    std::vector<cudaEvent_t> ev;
-    auto rec = [&]() -> bool {
-        if (!timing) return true;
-        cudaEvent_t e;
-        if (cudaEventCreate(&e) != cudaSuccess) return false;
-        ev.push_back(e);
-        return cudaEventRecord(e, st) == cudaSuccess;
-    };
-    // events around the main tensor-core kernel of each iteration's assignment
-    std::vector<cudaEvent_t> evm;
-    auto mk = [&](cudaEvent_t *e) -> bool {
-        *e = nullptr;
-        if (!timing) return true;
-        if (cudaEventCreate(e) != cudaSuccess) return false;
-        evm.push_back(*e);
-        return true;
-    };
-    auto cleanup = [&]() {
-        for (auto e : ev) cudaEventDestroy(e);
-        for (auto e : evm) cudaEventDestroy(e);
-    };
-    auto fail = [&](fk_status f) {
-        cleanup();
-        return f;
-    };
+    // Timing events: [0] call start, [1] end of the setup, then (pool or graph) 4 per
+    // iteration (after prep, assign, sort, update) and 2 per iteration around the
+    // assignment's tensor-core kernel; with kernel_only, only the last two.
+    const bool kernel_only = timing && timing->kernel_only != 0;
+    const bool phases = timing && !kernel_only;
+    std::vector<cudaEvent_t> *pool = nullptr;
+    if (timing && !pooled_events(2 + 6 * static_cast<size_t>(niter), &pool))
+        return FK_ERR_CUDA;
 
     NvtxRange call_range("fk_lloyd");
     if (cudaMemsetAsync(ws_ptr<uint32_t>(ws, L.err), 0, 2 * sizeof(uint32_t), st) != cudaSuccess)
         return FK_ERR_CUDA;
     const long launches0 = g_launches;
-    if (!rec()) return fail(FK_ERR_CUDA);
+    if (phases && cudaEventRecord((*pool)[0], st) != cudaSuccess) return FK_ERR_CUDA;
     const void *Xp = X;
     if (metric == FK_COSINE) {
         float *xn = ws_ptr<float>(ws, L.xn);
         if (launch_normalize(static_cast<const float *>(X), xn, N, d, st) != cudaSuccess ||
             launch_normalize(C, C, K, d, st) != cudaSuccess)
-            return fail(FK_ERR_CUDA);
+            return FK_ERR_CUDA;
         Xp = xn;
     }
     const void *planes = nullptr;
@@ -621,143 +805,266 @@ fk_status fk_lloyd(const void *X, fk_dtype dtype, int64_t N, int d, int K, fk_me
     float *xnorm = dtype == FK_F32 ? ws_ptr<float>(ws, L.xnorm) : nullptr;
     if (niter > 0 &&
         (s = prepare_x(Xp, dtype, N, d, L, ws, xnorm, st, &planes, &nplanes, &lda)) != FK_OK)
-        return fail(s);
+        return s;
 
-    float *Ccur = C, *Cnext = ws_ptr<float>(ws, L.calt);
+    float *C_alt = ws_ptr<float>(ws, L.calt);
     int32_t *cnt = counts ? counts : ws_ptr<int32_t>(ws, L.cnt);
     int32_t *off = offsets ? offsets : ws_ptr<int32_t>(ws, L.off);
     double *obj = ws_ptr<double>(ws, L.obj);
     float *cused = ws_ptr<float>(ws, L.cused);
-    int copied = 0;
     bool allow_screen = true;
-    int nscreened = 0;
-    bool last_screened = false;
     if (niter > 0 && dtype == FK_F32) {
         // Where the screened route applies, try it first on a sample of the rows with the
         // initial centroids and read how many would need the three-product pass (a single
         // host synchronisation per call); screen the call only if few would.
         bool probed = false;
-        if (launch_prep_centroids(Ccur, K, d, L.Kp, L.dp, dtype, ws_ptr<uint16_t>(ws, L.cs),
+        if (launch_prep_centroids(C, K, d, L.Kp, L.dp, dtype, ws_ptr<uint16_t>(ws, L.cs),
                                   ws_ptr<float>(ws, L.cn), cused, ws_ptr<uint16_t>(ws, L.caug),
                                   st) != cudaSuccess)
-            return fail(FK_ERR_CUDA);
+            return FK_ERR_CUDA;
         if ((s = run_assign(planes, nplanes, lda, N, d, K, L, ws, labels, xnorm, nullptr, st,
-                            static_cast<const float *>(Xp), Ccur, true, &probed, nullptr,
+                            static_cast<const float *>(Xp), C, true, &probed, nullptr,
                             nullptr, kScreenProbeRows)) != FK_OK)
-            return fail(s);
+            return s;
         if (probed) {
             uint32_t nfb = 0;
             if (cudaMemcpyAsync(&nfb, ws_ptr<uint32_t>(ws, L.nfb), sizeof(nfb),
                                 cudaMemcpyDeviceToHost, st) != cudaSuccess ||
                 cudaStreamSynchronize(st) != cudaSuccess)
-                return fail(FK_ERR_CUDA);
+                return FK_ERR_CUDA;
             const int64_t n = N < kScreenProbeRows ? N : kScreenProbeRows;
             allow_screen = static_cast<int64_t>(nfb) * kScreenMaxFallback <= n;
         }
     }
-    if (!rec()) return fail(FK_ERR_CUDA);  // end of the once-per-call setup
-    for (int t = 0; t < niter; ++t) {
-        NvtxRange iter_range("fk_lloyd iteration");
-        if (launch_prep_centroids(Ccur, K, d, L.Kp, L.dp, dtype, ws_ptr<uint16_t>(ws, L.cs),
-                                  ws_ptr<float>(ws, L.cn), cused, ws_ptr<uint16_t>(ws, L.caug),
-                                  st) != cudaSuccess)
-            return fail(FK_ERR_CUDA);
-        if (!rec()) return fail(FK_ERR_CUDA);
-        bool screened = false;
-        cudaEvent_t m0 = nullptr, m1 = nullptr;
-        if (!mk(&m0) || !mk(&m1)) return fail(FK_ERR_CUDA);
-        if ((s = run_assign(planes, nplanes, lda, N, d, K, L, ws, labels, xnorm, nullptr, st,
-                            dtype == FK_F32 ? static_cast<const float *>(Xp) : nullptr, Ccur,
-                            allow_screen, &screened, m0, m1)) != FK_OK)
-            return fail(s);
-        nscreened += screened ? 1 : 0;
-        last_screened = screened;
-        if (!rec()) return fail(FK_ERR_CUDA);
-        nvtxRangePushA("sort + update");
-        const int32_t *skeys = nullptr, *perm = nullptr;
-        if (launch_sort_csr(labels, N, K, L.sp, ws_ptr<int32_t>(ws, L.keys0),
-                            ws_ptr<int32_t>(ws, L.keys1), ws_ptr<int32_t>(ws, L.vals0),
-                            ws_ptr<int32_t>(ws, L.vals1), nullptr,
-                            ws_ptr<uint32_t>(ws, L.hist), ws_ptr<uint32_t>(ws, L.dtot), off,
-                            &skeys, &perm, ws_ptr<uint32_t>(ws, L.err), st) != cudaSuccess) {
-            nvtxRangePop();
-            return fail(FK_ERR_CUDA);
+    if (phases && cudaEventRecord((*pool)[1], st) != cudaSuccess) return FK_ERR_CUDA;
+
+    // The iteration loop, issued on stream s.  lev holds 4 events per iteration and mev 2,
+    // both null without timing.  With sync_objective the objective ring is copied to the
+    // host whenever it fills (never inside a graph, which is only used below the ring size).
+    int copied = 0;
+    auto issue_loop = [&](cudaStream_t s_, const cudaEvent_t *lev, const cudaEvent_t *mev,
+                          bool sync_objective, int *nscreened_out,
+                          bool *last_screened_out) -> fk_status {
+        float *Ccur = C, *Cnext = C_alt;
+        auto rec = [&](int i) { return !lev || record_event(lev[i], s_) == cudaSuccess; };
+        int nscr = 0;
+        bool last = false;
+        for (int t = 0; t < niter; ++t) {
+            NvtxRange iter_range("fk_lloyd iteration");
+            if (launch_prep_centroids(Ccur, K, d, L.Kp, L.dp, dtype, ws_ptr<uint16_t>(ws, L.cs),
+                                      ws_ptr<float>(ws, L.cn), cused,
+                                      ws_ptr<uint16_t>(ws, L.caug), s_) != cudaSuccess ||
+                !rec(4 * t))
+                return FK_ERR_CUDA;
+            bool screened = false;
+            fk_status r = run_assign(planes, nplanes, lda, N, d, K, L, ws, labels, xnorm, nullptr,
+                                     s_, dtype == FK_F32 ? static_cast<const float *>(Xp) : nullptr,
+                                     Ccur, allow_screen, &screened, mev ? mev[2 * t] : nullptr,
+                                     mev ? mev[2 * t + 1] : nullptr);
+            if (r != FK_OK) return r;
+            nscr += screened ? 1 : 0;
+            last = screened;
+            if (!rec(4 * t + 1)) return FK_ERR_CUDA;
+            NvtxRange upd_range("sort + update");
+            const int32_t *skeys = nullptr, *perm = nullptr;
+            if (launch_sort_csr(labels, N, K, L.sp, ws_ptr<int32_t>(ws, L.keys0),
+                                ws_ptr<int32_t>(ws, L.keys1), ws_ptr<int32_t>(ws, L.vals0),
+                                ws_ptr<int32_t>(ws, L.vals1), nullptr,
+                                ws_ptr<uint32_t>(ws, L.hist), ws_ptr<uint32_t>(ws, L.dtot), off,
+                                &skeys, &perm, ws_ptr<uint32_t>(ws, L.err), s_) != cudaSuccess ||
+                !rec(4 * t + 2))
+                return FK_ERR_CUDA;
+            if (launch_update(Xp, dtype, N, d, K, L.up, skeys, perm, off, Ccur,
+                              dtype == FK_F32 ? Ccur : cused, Cnext, cnt,
+                              ws_ptr<double>(ws, L.pieces), ws_ptr<int32_t>(ws, L.pkeys),
+                              ws_ptr<double>(ws, L.piecesb), ws_ptr<int32_t>(ws, L.pkeysb),
+                              ws_ptr<double>(ws, L.jpart), obj + (t % kObjRing),
+                              ws_ptr<uint32_t>(ws, L.err), nullptr, s_) != cudaSuccess ||
+                !rec(4 * t + 3))
+                return FK_ERR_CUDA;
+            float *tmp = Ccur;
+            Ccur = Cnext;
+            Cnext = tmp;
+            if (sync_objective && (t + 1) % kObjRing == 0) {
+                // the ring is full: hand it to the caller before it wraps
+                if (objective_host &&
+                    (cudaMemcpyAsync(objective_host + copied, obj, sizeof(double) * kObjRing,
+                                     cudaMemcpyDeviceToHost, s_) != cudaSuccess ||
+                     cudaStreamSynchronize(s_) != cudaSuccess))
+                    return FK_ERR_CUDA;
+                copied += kObjRing;
+            }
         }
-        if (!rec()) {
-            nvtxRangePop();
-            return fail(FK_ERR_CUDA);
+        *nscreened_out = nscr;
+        *last_screened_out = last;
+        return FK_OK;
+    };
+
+    // The end of the call on stream s: the final centroids back into C, the last
+    // iteration's statistics (timing of every phase), then the error words, the
+    // statistics and the objectives not yet copied into the pinned stage, and the error
+    // flags cleared for the next call.
+    CallStage *stage = call_stage();
+    if (!stage) return FK_ERR_CUDA;
+    auto issue_tail = [&](cudaStream_t s_, bool last_scr) -> fk_status {
+        float *Cfinal = niter % 2 ? C_alt : C;
+        uint32_t *errw = ws_ptr<uint32_t>(ws, L.err);
+        if (Cfinal != C &&
+            cudaMemcpyAsync(C, Cfinal, sizeof(float) * static_cast<size_t>(K) * d,
+                            cudaMemcpyDeviceToDevice, s_) != cudaSuccess)
+            return FK_ERR_CUDA;
+        if (phases && niter > 0) {
+            // words 4, 5 of the error block: the empty-cluster count and the largest cluster
+            if (launch_cluster_stats(cnt, K, errw + 4, s_) != cudaSuccess) return FK_ERR_CUDA;
+            if (last_scr && cudaMemcpyAsync(&stage->words[6], ws_ptr<uint32_t>(ws, L.nfb),
+                                            sizeof(uint32_t), cudaMemcpyDeviceToHost,
+                                            s_) != cudaSuccess)
+                return FK_ERR_CUDA;
         }
-        if (launch_update(Xp, dtype, N, d, K, L.up, skeys, perm, off, Ccur,
-                          dtype == FK_F32 ? Ccur : cused, Cnext, cnt,
-                          ws_ptr<double>(ws, L.pieces), ws_ptr<int32_t>(ws, L.pkeys),
-                          ws_ptr<double>(ws, L.piecesb), ws_ptr<int32_t>(ws, L.pkeysb),
-                          ws_ptr<double>(ws, L.jpart), obj + (t % kObjRing),
-                          ws_ptr<uint32_t>(ws, L.err), nullptr, st) != cudaSuccess) {
-            nvtxRangePop();
-            return fail(FK_ERR_CUDA);
+        if (cudaMemcpyAsync(stage->words, errw, 6 * sizeof(uint32_t), cudaMemcpyDeviceToHost,
+                            s_) != cudaSuccess ||
+            (niter > copied &&
+             cudaMemcpyAsync(stage->obj, obj, sizeof(double) * (niter - copied),
+                             cudaMemcpyDeviceToHost, s_) != cudaSuccess) ||
+            cudaMemsetAsync(errw, 0, 2 * sizeof(uint32_t), s_) != cudaSuccess)
+            return FK_ERR_CUDA;
+        return FK_OK;
+    };
+
+    int nscreened = 0;
+    bool last_screened = false;
+    const cudaEvent_t *lev = phases ? pool->data() + 2 : nullptr;
+    const cudaEvent_t *mev = timing ? pool->data() + 2 + 4 * static_cast<size_t>(niter) : nullptr;
+    bool replayed = false;
+    int dev = 0;
+    const uint64_t ctx = context_id();
+    if (niter > 0 && niter < kObjRing && loop_graphs_enabled() && ctx != 0 &&
+        cudaGetDevice(&dev) == cudaSuccess && dev >= 0 && dev < 64) {
+        LoopGraphCache &cache = loop_graphs();
+        // graphs and capture streams of another context are dropped unreleased
+        for (size_t i = cache.graphs.size(); i-- > 0;)
+            if (cache.graphs[i].key.ctx != ctx)
+                cache.graphs.erase(cache.graphs.begin() + static_cast<long>(i));
+        if (cache.capture_ctx[dev] != ctx) {
+            cache.capture[dev] = nullptr;
+            cache.capture_ctx[dev] = ctx;
         }
-        nvtxRangePop();
-        if (!rec()) return fail(FK_ERR_CUDA);
-        float *tmp = Ccur;
-        Ccur = Cnext;
-        Cnext = tmp;
-        if (objective_host && (t + 1) % kObjRing == 0) {
-            if (cudaMemcpyAsync(objective_host + copied, obj, sizeof(double) * kObjRing,
-                                cudaMemcpyDeviceToHost, st) != cudaSuccess ||
-                cudaStreamSynchronize(st) != cudaSuccess)
-                return fail(FK_ERR_CUDA);
-            copied += kObjRing;
+        const LoopKey key{X,    C,     labels, counts, offsets, ws,     ws_bytes, N,
+                          d,    K,     niter,  dev,    ctx,     dtype,  metric,
+                          timing ? (kernel_only ? 1 : 2) : 0, allow_screen};
+        LoopGraph *g = nullptr;
+        for (LoopGraph &c : cache.graphs)
+            if (c.key == key) g = &c;
+        if (!g && cache.have_last && cache.last == key) {
+            // second identical call in a row: capture the loop on this thread's capture
+            // stream (nothing runs during a capture) and keep the instantiated graph
+            LoopGraph ng;
+            ng.key = key;
+            bool ok = true;
+            if (timing) {
+                ng.ev.reserve(6 * static_cast<size_t>(niter));
+                for (int i = 0; ok && i < 6 * niter; ++i) {
+                    cudaEvent_t e;
+                    ok = cudaEventCreate(&e) == cudaSuccess;
+                    if (ok) ng.ev.push_back(e);
+                }
+            }
+            if (ok && !cache.capture[dev])
+                ok = cudaStreamCreateWithFlags(&cache.capture[dev], cudaStreamNonBlocking) ==
+                     cudaSuccess;
+            cudaStream_t cs = cache.capture[dev];
+            if (ok && timing) {  // the side stream is created outside the capture
+                SideStream *ss = side_stream();
+                ok = ss != nullptr;
+                if (ok) ss->used = false;  // nothing left over from a failed capture
+            }
+            if (ok && cudaStreamBeginCapture(cs, cudaStreamCaptureModeThreadLocal) == cudaSuccess) {
+                const long l0 = g_launches;
+                fk_status r =
+                    issue_loop(cs, phases ? ng.ev.data() : nullptr,
+                               timing ? ng.ev.data() + 4 * niter : nullptr, false,
+                               &ng.nscreened, &ng.last_screened);
+                if (r == FK_OK) r = issue_tail(cs, ng.last_screened);
+                if (join_side_stream(cs) != cudaSuccess) r = FK_ERR_CUDA;
+                cudaGraph_t graph = nullptr;
+                const cudaError_t ee = cudaStreamEndCapture(cs, &graph);
+                ng.launches = g_launches - l0;
+                g_launches = l0;
+                ok = r == FK_OK && ee == cudaSuccess && graph != nullptr &&
+                     cudaGraphInstantiate(&ng.exec, graph, 0) == cudaSuccess;
+                if (graph) cudaGraphDestroy(graph);
+            } else {
+                ok = false;
+            }
+            if (!ok) {
+                // a failed capture leaves this call (and, remembered, later ones with the
+                // same key) to the eager path
+                release(ng);
+                cudaGetLastError();
+            }
+            if (cache.graphs.size() >= kLoopGraphs) {
+                size_t lru = 0;
+                for (size_t i = 1; i < cache.graphs.size(); ++i)
+                    if (cache.graphs[i].used < cache.graphs[lru].used) lru = i;
+                release(cache.graphs[lru]);
+                cache.graphs.erase(cache.graphs.begin() + static_cast<long>(lru));
+            }
+            cache.graphs.push_back(std::move(ng));
+            g = &cache.graphs.back();
+        }
+        cache.last = key;
+        cache.have_last = true;
+        if (g) g->used = ++cache.clock;
+        if (g && g->exec) {
+            if (cudaGraphLaunch(g->exec, st) != cudaSuccess) return FK_ERR_CUDA;
+            note_launch(static_cast<int>(g->launches));
+            nscreened = g->nscreened;
+            last_screened = g->last_screened;
+            if (timing) {
+                lev = phases ? g->ev.data() : nullptr;
+                mev = g->ev.data() + 4 * niter;
+            }
+            replayed = true;
         }
     }
-    if (Ccur != C &&
-        cudaMemcpyAsync(C, Ccur, sizeof(float) * static_cast<size_t>(K) * d,
-                        cudaMemcpyDeviceToDevice, st) != cudaSuccess)
-        return fail(FK_ERR_CUDA);
-    if (objective_host && niter > copied &&
-        cudaMemcpyAsync(objective_host + copied, obj, sizeof(double) * (niter - copied),
-                        cudaMemcpyDeviceToHost, st) != cudaSuccess)
-        return fail(FK_ERR_CUDA);
-    // last-iteration statistics (timing only): words 4, 5 of the error block get the
-    // empty-cluster count and the largest cluster
+    if (!replayed &&
+        ((s = issue_loop(st, lev, mev, true, &nscreened, &last_screened)) != FK_OK ||
+         (s = issue_tail(st, last_screened)) != FK_OK))
+        return s;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return FK_ERR_CUDA;
+    if (objective_host && niter > copied)
+        std::memcpy(objective_host + copied, stage->obj, sizeof(double) * (niter - copied));
+    const uint32_t flags[2] = {stage->words[0], stage->words[1]};
+    const int code = decode_err(flags);
     uint32_t stats[3] = {0, 0, 0};
-    if (timing && niter > 0) {
-        uint32_t *sw = ws_ptr<uint32_t>(ws, L.err) + 4;
-        if (launch_cluster_stats(cnt, K, sw, st) != cudaSuccess ||
-            cudaMemcpyAsync(stats, sw, 2 * sizeof(uint32_t), cudaMemcpyDeviceToHost, st) !=
-                cudaSuccess)
-            return fail(FK_ERR_CUDA);
-        if (last_screened &&
-            cudaMemcpyAsync(stats + 2, ws_ptr<uint32_t>(ws, L.nfb), sizeof(uint32_t),
-                            cudaMemcpyDeviceToHost, st) != cudaSuccess)
-            return fail(FK_ERR_CUDA);
+    if (phases && niter > 0) {
+        stats[0] = stage->words[4];
+        stats[1] = stage->words[5];
+        stats[2] = last_screened ? stage->words[6] : 0u;
     }
-    int code = FK_OK;
-    if (read_err(ws, L, st, true, &code) != FK_OK) return fail(FK_ERR_CUDA);
-    if (timing && ev.size() >= 2) {
+    if (timing) {
         float ms = 0.f;
         std::memset(timing, 0, sizeof(*timing));
+        timing->kernel_only = kernel_only ? 1 : 0;
         timing->empty_clusters = static_cast<int>(stats[0]);
         timing->max_cluster = static_cast<int>(stats[1]);
         timing->fallback_rows = static_cast<int>(stats[2]);
-        cudaEventElapsedTime(&ms, ev[0], ev[1]);
-        timing->ms_setup = ms;
+        const cudaEvent_t e0 = (*pool)[0], e1 = (*pool)[1];
+        if (phases && elapsed_ms(e0, e1, &ms)) timing->ms_setup = ms;
         double *slot[4] = {&timing->ms_prep, &timing->ms_assign, &timing->ms_sort,
                            &timing->ms_update};
         for (int t = 0; t < niter; ++t) {
-            for (int p = 0; p < 4; ++p) {
-                const size_t a = 1 + 4 * t + p;
-                if (a + 1 < ev.size() && cudaEventElapsedTime(&ms, ev[a], ev[a + 1]) == cudaSuccess)
-                    *slot[p] += ms;
+            for (int p = 0; phases && p < 4; ++p) {
+                const int a = 4 * t + p;  // phase p of iteration t ends at lev[a]
+                const cudaEvent_t from = a == 0 ? e1 : lev[a - 1];
+                if (elapsed_ms(from, lev[a], &ms)) *slot[p] += ms;
             }
+            if (elapsed_ms(mev[2 * t], mev[2 * t + 1], &ms)) timing->ms_assign_mma += ms;
         }
         timing->iterations = niter;
         timing->launches = static_cast<int>(g_launches - launches0);
-        for (size_t a = 0; a + 1 < evm.size(); a += 2)
-            if (cudaEventElapsedTime(&ms, evm[a], evm[a + 1]) == cudaSuccess)
-                timing->ms_assign_mma += ms;
         timing->screened = nscreened;
     }
-    cleanup();
     return static_cast<fk_status>(code);
 }
 
@@ -1095,7 +1402,8 @@ fk_status fk_ivf_search(const float *Q, int64_t nq, int d, const float *C, int n
         }
         timing->fallback_queries = nfb;
         float ms[4] = {0, 0, 0, 0};
-        for (int i = 0; i < 4; ++i) cudaEventElapsedTime(&ms[i], ev[i], ev[i + 1]);
+        for (int i = 0; i < 4; ++i)
+            if (!elapsed_ms(ev[i], ev[i + 1], &ms[i])) ms[i] = 0.f;
         timing->ms_coarse = ms[0];
         timing->ms_sort = ms[1];
         timing->ms_fine = ms[2];

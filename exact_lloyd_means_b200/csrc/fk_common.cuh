@@ -534,6 +534,23 @@ cudaError_t smem_opt_in(Kernel kernel, int bytes, std::atomic<uint64_t> &done) {
     return e;
 }
 
+// A timing event at the current point of stream st.  Outside a capture, a plain record.
+// Under stream capture the record goes on a side branch: this thread's side stream forks
+// from st there and records the event as external (an event-record node of the graph; a
+// plain record during a capture records nothing when the graph runs).  The kernels on st
+// then keep their programmatic edges to one another, which an event node between them
+// would break.  join_side_stream(st) joins the branch back before the capture ends.
+cudaError_t record_event(cudaEvent_t e, cudaStream_t st);
+cudaError_t join_side_stream(cudaStream_t st);
+
+// Milliseconds between two recorded events; false (with the runtime's last-error state
+// cleared, so a later launch check does not see it) when they cannot be timed.
+inline bool elapsed_ms(cudaEvent_t a, cudaEvent_t b, float *ms) {
+    if (cudaEventElapsedTime(ms, a, b) == cudaSuccess) return true;
+    cudaGetLastError();
+    return false;
+}
+
 // Kernels launched by this host thread since the last reset (fk_lloyd reports it).
 extern thread_local long g_launches;
 inline void note_launch(int n = 1) { g_launches += n; }

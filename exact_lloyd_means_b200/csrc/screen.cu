@@ -288,9 +288,9 @@ cudaError_t launch_assign_screened(const AssignArgs &a, const float *X32, const 
     s1.mind = nullptr;
     s1.best = nullptr;
     s1.n_dev = nullptr;
-    if (ev_mma0 && (e = cudaEventRecord(ev_mma0, st)) != cudaSuccess) return e;
+    if (ev_mma0 && (e = record_event(ev_mma0, st)) != cudaSuccess) return e;
     if ((e = launch_assign(s1, st)) != cudaSuccess) return e;
-    if (ev_mma1 && (e = cudaEventRecord(ev_mma1, st)) != cudaSuccess) return e;
+    if (ev_mma1 && (e = record_event(ev_mma1, st)) != cudaSuccess) return e;
 
     const int64_t rr_blocks = ceil_div(a.N, 8);
     const int rgrid = static_cast<int>(rr_blocks < 148 * 16 ? rr_blocks : 148 * 16);

@@ -21,7 +21,9 @@
 //               place (digits, then blocks in order) with consecutive threads on
 //               consecutive addresses.  Ranks follow the index order, so the sort is
 //               stable and the output is unique.
-// offsets[k] = first sorted position whose key is >= k, written once per k.
+// offsets[k] = first sorted position whose key is >= k, written once per k: by the first
+// downsweep tile for a one-pass sort (the digit bases are the offsets), else by a kernel of
+// its own after the last pass.
 #include "fk_common.cuh"
 
 namespace fk {
@@ -200,7 +202,8 @@ __global__ void __launch_bounds__(kSortThreads)
     downsweep_kernel(const int32_t *__restrict__ kin, const int32_t *__restrict__ vin,
                      int32_t *__restrict__ kout, int32_t *__restrict__ vout, int64_t n64,
                      int shift, int bits, int K, const uint32_t *__restrict__ hist,
-                     const uint32_t *__restrict__ dtot, int64_t nblocks) {
+                     const uint32_t *__restrict__ dtot, int64_t nblocks,
+                     int32_t *__restrict__ offsets) {
     pdl_wait();
     pdl_trigger();
     constexpr int kTile = kSortThreads * ITEMS;
@@ -239,8 +242,13 @@ __global__ void __launch_bounds__(kSortThreads)
     // global digit bases: exclusive scan of the digit totals (its barriers also order the
     // zeroing above before the counting below)
     block_scan_bins(dtot, gofs, bins, part);
-    for (int b = threadIdx.x; b < bins; b += blockDim.x)
+    for (int b = threadIdx.x; b < bins; b += blockDim.x) {
+        // a one-pass sort's digit is the whole key: the CSR offsets are the digit bases,
+        // written by the first tile
+        if (offsets && blockIdx.x == 0 && b < K) offsets[b] = static_cast<int32_t>(gofs[b]);
         gofs[b] += hist[static_cast<int64_t>(b) * nblocks + blockIdx.x];
+    }
+    if (offsets && blockIdx.x == 0 && threadIdx.x == 0) offsets[K] = static_cast<int32_t>(n);
 
     uint32_t *h = wh + warp * bins;
     const uint32_t lt = lanemask_lt();
@@ -364,6 +372,8 @@ cudaError_t launch_sort_csr(const int32_t *labels, int64_t N, int K, const SortP
                               sizeof(int32_t) * 2 * kSortTile <= 48 * 1024,
                       "sort shared memory above the default limit");
         const bool small = sp.items == kSortItemsSmall;
+        // a one-pass sort's downsweep writes the CSR offsets (no offsets launch)
+        const bool one_pass = sp.passes == 1;
         const int32_t *kin = labels;
         const int32_t *vin = nullptr;
         int32_t *kb[2] = {keys0, keys1};
@@ -380,13 +390,14 @@ cudaError_t launch_sort_csr(const int32_t *labels, int64_t N, int K, const SortP
             int32_t *vo = (p == sp.passes - 1 && perm_out) ? perm_out : vb[p & 1];
             launch_pdl(small ? downsweep_kernel<kSortItemsSmall> : downsweep_kernel<kSortItems>,
                        grid, dim3(kSortThreads), dn_smem, st, kin, vin, kb[p & 1], vo, N, shift,
-                       sp.bits, K, hist, dtot, sp.nblocks);
+                       sp.bits, K, hist, dtot, sp.nblocks, one_pass ? offsets : nullptr);
             note_launch();
             kin = kb[p & 1];
             vin = vo;
         }
         *sorted_keys = kin;
         *perm = vin;
+        if (one_pass) return cudaGetLastError();  // offsets written by the downsweep
     }
     launch_pdl(csr_offsets_kernel, dim3(grid_cap(N + 1, 256)), dim3(256), 0, st, *sorted_keys, N,
                K, offsets);

@@ -641,6 +641,31 @@ __global__ void finalize_shards_kernel(const double *__restrict__ sums,
     }
 }
 
+// The objective partials summed in a fixed order by one block of 256 threads: thread t
+// adds entries t, t + 256, ... in index order (eight loads are issued before the eight
+// additions, so the loop is not a chain of dependent loads), then a fixed tree over the
+// threads.  sh: 256 doubles of shared memory.
+__device__ __forceinline__ void sum_objective(const double *__restrict__ part, int64_t n,
+                                              double *__restrict__ objective, double *sh) {
+    double s = 0.0;
+    int64_t i = threadIdx.x;
+    for (; i + 7 * 256 < n; i += 8 * 256) {
+        double v[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) v[j] = part[i + j * 256];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) s += v[j];
+    }
+    for (; i < n; i += 256) s += part[i];
+    sh[threadIdx.x] = s;
+    __syncthreads();
+    for (int o = 128; o > 0; o >>= 1) {
+        if (threadIdx.x < o) sh[threadIdx.x] += sh[threadIdx.x + o];
+        __syncthreads();
+    }
+    if (threadIdx.x == 0) *objective = sh[0];
+}
+
 // The update's tail steps in one launch.  Block 0 sums the n objective partials (thread t
 // adds t, t + 256, ... in order, then a fixed tree).  Blocks 1 .. nfin run the last combine
 // level (one unit; warp 0 of block 1 + cb handles column block cb).  The other blocks
@@ -661,25 +686,7 @@ __global__ void __launch_bounds__(256)
     if (blockIdx.x == 0) {
         if (objective == nullptr) return;
         __shared__ double sh[256];
-        // each thread adds its strided entries in index order; eight loads are issued
-        // before the eight additions so the loop is not a chain of dependent loads
-        double s = 0.0;
-        int64_t i = threadIdx.x;
-        for (; i + 7 * 256 < n; i += 8 * 256) {
-            double v[8];
-#pragma unroll
-            for (int j = 0; j < 8; ++j) v[j] = part[i + j * 256];
-#pragma unroll
-            for (int j = 0; j < 8; ++j) s += v[j];
-        }
-        for (; i < n; i += 256) s += part[i];
-        sh[threadIdx.x] = s;
-        __syncthreads();
-        for (int o = 128; o > 0; o >>= 1) {
-            if (threadIdx.x < o) sh[threadIdx.x] += sh[threadIdx.x + o];
-            __syncthreads();
-        }
-        if (threadIdx.x == 0) *objective = sh[0];
+        sum_objective(part, n, objective, sh);
         return;
     }
     if (static_cast<int>(blockIdx.x) <= nfin) {
@@ -706,6 +713,115 @@ __global__ void __launch_bounds__(256)
     }
 }
 
+// Every combine level of a small problem (at most kWideUnits level-1 units) in one launch.
+// A block evaluates, for one cluster at a time and one column block, the cluster's share of
+// every combine level: the sums it forms are those of seg_pieces_kernel and of the tail's
+// last level (the same pieces added in the same order, kGroup units of one level to a unit
+// of the next), so the centroids are bit for bit those of the level-by-level launches; only
+// the chain of dependent launches is gone.  A cluster's units are consecutive, so its
+// level-2 partials number at most kWideUnits / kGroup and fit in shared memory; higher
+// levels use a small second buffer.  The last block sums the objective.  counts[k] comes
+// from the offsets, and an empty cluster keeps C_old bit for bit (a zero sum for a shard).
+constexpr int kWideWarps = 8;
+constexpr int64_t kWideUnits = 1024;
+constexpr int kWideL2 = static_cast<int>(kWideUnits / kGroup);  // level-2 partials, at most
+constexpr int kWideL3 = 8;  // level >= 3 partials: (kWideL2 - 1) / kGroup + 2 at most
+static_assert(kWideL3 >= (kWideL2 - 1) / kGroup + 2, "level-3 buffer too small");
+static_assert(kWideWarps * 32 == 256, "sum_objective runs on 256 threads");
+constexpr size_t kWideSmem = size_t(kWideL2 + kWideL3) * 128 * sizeof(double);
+
+__global__ void __launch_bounds__(kWideWarps * 32)
+    wide_combine_kernel(const double *__restrict__ pieces, int rows_log2, int K, int d,
+                        int dcov, const int32_t *__restrict__ offsets,
+                        const float *__restrict__ C_old, float *__restrict__ C_new,
+                        double *__restrict__ sums_out, int32_t *__restrict__ counts,
+                        const double *__restrict__ jpart, int64_t njpart,
+                        double *__restrict__ objective) {
+    pdl_wait();
+    pdl_trigger();
+    extern __shared__ __align__(16) double s_part[];  // [kWideL2][128], then [kWideL3][128]
+    __shared__ double s_obj[256];
+    const int cb = blockIdx.y;
+    if (blockIdx.x == gridDim.x - 1) {
+        if (cb == 0 && objective) sum_objective(jpart, njpart, objective, s_obj);
+        return;
+    }
+    const int tid = threadIdx.x;
+    const int lane = tid & 31;
+    const int warp = tid >> 5;
+    const int col = cb * 128 + lane * 4;
+    const bool colv = col < d;
+    const int cend = d < cb * 128 + 128 ? d : cb * 128 + 128;
+    const int64_t R = int64_t(1) << rows_log2;
+    const int stride = static_cast<int>(gridDim.x) - 1;
+    for (int k = blockIdx.x; k < K; k += stride) {
+        const int64_t lo = offsets[k], hi = offsets[k + 1];
+        if (cb == 0 && tid == 0 && counts) counts[k] = static_cast<int32_t>(hi - lo);
+        if (hi == lo) {
+            for (int j = cb * 128 + tid; j < cend; j += kWideWarps * 32) {
+                if (sums_out)
+                    sums_out[int64_t(k) * d + j] = 0.0;
+                else
+                    C_new[int64_t(k) * d + j] = C_old[int64_t(k) * d + j];
+            }
+            continue;
+        }
+        int64_t a0 = lo >> rows_log2, a1 = (hi - 1) >> rows_log2;  // units of the level below
+        if (a0 == a1) continue;  // finished by the level-1 kernel
+        const double *src = nullptr;  // the level below in shared memory (level 1: pieces)
+        double *dst = s_part;
+        while (true) {
+            const int64_t g0 = a0 / kGroup, g1 = a1 / kGroup;
+            const bool done = g0 == g1;  // the cluster lies in one unit of this level
+            for (int64_t g = g0 + warp; g <= g1; g += kWideWarps) {
+                const int64_t ia = a0 > g * kGroup ? a0 : g * kGroup;
+                const int64_t ib = a1 < g * kGroup + kGroup - 1 ? a1 : g * kGroup + kGroup - 1;
+                double acc[4] = {0.0, 0.0, 0.0, 0.0};
+                for (int64_t b = ia; b <= ib; b += 8) {
+                    double2 va[8], vb[8];
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        const int64_t i = b + j;
+                        va[j] = vb[j] = make_double2(0.0, 0.0);
+                        if (i <= ib && colv) {
+                            const double *q;
+                            if (src == nullptr)  // a level-1 unit: slot 0 when the cluster
+                                                 // holds the unit's first position
+                                q = pieces + (i * 2 + (lo <= i * R ? 0 : 1)) * int64_t(dcov) + col;
+                            else
+                                q = src + (i - a0) * 128 + lane * 4;
+                            va[j] = reinterpret_cast<const double2 *>(q)[0];
+                            vb[j] = reinterpret_cast<const double2 *>(q)[1];
+                        }
+                    }
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        if (b + j > ib) break;
+                        acc[0] += va[j].x;
+                        acc[1] += va[j].y;
+                        acc[2] += vb[j].x;
+                        acc[3] += vb[j].y;
+                    }
+                }
+                if (done) {
+                    if (colv)
+                        store_done(C_new, sums_out, k, d, col, acc, static_cast<double>(hi - lo));
+                } else {
+                    double2 *o = reinterpret_cast<double2 *>(dst + (g - g0) * 128 + lane * 4);
+                    o[0] = make_double2(acc[0], acc[1]);
+                    o[1] = make_double2(acc[2], acc[3]);
+                }
+            }
+            __syncthreads();  // this level's partials are written before the next reads them
+            if (done) break;
+            a0 = g0;
+            a1 = g1;
+            src = dst;
+            dst = dst == s_part ? s_part + kWideL2 * 128 : s_part;
+        }
+    }
+}
+
 // The last combine level (a single unit), left for the update's tail launch.
 struct FinalLevel {
     bool pending = false;
@@ -722,7 +838,7 @@ cudaError_t run_levels(const void *X, bool bf16, int64_t N, int d, const UpdPlan
                        const float *C_used, float *C_new, double *sums_out, double *pa,
                        int32_t *ka,
                        double *pb, int32_t *kb, double *jpart, uint32_t *err,
-                       cudaStream_t st, FinalLevel *final_level) {
+                       cudaStream_t st, FinalLevel *final_level, bool level1_only) {
     static std::atomic<uint64_t> smem_set{0};
     {
         const cudaError_t e =
@@ -752,7 +868,7 @@ cudaError_t run_levels(const void *X, bool bf16, int64_t N, int d, const UpdPlan
     int64_t span = up.rows;
     double *pin = pa, *pout = pb;
     int32_t *kin = ka, *kout = kb;
-    while (units > 1) {
+    while (units > 1 && !level1_only) {
         const int64_t nunits = ceil_div(units, kGroup);
         span *= kGroup;
         if (nunits == 1) {  // the last level runs inside the tail launch
@@ -791,10 +907,29 @@ cudaError_t launch_update(const void *X, fk_dtype dtype, int64_t N, int d, int K
                           cudaStream_t st) {
     const bool bf16 = dtype == FK_BF16;
     FinalLevel fl;
+    const bool wide = up.nwarps <= kWideUnits;
     cudaError_t e = run_levels(X, bf16, N, d, up, skeys, perm, offsets, C_used, C_new,
                                sums_out, pieces_a, pkeys_a, pieces_b, pkeys_b, jpart, err, st,
-                               &fl);
+                               &fl, wide);
     if (e != cudaSuccess) return e;
+    if (wide) {
+        // a small problem: every combine level, the finalize and the objective in one launch
+        static std::atomic<uint64_t> smem_set{0};
+        if ((e = smem_opt_in(wide_combine_kernel, static_cast<int>(kWideSmem), smem_set)) !=
+            cudaSuccess)
+            return e;
+        int rows_log2 = 0;
+        while ((1 << rows_log2) < up.rows) ++rows_log2;  // rows is a power of two
+        int64_t blocks = K;
+        const int64_t cap = static_cast<int64_t>(device_sm_count()) * 3;  // 3 fit per SM
+        if (blocks > cap) blocks = cap;
+        launch_pdl(wide_combine_kernel, dim3(static_cast<unsigned>(blocks + 1), up.ncolblk),
+                   dim3(kWideWarps * 32), kWideSmem, st, pieces_a, rows_log2, K, d,
+                   up.dcov, offsets, C_old, C_new, sums_out, counts, jpart,
+                   up.nwarps * up.ncolblk, objective);
+        note_launch();
+        return cudaGetLastError();
+    }
     // the update's tail in one launch: the objective (block 0), the last combine level (one
     // block per 128-column block) and the empty clusters (the remaining blocks)
     int64_t fgrid = ceil_div(K, 8);

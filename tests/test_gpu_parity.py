@@ -74,7 +74,8 @@ def test_assign_tight_mixture_recovers_components():
 
 UPDATE_SHAPES = [(1000, 64, 10, "equal"), (20000, 128, 37, "equal"), (70000, 128, 3, "equal"),
                  (5000, 768, 50, "equal"), (3000, 1032, 20, "equal"), (200000, 16, 2, "equal"),
-                 (150000, 128, 4096, "zipf"), (777, 8, 700, "equal")]
+                 (150000, 128, 4096, "zipf"), (777, 8, 700, "equal"),
+                 (60000, 96, 500, "zipf")]
 
 
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
@@ -227,6 +228,72 @@ def test_fk_lloyd_deterministic_and_resumable():
     c = run(C0.to(DEV).clone(), 2)
     d = run(c[0].clone(), 3)
     assert torch.equal(d[0], a[0]) and torch.equal(d[1], a[1]) and d[2] == a[2][2:]
+
+
+def test_fk_lloyd_repeated_calls_replay_identically():
+    """A call that repeats the previous one replays its iteration loop from a CUDA graph
+    (captured on the second call): every call gives the eager call's result bit for bit,
+    new centroid values reach the replayed loop, and timing still works on a replay."""
+    N, d, K = 20000, 128, 200
+    X, C0, _ = _mixture(N, d, K, seed=12, centers="normal", sigma=0.3)
+    m = fk()
+    Xg = X.to(DEV)
+    ws = m.workspace(N, d, K, torch.float32, "l2")
+    C = torch.empty(K, d, dtype=torch.float32, device=DEV)
+    labels = torch.empty(N, dtype=torch.int32, device=DEV)
+    counts = torch.empty(K, dtype=torch.int32, device=DEV)
+
+    def run(Cinit, lab=labels, timing=False):
+        C.copy_(Cinit)
+        objs, tm = m.fk_lloyd(Xg, C, 4, lab, ws, counts=counts, timing=timing)
+        return C.clone(), lab.clone(), counts.clone(), objs, tm
+
+    C0g = C0.to(DEV)
+    ref = run(C0g)
+    for _ in range(3):
+        r = run(C0g)
+        assert all(torch.equal(a, b) for a, b in zip(r[:3], ref[:3])) and r[3] == ref[3]
+    timed = [run(C0g, timing=True) for _ in range(3)]
+    for r in timed:
+        assert all(torch.equal(a, b) for a, b in zip(r[:3], ref[:3])) and r[3] == ref[3]
+        tm = r[4]
+        assert tm["iterations"] == 4 and tm["launches"] == timed[0][4]["launches"] > 0
+        for k in ("ms_prep", "ms_assign", "ms_sort", "ms_update", "ms_assign_mma"):
+            assert tm[k] > 0, k
+    # kernel-only timing: the assignment kernel's time alone, the same results
+    for r in [run(C0g, timing="kernel") for _ in range(3)]:
+        assert all(torch.equal(a, b) for a, b in zip(r[:3], ref[:3])) and r[3] == ref[3]
+        tm = r[4]
+        assert tm["kernel_only"] == 1 and tm["iterations"] == 4 and tm["ms_assign_mma"] > 0
+        assert tm["ms_assign"] == 0 and tm["ms_update"] == 0 and tm["max_cluster"] == 0
+        assert tm["launches"] == timed[0][4]["launches"] - 1  # no statistics kernel
+    # other initial centroids: the eager result (another labels buffer, so another call)
+    # equals the replay of the cached loop with the original buffers
+    C1g = C0g[torch.randperm(K, generator=torch.Generator().manual_seed(5)).to(DEV)]
+    other = torch.empty_like(labels)
+    e = run(C1g, lab=other)
+    run(C0g)  # make the cached call the previous one again
+    r = run(C1g)
+    assert torch.equal(r[0], e[0]) and torch.equal(r[1], e[1]) and r[3] == e[3]
+    assert not torch.equal(r[0], ref[0])
+
+
+def test_fk_lloyd_objective_ring_wraps():
+    """More iterations than the device's objective ring (4096 entries): the full ring is
+    handed to the host before it wraps, and the run equals the same run in two calls."""
+    N, d, K = 2000, 16, 8
+    X, C0, _ = _mixture(N, d, K, seed=13, centers="normal", sigma=0.5)
+    m = fk()
+    Xg = X.to(DEV)
+    ws = m.workspace(N, d, K, torch.float32, "l2")
+    labels = torch.empty(N, dtype=torch.int32, device=DEV)
+    Ca = C0.to(DEV).clone()
+    oa, _ = m.fk_lloyd(Xg, Ca, 4099, labels, ws)
+    Cb = C0.to(DEV).clone()
+    ob1, _ = m.fk_lloyd(Xg, Cb, 4096, labels, ws)
+    ob2, _ = m.fk_lloyd(Xg, Cb, 3, labels, ws)
+    assert len(oa) == 4099 and oa == ob1 + ob2 and torch.equal(Ca, Cb)
+    assert all(o > 0 for o in oa)
 
 
 def test_fk_lloyd_k_equals_one_and_k_equals_n():
