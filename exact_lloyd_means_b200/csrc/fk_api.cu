@@ -308,7 +308,7 @@ fk_status read_err(void *ws, const WsLayout &L, cudaStream_t st, bool clear, int
     uint32_t e[2] = {0, 0};
     uint32_t *dev = ws_ptr<uint32_t>(ws, L.err);
     FK_TRY_CUDA(cudaMemcpyAsync(e, dev, sizeof(e), cudaMemcpyDeviceToHost, st));
-    if (clear) FK_TRY_CUDA(cudaMemsetAsync(dev, 0, sizeof(e), st));
+    if (clear) FK_TRY_CUDA(cudaMemsetAsync(dev, 0, kErrWords * sizeof(uint32_t), st));
     FK_TRY_CUDA(cudaStreamSynchronize(st));
     *code = e[0] ? FK_ERR_TIMEOUT : (e[1] ? FK_ERR_DEVICE : FK_OK);
     return FK_OK;
@@ -786,7 +786,7 @@ fk_status fk_lloyd(const void *X, fk_dtype dtype, int64_t N, int d, int K, fk_me
         return FK_ERR_CUDA;
 
     NvtxRange call_range("fk_lloyd");
-    if (cudaMemsetAsync(ws_ptr<uint32_t>(ws, L.err), 0, 2 * sizeof(uint32_t), st) != cudaSuccess)
+    if (cudaMemsetAsync(ws_ptr<uint32_t>(ws, L.err), 0, kErrWords * sizeof(uint32_t), st) != cudaSuccess)
         return FK_ERR_CUDA;
     const long launches0 = g_launches;
     if (phases && cudaEventRecord((*pool)[0], st) != cudaSuccess) return FK_ERR_CUDA;
@@ -849,11 +849,18 @@ fk_status fk_lloyd(const void *X, fk_dtype dtype, int64_t N, int d, int K, fk_me
         auto rec = [&](int i) { return !lev || record_event(lev[i], s_) == cudaSuccess; };
         int nscr = 0;
         bool last = false;
+        // the centroid operands; a small problem's update prepares the next iteration's
+        const CentroidOperands ops{ws_ptr<uint16_t>(ws, L.cs), ws_ptr<float>(ws, L.cn),
+                                   dtype == FK_F32 ? nullptr : cused,
+                                   ws_ptr<uint16_t>(ws, L.caug), L.Kp, L.dp,
+                                   dtype == FK_F32 ? 1 : 0};
+        bool prepped = false;
         for (int t = 0; t < niter; ++t) {
             NvtxRange iter_range("fk_lloyd iteration");
-            if (launch_prep_centroids(Ccur, K, d, L.Kp, L.dp, dtype, ws_ptr<uint16_t>(ws, L.cs),
-                                      ws_ptr<float>(ws, L.cn), cused,
-                                      ws_ptr<uint16_t>(ws, L.caug), s_) != cudaSuccess ||
+            if ((!prepped &&
+                 launch_prep_centroids(Ccur, K, d, L.Kp, L.dp, dtype, ws_ptr<uint16_t>(ws, L.cs),
+                                       ws_ptr<float>(ws, L.cn), cused,
+                                       ws_ptr<uint16_t>(ws, L.caug), s_) != cudaSuccess) ||
                 !rec(4 * t))
                 return FK_ERR_CUDA;
             bool screened = false;
@@ -879,7 +886,8 @@ fk_status fk_lloyd(const void *X, fk_dtype dtype, int64_t N, int d, int K, fk_me
                               ws_ptr<double>(ws, L.pieces), ws_ptr<int32_t>(ws, L.pkeys),
                               ws_ptr<double>(ws, L.piecesb), ws_ptr<int32_t>(ws, L.pkeysb),
                               ws_ptr<double>(ws, L.jpart), obj + (t % kObjRing),
-                              ws_ptr<uint32_t>(ws, L.err), nullptr, s_) != cudaSuccess ||
+                              ws_ptr<uint32_t>(ws, L.err), nullptr, s_, &ops,
+                              &prepped) != cudaSuccess ||
                 !rec(4 * t + 3))
                 return FK_ERR_CUDA;
             float *tmp = Ccur;
@@ -1180,7 +1188,7 @@ fk_status fk_lloyd_streamed(const void *X_host, fk_dtype dtype, int64_t N, int d
     float *cused = ws_ptr<float>(ws, L.cused);
     auto rows_of = [&](int64_t c) { return N - c * chunk_rows < chunk_rows ? N - c * chunk_rows : chunk_rows; };
 
-    if (cudaMemsetAsync(ws_ptr<uint32_t>(ws, L.err), 0, 2 * sizeof(uint32_t), st) != cudaSuccess)
+    if (cudaMemsetAsync(ws_ptr<uint32_t>(ws, L.err), 0, kErrWords * sizeof(uint32_t), st) != cudaSuccess)
         return fail(FK_ERR_CUDA);
     if (metric == FK_COSINE && launch_normalize(C, C, K, d, st) != cudaSuccess)
         return fail(FK_ERR_CUDA);

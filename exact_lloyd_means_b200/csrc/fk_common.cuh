@@ -30,6 +30,15 @@ constexpr int64_t kSortSmallN = int64_t(1) << 22;
 // digit width bound: 256 bins (a tile's per-digit bookkeeping grows with the bins, so two
 // narrow passes beat one wide one from about 1024 bins)
 constexpr int kSortMaxBits = 8;
+// Tiles up to which the upsweep's last tile scans the per-tile counts itself (its threads
+// read a digit's counts each: 256 tiles are 1 KB per thread)
+constexpr int64_t kSortScanInUpsweep = 256;
+// Words of the 256-byte error block at the start of a workspace: [0] a bounded wait
+// expired, [1] a label out of range, [4..5] the last iteration's statistics, [8] the
+// sort's tile ticket (zero between calls: the last tile resets it).  Cleared on entry by
+// fk_lloyd, and by fk_get_device_error.
+constexpr int kSortTicketWord = 8;
+constexpr int kErrWords = 9;
 
 // ----------------------------------------------------------------- update tiling
 constexpr int kUpdWarps = 8;          // warps per block of the update kernels
@@ -37,6 +46,8 @@ constexpr int kUpdGroup = 16;         // units of one combine level per unit of 
 constexpr int kUpdMinRows = 64;       // smallest chunk of sorted positions per warp
 constexpr int kUpdMaxRows = 256;      // largest chunk
 constexpr int64_t kUpdTargetWarps = 148 * 64;  // enough warps to cover the GPU twice
+// Level-1 units up to which every combine level runs in one launch (wide_combine_kernel)
+constexpr int64_t kUpdWideUnits = 2048;
 
 // ----------------------------------------------------------------- screening (fp32)
 // The single-product pass writes, per row, up to kCandPerRow candidate columns (unused
@@ -341,13 +352,28 @@ cudaError_t launch_sort_csr(const int32_t *labels, int64_t N, int K, const SortP
                             int32_t *perm_out, uint32_t *hist, uint32_t *dtot,
                             int32_t *offsets, const int32_t **sorted_keys,
                             const int32_t **perm, uint32_t *err, cudaStream_t st);
+// The assign operands of the centroids (prep_centroids_kernel's outputs): planes
+// [cplanes][Kp][dp] bf16, norms cn[Kp], cused[K][d] (bf16 points only) and the norm pieces
+// caug[Kp][kAug].
+struct CentroidOperands {
+    uint16_t *planes;
+    float *cn;
+    float *cused;
+    uint16_t *caug;
+    int64_t Kp, dp;
+    int two_planes;
+};
+// next (may be null): where a small problem's update (one column block, the one-launch
+// combine) may also prepare the new centroids' operands as it finishes them; *prepped
+// tells whether it did, so the next iteration can skip prep_centroids.
 cudaError_t launch_update(const void *X, fk_dtype dtype, int64_t N, int d, int K,
                           const UpdPlan &up, const int32_t *skeys, const int32_t *perm,
                           const int32_t *offsets, const float *C_old, const float *C_used,
                           float *C_new, int32_t *counts, double *pieces_a, int32_t *pkeys_a,
                           double *pieces_b, int32_t *pkeys_b, double *jpart,
                           double *objective, uint32_t *err, double *sums_out,
-                          cudaStream_t st);
+                          cudaStream_t st, const CentroidOperands *next = nullptr,
+                          bool *prepped = nullptr);
 cudaError_t launch_gather_rows(const void *X, int64_t N, int64_t row_bytes,
                                const int32_t *row_ids, void *out, cudaStream_t st);
 cudaError_t launch_accumulate_chunk(double *tot, const double *part, int64_t KD,

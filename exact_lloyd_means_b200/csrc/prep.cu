@@ -17,22 +17,10 @@
 #include <cuda_bf16.h>
 
 #include "fk_common.cuh"
+#include "prep_row.cuh"
 
 namespace fk {
 namespace {
-
-__device__ __forceinline__ uint16_t bf16_bits(float f) {
-    return __bfloat16_as_ushort(__float2bfloat16_rn(f));
-}
-__device__ __forceinline__ float bf16_val(uint16_t b) {
-    return __bfloat162float(__ushort_as_bfloat16(b));
-}
-
-__device__ __forceinline__ double warp_sum_d(double v) {
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-    return v;
-}
 
 // One warp per row; lanes walk the row four columns at a time.
 __global__ void split_x_kernel(const float *__restrict__ X, int64_t N, int d, int64_t dp,
@@ -129,51 +117,13 @@ __global__ void normalize_kernel(const float *__restrict__ X, float *__restrict_
     }
 }
 
-// One warp per (padded) centroid.  Planes: [cplanes][Kp][dp] bf16, holding -2*hi (and
-// -2*lo for the fp32 emulation).  cused (bf16 mode only): the bf16-rounded centroid
-// widened to fp32, i.e. exactly what the MMA sees.
-__global__ void prep_centroids_kernel(const float *__restrict__ C, int K, int d, int64_t Kp,
-                                      int64_t dp, int two_planes, uint16_t *__restrict__ planes,
-                                      float *__restrict__ cn, float *__restrict__ cused,
-                                      uint16_t *__restrict__ caug) {
+// One warp per (padded) centroid row (prep_row.cuh).
+__global__ void prep_centroids_kernel(const float *__restrict__ C, int K, int d,
+                                      CentroidOperands o) {
     const int lane = threadIdx.x & 31;
     const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
     const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
-    for (int64_t k = warp; k < Kp; k += nwarps) {
-        uint16_t *p0 = planes + k * dp;
-        uint16_t *p1 = planes + (Kp + k) * dp;
-        double s = 0.0;
-        for (int64_t j = lane; j < dp; j += 32) {
-            const float c = (k < K && j < d) ? C[k * d + j] : 0.f;
-            const uint16_t h = bf16_bits(c);
-            const float hv = bf16_val(h);
-            // -2 * bf16 value is exact in bf16 (a power-of-two scale)
-            p0[j] = bf16_bits(-2.f * hv);
-            if (two_planes) {
-                const uint16_t l = bf16_bits(c - hv);
-                p1[j] = bf16_bits(-2.f * bf16_val(l));
-                s += static_cast<double>(c) * c;
-            } else {
-                s += static_cast<double>(hv) * hv;
-                if (k < K && j < d && cused) cused[k * d + j] = hv;
-            }
-        }
-        s = warp_sum_d(s);
-        const float c2 = static_cast<float>(s);
-        if (lane == 0) cn[k] = k < K ? c2 : __int_as_float(0x7f800000);
-        if (caug != nullptr && lane < kAug) {
-            // exact split: hi captures the top 8 bits, mid the next 8, lo the rest (a
-            // multiple of the fp32 ulp with at most 8 significant bits)
-            const uint16_t h = bf16_bits(c2);
-            const float r1 = c2 - bf16_val(h);
-            const uint16_t m = bf16_bits(r1);
-            const uint16_t l = bf16_bits(r1 - bf16_val(m));
-            uint16_t v = 0;
-            if (k < K) v = lane == 0 ? h : (lane == 1 ? m : (lane == 2 ? l : 0));
-            else v = lane == 0 ? static_cast<uint16_t>(0x7f7f) : 0;  // largest finite bf16
-            caug[k * kAug + lane] = v;
-        }
-    }
+    for (int64_t k = warp; k < o.Kp; k += nwarps) prep_centroid_row(C, K, d, o, k, lane);
 }
 
 __global__ void centroid_norms_kernel(const float *__restrict__ C, int K, int d, int round_bf16,
@@ -233,8 +183,8 @@ cudaError_t launch_xnorm_bf16(const uint16_t *X, int64_t N, int d, float *xnorm,
 cudaError_t launch_prep_centroids(const float *C, int K, int d, int64_t Kp, int64_t dp,
                                   fk_dtype dtype, uint16_t *planes, float *cn, float *cused,
                                   uint16_t *caug, cudaStream_t st) {
-    prep_centroids_kernel<<<grid_for_warps(Kp, 256), 256, 0, st>>>(
-        C, K, d, Kp, dp, dtype == FK_BF16 ? 0 : 1, planes, cn, cused, caug);
+    const CentroidOperands o{planes, cn, cused, caug, Kp, dp, dtype == FK_BF16 ? 0 : 1};
+    prep_centroids_kernel<<<grid_for_warps(Kp, 256), 256, 0, st>>>(C, K, d, o);
     note_launch();
     return cudaGetLastError();
 }

@@ -29,6 +29,7 @@
 #include <cuda_bf16.h>
 
 #include "fk_common.cuh"
+#include "prep_row.cuh"
 #include "ptx_sm100.cuh"
 
 namespace fk {
@@ -713,33 +714,36 @@ __global__ void __launch_bounds__(256)
     }
 }
 
-// Every combine level of a small problem (at most kWideUnits level-1 units) in one launch.
-// A block evaluates, for one cluster at a time and one column block, the cluster's share of
-// every combine level: the sums it forms are those of seg_pieces_kernel and of the tail's
-// last level (the same pieces added in the same order, kGroup units of one level to a unit
-// of the next), so the centroids are bit for bit those of the level-by-level launches; only
-// the chain of dependent launches is gone.  A cluster's units are consecutive, so its
-// level-2 partials number at most kWideUnits / kGroup and fit in shared memory; higher
-// levels use a small second buffer.  The last block sums the objective.  counts[k] comes
-// from the offsets, and an empty cluster keeps C_old bit for bit (a zero sum for a shard).
+// Every combine level of a small problem (at most kUpdWideUnits level-1 units) in one
+// launch.  A block evaluates, for one cluster at a time and one column block, the cluster's
+// share of every combine level: the sums it forms are those of seg_pieces_kernel and of the
+// tail's last level (the same pieces added in the same order, kGroup units of one level to
+// a unit of the next), so the centroids are bit for bit those of the level-by-level
+// launches; only the chain of dependent launches is gone.  A cluster's units are
+// consecutive, so its level-2 partials number at most l2cap = (units - 1) / kGroup + 1 and
+// fit in shared memory; higher levels use a second buffer of l2cap / kGroup + 2 entries.
+// The last block sums the objective.  counts[k] comes from the offsets, and an empty
+// cluster keeps C_old bit for bit (a zero sum for a shard).
 constexpr int kWideWarps = 8;
-constexpr int64_t kWideUnits = 1024;
-constexpr int kWideL2 = static_cast<int>(kWideUnits / kGroup);  // level-2 partials, at most
-constexpr int kWideL3 = 8;  // level >= 3 partials: (kWideL2 - 1) / kGroup + 2 at most
-static_assert(kWideL3 >= (kWideL2 - 1) / kGroup + 2, "level-3 buffer too small");
 static_assert(kWideWarps * 32 == 256, "sum_objective runs on 256 threads");
-constexpr size_t kWideSmem = size_t(kWideL2 + kWideL3) * 128 * sizeof(double);
+
+// Shared-memory entries (128 doubles each) of the two level buffers for `units` units.
+inline int wide_l2cap(int64_t units) { return static_cast<int>((units - 1) / kGroup + 1); }
+inline int wide_l3cap(int64_t units) { return wide_l2cap(units) / kGroup + 2; }
+inline size_t wide_smem(int64_t units) {
+    return size_t(wide_l2cap(units) + wide_l3cap(units)) * 128 * sizeof(double);
+}
 
 __global__ void __launch_bounds__(kWideWarps * 32)
-    wide_combine_kernel(const double *__restrict__ pieces, int rows_log2, int K, int d,
-                        int dcov, const int32_t *__restrict__ offsets,
+    wide_combine_kernel(const double *__restrict__ pieces, int rows_log2, int l2cap, int K,
+                        int d, int dcov, const int32_t *__restrict__ offsets,
                         const float *__restrict__ C_old, float *__restrict__ C_new,
                         double *__restrict__ sums_out, int32_t *__restrict__ counts,
                         const double *__restrict__ jpart, int64_t njpart,
-                        double *__restrict__ objective) {
+                        double *__restrict__ objective, CentroidOperands next) {
     pdl_wait();
     pdl_trigger();
-    extern __shared__ __align__(16) double s_part[];  // [kWideL2][128], then [kWideL3][128]
+    extern __shared__ __align__(16) double s_part[];  // [l2cap][128], then [l3cap][128]
     __shared__ double s_obj[256];
     const int cb = blockIdx.y;
     if (blockIdx.x == gridDim.x - 1) {
@@ -757,6 +761,7 @@ __global__ void __launch_bounds__(kWideWarps * 32)
     for (int k = blockIdx.x; k < K; k += stride) {
         const int64_t lo = offsets[k], hi = offsets[k + 1];
         if (cb == 0 && tid == 0 && counts) counts[k] = static_cast<int32_t>(hi - lo);
+        int64_t a0 = lo >> rows_log2, a1 = (hi - 1) >> rows_log2;  // units of the level below
         if (hi == lo) {
             for (int j = cb * 128 + tid; j < cend; j += kWideWarps * 32) {
                 if (sums_out)
@@ -764,13 +769,11 @@ __global__ void __launch_bounds__(kWideWarps * 32)
                 else
                     C_new[int64_t(k) * d + j] = C_old[int64_t(k) * d + j];
             }
-            continue;
+            a1 = a0;  // no combine
         }
-        int64_t a0 = lo >> rows_log2, a1 = (hi - 1) >> rows_log2;  // units of the level below
-        if (a0 == a1) continue;  // finished by the level-1 kernel
         const double *src = nullptr;  // the level below in shared memory (level 1: pieces)
         double *dst = s_part;
-        while (true) {
+        while (a0 != a1) {  // a0 == a1: finished by the level-1 kernel (or empty)
             const int64_t g0 = a0 / kGroup, g1 = a1 / kGroup;
             const bool done = g0 == g1;  // the cluster lies in one unit of this level
             for (int64_t g = g0 + warp; g <= g1; g += kWideWarps) {
@@ -817,7 +820,13 @@ __global__ void __launch_bounds__(kWideWarps * 32)
             a0 = g0;
             a1 = g1;
             src = dst;
-            dst = dst == s_part ? s_part + kWideL2 * 128 : s_part;
+            dst = dst == s_part ? s_part + l2cap * 128 : s_part;
+        }
+        if (next.planes != nullptr) {
+            // row k of C_new is final (written by the level-1 kernel, or by this block
+            // before the barrier): its operands for the next iteration's assignment
+            __syncthreads();
+            if (warp == 0) prep_centroid_row(C_new, K, d, next, k, lane);
         }
     }
 }
@@ -904,10 +913,11 @@ cudaError_t launch_update(const void *X, fk_dtype dtype, int64_t N, int d, int K
                           float *C_new, int32_t *counts, double *pieces_a, int32_t *pkeys_a,
                           double *pieces_b, int32_t *pkeys_b, double *jpart,
                           double *objective, uint32_t *err, double *sums_out,
-                          cudaStream_t st) {
+                          cudaStream_t st, const CentroidOperands *next, bool *prepped) {
     const bool bf16 = dtype == FK_BF16;
+    if (prepped) *prepped = false;
     FinalLevel fl;
-    const bool wide = up.nwarps <= kWideUnits;
+    const bool wide = up.nwarps <= kUpdWideUnits;
     cudaError_t e = run_levels(X, bf16, N, d, up, skeys, perm, offsets, C_used, C_new,
                                sums_out, pieces_a, pkeys_a, pieces_b, pkeys_b, jpart, err, st,
                                &fl, wide);
@@ -915,20 +925,28 @@ cudaError_t launch_update(const void *X, fk_dtype dtype, int64_t N, int d, int K
     if (wide) {
         // a small problem: every combine level, the finalize and the objective in one launch
         static std::atomic<uint64_t> smem_set{0};
-        if ((e = smem_opt_in(wide_combine_kernel, static_cast<int>(kWideSmem), smem_set)) !=
-            cudaSuccess)
+        if ((e = smem_opt_in(wide_combine_kernel, static_cast<int>(wide_smem(kUpdWideUnits)),
+                             smem_set)) != cudaSuccess)
             return e;
         int rows_log2 = 0;
         while ((1 << rows_log2) < up.rows) ++rows_log2;  // rows is a power of two
+        const size_t smem = wide_smem(up.nwarps);
+        // one column block: a block owns whole rows and can prepare the next operands
+        const bool fuse = next != nullptr && sums_out == nullptr && up.ncolblk == 1;
+        // blocks that fit on an SM at once (228 KB of shared memory, 1 KB reserved and
+        // 2 KB static per block), so the cluster loop runs in one wave
+        const int64_t fit = static_cast<int64_t>((228u << 10) / (smem + (3u << 10)));
         int64_t blocks = K;
-        const int64_t cap = static_cast<int64_t>(device_sm_count()) * 3;  // 3 fit per SM
+        const int64_t cap = static_cast<int64_t>(device_sm_count()) * (fit < 1 ? 1 : fit);
         if (blocks > cap) blocks = cap;
         launch_pdl(wide_combine_kernel, dim3(static_cast<unsigned>(blocks + 1), up.ncolblk),
-                   dim3(kWideWarps * 32), kWideSmem, st, pieces_a, rows_log2, K, d,
+                   dim3(kWideWarps * 32), smem, st, pieces_a, rows_log2,
+                   wide_l2cap(up.nwarps), K, d,
                    up.dcov, offsets, C_old, C_new, sums_out, counts, jpart,
-                   up.nwarps * up.ncolblk, objective);
+                   up.nwarps * up.ncolblk, objective, fuse ? *next : CentroidOperands{});
         note_launch();
-        return cudaGetLastError();
+        if ((e = cudaGetLastError()) == cudaSuccess && prepped) *prepped = fuse;
+        return e;
     }
     // the update's tail in one launch: the objective (block 0), the last combine level (one
     // block per 128-column block) and the empty clusters (the remaining blocks)

@@ -75,7 +75,7 @@ def test_assign_tight_mixture_recovers_components():
 UPDATE_SHAPES = [(1000, 64, 10, "equal"), (20000, 128, 37, "equal"), (70000, 128, 3, "equal"),
                  (5000, 768, 50, "equal"), (3000, 1032, 20, "equal"), (200000, 16, 2, "equal"),
                  (150000, 128, 4096, "zipf"), (777, 8, 700, "equal"),
-                 (60000, 96, 500, "zipf")]
+                 (60000, 96, 500, "zipf"), (40960, 64, 1000, "zipf")]
 
 
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
