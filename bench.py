@@ -284,7 +284,7 @@ def fk_arm(args, spec, rank, world, dist):
                                    counts=counts, timing=mode if acc is not None else False)
             if acc is not None:
                 for k in ("ms_setup", "ms_prep", "ms_assign", "ms_sort", "ms_update",
-                          "ms_assign_mma", "screened"):
+                          "ms_assign_mma", "mma_timed", "screened"):
                     acc[k] = acc.get(k, 0) + tm[k]
             return objs
         Xp = Xin
@@ -322,9 +322,10 @@ def fk_arm(args, spec, rank, world, dist):
         dist.barrier()
     torch.cuda.synchronize()
     launches0 = fk.launch_count()
-    # the timed steps time only the assignment kernel (the roofline's launches); the
-    # per-phase breakdown comes from extra steps after the timed region
-    mode = True if sharded else "kernel"
+    # the timed steps time only the assignment kernel of each step's last iteration (the
+    # roofline's launches; two events per step, so that they barely perturb the steps);
+    # the per-phase breakdown comes from extra steps after the timed region
+    mode = True if sharded else "kernel_last"
     if flush is None:
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
@@ -378,7 +379,7 @@ def fk_arm(args, spec, rank, world, dist):
         mma_ms, screened = phase_ms, None
         scr = spec.dtype == "f32" and spec.d >= 256 and spec.n >= 18944
     else:
-        mma_ms, screened = acc["ms_assign_mma"] / n_assign, acc["screened"]
+        mma_ms, screened = acc["ms_assign_mma"] / max(1, acc["mma_timed"]), acc["screened"]
         scr = screened == n_assign
     # fp32 points: the screened route's main kernel runs one bf16 product per term (peak:
     # the bf16 peak); the three-product route runs three per useful product (bf16 / 3).
@@ -406,6 +407,9 @@ def fk_arm(args, spec, rank, world, dist):
             "frac": achieved / peak, "traffic": trec["bytes_per_launch"] if trec else None,
             "kernel": kernel, "algorithmic_flops_per_launch": flops,
             "avg_launch_ms": mma_ms, "peak_note": peak_note,
+            "launches_timed": n_assign if sharded else acc["mma_timed"],
+            "launches_timed_note": "the assignment kernel of each timed step's last iteration"
+                                   if not sharded else "every iteration's assignment",
             "frac_of_sustained": achieved / peak_sus,
             "assign_phase": {"ms_per_iteration": phase_ms,
                              "useful_tflops": flops / (phase_ms / 1e3) / 1e12,

@@ -8,7 +8,7 @@ CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libfk.so")
 SOURCES = ["fk_api.cu", "prep.cu", "assign_sm100.cu", "screen.cu", "sort_csr.cu", "update.cu",
            "ivf.cu", "ivf_search.cu", "fk_noalloc.cu"]
-HEADERS = ["fk_common.cuh", "ptx_sm100.cuh"]
+HEADERS = ["fk_common.cuh", "ptx_sm100.cuh", "prep_row.cuh"]
 
 
 def nvcc() -> str:

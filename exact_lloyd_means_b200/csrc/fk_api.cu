@@ -780,6 +780,7 @@ fk_status fk_lloyd(const void *X, fk_dtype dtype, int64_t N, int d, int K, fk_me
     // iteration (after prep, assign, sort, update) and 2 per iteration around the
     // assignment's tensor-core kernel; with kernel_only, only the last two.
     const bool kernel_only = timing && timing->kernel_only != 0;
+    const bool mma_last_only = kernel_only && timing->kernel_only == 2;
     const bool phases = timing && !kernel_only;
     std::vector<cudaEvent_t> *pool = nullptr;
     if (timing && !pooled_events(2 + 6 * static_cast<size_t>(niter), &pool))
@@ -864,10 +865,11 @@ fk_status fk_lloyd(const void *X, fk_dtype dtype, int64_t N, int d, int K, fk_me
                 !rec(4 * t))
                 return FK_ERR_CUDA;
             bool screened = false;
+            const bool timed = mev && (!mma_last_only || t == niter - 1);
             fk_status r = run_assign(planes, nplanes, lda, N, d, K, L, ws, labels, xnorm, nullptr,
                                      s_, dtype == FK_F32 ? static_cast<const float *>(Xp) : nullptr,
-                                     Ccur, allow_screen, &screened, mev ? mev[2 * t] : nullptr,
-                                     mev ? mev[2 * t + 1] : nullptr);
+                                     Ccur, allow_screen, &screened, timed ? mev[2 * t] : nullptr,
+                                     timed ? mev[2 * t + 1] : nullptr);
             if (r != FK_OK) return r;
             nscr += screened ? 1 : 0;
             last = screened;
@@ -959,7 +961,8 @@ fk_status fk_lloyd(const void *X, fk_dtype dtype, int64_t N, int d, int K, fk_me
         }
         const LoopKey key{X,    C,     labels, counts, offsets, ws,     ws_bytes, N,
                           d,    K,     niter,  dev,    ctx,     dtype,  metric,
-                          timing ? (kernel_only ? 1 : 2) : 0, allow_screen};
+                          timing ? (kernel_only ? (mma_last_only ? 3 : 1) : 2) : 0,
+                          allow_screen};
         LoopGraph *g = nullptr;
         for (LoopGraph &c : cache.graphs)
             if (c.key == key) g = &c;
@@ -1053,7 +1056,7 @@ fk_status fk_lloyd(const void *X, fk_dtype dtype, int64_t N, int d, int K, fk_me
     if (timing) {
         float ms = 0.f;
         std::memset(timing, 0, sizeof(*timing));
-        timing->kernel_only = kernel_only ? 1 : 0;
+        timing->kernel_only = kernel_only ? (mma_last_only ? 2 : 1) : 0;
         timing->empty_clusters = static_cast<int>(stats[0]);
         timing->max_cluster = static_cast<int>(stats[1]);
         timing->fallback_rows = static_cast<int>(stats[2]);
@@ -1067,7 +1070,10 @@ fk_status fk_lloyd(const void *X, fk_dtype dtype, int64_t N, int d, int K, fk_me
                 const cudaEvent_t from = a == 0 ? e1 : lev[a - 1];
                 if (elapsed_ms(from, lev[a], &ms)) *slot[p] += ms;
             }
-            if (elapsed_ms(mev[2 * t], mev[2 * t + 1], &ms)) timing->ms_assign_mma += ms;
+            if ((!mma_last_only || t == niter - 1) && elapsed_ms(mev[2 * t], mev[2 * t + 1], &ms)) {
+                timing->ms_assign_mma += ms;
+                ++timing->mma_timed;
+            }
         }
         timing->iterations = niter;
         timing->launches = static_cast<int>(g_launches - launches0);

@@ -30,15 +30,9 @@ constexpr int64_t kSortSmallN = int64_t(1) << 22;
 // digit width bound: 256 bins (a tile's per-digit bookkeeping grows with the bins, so two
 // narrow passes beat one wide one from about 1024 bins)
 constexpr int kSortMaxBits = 8;
-// Tiles up to which the upsweep's last tile scans the per-tile counts itself (its threads
-// read a digit's counts each: 256 tiles are 1 KB per thread)
-constexpr int64_t kSortScanInUpsweep = 256;
-// Words of the 256-byte error block at the start of a workspace: [0] a bounded wait
-// expired, [1] a label out of range, [4..5] the last iteration's statistics, [8] the
-// sort's tile ticket (zero between calls: the last tile resets it).  Cleared on entry by
-// fk_lloyd, and by fk_get_device_error.
-constexpr int kSortTicketWord = 8;
-constexpr int kErrWords = 9;
+// Words of the 256-byte error block at the start of a workspace that a call clears: [0] a
+// bounded wait expired, [1] a label out of range ([4..5]: the last iteration's statistics).
+constexpr int kErrWords = 2;
 
 // ----------------------------------------------------------------- update tiling
 constexpr int kUpdWarps = 8;          // warps per block of the update kernels

@@ -23,8 +23,7 @@
 //               stable and the output is unique.
 // offsets[k] = first sorted position whose key is >= k, written once per k: by the first
 // downsweep tile for a one-pass sort (the digit bases are the offsets), else by a kernel of
-// its own after the last pass.  With at most kSortScanInUpsweep tiles the scan runs in the
-// upsweep's last tile, so a small one-pass sort is two launches.
+// its own after the last pass.
 #include "fk_common.cuh"
 
 namespace fk {
@@ -80,20 +79,14 @@ __device__ __forceinline__ void count_tile(const int32_t *__restrict__ keys, int
     }
 }
 
-// With few tiles (scan_in_upsweep), the tile that finishes counting last (an atomic ticket
-// in the error block; every tile makes its counts visible device-wide first) also does the
-// scan launch's work: each of its threads scans one digit's per-tile counts in place (16-byte
-// loads from L2, eight in flight) and stores the digit total, then it resets the ticket.
-// Integer counts: the result does not depend on which tile is last.
 template <int ITEMS>
 __global__ void __launch_bounds__(kSortThreads)
     upsweep_kernel(const int32_t *__restrict__ keys, int64_t n, int shift, int bits, int K,
                    uint32_t *__restrict__ hist, int64_t nblocks, uint32_t *__restrict__ err,
-                   int check, uint32_t *__restrict__ dtot, int scan_in_upsweep) {
+                   int check) {
     pdl_wait();
     pdl_trigger();
     extern __shared__ uint32_t wh[];
-    __shared__ uint32_t s_last;
     const int bins = 1 << bits;
     for (int i = threadIdx.x; i < kWarps * bins; i += blockDim.x) wh[i] = 0;
     __syncthreads();
@@ -106,58 +99,6 @@ __global__ void __launch_bounds__(kSortThreads)
         for (int w = 0; w < kWarps; ++w) t += wh[w * bins + b];
         hist[static_cast<int64_t>(b) * nblocks + blockIdx.x] = t;
     }
-    if (!scan_in_upsweep) return;
-    uint32_t *ticket = err + kSortTicketWord;
-    __threadfence();  // this tile's counts are visible device-wide before its ticket
-    __syncthreads();
-    if (threadIdx.x == 0)
-        s_last = atomicAdd(ticket, 1u) == static_cast<uint32_t>(nblocks) - 1u ? 1u : 0u;
-    __syncthreads();
-    if (!s_last) return;
-    __threadfence();  // the other tiles' counts are read after their tickets
-    for (int b = threadIdx.x; b < bins; b += blockDim.x) {
-        uint32_t *r1 = hist + static_cast<int64_t>(b) * nblocks;
-        uint32_t run = 0;
-        if (nblocks % 4 != 0) {  // rows not 16-byte aligned: single counts, eight in flight
-            for (int64_t q = 0; q < nblocks; q += 8) {
-                uint32_t v[8];
-#pragma unroll
-                for (int j = 0; j < 8; ++j) v[j] = q + j < nblocks ? __ldcg(r1 + q + j) : 0u;
-#pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    if (q + j >= nblocks) break;
-                    r1[q + j] = run;
-                    run += v[j];
-                }
-            }
-            dtot[b] = run;
-            continue;
-        }
-        const int64_t nq = nblocks / 4;
-        uint4 *row = reinterpret_cast<uint4 *>(r1);
-        for (int64_t q = 0; q < nq; q += 8) {
-            uint4 v[8];
-#pragma unroll
-            for (int j = 0; j < 8; ++j)
-                if (q + j < nq) v[j] = __ldcg(row + q + j);
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                if (q + j >= nq) break;
-                uint4 o;
-                o.x = run;
-                run += v[j].x;
-                o.y = run;
-                run += v[j].y;
-                o.z = run;
-                run += v[j].z;
-                o.w = run;
-                run += v[j].w;
-                row[q + j] = o;
-            }
-        }
-        dtot[b] = run;
-    }
-    if (threadIdx.x == 0) *ticket = 0u;
 }
 
 // Exclusive scan of 1024 per-thread values held in registers; returns the exclusive
@@ -433,8 +374,6 @@ cudaError_t launch_sort_csr(const int32_t *labels, int64_t N, int K, const SortP
         const bool small = sp.items == kSortItemsSmall;
         // a one-pass sort's downsweep writes the CSR offsets (no offsets launch)
         const bool one_pass = sp.passes == 1;
-        // few tiles: the last upsweep tile scans the counts (no scan launch)
-        const bool scan_in_upsweep = sp.nblocks <= kSortScanInUpsweep;
         const int32_t *kin = labels;
         const int32_t *vin = nullptr;
         int32_t *kb[2] = {keys0, keys1};
@@ -444,13 +383,10 @@ cudaError_t launch_sort_csr(const int32_t *labels, int64_t N, int K, const SortP
             const dim3 grid(static_cast<unsigned>(sp.nblocks));
             launch_pdl(small ? upsweep_kernel<kSortItemsSmall> : upsweep_kernel<kSortItems>, grid,
                        dim3(kSortThreads), up_smem, st, kin, N, shift, sp.bits, K, hist,
-                       sp.nblocks, err, p == 0 ? 1 : 0, dtot, scan_in_upsweep ? 1 : 0);
+                       sp.nblocks, err, p == 0 ? 1 : 0);
             note_launch();
-            if (!scan_in_upsweep) {
-                launch_pdl(scan_rows_kernel, dim3(bins), dim3(1024), 0, st, hist, sp.nblocks,
-                           dtot);
-                note_launch();
-            }
+            launch_pdl(scan_rows_kernel, dim3(bins), dim3(1024), 0, st, hist, sp.nblocks, dtot);
+            note_launch();
             int32_t *vo = (p == sp.passes - 1 && perm_out) ? perm_out : vb[p & 1];
             launch_pdl(small ? downsweep_kernel<kSortItemsSmall> : downsweep_kernel<kSortItems>,
                        grid, dim3(kSortThreads), dn_smem, st, kin, vin, kb[p & 1], vo, N, shift,

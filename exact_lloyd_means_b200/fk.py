@@ -39,7 +39,7 @@ class FkTiming(ctypes.Structure):
                 ("launches", ctypes.c_int), ("ms_assign_mma", ctypes.c_double),
                 ("screened", ctypes.c_int), ("empty_clusters", ctypes.c_int),
                 ("max_cluster", ctypes.c_int), ("fallback_rows", ctypes.c_int),
-                ("kernel_only", ctypes.c_int)]
+                ("kernel_only", ctypes.c_int), ("mma_timed", ctypes.c_int)]
 
 
 class FkSearchTiming(ctypes.Structure):
@@ -285,13 +285,14 @@ def fk_lloyd(X: torch.Tensor, C: torch.Tensor, niter: int, labels: torch.Tensor,
              ws: torch.Tensor, metric="l2", counts: torch.Tensor | None = None,
              offsets: torch.Tensor | None = None, timing: bool | str = False, stream=None):
     """Run niter iterations in place on C.  Returns (objectives list, timing dict|None).
-    timing: True times every phase; "kernel" only the assignment's tensor-core kernel."""
+    timing: True times every phase; "kernel" only the assignment's tensor-core kernel of
+    every iteration; "kernel_last" only that of the last iteration."""
     N, d = X.shape
     K = C.shape[0]
     obj = (ctypes.c_double * max(niter, 1))()
     tm = FkTiming() if timing else None
     if tm is not None:
-        tm.kernel_only = 1 if timing == "kernel" else 0
+        tm.kernel_only = {"kernel": 1, "kernel_last": 2}.get(timing, 0)
     _check(_lib.fk_lloyd(_dev(X, "X"), _dtype_code(X), N, d, K, _metric_code(metric), niter,
                          _dev(C, "C", torch.float32, (K, d)),
                          _dev(labels, "labels", torch.int32, (N,)),

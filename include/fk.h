@@ -106,12 +106,15 @@ typedef struct fk_timing {
     int max_cluster;    /* last iteration: points in the largest cluster                */
     int fallback_rows;  /* last iteration, screened route: rows sent to the three-product
                            pass (0 when the iteration was not screened)                 */
-    int kernel_only;    /* IN: nonzero times only the main tensor-core kernel of each
-                           assignment (two events per iteration): ms_assign_mma,
+    int kernel_only;    /* IN: 1 times only the main tensor-core kernel of each
+                           assignment (two events per iteration), 2 only that of the last
+                           iteration (two events per call): ms_assign_mma, mma_timed,
                            iterations, launches and screened are filled, every other field
                            is 0.  The lightest timing, for loops of short calls, where the
-                           events between the phases would cost a noticeable share.  The
-                           call keeps this field as given.                               */
+                           events between the phases would cost a noticeable share.  0
+                           times every phase.  The call keeps this field as given.       */
+    int mma_timed;      /* launches of the main kernel whose device time ms_assign_mma
+                           sums (niter, or 1 with kernel_only = 2)                      */
 } fk_timing;
 
 /* Human-readable name of a status code (static string, never NULL). */

@@ -260,13 +260,16 @@ def test_fk_lloyd_repeated_calls_replay_identically():
         assert tm["iterations"] == 4 and tm["launches"] == timed[0][4]["launches"] > 0
         for k in ("ms_prep", "ms_assign", "ms_sort", "ms_update", "ms_assign_mma"):
             assert tm[k] > 0, k
-    # kernel-only timing: the assignment kernel's time alone, the same results
-    for r in [run(C0g, timing="kernel") for _ in range(3)]:
-        assert all(torch.equal(a, b) for a, b in zip(r[:3], ref[:3])) and r[3] == ref[3]
-        tm = r[4]
-        assert tm["kernel_only"] == 1 and tm["iterations"] == 4 and tm["ms_assign_mma"] > 0
-        assert tm["ms_assign"] == 0 and tm["ms_update"] == 0 and tm["max_cluster"] == 0
-        assert tm["launches"] == timed[0][4]["launches"] - 1  # no statistics kernel
+    # kernel-only timing: the assignment kernel's time alone (every iteration's, or the
+    # last iteration's), the same results
+    for mode, code, n in (("kernel", 1, 4), ("kernel_last", 2, 1)):
+        for r in [run(C0g, timing=mode) for _ in range(3)]:
+            assert all(torch.equal(a, b) for a, b in zip(r[:3], ref[:3])) and r[3] == ref[3]
+            tm = r[4]
+            assert tm["kernel_only"] == code and tm["iterations"] == 4
+            assert tm["mma_timed"] == n and tm["ms_assign_mma"] > 0
+            assert tm["ms_assign"] == 0 and tm["ms_update"] == 0 and tm["max_cluster"] == 0
+            assert tm["launches"] == timed[0][4]["launches"] - 1  # no statistics kernel
     # other initial centroids: the eager result (another labels buffer, so another call)
     # equals the replay of the cached loop with the original buffers
     C1g = C0g[torch.randperm(K, generator=torch.Generator().manual_seed(5)).to(DEV)]
