@@ -206,6 +206,16 @@ inline UpdPlan upd_plan(int64_t N, int d) {
     return p;
 }
 
+// The one-launch combine (at most kUpdWideUnits level-1 units): the shared-memory entries
+// (128 doubles each) of its two level buffers.  A cluster's units are consecutive, so its
+// level-2 partials span at most (units - 1) / kUpdGroup + 1 groups; its level-3 partials at
+// most that / kUpdGroup + 1, and the buffers alternate from there on.
+inline int upd_wide_l2cap(int64_t units) { return static_cast<int>((units - 1) / kUpdGroup + 1); }
+inline int upd_wide_l3cap(int64_t units) { return upd_wide_l2cap(units) / kUpdGroup + 2; }
+inline size_t upd_wide_smem(int64_t units) {
+    return size_t(upd_wide_l2cap(units) + upd_wide_l3cap(units)) * 128 * sizeof(double);
+}
+
 // Byte offsets of every scratch buffer inside the caller's workspace (256-byte aligned).
 struct WsLayout {
     size_t err = 0, obj = 0, xn = 0, xs = 0, xnorm = 0, cs = 0, cn = 0, cused = 0,

@@ -727,12 +727,6 @@ __global__ void __launch_bounds__(256)
 constexpr int kWideWarps = 8;
 static_assert(kWideWarps * 32 == 256, "sum_objective runs on 256 threads");
 
-// Shared-memory entries (128 doubles each) of the two level buffers for `units` units.
-inline int wide_l2cap(int64_t units) { return static_cast<int>((units - 1) / kGroup + 1); }
-inline int wide_l3cap(int64_t units) { return wide_l2cap(units) / kGroup + 2; }
-inline size_t wide_smem(int64_t units) {
-    return size_t(wide_l2cap(units) + wide_l3cap(units)) * 128 * sizeof(double);
-}
 
 __global__ void __launch_bounds__(kWideWarps * 32)
     wide_combine_kernel(const double *__restrict__ pieces, int rows_log2, int l2cap, int K,
@@ -925,12 +919,12 @@ cudaError_t launch_update(const void *X, fk_dtype dtype, int64_t N, int d, int K
     if (wide) {
         // a small problem: every combine level, the finalize and the objective in one launch
         static std::atomic<uint64_t> smem_set{0};
-        if ((e = smem_opt_in(wide_combine_kernel, static_cast<int>(wide_smem(kUpdWideUnits)),
+        if ((e = smem_opt_in(wide_combine_kernel, static_cast<int>(upd_wide_smem(kUpdWideUnits)),
                              smem_set)) != cudaSuccess)
             return e;
         int rows_log2 = 0;
         while ((1 << rows_log2) < up.rows) ++rows_log2;  // rows is a power of two
-        const size_t smem = wide_smem(up.nwarps);
+        const size_t smem = upd_wide_smem(up.nwarps);
         // one column block: a block owns whole rows and can prepare the next operands
         const bool fuse = next != nullptr && sums_out == nullptr && up.ncolblk == 1;
         // blocks that fit on an SM at once (228 KB of shared memory, 1 KB reserved and
@@ -941,7 +935,7 @@ cudaError_t launch_update(const void *X, fk_dtype dtype, int64_t N, int d, int K
         if (blocks > cap) blocks = cap;
         launch_pdl(wide_combine_kernel, dim3(static_cast<unsigned>(blocks + 1), up.ncolblk),
                    dim3(kWideWarps * 32), smem, st, pieces_a, rows_log2,
-                   wide_l2cap(up.nwarps), K, d,
+                   upd_wide_l2cap(up.nwarps), K, d,
                    up.dcov, offsets, C_old, C_new, sums_out, counts, jpart,
                    up.nwarps * up.ncolblk, objective, fuse ? *next : CentroidOperands{});
         note_launch();

@@ -122,6 +122,34 @@ int main() {
             }
         }
     }
+    // the one-launch combine: for every cluster range of level-1 units [a0, a1], each level
+    // it does not finish at writes its partials into a buffer large enough (level 2 into
+    // the first, then alternating), and its shared memory fits an SM
+    {
+        long long N = 0;
+        int K = 0, d = 128;
+        CHECK(upd_wide_smem(kUpdWideUnits) + 3 * 1024 <= 228 * 1024);
+        const long long units[] = {1, 2, 15, 16, 17, 255, 256, 257, 1000, 1024, 2047, 2048};
+        for (long long U : units) {
+            N = U;
+            const int l2 = upd_wide_l2cap(U), l3 = upd_wide_l3cap(U);
+            for (long long lo = 0; lo < U; ++lo) {
+                for (long long hi = lo; hi < U; hi += (U > 300 ? 7 : 1)) {
+                    long long a0 = lo, a1 = hi;
+                    bool first = true;
+                    while (a0 != a1) {
+                        const long long g0 = a0 / kUpdGroup, g1 = a1 / kUpdGroup;
+                        if (g0 == g1) break;  // finished at this level: nothing stored
+                        CHECK(g1 - g0 + 1 <= (first ? l2 : l3));
+                        a0 = g0;
+                        a1 = g1;
+                        first = !first;
+                    }
+                }
+            }
+            ++cases;
+        }
+    }
     std::printf("%d layouts checked, %d failures\n", cases, fails);
     return fails == 0 ? 0 : 1;
 }
