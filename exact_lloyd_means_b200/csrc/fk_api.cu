@@ -814,7 +814,12 @@ fk_status fk_lloyd(const void *X, fk_dtype dtype, int64_t N, int d, int K, fk_me
     double *obj = ws_ptr<double>(ws, L.obj);
     float *cused = ws_ptr<float>(ws, L.cused);
     bool allow_screen = true;
-    if (niter > 0 && dtype == FK_F32) {
+    // the probe runs where fk_assign would take the screened route for these fp32 points by
+    // choice (beyond kThreeProductMaxDp it has no choice: nothing to probe)
+    const bool probe = niter > 0 && dtype == FK_F32 && lda == L.dp &&
+                       L.dp <= kThreeProductMaxDp &&
+                       screened_route(N, static_cast<int>(L.dp), static_cast<int>(L.Kp), K);
+    if (probe) {
         // Where the screened route applies, try it first on a sample of the rows with the
         // initial centroids and read how many would need the three-product pass (a single
         // host synchronisation per call); screen the call only if few would.

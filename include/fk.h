@@ -216,15 +216,25 @@ FK_API fk_status fk_update(const void *X, fk_dtype dtype, int64_t N, int d, int 
 
 /* `niter` Lloyd iterations from the initial centroids in C (K x d fp32, overwritten with
  * the final centroids).  Cosine mode normalises X (into the workspace; X itself is not
- * modified) and the initial C first.  On return (this call synchronises `stream` once,
- * at the end):
+ * modified) and the initial C first.  On return (this call synchronises `stream` at the
+ * end, and once more after the screening probe where fp32 points may take the screened
+ * route):
  *   labels           N int32, the labels of the last assignment (device);
  *   counts, offsets  of the last assignment (device; optional, may be NULL);
  *   objective_host   niter doubles (HOST pointer, optional): entry t is the objective
  *                    of iteration t's labels against the centroids they were assigned
  *                    with;
- *   timing           HOST pointer (optional): per-phase device milliseconds.
- * niter = 0 only normalises C (cosine) and returns. */
+ *   timing           HOST pointer (optional): device milliseconds of every phase, or of
+ *                    the assignment kernel alone (see fk_timing.kernel_only).
+ * niter = 0 only normalises C (cosine) and returns.
+ * A call that repeats the previous call on the same host thread (same pointers, sizes,
+ * metric, iteration count below 4096, timing mode, device and probe decision) records
+ * its iteration loop and end-of-call copies into a CUDA graph, and later identical calls
+ * replay it (up to four graphs per thread).  The graph reads X and C when it runs, so new
+ * values need no new capture; results are the same bits either way.  FK_LOOP_GRAPH=0 in
+ * the environment runs every call eagerly.  For this the library keeps per-thread
+ * streams, events, pinned host staging and graphs, each tied to the CUDA context it was
+ * made in and dropped when that context changes. */
 FK_API fk_status fk_lloyd(const void *X, fk_dtype dtype, int64_t N, int d, int K,
                    fk_metric metric, int niter, float *C, int32_t *labels,
                    int32_t *counts, int32_t *offsets, double *objective_host,
