@@ -508,10 +508,10 @@ bool pooled_events(size_t n, std::vector<cudaEvent_t> **out) {
 }
 
 // fk_lloyd's iteration loop as a CUDA graph.  The loop's launches are fixed by the call's
-// arguments and by the screening probe's decision, so a call that repeats the previous call
-// on the same thread (same pointers, sizes, metric, iteration count, timing flag, device and
-// probe decision) captures its loop once and replays it as one graph launch, and later
-// identical calls replay it again.  The graph reads device memory when it runs, so new
+// arguments and by the screening probe's decision, so a short call (kLoopGraphMaxFlops)
+// that repeats the previous call on the same thread (same pointers, sizes, metric,
+// iteration count, timing flag, device and probe decision) captures its loop once and
+// replays it as one graph launch, and later identical calls replay it again.  The graph reads device memory when it runs, so new
 // point or centroid values need no new capture.  FK_LOOP_GRAPH=0 in the environment turns
 // the cache off.
 struct LoopKey {
@@ -547,6 +547,12 @@ struct LoopGraph {
 };
 
 constexpr size_t kLoopGraphs = 4;
+
+// Calls up to this many useful flops (2 N K d niter, about a millisecond of tensor work)
+// replay their loop from a graph.  There the launches are a large share of the call; above
+// it they are not, and a capture's host time (tens of milliseconds for a long loop with
+// timing events) would take hundreds of calls to repay.
+constexpr double kLoopGraphMaxFlops = 1e12;
 
 struct LoopGraphCache {
     bool have_last = false;
@@ -953,7 +959,8 @@ fk_status fk_lloyd(const void *X, fk_dtype dtype, int64_t N, int d, int K, fk_me
     bool replayed = false;
     int dev = 0;
     const uint64_t ctx = context_id();
-    if (niter > 0 && niter < kObjRing && loop_graphs_enabled() && ctx != 0 &&
+    const bool short_call = 2.0 * static_cast<double>(N) * K * d * niter <= kLoopGraphMaxFlops;
+    if (niter > 0 && niter < kObjRing && short_call && loop_graphs_enabled() && ctx != 0 &&
         cudaGetDevice(&dev) == cudaSuccess && dev >= 0 && dev < 64) {
         LoopGraphCache &cache = loop_graphs();
         // graphs and capture streams of another context are dropped unreleased

@@ -227,7 +227,8 @@ FK_API fk_status fk_update(const void *X, fk_dtype dtype, int64_t N, int d, int 
  *   timing           HOST pointer (optional): device milliseconds of every phase, or of
  *                    the assignment kernel alone (see fk_timing.kernel_only).
  * niter = 0 only normalises C (cosine) and returns.
- * A call that repeats the previous call on the same host thread (same pointers, sizes,
+ * A short call (at most 1e12 useful flops, 2 N K d niter: launches are a large share of
+ * it) that repeats the previous call on the same host thread (same pointers, sizes,
  * metric, iteration count below 4096, timing mode, device and probe decision) records
  * its iteration loop and end-of-call copies into a CUDA graph, and later identical calls
  * replay it (up to four graphs per thread).  The graph reads X and C when it runs, so new
