@@ -40,8 +40,12 @@ constexpr int kUpdGroup = 16;         // units of one combine level per unit of 
 constexpr int kUpdMinRows = 64;       // smallest chunk of sorted positions per warp
 constexpr int kUpdMaxRows = 256;      // largest chunk
 constexpr int64_t kUpdTargetWarps = 148 * 64;  // enough warps to cover the GPU twice
-// Level-1 units up to which every combine level runs in one launch (wide_combine_kernel)
+// Level-1 units up to which every combine level runs in one launch (wide_combine_kernel),
+// for at most kUpdWideMaxK clusters: its blocks walk their clusters one after another, so
+// beyond a few clusters per block the level-by-level launches (a warp per cluster in the
+// tail) are faster
 constexpr int64_t kUpdWideUnits = 2048;
+constexpr int kUpdWideMaxK = 4096;
 
 // ----------------------------------------------------------------- screening (fp32)
 // The single-product pass writes, per row, up to kCandPerRow candidate columns (unused

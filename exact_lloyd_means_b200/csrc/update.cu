@@ -911,7 +911,7 @@ cudaError_t launch_update(const void *X, fk_dtype dtype, int64_t N, int d, int K
     const bool bf16 = dtype == FK_BF16;
     if (prepped) *prepped = false;
     FinalLevel fl;
-    const bool wide = up.nwarps <= kUpdWideUnits;
+    const bool wide = up.nwarps <= kUpdWideUnits && K <= kUpdWideMaxK;
     cudaError_t e = run_levels(X, bf16, N, d, up, skeys, perm, offsets, C_used, C_new,
                                sums_out, pieces_a, pkeys_a, pieces_b, pkeys_b, jpart, err, st,
                                &fl, wide);
