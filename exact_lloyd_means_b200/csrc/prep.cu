@@ -7,10 +7,13 @@
 //  * prep_centroids: the same split of each centroid, scaled by -2 (exact in bf16), so the
 //               MMA accumulates -2 x.c directly; cn[k] = ||c_k||^2 (fp64 accumulation of
 //               the values the MMA consumes, rounded once to fp32); caug[k] = the three
-//               bf16 pieces hi + mid + lo that sum exactly to that fp32 value (then zeros),
-//               which one extra K = 16 MMA step against constant (1, 1, 1, 0, ...) columns
-//               of X folds into the accumulator.  Padding centroids get cn = +inf, a
-//               largest-finite bf16 first piece and zero planes, so they never win.
+//               bf16 pieces hi + mid + lo that sum exactly to that fp32 value (for norms
+//               of at least 2^-110), then zeros.  One extra K = 16 MMA step against
+//               constant (1, 1, 1, 0, ...) columns of X folds them into the accumulator,
+//               to within one fp32 ulp: the MMA adds the three products in an order the
+//               ISA does not fix, and hi + lo first can round.  Padding centroids get
+//               cn = +inf, a largest-finite bf16 first piece and zero planes, so they
+//               never win.
 //  * normalize: cosine mode (LEANN FlashLib guide, "距离度量只有 squared L2如何支持 mips /
 //               cosine"): x / ||x|| with a zero norm replaced by 1; the norm and the
 //               quotient are computed in fp64 and rounded once to fp32.
