@@ -10,8 +10,8 @@ every fp32 mantissa at several exponents, random fp32 values and the edge cases:
     lo (and whenever hi did not round up); adding hi and lo first can round, by at most
     one ulp of c2.  The ISA fixes no order for the products of one MMA step, so the
     folded norm is c2 to within one fp32 ulp: 6e-8 relative, inside the screening
-    window's allowance for the fp32 rounding of ||c||^2 and far inside the 1e-4 tie
-    window."""
+    window's allowance for the norm step's own fp32 accumulation (17 units of 2^-23 of
+    its partial sums, as for every MMA step) and far inside the 1e-4 tie window."""
 import itertools
 
 import numpy as np
